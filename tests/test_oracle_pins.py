@@ -1,0 +1,359 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself:
+a hand-worked example, closed forms, library routines (torch conv1d, rms_norm,
+softplus, a linear solve), brute force on tiny inputs, and invariants.
+
+The recurrence pinned here is the gated delta rule named on the Agnes-3.0-Flash
+pages (model card "Architecture" table, row "Delta-rule layers"; kongchang
+article, paragraph on the Gated Delta Rule):
+    S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from gated_delta_rule_81_b200 import inputs as gin
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def unit_rows(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+# ---------------------------------------------------------------- recurrence
+
+
+def test_worked_example_from_golden():
+    rows = np.loadtxt(os.path.join(GOLDEN, "recurrence_worked_example.txt"))
+    T = rows.shape[0]
+    k = rows[:, 1:3].reshape(T, 1, 2)
+    v = rows[:, 3:5].reshape(T, 1, 2)
+    q = rows[:, 5:7].reshape(T, 1, 2)
+    alpha, beta = rows[:, 7:8], rows[:, 8:9]
+    o, S = oracle.recurrence(q, k, v, alpha, beta, [0, T])
+    np.testing.assert_allclose(o[:, 0], rows[:, 9:11], rtol=0, atol=1e-14)
+    # state after the last step
+    np.testing.assert_allclose(S[0, 0].reshape(-1), rows[-1, 11:15], rtol=0, atol=1e-14)
+    # state after every step: run prefixes
+    for t in range(1, T + 1):
+        _, St = oracle.recurrence(q[:t], k[:t], v[:t], alpha[:t], beta[:t], [0, t])
+        np.testing.assert_allclose(St[0, 0].reshape(-1), rows[t - 1, 11:15], atol=1e-14)
+
+
+def test_identity_gate_keeps_state():
+    """alpha = 1, beta = 0: S_t = S_0 for all t and o_t = S_0 q_t."""
+    T, D = 37, 16
+    q = RNG.standard_normal((T, 1, D))
+    k = unit_rows(RNG.standard_normal((T, 1, D)))
+    v = RNG.standard_normal((T, 1, D))
+    S0 = RNG.standard_normal((1, 1, D, D))
+    o, S = oracle.recurrence(q, k, v, np.ones((T, 1)), np.zeros((T, 1)), [0, T], S0)
+    np.testing.assert_array_equal(S, S0)
+    np.testing.assert_allclose(o[:, 0], q[:, 0] @ S0[0, 0].T, rtol=1e-13, atol=1e-13)
+
+
+def test_orthonormal_keys_retrieve_values():
+    """alpha = 1, beta = 1, orthonormal keys: after writing (k_i, v_i), querying k_j
+    returns v_j (S (I - k k^T) + v k^T maps k to v and leaves orthogonal keys alone)."""
+    D, n = 128, 48
+    Qm, _ = np.linalg.qr(RNG.standard_normal((D, D)))
+    keys = Qm[:, :n].T  # n orthonormal rows
+    vals = RNG.standard_normal((n, D))
+    # n writes (query = own key), then n read-only queries (beta = 0) in shuffled order
+    order = RNG.permutation(n)
+    k = np.concatenate([keys, keys[order]])[:, None, :]
+    v = np.concatenate([vals, np.zeros((n, D))])[:, None, :]
+    q = np.concatenate([keys, keys[order]])[:, None, :]
+    beta = np.concatenate([np.ones(n), np.zeros(n)])[:, None]
+    o, _ = oracle.recurrence(q, k, v, np.ones((2 * n, 1)), beta, [0, 2 * n])
+    np.testing.assert_allclose(o[:n, 0], vals, atol=1e-13)
+    np.testing.assert_allclose(o[n:, 0], vals[order], atol=1e-13)
+
+
+def test_single_step_projector_form():
+    """T = 1: S_1 = alpha S_0 (I - beta k k^T) + beta v k^T (matrix form), o = S_1 q."""
+    D = 32
+    S0 = RNG.standard_normal((1, 1, D, D))
+    q, k, v = (RNG.standard_normal((1, 1, D)) for _ in range(3))
+    k = unit_rows(k)
+    alpha, beta = np.array([[0.37]]), np.array([[0.81]])
+    o, S = oracle.recurrence(q, k, v, alpha, beta, [0, 1], S0)
+    kk = np.outer(k[0, 0], k[0, 0])
+    S1 = 0.37 * S0[0, 0] @ (np.eye(D) - 0.81 * kk) + 0.81 * np.outer(v[0, 0], k[0, 0])
+    np.testing.assert_allclose(S[0, 0], S1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(o[0, 0], S1 @ q[0, 0], rtol=1e-13, atol=1e-13)
+
+
+def test_brute_force_products():
+    """T <= 8: S_T = S0 prod_t alpha_t (I - beta_t k_t k_t^T)
+    + sum_t beta_t v_t k_t^T prod_{tau > t} alpha_tau (I - beta_tau k_tau k_tau^T)."""
+    D = 24
+    for T in range(1, 9):
+        q = RNG.standard_normal((T, 1, D))
+        k = unit_rows(RNG.standard_normal((T, 1, D)))
+        v = RNG.standard_normal((T, 1, D))
+        alpha = RNG.uniform(0.2, 1.0, (T, 1))
+        beta = RNG.uniform(0.0, 1.0, (T, 1))
+        S0 = RNG.standard_normal((1, 1, D, D))
+        o, S = oracle.recurrence(q, k, v, alpha, beta, [0, T], S0)
+        P = [alpha[t, 0] * (np.eye(D) - beta[t, 0] * np.outer(k[t, 0], k[t, 0])) for t in range(T)]
+        for tt in range(1, T + 1):  # state after tt steps, as explicit products
+            St = S0[0, 0].copy()
+            for t in range(tt):
+                St = St @ P[t]
+            for t in range(tt):
+                term = beta[t, 0] * np.outer(v[t, 0], k[t, 0])
+                for tau in range(t + 1, tt):
+                    term = term @ P[tau]
+                St = St + term
+            np.testing.assert_allclose(o[tt - 1, 0], St @ q[tt - 1, 0], rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(S[0, 0], St, rtol=1e-11, atol=1e-11)
+
+
+def test_memoryless_when_alpha_zero():
+    """alpha -> 0: S_t = beta_t v_t k_t^T, o_t = beta_t (k_t . q_t) v_t."""
+    T, D = 20, 16
+    q = RNG.standard_normal((T, 1, D))
+    k = unit_rows(RNG.standard_normal((T, 1, D)))
+    v = RNG.standard_normal((T, 1, D))
+    beta = RNG.uniform(0, 1, (T, 1))
+    o, S = oracle.recurrence(q, k, v, np.zeros((T, 1)), beta, [0, T], RNG.standard_normal((1, 1, D, D)))
+    want = beta * np.sum(k[:, 0] * q[:, 0], axis=1, keepdims=True) * v[:, 0]
+    np.testing.assert_allclose(o[:, 0], want, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S[0, 0], beta[-1, 0] * np.outer(v[-1, 0], k[-1, 0]), atol=1e-14)
+
+
+@pytest.mark.parametrize("chunk", [1, 16, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_chunked_form_agrees(chunk, T):
+    """The UT-transform chunked form (library solve + matmuls) equals the sequential
+    recurrence to 1e-12, including partial chunks; chunk = 1 is the recurrence."""
+    D = 128
+    q = RNG.standard_normal((T, 1, D))
+    k = unit_rows(np.abs(RNG.standard_normal((T, 1, D))) + 0.3)  # correlated keys, as after SiLU
+    v = RNG.standard_normal((T, 1, D))
+    g = -RNG.uniform(0.0, 1.5, (T, 1))
+    beta = RNG.uniform(0, 1, (T, 1))
+    S0 = 0.1 * RNG.standard_normal((1, 1, D, D))
+    o_seq, S_seq = oracle.recurrence(q, k, v, np.exp(g), beta, [0, T], S0)
+    o_ch, S_ch = oracle.chunked_recurrence(q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0], S0[0, 0], chunk)
+    scale_o = max(1.0, np.sqrt(np.mean(o_seq**2)))
+    scale_s = max(1.0, np.sqrt(np.mean(S_seq**2)))
+    assert np.max(np.abs(o_ch - o_seq[:, 0])) <= 1e-12 * scale_o
+    assert np.max(np.abs(S_ch - S_seq[0, 0])) <= 1e-12 * scale_s
+
+
+def test_value_rows_are_independent():
+    """Changing value channel r of head h changes only output channel r of head h
+    and state row r (the state is d_v x d_k and o = S q)."""
+    T, D = 30, 16
+    q = RNG.standard_normal((T, 1, D))
+    k = unit_rows(RNG.standard_normal((T, 1, D)))
+    v = RNG.standard_normal((T, 2, D))
+    alpha, beta = RNG.uniform(0.5, 1, (T, 2)), RNG.uniform(0, 1, (T, 2))
+    o1, S1 = oracle.recurrence(q, k, v, alpha, beta, [0, T])
+    v2 = v.copy()
+    v2[:, 1, 5] += 1.0
+    o2, S2 = oracle.recurrence(q, k, v2, alpha, beta, [0, T])
+    diff_o = np.abs(o2 - o1).max(axis=0)
+    assert diff_o[1, 5] > 0
+    diff_o[1, 5] = 0
+    assert diff_o.max() == 0
+    diff_s = np.abs(S2 - S1)[0].max(axis=2)
+    assert diff_s[1, 5] > 0
+    diff_s[1, 5] = 0
+    assert diff_s.max() == 0
+
+
+# ---------------------------------------------------------------- front end / norm / gates
+
+
+def test_conv_identity_taps():
+    T, C = 50, 7
+    x = RNG.standard_normal((T, C))
+    w = np.zeros((C, 4))
+    w[:, 3] = 1.0
+    np.testing.assert_array_equal(oracle.conv(x, w, [0, T], silu=False), x)
+
+
+def test_conv_matches_torch_conv1d():
+    """Causal depthwise conv against torch.conv1d (fp64) on [history; x]."""
+    C = 9
+    cu = [0, 13, 14, 40]
+    x = RNG.standard_normal((cu[-1], C))
+    w = RNG.standard_normal((C, 4))
+    hist = RNG.standard_normal((3, 3, C))
+    for use_hist in (False, True):
+        y = oracle.conv(x, w, cu, hist if use_hist else None, silu=True)
+        for n in range(3):
+            seg = x[cu[n]:cu[n + 1]]
+            pre = hist[n] if use_hist else np.zeros((3, C))
+            full = torch.from_numpy(np.concatenate([pre, seg]).T[None])  # [1, C, 3 + L]
+            ref = F.conv1d(full, torch.from_numpy(w)[:, None, :], groups=C)[0].T  # [L, C]
+            ref = F.silu(ref).numpy()
+            np.testing.assert_allclose(y[cu[n]:cu[n + 1]], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_l2norm_unit_and_library():
+    x = RNG.standard_normal((40, 128)) * 3
+    y = oracle.l2norm(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), 1.0, atol=1e-9)
+    ref = F.normalize(torch.from_numpy(x), dim=-1).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-9, atol=1e-12)
+
+
+def test_gated_rmsnorm_matches_library():
+    o = RNG.standard_normal((25, 128))
+    z = RNG.standard_normal((25, 128)) * 2
+    w = RNG.uniform(0.5, 1.5, 128)
+    y = oracle.gated_rmsnorm(o, z, w)
+    ot, zt, wt = (torch.from_numpy(t) for t in (o, z, w))
+    ref = F.rms_norm(ot, (128,), weight=wt, eps=1e-6) * F.silu(zt)
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_gates_match_library_and_limits():
+    H = 3
+    A_log = np.log([1.0, 4.0, 16.0])
+    a = RNG.standard_normal((10, H)) * 3
+    b = RNG.standard_normal((10, H)) * 3
+    g, alpha, beta = oracle.gates(A_log, a, b)
+    ref_g = -np.exp(A_log)[None] * F.softplus(torch.from_numpy(a)).numpy()
+    np.testing.assert_allclose(g, ref_g, rtol=1e-13)
+    np.testing.assert_allclose(alpha, np.exp(ref_g), rtol=1e-13)
+    np.testing.assert_allclose(beta, torch.sigmoid(torch.from_numpy(b)).numpy(), rtol=1e-13)
+    lim = np.array([[-np.inf, -np.inf, np.inf]])
+    _, al, be = oracle.gates(np.zeros(3), lim, lim)
+    assert al[0, 0] == 1.0 and al[0, 1] == 1.0 and al[0, 2] == 0.0
+    assert be[0, 0] == 0.0 and be[0, 2] == 1.0
+
+
+# ---------------------------------------------------------------- whole mixer
+
+
+def _torch_composition(case, state_in=None, conv_in=None):
+    """The mixer rebuilt from library pieces (torch conv1d, normalize, softplus,
+    sigmoid, rms_norm) around the independent chunked form."""
+    inp, cu = case["inp"], case["cu_seqlens"].tolist()
+    H_k, H_v = case["H_k"], case["H_v"]
+    D = gin.D
+    G = H_v // H_k
+    f64 = lambda t: t.to(torch.float64)  # noqa: E731
+    x = torch.cat([f64(inp["q"]).reshape(-1, H_k * D), f64(inp["k"]).reshape(-1, H_k * D),
+                   f64(inp["v"]).reshape(-1, H_v * D)], dim=1)
+    C = x.shape[1]
+    w = f64(inp["conv_w"])
+    out = np.zeros((cu[-1], H_v, D))
+    S_fin = np.zeros((len(cu) - 1, H_v, D, D))
+    for n in range(len(cu) - 1):
+        seg = x[cu[n]:cu[n + 1]]
+        pre = f64(conv_in[n]) if conv_in is not None else torch.zeros(3, C, dtype=torch.float64)
+        y = F.conv1d(torch.cat([pre, seg]).T[None], w[:, None, :], groups=C)[0].T
+        y = F.silu(y)
+        L = seg.shape[0]
+        qh = y[:, :H_k * D].reshape(L, H_k, D)
+        kh = y[:, H_k * D:2 * H_k * D].reshape(L, H_k, D)
+        vh = y[:, 2 * H_k * D:].reshape(L, H_v, D)
+        qh = qh / torch.sqrt((qh * qh).sum(-1, keepdim=True) + 1e-6) * inp["scale"]
+        kh = kh / torch.sqrt((kh * kh).sum(-1, keepdim=True) + 1e-6)
+        a = f64(inp["a"][cu[n]:cu[n + 1]])
+        b = f64(inp["b"][cu[n]:cu[n + 1]])
+        g = -torch.exp(f64(inp["A_log"]))[None] * F.softplus(a)
+        beta = torch.sigmoid(b)
+        z = f64(inp["z"][cu[n]:cu[n + 1]])
+        for h in range(H_v):
+            S0 = None if state_in is None else state_in[n, h].double().numpy()
+            o, S = oracle.chunked_recurrence(qh[:, h // G].numpy(), kh[:, h // G].numpy(),
+                                             vh[:, h].numpy(), g[:, h].numpy(), beta[:, h].numpy(),
+                                             S0, chunk=64)
+            yv = F.rms_norm(torch.from_numpy(o), (D,), weight=f64(inp["norm_w"]), eps=1e-6) * F.silu(z[:, h])
+            out[cu[n]:cu[n + 1], h] = yv.numpy()
+            S_fin[n, h] = S
+    return out, S_fin
+
+
+def _small_case(lengths, H_k=2, H_v=6, seed=3):
+    case = gin.prefill_case(3, seed=seed, lengths=lengths)
+    # re-draw at the small head counts with the same recipe
+    T = sum(lengths)
+    inp = gin.token_inputs(T, H_k, H_v, seed)
+    inp.update(gin.weights(H_k, H_v, seed))
+    inp["scale"] = 1.0
+    case.update(inp=inp, H_k=H_k, H_v=H_v)
+    return case
+
+
+def test_mixer_matches_library_composition():
+    case = _small_case([70, 1, 130])
+    N, H_v = 3, case["H_v"]
+    st = gin.recurrent_state(N, H_v, seed=5)
+    cv = gin.conv_state(N, case["H_k"], H_v, seed=5)
+    res = oracle.mixer(case["inp"], case["cu_seqlens"], state_in=st, conv_in=cv)
+    ref_out, ref_S = _torch_composition(case, st, cv)
+    np.testing.assert_allclose(res["out"], ref_out, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(res["state"], ref_S, rtol=1e-10, atol=1e-12)
+
+
+def test_mixer_conv_out_is_last_three_raw_tokens():
+    case = _small_case([5, 1, 2])
+    H_k, H_v = case["H_k"], case["H_v"]
+    cv = gin.conv_state(3, H_k, H_v, seed=9)
+    res = oracle.mixer(case["inp"], case["cu_seqlens"], conv_in=cv)
+    inp = case["inp"]
+    x = torch.cat([inp["q"].reshape(8, -1), inp["k"].reshape(8, -1), inp["v"].reshape(8, -1)], 1).double()
+    hist = cv.double()
+    np.testing.assert_array_equal(res["conv"][0], x[2:5].numpy())
+    np.testing.assert_array_equal(res["conv"][1], torch.cat([hist[1, 1:], x[5:6]]).numpy())
+    np.testing.assert_array_equal(res["conv"][2], torch.cat([hist[2, 2:], x[6:8]]).numpy())
+
+
+def test_mixer_causal():
+    case = _small_case([90])
+    base = oracle.mixer(case["inp"], case["cu_seqlens"])["out"]
+    inp = dict(case["inp"])
+    for key in ("q", "k", "v", "z", "a", "b"):
+        inp[key] = inp[key].clone()
+        inp[key][60] = inp[key][60] + 1.0
+    pert = oracle.mixer(inp, case["cu_seqlens"])["out"]
+    np.testing.assert_array_equal(pert[:60], base[:60])
+    assert np.abs(pert[60:] - base[60:]).max() > 0
+
+
+def test_mixer_varlen_equals_solo_runs():
+    case = _small_case([33, 64, 2])
+    st = gin.recurrent_state(3, case["H_v"], seed=2)
+    packed = oracle.mixer(case["inp"], case["cu_seqlens"], state_in=st)
+    cu = case["cu_seqlens"].tolist()
+    for n in range(3):
+        sl = slice(cu[n], cu[n + 1])
+        sub = {k: (v[sl] if k in ("q", "k", "v", "z", "a", "b") else v) for k, v in case["inp"].items()}
+        solo = oracle.mixer(sub, [0, cu[n + 1] - cu[n]], state_in=st[n:n + 1])
+        np.testing.assert_array_equal(packed["out"][sl], solo["out"])
+        np.testing.assert_array_equal(packed["state"][n], solo["state"][0])
+
+
+def test_mixer_identity_gate_through_full_path():
+    """a = -inf, b = -inf (bf16 can hold them): alpha = 1, beta = 0 on every token, so
+    the state is returned unchanged and the pre-norm output is S_0 q_hat."""
+    case = _small_case([40], H_k=1, H_v=3)
+    inp = dict(case["inp"])
+    inp["a"] = torch.full_like(inp["a"], float("-inf"))
+    inp["b"] = torch.full_like(inp["b"], float("-inf"))
+    st = gin.recurrent_state(1, 3, seed=4)
+    res = oracle.mixer(inp, case["cu_seqlens"], state_in=st, want_pre_norm=True)
+    np.testing.assert_array_equal(res["state"], st.double().numpy())
+    # q_hat from library pieces
+    D = gin.D
+    qraw = inp["q"].double().reshape(40, D)
+    w = inp["conv_w"].double()[:D]
+    y = F.silu(F.conv1d(torch.cat([torch.zeros(3, D, dtype=torch.float64), qraw]).T[None], w[:, None, :],
+                        groups=D)[0].T)
+    qh = (y / torch.sqrt((y * y).sum(-1, keepdim=True) + 1e-6)).numpy()
+    for h in range(3):
+        np.testing.assert_allclose(res["pre_norm"][:, h], qh @ st[0, h].double().numpy().T,
+                                   rtol=1e-12, atol=1e-12)

@@ -1,0 +1,224 @@
+// C ABI of the gated-delta-rule mixer: argument validation, workspace layout
+// and kernel launches.  Declared in include/gdn.h.
+#include <limits.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+#include "gdn_kernels.cuh"
+
+using gdn::bf16;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+size_t chunk_base_bytes(int N) { return round_up(sizeof(int) * (static_cast<size_t>(N) + 1), 1024); }
+
+// Common checks of the per-token inputs; T_tot tokens.
+gdn_status check_inputs(const gdn_inputs* in, long long T_tot) {
+  if (!in) return GDN_ERR_INVALID_ARG;
+  if (in->H_k <= 0 || in->H_v <= 0 || in->H_v % in->H_k != 0) return GDN_ERR_INVALID_ARG;
+  if (in->H_v / in->H_k > 8) return GDN_ERR_UNSUPPORTED;
+  if (in->dv_slice != 0 && in->dv_slice != 32 && in->dv_slice != 64 && in->dv_slice != 128)
+    return GDN_ERR_INVALID_ARG;
+  if (in->dv_slice == 128) return GDN_ERR_UNSUPPORTED;
+  if (T_tot == 0) return GDN_OK;
+  if (!in->q || !in->k || !in->v || !in->a || !in->b || !in->z || !in->conv_w || !in->A_log || !in->norm_w)
+    return GDN_ERR_INVALID_ARG;
+  const long long qk = static_cast<long long>(in->H_k) * GDN_HEAD_DIM, vz = static_cast<long long>(in->H_v) * GDN_HEAD_DIM;
+  if (in->stride_q < qk || in->stride_k < qk || in->stride_v < vz || in->stride_z < vz || in->stride_a < in->H_v ||
+      in->stride_b < in->H_v)
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->v) || !aligned16(in->z) || !aligned16(in->conv_w))
+    return GDN_ERR_MISALIGNED;
+  if ((in->stride_q | in->stride_k | in->stride_v | in->stride_z) & 7) return GDN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(in->a) | reinterpret_cast<uintptr_t>(in->b) |
+       reinterpret_cast<uintptr_t>(in->norm_w)) & 1u)
+    return GDN_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(in->A_log) & 3u) return GDN_ERR_MISALIGNED;
+  return GDN_OK;
+}
+
+// `out` must not overlap any input read by the same call
+gdn_status check_out_alias(const gdn_inputs* in, long long T_tot, const void* out) {
+  const size_t ob = static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
+  const size_t tb = sizeof(bf16) * static_cast<size_t>(T_tot);
+  if (overlap(out, ob, in->q, tb * in->stride_q) || overlap(out, ob, in->k, tb * in->stride_k) ||
+      overlap(out, ob, in->v, tb * in->stride_v) || overlap(out, ob, in->z, tb * in->stride_z) ||
+      overlap(out, ob, in->a, tb * in->stride_a) || overlap(out, ob, in->b, tb * in->stride_b))
+    return GDN_ERR_ALIAS;
+  return GDN_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// smallest state-row slice that still fits all scan CTAs in one wave
+int pick_dv(const gdn_inputs* in, int N) {
+  if (in->dv_slice) return in->dv_slice;
+  const long long units = static_cast<long long>(N) * in->H_v;
+  const int sms = sm_count();
+  return units * 4 <= sms ? 32 : 64;
+}
+
+gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long long n_chunks, const int* cu,
+                          int T_uniform, const float* state_in, float* state_out, const void* conv_in,
+                          void* conv_out, void* out, void* workspace, size_t workspace_bytes, int* err,
+                          void* stream) {
+  gdn_status st = check_inputs(in, T_tot);
+  if (st != GDN_OK) return st;
+  if (N == 0) return GDN_OK;
+  if (T_tot > 0 && !out) return GDN_ERR_INVALID_ARG;
+  if (T_tot > 0 && (st = check_out_alias(in, T_tot, out)) != GDN_OK) return st;
+  const long long C_conv = static_cast<long long>(2 * in->H_k + in->H_v) * GDN_HEAD_DIM;
+  const size_t state_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(N) * 3 * C_conv * sizeof(bf16);
+  if (!aligned16(out) || !aligned16(state_in) || !aligned16(state_out) || !aligned16(conv_in) ||
+      !aligned16(conv_out) || !aligned16(workspace))
+    return GDN_ERR_MISALIGNED;
+  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
+    return GDN_ERR_ALIAS;
+  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
+  if (state_out && overlap(state_out, state_bytes, out, static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * 2))
+    return GDN_ERR_ALIAS;
+  const size_t need = gdn_prefill_workspace_size(in->H_k, in->H_v, N, n_chunks);
+  if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  gdn::PrefillParams p = {};
+  p.q = static_cast<const bf16*>(in->q);
+  p.k = static_cast<const bf16*>(in->k);
+  p.v = static_cast<const bf16*>(in->v);
+  p.a = static_cast<const bf16*>(in->a);
+  p.b = static_cast<const bf16*>(in->b);
+  p.z = static_cast<const bf16*>(in->z);
+  p.sq = in->stride_q; p.sk = in->stride_k; p.sv = in->stride_v; p.sz = in->stride_z;
+  p.sa = in->stride_a; p.sb = in->stride_b;
+  p.conv_w = static_cast<const bf16*>(in->conv_w);
+  p.A_log = in->A_log;
+  p.norm_w = static_cast<const bf16*>(in->norm_w);
+  p.scale = in->scale;
+  p.H_k = in->H_k;
+  p.H_v = in->H_v;
+  p.N = N;
+  p.cu = cu;
+  p.T_uniform = T_uniform;
+  p.n_chunks = n_chunks;
+  p.ws_flag = reinterpret_cast<int*>(ws);
+  p.chunk_base = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) : nullptr;
+  p.ws_qk = ws + gdn::kWsHeader + chunk_base_bytes(N);
+  p.ws_head = p.ws_qk + static_cast<size_t>(n_chunks) * in->H_k * gdn::kQKBytes;
+  p.state_in = state_in;
+  p.state_out = state_out;
+  p.conv_in = static_cast<const bf16*>(conv_in);
+  p.conv_out = static_cast<bf16*>(conv_out);
+  p.out = static_cast<bf16*>(out);
+  p.err = err;
+  cudaError_t e = gdn::launch_prefill(p, pick_dv(in, N), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks) {
+  if (H_k <= 0 || H_v <= 0 || N < 0 || n_chunks < 0) return 0;
+  return gdn::kWsHeader + chunk_base_bytes(N) +
+         static_cast<size_t>(n_chunks) * (static_cast<size_t>(H_k) * gdn::kQKBytes +
+                                          static_cast<size_t>(H_v) * gdn::kHeadBytes);
+}
+
+gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
+                       const void* conv_in, void* conv_out, void* out, void* workspace, size_t workspace_bytes,
+                       int* err, void* stream) {
+  if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
+  const long long n_chunks = static_cast<long long>(B) * ((T + GDN_CHUNK - 1) / GDN_CHUNK);
+  return prefill_common(in, B, T_tot, n_chunks, nullptr, T, state_in, state_out, conv_in, conv_out, out, workspace,
+                        workspace_bytes, err, stream);
+}
+
+gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens, const int* cu_seqlens_host,
+                              const float* state_in, float* state_out, const void* conv_in, void* conv_out,
+                              void* out, void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  if (N < 0) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return check_inputs(in, 0);
+  if (!cu_seqlens || !cu_seqlens_host) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens_host[0] != 0) return GDN_ERR_INVALID_ARG;
+  long long n_chunks = 0;
+  for (int n = 0; n < N; ++n) {
+    const long long L = static_cast<long long>(cu_seqlens_host[n + 1]) - cu_seqlens_host[n];
+    if (L < 0) return GDN_ERR_INVALID_ARG;
+    n_chunks += (L + GDN_CHUNK - 1) / GDN_CHUNK;
+  }
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return GDN_ERR_MISALIGNED;
+  return prefill_common(in, N, cu_seqlens_host[N], n_chunks, cu_seqlens, 0, state_in, state_out, conv_in, conv_out,
+                        out, workspace, workspace_bytes, err, stream);
+}
+
+gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out, int* err,
+                           void* stream) {
+  if (N < 0) return GDN_ERR_INVALID_ARG;
+  gdn_status st = check_inputs(in, N);
+  if (st != GDN_OK || N == 0) return st;
+  if (!state || !conv_state || !out) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(state) || !aligned16(conv_state) || !aligned16(out)) return GDN_ERR_MISALIGNED;
+  if ((st = check_out_alias(in, N, out)) != GDN_OK) return st;
+  const long long C_conv = static_cast<long long>(2 * in->H_k + in->H_v) * GDN_HEAD_DIM;
+  const size_t state_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(N) * 3 * C_conv * sizeof(bf16);
+  const size_t out_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
+  if (overlap(state, state_bytes, conv_state, conv_bytes) || overlap(state, state_bytes, out, out_bytes) ||
+      overlap(conv_state, conv_bytes, out, out_bytes))
+    return GDN_ERR_ALIAS;
+  gdn::DecodeParams p = {};
+  p.q = static_cast<const bf16*>(in->q);
+  p.k = static_cast<const bf16*>(in->k);
+  p.v = static_cast<const bf16*>(in->v);
+  p.a = static_cast<const bf16*>(in->a);
+  p.b = static_cast<const bf16*>(in->b);
+  p.z = static_cast<const bf16*>(in->z);
+  p.sq = in->stride_q; p.sk = in->stride_k; p.sv = in->stride_v; p.sz = in->stride_z;
+  p.sa = in->stride_a; p.sb = in->stride_b;
+  p.conv_w = static_cast<const bf16*>(in->conv_w);
+  p.A_log = in->A_log;
+  p.norm_w = static_cast<const bf16*>(in->norm_w);
+  p.scale = in->scale;
+  p.H_k = in->H_k;
+  p.H_v = in->H_v;
+  p.N = N;
+  p.state = state;
+  p.conv_state = static_cast<bf16*>(conv_state);
+  p.out = static_cast<bf16*>(out);
+  p.err = err;
+  return gdn::launch_decode(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+const char* gdn_status_string(gdn_status status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: null pointer, bad count or bad shape";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: request outside what this build implements";
+    case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointer or stride not suitably aligned";
+    case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: buffers that must be distinct overlap";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA launch failed";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a device-side wait timed out";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "unknown gdn_status";
+}
+
+}  // extern "C"

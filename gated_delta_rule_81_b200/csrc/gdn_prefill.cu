@@ -1,0 +1,949 @@
+// Chunked prefill of the gated-delta-rule mixer on sm_100a.
+//
+// Method: Agnes-3.0-Flash model card, "Architecture" table, row "Delta-rule
+// layers" (16 key / 48 value heads, head dim 128, causal conv kernel 4 in
+// front, gated RMS-norm after, fp32 recurrent state) and the kongchang
+// article's paragraph on the Gated Delta Rule (erase-then-write under a forget
+// gate).  Recurrence: S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T,
+// o_t = S_t q_t, evaluated 64 tokens at a time in its chunkwise (UT-transform)
+// form.  Inside a chunk that starts from state S (d_v x d_k), with G the
+// inclusive cumulative sum of g = log a, gamma_i = e^{G_i}:
+//   A_ij = b_i e^{G_i - G_j} (k_i . k_j) (j < i),   T = (I + A)^{-1},
+//   T~ = T diag(b),   P_ij = e^{G_i - G_j} (q_i . k_j) (j <= i),
+//   R = V - diag(gamma) K S^T,   U = T~ R,   O = diag(gamma) Q S^T + P T~ R,
+//   S^T <- gamma_C S^T + K^T diag(e^{G_C - G_j}) U.
+//
+// Two kernels (plus two small helpers):
+//   prep (one CTA per chunk x key head, all chunks in parallel): conv + SiLU +
+//     L2-norm front end, gates, [Q;K] K^T on tcgen05, the fp32 blocked
+//     triangular solve, and [P;I] T~ on tcgen05.  It writes the chunk's
+//     operand images to the workspace.
+//   scan (one CTA, or a cluster of 2 or 4 CTAs, per sequence x value head;
+//     each CTA owns 128/cluster value rows of the state): walks the chunks in
+//     order with S^T resident in tensor memory.  Per chunk three tcgen05 MMAs
+//     ([Q;K] S^T, [P T~; T~] R, K^T U) and the gated RMS-norm epilogue.
+#include "gdn_kernels.cuh"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kDevErrBadSeqlens = 4;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ long long seq_start(const PrefillParams& p, int n) {
+  return p.cu ? static_cast<long long>(p.cu[n]) : static_cast<long long>(n) * p.T_uniform;
+}
+
+__device__ __forceinline__ long long chunk_base_of(const PrefillParams& p, int n) {
+  return p.chunk_base ? static_cast<long long>(p.chunk_base[n])
+                      : static_cast<long long>(n) * ((p.T_uniform + kChunk - 1) / kChunk);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_shared_remote(const float* p, uint32_t cta) {
+  uint32_t local = smem_u32(p), remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(cta));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// unpack 8 bf16 from a uint4
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+// ============================================================ helpers
+
+// chunk_base[n] = sum_{m<n} ceil(L_m / 64) from the device cu_seqlens; checks
+// that it agrees with the host-side count and that cu_seqlens is valid.
+__global__ void __launch_bounds__(1024) setup_kernel(PrefillParams p) {
+  __shared__ long long part[1024];
+  __shared__ int bad_s;
+  const int tid = threadIdx.x;
+  if (tid == 0) bad_s = (p.cu[0] != 0);
+  __syncthreads();
+  const int per = (p.N + 1023) / 1024;
+  const int n0 = min(tid * per, p.N), n1 = min(n0 + per, p.N);
+  long long acc = 0;
+  int bad = 0;
+  for (int n = n0; n < n1; ++n) {
+    const int L = p.cu[n + 1] - p.cu[n];
+    if (L < 0) bad = 1;
+    acc += L > 0 ? (L + kChunk - 1) / kChunk : 0;
+  }
+  if (bad) atomicOr(&bad_s, 1);
+  part[tid] = acc;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan
+    const long long v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  long long base = part[tid] - acc;
+  for (int n = n0; n < n1; ++n) {
+    p.chunk_base[n] = static_cast<int>(base);
+    const int L = p.cu[n + 1] - p.cu[n];
+    base += L > 0 ? (L + kChunk - 1) / kChunk : 0;
+  }
+  if (tid == 1023) {
+    p.chunk_base[p.N] = static_cast<int>(part[1023]);
+    if (part[1023] != p.n_chunks) atomicOr(&bad_s, 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    *p.ws_flag = bad_s;
+    if (bad_s && p.err) atomicOr(p.err, kDevErrBadSeqlens);
+  }
+}
+
+// raw (pre-conv) value of conv channel c at token tau (tau inside the packed batch)
+__device__ __forceinline__ bf16 raw_channel(const PrefillParams& p, long long tau, long long c) {
+  const long long qk = static_cast<long long>(p.H_k) * kD;
+  if (c < qk) return p.q[tau * p.sq + c];
+  if (c < 2 * qk) return p.k[tau * p.sk + (c - qk)];
+  return p.v[tau * p.sv + (c - 2 * qk)];
+}
+
+// conv_out[n][j][c] = raw channel c at token end-3+j (history from conv_in before the start)
+__global__ void conv_out_kernel(PrefillParams p) {
+  const int n = blockIdx.y;
+  const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
+  const long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= C_conv) return;
+  if (p.cu && *p.ws_flag) return;
+  const long long s = seq_start(p, n), e = seq_start(p, n + 1);
+  for (int j = 0; j < 3; ++j) {
+    const long long tau = e - 3 + j;
+    bf16 val;
+    if (tau >= s) val = raw_channel(p, tau, c);
+    else if (p.conv_in) val = p.conv_in[(static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + c];
+    else val = __float2bfloat16(0.f);
+    p.conv_out[(static_cast<long long>(n) * 3 + j) * C_conv + c] = val;
+  }
+}
+
+// ============================================================ prep kernel
+
+constexpr int kPrepThreads = 256;
+constexpr int kLdA = 65;                               // fp32 row stride of A / T in shared memory
+constexpr int kPrepOffQK = 0;                          // [Q;K] image hi, lo    2 x 32768
+constexpr int kPrepOffPI = kPrepOffQK + 2 * 32768;     // [P;I] image hi, lo    2 x 16384
+constexpr int kPrepOffTt = kPrepOffPI + 2 * 16384;     // T~ image (B) hi, lo   2 x 8192
+constexpr int kPrepOffA = kPrepOffTt + 2 * 8192;       // A fp32                64*65*4
+constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32
+constexpr int kPrepOffM = kPrepOffT + 64 * kLdA * 4;   // block-solve temp      3*256*4
+constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum [8][64]
+constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta     [8][64]
+constexpr int kPrepSmem = kPrepOffB + 8 * 64 * 4 + 1024;
+
+// hi = bf16(f), lo = bf16(f - hi) for 8 values
+__device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    h[e] = __bfloat162float(__float2bfloat16(f[e]));
+    l[e] = f[e] - h[e];
+  }
+  hi = pack8(h);
+  lo = pack8(l);
+}
+
+// Conv (4 taps) + SiLU of 32 consecutive channels of one token.
+//   src: the token-0 address of the group's first channel; rows before the
+//   sequence start come from conv_in (or are zero).
+__device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, long long src_stride,
+                                       long long s, long long t, int n, long long conv_chan0, float* y) {
+  const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) y[e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kTaps; ++j) {
+    const long long tau = t - (kTaps - 1) + j;
+    const uint4* row = nullptr;
+    if (tau >= s) row = reinterpret_cast<const uint4*>(src + tau * src_stride);
+    else if (p.conv_in)
+      row = reinterpret_cast<const uint4*>(p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv +
+                                           conv_chan0);
+    if (row == nullptr) continue;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float x[8];
+      unpack8(__ldg(row + g), x);
+      const bf16* w = p.conv_w + (conv_chan0 + 8 * g) * kTaps + j;  // tap j of channels 8g .. 8g+7
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[8 * g + e] = fmaf(__bfloat162float(w[e * kTaps]), x[e], y[8 * g + e]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) y[e] = silu_f(y[e]);
+}
+
+// T = (I + A)^{-1} for a 64x64 strictly-lower A (fp32, shared memory), by 16x16
+// blocks: diagonal blocks by forward substitution, then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+// one block diagonal at a time.  All 256 threads.
+__device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid) {
+  if (tid < 64) {
+    const int blk = tid >> 4, col = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int l = 0; l < r; ++l) acc = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + l], x[l], acc);
+      x[r] = r < col ? 0.f : (r == col ? 1.f : -acc);
+      sT[(16 * blk + r) * kLdA + 16 * blk + col] = x[r];
+    }
+  }
+  __syncthreads();
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;
+    for (int x = tid; x < nb * 256; x += kPrepThreads) {
+      const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
+      float acc = 0.f;
+      for (int kk = 16 * J; kk < 16 * I; ++kk) acc = fmaf(sA[(16 * I + ii) * kLdA + kk], sT[kk * kLdA + 16 * J + jj], acc);
+      sM[x] = acc;
+    }
+    __syncthreads();
+    for (int x = tid; x < nb * 256; x += kPrepThreads) {
+      const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
+      float acc = 0.f;
+      for (int l = 0; l <= ii; ++l) acc = fmaf(sT[(16 * I + ii) * kLdA + 16 * I + l], sM[(J << 8) + (l << 4) + jj], acc);
+      sT[(16 * I + ii) * kLdA + 16 * J + jj] = -acc;
+    }
+    __syncthreads();
+  }
+}
+
+// D (+)= A B^T with both operands as hi/lo pairs: A_hi B_hi + A_hi B_lo + A_lo B_hi
+__device__ __forceinline__ void umma_split(uint32_t d, uint64_t a_hi, uint64_t a_lo, uint64_t b_hi, uint64_t b_lo,
+                                           uint32_t idesc, bool accumulate) {
+  umma_bf16(d, a_hi, b_hi, idesc, accumulate);
+  umma_bf16(d, a_hi, b_lo, idesc, true);
+  umma_bf16(d, a_lo, b_hi, idesc, true);
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) {
+  if (p.cu && *p.ws_flag) return;
+  extern __shared__ uint8_t prep_smem_raw[];
+  uint8_t* sm = align1024(prep_smem_raw);
+  uint8_t* sQK = sm + kPrepOffQK;   // hi at +0, lo at +32768
+  uint8_t* sPI = sm + kPrepOffPI;   // hi at +0, lo at +16384
+  uint8_t* sTt = sm + kPrepOffTt;   // hi at +0, lo at +8192
+  float* sA = reinterpret_cast<float*>(sm + kPrepOffA);
+  float* sT = reinterpret_cast<float*>(sm + kPrepOffT);
+  float* sM = reinterpret_cast<float*>(sm + kPrepOffM);
+  float* sG = reinterpret_cast<float*>(sm + kPrepOffG);
+  float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
+  __shared__ uint64_t bar[3];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long gc = blockIdx.x;
+  const int kh = blockIdx.y;
+  const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k;
+
+  // sequence of this chunk: the largest n with chunk_base(n) <= gc
+  int n;
+  if (p.chunk_base) {
+    int lo = 0, hi = p.N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.chunk_base[mid] <= gc) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+  } else {
+    n = static_cast<int>(gc / ((p.T_uniform + kChunk - 1) / kChunk));
+  }
+  const long long s = seq_start(p, n), e = seq_start(p, n + 1);
+  const long long t0 = s + (gc - chunk_base_of(p, n)) * kChunk;
+  const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - t0));
+
+  Abort ab{p.err, &abort_s};
+  if (tid == 0) {
+    abort_s = 0;
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_init(&bar[2], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc<128>(&tmem_base_s);
+
+  // identity rows 64..127 of the [P; I] image (hi = I, lo = 0)
+  for (int x = tid; x < 64 * 8; x += kPrepThreads) {
+    const int i = x >> 3, cc = x & 7;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (cc == (i >> 3)) {
+      const int e8 = i & 7;
+      w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
+    }
+    *reinterpret_cast<uint4*>(sPI + sw128_off(64 + i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(sPI + 16384 + sw128_off(64 + i, cc)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  // ---- front end of q and k: token i, channels 32*qq .. 32*qq+31
+  uint8_t* gQK = p.ws_qk + (gc * H_k + kh) * static_cast<long long>(kQKBytes);
+  {
+    const int i = tid >> 2, qq = tid & 3;
+    const bool valid = i < L;
+    for (int which = 0; which < 2; ++which) {
+      const bf16* X = which ? p.k : p.q;
+      const long long sx = which ? p.sk : p.sq;
+      const long long chan0 = static_cast<long long>(which) * H_k * kD + static_cast<long long>(kh) * kD + 32 * qq;
+      float y[32];
+      if (valid) conv32(p, X + static_cast<long long>(kh) * kD + 32 * qq, sx, s, t0 + i, n, chan0, y);
+      float ss = 0.f;
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) {
+        if (!valid) y[e2] = 0.f;
+        ss = fmaf(y[e2], y[e2], ss);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      const float inv = rsqrtf(ss + 1e-6f) * (which == 0 ? p.scale : 1.0f);
+      const int row = which * 64 + i, kb = qq >> 1;
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float f[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) f[e2] = y[8 * c2 + e2] * inv;
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t off = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
+        *reinterpret_cast<uint4*>(sQK + off) = hi;
+        *reinterpret_cast<uint4*>(sQK + kQKImg + off) = lo;
+        *reinterpret_cast<uint4*>(gQK + off) = hi;
+        *reinterpret_cast<uint4*>(gQK + kQKImg + off) = lo;
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+
+  // ---- [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
+  if (tid == 0) {
+    const uint32_t qh = smem_u32(sQK), ql = qh + kQKImg;
+    const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
+      umma_split(tbase, smem_desc(qh + ko, 16, 1024, Swz::k128), smem_desc(ql + ko, 16, 1024, Swz::k128),
+                 smem_desc(qh + ko + 8192, 16, 1024, Swz::k128), smem_desc(ql + ko + 8192, 16, 1024, Swz::k128),
+                 idesc, ks > 0);
+    }
+    umma_commit(&bar[0]);
+  }
+
+  // ---- gates of the key head's value heads (overlaps the MMA)
+  for (int base = 0; base < G * 64; base += kPrepThreads) {
+    const int x = base + tid;
+    if (x < G * 64) {  // warp-uniform: G*64 is a multiple of 64
+      const int j = x >> 6, i = x & 63, h = kh * G + j;
+      const bool valid = i < L;
+      float g = 0.f, beta = 0.f;
+      if (valid) {
+        const long long t = t0 + i;
+        g = -expf(p.A_log[h]) * softplus_f(__bfloat162float(p.a[t * p.sa + h]));
+        beta = sigmoid_f(__bfloat162float(p.b[t * p.sb + h]));
+      }
+      float v = g;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      sG[j * 64 + i] = v;
+      sB[j * 64 + i] = beta;
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < G * 32; x += kPrepThreads) {
+    const int j = x >> 5, i = 32 + (x & 31);
+    sG[j * 64 + i] += sG[j * 64 + 31];
+  }
+  __syncthreads();
+  // gate vectors for the scan: gamma_i, decay-to-end_i, gamma_C
+  for (int x = tid; x < G * 256; x += kPrepThreads) {
+    const int j = x >> 8, k2 = x & 255, h = kh * G + j;
+    const float Glast = sG[j * 64 + (L - 1)];
+    float val = 0.f;
+    if (k2 < 64) val = expf(sG[j * 64 + k2]);
+    else if (k2 < 128) val = (k2 - 64) < L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
+    else if (k2 == 128) val = expf(Glast);
+    float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes + kVBytes);
+    gdst[k2] = val;
+  }
+  // ---- v_hat of the value heads (fp32): token i, channels 32*qq..+31, stored [4 column blocks][64][32]
+  {
+    const int i = tid >> 2, qq = tid & 3;
+    const bool valid = i < L;
+    for (int j = 0; j < G; ++j) {
+      const int h = kh * G + j;
+      float y[32];
+      if (valid) {
+        conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,
+               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, y);
+      } else {
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
+      }
+      float4* dst = reinterpret_cast<float4*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes +
+                                              (qq * 64 + i) * 128);
+#pragma unroll
+      for (int c2 = 0; c2 < 8; ++c2) dst[c2] = make_float4(y[4 * c2], y[4 * c2 + 1], y[4 * c2 + 2], y[4 * c2 + 3]);
+    }
+  }
+
+  // ---- K K^T and Q K^T rows into registers: thread row = 32*(warp%4)+lane, columns cbase..cbase+31
+  const int row = 32 * (warp & 3) + lane;
+  const int cbase = 32 * (warp >> 2);
+  const bool isQ = row < 64;
+  const int ri = row & 63;
+  float acc[32];
+  if (mbar_wait_warp(&bar[0], 0, ab)) {
+    tc_fence_after();
+    tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), cbase), acc);
+    tmem_wait_ld();
+  } else {
+#pragma unroll
+    for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
+  }
+
+  for (int j = 0; j < G; ++j) {
+    const int h = kh * G + j;
+    const float Gi = sG[j * 64 + ri];
+    if (!isQ) {
+      const float bi = sB[j * 64 + ri];
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) {
+        const int col = cbase + e2;
+        sA[ri * kLdA + col] = col < ri ? bi * expf(Gi - sG[j * 64 + col]) * acc[e2] : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float f[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const int col = cbase + 8 * c2 + e2;
+          f[e2] = col <= ri ? expf(Gi - sG[j * 64 + col]) * acc[8 * c2 + e2] : 0.f;
+        }
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        *reinterpret_cast<uint4*>(sPI + sw128_off(ri, (cbase >> 3) + c2)) = hi;
+        *reinterpret_cast<uint4*>(sPI + 16384 + sw128_off(ri, (cbase >> 3) + c2)) = lo;
+      }
+    }
+    __syncthreads();
+    solve_unit_lower(sA, sT, sM, tid);
+    // T~ = T diag(beta): lower triangle incl. diagonal, as the MN-major B operand (row = k index)
+    for (int x = tid; x < 64 * 8; x += kPrepThreads) {
+      const int r = x >> 3, cc = x & 7;
+      float f[8];
+#pragma unroll
+      for (int e2 = 0; e2 < 8; ++e2) {
+        const int col = 8 * cc + e2;
+        f[e2] = col <= r ? sT[r * kLdA + col] * sB[j * 64 + col] : 0.f;
+      }
+      uint4 hi, lo;
+      split8(f, hi, lo);
+      *reinterpret_cast<uint4*>(sTt + sw128_off(r, cc)) = hi;
+      *reinterpret_cast<uint4*>(sTt + 8192 + sw128_off(r, cc)) = lo;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t pih = smem_u32(sPI), pil = pih + 16384, tth = smem_u32(sTt), ttl = tth + 8192;
+      const uint32_t idesc = idesc_bf16(128, 64, false, true);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_split(tbase + 64, smem_desc(pih + ks * 32, 16, 1024, Swz::k128),
+                   smem_desc(pil + ks * 32, 16, 1024, Swz::k128), smem_desc(tth + ks * 2048, 8192, 1024, Swz::k128),
+                   smem_desc(ttl + ks * 2048, 8192, 1024, Swz::k128), idesc, ks > 0);
+      umma_commit(&bar[1]);
+    }
+    __syncwarp();
+    float o[32];
+    if (mbar_wait_warp(&bar[1], j & 1, ab)) {
+      tc_fence_after();
+      tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), 64 + cbase), o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) o[e2] = 0.f;
+    }
+    uint8_t* dst = p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes);
+#pragma unroll
+    for (int c2 = 0; c2 < 4; ++c2) {
+      uint4 hi, lo;
+      split8(o + 8 * c2, hi, lo);
+      const uint32_t off = sw128_off(row, (cbase >> 3) + c2);
+      *reinterpret_cast<uint4*>(dst + off) = hi;
+      *reinterpret_cast<uint4*>(dst + kPTImg + off) = lo;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  // drain: every MMA this CTA issued has completed before TMEM is released
+  if (tid == 0) {
+    umma_commit(&bar[2]);
+    int drain_flag = 0;
+    Abort drain{nullptr, &drain_flag};
+    mbar_wait(&bar[2], 0, drain);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc<128>(tbase);
+}
+
+// ============================================================ scan kernel
+
+template <int DV>
+struct ScanCfg {
+  static constexpr int CS = 128 / DV;                  // CTAs per value head (cluster size)
+  static constexpr int NB = DV / 32;                   // 32-column blocks per CTA
+  static constexpr int TMEM_COLS = DV == 32 ? 256 : 512;
+  static constexpr int COL_Z = 0;                      // S^T: lanes = d_k, DV columns
+  static constexpr int COL_X = DV;                     // X[b] = [Q;K] S^T at DV + 2 DV b
+  static constexpr int COL_Y = 2 * DV;                 // Y[b] = [P T~; T~] R at 2 DV + 2 DV b
+  // shared memory (offsets from a 1024-aligned base)
+  static constexpr int OFF_GATE = kQKBytes;            // inside a [Q;K] stage
+  static constexpr int QK_STAGE = kQKBytes + kGateBytes;
+  static constexpr int OFF_PT = 2 * QK_STAGE;          // single [P T~; T~] buffer, hi then lo
+  static constexpr int OFF_V = OFF_PT + kPTBytes;      // single v_hat slice, fp32 [DV/32][64][32]
+  static constexpr int V_BYTES = 64 * DV * 4;
+  static constexpr int OFF_OP = OFF_V + V_BYTES;       // S, R and U operands (hi image, then lo image)
+  static constexpr int OP_IMG = 128 * DV * 2;
+  static constexpr int OFF_NW = OFF_OP + 2 * OP_IMG;   // norm weight slice, fp32 [DV]
+  static constexpr int OFF_SS = OFF_NW + 512;          // RMS partials [2][4][64] fp32
+  static constexpr int SMEM = OFF_SS + 2048 + 1024;
+  static constexpr uint32_t QK_TX = kQKBytes + kGateBytes;
+};
+
+// MN-major operand image with DV columns (8-element chunk index nch) and `krows` K-rows
+template <int DV>
+__device__ __forceinline__ uint32_t mn_off(uint32_t krow, uint32_t nch, uint32_t krows) {
+  if constexpr (DV == 32) return sw64_off(krow, nch);
+  else return (nch >> 3) * (krows * 128u) + sw128_off(krow, nch & 7u);
+}
+
+template <int DV>
+__device__ __forceinline__ uint64_t mn_desc(uint32_t base, int ks, uint32_t krows) {
+  if constexpr (DV == 32) return smem_desc(base + ks * 1024u, 512, 512, Swz::k64);
+  else return smem_desc(base + ks * 2048u, krows * 128u, 1024, Swz::k128);
+}
+
+// write 32 fp32 values (one thread's row segment, columns 32*cc..) as hi/lo bf16 into an MN-major image
+template <int DV>
+__device__ __forceinline__ void store_split_row(uint8_t* img_hi, int img_bytes, uint32_t krow, int cc, uint32_t krows,
+                                                const float* v) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 hi, lo;
+    split8(v + 8 * q4, hi, lo);
+    const uint32_t off = mn_off<DV>(krow, 4 * cc + q4, krows);
+    *reinterpret_cast<uint4*>(img_hi + off) = hi;
+    *reinterpret_cast<uint4*>(img_hi + img_bytes + off) = lo;
+  }
+}
+
+template <int DV>
+__global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
+  using Cfg = ScanCfg<DV>;
+  constexpr int CS = Cfg::CS, NB = Cfg::NB;
+  if (p.cu && *p.ws_flag) return;  // same value in every CTA of a cluster
+  extern __shared__ uint8_t scan_smem_raw[];
+  uint8_t* sm = align1024(scan_smem_raw);
+  __shared__ uint64_t qk_full[2], qk_empty[2], xyfree_b[2], mma2o_b[2], nfull_b[2], nack_b[2];
+  __shared__ uint64_t pt_full, pt_empty, v_full, v_empty;
+  __shared__ uint64_t sready_b, mma1_b, rready_b, mma2_b, uready_b, mma3_b, drain_b;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
+  const int unit = blockIdx.x / CS;
+  const int n = unit / p.H_v, h = unit % p.H_v;
+  const int G = p.H_v / p.H_k, kh = h / G;
+  const int slice = static_cast<int>(rank);
+  const long long s = seq_start(p, n), e = seq_start(p, n + 1);
+  const int nc = static_cast<int>((e - s + kChunk - 1) / kChunk);
+  const long long cb = chunk_base_of(p, n);
+
+  Abort ab{p.err, &abort_s};
+  float* sNW = reinterpret_cast<float*>(sm + Cfg::OFF_NW);
+  float* sSS = reinterpret_cast<float*>(sm + Cfg::OFF_SS);
+  uint8_t* sOP = sm + Cfg::OFF_OP;
+  if (tid == 0) {
+    abort_s = 0;
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&qk_full[b], 1);
+      mbar_init(&qk_empty[b], 1 + 64);
+      mbar_init(&xyfree_b[b], 64);
+      mbar_init(&mma2o_b[b], 1);
+      if (CS > 1) {
+        mbar_init(&nfull_b[b], (CS - 1) * 64);
+        mbar_init(&nack_b[b], (CS - 1) * 64);
+      }
+    }
+    mbar_init(&pt_full, 1);
+    mbar_init(&pt_empty, 1);
+    mbar_init(&v_full, 1);
+    mbar_init(&v_empty, 64);
+    mbar_init(&sready_b, 128);
+    mbar_init(&mma1_b, 1);
+    mbar_init(&rready_b, 64);
+    mbar_init(&mma2_b, 1);
+    mbar_init(&uready_b, 64);
+    mbar_init(&mma3_b, 1);
+    mbar_init(&drain_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 7) tmem_alloc<Cfg::TMEM_COLS>(&tmem_base_s);
+  if (tid < DV) sNW[tid] = __bfloat162float(p.norm_w[slice * DV + tid]);
+  tc_fence_before();
+  __syncthreads();
+  if (CS > 1) cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+  const uint32_t op_hi = smem_u32(sOP), op_lo = op_hi + Cfg::OP_IMG;
+
+  if (warp == 6) {
+    // ------------------------------------------------ bulk-copy producer
+    if (lane == 0) {
+      int qk_issued[2] = {0, 0}, pt_issued = 0, v_issued = 0;
+      for (int c = 0; c < nc; ++c) {
+        const int st = c & 1;
+        const long long gc = cb + c;
+        const uint8_t* hb = p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes);
+        uint8_t* stage = sm + st * Cfg::QK_STAGE;
+        if (c >= 2 && !mbar_wait(&qk_empty[st], ((c >> 1) - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&qk_full[st], Cfg::QK_TX);
+        bulk_g2s(stage, p.ws_qk + (gc * p.H_k + kh) * static_cast<long long>(kQKBytes), kQKBytes, &qk_full[st]);
+        bulk_g2s(stage + Cfg::OFF_GATE, hb + kPTBytes + kVBytes, kGateBytes, &qk_full[st]);
+        ++qk_issued[st];
+        if (c >= 1 && !mbar_wait(&pt_empty, (c - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&pt_full, kPTBytes);
+        bulk_g2s(sm + Cfg::OFF_PT, hb, kPTBytes, &pt_full);
+        ++pt_issued;
+        if (c >= 1 && !mbar_wait(&v_empty, (c - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&v_full, Cfg::V_BYTES);
+        bulk_g2s(sm + Cfg::OFF_V, hb + kPTBytes + slice * Cfg::V_BYTES, Cfg::V_BYTES, &v_full);
+        ++v_issued;
+      }
+      // drain copies still in flight (only possible after an abort)
+      int drain_flag = 0;
+      Abort drain{nullptr, &drain_flag};
+      for (int st = 0; st < 2; ++st)
+        if (qk_issued[st] > 0) mbar_wait(&qk_full[st], (qk_issued[st] - 1) & 1, drain);
+      if (pt_issued > 0) mbar_wait(&pt_full, (pt_issued - 1) & 1, drain);
+      if (v_issued > 0) mbar_wait(&v_full, (v_issued - 1) & 1, drain);
+    }
+    __syncwarp();
+  } else if (warp == 7) {
+    // ------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      const uint32_t idesc_xs = idesc_bf16(128, DV, false, true);
+      const uint32_t idesc_ku = idesc_bf16(128, DV, true, true);
+      const uint32_t pt_hi = smem_u32(sm + Cfg::OFF_PT), pt_lo = pt_hi + kPTImg;
+      for (int c = 0; c < nc; ++c) {
+        const int st = c & 1, xb = c & 1;
+        if (!mbar_wait(&qk_full[st], (c >> 1) & 1, ab)) break;
+        if (!mbar_wait(&sready_b, c & 1, ab)) break;
+        if (c >= 2 && !mbar_wait(&xyfree_b[xb], ((c >> 1) - 1) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t qk_hi = smem_u32(sm + st * Cfg::QK_STAGE), qk_lo = qk_hi + kQKImg;
+        const uint32_t dX = tbase + Cfg::COL_X + 2 * DV * xb, dY = tbase + Cfg::COL_Y + 2 * DV * xb;
+        // X = [Q;K] S^T
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
+          umma_split(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), smem_desc(qk_lo + ko, 16, 1024, Swz::k128),
+                     mn_desc<DV>(op_hi, ks, 128), mn_desc<DV>(op_lo, ks, 128), idesc_xs, ks > 0);
+        }
+        umma_commit(&mma1_b);
+        if (!mbar_wait(&rready_b, c & 1, ab)) break;
+        if (!mbar_wait(&pt_full, c & 1, ab)) break;
+        tc_fence_after();
+        // Y = [P T~; T~] R
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_split(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128),
+                     mn_desc<DV>(op_hi, ks, 64), mn_desc<DV>(op_lo, ks, 64), idesc_xs, ks > 0);
+        umma_commit(&mma2_b);
+        umma_commit(&mma2o_b[xb]);
+        umma_commit(&pt_empty);
+        if (!mbar_wait(&uready_b, c & 1, ab)) break;
+        tc_fence_after();
+        // S^T += K^T U_d
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_split(tbase + Cfg::COL_Z, smem_desc(qk_hi + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
+                     smem_desc(qk_lo + 8192u + ks * 2048u, 16384, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64),
+                     mn_desc<DV>(op_lo, ks, 64), idesc_ku, true);
+        umma_commit(&mma3_b);
+        umma_commit(&qk_empty[st]);
+      }
+      umma_commit(&drain_b);
+      int drain_flag = 0;
+      Abort drain{nullptr, &drain_flag};
+      mbar_wait(&drain_b, 0, drain);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------ state (threads 0..127) and chain (64..127)
+    const int t = tid;  // TMEM lane = d_k index
+    const uint32_t lb = 32 * warp;
+    const long long srow0 = (static_cast<long long>(n) * p.H_v + h) * kD + static_cast<long long>(slice) * DV;
+    bool ok = true;
+    for (int c = 0; c < nc && ok; ++c) {
+      const int st = c & 1, xb = c & 1;
+      const float* gates = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE);
+      if (c > 0) {
+        if (!(ok = mbar_wait_warp(&mma3_b, (c - 1) & 1, ab))) break;
+        tc_fence_after();
+      }
+      if (!(ok = mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab))) break;
+      const float gC = gates[128];
+#pragma unroll
+      for (int cc = 0; cc < NB; ++cc) {
+        float v[32];
+        if (c == 0) {
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2)
+            v[e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
+        } else {
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
+          tmem_wait_ld();
+        }
+        store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v);
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) v[e2] *= gC;
+        tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sready_b);
+      if (t >= 64) {
+        const int i = t - 64;
+        if (!(ok = mbar_wait_warp(&mma1_b, c & 1, ab))) break;
+        if (!(ok = mbar_wait_warp(&v_full, c & 1, ab))) break;
+        tc_fence_after();
+        const float gam = gates[i];
+        const float4* vrow = reinterpret_cast<const float4*>(sm + Cfg::OFF_V);
+        // R = v_hat - gamma (K S^T), into the operand buffer (S is no longer needed)
+#pragma unroll
+        for (int cc = 0; cc < NB; ++cc) {
+          float x[32];
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 2 * DV * xb + 32 * cc), x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 vv = vrow[(cc * 64 + i) * 8 + q];
+            x[4 * q + 0] = fmaf(-gam, x[4 * q + 0], vv.x);
+            x[4 * q + 1] = fmaf(-gam, x[4 * q + 1], vv.y);
+            x[4 * q + 2] = fmaf(-gam, x[4 * q + 2], vv.z);
+            x[4 * q + 3] = fmaf(-gam, x[4 * q + 3], vv.w);
+          }
+          store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, x);
+        }
+        mbar_arrive(&v_empty);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&rready_b);
+        if (!(ok = mbar_wait_warp(&mma2_b, c & 1, ab))) break;
+        tc_fence_after();
+        const float dcy = gates[64 + i];
+        // U_d = decay-to-end * U, into the operand buffer (R is no longer needed)
+#pragma unroll
+        for (int cc = 0; cc < NB; ++cc) {
+          float u[32];
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 2 * DV * xb + 32 * cc), u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) u[e2] *= dcy;
+          store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, u);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&uready_b);
+      }
+    }
+    // final state of this slice
+    if (p.state_out) {
+      if (nc == 0) {
+        for (int d = 0; d < DV; ++d)
+          p.state_out[(srow0 + d) * kD + t] = p.state_in ? p.state_in[(srow0 + d) * kD + t] : 0.f;
+      } else if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(&mma3_b, (nc - 1) & 1, ab)) {
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < NB; ++cc) {
+          float v[32];
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) p.state_out[(srow0 + 32 * cc + e2) * kD + t] = v[e2];
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ output (warps 4, 5): token i = TMEM lane i
+    const int i = tid - 128;
+    const uint32_t lb = 32 * (warp & 3);
+    for (int c = 0; c < nc; ++c) {
+      const int st = c & 1, xb = c & 1, pb = c & 1;
+      if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab)) break;
+      const float gam = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE)[i];
+      if (!mbar_wait_warp(&mma2o_b[xb], (c >> 1) & 1, ab)) break;
+      tc_fence_after();
+      const uint32_t cX = Cfg::COL_X + 2 * DV * xb, cY = Cfg::COL_Y + 2 * DV * xb;
+      // per-32-column partial sums of o^2, combined in a fixed order for every slicing
+      float part[NB];
+#pragma unroll
+      for (int cc = 0; cc < NB; ++cc) {
+        float x[32], y[32];
+        tmem_ld32(tmem_addr(tbase, lb, cX + 32 * cc), x);
+        tmem_ld32(tmem_addr(tbase, lb, cY + 32 * cc), y);
+        tmem_wait_ld();
+        float ss = 0.f;
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) {
+          const float o = fmaf(gam, x[e2], y[e2]);
+          ss = fmaf(o, o, ss);
+        }
+        part[cc] = ss;
+      }
+      float total;
+      if constexpr (CS == 1) {
+        total = part[0];
+#pragma unroll
+        for (int cc = 1; cc < NB; ++cc) total += part[cc];
+      } else {
+        if (c >= 2 && !mbar_wait_warp(&nack_b[pb], ((c >> 1) - 1) & 1, ab, true)) break;
+#pragma unroll
+        for (int cc = 0; cc < NB; ++cc) sSS[(pb * 4 + slice * NB + cc) * 64 + i] = part[cc];
+        for (int r = 0; r < CS; ++r)
+          if (r != slice) mbar_arrive_remote(&nfull_b[pb], static_cast<uint32_t>(r));
+        if (!mbar_wait_warp(&nfull_b[pb], (c >> 1) & 1, ab, true)) break;
+        float blk[4];
+#pragma unroll
+        for (int bidx = 0; bidx < 4; ++bidx) {
+          const int owner = bidx / NB;
+          blk[bidx] = owner == slice ? part[bidx % NB]
+                                     : ld_shared_remote(sSS + (pb * 4 + bidx) * 64 + i, static_cast<uint32_t>(owner));
+        }
+        total = ((blk[0] + blk[1]) + blk[2]) + blk[3];
+        for (int r = 0; r < CS; ++r)
+          if (r != slice) mbar_arrive_remote(&nack_b[pb], static_cast<uint32_t>(r));
+      }
+      const float inv = rsqrtf(total * (1.0f / kD) + 1e-6f);
+      const long long tok = s + static_cast<long long>(c) * kChunk + i;
+      const bool valid = tok < e;
+      const long long trow = valid ? tok : s;
+      const uint4* zrow = reinterpret_cast<const uint4*>(p.z + trow * p.sz + static_cast<long long>(h) * kD + slice * DV);
+      uint4* orow = reinterpret_cast<uint4*>(p.out + (trow * p.H_v + h) * kD + slice * DV);
+#pragma unroll
+      for (int cc = 0; cc < NB; ++cc) {
+        float x[32], y[32];
+        tmem_ld32(tmem_addr(tbase, lb, cX + 32 * cc), x);  // whole warp: tcgen05.ld is warp-aligned
+        tmem_ld32(tmem_addr(tbase, lb, cY + 32 * cc), y);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float zz[8], f[8];
+            unpack8(__ldg(zrow + cc * 4 + q4), zz);
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) {
+              const int col = 32 * cc + 8 * q4 + e2;
+              const float o = fmaf(gam, x[8 * q4 + e2], y[8 * q4 + e2]);
+              f[e2] = o * inv * sNW[col] * silu_f(zz[e2]);
+            }
+            orow[cc * 4 + q4] = pack8(f);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&xyfree_b[xb]);
+      mbar_arrive(&qk_empty[st]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (CS > 1) cluster_sync_all();
+  if (warp == 7) tmem_dealloc<Cfg::TMEM_COLS>(tbase);
+}
+
+template <int DV>
+cudaError_t launch_scan(const PrefillParams& p, cudaStream_t stream) {
+  using Cfg = ScanCfg<DV>;
+  cudaError_t err = cudaFuncSetAttribute(scan_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.N) * p.H_v * Cfg::CS, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = Cfg::CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, scan_kernel<DV>, p);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream) {
+  cudaError_t err;
+  if (p.cu) {
+    setup_kernel<<<1, 1024, 0, stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (p.conv_out) {
+    const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
+    conv_out_kernel<<<dim3(static_cast<unsigned>((C_conv + 255) / 256), p.N), 256, 0, stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (p.n_chunks > 0) {
+    err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
+    if (err != cudaSuccess) return err;
+    prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, kPrepSmem, stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  return dv_slice == 32 ? launch_scan<32>(p, stream) : launch_scan<64>(p, stream);
+}
+
+}  // namespace gdn

@@ -1,0 +1,186 @@
+"""Thin ctypes binding of libgdn.so (the C ABI in include/gdn.h).
+
+Argument marshalling only: every step of the mixer runs in the library's CUDA
+kernels.  torch supplies device memory and the current stream.  There is no
+fallback: if the library is missing or a call is rejected, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+HEAD_DIM = 128
+CHUNK = 64
+
+_STATUS = {
+    0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_MISALIGNED",
+    4: "GDN_ERR_ALIAS", 5: "GDN_ERR_CUDA", 6: "GDN_ERR_DEVICE_TIMEOUT", 7: "GDN_ERR_WORKSPACE",
+}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+class GdnInputs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("z", ctypes.c_void_p),
+        ("stride_q", ctypes.c_longlong), ("stride_k", ctypes.c_longlong), ("stride_v", ctypes.c_longlong),
+        ("stride_z", ctypes.c_longlong), ("stride_a", ctypes.c_longlong), ("stride_b", ctypes.c_longlong),
+        ("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
+        ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("scale", ctypes.c_float), ("dv_slice", ctypes.c_int),
+    ]
+
+
+_lib = None
+_vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
+
+EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
+           "gdn_status_string")
+
+
+def load(path: str | None = None):
+    """Load libgdn.so from the package directory (it must have been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or _build.lib_path("libgdn.so")
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: run gated_delta_rule_81_b200.build.build() first")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(GdnInputs)
+    lib.gdn_prefill_workspace_size.argtypes = [_i, _i, _i, _ll]
+    lib.gdn_prefill_workspace_size.restype = _sz
+    lib.gdn_prefill.argtypes = [P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+    lib.gdn_prefill.restype = _i
+    lib.gdn_prefill_varlen.argtypes = [P, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+    lib.gdn_prefill_varlen.restype = _i
+    lib.gdn_decode_step.argtypes = [P, _i, _vp, _vp, _vp, _vp, _vp]
+    lib.gdn_decode_step.restype = _i
+    lib.gdn_status_string.argtypes = [_i]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _tok_stride(t, T_tot):
+    """Token stride (elements) of a [T_tot, ...] tensor whose per-token channels are contiguous."""
+    if t.dim() == 1:
+        return t.numel() // max(T_tot, 1)
+    inner = t[0] if t.shape[0] > 0 else t
+    if t.shape[0] > 0 and not inner.is_contiguous():
+        raise ValueError("per-token channels must be contiguous")
+    return t.stride(0)
+
+
+def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0, dv_slice=0) -> GdnInputs:
+    T_tot = q.shape[0]
+    H_k = q.shape[1] if q.dim() == 3 else q.shape[-1] // HEAD_DIM
+    H_v = v.shape[1] if v.dim() == 3 else v.shape[-1] // HEAD_DIM
+    for name, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z), ("conv_w", conv_w),
+                    ("norm_w", norm_w)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bf16")
+    if A_log.dtype != torch.float32:
+        raise TypeError("A_log must be fp32")
+    s = GdnInputs()
+    s.q, s.k, s.v, s.a, s.b, s.z = (t.data_ptr() for t in (q, k, v, a, b, z))
+    s.stride_q, s.stride_k, s.stride_v = (_tok_stride(t, T_tot) for t in (q, k, v))
+    s.stride_z, s.stride_a, s.stride_b = (_tok_stride(t, T_tot) for t in (z, a, b))
+    s.conv_w, s.A_log, s.norm_w = conv_w.data_ptr(), A_log.data_ptr(), norm_w.data_ptr()
+    s.H_k, s.H_v, s.scale, s.dv_slice = int(H_k), int(H_v), float(scale), int(dv_slice)
+    return s
+
+
+def _check(status, where):
+    if status != 0:
+        raise GdnError(status, where)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def workspace_size(H_k: int, H_v: int, N: int, n_chunks: int) -> int:
+    return int(load().gdn_prefill_workspace_size(H_k, H_v, N, n_chunks))
+
+
+def chunk_count(lengths) -> int:
+    return sum((int(L) + CHUNK - 1) // CHUNK for L in lengths)
+
+
+def _outputs(dev, T_tot, H_k, H_v, N, want_state, want_conv, out, state_out, conv_out):
+    C_conv = (2 * H_k + H_v) * HEAD_DIM
+    if out is None:
+        out = torch.empty(T_tot, H_v, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    if state_out is None and want_state:
+        state_out = torch.empty(N, H_v, HEAD_DIM, HEAD_DIM, dtype=torch.float32, device=dev)
+    if conv_out is None and want_conv:
+        conv_out = torch.empty(N, 3, C_conv, dtype=torch.bfloat16, device=dev)
+    return out, state_out, conv_out
+
+
+def prefill(inp: GdnInputs, B: int, T: int, state_in=None, conv_in=None, *, want_state=True, want_conv=True,
+            out=None, state_out=None, conv_out=None, workspace=None, err=None, device=None):
+    """gdn_prefill: B sequences of T tokens, packed [B*T].  Returns (out, state_out, conv_out)."""
+    lib = load()
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    out, state_out, conv_out = _outputs(dev, B * T, inp.H_k, inp.H_v, B, want_state, want_conv, out, state_out,
+                                        conv_out)
+    n_chunks = B * ((T + CHUNK - 1) // CHUNK)
+    need = lib.gdn_prefill_workspace_size(inp.H_k, inp.H_v, B, n_chunks)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(lib.gdn_prefill(ctypes.byref(inp), B, T, _ptr(state_in), _ptr(state_out), _ptr(conv_in),
+                           _ptr(conv_out), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err), _stream()),
+           "gdn_prefill")
+    return out, state_out, conv_out
+
+
+def prefill_varlen(inp: GdnInputs, cu_seqlens, cu_seqlens_host, state_in=None, conv_in=None, *, want_state=True,
+                   want_conv=True, out=None, state_out=None, conv_out=None, workspace=None, err=None):
+    """gdn_prefill_varlen.  cu_seqlens: device int32 [N+1]; cu_seqlens_host: CPU int32 [N+1]."""
+    lib = load()
+    dev = cu_seqlens.device
+    host = cu_seqlens_host.to(torch.int32).contiguous()
+    N = host.numel() - 1
+    T_tot = int(host[-1])
+    out, state_out, conv_out = _outputs(dev, T_tot, inp.H_k, inp.H_v, N, want_state, want_conv, out, state_out,
+                                        conv_out)
+    n_chunks = chunk_count((host[1:] - host[:-1]).tolist())
+    need = lib.gdn_prefill_workspace_size(inp.H_k, inp.H_v, N, n_chunks)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    host_ptr = ctypes.cast(host.data_ptr(), ctypes.c_void_p)
+    _check(lib.gdn_prefill_varlen(ctypes.byref(inp), N, _ptr(cu_seqlens), host_ptr, _ptr(state_in),
+                                  _ptr(state_out), _ptr(conv_in), _ptr(conv_out), _ptr(out), _ptr(workspace),
+                                  workspace.numel(), _ptr(err), _stream()),
+           "gdn_prefill_varlen")
+    return out, state_out, conv_out
+
+
+def decode_step(inp: GdnInputs, N: int, state, conv_state, out=None, err=None):
+    """gdn_decode_step: one token per sequence; state and conv_state updated in place.  Returns out."""
+    lib = load()
+    if out is None:
+        out = torch.empty(N, inp.H_v, HEAD_DIM, dtype=torch.bfloat16, device=state.device)
+    _check(lib.gdn_decode_step(ctypes.byref(inp), N, _ptr(state), _ptr(conv_state), _ptr(out), _ptr(err),
+                               _stream()),
+           "gdn_decode_step")
+    return out
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(status).decode()

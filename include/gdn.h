@@ -1,0 +1,144 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated-delta-rule token mixer.
+ *
+ * The mixer is the recurrent token mixer of the hybrid decoder described on
+ * the Agnes-3.0-Flash pages: model card, "Architecture" table, row
+ * "Delta-rule layers" (16 key heads / 48 value heads, head dim 128, a causal
+ * conv of kernel 4 in front, a gated RMS-norm after, recurrent state in fp32);
+ * kongchang article, paragraph on the Gated Delta Rule (each step erases the
+ * key's old association and then writes the new value, and a forget gate
+ * decays the memory).  Per value head h (key head h / (H_v / H_k)) and token t:
+ *
+ *   x_t      = [q | k | v] raw channels; y = SiLU(causal depthwise conv_4(x))
+ *   q_t, k_t = per-head L2-normalised y (x / sqrt(sum x^2 + 1e-6)), q_t *= scale
+ *   g_t      = -exp(A_log[h]) * softplus(a_t),  alpha_t = exp(g_t),  beta_t = sigmoid(b_t)
+ *   S_t      = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T   (S: d_v x d_k, fp32)
+ *   o_t      = S_t q_t
+ *   out_t    = o_t / sqrt(mean(o_t^2) + 1e-6) * norm_w * SiLU(z_t)           (bf16, RNE)
+ *
+ * Conventions common to every call:
+ *   - All tensor pointers are DEVICE pointers unless named *_host.  The caller
+ *     owns every buffer; the library keeps no state between calls and
+ *     allocates no memory (prefill scratch is the caller's `workspace`).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise.  A returned GDN_OK means the work was
+ *     validated and launched.
+ *   - Head dim is fixed at 128 (GDN_HEAD_DIM), H_v % H_k == 0 and
+ *     1 <= H_v / H_k <= 8.  Every tensor base pointer and every token stride
+ *     (in bytes) must be a multiple of 16.
+ *   - Layouts: q, k [T_tot][stride_q|k] with the H_k*128 head channels first;
+ *     v, z [T_tot][stride_v|z] with H_v*128 channels; a, b [T_tot][stride_a|b]
+ *     with H_v gate logits; out [T_tot][H_v][128] contiguous.  All bf16.
+ *     conv_w bf16 [C_conv][4] with C_conv = (2 H_k + H_v) * 128 channels
+ *     ordered q | k | v and tap 3 applied to the current token; A_log fp32
+ *     [H_v]; norm_w bf16 [128] shared by all heads.
+ *   - Recurrent state: fp32 [N][H_v][128 (d_v)][128 (d_k)], row-major.
+ *     Conv state: bf16 [N][3][C_conv], the 3 most recent raw tokens, oldest first.
+ *   - `err` (nullable) is a device int the kernels OR error bits into
+ *     (1 = a bounded wait timed out, 2 = cluster exchange failed,
+ *     4 = cu_seqlens on the device disagreed with cu_seqlens_host).  It is
+ *     never cleared by the library.  Read it after synchronising.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_HEAD_DIM 128
+#define GDN_CHUNK 64
+#define GDN_CONV_TAPS 4
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,   /* null required pointer, bad count, bad shape */
+  GDN_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  GDN_ERR_MISALIGNED = 3,    /* a pointer or stride is not 16-byte aligned */
+  GDN_ERR_ALIAS = 4,         /* buffers that must be distinct overlap */
+  GDN_ERR_CUDA = 5,          /* a CUDA launch failed */
+  GDN_ERR_DEVICE_TIMEOUT = 6,/* reserved for callers mapping *err bit 1 */
+  GDN_ERR_WORKSPACE = 7      /* workspace null or smaller than required */
+} gdn_status;
+
+/* Per-token inputs and per-layer parameters shared by all entry points. */
+typedef struct {
+  const void* q;          /* bf16 [T_tot] x stride_q, first H_k*128 channels used (pre-conv) */
+  const void* k;          /* bf16 [T_tot] x stride_k (pre-conv) */
+  const void* v;          /* bf16 [T_tot] x stride_v, first H_v*128 channels used (pre-conv) */
+  const void* a;          /* bf16 [T_tot] x stride_a, H_v decay logits */
+  const void* b;          /* bf16 [T_tot] x stride_b, H_v beta logits */
+  const void* z;          /* bf16 [T_tot] x stride_z, H_v*128 output-gate channels */
+  long long stride_q, stride_k, stride_v, stride_z, stride_a, stride_b; /* token strides, elements */
+  const void* conv_w;     /* bf16 [C_conv][4] */
+  const float* A_log;     /* fp32 [H_v] */
+  const void* norm_w;     /* bf16 [128] */
+  int H_k, H_v;
+  float scale;            /* multiplies the normalised q; 1.0 = o_t = S_t q_t as written above */
+  int dv_slice;           /* prefill only: state rows per scan CTA, 32 or 64, or 0 = automatic
+                             (128 is rejected with GDN_ERR_UNSUPPORTED); results do not depend on it */
+} gdn_inputs;
+
+/*
+ * Bytes of device workspace gdn_prefill / gdn_prefill_varlen need for a batch
+ * of N sequences that splits into n_chunks chunks of 64 tokens
+ * (n_chunks = sum over sequences of ceil(L_n / 64)).  0 on bad arguments.
+ */
+size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks);
+
+/*
+ * Prefill of B sequences of T tokens each, packed as [B*T] tokens (sequence n
+ * holds tokens n*T .. n*T+T-1).  Computes out for every token, and optionally
+ * the final recurrent state and conv state of each sequence.
+ *   state_in   fp32 [B][H_v][128][128] or NULL (zero initial state)
+ *   state_out  fp32 [B][H_v][128][128] or NULL; may equal state_in (in place)
+ *   conv_in    bf16 [B][3][C_conv] or NULL (zero history)
+ *   conv_out   bf16 [B][3][C_conv] or NULL; must not overlap conv_in
+ *   out        bf16 [B*T][H_v][128]
+ *   workspace  device scratch of gdn_prefill_workspace_size(H_k, H_v, B, B*ceil(T/64))
+ *              bytes, 16-byte aligned; contents need no initialisation
+ * B = 0 or T = 0 is a no-op apart from state_out = state_in and conv_out = conv_in history.
+ */
+gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
+                       const void* conv_in, void* conv_out, void* out, void* workspace,
+                       size_t workspace_bytes, int* err, void* stream);
+
+/*
+ * Prefill of N variable-length sequences packed back to back.
+ *   cu_seqlens       device int32 [N+1], cu[0] = 0, non-decreasing; sequence n is
+ *                    tokens cu[n] .. cu[n+1]-1
+ *   cu_seqlens_host  host copy of the same values (used to size the launch);
+ *                    validated on the host, and the device copy is checked
+ *                    against it on the device (mismatch: nothing is computed
+ *                    and *err gets bit 4)
+ * Every sequence starts from its own state_in[n] / conv_in[n] (or zeros): state
+ * and conv history never cross a cu_seqlens boundary.  Results for sequence n
+ * are bitwise identical to a gdn_prefill of that sequence alone with the same
+ * dv_slice.  Other arguments as in gdn_prefill with leading dimension N; the
+ * workspace size uses n_chunks = sum ceil((cu[n+1]-cu[n]) / 64).
+ */
+gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens,
+                              const int* cu_seqlens_host, const float* state_in, float* state_out,
+                              const void* conv_in, void* conv_out, void* out, void* workspace,
+                              size_t workspace_bytes, int* err, void* stream);
+
+/*
+ * One decode step for N sequences, one new token each (token n of the inputs
+ * belongs to sequence n, so T_tot = N).  Updates, in place,
+ *   state       fp32 [N][H_v][128][128]
+ *   conv_state  bf16 [N][3][C_conv]  (shifted by one token)
+ * and writes out bf16 [N][H_v][128].  Inputs must not overlap state, conv_state or out.
+ */
+gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out,
+                           int* err, void* stream);
+
+/* Static description of a status code. */
+const char* gdn_status_string(gdn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

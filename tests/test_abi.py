@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/gdn.h declares, sizes workspaces, and rejects bad
+arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_81_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gdn.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:size_t|gdn_status|const char\*)\s+(gdn_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) >= set(gdn.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert gdn.status_string(code).startswith("GDN_")
+
+
+def test_workspace_size(lib):
+    base = gdn.workspace_size(16, 48, 1, 0)
+    assert base > 0
+    per_chunk = gdn.workspace_size(16, 48, 1, 1) - base
+    assert per_chunk == 16 * 65536 + 48 * 66560
+    assert gdn.workspace_size(0, 48, 1, 1) == 0
+    assert gdn.workspace_size(16, 48, -1, 1) == 0
+
+
+def fake_inputs(H_k=2, H_v=6, ptr=0x10000):
+    s = gdn.GdnInputs()
+    for f in ("q", "k", "v", "a", "b", "z", "conv_w", "A_log", "norm_w"):
+        setattr(s, f, ptr)
+    s.stride_q = s.stride_k = H_k * 128
+    s.stride_v = s.stride_z = H_v * 128
+    s.stride_a = s.stride_b = H_v
+    s.H_k, s.H_v, s.scale, s.dv_slice = H_k, H_v, 1.0, 0
+    return s
+
+
+def call_prefill(lib, s, B=1, T=64, out=0x900000, ws=0x2000000, ws_bytes=1 << 30, conv_in=None, conv_out=None,
+                 state_in=None, state_out=None):
+    return lib.gdn_prefill(ctypes.byref(s), B, T, state_in, state_out, conv_in, conv_out, out, ws, ws_bytes, None,
+                           None)
+
+
+def test_rejects_bad_shapes(lib):
+    s = fake_inputs(H_k=4, H_v=6)  # 6 % 4 != 0
+    assert call_prefill(lib, s) == 1
+    s = fake_inputs(H_k=1, H_v=16)  # group of 16 value heads per key head
+    assert call_prefill(lib, s) == 2
+    s = fake_inputs()
+    s.dv_slice = 48
+    assert call_prefill(lib, s) == 1
+    s.dv_slice = 128
+    assert call_prefill(lib, s) == 2
+    s = fake_inputs()
+    s.stride_q = 100  # below H_k * 128
+    assert call_prefill(lib, s) == 1
+    assert call_prefill(lib, fake_inputs(), B=-1) == 1
+
+
+def test_rejects_null_and_misaligned(lib):
+    s = fake_inputs()
+    s.z = None
+    assert call_prefill(lib, s) == 1
+    s = fake_inputs()
+    s.q = 0x10008  # 8-byte aligned only
+    assert call_prefill(lib, s) == 3
+    s = fake_inputs()
+    s.stride_v = 6 * 128 + 4  # token stride not a multiple of 16 bytes
+    assert call_prefill(lib, s) == 3
+    assert call_prefill(lib, fake_inputs(), out=0x900008) == 3
+
+
+def test_rejects_aliasing_and_small_workspace(lib):
+    s = fake_inputs()
+    assert call_prefill(lib, s, conv_in=0x5000000, conv_out=0x5000000 + 16) == 4
+    assert call_prefill(lib, s, out=0x10000) == 4  # out over the inputs
+    assert call_prefill(lib, s, state_in=0x7000000, state_out=0x7000000 + 4096) == 4
+    assert call_prefill(lib, s, ws_bytes=1024) == 7
+    assert call_prefill(lib, s, ws=None) == 7
+
+
+def test_varlen_rejects_bad_cu_seqlens(lib):
+    s = fake_inputs()
+    for host in ([1, 5, 9], [0, 9, 5]):
+        arr = (ctypes.c_int * 3)(*host)
+        rc = lib.gdn_prefill_varlen(ctypes.byref(s), 2, 0x3000000, arr, None, None, None, None, 0x900000, 0x2000000,
+                                    1 << 30, None, None)
+        assert rc == 1
+    arr = (ctypes.c_int * 3)(0, 5, 9)
+    assert lib.gdn_prefill_varlen(ctypes.byref(s), 2, None, arr, None, None, None, None, 0x900000, 0x2000000,
+                                  1 << 30, None, None) == 1
+
+
+def test_decode_rejects_aliasing(lib):
+    s = fake_inputs()
+    assert lib.gdn_decode_step(ctypes.byref(s), 4, 0x7000000, 0x7000000 + 64, 0x900000, None, None) == 4
+    assert lib.gdn_decode_step(ctypes.byref(s), 4, None, 0x7000000, 0x900000, None, None) == 1
+    assert lib.gdn_decode_step(ctypes.byref(s), 0, None, None, None, None, None) == 0

@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the gated-delta-rule mixer on B200.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Default workload: one delta-layer prefill, B = 1, T = 4096 tokens, 16 key / 48
+value heads, head dim 128 (the headline configuration), metric tokens/s per
+layer.  One step = one gdn_prefill call (conv-state kernel, prep kernel, scan
+kernel) over the whole batch, inputs resident in HBM; the L2 is flushed
+(256 MiB write) between timed steps and the flush is outside the timed events.
+A secondary line item measures batched decode (256 sequences x 64 steps),
+state GB/s.  Under torchrun (N > 1) every rank runs its own batch (weak
+scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on the
+host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_81_b200 import inputs as gin  # noqa: E402
+
+METRIC = "gated-delta prefill tokens/s per layer; decode state GB/s vs B200 HBM peak"
+
+# Algorithmic work per token of a chunk-64 prefill with d = 128 (16 key / 48 value heads):
+#   prep kernel: [Q;K]K^T per key head (4 C d) and the two T-products per value head (4 C d)
+#   scan kernel: W S^T, Q S^T, U^T K per value head (6 d^2) and P U (2 C d)
+PREP_FLOP_PER_TOKEN = 16 * 4 * 64 * 128 + 48 * 4 * 64 * 128          # 2,097,152
+SCAN_FLOP_PER_TOKEN = 48 * (6 * 128 * 128 + 2 * 64 * 128)             # 5,505,024
+PREFILL_FLOP_PER_TOKEN = PREP_FLOP_PER_TOKEN + SCAN_FLOP_PER_TOKEN     # 7,602,176
+PREFILL_BYTES_PER_TOKEN = 20480 + 12288 + 12288 + 192                  # q,k,v + z + out + a,b
+DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 state read + write
+
+# DRAM traffic of one launch from an ncu capture, valid only for the kernel source
+# it was taken on (sha256 of the .cu file, first 16 hex digits).
+TRAFFIC = {}
+
+
+def src_sha(name):
+    with open(os.path.join(ROOT, "gated_delta_rule_81_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]),
+                "bf16_tflops_sustained": float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks (NVML, sampled during the timed region)
+
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.01):
+        self.samples, self.reasons, self.period = [], 0, period
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workloads
+
+
+def flush_l2(buf):
+    buf.add_(1)  # 256 MiB read + write, more than the 126 MB L2
+
+
+def prefill_workload(seed, dev):
+    case = gin.prefill_case(1, seed=seed)
+    inp = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in case["inp"].items()}
+    st = case["state_in"].to(dev)
+    return case, inp, st
+
+
+def run_prefill_ours(args, world, rank, dev, pk):
+    from gated_delta_rule_81_b200 import gdn
+
+    case, inp, st = prefill_workload(seed=rank, dev=dev)
+    B, T = 1, case["T_tot"]
+    s = gdn.make_inputs(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["z"], inp["conv_w"], inp["A_log"],
+                        inp["norm_w"], scale=inp["scale"])
+    H_k, H_v = s.H_k, s.H_v
+    n_chunks = B * math.ceil(T / 64)
+    ws = torch.empty(gdn.workspace_size(H_k, H_v, B, n_chunks), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, H_v, 128, dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty_like(st)
+    C_out = torch.empty(B, 3, (2 * H_k + H_v) * 128, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.prefill(s, B, T, st, None, out=out, state_out=S_out, conv_out=C_out, workspace=ws, err=err)
+
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    # per timed step: [step start] conv-state kernel [lib 0] prep [lib 1] scan [lib 2] [step end]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    hooks = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for ev in evs:
+            flush_l2(flush)
+            hooks.append(gdn.set_timing_events(s, ev[1:4]))
+            ev[0].record(stream)
+            step()
+            ev[4].record(stream)
+        torch.cuda.synchronize()
+    gdn.set_timing_events(s, None)
+    barrier(world)
+    step_ms = [ev[0].elapsed_time(ev[4]) for ev in evs]
+    prep_ms = [ev[1].elapsed_time(ev[2]) for ev in evs]
+    scan_ms = [ev[2].elapsed_time(ev[3]) for ev in evs]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    return {"total_ms": total_ms, "step_ms": step_ms, "T": T, "clocks": clk.report(), "launches_per_step": 3,
+            "case": case, "kernel_ms": {"prep": statistics.mean(prep_ms), "scan": statistics.mean(scan_ms),
+                                        "conv_state+gaps": statistics.mean(step_ms) - statistics.mean(prep_ms)
+                                        - statistics.mean(scan_ms)}}
+
+
+def run_e2e_prefill(args, world, rank, dev, case):
+    """Same workload through the public binding with host buffers: pinned host
+    inputs -> device, gdn_prefill, output and final state -> pinned host, all inside
+    the timed region."""
+    from gated_delta_rule_81_b200 import gdn
+
+    keys = ("q", "k", "v", "a", "b", "z")
+    host = {k: case["inp"][k].pin_memory() for k in keys}
+    host_state = case["state_in"].pin_memory()
+    wts = {k: case["inp"][k].to(dev) for k in ("conv_w", "A_log", "norm_w")}
+    T = case["T_tot"]
+    H_k, H_v = case["H_k"], case["H_v"]
+    dev_in = {k: torch.empty_like(host[k], device=dev) for k in keys}
+    st = torch.empty_like(host_state, device=dev)
+    ws = torch.empty(gdn.workspace_size(H_k, H_v, 1, math.ceil(T / 64)), dtype=torch.uint8, device=dev)
+    out_h = torch.empty(T, H_v, 128, dtype=torch.bfloat16).pin_memory()
+    S_h = torch.empty_like(host_state).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_state.numel() * 4
+    d2h = out_h.numel() * 2 + S_h.numel() * 4
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k in keys:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        st.copy_(host_state, non_blocking=True)
+        s = gdn.make_inputs(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a"], dev_in["b"], dev_in["z"],
+                            wts["conv_w"], wts["A_log"], wts["norm_w"])
+        out, S, _ = gdn.prefill(s, 1, T, st, None, want_conv=False, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+        S_h.copy_(S, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": world * T * args.steps / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def run_decode_ours(args, dev, steps_per_pass=64):
+    from gated_delta_rule_81_b200 import gdn
+
+    case = gin.decode_case(4)
+    N = case["N"]
+    state = case["state"].to(dev)
+    conv = case["conv_state"].to(dev)
+    tok = {k: case["tok"][k].to(dev) for k in ("q", "k", "v", "a", "b", "z")}
+    w = {k: v.to(dev) for k, v in case["w"].items()}
+    ins = [gdn.make_inputs(*(tok[k][i * N:(i + 1) * N] for k in ("q", "k", "v", "a", "b", "z")), w["conv_w"],
+                           w["A_log"], w["norm_w"]) for i in range(steps_per_pass)]
+    out = torch.empty(N, 48, 128, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        gdn.decode_step(ins[i], N, state, conv, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps_per_pass):
+        gdn.decode_step(ins[i], N, state, conv, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    per_launch_s = ms / 1e3 / steps_per_pass
+    gbs = N * DECODE_BYTES_PER_SEQ / per_launch_s / 1e9
+    return {"ms_per_launch": ms / steps_per_pass, "gbs": gbs, "launches": steps_per_pass}
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+
+
+def cpu_oracle_tokens_per_s(min_seconds=10.0, max_reps=8):
+    import oracle
+
+    case = gin.prefill_case(1)
+    cu = case["cu_seqlens"].tolist()
+    oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=[0], want_conv=False)  # build + warm
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.mixer(case["inp"], cu, state_in=case["state_in"], want_conv=False)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    return {"value": reps * case["T_tot"] / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"full T=4096 layer (48 value heads), fp64, repeated {reps}x ({el:.1f} s)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+
+    case = gin.prefill_case(1)
+    cu = case["cu_seqlens"].tolist()
+    heads = list(range(8))  # bounded sample per step: 8 of 48 value heads, scaled to the layer
+    oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=[0], want_conv=False)
+    for _ in range(args.warmup):
+        oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=heads, want_conv=False)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=heads, want_conv=False)
+    el = time.perf_counter() - t0
+    layer_s_per_step = el / args.steps * (48 / len(heads))
+    value = case["T_tot"] / layer_s_per_step
+    cfg = {"workload": gin.CONFIGS[1]["name"], "batch": 1, "seq_len": case["T_tot"], "H_k": 16, "H_v": 48,
+           "head_dim": 128}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s_per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"each step: value heads 0-7 of 48 over T=4096, time scaled x6"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: warm-up raised to 3 steps", file=sys.stderr)
+        args.warmup = 3
+
+    world, rank, local = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                          int(os.environ.get("LOCAL_RANK", "0")))
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from gated_delta_rule_81_b200 import build, gdn
+
+    build.build()
+    gdn.load()
+    pk = peaks()
+
+    res = run_prefill_ours(args, world, rank, dev, pk)
+    T = res["T"]
+    total_ms = res["total_ms"]
+    value = world * T * args.steps / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    # dominant kernel, timed live in the timed region with the library's event hook
+    kt = res["kernel_ms"]
+    dom = "scan" if kt["scan"] >= kt["prep"] else "prep"
+    flops = (SCAN_FLOP_PER_TOKEN if dom == "scan" else PREP_FLOP_PER_TOKEN) * T
+    achieved = flops / (kt[dom] * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    tr = TRAFFIC.get(dom)
+    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") else None
+    roof = {"kernel": f"{dom}_kernel", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic, "peak_source": f"{pk['source']} (bf16 burst)",
+            "algorithmic_flop_per_launch": flops, "launch_ms": kt[dom],
+            "kernel_ms": {k: round(v, 5) for k, v in kt.items()},
+            "whole_step": {"achieved": PREFILL_FLOP_PER_TOKEN * T / (ms_per_step * 1e-3) / 1e12,
+                           "frac": PREFILL_FLOP_PER_TOKEN * T / (ms_per_step * 1e-3) / 1e12 / peak}}
+
+    e2e = None if args.no_e2e else run_e2e_prefill(args, world, rank, dev, res["case"])
+    decode = None
+    if not args.no_decode:
+        d = run_decode_ours(args, dev)
+        decode = {"workload": gin.CONFIGS[4]["name"], "metric": "decode state GB/s", "value": d["gbs"],
+                  "unit": "GB/s", "ms_per_launch": d["ms_per_launch"],
+                  "roofline": {"bound": "hbm", "achieved": d["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                               "frac": d["gbs"] / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_tokens_per_s()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": gin.CONFIGS[1]["name"], "batch": 1, "seq_len": T, "H_k": 16, "H_v": 48,
+                       "head_dim": 128, "chunk": 64, "state_in": "N(0,0.01) fp32",
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+                       "parallelism": f"dp{world} (independent batch per GPU)"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": res["launches_per_step"] * args.steps,
+            "clocks": res["clocks"],
+            "secondary": decode,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

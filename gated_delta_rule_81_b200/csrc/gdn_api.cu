@@ -125,7 +125,7 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.conv_out = static_cast<bf16*>(conv_out);
   p.out = static_cast<bf16*>(out);
   p.err = err;
-  cudaError_t e = gdn::launch_prefill(p, pick_dv(in, N), static_cast<cudaStream_t>(stream));
+  cudaError_t e = gdn::launch_prefill(p, pick_dv(in, N), static_cast<cudaStream_t>(stream), in->events);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -204,7 +204,8 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
   p.conv_state = static_cast<bf16*>(conv_state);
   p.out = static_cast<bf16*>(out);
   p.err = err;
-  return gdn::launch_decode(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  return gdn::launch_decode(p, static_cast<cudaStream_t>(stream), in->events) == cudaSuccess ? GDN_OK
+                                                                                         : GDN_ERR_CUDA;
 }
 
 const char* gdn_status_string(gdn_status status) {

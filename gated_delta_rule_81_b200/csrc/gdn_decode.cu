@@ -145,12 +145,15 @@ __global__ void __launch_bounds__(kDecThreads) gdn_decode_kernel(DecodeParams p)
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events) {
   const int G = p.H_v / p.H_k;
   const size_t smem = static_cast<size_t>((2 + G) * kD + G * kD) * sizeof(float);
   dim3 grid(p.H_k, p.N);
+  if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
   gdn_decode_kernel<<<grid, kDecThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaError_t err = cudaGetLastError();
+  if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);
+  return err;
 }
 
 }  // namespace gdn

@@ -61,8 +61,9 @@ struct PrefillParams {
   int* err;
 };
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+// events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events);
 // dv_slice: 64 or 32 value rows of the state per scan CTA (a cluster of 128/dv_slice CTAs per head)
-cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream, void* const* events);
 
 }  // namespace gdn

@@ -926,7 +926,7 @@ cudaError_t launch_scan(const PrefillParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream, void* const* events) {
   cudaError_t err;
   if (p.cu) {
     setup_kernel<<<1, 1024, 0, stream>>>(p);
@@ -937,13 +937,17 @@ cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t st
     conv_out_kernel<<<dim3(static_cast<unsigned>((C_conv + 255) / 256), p.N), 256, 0, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
+  if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
   if (p.n_chunks > 0) {
     err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
     if (err != cudaSuccess) return err;
     prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, kPrepSmem, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  return dv_slice == 32 ? launch_scan<32>(p, stream) : launch_scan<64>(p, stream);
+  if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);
+  err = dv_slice == 32 ? launch_scan<32>(p, stream) : launch_scan<64>(p, stream);
+  if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), stream);
+  return err;
 }
 
 }  // namespace gdn

@@ -37,6 +37,7 @@ class GdnInputs(ctypes.Structure):
         ("stride_z", ctypes.c_longlong), ("stride_a", ctypes.c_longlong), ("stride_b", ctypes.c_longlong),
         ("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
         ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("scale", ctypes.c_float), ("dv_slice", ctypes.c_int),
+        ("events", ctypes.c_void_p),
     ]
 
 
@@ -102,6 +103,21 @@ def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0, dv_slice=0) 
     s.conv_w, s.A_log, s.norm_w = conv_w.data_ptr(), A_log.data_ptr(), norm_w.data_ptr()
     s.H_k, s.H_v, s.scale, s.dv_slice = int(H_k), int(H_v), float(scale), int(dv_slice)
     return s
+
+
+def set_timing_events(inp: GdnInputs, events):
+    """Attach torch.cuda.Event objects (enable_timing=True) that the library records
+    around its kernels (3 for prefill, 2 for decode); None detaches.  Returns the
+    ctypes array, which must stay alive while the call is in use."""
+    if events is None:
+        inp.events = None
+        return None
+    for ev in events:
+        if not ev.cuda_event:
+            ev.record()  # materialise the handle
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    inp.events = ctypes.cast(arr, ctypes.c_void_p)
+    return arr
 
 
 def _check(status, where):

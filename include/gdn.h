@@ -79,6 +79,10 @@ typedef struct {
   float scale;            /* multiplies the normalised q; 1.0 = o_t = S_t q_t as written above */
   int dv_slice;           /* prefill only: state rows per scan CTA, 32 or 64, or 0 = automatic
                              (128 is rejected with GDN_ERR_UNSUPPORTED); results do not depend on it */
+  void* const* events;    /* optional timing hook: NULL, or caller-created cudaEvent_t handles that
+                             the library records on `stream` around its kernels.  Prefill: 3 events,
+                             [0] before the prep kernel, [1] between prep and scan, [2] after the
+                             scan.  Decode: 2 events, before and after the decode kernel. */
 } gdn_inputs;
 
 /*

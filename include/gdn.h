@@ -138,6 +138,33 @@ gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens
 gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out,
                            int* err, void* stream);
 
+/*
+ * Allocation-free prefill.  The pages have no counterpart to this call; it
+ * exists for callers that cannot allocate device memory (code running inside a
+ * memory budget fixed by a host framework, an allocator hook that must not
+ * re-enter the allocator, a runtime whose memory plan is frozen before its
+ * first launch).  Same inputs, outputs and results as gdn_prefill, but no
+ * workspace argument: the scratch is a file-scope device array of
+ * GDN_NOALLOC_SCRATCH_BYTES inside libgdn.so, which every GPU that loads the
+ * library holds until the process exits.
+ *   - Limit: gdn_prefill_workspace_size(H_k, H_v, B, B*ceil(T/64)) must not
+ *     exceed GDN_NOALLOC_SCRATCH_BYTES (64 MiB: e.g. up to 15 chunks of 64
+ *     tokens in total at 16/48 heads, 126 at 2/6 heads); larger requests return
+ *     GDN_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the previous
+ *     call's contents (nothing in it needs to start at zero).  Calls whose work
+ *     overlaps on the GPU -- on different streams, or from different host
+ *     threads without ordering -- race on it; order them on one stream.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64u << 20)
+gdn_status gdn_prefill_noalloc(const gdn_inputs* in, int B, int T, const float* state_in,
+                               float* state_out, const void* conv_in, void* conv_out, void* out,
+                               int* err, void* stream);
+
 /* Static description of a status code. */
 const char* gdn_status_string(gdn_status status);
 

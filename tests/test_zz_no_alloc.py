@@ -1,0 +1,81 @@
+"""gdn_prefill_noalloc: the prefill for callers that cannot allocate device
+memory (a fixed memory budget handed down by a host framework, an allocator
+hook that must not re-enter the allocator, a pre-planned runtime).  It uses the
+library's own static device scratch instead of a caller workspace.
+
+Checked through the C ABI against gdn_prefill (the entry point with a caller
+workspace) on two calls in a row with different inputs, so the second call
+runs on the scratch contents the first left behind; oversize requests must be
+rejected without a launch.  Collected last so a failure here cannot hide
+another test's.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_81_b200 import build, gdn
+from gated_delta_rule_81_b200 import inputs as gin
+from gpu_helpers import OUT_TOL, STATE_TOL, out_error, state_error
+
+pytestmark = pytest.mark.gpu
+
+NOALLOC_BYTES = 64 << 20
+
+
+def noalloc_fn():
+    build.build()
+    lib = gdn.load()
+    f = lib.gdn_prefill_noalloc
+    f.argtypes = [ctypes.POINTER(gdn.GdnInputs), ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 7
+    f.restype = ctypes.c_int
+    return f
+
+
+def one_case(seed, B, T, H_k, H_v):
+    inp = gin.token_inputs(B * T, H_k, H_v, seed=seed)
+    inp.update(gin.weights(H_k, H_v, seed=seed))
+    dev = {k: v.cuda() for k, v in inp.items()}
+    s = gdn.make_inputs(dev["q"], dev["k"], dev["v"], dev["a"], dev["b"], dev["z"], dev["conv_w"], dev["A_log"],
+                        dev["norm_w"])
+    st = gin.recurrent_state(B, H_v, seed=seed + 1).cuda()
+    cv = gin.conv_state(B, H_k, H_v, seed=seed + 2).cuda()
+    return dev, s, st, cv
+
+
+def run_noalloc(f, s, B, T, st, cv):
+    H_k, H_v = s.H_k, s.H_v
+    out = torch.empty(B * T, H_v, 128, dtype=torch.bfloat16, device="cuda")
+    S = torch.empty_like(st)
+    C = torch.empty(B, 3, (2 * H_k + H_v) * 128, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    rc = f(ctypes.byref(s), B, T, p(st), p(S), p(cv), p(C), p(out), p(err),
+           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return rc, out, S, C, err
+
+
+@pytest.mark.parametrize("B,T,H_k,H_v", [(2, 200, 2, 6), (1, 900, 16, 48)])
+def test_noalloc_matches_workspace_prefill_twice(B, T, H_k, H_v):
+    f = noalloc_fn()
+    assert gdn.workspace_size(H_k, H_v, B, B * ((T + 63) // 64)) <= NOALLOC_BYTES
+    for seed in (31, 47):  # two calls in a row, different inputs
+        dev, s, st, cv = one_case(seed, B, T, H_k, H_v)
+        rc, out, S, C, err = run_noalloc(f, s, B, T, st, cv)
+        assert rc == 0, gdn.status_string(rc)
+        ref_out, ref_S, ref_C = gdn.prefill(s, B, T, st, cv)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert out_error(out, ref_out.float().cpu().numpy()) <= OUT_TOL
+        assert state_error(S, ref_S.double().cpu().numpy()) <= STATE_TOL
+        np.testing.assert_array_equal(C.cpu().float().numpy(), ref_C.cpu().float().numpy())
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch():
+    f = noalloc_fn()
+    B, T, H_k, H_v = 1, 4096, 16, 48
+    assert gdn.workspace_size(H_k, H_v, B, 64) > NOALLOC_BYTES
+    dev, s, st, cv = one_case(5, 1, 64, H_k, H_v)  # small real buffers; the size check comes first
+    rc = f(ctypes.byref(s), B, T, None, None, None, None, ctypes.c_void_p(dev["q"].data_ptr()), None, None)
+    assert rc == 7  # GDN_ERR_WORKSPACE, nothing launched

@@ -2,8 +2,9 @@
 //
 // Agnes-3.0-Flash model card, "Architecture" table, row "Delta-rule layers":
 // causal conv (kernel 4) in front, gated RMS-norm after, fp32 recurrent state;
-// kongchang article, paragraph on the Gated Delta Rule: erase the key's old
-// association, then write, under a forget gate.  Per value head and state row
+// "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention Multimodal Model", section
+// "Feed-Forward and Positional Encoding", paragraph on the Gated Delta Rule:
+// erase the key's old association, then write, under a forget gate.  Per value head and state row
 // r (d_v index) the step reads the row once and writes it once:
 //   sk = s_r . k, sq = s_r . q,  delta = beta (v_r - alpha sk),
 //   s_r <- alpha s_r + delta k,   o_r = alpha sq + delta (k . q),

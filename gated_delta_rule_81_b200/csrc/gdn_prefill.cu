@@ -2,9 +2,10 @@
 //
 // Method: Agnes-3.0-Flash model card, "Architecture" table, row "Delta-rule
 // layers" (16 key / 48 value heads, head dim 128, causal conv kernel 4 in
-// front, gated RMS-norm after, fp32 recurrent state) and the kongchang
-// article's paragraph on the Gated Delta Rule (erase-then-write under a forget
-// gate).  Recurrence: S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T,
+// front, gated RMS-norm after, fp32 recurrent state) and "Agnes-3.0-Flash
+// Deep Dive: A 33B Hybrid-Attention Multimodal Model", section "Feed-Forward
+// and Positional Encoding", paragraph on the Gated Delta Rule (erase-then-write
+// under a forget gate).  Recurrence: S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T,
 // o_t = S_t q_t, evaluated 64 tokens at a time in its chunkwise (UT-transform)
 // form.  Inside a chunk that starts from state S (d_v x d_k), with G the
 // inclusive cumulative sum of g = log a, gamma_i = e^{G_i}:

@@ -5,9 +5,10 @@
  * the Agnes-3.0-Flash pages: model card, "Architecture" table, row
  * "Delta-rule layers" (16 key heads / 48 value heads, head dim 128, a causal
  * conv of kernel 4 in front, a gated RMS-norm after, recurrent state in fp32);
- * kongchang article, paragraph on the Gated Delta Rule (each step erases the
- * key's old association and then writes the new value, and a forget gate
- * decays the memory).  Per value head h (key head h / (H_v / H_k)) and token t:
+ * "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention Multimodal Model",
+ * section "Feed-Forward and Positional Encoding", paragraph on the Gated Delta
+ * Rule (each step erases the key's old association and then writes the new
+ * value, and a forget gate decays the memory).  Per value head h (key head h / (H_v / H_k)) and token t:
  *
  *   x_t      = [q | k | v] raw channels; y = SiLU(causal depthwise conv_4(x))
  *   q_t, k_t = per-head L2-normalised y (x / sqrt(sum x^2 + 1e-6)), q_t *= scale

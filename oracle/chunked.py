@@ -2,8 +2,10 @@
 
 It validates the chunk algebra that the GPU path uses; it is not the reference
 (the sequential recurrence in gdn_oracle.c is).  Derivation, written out from
-the recurrence the Agnes-3.0-Flash pages name (model card "Architecture" table,
-row "Delta-rule layers"; kongchang article, paragraph on the Gated Delta Rule):
+the recurrence the Agnes-3.0-Flash pages name (model card, "Architecture" table,
+row "Delta-rule layers"; "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention
+Multimodal Model", section "Feed-Forward and Positional Encoding", paragraph on
+the Gated Delta Rule):
 
   S_i = alpha_i S_{i-1} + u_i k_i^T   with   u_i = beta_i (v_i - alpha_i S_{i-1} k_i).
 

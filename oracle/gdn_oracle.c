@@ -10,15 +10,17 @@
  *   Agnes-3.0-Flash model card, "Architecture" table, row "Delta-rule layers":
  *     16 key heads / 48 value heads, head dim 128, a causal conv of kernel 4 in
  *     front, a gated RMS-norm after, recurrent state in fp32.
- *   kongchang article, paragraph on the Gated Delta Rule: each step first
- *     erases the old association of the key and then writes the new value
- *     ("erase then update"), and a forget gate decays the whole memory.
+ *   "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention Multimodal Model",
+ *     section "Feed-Forward and Positional Encoding", paragraph on the Gated
+ *     Delta Rule: each step first erases the old association of the key and
+ *     then writes the new value ("erase then update"), and a forget gate
+ *     decays the whole memory.
  *   The recurrence those two passages name, written out (the standard gated
  *   delta rule; the pages give no equation, so this is the reading taken):
  *       S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t
  *   with S_t a d_v x d_k matrix per value head.
  *
- * Readings of points the pages leave open (each also listed in the design doc):
+ * Readings of points the pages leave open:
  *   - conv: depthwise over the q|k|v channels, no bias, tap 3 on the current
  *     token, history before a sequence start from conv_in (zeros if absent);
  *     SiLU after the conv.

@@ -1,11 +1,12 @@
 """ctypes front of the fp64 C oracle (gdn_oracle.c) -- test infrastructure only.
 
 The sequential fp64 recurrence is the reference every GPU result is checked
-against.  Its passages: the model card's "Architecture" table (row "Delta-rule
-layers": 16 key / 48 value heads, head dim 128, causal conv kernel 4 in front,
-gated RMS-norm after, fp32 state) and the kongchang article's paragraph on the
-Gated Delta Rule (erase the key's old association, then write; a forget gate
-decays the memory).  The recurrence itself, S_t = a_t S_{t-1}(I - b_t k_t k_t^T)
+against.  Its passages: the Agnes-3.0-Flash model card, "Architecture" table,
+row "Delta-rule layers" (16 key / 48 value heads, head dim 128, causal conv
+kernel 4 in front, gated RMS-norm after, fp32 state), and "Agnes-3.0-Flash Deep
+Dive: A 33B Hybrid-Attention Multimodal Model", section "Feed-Forward and
+Positional Encoding", paragraph on the Gated Delta Rule (erase the key's old
+association, then write; a forget gate decays the memory).  The recurrence itself, S_t = a_t S_{t-1}(I - b_t k_t k_t^T)
 + b_t v_t k_t^T with o_t = S_t q_t, is the standard gated delta rule those
 passages name.
 """

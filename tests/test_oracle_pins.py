@@ -3,8 +3,9 @@ a hand-worked example, closed forms, library routines (torch conv1d, rms_norm,
 softplus, a linear solve), brute force on tiny inputs, and invariants.
 
 The recurrence pinned here is the gated delta rule named on the Agnes-3.0-Flash
-pages (model card "Architecture" table, row "Delta-rule layers"; kongchang
-article, paragraph on the Gated Delta Rule):
+pages (model card, "Architecture" table, row "Delta-rule layers"; "Agnes-3.0-Flash
+Deep Dive: A 33B Hybrid-Attention Multimodal Model", section "Feed-Forward and
+Positional Encoding", paragraph on the Gated Delta Rule):
     S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t.
 """
 import os

@@ -156,7 +156,8 @@ constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32
 constexpr int kPrepOffM = kPrepOffT + 64 * kLdA * 4;   // block-solve temp      3*256*4
 constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum [8][64]
 constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta     [8][64]
-constexpr int kPrepSmem = kPrepOffB + 8 * 64 * 4 + 1024;
+constexpr int kPrepOffW = kPrepOffB + 8 * 64 * 4;      // conv weights of the CTA's channels, (2+8)*128*8 B
+constexpr int kPrepSmem = kPrepOffW + 10 * 128 * 8 + 1024;
 
 // hi = bf16(f), lo = bf16(f - hi) for 8 values
 __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
@@ -172,12 +173,14 @@ __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
 
 // Conv (4 taps) + SiLU of 32 consecutive channels of one token.
 //   src: the token-0 address of the group's first channel; rows before the
-//   sequence start come from conv_in (or are zero).
+//   sequence start come from conv_in (or are zero).  wsm: the 32 channels'
+//   weights in shared memory, 16 x uint4 (channels 2u, 2u+1; taps 0..3 each).
+//   All 16 input loads are issued before any arithmetic.
 __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, long long src_stride,
-                                       long long s, long long t, int n, long long conv_chan0, float* y) {
+                                       long long s, long long t, int n, long long conv_chan0, const uint4* wsm,
+                                       float* y) {
   const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) y[e] = 0.f;
+  uint4 xin[kTaps][4];
 #pragma unroll
   for (int j = 0; j < kTaps; ++j) {
     const long long tau = t - (kTaps - 1) + j;
@@ -186,54 +189,91 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
     else if (p.conv_in)
       row = reinterpret_cast<const uint4*>(p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv +
                                            conv_chan0);
-    if (row == nullptr) continue;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      float x[8];
-      unpack8(__ldg(row + g), x);
-      const bf16* w = p.conv_w + (conv_chan0 + 8 * g) * kTaps + j;  // tap j of channels 8g .. 8g+7
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[8 * g + e] = fmaf(__bfloat162float(w[e * kTaps]), x[e], y[8 * g + e]);
-    }
+    for (int g = 0; g < 4; ++g) xin[j][g] = row ? __ldg(row + g) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int e = 0; e < 32; ++e) y[e] = silu_f(y[e]);
+  for (int g = 0; g < 4; ++g) {
+    float x[kTaps][8];
+#pragma unroll
+    for (int j = 0; j < kTaps; ++j) unpack8(xin[j][g], x[j]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // channel pair 8g + 2u, 8g + 2u + 1
+      const uint4 w = wsm[4 * g + u];
+      const int e0 = 2 * u, e1 = 2 * u + 1;
+      float a0 = bf16_lo(w.x) * x[0][e0];
+      a0 = fmaf(bf16_hi(w.x), x[1][e0], a0);
+      a0 = fmaf(bf16_lo(w.y), x[2][e0], a0);
+      a0 = fmaf(bf16_hi(w.y), x[3][e0], a0);
+      float a1 = bf16_lo(w.z) * x[0][e1];
+      a1 = fmaf(bf16_hi(w.z), x[1][e1], a1);
+      a1 = fmaf(bf16_lo(w.w), x[2][e1], a1);
+      a1 = fmaf(bf16_hi(w.w), x[3][e1], a1);
+      y[8 * g + e0] = silu_f(a0);
+      y[8 * g + e1] = silu_f(a1);
+    }
+  }
+}
+
+// One block diagonal of the blocked inverse: for blocks (I, J = I - d),
+//   M = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II M
+// with 16x16 blocks; all 256 threads, fixed trip counts.
+template <int d>
+__device__ __forceinline__ void solve_level(const float* sA, float* sT, float* sM, int tid) {
+  constexpr int nb = 4 - d;
+  for (int x = tid; x < nb * 256; x += kPrepThreads) {
+    const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
+    const float* arow = sA + (16 * I + ii) * kLdA + 16 * J;
+    const float* tcol = sT + (16 * J) * kLdA + 16 * J + jj;
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 16 * d; kk += 2) {
+      acc0 = fmaf(arow[kk], tcol[kk * kLdA], acc0);
+      acc1 = fmaf(arow[kk + 1], tcol[(kk + 1) * kLdA], acc1);
+    }
+    sM[x] = acc0 + acc1;
+  }
+  __syncthreads();
+  for (int x = tid; x < nb * 256; x += kPrepThreads) {
+    const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
+    const float* trow = sT + (16 * I + ii) * kLdA + 16 * I;
+    const float* mcol = sM + (J << 8) + jj;
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int l = 0; l < 16; l += 2) {  // T_II is lower triangular: entries l > ii are zero
+      acc0 = fmaf(l <= ii ? trow[l] : 0.f, mcol[l << 4], acc0);
+      acc1 = fmaf(l + 1 <= ii ? trow[l + 1] : 0.f, mcol[(l + 1) << 4], acc1);
+    }
+    sT[(16 * I + ii) * kLdA + 16 * J + jj] = -(acc0 + acc1);
+  }
+  __syncthreads();
 }
 
 // T = (I + A)^{-1} for a 64x64 strictly-lower A (fp32, shared memory), by 16x16
-// blocks: diagonal blocks by forward substitution, then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
-// one block diagonal at a time.  All 256 threads.
+// blocks: diagonal blocks by forward substitution, then the three block
+// diagonals below.  All 256 threads.
 __device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid) {
   if (tid < 64) {
     const int blk = tid >> 4, col = tid & 15;
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int l = 0; l < r; ++l) acc = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + l], x[l], acc);
+      for (int l = 0; l + 1 < r; l += 2) {
+        acc0 = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + l], x[l], acc0);
+        acc1 = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + l + 1], x[l + 1], acc1);
+      }
+      if (r & 1) acc0 = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + r - 1], x[r - 1], acc0);
+      const float acc = acc0 + acc1;
       x[r] = r < col ? 0.f : (r == col ? 1.f : -acc);
       sT[(16 * blk + r) * kLdA + 16 * blk + col] = x[r];
     }
   }
   __syncthreads();
-  for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;
-    for (int x = tid; x < nb * 256; x += kPrepThreads) {
-      const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
-      float acc = 0.f;
-      for (int kk = 16 * J; kk < 16 * I; ++kk) acc = fmaf(sA[(16 * I + ii) * kLdA + kk], sT[kk * kLdA + 16 * J + jj], acc);
-      sM[x] = acc;
-    }
-    __syncthreads();
-    for (int x = tid; x < nb * 256; x += kPrepThreads) {
-      const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
-      float acc = 0.f;
-      for (int l = 0; l <= ii; ++l) acc = fmaf(sT[(16 * I + ii) * kLdA + 16 * I + l], sM[(J << 8) + (l << 4) + jj], acc);
-      sT[(16 * I + ii) * kLdA + 16 * J + jj] = -acc;
-    }
-    __syncthreads();
-  }
+  solve_level<1>(sA, sT, sM, tid);
+  solve_level<2>(sA, sT, sM, tid);
+  solve_level<3>(sA, sT, sM, tid);
 }
 
 // D (+)= A B^T with both operands as hi/lo pairs: A_hi B_hi + A_hi B_lo + A_lo B_hi
@@ -256,6 +296,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
   float* sM = reinterpret_cast<float*>(sm + kPrepOffM);
   float* sG = reinterpret_cast<float*>(sm + kPrepOffG);
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
+  uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2+G)*128 channels / 2] pairs: q | k | v heads
   __shared__ uint64_t bar[3];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
@@ -291,6 +332,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
   }
   if (warp == 0) tmem_alloc<128>(&tmem_base_s);
 
+  // conv weights of this CTA's channels (q, k of key head kh; v of its G value heads)
+  for (int x = tid; x < (2 + G) * 64; x += kPrepThreads) {
+    const int pair = x % 64, grp = x / 64;  // grp 0 = q, 1 = k, 2.. = value head grp-2
+    const long long ch0 = grp == 0 ? static_cast<long long>(kh) * kD
+                        : grp == 1 ? static_cast<long long>(H_k + kh) * kD
+                                   : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh * G + grp - 2) * kD;
+    sW[x] = __ldg(reinterpret_cast<const uint4*>(p.conv_w + (ch0 + 2 * pair) * kTaps));
+  }
+  __syncthreads();
+
   // identity rows 64..127 of the [P; I] image (hi = I, lo = 0)
   for (int x = tid; x < 64 * 8; x += kPrepThreads) {
     const int i = x >> 3, cc = x & 7;
@@ -313,7 +364,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
       const long long sx = which ? p.sk : p.sq;
       const long long chan0 = static_cast<long long>(which) * H_k * kD + static_cast<long long>(kh) * kD + 32 * qq;
       float y[32];
-      if (valid) conv32(p, X + static_cast<long long>(kh) * kD + 32 * qq, sx, s, t0 + i, n, chan0, y);
+      if (valid) conv32(p, X + static_cast<long long>(kh) * kD + 32 * qq, sx, s, t0 + i, n, chan0, sW + which * 64 + 16 * qq, y);
       float ss = 0.f;
 #pragma unroll
       for (int e2 = 0; e2 < 32; ++e2) {
@@ -398,7 +449,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
     float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes + kVBytes);
     gdst[k2] = val;
   }
-  // ---- v_hat of the value heads (fp32): token i, channels 32*qq..+31, stored [4 column blocks][64][32]
+  // ---- v_hat of the value heads (fp32): token i, channels 32*qq..+31
   {
     const int i = tid >> 2, qq = tid & 3;
     const bool valid = i < L;
@@ -407,15 +458,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
       float y[32];
       if (valid) {
         conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,
-               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, y);
+               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, sW + (2 + j) * 64 + 16 * qq, y);
       } else {
 #pragma unroll
         for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
       }
-      float4* dst = reinterpret_cast<float4*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes +
-                                              (qq * 64 + i) * 128);
+      // [column block qq][quad q][token i] float4: a warp's reads of one quad are contiguous
+      float4* dst = reinterpret_cast<float4*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes) +
+                    qq * 8 * 64 + i;
 #pragma unroll
-      for (int c2 = 0; c2 < 8; ++c2) dst[c2] = make_float4(y[4 * c2], y[4 * c2 + 1], y[4 * c2 + 2], y[4 * c2 + 3]);
+      for (int c2 = 0; c2 < 8; ++c2) dst[c2 * 64] = make_float4(y[4 * c2], y[4 * c2 + 1], y[4 * c2 + 2], y[4 * c2 + 3]);
     }
   }
 
@@ -769,7 +821,7 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 vv = vrow[(cc * 64 + i) * 8 + q];
+            const float4 vv = vrow[(cc * 8 + q) * 64 + i];
             x[4 * q + 0] = fmaf(-gam, x[4 * q + 0], vv.x);
             x[4 * q + 1] = fmaf(-gam, x[4 * q + 1], vv.y);
             x[4 * q + 2] = fmaf(-gam, x[4 * q + 2], vv.z);
@@ -820,10 +872,21 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     // ------------------------------------------------ output (warps 4, 5): token i = TMEM lane i
     const int i = tid - 128;
     const uint32_t lb = 32 * (warp & 3);
+    // z of the next chunk is loaded while this chunk's products are still running
+    uint4 zbuf[NB * 4];
+    auto load_z = [&](int c) {
+      const long long tok = s + static_cast<long long>(c) * kChunk + i;
+      const uint4* zrow = reinterpret_cast<const uint4*>(p.z + (tok < e ? tok : s) * p.sz +
+                                                         static_cast<long long>(h) * kD + slice * DV);
+#pragma unroll
+      for (int q = 0; q < NB * 4; ++q) zbuf[q] = tok < e ? __ldg(zrow + q) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    if (nc > 0) load_z(0);
     for (int c = 0; c < nc; ++c) {
       const int st = c & 1, xb = c & 1, pb = c & 1;
       if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab)) break;
       const float gam = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE)[i];
+      mbar_arrive(&qk_empty[st]);  // only gamma is read from the stage
       if (!mbar_wait_warp(&mma2o_b[xb], (c >> 1) & 1, ab)) break;
       tc_fence_after();
       const uint32_t cX = Cfg::COL_X + 2 * DV * xb, cY = Cfg::COL_Y + 2 * DV * xb;
@@ -869,33 +932,34 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
       const float inv = rsqrtf(total * (1.0f / kD) + 1e-6f);
       const long long tok = s + static_cast<long long>(c) * kChunk + i;
       const bool valid = tok < e;
-      const long long trow = valid ? tok : s;
-      const uint4* zrow = reinterpret_cast<const uint4*>(p.z + trow * p.sz + static_cast<long long>(h) * kD + slice * DV);
-      uint4* orow = reinterpret_cast<uint4*>(p.out + (trow * p.H_v + h) * kD + slice * DV);
+      uint4* orow = reinterpret_cast<uint4*>(p.out + ((valid ? tok : s) * p.H_v + h) * kD + slice * DV);
+      uint4 ob[NB * 4];
 #pragma unroll
       for (int cc = 0; cc < NB; ++cc) {
         float x[32], y[32];
         tmem_ld32(tmem_addr(tbase, lb, cX + 32 * cc), x);  // whole warp: tcgen05.ld is warp-aligned
         tmem_ld32(tmem_addr(tbase, lb, cY + 32 * cc), y);
         tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float zz[8], f[8];
-            unpack8(__ldg(zrow + cc * 4 + q4), zz);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float zz[8], f[8];
+          unpack8(zbuf[cc * 4 + q4], zz);
 #pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2) {
-              const int col = 32 * cc + 8 * q4 + e2;
-              const float o = fmaf(gam, x[8 * q4 + e2], y[8 * q4 + e2]);
-              f[e2] = o * inv * sNW[col] * silu_f(zz[e2]);
-            }
-            orow[cc * 4 + q4] = pack8(f);
+          for (int e2 = 0; e2 < 8; ++e2) {
+            const int col = 32 * cc + 8 * q4 + e2;
+            const float o = fmaf(gam, x[8 * q4 + e2], y[8 * q4 + e2]);
+            f[e2] = o * inv * sNW[col] * silu_f(zz[e2]);
           }
+          ob[cc * 4 + q4] = pack8(f);
         }
       }
       tc_fence_before();
       mbar_arrive(&xyfree_b[xb]);
-      mbar_arrive(&qk_empty[st]);
+      if (c + 1 < nc) load_z(c + 1);
+      if (valid) {
+#pragma unroll
+        for (int q = 0; q < NB * 4; ++q) orow[q] = ob[q];
+      }
     }
   }
 

@@ -948,7 +948,7 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
           for (int e2 = 0; e2 < 8; ++e2) {
             const int col = 32 * cc + 8 * q4 + e2;
             const float o = fmaf(gam, x[8 * q4 + e2], y[8 * q4 + e2]);
-            f[e2] = o * inv * sNW[col] * silu_f(zz[e2]);
+            f[e2] = o * inv * sNW[col] * silu_fast(zz[e2]);
           }
           ob[cc * 4 + q4] = pack8(f);
         }

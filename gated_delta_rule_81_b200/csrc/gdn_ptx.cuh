@@ -274,6 +274,9 @@ __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u 
 
 __device__ __forceinline__ float silu_f(float y) { return y / (1.0f + __expf(-y)); }
 
+// SiLU with the fast approximate division (about 2 ulp; y -> -inf gives -0)
+__device__ __forceinline__ float silu_fast(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+
 // softplus(a) = log(1 + e^a), computed as max(a, 0) + log1p(e^{-|a|})
 __device__ __forceinline__ float softplus_f(float a) { return fmaxf(a, 0.0f) + log1pf(expf(-fabsf(a))); }
 

@@ -147,13 +147,14 @@ __global__ void conv_out_kernel(PrefillParams p) {
 // ============================================================ prep kernel
 
 constexpr int kPrepThreads = 256;
-constexpr int kLdA = 65;                               // fp32 row stride of A / T in shared memory
+constexpr int kLdA = 65;                               // fp32 row stride of A in shared memory
+constexpr int kLdT = 68;                               // fp32 row stride of T (16-byte aligned rows)
 constexpr int kPrepOffQK = 0;                          // [Q;K] image hi, lo    2 x 32768
 constexpr int kPrepOffPI = kPrepOffQK + 2 * 32768;     // [P;I] image hi, lo    2 x 16384
 constexpr int kPrepOffTt = kPrepOffPI + 2 * 16384;     // T~ image (B) hi, lo   2 x 8192
 constexpr int kPrepOffA = kPrepOffTt + 2 * 8192;       // A fp32                64*65*4
 constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32
-constexpr int kPrepOffM = kPrepOffT + 64 * kLdA * 4;   // block-solve temp      3*256*4
+constexpr int kPrepOffM = kPrepOffT + 64 * kLdT * 4;   // block-solve temp      3*256*4
 constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum [8][64]
 constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta     [8][64]
 constexpr int kPrepOffW = kPrepOffB + 8 * 64 * 4;      // conv weights of the CTA's channels, (2+8)*128*8 B
@@ -209,42 +210,50 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
       a1 = fmaf(bf16_hi(w.z), x[1][e1], a1);
       a1 = fmaf(bf16_lo(w.w), x[2][e1], a1);
       a1 = fmaf(bf16_hi(w.w), x[3][e1], a1);
-      y[8 * g + e0] = silu_f(a0);
-      y[8 * g + e1] = silu_f(a1);
+      y[8 * g + e0] = silu_fast(a0);
+      y[8 * g + e1] = silu_fast(a1);
     }
   }
 }
 
 // One block diagonal of the blocked inverse: for blocks (I, J = I - d),
 //   M = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II M
-// with 16x16 blocks; all 256 threads, fixed trip counts.
+// with 16x16 blocks; each thread computes four adjacent columns of one row.
 template <int d>
 __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* sM, int tid) {
   constexpr int nb = 4 - d;
-  for (int x = tid; x < nb * 256; x += kPrepThreads) {
-    const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
+  if (tid < nb * 64) {
+    const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
     const float* arow = sA + (16 * I + ii) * kLdA + 16 * J;
-    const float* tcol = sT + (16 * J) * kLdA + 16 * J + jj;
-    float acc0 = 0.f, acc1 = 0.f;
+    const float* tcol = sT + (16 * J) * kLdT + 16 * J + j4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int kk = 0; kk < 16 * d; kk += 2) {
-      acc0 = fmaf(arow[kk], tcol[kk * kLdA], acc0);
-      acc1 = fmaf(arow[kk + 1], tcol[(kk + 1) * kLdA], acc1);
+    for (int kk = 0; kk < 16 * d; ++kk) {
+      const float a = arow[kk];
+      const float4 t = *reinterpret_cast<const float4*>(tcol + kk * kLdT);
+      acc.x = fmaf(a, t.x, acc.x);
+      acc.y = fmaf(a, t.y, acc.y);
+      acc.z = fmaf(a, t.z, acc.z);
+      acc.w = fmaf(a, t.w, acc.w);
     }
-    sM[x] = acc0 + acc1;
+    *reinterpret_cast<float4*>(sM + (J << 8) + (ii << 4) + j4) = acc;
   }
   __syncthreads();
-  for (int x = tid; x < nb * 256; x += kPrepThreads) {
-    const int J = x >> 8, I = J + d, ii = (x >> 4) & 15, jj = x & 15;
-    const float* trow = sT + (16 * I + ii) * kLdA + 16 * I;
-    const float* mcol = sM + (J << 8) + jj;
-    float acc0 = 0.f, acc1 = 0.f;
+  if (tid < nb * 64) {
+    const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
+    const float* trow = sT + (16 * I + ii) * kLdT + 16 * I;
+    const float* mcol = sM + (J << 8) + j4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int l = 0; l < 16; l += 2) {  // T_II is lower triangular: entries l > ii are zero
-      acc0 = fmaf(l <= ii ? trow[l] : 0.f, mcol[l << 4], acc0);
-      acc1 = fmaf(l + 1 <= ii ? trow[l + 1] : 0.f, mcol[(l + 1) << 4], acc1);
+    for (int l = 0; l < 16; ++l) {  // T_II is lower triangular (its upper part is stored as zeros)
+      const float a = trow[l];
+      const float4 m = *reinterpret_cast<const float4*>(mcol + (l << 4));
+      acc.x = fmaf(a, m.x, acc.x);
+      acc.y = fmaf(a, m.y, acc.y);
+      acc.z = fmaf(a, m.z, acc.z);
+      acc.w = fmaf(a, m.w, acc.w);
     }
-    sT[(16 * I + ii) * kLdA + 16 * J + jj] = -(acc0 + acc1);
+    *reinterpret_cast<float4*>(sT + (16 * I + ii) * kLdT + 16 * J + j4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
   }
   __syncthreads();
 }
@@ -267,7 +276,7 @@ __device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid)
       if (r & 1) acc0 = fmaf(sA[(16 * blk + r) * kLdA + 16 * blk + r - 1], x[r - 1], acc0);
       const float acc = acc0 + acc1;
       x[r] = r < col ? 0.f : (r == col ? 1.f : -acc);
-      sT[(16 * blk + r) * kLdA + 16 * blk + col] = x[r];
+      sT[(16 * blk + r) * kLdT + 16 * blk + col] = x[r];
     }
   }
   __syncthreads();
@@ -494,7 +503,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
 #pragma unroll
       for (int e2 = 0; e2 < 32; ++e2) {
         const int col = cbase + e2;
-        sA[ri * kLdA + col] = col < ri ? bi * expf(Gi - sG[j * 64 + col]) * acc[e2] : 0.f;
+        sA[ri * kLdA + col] = col < ri ? bi * __expf(Gi - sG[j * 64 + col]) * acc[e2] : 0.f;
       }
     } else {
 #pragma unroll
@@ -503,7 +512,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
           const int col = cbase + 8 * c2 + e2;
-          f[e2] = col <= ri ? expf(Gi - sG[j * 64 + col]) * acc[8 * c2 + e2] : 0.f;
+          f[e2] = col <= ri ? __expf(Gi - sG[j * 64 + col]) * acc[8 * c2 + e2] : 0.f;
         }
         uint4 hi, lo;
         split8(f, hi, lo);
@@ -520,7 +529,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) 
 #pragma unroll
       for (int e2 = 0; e2 < 8; ++e2) {
         const int col = 8 * cc + e2;
-        f[e2] = col <= r ? sT[r * kLdA + col] * sB[j * 64 + col] : 0.f;
+        f[e2] = col <= r ? sT[r * kLdT + col] * sB[j * 64 + col] : 0.f;
       }
       uint4 hi, lo;
       split8(f, hi, lo);

@@ -150,15 +150,18 @@ constexpr int kPrepThreads = 256;
 constexpr int kLdA = 65;                               // fp32 row stride of A in shared memory
 constexpr int kLdT = 68;                               // fp32 row stride of T (16-byte aligned rows)
 constexpr int kPrepOffQK = 0;                          // [Q;K] image hi, lo    2 x 32768
-constexpr int kPrepOffPI = kPrepOffQK + 2 * 32768;     // [P;I] image hi, lo    2 x 16384
-constexpr int kPrepOffTt = kPrepOffPI + 2 * 16384;     // T~ image (B) hi, lo   2 x 8192
+// After the [Q;K] K^T product has completed, the [Q;K] region is reused by the head loop:
+constexpr int kPrepOffTt = kPrepOffQK;                 // T~ image (B) hi, lo   2 x 8192
 constexpr int kPrepOffA = kPrepOffTt + 2 * 8192;       // A fp32                64*65*4
-constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32
+constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32                64*68*4
 constexpr int kPrepOffM = kPrepOffT + 64 * kLdT * 4;   // block-solve temp      3*256*4
-constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum [8][64]
+static_assert(kPrepOffM + 3 * 256 * 4 <= 2 * 32768, "head-loop buffers must fit the [Q;K] region");
+constexpr int kPrepOffPI = 2 * 32768;                  // [P;I] image hi, lo    2 x 16384
+constexpr int kPrepOffG = kPrepOffPI + 2 * 16384;      // G cumsum [8][64]
 constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta     [8][64]
-constexpr int kPrepOffW = kPrepOffB + 8 * 64 * 4;      // conv weights of the CTA's channels, (2+8)*128*8 B
-constexpr int kPrepSmem = kPrepOffW + 10 * 128 * 8 + 1024;
+constexpr int kPrepOffW = kPrepOffB + 8 * 64 * 4;      // conv weights of the CTA's channels, (2+G)*128*8 B
+// dynamic shared memory for G value heads per key head (1 KiB of alignment slack)
+__host__ __device__ constexpr int prep_smem_bytes(int G) { return kPrepOffW + (2 + G) * 128 * 8 + 1024; }
 
 // hi = bf16(f), lo = bf16(f - hi) for 8 values
 __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
@@ -293,7 +296,7 @@ __device__ __forceinline__ void umma_split(uint32_t d, uint64_t a_hi, uint64_t a
   umma_bf16(d, a_lo, b_hi, idesc, true);
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(PrefillParams p) {
+__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;
   extern __shared__ uint8_t prep_smem_raw[];
   uint8_t* sm = align1024(prep_smem_raw);
@@ -1013,9 +1016,10 @@ cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t st
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
   if (p.n_chunks > 0) {
-    err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrepSmem);
+    const int smem = prep_smem_bytes(p.H_v / p.H_k);
+    err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, kPrepSmem, stream>>>(p);
+    prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, smem, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);

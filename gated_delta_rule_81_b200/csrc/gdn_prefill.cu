@@ -597,8 +597,11 @@ struct ScanCfg {
   static constexpr int NB = DV / 32;                   // 32-column blocks per CTA
   static constexpr int TMEM_COLS = DV == 32 ? 256 : 512;
   static constexpr int COL_Z = 0;                      // S^T: lanes = d_k, DV columns
-  static constexpr int COL_X = DV;                     // X[b] = [Q;K] S^T at DV + 2 DV b
-  static constexpr int COL_Y = 2 * DV;                 // Y[b] = [P T~; T~] R at 2 DV + 2 DV b
+  // X = [Q;K] S^T and Y = [P T~; T~] R, each as two DV-column halves whose sum is
+  // the product: (hi.hi + lo.hi | hi.lo) -- the hi and lo B operands sit side by
+  // side along N so that A_hi [B_hi | B_lo] is one instruction.
+  static constexpr int COL_X = DV;
+  static constexpr int COL_Y = 3 * DV;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int OFF_GATE = kQKBytes;            // inside a [Q;K] stage
   static constexpr int QK_STAGE = kQKBytes + kGateBytes;
@@ -626,6 +629,13 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t base, int ks, uint32_t krow
   else return smem_desc(base + ks * 2048u, krows * 128u, 1024, Swz::k128);
 }
 
+// [hi | lo] as one 2*DV-wide MN-major operand: the lo image is the next MN block, img_bytes on
+template <int DV>
+__device__ __forceinline__ uint64_t mn_desc_cat(uint32_t base_hi, int ks, uint32_t img_bytes) {
+  if constexpr (DV == 32) return smem_desc(base_hi + ks * 1024u, img_bytes, 512, Swz::k64);
+  else return smem_desc(base_hi + ks * 2048u, img_bytes, 1024, Swz::k128);
+}
+
 // write 32 fp32 values (one thread's row segment, columns 32*cc..) as hi/lo bf16 into an MN-major image
 template <int DV>
 __device__ __forceinline__ void store_split_row(uint8_t* img_hi, int img_bytes, uint32_t krow, int cc, uint32_t krows,
@@ -647,7 +657,7 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;  // same value in every CTA of a cluster
   extern __shared__ uint8_t scan_smem_raw[];
   uint8_t* sm = align1024(scan_smem_raw);
-  __shared__ uint64_t qk_full[2], qk_empty[2], xyfree_b[2], mma2o_b[2], nfull_b[2], nack_b[2];
+  __shared__ uint64_t qk_full[2], qk_empty[2], xyfree_b, mma2o_b, nfull_b[2], nack_b[2];
   __shared__ uint64_t pt_full, pt_empty, v_full, v_empty;
   __shared__ uint64_t sready_b, mma1_b, rready_b, mma2_b, uready_b, mma3_b, drain_b;
   __shared__ uint32_t tmem_base_s;
@@ -672,13 +682,13 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&qk_full[b], 1);
       mbar_init(&qk_empty[b], 1 + 64);
-      mbar_init(&xyfree_b[b], 64);
-      mbar_init(&mma2o_b[b], 1);
       if (CS > 1) {
         mbar_init(&nfull_b[b], (CS - 1) * 64);
         mbar_init(&nack_b[b], (CS - 1) * 64);
       }
     }
+    mbar_init(&xyfree_b, 64);
+    mbar_init(&mma2o_b, 1);
     mbar_init(&pt_full, 1);
     mbar_init(&pt_empty, 1);
     mbar_init(&v_full, 1);
@@ -736,23 +746,25 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
   } else if (warp == 7) {
     // ------------------------------------------------ MMA issuer (one thread)
     if (lane == 0) {
-      const uint32_t idesc_xs = idesc_bf16(128, DV, false, true);
+      const uint32_t idesc_1 = idesc_bf16(128, DV, false, true);       // A_lo B_hi
+      const uint32_t idesc_2 = idesc_bf16(128, 2 * DV, false, true);   // A_hi [B_hi | B_lo]
       const uint32_t idesc_ku = idesc_bf16(128, DV, true, true);
       const uint32_t pt_hi = smem_u32(sm + Cfg::OFF_PT), pt_lo = pt_hi + kPTImg;
+      const uint32_t dX = tbase + Cfg::COL_X, dY = tbase + Cfg::COL_Y;
       for (int c = 0; c < nc; ++c) {
-        const int st = c & 1, xb = c & 1;
+        const int st = c & 1;
         if (!mbar_wait(&qk_full[st], (c >> 1) & 1, ab)) break;
         if (!mbar_wait(&sready_b, c & 1, ab)) break;
-        if (c >= 2 && !mbar_wait(&xyfree_b[xb], ((c >> 1) - 1) & 1, ab)) break;
+        if (c >= 1 && !mbar_wait(&xyfree_b, (c - 1) & 1, ab)) break;
         tc_fence_after();
         const uint32_t qk_hi = smem_u32(sm + st * Cfg::QK_STAGE), qk_lo = qk_hi + kQKImg;
-        const uint32_t dX = tbase + Cfg::COL_X + 2 * DV * xb, dY = tbase + Cfg::COL_Y + 2 * DV * xb;
         // X = [Q;K] S^T
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-          umma_split(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), smem_desc(qk_lo + ko, 16, 1024, Swz::k128),
-                     mn_desc<DV>(op_hi, ks, 128), mn_desc<DV>(op_lo, ks, 128), idesc_xs, ks > 0);
+          umma_bf16(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG), idesc_2,
+                    ks > 0);
+          umma_bf16(dX, smem_desc(qk_lo + ko, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 128), idesc_1, true);
         }
         umma_commit(&mma1_b);
         if (!mbar_wait(&rready_b, c & 1, ab)) break;
@@ -760,11 +772,13 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         tc_fence_after();
         // Y = [P T~; T~] R
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_split(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128),
-                     mn_desc<DV>(op_hi, ks, 64), mn_desc<DV>(op_lo, ks, 64), idesc_xs, ks > 0);
+        for (int ks = 0; ks < 4; ++ks) {
+          umma_bf16(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
+                    idesc_2, ks > 0);
+          umma_bf16(dY, smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64), idesc_1, true);
+        }
         umma_commit(&mma2_b);
-        umma_commit(&mma2o_b[xb]);
+        umma_commit(&mma2o_b);
         umma_commit(&pt_empty);
         if (!mbar_wait(&uready_b, c & 1, ab)) break;
         tc_fence_after();
@@ -790,7 +804,7 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     const long long srow0 = (static_cast<long long>(n) * p.H_v + h) * kD + static_cast<long long>(slice) * DV;
     bool ok = true;
     for (int c = 0; c < nc && ok; ++c) {
-      const int st = c & 1, xb = c & 1;
+      const int st = c & 1;
       const float* gates = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE);
       if (c > 0) {
         if (!(ok = mbar_wait_warp(&mma3_b, (c - 1) & 1, ab))) break;
@@ -828,9 +842,12 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         // R = v_hat - gamma (K S^T), into the operand buffer (S is no longer needed)
 #pragma unroll
         for (int cc = 0; cc < NB; ++cc) {
-          float x[32];
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 2 * DV * xb + 32 * cc), x);
+          float x[32], x2[32];
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), x);
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), x2);
           tmem_wait_ld();
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) x[e2] += x2[e2];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const float4 vv = vrow[(cc * 8 + q) * 64 + i];
@@ -851,11 +868,12 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         // U_d = decay-to-end * U, into the operand buffer (R is no longer needed)
 #pragma unroll
         for (int cc = 0; cc < NB; ++cc) {
-          float u[32];
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 2 * DV * xb + 32 * cc), u);
+          float u[32], u2[32];
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), u);
+          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), u2);
           tmem_wait_ld();
 #pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) u[e2] *= dcy;
+          for (int e2 = 0; e2 < 32; ++e2) u[e2] = (u[e2] + u2[e2]) * dcy;
           store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, u);
         }
         fence_proxy_async_smem();
@@ -895,29 +913,35 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     };
     if (nc > 0) load_z(0);
     for (int c = 0; c < nc; ++c) {
-      const int st = c & 1, xb = c & 1, pb = c & 1;
+      const int st = c & 1, pb = c & 1;
       if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab)) break;
       const float gam = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE)[i];
       mbar_arrive(&qk_empty[st]);  // only gamma is read from the stage
-      if (!mbar_wait_warp(&mma2o_b[xb], (c >> 1) & 1, ab)) break;
+      if (!mbar_wait_warp(&mma2o_b, c & 1, ab)) break;
       tc_fence_after();
-      const uint32_t cX = Cfg::COL_X + 2 * DV * xb, cY = Cfg::COL_Y + 2 * DV * xb;
-      // per-32-column partial sums of o^2, combined in a fixed order for every slicing
+      // o = gamma (X_a + X_b) + (Y_a + Y_b), kept in registers; per-32-column
+      // partial sums of o^2 are combined in a fixed order for every slicing
+      float o[DV];
       float part[NB];
 #pragma unroll
       for (int cc = 0; cc < NB; ++cc) {
-        float x[32], y[32];
-        tmem_ld32(tmem_addr(tbase, lb, cX + 32 * cc), x);
-        tmem_ld32(tmem_addr(tbase, lb, cY + 32 * cc), y);
+        float xa[32], xb2[32], ya[32], yb[32];
+        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), xa);
+        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), xb2);
+        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), ya);
+        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), yb);
         tmem_wait_ld();
         float ss = 0.f;
 #pragma unroll
         for (int e2 = 0; e2 < 32; ++e2) {
-          const float o = fmaf(gam, x[e2], y[e2]);
-          ss = fmaf(o, o, ss);
+          const float v = fmaf(gam, xa[e2] + xb2[e2], ya[e2] + yb[e2]);
+          o[32 * cc + e2] = v;
+          ss = fmaf(v, v, ss);
         }
         part[cc] = ss;
       }
+      tc_fence_before();
+      mbar_arrive(&xyfree_b);  // X and Y may be overwritten by the next chunk's products
       float total;
       if constexpr (CS == 1) {
         total = part[0];
@@ -947,26 +971,13 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
       uint4* orow = reinterpret_cast<uint4*>(p.out + ((valid ? tok : s) * p.H_v + h) * kD + slice * DV);
       uint4 ob[NB * 4];
 #pragma unroll
-      for (int cc = 0; cc < NB; ++cc) {
-        float x[32], y[32];
-        tmem_ld32(tmem_addr(tbase, lb, cX + 32 * cc), x);  // whole warp: tcgen05.ld is warp-aligned
-        tmem_ld32(tmem_addr(tbase, lb, cY + 32 * cc), y);
-        tmem_wait_ld();
+      for (int q = 0; q < NB * 4; ++q) {
+        float zz[8], f[8];
+        unpack8(zbuf[q], zz);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float zz[8], f[8];
-          unpack8(zbuf[cc * 4 + q4], zz);
-#pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) {
-            const int col = 32 * cc + 8 * q4 + e2;
-            const float o = fmaf(gam, x[8 * q4 + e2], y[8 * q4 + e2]);
-            f[e2] = o * inv * sNW[col] * silu_fast(zz[e2]);
-          }
-          ob[cc * 4 + q4] = pack8(f);
-        }
+        for (int e2 = 0; e2 < 8; ++e2) f[e2] = o[8 * q + e2] * inv * sNW[8 * q + e2] * silu_fast(zz[e2]);
+        ob[q] = pack8(f);
       }
-      tc_fence_before();
-      mbar_arrive(&xyfree_b[xb]);
       if (c + 1 < nc) load_z(c + 1);
       if (valid) {
 #pragma unroll

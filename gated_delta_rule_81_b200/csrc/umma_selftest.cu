@@ -12,7 +12,7 @@ namespace {
 // layout codes
 constexpr int kKMajor = 0;     // SW128, K-major
 constexpr int kMN128 = 1;      // SW128, MN-major (64-wide MN blocks, LBO apart)
-constexpr int kMN64 = 2;       // SW64, MN-major (32-wide MN block)
+constexpr int kMN64 = 2;       // SW64, MN-major (32-wide MN blocks, LBO apart)
 
 __device__ __forceinline__ uint32_t operand_off(int layout, int mn, int k, int MN, int K) {
   if (layout == kKMajor) {  // K blocks of 64 elements, each MN rows x 128 B
@@ -21,7 +21,8 @@ __device__ __forceinline__ uint32_t operand_off(int layout, int mn, int k, int M
   if (layout == kMN128) {  // MN blocks of 64 elements, each K rows x 128 B
     return static_cast<uint32_t>((mn >> 6) * (K * 128)) + sw128_off(k, (mn & 63) >> 3) + (mn & 7) * 2;
   }
-  return sw64_off(k, (mn & 31) >> 3) + (mn & 7) * 2;  // one 32-wide MN block
+  // 32-wide MN blocks of K rows x 64 B each
+  return static_cast<uint32_t>((mn >> 5) * (K * 64)) + sw64_off(k, (mn & 31) >> 3) + (mn & 7) * 2;
 }
 
 __device__ __forceinline__ uint64_t operand_desc(int layout, uint32_t base, int ks, int MN, int K) {
@@ -30,7 +31,7 @@ __device__ __forceinline__ uint64_t operand_desc(int layout, uint32_t base, int 
     return smem_desc(addr, 16, 1024, Swz::k128);
   }
   if (layout == kMN128) return smem_desc(base + ks * 2048, K * 128, 1024, Swz::k128);
-  return smem_desc(base + ks * 1024, 512, 512, Swz::k64);
+  return smem_desc(base + ks * 1024, K * 64, 512, Swz::k64);
 }
 
 __global__ void __launch_bounds__(128) umma_selftest_kernel(int a_layout, int b_layout, int N, int K,
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(128) umma_selftest_kernel(int a_layout, int b_
 }  // namespace
 
 // D = A * B^T for a 128 x K A and an N x K B (both bf16 row-major, device), fp32 D [128][N].
-// a_layout / b_layout: 0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64 (N = 32).
+// a_layout / b_layout: 0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64 (32-wide MN blocks).
 // Returns 0 on launch success, -1 on a bad argument, else the CUDA error code.
 extern "C" int gdn_selftest_umma(int a_layout, int b_layout, int N, int K, const void* A, const void* B,
                                  float* D, int* err, void* stream) {
@@ -104,7 +105,7 @@ extern "C" int gdn_selftest_umma(int a_layout, int b_layout, int N, int K, const
   if (a_layout == 2) return -1;
   if (a_layout == 1 && K % 16 != 0) return -1;
   if (b_layout == 1 && N % 64 != 0) return -1;
-  if (b_layout == 2 && N != 32) return -1;
+  if (b_layout == 2 && N % 32 != 0) return -1;
   size_t smem = static_cast<size_t>(128 + N) * K * 2 + 1024;
   cudaFuncSetAttribute(umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   umma_selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(

@@ -19,6 +19,8 @@ CASES = [
     (0, 1, 64, 128),    # [Q;K] S^T, 64 state rows
     (0, 2, 32, 128),    # [Q;K] S^T, 32 state rows
     (0, 2, 32, 64),     # [P T~; T~] R, 32 state rows
+    (0, 2, 64, 128),    # [Q;K] [S_hi | S_lo], 32 state rows (two SW64 blocks)
+    (0, 2, 64, 64),     # [P T~; T~] [R_hi | R_lo], 32 state rows
     (1, 1, 128, 64),    # K^T U
     (1, 1, 64, 64),
     (1, 2, 32, 64),

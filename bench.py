@@ -39,15 +39,23 @@ METRIC = "gated-delta prefill tokens/s per layer; decode state GB/s vs B200 HBM 
 # Algorithmic work per token of a chunk-64 prefill with d = 128 (16 key / 48 value heads):
 #   prep kernel: [Q;K]K^T per key head (4 C d) and the two T-products per value head (4 C d)
 #   scan kernel: W S^T, Q S^T, U^T K per value head (6 d^2) and P U (2 C d)
-PREP_FLOP_PER_TOKEN = 16 * 4 * 64 * 128 + 48 * 4 * 64 * 128          # 2,097,152
-SCAN_FLOP_PER_TOKEN = 48 * (6 * 128 * 128 + 2 * 64 * 128)             # 5,505,024
+def prep_flop_per_token(H_k=16, H_v=48, C=64, d=128):
+    return H_k * 4 * C * d + H_v * 4 * C * d          # 2,097,152 at 16/48 heads
+
+
+def scan_flop_per_token(H_v=48, C=64, d=128):
+    return H_v * (6 * d * d + 2 * C * d)              # 5,505,024 at 48 value heads
+
+
+PREP_FLOP_PER_TOKEN = prep_flop_per_token()
+SCAN_FLOP_PER_TOKEN = scan_flop_per_token()
 PREFILL_FLOP_PER_TOKEN = PREP_FLOP_PER_TOKEN + SCAN_FLOP_PER_TOKEN     # 7,602,176
 PREFILL_BYTES_PER_TOKEN = 20480 + 12288 + 12288 + 192                  # q,k,v + z + out + a,b
 DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 state read + write
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {}
+TRAFFIC = {"scan": {"bytes": 325274624 + 42740736, "sha": "eb5fa90e952f2519"}}  # ncu, T=4096 layer
 
 
 def src_sha(name):
@@ -164,32 +172,37 @@ def flush_l2(buf):
     buf.add_(1)  # 256 MiB read + write, more than the 126 MB L2
 
 
-def prefill_workload(seed, dev):
-    case = gin.prefill_case(1, seed=seed)
-    inp = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in case["inp"].items()}
-    st = case["state_in"].to(dev)
-    return case, inp, st
+WORKLOADS = {"prefill4k": 1, "tiny": 0, "fullctx": 2, "varlen": 3}
 
 
-def run_prefill_ours(args, world, rank, dev, pk):
+def run_prefill_ours(args, world, rank, dev, pk, cfg_id=1):
     from gated_delta_rule_81_b200 import gdn
 
-    case, inp, st = prefill_workload(seed=rank, dev=dev)
-    B, T = 1, case["T_tot"]
+    case = gin.prefill_case(cfg_id, seed=rank)
+    inp = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in case["inp"].items()}
+    st = case["state_in"].to(dev) if case["state_in"] is not None else None
+    varlen = gin.CONFIGS[cfg_id]["kind"] == "varlen"
+    N, T_tot = case["N"], case["T_tot"]
     s = gdn.make_inputs(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["z"], inp["conv_w"], inp["A_log"],
                         inp["norm_w"], scale=inp["scale"])
     H_k, H_v = s.H_k, s.H_v
-    n_chunks = B * math.ceil(T / 64)
-    ws = torch.empty(gdn.workspace_size(H_k, H_v, B, n_chunks), dtype=torch.uint8, device=dev)
-    out = torch.empty(T, H_v, 128, dtype=torch.bfloat16, device=dev)
-    S_out = torch.empty_like(st)
-    C_out = torch.empty(B, 3, (2 * H_k + H_v) * 128, dtype=torch.bfloat16, device=dev)
+    n_chunks = gdn.chunk_count(case["lengths"])
+    ws = torch.empty(gdn.workspace_size(H_k, H_v, N, n_chunks), dtype=torch.uint8, device=dev)
+    out = torch.empty(T_tot, H_v, 128, dtype=torch.bfloat16, device=dev)
+    S_out = torch.empty(N, H_v, 128, 128, dtype=torch.float32, device=dev)
+    C_out = torch.empty(N, 3, (2 * H_k + H_v) * 128, dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
     stream = torch.cuda.current_stream()
+    cu_dev = case["cu_seqlens"].to(dev)
 
     def step():
-        gdn.prefill(s, B, T, st, None, out=out, state_out=S_out, conv_out=C_out, workspace=ws, err=err)
+        if varlen:
+            gdn.prefill_varlen(s, cu_dev, case["cu_seqlens"], st, None, out=out, state_out=S_out, conv_out=C_out,
+                               workspace=ws, err=err)
+        else:
+            gdn.prefill(s, N, case["lengths"][0], st, None, out=out, state_out=S_out, conv_out=C_out, workspace=ws,
+                        err=err)
 
     for _ in range(args.warmup):
         flush_l2(flush)
@@ -197,7 +210,7 @@ def run_prefill_ours(args, world, rank, dev, pk):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    # per timed step: [step start] conv-state kernel [lib 0] prep [lib 1] scan [lib 2] [step end]
+    # per timed step: [step start] helper kernels [lib 0] prep [lib 1] scan [lib 2] [step end]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     hooks = []
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -216,10 +229,11 @@ def run_prefill_ours(args, world, rank, dev, pk):
     total_ms = max_over_ranks(sum(step_ms), world)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())}")
-    return {"total_ms": total_ms, "step_ms": step_ms, "T": T, "clocks": clk.report(), "launches_per_step": 3,
-            "case": case, "kernel_ms": {"prep": statistics.mean(prep_ms), "scan": statistics.mean(scan_ms),
-                                        "conv_state+gaps": statistics.mean(step_ms) - statistics.mean(prep_ms)
-                                        - statistics.mean(scan_ms)}}
+    return {"total_ms": total_ms, "step_ms": step_ms, "T": T_tot, "clocks": clk.report(),
+            "launches_per_step": 4 if varlen else 3, "case": case, "H_k": H_k, "H_v": H_v, "N": N,
+            "kernel_ms": {"prep": statistics.mean(prep_ms), "scan": statistics.mean(scan_ms),
+                          "helpers+gaps": statistics.mean(step_ms) - statistics.mean(prep_ms)
+                          - statistics.mean(scan_ms)}}
 
 
 def run_e2e_prefill(args, world, rank, dev, case):
@@ -358,6 +372,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode"], default="prefill4k",
+                    help="prefill4k (default, the headline line) or another configuration for the record")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
@@ -376,7 +392,19 @@ def main():
     gdn.load()
     pk = peaks()
 
-    res = run_prefill_ours(args, world, rank, dev, pk)
+    if args.workload == "decode":
+        d = run_decode_ours(args, dev)
+        if rank == 0:
+            print(json.dumps({"metric": "decode state GB/s", "value": d["gbs"], "unit": "GB/s", "n_gpus": world,
+                              "steps": 64, "warmup": 3, "ms_per_step": d["ms_per_launch"], "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                              "config": {"workload": gin.CONFIGS[4]["name"]},
+                              "roofline": {"bound": "hbm", "achieved": d["gbs"], "peak": pk["hbm_gbs"],
+                                           "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"], "traffic": None},
+                              "gpu_launches": 64}), flush=True)
+        return 0
+    cfg_id = WORKLOADS[args.workload]
+    res = run_prefill_ours(args, world, rank, dev, pk, cfg_id)
     T = res["T"]
     total_ms = res["total_ms"]
     value = world * T * args.steps / (total_ms / 1e3)
@@ -385,17 +413,31 @@ def main():
     # dominant kernel, timed live in the timed region with the library's event hook
     kt = res["kernel_ms"]
     dom = "scan" if kt["scan"] >= kt["prep"] else "prep"
-    flops = (SCAN_FLOP_PER_TOKEN if dom == "scan" else PREP_FLOP_PER_TOKEN) * T
+    flops = (scan_flop_per_token(res["H_v"]) if dom == "scan" else prep_flop_per_token(res["H_k"], res["H_v"])) * T
+    step_flops = (scan_flop_per_token(res["H_v"]) + prep_flop_per_token(res["H_k"], res["H_v"])) * T
     achieved = flops / (kt[dom] * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
     tr = TRAFFIC.get(dom)
-    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") else None
+    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") and cfg_id == 1 else None
     roof = {"kernel": f"{dom}_kernel", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic, "peak_source": f"{pk['source']} (bf16 burst)",
             "algorithmic_flop_per_launch": flops, "launch_ms": kt[dom],
             "kernel_ms": {k: round(v, 5) for k, v in kt.items()},
-            "whole_step": {"achieved": PREFILL_FLOP_PER_TOKEN * T / (ms_per_step * 1e-3) / 1e12,
-                           "frac": PREFILL_FLOP_PER_TOKEN * T / (ms_per_step * 1e-3) / 1e12 / peak}}
+            "whole_step": {"achieved": step_flops / (ms_per_step * 1e-3) / 1e12,
+                           "frac": step_flops / (ms_per_step * 1e-3) / 1e12 / peak}}
+    if cfg_id != 1:
+        if rank == 0:
+            c = gin.CONFIGS[cfg_id]
+            print(json.dumps({"metric": "gated-delta prefill tokens/s per layer", "value": value, "unit": "tokens/s",
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                              "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                              "config": {"workload": c["name"], "sequences": res["N"], "tokens": T,
+                                         "H_k": res["H_k"], "H_v": res["H_v"], "head_dim": 128, "chunk": 64,
+                                         "l2": "flushed between timed steps"},
+                              "roofline": roof, "gpu_launches": res["launches_per_step"] * args.steps,
+                              "clocks": res["clocks"]}), flush=True)
+        return 0
 
     e2e = None if args.no_e2e else run_e2e_prefill(args, world, rank, dev, res["case"])
     decode = None

@@ -155,14 +155,26 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_sequences(lengths, world, rank):
+    """Indices of the sequences rank `rank` runs: greedy longest-first onto the
+    least-loaded rank (sequences are independent, so no exchange is needed)."""
+    loads = [0] * world
+    owner = {}
+    for i in sorted(range(len(lengths)), key=lambda j: (-lengths[j], j)):
+        r = min(range(world), key=lambda k: (loads[k], k))
+        owner[i] = r
+        loads[r] += lengths[i]
+    return [i for i in range(len(lengths)) if owner[i] == rank]
 
 
 # ------------------------------------------------------------------ workloads

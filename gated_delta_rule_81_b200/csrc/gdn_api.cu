@@ -115,6 +115,7 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.cu = cu;
   p.T_uniform = T_uniform;
   p.n_chunks = n_chunks;
+  p.T_total = T_tot;
   p.ws_flag = reinterpret_cast<int*>(ws);
   p.chunk_base = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) : nullptr;
   p.ws_qk = ws + gdn::kWsHeader + chunk_base_bytes(N);

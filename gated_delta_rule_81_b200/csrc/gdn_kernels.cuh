@@ -49,6 +49,7 @@ struct PrefillParams {
   const int* cu;          // device cu_seqlens [N+1], or null for uniform length T_uniform
   int T_uniform;
   long long n_chunks;     // total chunks (host count)
+  long long T_total;      // total tokens (host count)
   int* chunk_base;        // [N+1] in the workspace (varlen), or null (uniform)
   int* ws_flag;           // workspace header word: nonzero = inconsistent cu_seqlens
   uint8_t* ws_qk;         // [n_chunks][H_k][kQKBytes]

@@ -76,12 +76,13 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
 // ============================================================ helpers
 
 // chunk_base[n] = sum_{m<n} ceil(L_m / 64) from the device cu_seqlens; checks
-// that it agrees with the host-side count and that cu_seqlens is valid.
+// that the device copy is valid (cu[0] = 0, non-decreasing) and agrees with the
+// host copy in its number of chunks and its total number of tokens.
 __global__ void __launch_bounds__(1024) setup_kernel(PrefillParams p) {
   __shared__ long long part[1024];
   __shared__ int bad_s;
   const int tid = threadIdx.x;
-  if (tid == 0) bad_s = (p.cu[0] != 0);
+  if (tid == 0) bad_s = (p.cu[0] != 0) || (static_cast<long long>(p.cu[p.N]) != p.T_total);
   __syncthreads();
   const int per = (p.N + 1023) / 1024;
   const int n0 = min(tid * per, p.N), n1 = min(n0 + per, p.N);

@@ -115,9 +115,10 @@ gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in
  *   cu_seqlens       device int32 [N+1], cu[0] = 0, non-decreasing; sequence n is
  *                    tokens cu[n] .. cu[n+1]-1
  *   cu_seqlens_host  host copy of the same values (used to size the launch);
- *                    validated on the host, and the device copy is checked
- *                    against it on the device (mismatch: nothing is computed
- *                    and *err gets bit 4)
+ *                    validated on the host.  The device copy is checked on the
+ *                    device: cu[0] = 0, non-decreasing, and the same number of
+ *                    chunks and total tokens as the host copy (otherwise nothing
+ *                    is computed and *err gets bit 4)
  * Every sequence starts from its own state_in[n] / conv_in[n] (or zeros): state
  * and conv history never cross a cu_seqlens boundary.  Results for sequence n
  * are bitwise identical to a gdn_prefill of that sequence alone with the same

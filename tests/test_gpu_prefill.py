@@ -206,3 +206,57 @@ def test_empty_batch_and_empty_sequences():
     assert torch.equal(S.cpu(), case["state_in"])
     ref = run_oracle(case)
     np.testing.assert_array_equal(C.float().cpu().numpy(), ref["conv"])
+
+
+# ------------------------------------------------------------------ layouts, head groupings, failure detection
+
+
+def test_strided_inputs_from_one_projection_buffer():
+    """q, k, v, z, a, b as column slices of one [T, proj] buffer (token stride = proj width)."""
+    H_k, H_v, T = 2, 6, 150
+    case = small_case([T], H_k=H_k, H_v=H_v, with_conv=True)
+    inp = case["inp"]
+    parts = [inp["q"].reshape(T, -1), inp["k"].reshape(T, -1), inp["v"].reshape(T, -1), inp["z"].reshape(T, -1),
+             inp["a"], inp["b"], torch.zeros(T, 4, dtype=torch.bfloat16)]  # pad the row to a 16-byte multiple
+    proj = torch.cat(parts, dim=1).cuda()
+    assert (proj.shape[1] * 2) % 16 == 0
+    o = 0
+    views = {}
+    for name, t in zip(("q", "k", "v", "z", "a", "b"), parts):
+        views[name] = proj[:, o:o + t.shape[1]]
+        o += t.shape[1]
+    views["q"] = views["q"].unflatten(1, (H_k, 128))
+    views["k"] = views["k"].unflatten(1, (H_k, 128))
+    views["v"] = views["v"].unflatten(1, (H_v, 128))
+    views["z"] = views["z"].unflatten(1, (H_v, 128))
+    w = {k: inp[k].cuda() for k in ("conv_w", "A_log", "norm_w")}
+    s = gdn.make_inputs(views["q"], views["k"], views["v"], views["a"], views["b"], views["z"], w["conv_w"],
+                        w["A_log"], w["norm_w"])
+    assert s.stride_q == proj.shape[1] and s.stride_a == proj.shape[1]
+    err = err_word()
+    out, S, C = gdn.prefill(s, 1, T, case["state_in"].cuda(), case["conv_in"].cuda(), err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    check(case, out, S, C, run_oracle(case))
+
+
+@pytest.mark.parametrize("H_k,H_v", [(4, 8), (1, 8), (3, 3)])
+def test_other_head_groupings(H_k, H_v):
+    case = small_case([70, 129], H_k=H_k, H_v=H_v, with_conv=True)
+    out, S, C = run_gpu(case)
+    check(case, out, S, C, run_oracle(case))
+
+
+def test_device_cu_seqlens_mismatch_is_reported_not_computed():
+    """The device copy of cu_seqlens disagrees with the host copy: the setup kernel
+    detects it, sets error bit 4 and every other kernel skips its work."""
+    case = small_case([64, 64])
+    keep, s = device_inputs(case["inp"])
+    cu_host = case["cu_seqlens"]
+    cu_bad = torch.tensor([0, 64, 100], dtype=torch.int32, device="cuda")  # host says 128 tokens
+    err = err_word()
+    out = torch.full((128, case["H_v"], 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    gdn.prefill_varlen(s, cu_bad, cu_host, None, None, out=out, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 4
+    assert torch.all(out == 7.0)  # nothing was written

@@ -813,21 +813,24 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
       }
       if (!(ok = mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab))) break;
       const float gC = gates[128];
+      float v[NB][32];
+      if (c == 0) {
 #pragma unroll
-      for (int cc = 0; cc < NB; ++cc) {
-        float v[32];
-        if (c == 0) {
+        for (int cc = 0; cc < NB; ++cc)
 #pragma unroll
           for (int e2 = 0; e2 < 32; ++e2)
-            v[e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
-        } else {
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
-          tmem_wait_ld();
-        }
-        store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v);
+            v[cc][e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
+      } else {
 #pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) v[e2] *= gC;
-        tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
+        for (int cc = 0; cc < NB; ++cc) tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
+        tmem_wait_ld();  // one wait for all column blocks
+      }
+#pragma unroll
+      for (int cc = 0; cc < NB; ++cc) {
+        store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v[cc]);
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) v[cc][e2] *= gC;
+        tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
       }
       tmem_wait_st();
       fence_proxy_async_smem();

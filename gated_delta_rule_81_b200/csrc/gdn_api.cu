@@ -20,7 +20,8 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
-size_t chunk_base_bytes(int N) { return round_up(sizeof(int) * (static_cast<size_t>(N) + 1), 1024); }
+// chunk_base[N+1] and seq_order[N] (ints) after the 1 KiB header
+size_t chunk_base_bytes(int N) { return round_up(sizeof(int) * (2 * static_cast<size_t>(N) + 1), 1024); }
 
 // Common checks of the per-token inputs; T_tot tokens.
 gdn_status check_inputs(const gdn_inputs* in, long long T_tot) {
@@ -118,6 +119,7 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.T_total = T_tot;
   p.ws_flag = reinterpret_cast<int*>(ws);
   p.chunk_base = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) : nullptr;
+  p.seq_order = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) + (N + 1) : nullptr;
   p.ws_qk = ws + gdn::kWsHeader + chunk_base_bytes(N);
   p.ws_head = p.ws_qk + static_cast<size_t>(n_chunks) * in->H_k * gdn::kQKBytes;
   p.state_in = state_in;

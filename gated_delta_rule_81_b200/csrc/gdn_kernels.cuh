@@ -51,6 +51,7 @@ struct PrefillParams {
   long long n_chunks;     // total chunks (host count)
   long long T_total;      // total tokens (host count)
   int* chunk_base;        // [N+1] in the workspace (varlen), or null (uniform)
+  int* seq_order;         // [N] scan order, longest first (varlen), or null
   int* ws_flag;           // workspace header word: nonzero = inconsistent cu_seqlens
   uint8_t* ws_qk;         // [n_chunks][H_k][kQKBytes]
   uint8_t* ws_head;       // [n_chunks][H_v][kHeadBytes]

@@ -30,6 +30,8 @@ namespace gdn {
 namespace {
 
 constexpr int kDevErrBadSeqlens = 4;
+constexpr int kMaxOrdered = 8192;  // sequences reordered longest-first for the scan
+constexpr unsigned kBackoffNs = 64;  // poll back-off of the producer and output warps
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -52,6 +54,22 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Named barrier over `nthreads` threads that also ORs a per-thread predicate:
+// every participant gets the same answer.  The non-aligned form, so the lanes of
+// a warp may arrive at different times (one lane may still be issuing MMAs).
+__device__ __forceinline__ bool bar_sync_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ float ld_shared_remote(const float* p, uint32_t cta) {
@@ -111,6 +129,19 @@ __global__ void __launch_bounds__(1024) setup_kernel(PrefillParams p) {
   if (tid == 1023) {
     p.chunk_base[p.N] = static_cast<int>(part[1023]);
     if (part[1023] != p.n_chunks) atomicOr(&bad_s, 1);
+  }
+  // scan order: longest sequence first (ties by index), so the longest chains start
+  // in the first wave; beyond kMaxOrdered sequences the pack order is kept
+  if (p.N <= kMaxOrdered) {
+    for (int nn = tid; nn < p.N; nn += 1024) {
+      const int Ln = p.cu[nn + 1] - p.cu[nn];
+      int rank = 0;
+      for (int m = 0; m < p.N; ++m) {
+        const int Lm = p.cu[m + 1] - p.cu[m];
+        rank += (Lm > Ln || (Lm == Ln && m < nn)) ? 1 : 0;
+      }
+      p.seq_order[rank] = nn;
+    }
   }
   __syncthreads();
   if (tid == 0) {
@@ -660,14 +691,15 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
   uint8_t* sm = align1024(scan_smem_raw);
   __shared__ uint64_t qk_full[2], qk_empty[2], xyfree_b, mma2o_b, nfull_b[2], nack_b[2];
   __shared__ uint64_t pt_full, pt_empty, v_full, v_empty;
-  __shared__ uint64_t sready_b, mma1_b, rready_b, mma2_b, uready_b, mma3_b, drain_b;
+  __shared__ uint64_t mma1_b, mma2_b, mma3_b, drain_b, drain2_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
   const int unit = blockIdx.x / CS;
-  const int n = unit / p.H_v, h = unit % p.H_v;
+  const int n_rank = unit / p.H_v, h = unit % p.H_v;
+  const int n = (p.seq_order && p.N <= kMaxOrdered) ? p.seq_order[n_rank] : n_rank;
   const int G = p.H_v / p.H_k, kh = h / G;
   const int slice = static_cast<int>(rank);
   const long long s = seq_start(p, n), e = seq_start(p, n + 1);
@@ -694,13 +726,11 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     mbar_init(&pt_empty, 1);
     mbar_init(&v_full, 1);
     mbar_init(&v_empty, 64);
-    mbar_init(&sready_b, 128);
     mbar_init(&mma1_b, 1);
-    mbar_init(&rready_b, 64);
     mbar_init(&mma2_b, 1);
-    mbar_init(&uready_b, 64);
     mbar_init(&mma3_b, 1);
     mbar_init(&drain_b, 1);
+    mbar_init(&drain2_b, 1);
     fence_mbar_init();
   }
   if (warp == 7) tmem_alloc<Cfg::TMEM_COLS>(&tmem_base_s);
@@ -721,12 +751,12 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         const long long gc = cb + c;
         const uint8_t* hb = p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes);
         uint8_t* stage = sm + st * Cfg::QK_STAGE;
-        if (c >= 2 && !mbar_wait(&qk_empty[st], ((c >> 1) - 1) & 1, ab)) break;
+        if (c >= 2 && !mbar_wait(&qk_empty[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&qk_full[st], Cfg::QK_TX);
         bulk_g2s(stage, p.ws_qk + (gc * p.H_k + kh) * static_cast<long long>(kQKBytes), kQKBytes, &qk_full[st]);
         bulk_g2s(stage + Cfg::OFF_GATE, hb + kPTBytes + kVBytes, kGateBytes, &qk_full[st]);
         ++qk_issued[st];
-        if (c >= 1 && !mbar_wait(&pt_empty, (c - 1) & 1, ab)) break;
+        if (c >= 1 && !mbar_wait(&pt_empty, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&pt_full, kPTBytes);
         bulk_g2s(sm + Cfg::OFF_PT, hb, kPTBytes, &pt_full);
         ++pt_issued;
@@ -744,46 +774,143 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
       if (v_issued > 0) mbar_wait(&v_full, (v_issued - 1) & 1, drain);
     }
     __syncwarp();
-  } else if (warp == 7) {
-    // ------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
-      const uint32_t idesc_1 = idesc_bf16(128, DV, false, true);       // A_lo B_hi
-      const uint32_t idesc_2 = idesc_bf16(128, 2 * DV, false, true);   // A_hi [B_hi | B_lo]
-      const uint32_t idesc_ku = idesc_bf16(128, DV, true, true);
-      const uint32_t pt_hi = smem_u32(sm + Cfg::OFF_PT), pt_lo = pt_hi + kPTImg;
-      const uint32_t dX = tbase + Cfg::COL_X, dY = tbase + Cfg::COL_Y;
-      for (int c = 0; c < nc; ++c) {
-        const int st = c & 1;
-        if (!mbar_wait(&qk_full[st], (c >> 1) & 1, ab)) break;
-        if (!mbar_wait(&sready_b, c & 1, ab)) break;
-        if (c >= 1 && !mbar_wait(&xyfree_b, (c - 1) & 1, ab)) break;
+  } else if (warp < 4) {
+    // ------------------------------------------------ state (threads 0..127), chain (64..127) and
+    // the tensor-core issue: thread 0 issues X = [Q;K] S^T, thread 64 issues Y and the state
+    // update.  Warps 0-3 pass the same three named barriers every chunk; each barrier ORs a
+    // "something failed" predicate, so all four warps leave the loop at the same barrier.
+    const int t = tid;  // TMEM lane = d_k index
+    const uint32_t lb = 32 * warp;
+    const long long srow0 = (static_cast<long long>(n) * p.H_v + h) * kD + static_cast<long long>(slice) * DV;
+    const uint32_t idesc_1 = idesc_bf16(128, DV, false, true);       // A_lo B_hi
+    const uint32_t idesc_2 = idesc_bf16(128, 2 * DV, false, true);   // A_hi [B_hi | B_lo]
+    const uint32_t idesc_ku = idesc_bf16(128, DV, true, true);
+    const uint32_t pt_hi = smem_u32(sm + Cfg::OFF_PT), pt_lo = pt_hi + kPTImg;
+    const uint32_t dX = tbase + Cfg::COL_X, dY = tbase + Cfg::COL_Y;
+    bool ok = true;
+    for (int c = 0; c < nc; ++c) {
+      const int st = c & 1;
+      const float* gates = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE);
+      const uint32_t qk_hi = smem_u32(sm + st * Cfg::QK_STAGE), qk_lo = qk_hi + kQKImg;
+      // ---- state: S_{c-1} -> hi/lo operand image; S^T <- gamma_C S^T in TMEM
+      bool w = c == 0 || mbar_wait_warp(&mma3_b, (c - 1) & 1, ab);
+      if (w) w = mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab);
+      if (w) {
         tc_fence_after();
-        const uint32_t qk_hi = smem_u32(sm + st * Cfg::QK_STAGE), qk_lo = qk_hi + kQKImg;
-        // X = [Q;K] S^T
+        const float gC = gates[128];
+        float v[NB][32];
+        if (c == 0) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-          umma_bf16(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG), idesc_2,
-                    ks > 0);
-          umma_bf16(dX, smem_desc(qk_lo + ko, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 128), idesc_1, true);
-        }
-        umma_commit(&mma1_b);
-        if (!mbar_wait(&rready_b, c & 1, ab)) break;
-        if (!mbar_wait(&pt_full, c & 1, ab)) break;
-        tc_fence_after();
-        // Y = [P T~; T~] R
+          for (int cc = 0; cc < NB; ++cc)
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          umma_bf16(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
-                    idesc_2, ks > 0);
-          umma_bf16(dY, smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64), idesc_1, true);
+            for (int e2 = 0; e2 < 32; ++e2)
+              v[cc][e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < NB; ++cc) tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
+          tmem_wait_ld();  // one wait for all column blocks
         }
-        umma_commit(&mma2_b);
-        umma_commit(&mma2o_b);
-        umma_commit(&pt_empty);
-        if (!mbar_wait(&uready_b, c & 1, ab)) break;
+#pragma unroll
+        for (int cc = 0; cc < NB; ++cc) {
+          store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v[cc]);
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) v[cc][e2] *= gC;
+          tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      if (bar_sync_or(1, 128, !w)) { ok = false; break; }
+      bool issued = true;
+      if (t == 0) {  // X = [Q;K] S^T
+        issued = c == 0 || mbar_wait(&xyfree_b, (c - 1) & 1, ab);
+        if (issued) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
+            umma_bf16(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
+                      idesc_2, ks > 0);
+            umma_bf16(dX, smem_desc(qk_lo + ko, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 128), idesc_1, true);
+          }
+          umma_commit(&mma1_b);
+        }
+      }
+      // ---- chain: R = v_hat - gamma (K S^T)
+      w = true;
+      if (t >= 64) {
+        const int i = t - 64;
+        w = mbar_wait_warp(&mma1_b, c & 1, ab);
+        if (w) w = mbar_wait_warp(&v_full, c & 1, ab);
+        if (w) {
+          tc_fence_after();
+          const float gam = gates[i];
+          const float4* vrow = reinterpret_cast<const float4*>(sm + Cfg::OFF_V);
+#pragma unroll
+          for (int cc = 0; cc < NB; ++cc) {
+            float x[32], x2[32];
+            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), x);
+            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), x2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) x[e2] += x2[e2];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 vv = vrow[(cc * 8 + q) * 64 + i];
+              x[4 * q + 0] = fmaf(-gam, x[4 * q + 0], vv.x);
+              x[4 * q + 1] = fmaf(-gam, x[4 * q + 1], vv.y);
+              x[4 * q + 2] = fmaf(-gam, x[4 * q + 2], vv.z);
+              x[4 * q + 3] = fmaf(-gam, x[4 * q + 3], vv.w);
+            }
+            store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, x);
+          }
+          mbar_arrive(&v_empty);
+          fence_proxy_async_smem();
+        }
+      }
+      tc_fence_before();
+      if (bar_sync_or(2, 128, !w || !issued)) { ok = false; break; }
+      if (t == 64) {  // Y = [P T~; T~] R
+        issued = mbar_wait(&pt_full, c & 1, ab);
+        if (issued) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            umma_bf16(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
+                      idesc_2, ks > 0);
+            umma_bf16(dY, smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64), idesc_1, true);
+          }
+          umma_commit(&mma2_b);
+          umma_commit(&mma2o_b);
+          umma_commit(&pt_empty);
+        }
+      }
+      // ---- chain: U_d = decay-to-end * U
+      w = true;
+      if (t >= 64) {
+        const int i = t - 64;
+        w = mbar_wait_warp(&mma2_b, c & 1, ab);
+        if (w) {
+          tc_fence_after();
+          const float dcy = gates[64 + i];
+#pragma unroll
+          for (int cc = 0; cc < NB; ++cc) {
+            float u[32], u2[32];
+            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), u);
+            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), u2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) u[e2] = (u[e2] + u2[e2]) * dcy;
+            store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, u);
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      tc_fence_before();
+      if (bar_sync_or(3, 128, !w || !issued)) { ok = false; break; }
+      if (t == 64) {  // S^T += K^T U_d
         tc_fence_after();
-        // S^T += K^T U_d
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           umma_split(tbase + Cfg::COL_Z, smem_desc(qk_hi + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
@@ -792,98 +919,14 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         umma_commit(&mma3_b);
         umma_commit(&qk_empty[st]);
       }
-      umma_commit(&drain_b);
+    }
+    // every MMA this thread issued has completed before TMEM is read or released
+    if (t == 0 || t == 64) {
+      uint64_t* db = t == 0 ? &drain_b : &drain2_b;
+      umma_commit(db);
       int drain_flag = 0;
       Abort drain{nullptr, &drain_flag};
-      mbar_wait(&drain_b, 0, drain);
-    }
-    __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------ state (threads 0..127) and chain (64..127)
-    const int t = tid;  // TMEM lane = d_k index
-    const uint32_t lb = 32 * warp;
-    const long long srow0 = (static_cast<long long>(n) * p.H_v + h) * kD + static_cast<long long>(slice) * DV;
-    bool ok = true;
-    for (int c = 0; c < nc && ok; ++c) {
-      const int st = c & 1;
-      const float* gates = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE);
-      if (c > 0) {
-        if (!(ok = mbar_wait_warp(&mma3_b, (c - 1) & 1, ab))) break;
-        tc_fence_after();
-      }
-      if (!(ok = mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab))) break;
-      const float gC = gates[128];
-      float v[NB][32];
-      if (c == 0) {
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc)
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2)
-            v[cc][e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc) tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
-        tmem_wait_ld();  // one wait for all column blocks
-      }
-#pragma unroll
-      for (int cc = 0; cc < NB; ++cc) {
-        store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v[cc]);
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) v[cc][e2] *= gC;
-        tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&sready_b);
-      if (t >= 64) {
-        const int i = t - 64;
-        if (!(ok = mbar_wait_warp(&mma1_b, c & 1, ab))) break;
-        if (!(ok = mbar_wait_warp(&v_full, c & 1, ab))) break;
-        tc_fence_after();
-        const float gam = gates[i];
-        const float4* vrow = reinterpret_cast<const float4*>(sm + Cfg::OFF_V);
-        // R = v_hat - gamma (K S^T), into the operand buffer (S is no longer needed)
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc) {
-          float x[32], x2[32];
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), x);
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), x2);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) x[e2] += x2[e2];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 vv = vrow[(cc * 8 + q) * 64 + i];
-            x[4 * q + 0] = fmaf(-gam, x[4 * q + 0], vv.x);
-            x[4 * q + 1] = fmaf(-gam, x[4 * q + 1], vv.y);
-            x[4 * q + 2] = fmaf(-gam, x[4 * q + 2], vv.z);
-            x[4 * q + 3] = fmaf(-gam, x[4 * q + 3], vv.w);
-          }
-          store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, x);
-        }
-        mbar_arrive(&v_empty);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&rready_b);
-        if (!(ok = mbar_wait_warp(&mma2_b, c & 1, ab))) break;
-        tc_fence_after();
-        const float dcy = gates[64 + i];
-        // U_d = decay-to-end * U, into the operand buffer (R is no longer needed)
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc) {
-          float u[32], u2[32];
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), u);
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), u2);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) u[e2] = (u[e2] + u2[e2]) * dcy;
-          store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, u);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&uready_b);
-      }
+      mbar_wait(db, 0, drain);
     }
     // final state of this slice
     if (p.state_out) {
@@ -902,7 +945,7 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
         }
       }
     }
-  } else {
+  } else if (warp >= 4 && warp < 6) {
     // ------------------------------------------------ output (warps 4, 5): token i = TMEM lane i
     const int i = tid - 128;
     const uint32_t lb = 32 * (warp & 3);
@@ -918,10 +961,10 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
     if (nc > 0) load_z(0);
     for (int c = 0; c < nc; ++c) {
       const int st = c & 1, pb = c & 1;
-      if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab)) break;
+      if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab, false, kBackoffNs)) break;
       const float gam = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE)[i];
       mbar_arrive(&qk_empty[st]);  // only gamma is read from the stage
-      if (!mbar_wait_warp(&mma2o_b, c & 1, ab)) break;
+      if (!mbar_wait_warp(&mma2o_b, c & 1, ab, false, kBackoffNs)) break;
       tc_fence_after();
       // o = gamma (X_a + X_b) + (Y_a + Y_b), kept in registers; per-32-column
       // partial sums of o^2 are combined in a fixed order for every slicing
@@ -952,12 +995,12 @@ __global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
 #pragma unroll
         for (int cc = 1; cc < NB; ++cc) total += part[cc];
       } else {
-        if (c >= 2 && !mbar_wait_warp(&nack_b[pb], ((c >> 1) - 1) & 1, ab, true)) break;
+        if (c >= 2 && !mbar_wait_warp(&nack_b[pb], ((c >> 1) - 1) & 1, ab, true, kBackoffNs)) break;
 #pragma unroll
         for (int cc = 0; cc < NB; ++cc) sSS[(pb * 4 + slice * NB + cc) * 64 + i] = part[cc];
         for (int r = 0; r < CS; ++r)
           if (r != slice) mbar_arrive_remote(&nfull_b[pb], static_cast<uint32_t>(r));
-        if (!mbar_wait_warp(&nfull_b[pb], (c >> 1) & 1, ab, true)) break;
+        if (!mbar_wait_warp(&nfull_b[pb], (c >> 1) & 1, ab, true, kBackoffNs)) break;
         float blk[4];
 #pragma unroll
         for (int bidx = 0; bidx < 4; ++bidx) {

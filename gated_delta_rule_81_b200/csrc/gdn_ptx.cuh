@@ -93,8 +93,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // Bounded wait for phase `parity` of `bar`.  False on timeout or abort.
+// sleep_ns > 0 backs off between polls: for waits off the critical path, so that
+// the polling warp leaves issue slots to the warps it shares a sub-partition with.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
-                                          bool cluster_scope = false) {
+                                          bool cluster_scope = false, unsigned sleep_ns = 0) {
   if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
@@ -104,6 +106,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
       ab.raise(kDevErrTimeout);
       return false;
     }
+    if (sleep_ns) __nanosleep(sleep_ns);
   }
 }
 
@@ -111,8 +114,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 // same answer, so a following warp-aligned instruction (tcgen05.ld/st) is
 // either executed by the whole warp or skipped by the whole warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const Abort& ab,
-                                               bool cluster_scope = false) {
-  const bool ok = mbar_wait(bar, parity, ab, cluster_scope);
+                                               bool cluster_scope = false, unsigned sleep_ns = 0) {
+  const bool ok = mbar_wait(bar, parity, ab, cluster_scope, sleep_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

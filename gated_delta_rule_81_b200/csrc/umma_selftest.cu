@@ -13,6 +13,7 @@ namespace {
 constexpr int kKMajor = 0;     // SW128, K-major
 constexpr int kMN128 = 1;      // SW128, MN-major (64-wide MN blocks, LBO apart)
 constexpr int kMN64 = 2;       // SW64, MN-major (32-wide MN blocks, LBO apart)
+constexpr int kTmemA = 3;      // A only: in tensor memory, lane = row m, bf16 pairs along K per column
 
 __device__ __forceinline__ uint32_t operand_off(int layout, int mn, int k, int MN, int K) {
   if (layout == kKMajor) {  // K blocks of 64 elements, each MN rows x 128 B
@@ -53,10 +54,12 @@ __global__ void __launch_bounds__(128) umma_selftest_kernel(int a_layout, int b_
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc<256>(&tmem_base);
-  for (int i = tid; i < 128 * K; i += blockDim.x) {
-    int m = i / K, k = i % K;
-    *reinterpret_cast<__nv_bfloat16*>(sA + operand_off(a_layout, m, k, 128, K)) = A[i];
+  if (warp == 0) tmem_alloc<512>(&tmem_base);
+  if (a_layout != kTmemA) {
+    for (int i = tid; i < 128 * K; i += blockDim.x) {
+      int m = i / K, k = i % K;
+      *reinterpret_cast<__nv_bfloat16*>(sA + operand_off(a_layout, m, k, 128, K)) = A[i];
+    }
   }
   for (int i = tid; i < N * K; i += blockDim.x) {
     int n = i / K, k = i % K;
@@ -67,12 +70,29 @@ __global__ void __launch_bounds__(128) umma_selftest_kernel(int a_layout, int b_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base;
+  if (a_layout == kTmemA) {
+    // row m = TMEM lane m, columns 256 + c hold the bf16 pair (A[m][2c], A[m][2c+1]), even k in the low half
+    const uint32_t* A32 = reinterpret_cast<const uint32_t*>(A);
+    for (int c0 = 0; c0 < K / 2; c0 += 32) {
+      uint32_t w[32];
+      for (int j = 0; j < 32; ++j) w[j] = A32[(tid * K) / 2 + c0 + j];
+      tmem_st32(tmem_addr(tbase, warp * 32, 256 + c0), reinterpret_cast<const float*>(w));
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   if (tid == 0) {
-    uint32_t idesc = idesc_bf16(128, N, a_layout != kKMajor, b_layout != kKMajor);
+    uint32_t idesc = idesc_bf16(128, N, a_layout == kMN128 || a_layout == kMN64, b_layout != kKMajor);
     for (int ks = 0; ks < K / 16; ++ks) {
-      uint64_t da = operand_desc(a_layout, smem_u32(sA), ks, 128, K);
       uint64_t db = operand_desc(b_layout, smem_u32(sB), ks, N, K);
-      umma_bf16(tbase, da, db, idesc, ks > 0);
+      if (a_layout == kTmemA) {
+        umma_bf16_ts(tbase, tbase + 256 + 8 * ks, db, idesc, ks > 0);
+      } else {
+        uint64_t da = operand_desc(a_layout, smem_u32(sA), ks, 128, K);
+        umma_bf16(tbase, da, db, idesc, ks > 0);
+      }
     }
     umma_commit(&bar);
   }
@@ -90,19 +110,20 @@ __global__ void __launch_bounds__(128) umma_selftest_kernel(int a_layout, int b_
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc<256>(tbase);
+  if (warp == 0) tmem_dealloc<512>(tbase);
 }
 
 }  // namespace
 
 // D = A * B^T for a 128 x K A and an N x K B (both bf16 row-major, device), fp32 D [128][N].
-// a_layout / b_layout: 0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64 (32-wide MN blocks).
+// a_layout / b_layout: 0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64 (32-wide MN blocks);
+// a_layout 3 = A in tensor memory (K <= 256).
 // Returns 0 on launch success, -1 on a bad argument, else the CUDA error code.
 extern "C" int gdn_selftest_umma(int a_layout, int b_layout, int N, int K, const void* A, const void* B,
                                  float* D, int* err, void* stream) {
   if (K % 64 != 0 || K < 64 || K > 256) return -1;
   if (N % 16 != 0 || N < 16 || N > 256) return -1;
-  if (a_layout == 2) return -1;
+  if (a_layout == 2 || a_layout > 3 || b_layout > 2) return -1;
   if (a_layout == 1 && K % 16 != 0) return -1;
   if (b_layout == 1 && N % 64 != 0) return -1;
   if (b_layout == 2 && N % 32 != 0) return -1;

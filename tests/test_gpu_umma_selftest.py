@@ -10,7 +10,7 @@ from gpu_helpers import selftest_lib
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # a_layout, b_layout, N, K   (0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64)
+    # a_layout, b_layout, N, K   (0 = K-major SW128, 1 = MN-major SW128, 2 = MN-major SW64, 3 = A in TMEM)
     (0, 0, 64, 128),    # [Q;K] K^T
     (0, 0, 128, 128),
     (0, 0, 256, 64),
@@ -24,6 +24,13 @@ CASES = [
     (1, 1, 128, 64),    # K^T U
     (1, 1, 64, 64),
     (1, 2, 32, 64),
+    # A in tensor memory (3): state rows x operand, the TMEM-resident chain
+    (3, 1, 64, 128),    # S [W^T] : W^T MN-major, one 64-wide block
+    (3, 0, 64, 128),    # S Q^T   : Q K-major, two K blocks
+    (3, 1, 128, 64),    # U_d K   : K MN-major, two 64-wide blocks
+    (3, 0, 64, 64),     # U P^T   : P K-major
+    (3, 0, 256, 64),
+    (3, 1, 128, 128),
 ]
 
 

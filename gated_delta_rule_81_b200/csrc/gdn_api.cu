@@ -28,9 +28,6 @@ gdn_status check_inputs(const gdn_inputs* in, long long T_tot) {
   if (!in) return GDN_ERR_INVALID_ARG;
   if (in->H_k <= 0 || in->H_v <= 0 || in->H_v % in->H_k != 0) return GDN_ERR_INVALID_ARG;
   if (in->H_v / in->H_k > 8) return GDN_ERR_UNSUPPORTED;
-  if (in->dv_slice != 0 && in->dv_slice != 32 && in->dv_slice != 64 && in->dv_slice != 128)
-    return GDN_ERR_INVALID_ARG;
-  if (in->dv_slice == 128) return GDN_ERR_UNSUPPORTED;
   if (T_tot == 0) return GDN_OK;
   if (!in->q || !in->k || !in->v || !in->a || !in->b || !in->z || !in->conv_w || !in->A_log || !in->norm_w)
     return GDN_ERR_INVALID_ARG;
@@ -57,20 +54,6 @@ gdn_status check_out_alias(const gdn_inputs* in, long long T_tot, const void* ou
       overlap(out, ob, in->a, tb * in->stride_a) || overlap(out, ob, in->b, tb * in->stride_b))
     return GDN_ERR_ALIAS;
   return GDN_OK;
-}
-
-int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
-// smallest state-row slice that still fits all scan CTAs in one wave
-int pick_dv(const gdn_inputs* in, int N) {
-  if (in->dv_slice) return in->dv_slice;
-  const long long units = static_cast<long long>(N) * in->H_v;
-  const int sms = sm_count();
-  return units * 4 <= sms ? 32 : 64;
 }
 
 gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long long n_chunks, const int* cu,
@@ -120,15 +103,15 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.ws_flag = reinterpret_cast<int*>(ws);
   p.chunk_base = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) : nullptr;
   p.seq_order = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) + (N + 1) : nullptr;
-  p.ws_qk = ws + gdn::kWsHeader + chunk_base_bytes(N);
-  p.ws_head = p.ws_qk + static_cast<size_t>(n_chunks) * in->H_k * gdn::kQKBytes;
+  p.ws_k = ws + gdn::kWsHeader + chunk_base_bytes(N);
+  p.ws_head = p.ws_k + static_cast<size_t>(n_chunks) * in->H_k * gdn::kKBytes;
   p.state_in = state_in;
   p.state_out = state_out;
   p.conv_in = static_cast<const bf16*>(conv_in);
   p.conv_out = static_cast<bf16*>(conv_out);
   p.out = static_cast<bf16*>(out);
   p.err = err;
-  cudaError_t e = gdn::launch_prefill(p, pick_dv(in, N), static_cast<cudaStream_t>(stream), in->events);
+  cudaError_t e = gdn::launch_prefill(p, static_cast<cudaStream_t>(stream), in->events);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -139,7 +122,7 @@ extern "C" {
 size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks) {
   if (H_k <= 0 || H_v <= 0 || N < 0 || n_chunks < 0) return 0;
   return gdn::kWsHeader + chunk_base_bytes(N) +
-         static_cast<size_t>(n_chunks) * (static_cast<size_t>(H_k) * gdn::kQKBytes +
+         static_cast<size_t>(n_chunks) * (static_cast<size_t>(H_k) * gdn::kKBytes +
                                           static_cast<size_t>(H_v) * gdn::kHeadBytes);
 }
 

@@ -9,18 +9,29 @@ using bf16 = __nv_bfloat16;
 
 // Per-chunk workspace written by the prep kernel and read by the scan kernel.
 // Every tensor-core operand is stored as a bf16 pair (hi = bf16(x), lo =
-// bf16(x - hi)) so that products keep ~16 significant bits:
-//   per (chunk, key head):   [Q;K] operand image, 128 rows x 128, SW128 K-major: hi, then lo
-//   per (chunk, value head): [P T~; T~] image (128 x 64, SW128 K-major): hi, then lo;
-//                            v_hat fp32 (64 tokens x 128, four 32-wide column blocks);
-//                            gates fp32 (gamma[64], decay-to-end[64], gamma_C)
-constexpr int kQKImg = 32768;                                // one bf16 image
-constexpr int kQKBytes = 2 * kQKImg;                         // hi + lo
-constexpr int kPTImg = 16384;
-constexpr int kPTBytes = 2 * kPTImg;
-constexpr int kVBytes = 64 * 128 * 4;                        // fp32
+// bf16(x - hi)) so that products keep ~16 significant bits.  Operand images use
+// the 128-byte swizzled layout (rows of 64 bf16 = 128 B, 8-row groups of 1 KiB).
+//   per (chunk, key head), kKBytes:
+//     K hi | K lo: 64 tokens x 128 channels as two 8 KiB blocks of 64 channels
+//     (row = token), read by the scan as an MN-major operand (N = channels).
+//   per (chunk, value head), kHeadBytes:
+//     W^T lo | W^T hi | (gamma Q)^T hi | (gamma Q)^T lo: four 16 KiB images of
+//       128 rows (d_k) x 64 tokens, W = T diag(beta gamma) K and gamma Q = diag(gamma) Q;
+//       side by side they form one MN-major operand of N = 256 (or N = 128 from the second)
+//     P hi | P lo: P_ij = e^{G_i - G_j} q_i.k_j for j <= i, row = i, 64 j per row
+//     U0 fp32 [64 tokens][128 d_v]   (U0 = T diag(beta) V)
+//     gates fp32: gamma_i [64], e^{G_C - G_i} [64], gamma_C
+constexpr int kImg64 = 16384;                                // 64 rows x 128 channels (or 128 x 64), bf16
+constexpr int kKBytes = 2 * kImg64;                          // K hi, K lo
+constexpr int kHeadOffWQ = 0;                                // W^T lo, W^T hi, (gQ)^T hi, (gQ)^T lo
+constexpr int kWQBytes = 4 * kImg64;
+constexpr int kHeadOffP = kHeadOffWQ + kWQBytes;             // P hi, lo (8 KiB each)
+constexpr int kPImg = 8192;
+constexpr int kHeadOffU0 = kHeadOffP + 2 * kPImg;
+constexpr int kU0Bytes = 64 * 128 * 4;
+constexpr int kHeadOffGate = kHeadOffU0 + kU0Bytes;
 constexpr int kGateBytes = 1024;
-constexpr int kHeadBytes = kPTBytes + kVBytes + kGateBytes;  // 66560
+constexpr int kHeadBytes = kHeadOffGate + kGateBytes;        // 115712
 constexpr int kWsHeader = 1024;                              // error/consistency word
 
 struct DecodeParams {
@@ -53,7 +64,7 @@ struct PrefillParams {
   int* chunk_base;        // [N+1] in the workspace (varlen), or null (uniform)
   int* seq_order;         // [N] scan order, longest first (varlen), or null
   int* ws_flag;           // workspace header word: nonzero = inconsistent cu_seqlens
-  uint8_t* ws_qk;         // [n_chunks][H_k][kQKBytes]
+  uint8_t* ws_k;          // [n_chunks][H_k][kKBytes]
   uint8_t* ws_head;       // [n_chunks][H_v][kHeadBytes]
   const float* state_in;  // [N][H_v][128][128] or null (zeros)
   float* state_out;       // [N][H_v][128][128] or null
@@ -65,7 +76,6 @@ struct PrefillParams {
 
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events);
-// dv_slice: 64 or 32 value rows of the state per scan CTA (a cluster of 128/dv_slice CTAs per head)
-cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream, void* const* events);
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* const* events);
 
 }  // namespace gdn

@@ -11,18 +11,20 @@
 // inclusive cumulative sum of g = log a, gamma_i = e^{G_i}:
 //   A_ij = b_i e^{G_i - G_j} (k_i . k_j) (j < i),   T = (I + A)^{-1},
 //   T~ = T diag(b),   P_ij = e^{G_i - G_j} (q_i . k_j) (j <= i),
-//   R = V - diag(gamma) K S^T,   U = T~ R,   O = diag(gamma) Q S^T + P T~ R,
-//   S^T <- gamma_C S^T + K^T diag(e^{G_C - G_j}) U.
+//   W = T diag(b gamma) K,   U0 = T diag(b) V,   U = U0 - W S^T,
+//   O = diag(gamma) Q S^T + P U,   S <- gamma_C S + U^T diag(e^{G_C - G_j}) K.
 //
 // Two kernels (plus two small helpers):
 //   prep (one CTA per chunk x key head, all chunks in parallel): conv + SiLU +
 //     L2-norm front end, gates, [Q;K] K^T on tcgen05, the fp32 blocked
-//     triangular solve, and [P;I] T~ on tcgen05.  It writes the chunk's
-//     operand images to the workspace.
-//   scan (one CTA, or a cluster of 2 or 4 CTAs, per sequence x value head;
-//     each CTA owns 128/cluster value rows of the state): walks the chunks in
-//     order with S^T resident in tensor memory.  Per chunk three tcgen05 MMAs
-//     ([Q;K] S^T, [P T~; T~] R, K^T U) and the gated RMS-norm epilogue.
+//     triangular solve, and per value head W = T diag(b gamma) K and
+//     U0 = T diag(b) V on tcgen05 (so that U = U0 - W S^T).  It writes the
+//     chunk's operand images to the workspace.
+//   scan (one CTA per sequence x value head): walks the chunks in order with
+//     the whole fp32 state in tensor memory (lane = value row), the state and
+//     U as bf16 hi/lo A operands read by tcgen05 straight from tensor memory.
+//     Per chunk four tcgen05 products (S W^T, S Q^T, U_d^T K, U^T P^T) and the
+//     gated RMS-norm epilogue.
 #include "gdn_kernels.cuh"
 
 namespace gdn {
@@ -46,19 +48,8 @@ __device__ __forceinline__ long long chunk_base_of(const PrefillParams& p, int n
                       : static_cast<long long>(n) * ((p.T_uniform + kChunk - 1) / kChunk);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Named barrier over `nthreads` threads that also ORs a per-thread predicate:
-// every participant gets the same answer.  The non-aligned form, so the lanes of
-// a warp may arrive at different times (one lane may still be issuing MMAs).
+// every participant gets the same answer.
 __device__ __forceinline__ bool bar_sync_or(int id, int nthreads, bool pred) {
   uint32_t r;
   asm volatile(
@@ -70,14 +61,6 @@ __device__ __forceinline__ bool bar_sync_or(int id, int nthreads, bool pred) {
       : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
-}
-
-__device__ __forceinline__ float ld_shared_remote(const float* p, uint32_t cta) {
-  uint32_t local = smem_u32(p), remote;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(cta));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
 }
 
 // unpack 8 bf16 from a uint4
@@ -176,24 +159,36 @@ __global__ void conv_out_kernel(PrefillParams p) {
   }
 }
 
+
 // ============================================================ prep kernel
 
 constexpr int kPrepThreads = 256;
 constexpr int kLdA = 65;                               // fp32 row stride of A in shared memory
 constexpr int kLdT = 68;                               // fp32 row stride of T (16-byte aligned rows)
-constexpr int kPrepOffQK = 0;                          // [Q;K] image hi, lo    2 x 32768
-// After the [Q;K] K^T product has completed, the [Q;K] region is reused by the head loop:
-constexpr int kPrepOffTt = kPrepOffQK;                 // T~ image (B) hi, lo   2 x 8192
-constexpr int kPrepOffA = kPrepOffTt + 2 * 8192;       // A fp32                64*65*4
-constexpr int kPrepOffT = kPrepOffA + 64 * kLdA * 4;   // T fp32                64*68*4
-constexpr int kPrepOffM = kPrepOffT + 64 * kLdT * 4;   // block-solve temp      3*256*4
-static_assert(kPrepOffM + 3 * 256 * 4 <= 2 * 32768, "head-loop buffers must fit the [Q;K] region");
-constexpr int kPrepOffPI = 2 * 32768;                  // [P;I] image hi, lo    2 x 16384
-constexpr int kPrepOffG = kPrepOffPI + 2 * 16384;      // G cumsum [8][64]
-constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta     [8][64]
-constexpr int kPrepOffW = kPrepOffB + 8 * 64 * 4;      // conv weights of the CTA's channels, (2+G)*128*8 B
-// dynamic shared memory for G value heads per key head (1 KiB of alignment slack)
+// [Q;K] operand image in shared memory: hi at +0, lo at +32768; K-block kb (channels
+// 64 kb .. 64 kb + 63) at kb * 16384, rows 0..63 = Q tokens, rows 64..127 = K tokens.
+constexpr int kPrepOffQK = 0;
+// Once the [Q;K] K^T product has completed, the Q rows of the four K-block halves
+// hold the head loop's K-major B images: B_W = T diag(beta gamma), B_U = T diag(beta)
+constexpr int kPrepOffBWhi = 0, kPrepOffBUhi = 16384, kPrepOffBWlo = 32768, kPrepOffBUlo = 49152;
+constexpr int kPrepOffT = 65536;                       // T fp32                64*68*4
+// Once the B images are built, T, A and the block-solve temp are dead: the
+// region then holds the value head's v_hat image (A operand of U0^T, MN-major:
+// rows = tokens, two 64-channel blocks, hi then lo; 32 KiB)
+constexpr int kPrepOffV = kPrepOffT;
+constexpr int kPrepOffA = kPrepOffT + 64 * kLdT * 4;   // A fp32                64*65*4
+constexpr int kPrepOffM = kPrepOffA + 64 * kLdA * 4;   // block-solve temp      3*256*4
+constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum   [8][64]
+constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta       [8][64]
+constexpr int kPrepOffGam = kPrepOffB + 8 * 64 * 4;    // gamma = e^G [8][64]
+constexpr int kPrepOffW = kPrepOffGam + 8 * 64 * 4;    // conv weights of the q, k and v channels, (2+G)*128*8 B
 __host__ __device__ constexpr int prep_smem_bytes(int G) { return kPrepOffW + (2 + G) * 128 * 8 + 1024; }
+static_assert(kPrepOffV + 2 * kImg64 <= kPrepOffG, "the v_hat image must fit the solve buffers");
+// tensor memory columns (256 per CTA, two CTAs per SM)
+constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns);
+                                      // then q^T (lane = d_k, column = token)
+constexpr uint32_t kPrepColW = 128;   // W^T (lane = d_k, column = token)
+constexpr uint32_t kPrepColU = 192;   // U0^T (lane = d_v, column = token)
 
 // hi = bf16(f), lo = bf16(f - hi) for 8 values
 __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
@@ -328,20 +323,35 @@ __device__ __forceinline__ void umma_split(uint32_t d, uint64_t a_hi, uint64_t a
   umma_bf16(d, a_lo, b_hi, idesc, true);
 }
 
+
+// W words of bf16 pairs from 2W fp32 values: hi[m] = (bf16(x[2m]), bf16(x[2m+1])) with
+// the even element in the low half, lo[m] the same for the residuals x - hi.
+template <int W>
+__device__ __forceinline__ void split_pairs(const float* x, uint32_t* hi, uint32_t* lo) {
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    const uint32_t h = pack_bf16x2(x[2 * m], x[2 * m + 1]);
+    hi[m] = h;
+    lo[m] = pack_bf16x2(x[2 * m] - bf16_lo(h), x[2 * m + 1] - bf16_hi(h));
+  }
+}
+
+// One CTA per (chunk, key head).  Writes the chunk's K image for the key head
+// and, for each of its value heads, W^T, (gamma Q)^T, P, U0 and the gate vectors.
 __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;
   extern __shared__ uint8_t prep_smem_raw[];
   uint8_t* sm = align1024(prep_smem_raw);
-  uint8_t* sQK = sm + kPrepOffQK;   // hi at +0, lo at +32768
-  uint8_t* sPI = sm + kPrepOffPI;   // hi at +0, lo at +16384
-  uint8_t* sTt = sm + kPrepOffTt;   // hi at +0, lo at +8192
+  uint8_t* sQK = sm + kPrepOffQK;
   float* sA = reinterpret_cast<float*>(sm + kPrepOffA);
   float* sT = reinterpret_cast<float*>(sm + kPrepOffT);
   float* sM = reinterpret_cast<float*>(sm + kPrepOffM);
   float* sG = reinterpret_cast<float*>(sm + kPrepOffG);
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
-  uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2+G)*128 channels / 2] pairs: q | k | v heads
-  __shared__ uint64_t bar[3];
+  float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
+  uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2 + G) * 64] channel pairs: q | k | v heads
+  uint8_t* sV = sm + kPrepOffV;
+  __shared__ uint64_t bar[4];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -349,6 +359,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   const long long gc = blockIdx.x;
   const int kh = blockIdx.y;
   const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k;
+  const long long C_conv = static_cast<long long>(2 * H_k + H_v) * kD;
 
   // sequence of this chunk: the largest n with chunk_base(n) <= gc
   int n;
@@ -372,9 +383,10 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     mbar_init(&bar[2], 1);
+    mbar_init(&bar[3], 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc<128>(&tmem_base_s);
+  if (warp == 0) tmem_alloc<256>(&tmem_base_s);
 
   // conv weights of this CTA's channels (q, k of key head kh; v of its G value heads)
   for (int x = tid; x < (2 + G) * 64; x += kPrepThreads) {
@@ -384,22 +396,17 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
                                    : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh * G + grp - 2) * kD;
     sW[x] = __ldg(reinterpret_cast<const uint4*>(p.conv_w + (ch0 + 2 * pair) * kTaps));
   }
+  // the raw v rows of the key head's value heads are read later in the head loop: into L2 now
+  if (warp == 7) {
+    for (int r = lane; r < L + 3; r += 32) {
+      const long long tau = t0 - 3 + r;
+      if (tau >= s) prefetch_l2(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD, static_cast<uint32_t>(G * kD * 2));
+    }
+  }
   __syncthreads();
 
-  // identity rows 64..127 of the [P; I] image (hi = I, lo = 0)
-  for (int x = tid; x < 64 * 8; x += kPrepThreads) {
-    const int i = x >> 3, cc = x & 7;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (cc == (i >> 3)) {
-      const int e8 = i & 7;
-      w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
-    }
-    *reinterpret_cast<uint4*>(sPI + sw128_off(64 + i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(sPI + 16384 + sw128_off(64 + i, cc)) = make_uint4(0u, 0u, 0u, 0u);
-  }
-
   // ---- front end of q and k: token i, channels 32*qq .. 32*qq+31
-  uint8_t* gQK = p.ws_qk + (gc * H_k + kh) * static_cast<long long>(kQKBytes);
+  uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
   {
     const int i = tid >> 2, qq = tid & 3;
     const bool valid = i < L;
@@ -426,11 +433,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         for (int e2 = 0; e2 < 8; ++e2) f[e2] = y[8 * c2 + e2] * inv;
         uint4 hi, lo;
         split8(f, hi, lo);
-        const uint32_t off = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
-        *reinterpret_cast<uint4*>(sQK + off) = hi;
-        *reinterpret_cast<uint4*>(sQK + kQKImg + off) = lo;
-        *reinterpret_cast<uint4*>(gQK + off) = hi;
-        *reinterpret_cast<uint4*>(gQK + kQKImg + off) = lo;
+        const uint32_t soff = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
+        *reinterpret_cast<uint4*>(sQK + soff) = hi;
+        *reinterpret_cast<uint4*>(sQK + 32768 + soff) = lo;
+        if (which == 1) {
+          const uint32_t goff = kb * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
+          *reinterpret_cast<uint4*>(gK + goff) = hi;
+          *reinterpret_cast<uint4*>(gK + kImg64 + goff) = lo;
+        }
       }
     }
   }
@@ -442,12 +452,12 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 
   // ---- [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
   if (tid == 0) {
-    const uint32_t qh = smem_u32(sQK), ql = qh + kQKImg;
+    const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
     const uint32_t idesc = idesc_bf16(128, 64, false, false);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-      umma_split(tbase, smem_desc(qh + ko, 16, 1024, Swz::k128), smem_desc(ql + ko, 16, 1024, Swz::k128),
+      umma_split(tbase + kPrepColQK, smem_desc(qh + ko, 16, 1024, Swz::k128), smem_desc(ql + ko, 16, 1024, Swz::k128),
                  smem_desc(qh + ko + 8192, 16, 1024, Swz::k128), smem_desc(ql + ko + 8192, 16, 1024, Swz::k128),
                  idesc, ks > 0);
     }
@@ -482,37 +492,21 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     sG[j * 64 + i] += sG[j * 64 + 31];
   }
   __syncthreads();
-  // gate vectors for the scan: gamma_i, decay-to-end_i, gamma_C
+  // gate vectors for the scan: gamma_i, decay-to-end_i (0 past the chunk's last token), gamma_C
   for (int x = tid; x < G * 256; x += kPrepThreads) {
     const int j = x >> 8, k2 = x & 255, h = kh * G + j;
     const float Glast = sG[j * 64 + (L - 1)];
     float val = 0.f;
-    if (k2 < 64) val = expf(sG[j * 64 + k2]);
-    else if (k2 < 128) val = (k2 - 64) < L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
-    else if (k2 == 128) val = expf(Glast);
-    float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes + kVBytes);
-    gdst[k2] = val;
-  }
-  // ---- v_hat of the value heads (fp32): token i, channels 32*qq..+31
-  {
-    const int i = tid >> 2, qq = tid & 3;
-    const bool valid = i < L;
-    for (int j = 0; j < G; ++j) {
-      const int h = kh * G + j;
-      float y[32];
-      if (valid) {
-        conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,
-               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, sW + (2 + j) * 64 + 16 * qq, y);
-      } else {
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
-      }
-      // [column block qq][quad q][token i] float4: a warp's reads of one quad are contiguous
-      float4* dst = reinterpret_cast<float4*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kPTBytes) +
-                    qq * 8 * 64 + i;
-#pragma unroll
-      for (int c2 = 0; c2 < 8; ++c2) dst[c2 * 64] = make_float4(y[4 * c2], y[4 * c2 + 1], y[4 * c2 + 2], y[4 * c2 + 3]);
+    if (k2 < 64) {
+      val = expf(sG[j * 64 + k2]);
+      sGam[j * 64 + k2] = val;
+    } else if (k2 < 128) {
+      val = (k2 - 64) < L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
+    } else if (k2 == 128) {
+      val = expf(Glast);
     }
+    float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate);
+    gdst[k2] = val;
   }
 
   // ---- K K^T and Q K^T rows into registers: thread row = 32*(warp%4)+lane, columns cbase..cbase+31
@@ -523,15 +517,49 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   float acc[32];
   if (mbar_wait_warp(&bar[0], 0, ab)) {
     tc_fence_after();
-    tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), cbase), acc);
+    tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + cbase), acc);
     tmem_wait_ld();
   } else {
 #pragma unroll
     for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
   }
+  // ---- q^T (lane = d_k, column = token) into TMEM columns 0..63, which the [Q;K] K^T
+  // product no longer needs: Q_hi^T I + Q_lo^T I with an identity B, exact in fp32
+  {
+    uint8_t* sId = sm + kPrepOffA;  // 64 x 64 bf16 identity, K-major (before sA is built)
+    for (int x = tid; x < 64 * 8; x += kPrepThreads) {
+      const int i = x >> 3, cc = x & 7;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (cc == (i >> 3)) {
+        const int e8 = i & 7;
+        w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
+      }
+      *reinterpret_cast<uint4*>(sId + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();  // sG's second half, sGam and the identity are complete; acc has been read
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t qk = smem_u32(sQK), id = smem_u32(sId);
+      const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
+        umma_bf16(tbase + kPrepColQK, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
+        umma_bf16(tbase + kPrepColQK, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
+      }
+      umma_commit(&bar[3]);
+    }
+    __syncwarp();
+    mbar_wait_warp(&bar[3], 0, ab);
+    tc_fence_after();
+    __syncthreads();  // the identity (sA region) may now be overwritten
+  }
 
   for (int j = 0; j < G; ++j) {
     const int h = kh * G + j;
+    uint8_t* hb = p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes);
     const float Gi = sG[j * 64 + ri];
     if (!isQ) {
       const float bi = sB[j * 64 + ri];
@@ -541,6 +569,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         sA[ri * kLdA + col] = col < ri ? bi * __expf(Gi - sG[j * 64 + col]) * acc[e2] : 0.f;
       }
     } else {
+      // P_ij = e^{G_i - G_j} (q_i . k_j) for j <= i, as the K-major image (row i) in the workspace
 #pragma unroll
       for (int c2 = 0; c2 < 4; ++c2) {
         float f[8];
@@ -551,58 +580,123 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         }
         uint4 hi, lo;
         split8(f, hi, lo);
-        *reinterpret_cast<uint4*>(sPI + sw128_off(ri, (cbase >> 3) + c2)) = hi;
-        *reinterpret_cast<uint4*>(sPI + 16384 + sw128_off(ri, (cbase >> 3) + c2)) = lo;
+        const uint32_t off = sw128_off(ri, (cbase >> 3) + c2);
+        *reinterpret_cast<uint4*>(hb + kHeadOffP + off) = hi;
+        *reinterpret_cast<uint4*>(hb + kHeadOffP + kPImg + off) = lo;
       }
     }
     __syncthreads();
     solve_unit_lower(sA, sT, sM, tid);
-    // T~ = T diag(beta): lower triangle incl. diagonal, as the MN-major B operand (row = k index)
+    // B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
     for (int x = tid; x < 64 * 8; x += kPrepThreads) {
       const int r = x >> 3, cc = x & 7;
-      float f[8];
+      float fu[8], fw[8];
 #pragma unroll
       for (int e2 = 0; e2 < 8; ++e2) {
         const int col = 8 * cc + e2;
-        f[e2] = col <= r ? sT[r * kLdT + col] * sB[j * 64 + col] : 0.f;
+        const float tb = col <= r ? sT[r * kLdT + col] * sB[j * 64 + col] : 0.f;
+        fu[e2] = tb;
+        fw[e2] = tb * sGam[j * 64 + col];
       }
       uint4 hi, lo;
-      split8(f, hi, lo);
-      *reinterpret_cast<uint4*>(sTt + sw128_off(r, cc)) = hi;
-      *reinterpret_cast<uint4*>(sTt + 8192 + sw128_off(r, cc)) = lo;
+      const uint32_t off = sw128_off(r, cc);
+      split8(fw, hi, lo);
+      *reinterpret_cast<uint4*>(sQK + kPrepOffBWhi + off) = hi;
+      *reinterpret_cast<uint4*>(sQK + kPrepOffBWlo + off) = lo;
+      split8(fu, hi, lo);
+      *reinterpret_cast<uint4*>(sQK + kPrepOffBUhi + off) = hi;
+      *reinterpret_cast<uint4*>(sQK + kPrepOffBUlo + off) = lo;
+    }
+    __syncthreads();  // T is dead: its region takes the v_hat image
+    {
+      // v_hat of value head h: token i, channels 32*qq .. 32*qq+31, as the MN-major image
+      const int i = tid >> 2, qq = tid & 3;
+      float y[32];
+      if (i < L) {
+        conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,
+               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, sW + (2 + j) * 64 + 16 * qq, y);
+      } else {
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
+      }
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        uint4 hi, lo;
+        split8(y + 8 * c2, hi, lo);
+        const uint32_t off = (qq >> 1) * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
+        *reinterpret_cast<uint4*>(sV + off) = hi;
+        *reinterpret_cast<uint4*>(sV + kImg64 + off) = lo;
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-      const uint32_t pih = smem_u32(sPI), pil = pih + 16384, tth = smem_u32(sTt), ttl = tth + 8192;
-      const uint32_t idesc = idesc_bf16(128, 64, false, true);
+      // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
+      const uint32_t qk = smem_u32(sQK);
+      const uint32_t idesc_w = idesc_bf16(128, 64, true, false);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        umma_split(tbase + 64, smem_desc(pih + ks * 32, 16, 1024, Swz::k128),
-                   smem_desc(pil + ks * 32, 16, 1024, Swz::k128), smem_desc(tth + ks * 2048, 8192, 1024, Swz::k128),
-                   smem_desc(ttl + ks * 2048, 8192, 1024, Swz::k128), idesc, ks > 0);
+        umma_split(tbase + kPrepColW, smem_desc(qk + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
+                   smem_desc(qk + 32768u + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
+                   smem_desc(qk + kPrepOffBWhi + ks * 32u, 16, 1024, Swz::k128),
+                   smem_desc(qk + kPrepOffBWlo + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
+      // U0^T = V^T B_U^T: A = v_hat (MN-major, rows = tokens), B = B_U (K-major)
+      const uint32_t vv = smem_u32(sV);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_split(tbase + kPrepColU, smem_desc(vv + ks * 2048u, 8192, 1024, Swz::k128),
+                   smem_desc(vv + kImg64 + ks * 2048u, 8192, 1024, Swz::k128),
+                   smem_desc(qk + kPrepOffBUhi + ks * 32u, 16, 1024, Swz::k128),
+                   smem_desc(qk + kPrepOffBUlo + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
       umma_commit(&bar[1]);
     }
     __syncwarp();
-    float o[32];
     if (mbar_wait_warp(&bar[1], j & 1, ab)) {
       tc_fence_after();
-      tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), 64 + cbase), o);
-      tmem_wait_ld();
-    } else {
+      float o[64];
+      {
+        // (gamma Q)^T row d_k = lane, tokens 32*(warp/4) .. +31: hi and lo images
+        const int kr = 32 * (warp & 3) + lane, half = warp >> 2;
+        float qg[32];
+        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + 32 * half), qg);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) o[e2] = 0.f;
-    }
-    uint8_t* dst = p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes);
+        for (int c2 = 0; c2 < 4; ++c2) {
+          float f[8];
 #pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2) {
-      uint4 hi, lo;
-      split8(o + 8 * c2, hi, lo);
-      const uint32_t off = sw128_off(row, (cbase >> 3) + c2);
-      *reinterpret_cast<uint4*>(dst + off) = hi;
-      *reinterpret_cast<uint4*>(dst + kPTImg + off) = lo;
+          for (int e2 = 0; e2 < 8; ++e2) f[e2] = qg[8 * c2 + e2] * sGam[j * 64 + 32 * half + 8 * c2 + e2];
+          uint4 hi, lo;
+          split8(f, hi, lo);
+          const uint32_t off = sw128_off(kr, 4 * half + c2);
+          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 2 * kImg64 + off) = hi;
+          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 3 * kImg64 + off) = lo;
+        }
+      }
+      if (warp < 4) {
+        // W^T row d_k = lane: the MN-major image row (64 tokens), lo image then hi image
+        tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW), o);
+        tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW + 32), o + 32);
+        tmem_wait_ld();
+        const int kr = 32 * warp + lane;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint4 hi, lo;
+          split8(o + 8 * cc, hi, lo);
+          const uint32_t off = sw128_off(kr, cc);
+          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + kImg64 + off) = hi;
+          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + off) = lo;
+        }
+      } else {
+        // U0 [token][d_v] fp32: a warp writes 128 contiguous bytes per token
+        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU), o);
+        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU + 32), o + 32);
+        tmem_wait_ld();
+        float* u0 = reinterpret_cast<float*>(hb + kHeadOffU0) + 32 * (warp & 3) + lane;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) u0[i * kD] = o[i];
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -618,450 +712,416 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc<128>(tbase);
+  if (warp == 0) tmem_dealloc<256>(tbase);
 }
 
 // ============================================================ scan kernel
+//
+// One CTA per (sequence, value head); the whole 128 x 128 state lives in tensor
+// memory with lane = d_v row.  Per chunk, every product summed over the hi/lo
+// split terms (hi.hi + hi.lo + lo.hi):
+//   [U^T | O^T] = S [W^T | (gamma Q)^T]  (A = S hi/lo from TMEM; the U^T half first)
+//   U^T  = U0^T - (S W^T)
+//   S    = gamma_C S + (U^T diag(e^{G_C - G_j})) K   (A = U_d hi/lo from TMEM)
+//   O^T += U^T P^T                       (A = U hi/lo from TMEM)
+//   then the gated RMS-norm of o_i over d_v.
+// Warps 0-7 (thread = d_v row; warps w and w + 4 share a TMEM lane quarter and
+// split its columns) convert S and U between fp32 accumulators and bf16 hi/lo
+// operands in tensor memory, each conversion publishing first the part the next
+// product waits for; warps 8-11 run the output stage; warp 12 lane 0 issues the
+// MMAs in the order S W^T, S (gamma Q)^T, state update, U^T P^T, so that the
+// output's products fill the tensor pipe while the chain converts; warp 13
+// lane 0 issues the bulk copies.
 
-template <int DV>
-struct ScanCfg {
-  static constexpr int CS = 128 / DV;                  // CTAs per value head (cluster size)
-  static constexpr int NB = DV / 32;                   // 32-column blocks per CTA
-  static constexpr int TMEM_COLS = DV == 32 ? 256 : 512;
-  static constexpr int COL_Z = 0;                      // S^T: lanes = d_k, DV columns
-  // X = [Q;K] S^T and Y = [P T~; T~] R, each as two DV-column halves whose sum is
-  // the product: (hi.hi + lo.hi | hi.lo) -- the hi and lo B operands sit side by
-  // side along N so that A_hi [B_hi | B_lo] is one instruction.
-  static constexpr int COL_X = DV;
-  static constexpr int COL_Y = 3 * DV;
-  // shared memory (offsets from a 1024-aligned base)
-  static constexpr int OFF_GATE = kQKBytes;            // inside a [Q;K] stage
-  static constexpr int QK_STAGE = kQKBytes + kGateBytes;
-  static constexpr int OFF_PT = 2 * QK_STAGE;          // single [P T~; T~] buffer, hi then lo
-  static constexpr int OFF_V = OFF_PT + kPTBytes;      // single v_hat slice, fp32 [DV/32][64][32]
-  static constexpr int V_BYTES = 64 * DV * 4;
-  static constexpr int OFF_OP = OFF_V + V_BYTES;       // S, R and U operands (hi image, then lo image)
-  static constexpr int OP_IMG = 128 * DV * 2;
-  static constexpr int OFF_NW = OFF_OP + 2 * OP_IMG;   // norm weight slice, fp32 [DV]
-  static constexpr int OFF_SS = OFF_NW + 512;          // RMS partials [2][4][64] fp32
-  static constexpr int SMEM = OFF_SS + 2048 + 1024;
-  static constexpr uint32_t QK_TX = kQKBytes + kGateBytes;
-};
+constexpr int kScanThreads = 448;
+constexpr int kWarpIssue = 12, kWarpProd = 13;
+// tensor memory columns (512 allocated)
+constexpr uint32_t kColS = 0;      // S fp32, 128 columns (d_k)
+constexpr uint32_t kColSH = 128;   // S hi, bf16 pairs along d_k (64 columns)
+constexpr uint32_t kColSL = 192;   // S lo
+// [S_hi W_lo^T | (S_hi + S_lo) W_hi^T | O part 1 | O part 2], 4 x 64 columns
+constexpr uint32_t kColU2 = 256;   //   U^T = U0^T - (U2 + U1)
+constexpr uint32_t kColU1 = 320;
+constexpr uint32_t kColO = 384;    //   o = O1 + O2 (gamma Q S^T, then + P U accumulated by the last product)
+// After the U conversion, in place: the chain warp of token half th (tokens 32 th .. +31)
+// read U2 / U1 columns 256 + 32 th / 320 + 32 th and writes there, 16 columns each,
+//   U hi at 256 + 32 th, U lo at 272 + 32 th, U_d hi at 320 + 32 th, U_d lo at 336 + 32 th,
+// so K step ks (tokens 16 ks .. +15) of an A operand sits at base + 32 (ks / 2) + 8 (ks % 2).
+constexpr uint32_t kColUH = 256;
+constexpr uint32_t kColUL = 272;
+constexpr uint32_t kColUDH = 320;
+constexpr uint32_t kColUDL = 336;
+__host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base + 32u * (ks >> 1) + 8u * (ks & 1); }
+// shared memory (offsets from a 1024-aligned base)
+constexpr int kScOffWQ = 0;                            // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
+constexpr int kScOffK = kScOffWQ + kWQBytes;           // K hi, lo
+constexpr int kScOffP = kScOffK + kKBytes;             // P hi, lo
+constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // U0 fp32 [64][128]
+constexpr int kScOffO = kScOffU0 + kU0Bytes;           // o fp32 [64 tokens][128 d_v] for the token-major epilogue
+constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
+constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 
-// MN-major operand image with DV columns (8-element chunk index nch) and `krows` K-rows
-template <int DV>
-__device__ __forceinline__ uint32_t mn_off(uint32_t krow, uint32_t nch, uint32_t krows) {
-  if constexpr (DV == 32) return sw64_off(krow, nch);
-  else return (nch >> 3) * (krows * 128u) + sw128_off(krow, nch & 7u);
-}
-
-template <int DV>
-__device__ __forceinline__ uint64_t mn_desc(uint32_t base, int ks, uint32_t krows) {
-  if constexpr (DV == 32) return smem_desc(base + ks * 1024u, 512, 512, Swz::k64);
-  else return smem_desc(base + ks * 2048u, krows * 128u, 1024, Swz::k128);
-}
-
-// [hi | lo] as one 2*DV-wide MN-major operand: the lo image is the next MN block, img_bytes on
-template <int DV>
-__device__ __forceinline__ uint64_t mn_desc_cat(uint32_t base_hi, int ks, uint32_t img_bytes) {
-  if constexpr (DV == 32) return smem_desc(base_hi + ks * 1024u, img_bytes, 512, Swz::k64);
-  else return smem_desc(base_hi + ks * 2048u, img_bytes, 1024, Swz::k128);
-}
-
-// write 32 fp32 values (one thread's row segment, columns 32*cc..) as hi/lo bf16 into an MN-major image
-template <int DV>
-__device__ __forceinline__ void store_split_row(uint8_t* img_hi, int img_bytes, uint32_t krow, int cc, uint32_t krows,
-                                                const float* v) {
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    uint4 hi, lo;
-    split8(v + 8 * q4, hi, lo);
-    const uint32_t off = mn_off<DV>(krow, 4 * cc + q4, krows);
-    *reinterpret_cast<uint4*>(img_hi + off) = hi;
-    *reinterpret_cast<uint4*>(img_hi + img_bytes + off) = lo;
-  }
-}
-
-template <int DV>
-__global__ void __launch_bounds__(256, 1) scan_kernel(PrefillParams p) {
-  using Cfg = ScanCfg<DV>;
-  constexpr int CS = Cfg::CS, NB = Cfg::NB;
-  if (p.cu && *p.ws_flag) return;  // same value in every CTA of a cluster
+__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) {
+  if (p.cu && *p.ws_flag) return;
   extern __shared__ uint8_t scan_smem_raw[];
   uint8_t* sm = align1024(scan_smem_raw);
-  __shared__ uint64_t qk_full[2], qk_empty[2], xyfree_b, mma2o_b, nfull_b[2], nack_b[2];
-  __shared__ uint64_t pt_full, pt_empty, v_full, v_empty;
-  __shared__ uint64_t mma1_b, mma2_b, mma3_b, drain_b, drain2_b;
+  __shared__ uint64_t g_full[2], g_free[2];
+  __shared__ uint64_t wq_full, wq_free, k_full, k_free, p_full, p_free, u0_full, u0_free;
+  __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
-  const int unit = blockIdx.x / CS;
-  const int n_rank = unit / p.H_v, h = unit % p.H_v;
+  const int n_rank = blockIdx.x / p.H_v, h = blockIdx.x % p.H_v;
   const int n = (p.seq_order && p.N <= kMaxOrdered) ? p.seq_order[n_rank] : n_rank;
   const int G = p.H_v / p.H_k, kh = h / G;
-  const int slice = static_cast<int>(rank);
   const long long s = seq_start(p, n), e = seq_start(p, n + 1);
   const int nc = static_cast<int>((e - s + kChunk - 1) / kChunk);
   const long long cb = chunk_base_of(p, n);
 
   Abort ab{p.err, &abort_s};
-  float* sNW = reinterpret_cast<float*>(sm + Cfg::OFF_NW);
-  float* sSS = reinterpret_cast<float*>(sm + Cfg::OFF_SS);
-  uint8_t* sOP = sm + Cfg::OFF_OP;
   if (tid == 0) {
     abort_s = 0;
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&qk_full[b], 1);
-      mbar_init(&qk_empty[b], 1 + 64);
-      if (CS > 1) {
-        mbar_init(&nfull_b[b], (CS - 1) * 64);
-        mbar_init(&nack_b[b], (CS - 1) * 64);
-      }
+      mbar_init(&g_full[b], 1);
+      mbar_init(&g_free[b], 256);
     }
-    mbar_init(&xyfree_b, 64);
-    mbar_init(&mma2o_b, 1);
-    mbar_init(&pt_full, 1);
-    mbar_init(&pt_empty, 1);
-    mbar_init(&v_full, 1);
-    mbar_init(&v_empty, 64);
-    mbar_init(&mma1_b, 1);
-    mbar_init(&mma2_b, 1);
-    mbar_init(&mma3_b, 1);
+    mbar_init(&wq_full, 1);
+    mbar_init(&wq_free, 1);
+    mbar_init(&k_full, 1);
+    mbar_init(&k_free, 1);
+    mbar_init(&p_full, 1);
+    mbar_init(&p_free, 1);
+    mbar_init(&u0_full, 1);
+    mbar_init(&u0_free, 256);
+    mbar_init(&s_conv, 256);
+    mbar_init(&u_conv, 256);
+    mbar_init(&u_conv2, 256);
+    mbar_init(&u_done, 1);
+    mbar_init(&s_done, 1);
+    mbar_init(&y_done, 1);
+    mbar_init(&o_free, 128);
     mbar_init(&drain_b, 1);
-    mbar_init(&drain2_b, 1);
     fence_mbar_init();
   }
-  if (warp == 7) tmem_alloc<Cfg::TMEM_COLS>(&tmem_base_s);
-  if (tid < DV) sNW[tid] = __bfloat162float(p.norm_w[slice * DV + tid]);
+  if (warp == kWarpIssue) tmem_alloc<512>(&tmem_base_s);
   tc_fence_before();
   __syncthreads();
-  if (CS > 1) cluster_sync_all();
   tc_fence_after();
   const uint32_t tbase = tmem_base_s;
-  const uint32_t op_hi = smem_u32(sOP), op_lo = op_hi + Cfg::OP_IMG;
 
-  if (warp == 6) {
-    // ------------------------------------------------ bulk-copy producer
+  if (warp < 8) {
+    // ------------------------------------------------ S and U conversions; thread = d_v row v,
+    // columns / tokens of half th
+    const int v = 32 * (warp & 3) + lane, th = warp >> 2;
+    const uint32_t tl = tmem_addr(tbase, 32 * (warp & 3), 0);
+    const long long srow = ((static_cast<long long>(n) * p.H_v + h) * kD + v) * kD;
+    const float* U0 = reinterpret_cast<const float*>(sm + kScOffU0);
+    bool ok = true;
+    for (int c = 0; c < nc && ok; ++c) {
+      const int gs = c & 1;
+      const float* gates = reinterpret_cast<const float*>(sm + kScOffG + gs * kGateBytes);
+      // ---- S_c (columns 64 th .. +63) -> hi/lo operand; then S <- gamma_C S for the update
+      // (the previous chunk's products that read S hi/lo were issued before its state update)
+      ok = c == 0 || mbar_wait_warp(&s_done, (c - 1) & 1, ab);
+      if (ok) ok = mbar_wait_warp(&g_full[gs], (c >> 1) & 1, ab);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[64];
+      if (c == 0) {
+        if (p.state_in) {
+          const float4* src = reinterpret_cast<const float4*>(p.state_in + srow + 64 * th);
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const float4 f = __ldg(src + q4);
+            sv[4 * q4] = f.x; sv[4 * q4 + 1] = f.y; sv[4 * q4 + 2] = f.z; sv[4 * q4 + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int e2 = 0; e2 < 64; ++e2) sv[e2] = 0.f;
+        }
+      } else {
+        tmem_ld32(tl + kColS + 64 * th, sv);
+        tmem_ld32(tl + kColS + 64 * th + 32, sv + 32);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t hi[16], lo[16];
+        split_pairs<16>(sv + 32 * cc, hi, lo);
+        tmem_st16(tl + kColSH + 32 * th + 16 * cc, hi);
+        tmem_st16(tl + kColSL + 32 * th + 16 * cc, lo);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&s_conv);
+      const float gC = gates[128];
+#pragma unroll
+      for (int e2 = 0; e2 < 64; ++e2) sv[e2] *= gC;
+      tmem_st32(tl + kColS + 64 * th, sv);
+      tmem_st32(tl + kColS + 64 * th + 32, sv + 32);
+      // ---- U^T = U0^T - S W^T for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first
+      // (the state update waits for it), then U (the output product waits for it)
+      ok = mbar_wait_warp(&u_done, c & 1, ab);
+      if (ok) ok = mbar_wait_warp(&u0_full, c & 1, ab);
+      if (!ok) break;
+      tc_fence_after();
+      float u[32], ud[32];
+      {
+        float u1[32];
+        tmem_ld32(tl + kColU2 + 32 * th, u);
+        tmem_ld32(tl + kColU1 + 32 * th, u1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = U0[(32 * th + i) * kD + v] - (u1[i] + u[i]);
+      }
+      mbar_arrive(&u0_free);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ud[i] = u[i] * gates[64 + 32 * th + i];
+      mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time
+      {
+        uint32_t hi[16], lo[16];
+        split_pairs<16>(ud, hi, lo);
+        tmem_st16(tl + kColUDH + 32 * th, hi);
+        tmem_st16(tl + kColUDL + 32 * th, lo);
+      }
+      tmem_wait_st();  // also covers the rescaled S
+      tc_fence_before();
+      mbar_arrive(&u_conv);
+      {
+        uint32_t hi[16], lo[16];
+        split_pairs<16>(u, hi, lo);
+        tmem_st16(tl + kColUH + 32 * th, hi);
+        tmem_st16(tl + kColUL + 32 * th, lo);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&u_conv2);
+    }
+    // final state of this head (row v, columns 64 th .. +63)
+    if (p.state_out) {
+      if (nc == 0) {
+        for (int k = 64 * th; k < 64 * th + 64; ++k) p.state_out[srow + k] = p.state_in ? p.state_in[srow + k] : 0.f;
+      } else if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(&s_done, (nc - 1) & 1, ab)) {
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float sv2[32];
+          tmem_ld32(tl + kColS + 64 * th + 32 * cc, sv2);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(p.state_out + srow + 64 * th + 32 * cc);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(sv2[4 * q4], sv2[4 * q4 + 1], sv2[4 * q4 + 2], sv2[4 * q4 + 3]);
+        }
+      }
+    }
+  } else if (warp == kWarpIssue) {
+    // ------------------------------------------------ tensor-core issue (one thread)
     if (lane == 0) {
-      int qk_issued[2] = {0, 0}, pt_issued = 0, v_issued = 0;
+      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [W_lo | W_hi], S_hi [gQ_hi | gQ_lo]
+      const uint32_t idesc_u2 = idesc_bf16(128, 64, false, true);   // S_lo W_hi, S_lo gQ_hi
+      const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
+      const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
+      const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
+      const uint32_t wq = smem_u32(sm + kScOffWQ);
+      const uint32_t k_hi = smem_u32(sm + kScOffK), k_lo = k_hi + kImg64;
+      const uint32_t p_hi = smem_u32(sm + kScOffP);
+      for (int c = 0; c < nc; ++c) {
+        if (!mbar_wait(&s_conv, c & 1, ab)) break;
+        if (!mbar_wait(&wq_full, c & 1, ab)) break;
+        if (c > 0 && !mbar_wait(&y_done, (c - 1) & 1, ab)) break;  // U^T P^T of the last chunk read the U columns
+        tc_fence_after();
+        // the chain's product first: [U2 | U1] = S_hi [W_lo | W_hi], U1 += S_lo W_hi
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
+          const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, ks > 0);
+          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
+        }
+        umma_commit(&u_done);
+        // then the output's: [O1 | O2] = S_hi [gQ_hi | gQ_lo], O1 += S_lo gQ_hi, once o(c-1) has been read
+        if (c > 0 && !mbar_wait(&o_free, (c - 1) & 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bq = smem_desc(wq + 2 * kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, ks > 0);
+          umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, bq, idesc_u2, true);
+        }
+        umma_commit(&wq_free);
+        if (!mbar_wait(&u_conv, c & 1, ab)) break;
+        if (!mbar_wait(&k_full, c & 1, ab)) break;
+        tc_fence_after();
+        // S += U_d^T K (onto gamma_C S)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
+          const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
+        }
+        umma_commit(&s_done);
+        umma_commit(&k_free);
+        if (!mbar_wait(&u_conv2, c & 1, ab)) break;
+        if (!mbar_wait(&p_full, c & 1, ab)) break;
+        tc_fence_after();
+        // [O1 | O2] += U_hi [P_hi | P_lo], O1 += U_lo P_hi
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t b2 = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);  // 128 rows: P hi then P lo
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUH, ks), b2, idesc_y, true);
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUL, ks), b2, idesc_y2, true);
+        }
+        umma_commit(&y_done);
+        umma_commit(&p_free);
+      }
+      // every MMA issued has completed before TMEM is read for the last time or released
+      umma_commit(&drain_b);
+      int drain_flag = 0;
+      Abort drain{nullptr, &drain_flag};
+      mbar_wait(&drain_b, 0, drain);
+    }
+    __syncwarp();
+  } else if (warp == kWarpProd) {
+    // ------------------------------------------------ bulk-copy producer (lane 0)
+    if (lane == 0) {
+      int n_g[2] = {0, 0}, n_wq = 0, n_k = 0, n_p = 0, n_u0 = 0;
       for (int c = 0; c < nc; ++c) {
         const int st = c & 1;
         const long long gc = cb + c;
         const uint8_t* hb = p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes);
-        uint8_t* stage = sm + st * Cfg::QK_STAGE;
-        if (c >= 2 && !mbar_wait(&qk_empty[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&qk_full[st], Cfg::QK_TX);
-        bulk_g2s(stage, p.ws_qk + (gc * p.H_k + kh) * static_cast<long long>(kQKBytes), kQKBytes, &qk_full[st]);
-        bulk_g2s(stage + Cfg::OFF_GATE, hb + kPTBytes + kVBytes, kGateBytes, &qk_full[st]);
-        ++qk_issued[st];
-        if (c >= 1 && !mbar_wait(&pt_empty, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&pt_full, kPTBytes);
-        bulk_g2s(sm + Cfg::OFF_PT, hb, kPTBytes, &pt_full);
-        ++pt_issued;
-        if (c >= 1 && !mbar_wait(&v_empty, (c - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&v_full, Cfg::V_BYTES);
-        bulk_g2s(sm + Cfg::OFF_V, hb + kPTBytes + slice * Cfg::V_BYTES, Cfg::V_BYTES, &v_full);
-        ++v_issued;
+        const uint8_t* kb = p.ws_k + (gc * p.H_k + kh) * static_cast<long long>(kKBytes);
+        if (c + 2 < nc) {  // two chunks ahead into L2
+          prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
+          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
+        }
+        if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&g_full[st], kGateBytes);
+        bulk_g2s(sm + kScOffG + st * kGateBytes, hb + kHeadOffGate, kGateBytes, &g_full[st]);
+        ++n_g[st];
+        if (c >= 1 && !mbar_wait(&wq_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&wq_full, kWQBytes);
+        bulk_g2s(sm + kScOffWQ, hb + kHeadOffWQ, kWQBytes, &wq_full);
+        ++n_wq;
+        if (c >= 1 && !mbar_wait(&u0_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&u0_full, kU0Bytes);
+        bulk_g2s(sm + kScOffU0, hb + kHeadOffU0, kU0Bytes, &u0_full);
+        ++n_u0;
+        if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&k_full, kKBytes);
+        bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
+        ++n_k;
+        if (c >= 1 && !mbar_wait(&p_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&p_full, 2 * kPImg);
+        bulk_g2s(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
+        ++n_p;
       }
-      // drain copies still in flight (only possible after an abort)
+      // copies still in flight (only possible after an abort) land before the CTA exits
       int drain_flag = 0;
       Abort drain{nullptr, &drain_flag};
-      for (int st = 0; st < 2; ++st)
-        if (qk_issued[st] > 0) mbar_wait(&qk_full[st], (qk_issued[st] - 1) & 1, drain);
-      if (pt_issued > 0) mbar_wait(&pt_full, (pt_issued - 1) & 1, drain);
-      if (v_issued > 0) mbar_wait(&v_full, (v_issued - 1) & 1, drain);
+      for (int b = 0; b < 2; ++b)
+        if (n_g[b] > 0) mbar_wait(&g_full[b], (n_g[b] - 1) & 1, drain);
+      if (n_wq > 0) mbar_wait(&wq_full, (n_wq - 1) & 1, drain);
+      if (n_u0 > 0) mbar_wait(&u0_full, (n_u0 - 1) & 1, drain);
+      if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
+      if (n_p > 0) mbar_wait(&p_full, (n_p - 1) & 1, drain);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------ state (threads 0..127), chain (64..127) and
-    // the tensor-core issue: thread 0 issues X = [Q;K] S^T, thread 64 issues Y and the state
-    // update.  Warps 0-3 pass the same three named barriers every chunk; each barrier ORs a
-    // "something failed" predicate, so all four warps leave the loop at the same barrier.
-    const int t = tid;  // TMEM lane = d_k index
-    const uint32_t lb = 32 * warp;
-    const long long srow0 = (static_cast<long long>(n) * p.H_v + h) * kD + static_cast<long long>(slice) * DV;
-    const uint32_t idesc_1 = idesc_bf16(128, DV, false, true);       // A_lo B_hi
-    const uint32_t idesc_2 = idesc_bf16(128, 2 * DV, false, true);   // A_hi [B_hi | B_lo]
-    const uint32_t idesc_ku = idesc_bf16(128, DV, true, true);
-    const uint32_t pt_hi = smem_u32(sm + Cfg::OFF_PT), pt_lo = pt_hi + kPTImg;
-    const uint32_t dX = tbase + Cfg::COL_X, dY = tbase + Cfg::COL_Y;
-    bool ok = true;
+  } else {
+    // ------------------------------------------------ output stage (warps 8-11)
+    // o leaves tensor memory row-wise (thread = d_v row) into shared memory as fp32
+    // [token][d_v]; then each thread owns 8 consecutive d_v of a token, 16 threads per
+    // token: the sum of o^2 over d_v is a 4-step shuffle inside that group (a fixed
+    // order), z is read and out written with 16-byte accesses.
+    const int ow = warp & 3;              // TMEM lane quarter
+    const int v = 32 * ow + lane;
+    const int otid = tid - 256;           // 0..127 within the output group
+    const uint32_t tl = tmem_addr(tbase, 32 * ow, 0);
+    float* sO = reinterpret_cast<float*>(sm + kScOffO);
+    const int v8 = (otid & 15) * 8;       // this thread's 8 channels; its tokens are otid / 16 + 8 m
+    float w8[8];  // norm_w is only 2-byte aligned: element loads
+#pragma unroll
+    for (int e2 = 0; e2 < 8; ++e2) w8[e2] = __bfloat162float(p.norm_w[v8 + e2]);
+    // Every output warp reaches every named barrier; a failed wait is OR-ed into the
+    // first barrier so that the four warps leave the loop together.
     for (int c = 0; c < nc; ++c) {
-      const int st = c & 1;
-      const float* gates = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE);
-      const uint32_t qk_hi = smem_u32(sm + st * Cfg::QK_STAGE), qk_lo = qk_hi + kQKImg;
-      // ---- state: S_{c-1} -> hi/lo operand image; S^T <- gamma_C S^T in TMEM
-      bool w = c == 0 || mbar_wait_warp(&mma3_b, (c - 1) & 1, ab);
-      if (w) w = mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab);
-      if (w) {
-        tc_fence_after();
-        const float gC = gates[128];
-        float v[NB][32];
-        if (c == 0) {
+      const long long tok0 = s + static_cast<long long>(c) * kChunk;
+      const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - tok0));
+      // z of the chunk (loaded while the products run)
+      uint4 zr[8];
 #pragma unroll
-          for (int cc = 0; cc < NB; ++cc)
-#pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2)
-              v[cc][e2] = p.state_in ? p.state_in[(srow0 + 32 * cc + e2) * kD + t] : 0.f;
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < NB; ++cc) tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
-          tmem_wait_ld();  // one wait for all column blocks
-        }
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc) {
-          store_split_row<DV>(sOP, Cfg::OP_IMG, t, cc, 128, v[cc]);
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) v[cc][e2] *= gC;
-          tmem_st32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v[cc]);
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
+      for (int m = 0; m < 8; ++m) {
+        const int r = (otid >> 4) + 8 * m;
+        zr[m] = r < L ? __ldg(reinterpret_cast<const uint4*>(p.z + (tok0 + r) * p.sz + static_cast<long long>(h) * kD + v8))
+                      : make_uint4(0u, 0u, 0u, 0u);
       }
-      tc_fence_before();
-      if (bar_sync_or(1, 128, !w)) { ok = false; break; }
-      bool issued = true;
-      if (t == 0) {  // X = [Q;K] S^T
-        issued = c == 0 || mbar_wait(&xyfree_b, (c - 1) & 1, ab);
-        if (issued) {
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-            umma_bf16(dX, smem_desc(qk_hi + ko, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
-                      idesc_2, ks > 0);
-            umma_bf16(dX, smem_desc(qk_lo + ko, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 128), idesc_1, true);
-          }
-          umma_commit(&mma1_b);
-        }
-      }
-      // ---- chain: R = v_hat - gamma (K S^T)
-      w = true;
-      if (t >= 64) {
-        const int i = t - 64;
-        w = mbar_wait_warp(&mma1_b, c & 1, ab);
-        if (w) w = mbar_wait_warp(&v_full, c & 1, ab);
-        if (w) {
-          tc_fence_after();
-          const float gam = gates[i];
-          const float4* vrow = reinterpret_cast<const float4*>(sm + Cfg::OFF_V);
-#pragma unroll
-          for (int cc = 0; cc < NB; ++cc) {
-            float x[32], x2[32];
-            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), x);
-            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), x2);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) x[e2] += x2[e2];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 vv = vrow[(cc * 8 + q) * 64 + i];
-              x[4 * q + 0] = fmaf(-gam, x[4 * q + 0], vv.x);
-              x[4 * q + 1] = fmaf(-gam, x[4 * q + 1], vv.y);
-              x[4 * q + 2] = fmaf(-gam, x[4 * q + 2], vv.z);
-              x[4 * q + 3] = fmaf(-gam, x[4 * q + 3], vv.w);
-            }
-            store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, x);
-          }
-          mbar_arrive(&v_empty);
-          fence_proxy_async_smem();
-        }
-      }
-      tc_fence_before();
-      if (bar_sync_or(2, 128, !w || !issued)) { ok = false; break; }
-      if (t == 64) {  // Y = [P T~; T~] R
-        issued = mbar_wait(&pt_full, c & 1, ab);
-        if (issued) {
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            umma_bf16(dY, smem_desc(pt_hi + ks * 32u, 16, 1024, Swz::k128), mn_desc_cat<DV>(op_hi, ks, Cfg::OP_IMG),
-                      idesc_2, ks > 0);
-            umma_bf16(dY, smem_desc(pt_lo + ks * 32u, 16, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64), idesc_1, true);
-          }
-          umma_commit(&mma2_b);
-          umma_commit(&mma2o_b);
-          umma_commit(&pt_empty);
-        }
-      }
-      // ---- chain: U_d = decay-to-end * U
-      w = true;
-      if (t >= 64) {
-        const int i = t - 64;
-        w = mbar_wait_warp(&mma2_b, c & 1, ab);
-        if (w) {
-          tc_fence_after();
-          const float dcy = gates[64 + i];
-#pragma unroll
-          for (int cc = 0; cc < NB; ++cc) {
-            float u[32], u2[32];
-            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), u);
-            tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), u2);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) u[e2] = (u[e2] + u2[e2]) * dcy;
-            store_split_row<DV>(sOP, Cfg::OP_IMG, i, cc, 64, u);
-          }
-          fence_proxy_async_smem();
-        }
-      }
-      tc_fence_before();
-      if (bar_sync_or(3, 128, !w || !issued)) { ok = false; break; }
-      if (t == 64) {  // S^T += K^T U_d
+      bool ok = mbar_wait_warp(&y_done, c & 1, ab, false, kBackoffNs);
+      if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_split(tbase + Cfg::COL_Z, smem_desc(qk_hi + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
-                     smem_desc(qk_lo + 8192u + ks * 2048u, 16384, 1024, Swz::k128), mn_desc<DV>(op_hi, ks, 64),
-                     mn_desc<DV>(op_lo, ks, 64), idesc_ku, true);
-        umma_commit(&mma3_b);
-        umma_commit(&qk_empty[st]);
-      }
-    }
-    // every MMA this thread issued has completed before TMEM is read or released
-    if (t == 0 || t == 64) {
-      uint64_t* db = t == 0 ? &drain_b : &drain2_b;
-      umma_commit(db);
-      int drain_flag = 0;
-      Abort drain{nullptr, &drain_flag};
-      mbar_wait(db, 0, drain);
-    }
-    // final state of this slice
-    if (p.state_out) {
-      if (nc == 0) {
-        for (int d = 0; d < DV; ++d)
-          p.state_out[(srow0 + d) * kD + t] = p.state_in ? p.state_in[(srow0 + d) * kD + t] : 0.f;
-      } else if (__all_sync(0xffffffffu, ok) && mbar_wait_warp(&mma3_b, (nc - 1) & 1, ab)) {
-        tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < NB; ++cc) {
-          float v[32];
-          tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Z + 32 * cc), v);
+        for (int cc = 0; cc < 2; ++cc) {
+          float o1[32], o2[32];
+          tmem_ld32(tl + kColO + 32 * cc, o1);
+          tmem_ld32(tl + kColO + 64 + 32 * cc, o2);
           tmem_wait_ld();
 #pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) p.state_out[(srow0 + 32 * cc + e2) * kD + t] = v[e2];
+          for (int i = 0; i < 32; ++i) sO[(32 * cc + i) * kD + v] = o1[i] + o2[i];
         }
+        tc_fence_before();
+        mbar_arrive(&o_free);
       }
-    }
-  } else if (warp >= 4 && warp < 6) {
-    // ------------------------------------------------ output (warps 4, 5): token i = TMEM lane i
-    const int i = tid - 128;
-    const uint32_t lb = 32 * (warp & 3);
-    // z of the next chunk is loaded while this chunk's products are still running
-    uint4 zbuf[NB * 4];
-    auto load_z = [&](int c) {
-      const long long tok = s + static_cast<long long>(c) * kChunk + i;
-      const uint4* zrow = reinterpret_cast<const uint4*>(p.z + (tok < e ? tok : s) * p.sz +
-                                                         static_cast<long long>(h) * kD + slice * DV);
+      if (bar_sync_or(1, 128, !ok)) break;
+      // the eight tokens' sums of squares side by side (independent shuffles), then the outputs
+      float inv[8];
 #pragma unroll
-      for (int q = 0; q < NB * 4; ++q) zbuf[q] = tok < e ? __ldg(zrow + q) : make_uint4(0u, 0u, 0u, 0u);
-    };
-    if (nc > 0) load_z(0);
-    for (int c = 0; c < nc; ++c) {
-      const int st = c & 1, pb = c & 1;
-      if (!mbar_wait_warp(&qk_full[st], (c >> 1) & 1, ab, false, kBackoffNs)) break;
-      const float gam = reinterpret_cast<const float*>(sm + st * Cfg::QK_STAGE + Cfg::OFF_GATE)[i];
-      mbar_arrive(&qk_empty[st]);  // only gamma is read from the stage
-      if (!mbar_wait_warp(&mma2o_b, c & 1, ab, false, kBackoffNs)) break;
-      tc_fence_after();
-      // o = gamma (X_a + X_b) + (Y_a + Y_b), kept in registers; per-32-column
-      // partial sums of o^2 are combined in a fixed order for every slicing
-      float o[DV];
-      float part[NB];
-#pragma unroll
-      for (int cc = 0; cc < NB; ++cc) {
-        float xa[32], xb2[32], ya[32], yb[32];
-        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + 32 * cc), xa);
-        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_X + DV + 32 * cc), xb2);
-        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + 32 * cc), ya);
-        tmem_ld32(tmem_addr(tbase, lb, Cfg::COL_Y + DV + 32 * cc), yb);
-        tmem_wait_ld();
-        float ss = 0.f;
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) {
-          const float v = fmaf(gam, xa[e2] + xb2[e2], ya[e2] + yb[e2]);
-          o[32 * cc + e2] = v;
-          ss = fmaf(v, v, ss);
-        }
-        part[cc] = ss;
+      for (int m = 0; m < 8; ++m) {
+        const float4* orow = reinterpret_cast<const float4*>(sO + ((otid >> 4) + 8 * m) * kD + v8);
+        const float4 a0 = orow[0], a1 = orow[1];
+        float ss = a0.x * a0.x;
+        ss = fmaf(a0.y, a0.y, ss); ss = fmaf(a0.z, a0.z, ss); ss = fmaf(a0.w, a0.w, ss);
+        ss = fmaf(a1.x, a1.x, ss); ss = fmaf(a1.y, a1.y, ss); ss = fmaf(a1.z, a1.z, ss); ss = fmaf(a1.w, a1.w, ss);
+        inv[m] = ss;
       }
-      tc_fence_before();
-      mbar_arrive(&xyfree_b);  // X and Y may be overwritten by the next chunk's products
-      float total;
-      if constexpr (CS == 1) {
-        total = part[0];
 #pragma unroll
-        for (int cc = 1; cc < NB; ++cc) total += part[cc];
-      } else {
-        if (c >= 2 && !mbar_wait_warp(&nack_b[pb], ((c >> 1) - 1) & 1, ab, true, kBackoffNs)) break;
+      for (int sh = 8; sh >= 1; sh >>= 1)
 #pragma unroll
-        for (int cc = 0; cc < NB; ++cc) sSS[(pb * 4 + slice * NB + cc) * 64 + i] = part[cc];
-        for (int r = 0; r < CS; ++r)
-          if (r != slice) mbar_arrive_remote(&nfull_b[pb], static_cast<uint32_t>(r));
-        if (!mbar_wait_warp(&nfull_b[pb], (c >> 1) & 1, ab, true, kBackoffNs)) break;
-        float blk[4];
+        for (int m = 0; m < 8; ++m) inv[m] += __shfl_xor_sync(0xffffffffu, inv[m], sh);
 #pragma unroll
-        for (int bidx = 0; bidx < 4; ++bidx) {
-          const int owner = bidx / NB;
-          blk[bidx] = owner == slice ? part[bidx % NB]
-                                     : ld_shared_remote(sSS + (pb * 4 + bidx) * 64 + i, static_cast<uint32_t>(owner));
-        }
-        total = ((blk[0] + blk[1]) + blk[2]) + blk[3];
-        for (int r = 0; r < CS; ++r)
-          if (r != slice) mbar_arrive_remote(&nack_b[pb], static_cast<uint32_t>(r));
+      for (int m = 0; m < 8; ++m) inv[m] = rsqrtf(inv[m] * (1.0f / kD) + 1e-6f);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int r = (otid >> 4) + 8 * m;
+        const float4* orow = reinterpret_cast<const float4*>(sO + r * kD + v8);
+        const float4 a0 = orow[0], a1 = orow[1];
+        const float o8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        float z8[8], y8[8];
+        unpack8(zr[m], z8);
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) y8[e2] = o8[e2] * inv[m] * w8[e2] * silu_fast(z8[e2]);
+        if (r < L)
+          *reinterpret_cast<uint4*>(p.out + ((tok0 + r) * p.H_v + h) * kD + v8) = pack8(y8);
       }
-      const float inv = rsqrtf(total * (1.0f / kD) + 1e-6f);
-      const long long tok = s + static_cast<long long>(c) * kChunk + i;
-      const bool valid = tok < e;
-      uint4* orow = reinterpret_cast<uint4*>(p.out + ((valid ? tok : s) * p.H_v + h) * kD + slice * DV);
-      uint4 ob[NB * 4];
-#pragma unroll
-      for (int q = 0; q < NB * 4; ++q) {
-        float zz[8], f[8];
-        unpack8(zbuf[q], zz);
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) f[e2] = o[8 * q + e2] * inv * sNW[8 * q + e2] * silu_fast(zz[e2]);
-        ob[q] = pack8(f);
-      }
-      if (c + 1 < nc) load_z(c + 1);
-      if (valid) {
-#pragma unroll
-        for (int q = 0; q < NB * 4; ++q) orow[q] = ob[q];
-      }
+      named_bar_sync(1, 128);  // sO is rewritten by the next chunk
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (CS > 1) cluster_sync_all();
-  if (warp == 7) tmem_dealloc<Cfg::TMEM_COLS>(tbase);
+  if (warp == kWarpIssue) tmem_dealloc<512>(tbase);
 }
 
-template <int DV>
 cudaError_t launch_scan(const PrefillParams& p, cudaStream_t stream) {
-  using Cfg = ScanCfg<DV>;
-  cudaError_t err = cudaFuncSetAttribute(scan_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  cudaError_t err = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScSmem);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.N) * p.H_v * Cfg::CS, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::SMEM;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = Cfg::CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, scan_kernel<DV>, p);
+  scan_kernel<<<static_cast<unsigned>(p.N) * p.H_v, kScanThreads, kScSmem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t stream, void* const* events) {
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* const* events) {
   cudaError_t err;
   if (p.cu) {
     setup_kernel<<<1, 1024, 0, stream>>>(p);
@@ -1081,7 +1141,7 @@ cudaError_t launch_prefill(const PrefillParams& p, int dv_slice, cudaStream_t st
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);
-  err = dv_slice == 32 ? launch_scan<32>(p, stream) : launch_scan<64>(p, stream);
+  err = launch_scan(p, stream);
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), stream);
   return err;
 }

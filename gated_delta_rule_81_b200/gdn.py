@@ -36,7 +36,7 @@ class GdnInputs(ctypes.Structure):
         ("stride_q", ctypes.c_longlong), ("stride_k", ctypes.c_longlong), ("stride_v", ctypes.c_longlong),
         ("stride_z", ctypes.c_longlong), ("stride_a", ctypes.c_longlong), ("stride_b", ctypes.c_longlong),
         ("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
-        ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("scale", ctypes.c_float), ("dv_slice", ctypes.c_int),
+        ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("scale", ctypes.c_float),
         ("events", ctypes.c_void_p),
     ]
 
@@ -86,7 +86,7 @@ def _tok_stride(t, T_tot):
     return t.stride(0)
 
 
-def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0, dv_slice=0) -> GdnInputs:
+def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0) -> GdnInputs:
     T_tot = q.shape[0]
     H_k = q.shape[1] if q.dim() == 3 else q.shape[-1] // HEAD_DIM
     H_v = v.shape[1] if v.dim() == 3 else v.shape[-1] // HEAD_DIM
@@ -101,7 +101,7 @@ def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0, dv_slice=0) 
     s.stride_q, s.stride_k, s.stride_v = (_tok_stride(t, T_tot) for t in (q, k, v))
     s.stride_z, s.stride_a, s.stride_b = (_tok_stride(t, T_tot) for t in (z, a, b))
     s.conv_w, s.A_log, s.norm_w = conv_w.data_ptr(), A_log.data_ptr(), norm_w.data_ptr()
-    s.H_k, s.H_v, s.scale, s.dv_slice = int(H_k), int(H_v), float(scale), int(dv_slice)
+    s.H_k, s.H_v, s.scale = int(H_k), int(H_v), float(scale)
     return s
 
 

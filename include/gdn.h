@@ -78,8 +78,6 @@ typedef struct {
   const void* norm_w;     /* bf16 [128] */
   int H_k, H_v;
   float scale;            /* multiplies the normalised q; 1.0 = o_t = S_t q_t as written above */
-  int dv_slice;           /* prefill only: state rows per scan CTA, 32 or 64, or 0 = automatic
-                             (128 is rejected with GDN_ERR_UNSUPPORTED); results do not depend on it */
   void* const* events;    /* optional timing hook: NULL, or caller-created cudaEvent_t handles that
                              the library records on `stream` around its kernels.  Prefill: 3 events,
                              [0] before the prep kernel, [1] between prep and scan, [2] after the
@@ -121,8 +119,7 @@ gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in
  *                    is computed and *err gets bit 4)
  * Every sequence starts from its own state_in[n] / conv_in[n] (or zeros): state
  * and conv history never cross a cu_seqlens boundary.  Results for sequence n
- * are bitwise identical to a gdn_prefill of that sequence alone with the same
- * dv_slice.  Other arguments as in gdn_prefill with leading dimension N; the
+ * are bitwise identical to a gdn_prefill of that sequence alone.  Other arguments as in gdn_prefill with leading dimension N; the
  * workspace size uses n_chunks = sum ceil((cu[n+1]-cu[n]) / 64).
  */
 gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens,
@@ -150,8 +147,8 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
  * GDN_NOALLOC_SCRATCH_BYTES inside libgdn.so, which every GPU that loads the
  * library holds until the process exits.
  *   - Limit: gdn_prefill_workspace_size(H_k, H_v, B, B*ceil(T/64)) must not
- *     exceed GDN_NOALLOC_SCRATCH_BYTES (64 MiB: e.g. up to 15 chunks of 64
- *     tokens in total at 16/48 heads, 126 at 2/6 heads); larger requests return
+ *     exceed GDN_NOALLOC_SCRATCH_BYTES (64 MiB: e.g. up to 11 chunks of 64
+ *     tokens in total at 16/48 heads, 88 at 2/6 heads); larger requests return
  *     GDN_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call

@@ -16,11 +16,11 @@ BF16_ULP = 2.0 ** -8
 STATE_TOL = 5e-3   # ||S_gpu - S_ref||_F / ||S_ref||_F <= STATE_TOL per sequence
 
 
-def device_inputs(inp, dev="cuda", dv_slice=0):
+def device_inputs(inp, dev="cuda"):
     """Copy the per-token inputs and parameters to the device; returns (keep, GdnInputs)."""
     keep = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
     s = gdn.make_inputs(keep["q"], keep["k"], keep["v"], keep["a"], keep["b"], keep["z"], keep["conv_w"],
-                        keep["A_log"], keep["norm_w"], scale=keep.get("scale", 1.0), dv_slice=dv_slice)
+                        keep["A_log"], keep["norm_w"], scale=keep.get("scale", 1.0))
     return keep, s
 
 

@@ -39,7 +39,7 @@ def test_workspace_size(lib):
     base = gdn.workspace_size(16, 48, 1, 0)
     assert base > 0
     per_chunk = gdn.workspace_size(16, 48, 1, 1) - base
-    assert per_chunk == 16 * 65536 + 48 * 66560
+    assert per_chunk == 16 * 32768 + 48 * 115712
     assert gdn.workspace_size(0, 48, 1, 1) == 0
     assert gdn.workspace_size(16, 48, -1, 1) == 0
 
@@ -51,7 +51,7 @@ def fake_inputs(H_k=2, H_v=6, ptr=0x10000):
     s.stride_q = s.stride_k = H_k * 128
     s.stride_v = s.stride_z = H_v * 128
     s.stride_a = s.stride_b = H_v
-    s.H_k, s.H_v, s.scale, s.dv_slice = H_k, H_v, 1.0, 0
+    s.H_k, s.H_v, s.scale = H_k, H_v, 1.0
     return s
 
 
@@ -65,11 +65,6 @@ def test_rejects_bad_shapes(lib):
     s = fake_inputs(H_k=4, H_v=6)  # 6 % 4 != 0
     assert call_prefill(lib, s) == 1
     s = fake_inputs(H_k=1, H_v=16)  # group of 16 value heads per key head
-    assert call_prefill(lib, s) == 2
-    s = fake_inputs()
-    s.dv_slice = 48
-    assert call_prefill(lib, s) == 1
-    s.dv_slice = 128
     assert call_prefill(lib, s) == 2
     s = fake_inputs()
     s.stride_q = 100  # below H_k * 128

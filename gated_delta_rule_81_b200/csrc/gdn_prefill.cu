@@ -167,39 +167,82 @@ constexpr int kLdA = 65;                               // fp32 row stride of A i
 constexpr int kLdT = 68;                               // fp32 row stride of T (16-byte aligned rows)
 // [Q;K] operand image in shared memory: hi at +0, lo at +32768; K-block kb (channels
 // 64 kb .. 64 kb + 63) at kb * 16384, rows 0..63 = Q tokens, rows 64..127 = K tokens.
+// The K rows are the workspace's K image (four 8 KiB pieces, bulk-stored from here).
 constexpr int kPrepOffQK = 0;
-// Once the [Q;K] K^T product has completed, the Q rows of the four K-block halves
-// hold the head loop's K-major B images: B_W = T diag(beta gamma), B_U = T diag(beta)
+// Once the products that read Q have completed, the four 8 KiB Q pieces are scratch:
+// per value head they stage P (hi, lo), then hold the B images B_W = T diag(beta gamma)
+// and B_U = T diag(beta), then stage W^T (lo rows 0..63, 64..127, hi rows 0..63, 64..127).
 constexpr int kPrepOffBWhi = 0, kPrepOffBUhi = 16384, kPrepOffBWlo = 32768, kPrepOffBUlo = 49152;
-constexpr int kPrepOffT = 65536;                       // T fp32                64*68*4
-// Once the B images are built, T, A and the block-solve temp are dead: the
-// region then holds the value head's v_hat image (A operand of U0^T, MN-major:
-// rows = tokens, two 64-channel blocks, hi then lo; 32 KiB)
-constexpr int kPrepOffV = kPrepOffT;
+// Region R (37 KiB) changes role through the kernel:
+//   the raw q | k rows of the chunk (front-end input, rows of kRawStride bytes);
+//   the identity B image of the q^T transpose;
+//   per value head: T, A and the block-solve temp; then the v_hat image (A operand
+//   of U0^T, MN-major: rows = tokens, two 64-channel blocks, hi then lo); then the
+//   staged (gamma Q)^T images (hi, lo).
+constexpr int kPrepOffR = 65536;
+constexpr int kRawStride = 2 * kD * 2 + 16;            // q row | k row, 16 B of padding against bank conflicts
+constexpr int kPrepOffT = kPrepOffR;                   // T fp32                64*68*4
 constexpr int kPrepOffA = kPrepOffT + 64 * kLdT * 4;   // A fp32                64*65*4
 constexpr int kPrepOffM = kPrepOffA + 64 * kLdA * 4;   // block-solve temp      3*256*4
-constexpr int kPrepOffG = kPrepOffM + 3 * 256 * 4;     // G cumsum   [8][64]
+constexpr int kPrepRBytes = 64 * kLdT * 4 + 64 * kLdA * 4 + 3 * 256 * 4;
+constexpr int kPrepOffG = kPrepOffR + kPrepRBytes;     // G cumsum   [8][64]
 constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta       [8][64]
 constexpr int kPrepOffGam = kPrepOffB + 8 * 64 * 4;    // gamma = e^G [8][64]
 constexpr int kPrepOffW = kPrepOffGam + 8 * 64 * 4;    // conv weights of the q, k and v channels, (2+G)*128*8 B
 __host__ __device__ constexpr int prep_smem_bytes(int G) { return kPrepOffW + (2 + G) * 128 * 8 + 1024; }
-static_assert(kPrepOffV + 2 * kImg64 <= kPrepOffG, "the v_hat image must fit the solve buffers");
+static_assert(2 * kImg64 <= kPrepRBytes, "the v_hat and (gamma Q)^T images must fit region R");
+static_assert((kChunk + kTaps - 1) * kRawStride <= kPrepRBytes, "the raw q | k rows must fit region R");
 // tensor memory columns (256 per CTA, two CTAs per SM)
 constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns);
                                       // then q^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColW = 128;   // W^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColU = 192;   // U0^T (lane = d_v, column = token)
 
-// hi = bf16(f), lo = bf16(f - hi) for 8 values
-__device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
-  float h[8], l[8];
+// W words of bf16 pairs from 2W fp32 values: hi[m] = (bf16(x[2m]), bf16(x[2m+1])) with
+// the even element in the low half, lo[m] the same for the residuals x - hi.  One paired
+// conversion per two values for each of hi and lo.
+template <int W>
+__device__ __forceinline__ void split_pairs(const float* x, uint32_t* hi, uint32_t* lo) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    h[e] = __bfloat162float(__float2bfloat16(f[e]));
-    l[e] = f[e] - h[e];
+  for (int m = 0; m < W; ++m) {
+    const uint32_t h = pack_bf16x2(x[2 * m], x[2 * m + 1]);
+    hi[m] = h;
+    lo[m] = pack_bf16x2(x[2 * m] - bf16_lo(h), x[2 * m + 1] - bf16_hi(h));
   }
-  hi = pack8(h);
-  lo = pack8(l);
+}
+
+// hi = bf16(f), lo = bf16(f - hi) for 8 values, packed as 16-byte rows
+__device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+  split_pairs<4>(f, h, l);
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// The 4-tap conv + SiLU of 32 channels from their raw inputs (tap j = token t - 3 + j, 4 x 8 bf16
+// per tap): wsm holds the 32 channels' weights, 16 x uint4 (channels 2u, 2u+1; taps 0..3 each).
+__device__ __forceinline__ void conv_taps(const uint4 (&xin)[kTaps][4], const uint4* wsm, float* y) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float x[kTaps][8];
+#pragma unroll
+    for (int j = 0; j < kTaps; ++j) unpack8(xin[j][g], x[j]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {  // channel pair 8g + 2u, 8g + 2u + 1
+      const uint4 w = wsm[4 * g + u];
+      const int e0 = 2 * u, e1 = 2 * u + 1;
+      float a0 = bf16_lo(w.x) * x[0][e0];
+      a0 = fmaf(bf16_hi(w.x), x[1][e0], a0);
+      a0 = fmaf(bf16_lo(w.y), x[2][e0], a0);
+      a0 = fmaf(bf16_hi(w.y), x[3][e0], a0);
+      float a1 = bf16_lo(w.z) * x[0][e1];
+      a1 = fmaf(bf16_hi(w.z), x[1][e1], a1);
+      a1 = fmaf(bf16_lo(w.w), x[2][e1], a1);
+      a1 = fmaf(bf16_hi(w.w), x[3][e1], a1);
+      y[8 * g + e0] = silu_fast(a0);
+      y[8 * g + e1] = silu_fast(a1);
+    }
+  }
 }
 
 // Conv (4 taps) + SiLU of 32 consecutive channels of one token.
@@ -223,27 +266,7 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
 #pragma unroll
     for (int g = 0; g < 4; ++g) xin[j][g] = row ? __ldg(row + g) : make_uint4(0u, 0u, 0u, 0u);
   }
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float x[kTaps][8];
-#pragma unroll
-    for (int j = 0; j < kTaps; ++j) unpack8(xin[j][g], x[j]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {  // channel pair 8g + 2u, 8g + 2u + 1
-      const uint4 w = wsm[4 * g + u];
-      const int e0 = 2 * u, e1 = 2 * u + 1;
-      float a0 = bf16_lo(w.x) * x[0][e0];
-      a0 = fmaf(bf16_hi(w.x), x[1][e0], a0);
-      a0 = fmaf(bf16_lo(w.y), x[2][e0], a0);
-      a0 = fmaf(bf16_hi(w.y), x[3][e0], a0);
-      float a1 = bf16_lo(w.z) * x[0][e1];
-      a1 = fmaf(bf16_hi(w.z), x[1][e1], a1);
-      a1 = fmaf(bf16_lo(w.w), x[2][e1], a1);
-      a1 = fmaf(bf16_hi(w.w), x[3][e1], a1);
-      y[8 * g + e0] = silu_fast(a0);
-      y[8 * g + e1] = silu_fast(a1);
-    }
-  }
+  conv_taps(xin, wsm, y);
 }
 
 // One block diagonal of the blocked inverse: for blocks (I, J = I - d),
@@ -326,23 +349,28 @@ __device__ __forceinline__ void umma_split(uint32_t d, uint64_t a_hi, uint64_t a
 
 // W words of bf16 pairs from 2W fp32 values: hi[m] = (bf16(x[2m]), bf16(x[2m+1])) with
 // the even element in the low half, lo[m] the same for the residuals x - hi.
-template <int W>
-__device__ __forceinline__ void split_pairs(const float* x, uint32_t* hi, uint32_t* lo) {
+// Conv (4 taps) + SiLU of 32 consecutive channels of token i from the staged raw rows
+// (row r holds token t0 - 3 + r; `off` = byte offset of the 32-channel group in a row).
+__device__ __forceinline__ void conv32_rows(const uint8_t* raw, int i, int off, const uint4* wsm, float* y) {
+  uint4 xin[kTaps][4];
 #pragma unroll
-  for (int m = 0; m < W; ++m) {
-    const uint32_t h = pack_bf16x2(x[2 * m], x[2 * m + 1]);
-    hi[m] = h;
-    lo[m] = pack_bf16x2(x[2 * m] - bf16_lo(h), x[2 * m + 1] - bf16_hi(h));
+  for (int j = 0; j < kTaps; ++j) {
+    const uint4* row = reinterpret_cast<const uint4*>(raw + (i + j) * kRawStride + off);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) xin[j][g] = row[g];
   }
+  conv_taps(xin, wsm, y);
 }
 
 // One CTA per (chunk, key head).  Writes the chunk's K image for the key head
 // and, for each of its value heads, W^T, (gamma Q)^T, P, U0 and the gate vectors.
+// The operand images leave shared memory as bulk stores.
 __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;
   extern __shared__ uint8_t prep_smem_raw[];
   uint8_t* sm = align1024(prep_smem_raw);
   uint8_t* sQK = sm + kPrepOffQK;
+  uint8_t* sR = sm + kPrepOffR;
   float* sA = reinterpret_cast<float*>(sm + kPrepOffA);
   float* sT = reinterpret_cast<float*>(sm + kPrepOffT);
   float* sM = reinterpret_cast<float*>(sm + kPrepOffM);
@@ -350,8 +378,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
   float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
   uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2 + G) * 64] channel pairs: q | k | v heads
-  uint8_t* sV = sm + kPrepOffV;
-  __shared__ uint64_t bar[4];
+  __shared__ uint64_t bar[5];  // [Q;K] K^T, W / U0 (per head), drain, q^T, raw rows landed
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -376,17 +403,45 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   const long long s = seq_start(p, n), e = seq_start(p, n + 1);
   const long long t0 = s + (gc - chunk_base_of(p, n)) * kChunk;
   const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - t0));
+  const int nrows = L + kTaps - 1;  // raw rows of tokens t0 - 3 .. t0 + L - 1
 
   Abort ab{p.err, &abort_s};
   if (tid == 0) {
     abort_s = 0;
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    mbar_init(&bar[2], 1);
-    mbar_init(&bar[3], 1);
+    for (int b = 0; b < 5; ++b) mbar_init(&bar[b], 1);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc<256>(&tmem_base_s);
+  __syncthreads();
+
+  // ---- raw q | k rows into region R (bulk copies by warp 7; rows before the sequence start
+  // come from conv_in, or are zero), and the value heads' raw v rows into L2 for later
+  if (warp == 7) {
+    uint32_t bytes = 0;
+    for (int r = 0; r < nrows; ++r)
+      if (t0 - (kTaps - 1) + r >= s || p.conv_in) bytes += 2 * kD * 2;
+    if (lane == 0) mbar_arrive_expect_tx(&bar[4], bytes);
+    __syncwarp();
+    for (int x = lane; x < 2 * nrows; x += 32) {
+      const int r = x >> 1, which = x & 1;
+      const long long tau = t0 - (kTaps - 1) + r;
+      uint8_t* dst = sR + r * kRawStride + which * kD * 2;
+      const bf16* src = nullptr;
+      if (tau >= s) src = (which ? p.k + tau * p.sk : p.q + tau * p.sq) + static_cast<long long>(kh) * kD;
+      else if (p.conv_in)
+        src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + static_cast<long long>(which * H_k + kh) * kD;
+      if (src) {
+        bulk_g2s(dst, src, kD * 2, &bar[4]);
+      } else {
+#pragma unroll
+        for (int q4 = 0; q4 < 16; ++q4) reinterpret_cast<uint4*>(dst)[q4] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    for (int r = lane; r < nrows; r += 32) {
+      const long long tau = t0 - (kTaps - 1) + r;
+      if (tau >= s) prefetch_l2(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD, static_cast<uint32_t>(G * kD * 2));
+    }
+  }
 
   // conv weights of this CTA's channels (q, k of key head kh; v of its G value heads)
   for (int x = tid; x < (2 + G) * 64; x += kPrepThreads) {
@@ -396,75 +451,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
                                    : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh * G + grp - 2) * kD;
     sW[x] = __ldg(reinterpret_cast<const uint4*>(p.conv_w + (ch0 + 2 * pair) * kTaps));
   }
-  // the raw v rows of the key head's value heads are read later in the head loop: into L2 now
-  if (warp == 7) {
-    for (int r = lane; r < L + 3; r += 32) {
-      const long long tau = t0 - 3 + r;
-      if (tau >= s) prefetch_l2(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD, static_cast<uint32_t>(G * kD * 2));
-    }
-  }
-  __syncthreads();
 
-  // ---- front end of q and k: token i, channels 32*qq .. 32*qq+31
-  uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
-  {
-    const int i = tid >> 2, qq = tid & 3;
-    const bool valid = i < L;
-    for (int which = 0; which < 2; ++which) {
-      const bf16* X = which ? p.k : p.q;
-      const long long sx = which ? p.sk : p.sq;
-      const long long chan0 = static_cast<long long>(which) * H_k * kD + static_cast<long long>(kh) * kD + 32 * qq;
-      float y[32];
-      if (valid) conv32(p, X + static_cast<long long>(kh) * kD + 32 * qq, sx, s, t0 + i, n, chan0, sW + which * 64 + 16 * qq, y);
-      float ss = 0.f;
-#pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) {
-        if (!valid) y[e2] = 0.f;
-        ss = fmaf(y[e2], y[e2], ss);
-      }
-      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-      const float inv = rsqrtf(ss + 1e-6f) * (which == 0 ? p.scale : 1.0f);
-      const int row = which * 64 + i, kb = qq >> 1;
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        float f[8];
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) f[e2] = y[8 * c2 + e2] * inv;
-        uint4 hi, lo;
-        split8(f, hi, lo);
-        const uint32_t soff = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
-        *reinterpret_cast<uint4*>(sQK + soff) = hi;
-        *reinterpret_cast<uint4*>(sQK + 32768 + soff) = lo;
-        if (which == 1) {
-          const uint32_t goff = kb * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
-          *reinterpret_cast<uint4*>(gK + goff) = hi;
-          *reinterpret_cast<uint4*>(gK + kImg64 + goff) = lo;
-        }
-      }
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = tmem_base_s;
-
-  // ---- [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
-  if (tid == 0) {
-    const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
-    const uint32_t idesc = idesc_bf16(128, 64, false, false);
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-      umma_split(tbase + kPrepColQK, smem_desc(qh + ko, 16, 1024, Swz::k128), smem_desc(ql + ko, 16, 1024, Swz::k128),
-                 smem_desc(qh + ko + 8192, 16, 1024, Swz::k128), smem_desc(ql + ko + 8192, 16, 1024, Swz::k128),
-                 idesc, ks > 0);
-    }
-    umma_commit(&bar[0]);
-  }
-
-  // ---- gates of the key head's value heads (overlaps the MMA)
+  // ---- gates of the key head's value heads
   for (int base = 0; base < G * 64; base += kPrepThreads) {
     const int x = base + tid;
     if (x < G * 64) {  // warp-uniform: G*64 is a multiple of 64
@@ -486,7 +474,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       sB[j * 64 + i] = beta;
     }
   }
-  __syncthreads();
+  __syncthreads();  // also publishes warp 7's zero rows and sW
   for (int x = tid; x < G * 32; x += kPrepThreads) {
     const int j = x >> 5, i = 32 + (x & 31);
     sG[j * 64 + i] += sG[j * 64 + 31];
@@ -509,6 +497,77 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     gdst[k2] = val;
   }
 
+  // ---- front end of q and k from the staged rows: token i, channels 32*qq .. 32*qq+31
+  mbar_wait_warp(&bar[4], 0, ab);
+  {
+    const int i = tid >> 2, qq = tid & 3;
+    const bool valid = i < L;
+    for (int which = 0; which < 2; ++which) {
+      float y[32];
+      if (valid) conv32_rows(sR, i, which * kD * 2 + qq * 64, sW + which * 64 + 16 * qq, y);
+      float ss = 0.f;
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) {
+        if (!valid) y[e2] = 0.f;
+        ss = fmaf(y[e2], y[e2], ss);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      const float inv = rsqrtf(ss + 1e-6f) * (which == 0 ? p.scale : 1.0f);
+      const int row = which * 64 + i, kb = qq >> 1;
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float f[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) f[e2] = y[8 * c2 + e2] * inv;
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t soff = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
+        *reinterpret_cast<uint4*>(sQK + soff) = hi;
+        *reinterpret_cast<uint4*>(sQK + 32768 + soff) = lo;
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+
+  // ---- the K image to the workspace (the K rows of the four K-block halves), and
+  // [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
+  if (tid == 0) {
+    uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
+    bulk_s2g(gK, sQK + 8192, 8192);
+    bulk_s2g(gK + 8192, sQK + 24576, 8192);
+    bulk_s2g(gK + 16384, sQK + 40960, 8192);
+    bulk_s2g(gK + 24576, sQK + 57344, 8192);
+    bulk_commit();
+    const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
+    const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
+      umma_split(tbase + kPrepColQK, smem_desc(qh + ko, 16, 1024, Swz::k128), smem_desc(ql + ko, 16, 1024, Swz::k128),
+                 smem_desc(qh + ko + 8192, 16, 1024, Swz::k128), smem_desc(ql + ko + 8192, 16, 1024, Swz::k128),
+                 idesc, ks > 0);
+    }
+    umma_commit(&bar[0]);
+  }
+  // identity B image for the q^T transpose, in region R (the raw rows are dead)
+  {
+    uint8_t* sId = sR;
+    for (int x = tid; x < 64 * 8; x += kPrepThreads) {
+      const int i = x >> 3, cc = x & 7;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (cc == (i >> 3)) {
+        const int e8 = i & 7;
+        w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
+      }
+      *reinterpret_cast<uint4*>(sId + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+
   // ---- K K^T and Q K^T rows into registers: thread row = 32*(warp%4)+lane, columns cbase..cbase+31
   const int row = 32 * (warp & 3) + lane;
   const int cbase = 32 * (warp >> 2);
@@ -523,39 +582,28 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 #pragma unroll
     for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
   }
+
   // ---- q^T (lane = d_k, column = token) into TMEM columns 0..63, which the [Q;K] K^T
   // product no longer needs: Q_hi^T I + Q_lo^T I with an identity B, exact in fp32
-  {
-    uint8_t* sId = sm + kPrepOffA;  // 64 x 64 bf16 identity, K-major (before sA is built)
-    for (int x = tid; x < 64 * 8; x += kPrepThreads) {
-      const int i = x >> 3, cc = x & 7;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (cc == (i >> 3)) {
-        const int e8 = i & 7;
-        w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
-      }
-      *reinterpret_cast<uint4*>(sId + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();  // sG's second half, sGam and the identity are complete; acc has been read
-    tc_fence_after();
-    if (tid == 0) {
-      const uint32_t qk = smem_u32(sQK), id = smem_u32(sId);
-      const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();  // the identity is complete; acc has been read
+  tc_fence_after();
+  if (tid == 0) {
+    const uint32_t qk = smem_u32(sQK), id = smem_u32(sR);
+    const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
-        umma_bf16(tbase + kPrepColQK, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
-        umma_bf16(tbase + kPrepColQK, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
-      }
-      umma_commit(&bar[3]);
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
+      umma_bf16(tbase + kPrepColQK, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
+      umma_bf16(tbase + kPrepColQK, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
     }
-    __syncwarp();
-    mbar_wait_warp(&bar[3], 0, ab);
-    tc_fence_after();
-    __syncthreads();  // the identity (sA region) may now be overwritten
+    umma_commit(&bar[3]);
   }
+  __syncwarp();
+  mbar_wait_warp(&bar[3], 0, ab);
+  tc_fence_after();
+  __syncthreads();  // Q and the identity are dead: the Q pieces and region R are scratch from here
 
   for (int j = 0; j < G; ++j) {
     const int h = kh * G + j;
@@ -569,7 +617,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         sA[ri * kLdA + col] = col < ri ? bi * __expf(Gi - sG[j * 64 + col]) * acc[e2] : 0.f;
       }
     } else {
-      // P_ij = e^{G_i - G_j} (q_i . k_j) for j <= i, as the K-major image (row i) in the workspace
+      // P_ij = e^{G_i - G_j} (q_i . k_j) for j <= i: K-major image (row i), staged hi in the Q
+      // piece at 0 and lo in the one at 32768
 #pragma unroll
       for (int c2 = 0; c2 < 4; ++c2) {
         float f[8];
@@ -581,12 +630,20 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         uint4 hi, lo;
         split8(f, hi, lo);
         const uint32_t off = sw128_off(ri, (cbase >> 3) + c2);
-        *reinterpret_cast<uint4*>(hb + kHeadOffP + off) = hi;
-        *reinterpret_cast<uint4*>(hb + kHeadOffP + kPImg + off) = lo;
+        *reinterpret_cast<uint4*>(sQK + off) = hi;
+        *reinterpret_cast<uint4*>(sQK + 32768 + off) = lo;
       }
+      fence_proxy_async_smem();
     }
     __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(hb + kHeadOffP, sQK, kPImg);
+      bulk_s2g(hb + kHeadOffP + kPImg, sQK + 32768, kPImg);
+      bulk_commit();
+    }
     solve_unit_lower(sA, sT, sM, tid);
+    if (tid == 0) bulk_wait_read<0>();  // P has left the Q pieces
+    __syncthreads();
     // B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
     for (int x = tid; x < 64 * 8; x += kPrepThreads) {
       const int r = x >> 3, cc = x & 7;
@@ -607,7 +664,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       *reinterpret_cast<uint4*>(sQK + kPrepOffBUhi + off) = hi;
       *reinterpret_cast<uint4*>(sQK + kPrepOffBUlo + off) = lo;
     }
-    __syncthreads();  // T is dead: its region takes the v_hat image
+    __syncthreads();  // T is dead: region R takes the v_hat image
     {
       // v_hat of value head h: token i, channels 32*qq .. 32*qq+31, as the MN-major image
       const int i = tid >> 2, qq = tid & 3;
@@ -624,8 +681,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
         uint4 hi, lo;
         split8(y + 8 * c2, hi, lo);
         const uint32_t off = (qq >> 1) * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
-        *reinterpret_cast<uint4*>(sV + off) = hi;
-        *reinterpret_cast<uint4*>(sV + kImg64 + off) = lo;
+        *reinterpret_cast<uint4*>(sR + off) = hi;
+        *reinterpret_cast<uint4*>(sR + kImg64 + off) = lo;
       }
     }
     fence_proxy_async_smem();
@@ -643,7 +700,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
                    smem_desc(qk + kPrepOffBWhi + ks * 32u, 16, 1024, Swz::k128),
                    smem_desc(qk + kPrepOffBWlo + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
       // U0^T = V^T B_U^T: A = v_hat (MN-major, rows = tokens), B = B_U (K-major)
-      const uint32_t vv = smem_u32(sV);
+      const uint32_t vv = smem_u32(sR);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         umma_split(tbase + kPrepColU, smem_desc(vv + ks * 2048u, 8192, 1024, Swz::k128),
@@ -655,9 +712,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     __syncwarp();
     if (mbar_wait_warp(&bar[1], j & 1, ab)) {
       tc_fence_after();
-      float o[64];
       {
-        // (gamma Q)^T row d_k = lane, tokens 32*(warp/4) .. +31: hi and lo images
+        // (gamma Q)^T row d_k = lane, tokens 32*(warp/4) .. +31: staged in region R, hi then lo
         const int kr = 32 * (warp & 3) + lane, half = warp >> 2;
         float qg[32];
         tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + 32 * half), qg);
@@ -670,23 +726,26 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
           uint4 hi, lo;
           split8(f, hi, lo);
           const uint32_t off = sw128_off(kr, 4 * half + c2);
-          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 2 * kImg64 + off) = hi;
-          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 3 * kImg64 + off) = lo;
+          *reinterpret_cast<uint4*>(sR + off) = hi;
+          *reinterpret_cast<uint4*>(sR + kImg64 + off) = lo;
         }
       }
+      float o[64];
       if (warp < 4) {
-        // W^T row d_k = lane: the MN-major image row (64 tokens), lo image then hi image
+        // W^T row d_k = lane (64 tokens): staged lo rows 0..63 | 64..127 in the Q pieces at 0 | 16384,
+        // hi rows 0..63 | 64..127 at 32768 | 49152
         tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW), o);
         tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW + 32), o + 32);
         tmem_wait_ld();
         const int kr = 32 * warp + lane;
+        const uint32_t half_off = kr < 64 ? 0u : 16384u;
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           uint4 hi, lo;
           split8(o + 8 * cc, hi, lo);
-          const uint32_t off = sw128_off(kr, cc);
-          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + kImg64 + off) = hi;
-          *reinterpret_cast<uint4*>(hb + kHeadOffWQ + off) = lo;
+          const uint32_t off = sw128_off(kr & 63, cc);
+          *reinterpret_cast<uint4*>(sQK + half_off + off) = lo;
+          *reinterpret_cast<uint4*>(sQK + 32768 + half_off + off) = hi;
         }
       } else {
         // U0 [token][d_v] fp32: a warp writes 128 contiguous bytes per token
@@ -697,18 +756,31 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 #pragma unroll
         for (int i = 0; i < 64; ++i) u0[i * kD] = o[i];
       }
+      fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 0) {
+      uint8_t* wq = hb + kHeadOffWQ;  // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
+      bulk_s2g(wq, sQK, 8192);
+      bulk_s2g(wq + 8192, sQK + 16384, 8192);
+      bulk_s2g(wq + 16384, sQK + 32768, 8192);
+      bulk_s2g(wq + 24576, sQK + 49152, 8192);
+      bulk_s2g(wq + 2 * kImg64, sR, 2 * kImg64);
+      bulk_commit();
+      bulk_wait_read<0>();  // the staging areas are rewritten by the next value head
+    }
+    __syncthreads();
   }
 
-  // drain: every MMA this CTA issued has completed before TMEM is released
+  // drain: every MMA this CTA issued and every bulk store has completed
   if (tid == 0) {
     umma_commit(&bar[2]);
     int drain_flag = 0;
     Abort drain{nullptr, &drain_flag};
     mbar_wait(&bar[2], 0, drain);
+    bulk_wait<0>();
   }
   tc_fence_before();
   __syncthreads();

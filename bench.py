@@ -55,12 +55,19 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {"scan": {"bytes": 325274624 + 42740736, "sha": "eb5fa90e952f2519"}}  # ncu, T=4096 layer
+TRAFFIC = {"scan": {"bytes": 442649856 + 44844288, "sha": "f74aec2f444d2102"},   # ncu, T=4096 layer
+           "prep": {"bytes": 100750336 + 339516416, "sha": "f74aec2f444d2102"}}
+DECODE_TRAFFIC = {"bytes": 829621504 + 767561728, "sha": "6ad12188ad3a4536"}  # ncu, one step of 256 sequences
 
 
 def src_sha(name):
     with open(os.path.join(ROOT, "gated_delta_rule_81_b200", "csrc", name), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def decode_traffic():
+    """DRAM bytes of one 256-sequence decode launch from the ncu capture, if the source is unchanged."""
+    return DECODE_TRAFFIC["bytes"] if DECODE_TRAFFIC["sha"] == src_sha("gdn_decode.cu") else None
 
 
 def peaks():
@@ -412,7 +419,8 @@ def main():
                               "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                               "config": {"workload": gin.CONFIGS[4]["name"]},
                               "roofline": {"bound": "hbm", "achieved": d["gbs"], "peak": pk["hbm_gbs"],
-                                           "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"], "traffic": None},
+                                           "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"],
+                                           "traffic": decode_traffic()},
                               "gpu_launches": 64}), flush=True)
         return 0
     cfg_id = WORKLOADS[args.workload]
@@ -458,7 +466,8 @@ def main():
         decode = {"workload": gin.CONFIGS[4]["name"], "metric": "decode state GB/s", "value": d["gbs"],
                   "unit": "GB/s", "ms_per_launch": d["ms_per_launch"],
                   "roofline": {"bound": "hbm", "achieved": d["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                               "frac": d["gbs"] / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}}
+                               "frac": d["gbs"] / pk["hbm_gbs"], "traffic": decode_traffic(),
+                               "peak_source": pk["source"]}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
   float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
   uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2 + G) * 64] channel pairs: q | k | v heads
-  __shared__ uint64_t bar[5];  // [Q;K] K^T, W / U0 (per head), drain, q^T, raw rows landed
+  __shared__ uint64_t bar[4];  // [Q;K] K^T, W / U0 (per head), drain, q^T
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -408,39 +408,31 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   Abort ab{p.err, &abort_s};
   if (tid == 0) {
     abort_s = 0;
-    for (int b = 0; b < 5; ++b) mbar_init(&bar[b], 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&bar[b], 1);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc<256>(&tmem_base_s);
   __syncthreads();
 
-  // ---- raw q | k rows into region R (bulk copies by warp 7; rows before the sequence start
-  // come from conv_in, or are zero), and the value heads' raw v rows into L2 for later
-  if (warp == 7) {
-    uint32_t bytes = 0;
-    for (int r = 0; r < nrows; ++r)
-      if (t0 - (kTaps - 1) + r >= s || p.conv_in) bytes += 2 * kD * 2;
-    if (lane == 0) mbar_arrive_expect_tx(&bar[4], bytes);
-    __syncwarp();
-    for (int x = lane; x < 2 * nrows; x += 32) {
-      const int r = x >> 1, which = x & 1;
-      const long long tau = t0 - (kTaps - 1) + r;
-      uint8_t* dst = sR + r * kRawStride + which * kD * 2;
-      const bf16* src = nullptr;
-      if (tau >= s) src = (which ? p.k + tau * p.sk : p.q + tau * p.sq) + static_cast<long long>(kh) * kD;
-      else if (p.conv_in)
-        src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + static_cast<long long>(which * H_k + kh) * kD;
-      if (src) {
-        bulk_g2s(dst, src, kD * 2, &bar[4]);
-      } else {
-#pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) reinterpret_cast<uint4*>(dst)[q4] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    for (int r = lane; r < nrows; r += 32) {
-      const long long tau = t0 - (kTaps - 1) + r;
-      if (tau >= s) prefetch_l2(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD, static_cast<uint32_t>(G * kD * 2));
-    }
+  // ---- raw q | k rows into region R: 16-byte asynchronous copies by all threads (a warp
+  // moves one 512-byte row per instruction); rows before the sequence start come from
+  // conv_in, or are zero.  The value heads' raw v rows are prefetched into L2 for later.
+  for (int x = tid; x < nrows * 32; x += kPrepThreads) {
+    const int r = x >> 5, piece = x & 31, which = piece >> 4;
+    const long long tau = t0 - (kTaps - 1) + r;
+    uint8_t* dst = sR + r * kRawStride + piece * 16;
+    const bf16* src = nullptr;
+    if (tau >= s) src = (which ? p.k + tau * p.sk : p.q + tau * p.sq) + static_cast<long long>(kh) * kD;
+    else if (p.conv_in)
+      src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + static_cast<long long>(which * H_k + kh) * kD;
+    if (src) cp_async16(dst, src + (piece & 15) * 8);
+    else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  cp_async_commit();
+  for (int x = tid; x < nrows * G * 2; x += kPrepThreads) {  // 128-byte lines of G*256-byte rows
+    const int r = x / (G * 2), line = x % (G * 2);
+    const long long tau = t0 - (kTaps - 1) + r;
+    if (tau >= s) prefetch_l2_line(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD + line * 64);
   }
 
   // conv weights of this CTA's channels (q, k of key head kh; v of its G value heads)
@@ -474,31 +466,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       sB[j * 64 + i] = beta;
     }
   }
-  __syncthreads();  // also publishes warp 7's zero rows and sW
+  __syncthreads();
   for (int x = tid; x < G * 32; x += kPrepThreads) {
     const int j = x >> 5, i = 32 + (x & 31);
     sG[j * 64 + i] += sG[j * 64 + 31];
   }
   __syncthreads();
-  // gate vectors for the scan: gamma_i, decay-to-end_i (0 past the chunk's last token), gamma_C
-  for (int x = tid; x < G * 256; x += kPrepThreads) {
-    const int j = x >> 8, k2 = x & 255, h = kh * G + j;
-    const float Glast = sG[j * 64 + (L - 1)];
-    float val = 0.f;
-    if (k2 < 64) {
-      val = expf(sG[j * 64 + k2]);
-      sGam[j * 64 + k2] = val;
-    } else if (k2 < 128) {
-      val = (k2 - 64) < L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
-    } else if (k2 == 128) {
-      val = expf(Glast);
-    }
-    float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate);
-    gdst[k2] = val;
-  }
-
+  for (int x = tid; x < G * 64; x += kPrepThreads) sGam[x] = expf(sG[x]);
   // ---- front end of q and k from the staged rows: token i, channels 32*qq .. 32*qq+31
-  mbar_wait_warp(&bar[4], 0, ab);
+  cp_async_wait_all();
+  __syncthreads();
   {
     const int i = tid >> 2, qq = tid & 3;
     const bool valid = i < L;
@@ -554,6 +531,22 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     }
     umma_commit(&bar[0]);
   }
+  // gate vectors for the scan: gamma_i, decay-to-end_i (0 past the chunk's last token), gamma_C
+  for (int x = tid; x < G * 256; x += kPrepThreads) {
+    const int j = x >> 8, k2 = x & 255, h = kh * G + j;
+    const float Glast = sG[j * 64 + (L - 1)];
+    float val = 0.f;
+    if (k2 < 64) {
+      val = sGam[j * 64 + k2];
+    } else if (k2 < 128) {
+      val = (k2 - 64) < L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
+    } else if (k2 == 128) {
+      val = expf(Glast);
+    }
+    float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate);
+    gdst[k2] = val;
+  }
+
   // identity B image for the q^T transpose, in region R (the raw rows are dead)
   {
     uint8_t* sId = sR;

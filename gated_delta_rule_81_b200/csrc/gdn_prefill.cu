@@ -211,6 +211,20 @@ __device__ __forceinline__ void split_pairs(const float* x, uint32_t* hi, uint32
   }
 }
 
+// The same split with the residual pair x - hi as one packed fp32x2 fma (hi * (-1) + x;
+// exact, as x - hi is representable): fewer instructions, one more live register pair.
+template <int W>
+__device__ __forceinline__ void split_pairs_x2(const float* x, uint32_t* hi, uint32_t* lo) {
+#pragma unroll
+  for (int m = 0; m < W; ++m) {
+    const uint32_t h = pack_bf16x2(x[2 * m], x[2 * m + 1]);
+    hi[m] = h;
+    const float2 r = __ffma2_rn(make_float2(bf16_lo(h), bf16_hi(h)), make_float2(-1.f, -1.f),
+                                make_float2(x[2 * m], x[2 * m + 1]));
+    lo[m] = pack_bf16x2(r.x, r.y);
+  }
+}
+
 // hi = bf16(f), lo = bf16(f - hi) for 8 values, packed as 16-byte rows
 __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
   uint32_t h[4], l[4];
@@ -796,7 +810,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // product waits for; warps 8-11 run the output stage; warp 12 lane 0 issues the
 // MMAs in the order S W^T, S (gamma Q)^T, state update, U^T P^T, so that the
 // output's products fill the tensor pipe while the chain converts; warp 13
-// lane 0 issues the bulk copies.
+// lane 0 issues the bulk copies (W, gamma Q, K, P single-buffered, gates and U0 double-buffered).
 
 constexpr int kScanThreads = 448;
 constexpr int kWarpIssue = 12, kWarpProd = 13;
@@ -821,8 +835,8 @@ __host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base
 constexpr int kScOffWQ = 0;                            // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
 constexpr int kScOffK = kScOffWQ + kWQBytes;           // K hi, lo
 constexpr int kScOffP = kScOffK + kKBytes;             // P hi, lo
-constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // U0 fp32 [64][128]
-constexpr int kScOffO = kScOffU0 + kU0Bytes;           // o fp32 [64 tokens][128 d_v] for the token-major epilogue
+constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // 2 stages of U0 fp32 [64][128]
+constexpr int kScOffO = kScOffU0 + 2 * kU0Bytes;       // o fp32 [64 tokens][128 d_v] for the token-major epilogue
 constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 
@@ -831,7 +845,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
   extern __shared__ uint8_t scan_smem_raw[];
   uint8_t* sm = align1024(scan_smem_raw);
   __shared__ uint64_t g_full[2], g_free[2];
-  __shared__ uint64_t wq_full, wq_free, k_full, k_free, p_full, p_free, u0_full, u0_free;
+  __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, u0_full[2], u0_free[2];
   __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
@@ -850,15 +864,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
     for (int b = 0; b < 2; ++b) {
       mbar_init(&g_full[b], 1);
       mbar_init(&g_free[b], 256);
+      mbar_init(&u0_full[b], 1);
+      mbar_init(&u0_free[b], 256);
     }
-    mbar_init(&wq_full, 1);
-    mbar_init(&wq_free, 1);
+    mbar_init(&w_full, 1);
+    mbar_init(&w_free, 1);
+    mbar_init(&q_full, 1);
+    mbar_init(&q_free, 1);
     mbar_init(&k_full, 1);
     mbar_init(&k_free, 1);
     mbar_init(&p_full, 1);
     mbar_init(&p_free, 1);
-    mbar_init(&u0_full, 1);
-    mbar_init(&u0_free, 256);
     mbar_init(&s_conv, 256);
     mbar_init(&u_conv, 256);
     mbar_init(&u_conv2, 256);
@@ -881,7 +897,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
     const int v = 32 * (warp & 3) + lane, th = warp >> 2;
     const uint32_t tl = tmem_addr(tbase, 32 * (warp & 3), 0);
     const long long srow = ((static_cast<long long>(n) * p.H_v + h) * kD + v) * kD;
-    const float* U0 = reinterpret_cast<const float*>(sm + kScOffU0);
     bool ok = true;
     for (int c = 0; c < nc && ok; ++c) {
       const int gs = c & 1;
@@ -913,7 +928,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t hi[16], lo[16];
-        split_pairs<16>(sv + 32 * cc, hi, lo);
+        split_pairs_x2<16>(sv + 32 * cc, hi, lo);
         tmem_st16(tl + kColSH + 32 * th + 16 * cc, hi);
         tmem_st16(tl + kColSL + 32 * th + 16 * cc, lo);
       }
@@ -922,13 +937,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
       mbar_arrive(&s_conv);
       const float gC = gates[128];
 #pragma unroll
-      for (int e2 = 0; e2 < 64; ++e2) sv[e2] *= gC;
+      for (int e2 = 0; e2 < 64; e2 += 2) {
+        const float2 r = __fmul2_rn(make_float2(sv[e2], sv[e2 + 1]), make_float2(gC, gC));
+        sv[e2] = r.x;
+        sv[e2 + 1] = r.y;
+      }
       tmem_st32(tl + kColS + 64 * th, sv);
       tmem_st32(tl + kColS + 64 * th + 32, sv + 32);
       // ---- U^T = U0^T - S W^T for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first
       // (the state update waits for it), then U (the output product waits for it)
       ok = mbar_wait_warp(&u_done, c & 1, ab);
-      if (ok) ok = mbar_wait_warp(&u0_full, c & 1, ab);
+      if (ok) ok = mbar_wait_warp(&u0_full[gs], (c >> 1) & 1, ab);
+      const float* U0 = reinterpret_cast<const float*>(sm + kScOffU0 + gs * kU0Bytes);
       if (!ok) break;
       tc_fence_after();
       float u[32], ud[32];
@@ -938,15 +958,26 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
         tmem_ld32(tl + kColU1 + 32 * th, u1);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = U0[(32 * th + i) * kD + v] - (u1[i] + u[i]);
+        for (int i = 0; i < 32; i += 2) {  // u = U0 - (U1 + U2), packed in token pairs
+          const float2 acc = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
+          const float2 r = __ffma2_rn(acc, make_float2(-1.f, -1.f),
+                                      make_float2(U0[(32 * th + i) * kD + v], U0[(32 * th + i + 1) * kD + v]));
+          u[i] = r.x;
+          u[i + 1] = r.y;
+        }
       }
-      mbar_arrive(&u0_free);
+      mbar_arrive(&u0_free[gs]);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ud[i] = u[i] * gates[64 + 32 * th + i];
+      for (int i = 0; i < 32; i += 2) {
+        const float2 d = *reinterpret_cast<const float2*>(gates + 64 + 32 * th + i);
+        const float2 r = __fmul2_rn(make_float2(u[i], u[i + 1]), d);
+        ud[i] = r.x;
+        ud[i + 1] = r.y;
+      }
       mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time
       {
         uint32_t hi[16], lo[16];
-        split_pairs<16>(ud, hi, lo);
+        split_pairs_x2<16>(ud, hi, lo);
         tmem_st16(tl + kColUDH + 32 * th, hi);
         tmem_st16(tl + kColUDL + 32 * th, lo);
       }
@@ -955,7 +986,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
       mbar_arrive(&u_conv);
       {
         uint32_t hi[16], lo[16];
-        split_pairs<16>(u, hi, lo);
+        split_pairs_x2<16>(u, hi, lo);
         tmem_st16(tl + kColUH + 32 * th, hi);
         tmem_st16(tl + kColUL + 32 * th, lo);
       }
@@ -993,7 +1024,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
       const uint32_t p_hi = smem_u32(sm + kScOffP);
       for (int c = 0; c < nc; ++c) {
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
-        if (!mbar_wait(&wq_full, c & 1, ab)) break;
+        if (!mbar_wait(&w_full, c & 1, ab)) break;
         if (c > 0 && !mbar_wait(&y_done, (c - 1) & 1, ab)) break;  // U^T P^T of the last chunk read the U columns
         tc_fence_after();
         // the chain's product first: [U2 | U1] = S_hi [W_lo | W_hi], U1 += S_lo W_hi
@@ -1005,7 +1036,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
           umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
         }
         umma_commit(&u_done);
+        umma_commit(&w_free);
         // then the output's: [O1 | O2] = S_hi [gQ_hi | gQ_lo], O1 += S_lo gQ_hi, once o(c-1) has been read
+        if (!mbar_wait(&q_full, c & 1, ab)) break;
         if (c > 0 && !mbar_wait(&o_free, (c - 1) & 1, ab)) break;
         tc_fence_after();
 #pragma unroll
@@ -1014,7 +1047,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
           umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, ks > 0);
           umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, bq, idesc_u2, true);
         }
-        umma_commit(&wq_free);
+        umma_commit(&q_free);
         if (!mbar_wait(&u_conv, c & 1, ab)) break;
         if (!mbar_wait(&k_full, c & 1, ab)) break;
         tc_fence_after();
@@ -1052,28 +1085,37 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
   } else if (warp == kWarpProd) {
     // ------------------------------------------------ bulk-copy producer (lane 0)
     if (lane == 0) {
-      int n_g[2] = {0, 0}, n_wq = 0, n_k = 0, n_p = 0, n_u0 = 0;
-      for (int c = 0; c < nc; ++c) {
+      // Order of need: W, gamma Q, K, P of chunk c (single stages, each refilled as soon as the
+      // product that reads it has completed), then the double-buffered gates and U0 of chunk c + 1.
+      int n_g[2] = {0, 0}, n_u0[2] = {0, 0}, n_w = 0, n_q = 0, n_k = 0, n_p = 0;
+      auto head_blob = [&](int c) {
+        return p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes);
+      };
+      auto load_gates_u0 = [&](int c) -> bool {  // chunk c into stage c & 1
         const int st = c & 1;
-        const long long gc = cb + c;
-        const uint8_t* hb = p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes);
-        const uint8_t* kb = p.ws_k + (gc * p.H_k + kh) * static_cast<long long>(kKBytes);
-        if (c + 2 < nc) {  // two chunks ahead into L2
-          prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
-          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
-        }
-        if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) break;
+        const uint8_t* hb = head_blob(c);
+        if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
         mbar_arrive_expect_tx(&g_full[st], kGateBytes);
         bulk_g2s(sm + kScOffG + st * kGateBytes, hb + kHeadOffGate, kGateBytes, &g_full[st]);
         ++n_g[st];
-        if (c >= 1 && !mbar_wait(&wq_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&wq_full, kWQBytes);
-        bulk_g2s(sm + kScOffWQ, hb + kHeadOffWQ, kWQBytes, &wq_full);
-        ++n_wq;
-        if (c >= 1 && !mbar_wait(&u0_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&u0_full, kU0Bytes);
-        bulk_g2s(sm + kScOffU0, hb + kHeadOffU0, kU0Bytes, &u0_full);
-        ++n_u0;
+        if (c >= 2 && !mbar_wait(&u0_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
+        mbar_arrive_expect_tx(&u0_full[st], kU0Bytes);
+        bulk_g2s(sm + kScOffU0 + st * kU0Bytes, hb + kHeadOffU0, kU0Bytes, &u0_full[st]);
+        ++n_u0[st];
+        return true;
+      };
+      bool ok = nc == 0 || load_gates_u0(0);
+      for (int c = 0; c < nc && ok; ++c) {
+        const uint8_t* hb = head_blob(c);
+        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes);
+        if (c >= 1 && !mbar_wait(&w_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&w_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffWQ, hb + kHeadOffWQ, 2 * kImg64, &w_full);
+        ++n_w;
+        if (c >= 1 && !mbar_wait(&q_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&q_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffWQ + 2 * kImg64, hb + kHeadOffWQ + 2 * kImg64, 2 * kImg64, &q_full);
+        ++n_q;
         if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&k_full, kKBytes);
         bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
@@ -1082,14 +1124,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
         mbar_arrive_expect_tx(&p_full, 2 * kPImg);
         bulk_g2s(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
         ++n_p;
+        if (c + 1 < nc) ok = load_gates_u0(c + 1);
+        if (c + 2 < nc) {  // two chunks ahead into L2, behind this chunk's copies
+          prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
+          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
+        }
       }
       // copies still in flight (only possible after an abort) land before the CTA exits
       int drain_flag = 0;
       Abort drain{nullptr, &drain_flag};
-      for (int b = 0; b < 2; ++b)
+      for (int b = 0; b < 2; ++b) {
         if (n_g[b] > 0) mbar_wait(&g_full[b], (n_g[b] - 1) & 1, drain);
-      if (n_wq > 0) mbar_wait(&wq_full, (n_wq - 1) & 1, drain);
-      if (n_u0 > 0) mbar_wait(&u0_full, (n_u0 - 1) & 1, drain);
+        if (n_u0[b] > 0) mbar_wait(&u0_full[b], (n_u0[b] - 1) & 1, drain);
+      }
+      if (n_w > 0) mbar_wait(&w_full, (n_w - 1) & 1, drain);
+      if (n_q > 0) mbar_wait(&q_full, (n_q - 1) & 1, drain);
       if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
       if (n_p > 0) mbar_wait(&p_full, (n_p - 1) & 1, drain);
     }
@@ -1114,7 +1163,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
     for (int c = 0; c < nc; ++c) {
       const long long tok0 = s + static_cast<long long>(c) * kChunk;
       const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - tok0));
-      // z of the chunk (loaded while the products run)
+      // z of the next chunk into L2 (one 128-byte line per thread), z of this chunk into
+      // registers while the products run
+      if (c + 1 < nc) {
+        const long long r = tok0 + kChunk + (otid >> 1);
+        if (r < e) prefetch_l2_line(p.z + r * p.sz + static_cast<long long>(h) * kD + (otid & 1) * 64);
+      }
       uint4 zr[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -1132,7 +1186,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
           tmem_ld32(tl + kColO + 64 + 32 * cc, o2);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sO[(32 * cc + i) * kD + v] = o1[i] + o2[i];
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = __fadd2_rn(make_float2(o1[i], o1[i + 1]), make_float2(o2[i], o2[i + 1]));
+            sO[(32 * cc + i) * kD + v] = r.x;
+            sO[(32 * cc + i + 1) * kD + v] = r.y;
+          }
         }
         tc_fence_before();
         mbar_arrive(&o_free);
@@ -1155,18 +1213,35 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
         for (int m = 0; m < 8; ++m) inv[m] += __shfl_xor_sync(0xffffffffu, inv[m], sh);
 #pragma unroll
       for (int m = 0; m < 8; ++m) inv[m] = rsqrtf(inv[m] * (1.0f / kD) + 1e-6f);
+      // two tokens per step, so that their exponential / reciprocal chains overlap
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int r = (otid >> 4) + 8 * m;
-        const float4* orow = reinterpret_cast<const float4*>(sO + r * kD + v8);
-        const float4 a0 = orow[0], a1 = orow[1];
-        const float o8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        float z8[8], y8[8];
-        unpack8(zr[m], z8);
+      for (int m = 0; m < 8; m += 2) {
+        float o8[2][8], y8[2][8], z8[2][8];
 #pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) y8[e2] = o8[e2] * inv[m] * w8[e2] * silu_fast(z8[e2]);
-        if (r < L)
-          *reinterpret_cast<uint4*>(p.out + ((tok0 + r) * p.H_v + h) * kD + v8) = pack8(y8);
+        for (int u = 0; u < 2; ++u) {
+          const float4* orow = reinterpret_cast<const float4*>(sO + ((otid >> 4) + 8 * (m + u)) * kD + v8);
+          const float4 a0 = orow[0], a1 = orow[1];
+          o8[u][0] = a0.x; o8[u][1] = a0.y; o8[u][2] = a0.z; o8[u][3] = a0.w;
+          o8[u][4] = a1.x; o8[u][5] = a1.y; o8[u][6] = a1.z; o8[u][7] = a1.w;
+          unpack8(zr[m + u], z8[u]);
+        }
+#pragma unroll
+        for (int e2 = 0; e2 < 8; e2 += 2) {  // ((o inv) w) silu(z), packed in channel pairs
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const float2 a = __fmul2_rn(make_float2(o8[u][e2], o8[u][e2 + 1]), make_float2(inv[m + u], inv[m + u]));
+            const float2 b = __fmul2_rn(a, make_float2(w8[e2], w8[e2 + 1]));
+            const float2 r = __fmul2_rn(b, make_float2(silu_fast(z8[u][e2]), silu_fast(z8[u][e2 + 1])));
+            y8[u][e2] = r.x;
+            y8[u][e2 + 1] = r.y;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = (otid >> 4) + 8 * (m + u);
+          if (r < L)
+            *reinterpret_cast<uint4*>(p.out + ((tok0 + r) * p.H_v + h) * kD + v8) = pack8(y8[u]);
+        }
       }
       named_bar_sync(1, 128);  // sO is rewritten by the next chunk
     }

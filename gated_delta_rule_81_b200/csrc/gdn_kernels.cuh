@@ -19,7 +19,7 @@ using bf16 = __nv_bfloat16;
 //       128 rows (d_k) x 64 tokens, W = T diag(beta gamma) K and gamma Q = diag(gamma) Q;
 //       side by side they form one MN-major operand of N = 256 (or N = 128 from the second)
 //     P hi | P lo: P_ij = e^{G_i - G_j} q_i.k_j for j <= i, row = i, 64 j per row
-//     U0 fp32 [64 tokens][128 d_v]   (U0 = T diag(beta) V)
+//     U0 fp32 [16 token quads][128 d_v][4 tokens]   (U0 = T diag(beta) V)
 //     gates fp32: gamma_i [64], e^{G_C - G_i} [64], gamma_C
 constexpr int kImg64 = 16384;                                // 64 rows x 128 channels (or 128 x 64), bf16
 constexpr int kKBytes = 2 * kImg64;                          // K hi, K lo

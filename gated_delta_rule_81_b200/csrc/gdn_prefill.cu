@@ -755,13 +755,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
           *reinterpret_cast<uint4*>(sQK + 32768 + half_off + off) = hi;
         }
       } else {
-        // U0 [token][d_v] fp32: a warp writes 128 contiguous bytes per token
+        // U0 [token / 4][d_v][4] fp32: a warp writes 512 contiguous bytes per token quad
         tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU), o);
         tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU + 32), o + 32);
         tmem_wait_ld();
-        float* u0 = reinterpret_cast<float*>(hb + kHeadOffU0) + 32 * (warp & 3) + lane;
+        float4* u0 = reinterpret_cast<float4*>(hb + kHeadOffU0) + 32 * (warp & 3) + lane;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) u0[i * kD] = o[i];
+        for (int q4 = 0; q4 < 16; ++q4) u0[q4 * kD] = make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
       }
       fence_proxy_async_smem();
     }
@@ -835,7 +835,7 @@ __host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base
 constexpr int kScOffWQ = 0;                            // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
 constexpr int kScOffK = kScOffWQ + kWQBytes;           // K hi, lo
 constexpr int kScOffP = kScOffK + kKBytes;             // P hi, lo
-constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // 2 stages of U0 fp32 [64][128]
+constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // 2 stages of U0 fp32 [16 token quads][128][4]
 constexpr int kScOffO = kScOffU0 + 2 * kU0Bytes;       // o fp32 [64 tokens][128 d_v] for the token-major epilogue
 constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
@@ -957,13 +957,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
         tmem_ld32(tl + kColU2 + 32 * th, u);
         tmem_ld32(tl + kColU1 + 32 * th, u1);
         tmem_wait_ld();
+        const float4* U0q = reinterpret_cast<const float4*>(U0) + (8 * th) * kD + v;  // [token / 4][d_v][4]
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {  // u = U0 - (U1 + U2), packed in token pairs
-          const float2 acc = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
-          const float2 r = __ffma2_rn(acc, make_float2(-1.f, -1.f),
-                                      make_float2(U0[(32 * th + i) * kD + v], U0[(32 * th + i + 1) * kD + v]));
-          u[i] = r.x;
-          u[i + 1] = r.y;
+        for (int q4 = 0; q4 < 8; ++q4) {  // u = U0 - (U1 + U2), packed in token pairs
+          const float4 u0 = U0q[q4 * kD];
+          const int i = 4 * q4;
+          const float2 a0 = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
+          const float2 a1 = __fadd2_rn(make_float2(u1[i + 2], u1[i + 3]), make_float2(u[i + 2], u[i + 3]));
+          const float2 r0 = __ffma2_rn(a0, make_float2(-1.f, -1.f), make_float2(u0.x, u0.y));
+          const float2 r1 = __ffma2_rn(a1, make_float2(-1.f, -1.f), make_float2(u0.z, u0.w));
+          u[i] = r0.x; u[i + 1] = r0.y; u[i + 2] = r1.x; u[i + 3] = r1.y;
         }
       }
       mbar_arrive(&u0_free[gs]);

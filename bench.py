@@ -301,32 +301,53 @@ def run_e2e_prefill(args, world, rank, dev, case):
             "d2h_bytes_per_step": d2h}
 
 
-def run_decode_ours(args, dev, steps_per_pass=64):
+def run_decode_ours(args, dev, steps_per_pass=64, T=1):
+    """The decode workload (256 sequences, 64 new tokens each) as 64 / T launches of
+    T tokens per sequence.  T = 1 goes through gdn_decode_step; T > 1 through
+    gdn_decode_multi with the states in a pool addressed by a permuted slot list."""
     from gated_delta_rule_81_b200 import gdn
 
     case = gin.decode_case(4)
     N = case["N"]
     state = case["state"].to(dev)
     conv = case["conv_state"].to(dev)
-    tok = {k: case["tok"][k].to(dev) for k in ("q", "k", "v", "a", "b", "z")}
+    tok = case["tok"]
     w = {k: v.to(dev) for k, v in case["w"].items()}
-    ins = [gdn.make_inputs(*(tok[k][i * N:(i + 1) * N] for k in ("q", "k", "v", "a", "b", "z")), w["conv_w"],
-                           w["A_log"], w["norm_w"]) for i in range(steps_per_pass)]
-    out = torch.empty(N, 48, 128, dtype=torch.bfloat16, device=dev)
+    launches = steps_per_pass // T
+    if T == 1:
+        dtok = {k: tok[k].to(dev) for k in ("q", "k", "v", "a", "b", "z")}
+        ins = [gdn.make_inputs(*(dtok[k][i * N:(i + 1) * N] for k in ("q", "k", "v", "a", "b", "z")),
+                               w["conv_w"], w["A_log"], w["norm_w"]) for i in range(launches)]
+    else:
+        # launch i takes steps i*T .. i*T+T-1 of every sequence, sequence-major
+        idx = torch.tensor([(i * T + t) * N + n for i in range(launches) for n in range(N) for t in range(T)])
+        dtok = {k: tok[k][idx].to(dev) for k in ("q", "k", "v", "a", "b", "z")}
+        ins = [gdn.make_inputs(*(dtok[k][i * N * T:(i + 1) * N * T] for k in ("q", "k", "v", "a", "b", "z")),
+                               w["conv_w"], w["A_log"], w["norm_w"]) for i in range(launches)]
+        slots = torch.randperm(N, generator=torch.Generator().manual_seed(5)).to(torch.int32).to(dev)
+    out = torch.empty(N * T, 48, 128, dtype=torch.bfloat16, device=dev)
+
+    def launch(i):
+        if T == 1:
+            gdn.decode_step(ins[i], N, state, conv, out=out)
+        else:
+            gdn.decode_multi(ins[i], N, T, state, conv, state_slot=slots, out=out)
+
     stream = torch.cuda.current_stream()
     for i in range(3):
-        gdn.decode_step(ins[i], N, state, conv, out=out)
+        launch(i % launches)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(steps_per_pass):
-        gdn.decode_step(ins[i], N, state, conv, out=out)
+    for i in range(launches):
+        launch(i)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    per_launch_s = ms / 1e3 / steps_per_pass
+    per_launch_s = ms / 1e3 / launches
     gbs = N * DECODE_BYTES_PER_SEQ / per_launch_s / 1e9
-    return {"ms_per_launch": ms / steps_per_pass, "gbs": gbs, "launches": steps_per_pass}
+    return {"ms_per_launch": ms / launches, "gbs": gbs, "launches": launches, "T": T,
+            "tokens_per_s": N * T / per_launch_s}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
@@ -393,6 +414,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode"], default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
+    ap.add_argument("--decode-tokens", type=int, default=1,
+                    help="decode workload: new tokens per sequence per launch (1 .. 8)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
@@ -412,16 +435,19 @@ def main():
     pk = peaks()
 
     if args.workload == "decode":
-        d = run_decode_ours(args, dev)
+        d = run_decode_ours(args, dev, T=args.decode_tokens)
         if rank == 0:
             print(json.dumps({"metric": "decode state GB/s", "value": d["gbs"], "unit": "GB/s", "n_gpus": world,
-                              "steps": 64, "warmup": 3, "ms_per_step": d["ms_per_launch"], "higher_is_better": True,
-                              "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                              "config": {"workload": gin.CONFIGS[4]["name"]},
+                              "steps": d["launches"], "warmup": 3, "ms_per_step": d["ms_per_launch"],
+                              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                              "data": "synthetic",
+                              "config": {"workload": gin.CONFIGS[4]["name"], "tokens_per_launch": d["T"],
+                                         "state_slots": "permuted pool" if d["T"] > 1 else "slot n",
+                                         "tokens_per_s": d["tokens_per_s"]},
                               "roofline": {"bound": "hbm", "achieved": d["gbs"], "peak": pk["hbm_gbs"],
                                            "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"],
-                                           "traffic": decode_traffic()},
-                              "gpu_launches": 64}), flush=True)
+                                           "traffic": decode_traffic() if d["T"] == 1 else None},
+                              "gpu_launches": d["launches"]}), flush=True)
         return 0
     cfg_id = WORKLOADS[args.workload]
     res = run_prefill_ours(args, world, rank, dev, pk, cfg_id)

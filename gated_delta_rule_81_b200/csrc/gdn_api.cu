@@ -155,18 +155,21 @@ gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens
                         out, workspace, workspace_bytes, err, stream);
 }
 
-gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out, int* err,
-                           void* stream) {
-  if (N < 0) return GDN_ERR_INVALID_ARG;
-  gdn_status st = check_inputs(in, N);
+gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,
+                            const int* state_slot, int n_slots, void* out, int* err, void* stream) {
+  if (N < 0 || T < 1 || T > gdn::kMaxDecodeTokens || n_slots < 0) return GDN_ERR_INVALID_ARG;
+  const long long T_tot = static_cast<long long>(N) * T;
+  gdn_status st = check_inputs(in, T_tot);
   if (st != GDN_OK || N == 0) return st;
   if (!state || !conv_state || !out) return GDN_ERR_INVALID_ARG;
+  if (!state_slot && n_slots < N) return GDN_ERR_INVALID_ARG;  // slot n for sequence n
   if (!aligned16(state) || !aligned16(conv_state) || !aligned16(out)) return GDN_ERR_MISALIGNED;
-  if ((st = check_out_alias(in, N, out)) != GDN_OK) return st;
+  if (reinterpret_cast<uintptr_t>(state_slot) & 3u) return GDN_ERR_MISALIGNED;
+  if ((st = check_out_alias(in, T_tot, out)) != GDN_OK) return st;
   const long long C_conv = static_cast<long long>(2 * in->H_k + in->H_v) * GDN_HEAD_DIM;
-  const size_t state_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
-  const size_t conv_bytes = static_cast<size_t>(N) * 3 * C_conv * sizeof(bf16);
-  const size_t out_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
+  const size_t state_bytes = static_cast<size_t>(n_slots) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(n_slots) * 3 * C_conv * sizeof(bf16);
+  const size_t out_bytes = static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
   if (overlap(state, state_bytes, conv_state, conv_bytes) || overlap(state, state_bytes, out, out_bytes) ||
       overlap(conv_state, conv_bytes, out, out_bytes))
     return GDN_ERR_ALIAS;
@@ -186,12 +189,20 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
   p.H_k = in->H_k;
   p.H_v = in->H_v;
   p.N = N;
+  p.T = T;
+  p.state_slot = state_slot;
+  p.n_slots = n_slots;
   p.state = state;
   p.conv_state = static_cast<bf16*>(conv_state);
   p.out = static_cast<bf16*>(out);
   p.err = err;
   return gdn::launch_decode(p, static_cast<cudaStream_t>(stream), in->events) == cudaSuccess ? GDN_OK
                                                                                          : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out, int* err,
+                           void* stream) {
+  return gdn_decode_multi(in, N, 1, state, conv_state, nullptr, N, out, err, stream);
 }
 
 const char* gdn_status_string(gdn_status status) {

@@ -34,17 +34,23 @@ constexpr int kGateBytes = 1024;
 constexpr int kHeadBytes = kHeadOffGate + kGateBytes;        // 115712
 constexpr int kWsHeader = 1024;                              // error/consistency word
 
+constexpr int kMaxDecodeTokens = 8;   // new tokens per sequence in one decode call
+constexpr int kDevErrBadSlot = 8;      // a state_slot entry outside [0, n_slots)
+
 struct DecodeParams {
-  const bf16 *q, *k, *v, *a, *b, *z;
-  long long sq, sk, sv, sz, sa, sb;  // token strides (elements)
+  const bf16 *q, *k, *v, *a, *b, *z;  // token n * T + t is new token t of sequence n
+  long long sq, sk, sv, sz, sa, sb;   // token strides (elements)
   const bf16* conv_w;
   const float* A_log;
   const bf16* norm_w;
   float scale;
   int H_k, H_v, N;
-  float* state;     // [N][H_v][128][128], updated in place
-  bf16* conv_state; // [N][3][C_conv], updated in place
-  bf16* out;        // [N][H_v][128]
+  int T;                  // new tokens per sequence, 1 .. kMaxDecodeTokens
+  const int* state_slot;  // [N] slot of each sequence in the state pools, or null (slot n)
+  int n_slots;            // slots in the pools
+  float* state;           // [n_slots][H_v][128][128], updated in place
+  bf16* conv_state;       // [n_slots][3][C_conv], updated in place
+  bf16* out;              // [N * T][H_v][128]
   int* err;
 };
 

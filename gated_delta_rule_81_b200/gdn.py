@@ -45,7 +45,8 @@ _lib = None
 _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
-           "gdn_status_string")
+           "gdn_decode_multi", "gdn_status_string")
+MAX_DECODE_TOKENS = 8
 
 
 def load(path: str | None = None):
@@ -66,6 +67,8 @@ def load(path: str | None = None):
     lib.gdn_prefill_varlen.restype = _i
     lib.gdn_decode_step.argtypes = [P, _i, _vp, _vp, _vp, _vp, _vp]
     lib.gdn_decode_step.restype = _i
+    lib.gdn_decode_multi.argtypes = [P, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]
+    lib.gdn_decode_multi.restype = _i
     lib.gdn_status_string.argtypes = [_i]
     lib.gdn_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -195,6 +198,22 @@ def decode_step(inp: GdnInputs, N: int, state, conv_state, out=None, err=None):
     _check(lib.gdn_decode_step(ctypes.byref(inp), N, _ptr(state), _ptr(conv_state), _ptr(out), _ptr(err),
                                _stream()),
            "gdn_decode_step")
+    return out
+
+
+def decode_multi(inp: GdnInputs, N: int, T: int, state, conv_state, state_slot=None, out=None, err=None):
+    """gdn_decode_multi: T new tokens per sequence (token n*T + t), states in pool slots.
+
+    state [n_slots][H_v][128][128] fp32 and conv_state [n_slots][3][C_conv] bf16 are
+    updated in place; state_slot is a device int32 [N] (None: sequence n uses slot n).
+    Returns out [N*T][H_v][128] bf16."""
+    lib = load()
+    if out is None:
+        out = torch.empty(N * T, inp.H_v, HEAD_DIM, dtype=torch.bfloat16, device=state.device)
+    n_slots = state.shape[0]
+    _check(lib.gdn_decode_multi(ctypes.byref(inp), N, T, _ptr(state), _ptr(conv_state), _ptr(state_slot), n_slots,
+                                _ptr(out), _ptr(err), _stream()),
+           "gdn_decode_multi")
     return out
 
 

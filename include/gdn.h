@@ -37,7 +37,8 @@
  *     Conv state: bf16 [N][3][C_conv], the 3 most recent raw tokens, oldest first.
  *   - `err` (nullable) is a device int the kernels OR error bits into
  *     (1 = a bounded wait timed out, 2 = cluster exchange failed,
- *     4 = cu_seqlens on the device disagreed with cu_seqlens_host).  It is
+ *     4 = cu_seqlens on the device disagreed with cu_seqlens_host, 8 = a decode
+ *     state_slot outside the pool).  It is
  *     never cleared by the library.  Read it after synchronising.
  */
 #ifndef GDN_H_
@@ -136,6 +137,26 @@ gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens
  */
 gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out,
                            int* err, void* stream);
+
+/*
+ * T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N sequences in one call
+ * (decode with several tokens per step, e.g. verifying drafted tokens), with
+ * the states held in slots of a state pool.  Token n * T + t of the inputs is
+ * new token t of sequence n (T_tot = N * T); out is bf16 [N * T][H_v][128].
+ * The tokens of a sequence are applied in order exactly as T gdn_decode_step
+ * calls would apply them (same arithmetic: results are bitwise equal), but each
+ * state row is read from HBM once and written once for all T tokens.
+ *   state       fp32 [n_slots][H_v][128][128], updated in place
+ *   conv_state  bf16 [n_slots][3][C_conv], updated in place (the last 3 raw tokens)
+ *   state_slot  device int32 [N]: the slot of sequence n, or NULL for slot n
+ *               (then n_slots >= N).  Slots must be distinct within a call.  A slot
+ *               outside [0, n_slots) leaves that sequence untouched and sets bit 8
+ *               of *err.
+ * Inputs must not overlap state, conv_state or out.
+ */
+#define GDN_MAX_DECODE_TOKENS 8
+gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,
+                            const int* state_slot, int n_slots, void* out, int* err, void* stream);
 
 /*
  * Allocation-free prefill.  The pages have no counterpart to this call; it

@@ -111,3 +111,20 @@ def test_decode_rejects_aliasing(lib):
     assert lib.gdn_decode_step(ctypes.byref(s), 4, 0x7000000, 0x7000000 + 64, 0x900000, None, None) == 4
     assert lib.gdn_decode_step(ctypes.byref(s), 4, None, 0x7000000, 0x900000, None, None) == 1
     assert lib.gdn_decode_step(ctypes.byref(s), 0, None, None, None, None, None) == 0
+
+
+def test_decode_multi_rejects_bad_arguments(lib):
+    s = fake_inputs()
+    st, cv, out = 0x7000000, 0x5000000, 0x900000
+    # T outside 1 .. GDN_MAX_DECODE_TOKENS, negative N or pool size
+    for T in (0, gdn.MAX_DECODE_TOKENS + 1):
+        assert lib.gdn_decode_multi(ctypes.byref(s), 2, T, st, cv, None, 2, out, None, None) == 1
+    assert lib.gdn_decode_multi(ctypes.byref(s), -1, 1, st, cv, None, 2, out, None, None) == 1
+    assert lib.gdn_decode_multi(ctypes.byref(s), 2, 1, st, cv, 0x3000000, -1, out, None, None) == 1
+    # without slots sequence n uses slot n, so the pool must hold N states
+    assert lib.gdn_decode_multi(ctypes.byref(s), 3, 1, st, cv, None, 2, out, None, None) == 1
+    # a misaligned slot array, a state overlapping the output
+    assert lib.gdn_decode_multi(ctypes.byref(s), 2, 2, st, cv, 0x3000002, 4, out, None, None) == 3
+    assert lib.gdn_decode_multi(ctypes.byref(s), 2, 2, st, cv, None, 2, st + 1024, None, None) == 4
+    # N = 0 is a no-op
+    assert lib.gdn_decode_multi(ctypes.byref(s), 0, 4, None, None, None, 0, None, None, None) == 0

@@ -55,9 +55,9 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {"scan": {"bytes": 442649856 + 44844288, "sha": "f74aec2f444d2102"},   # ncu, T=4096 layer
-           "prep": {"bytes": 100750336 + 339516416, "sha": "f74aec2f444d2102"}}
-DECODE_TRAFFIC = {"bytes": 829621504 + 767561728, "sha": "6ad12188ad3a4536"}  # ncu, one step of 256 sequences
+TRAFFIC = {"scan": {"bytes": 442659072 + 44793088, "sha": "daba6480c7058e35"},   # ncu, T=4096 layer
+           "prep": {"bytes": 103497984 + 341519104, "sha": "daba6480c7058e35"}}
+DECODE_TRAFFIC = {"bytes": 829675264 + 766249984, "sha": "852a2d42cccfe44d"}  # ncu, one step of 256 sequences
 
 
 def src_sha(name):

@@ -31,6 +31,7 @@ constexpr int kHeadOffU0 = kHeadOffP + 2 * kPImg;
 constexpr int kU0Bytes = 64 * 128 * 4;
 constexpr int kHeadOffGate = kHeadOffU0 + kU0Bytes;
 constexpr int kGateBytes = 1024;
+constexpr int kReadyFlagWord = 255;  // word of the gate area a fused prefill launch uses as a ready flag
 constexpr int kHeadBytes = kHeadOffGate + kGateBytes;        // 115712
 constexpr int kWsHeader = 1024;                              // error/consistency word
 
@@ -78,6 +79,9 @@ struct PrefillParams {
   bf16* conv_out;         // [N][3][C_conv] or null
   bf16* out;              // [T_tot][H_v][128]
   int* err;
+  int allow_fused;        // 0 = two launches, 1 = automatic, 2 = one fused launch whenever possible
+  int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, scan CTAs first, prep items
+                          // published by ready flags; 0 = prep kernel, then scan kernel
 };
 
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)

@@ -193,8 +193,8 @@ __host__ __device__ constexpr int prep_smem_bytes(int G) { return kPrepOffW + (2
 static_assert(2 * kImg64 <= kPrepRBytes, "the v_hat and (gamma Q)^T images must fit region R");
 static_assert((kChunk + kTaps - 1) * kRawStride <= kPrepRBytes, "the raw q | k rows must fit region R");
 // tensor memory columns (256 per CTA, two CTAs per SM)
-constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns);
-                                      // then q^T (lane = d_k, column = token)
+constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns)
+constexpr uint32_t kPrepColQT = 64;   // q^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColW = 128;   // W^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColU = 192;   // U0^T (lane = d_v, column = token)
 
@@ -287,7 +287,7 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
 //   M = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II M
 // with 16x16 blocks; each thread computes four adjacent columns of one row.
 template <int d>
-__device__ __forceinline__ void solve_level(const float* sA, float* sT, float* sM, int tid) {
+__device__ __forceinline__ void solve_level(const float* sA, float* sT, float* sM, int tid, int bar_id) {
   constexpr int nb = 4 - d;
   if (tid < nb * 64) {
     const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
@@ -305,7 +305,7 @@ __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* s
     }
     *reinterpret_cast<float4*>(sM + (J << 8) + (ii << 4) + j4) = acc;
   }
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
   if (tid < nb * 64) {
     const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
     const float* trow = sT + (16 * I + ii) * kLdT + 16 * I;
@@ -322,13 +322,13 @@ __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* s
     }
     *reinterpret_cast<float4*>(sT + (16 * I + ii) * kLdT + 16 * J + j4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
   }
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
 }
 
 // T = (I + A)^{-1} for a 64x64 strictly-lower A (fp32, shared memory), by 16x16
 // blocks: diagonal blocks by forward substitution, then the three block
 // diagonals below.  All 256 threads.
-__device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid) {
+__device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid, int bar_id) {
   if (tid < 64) {
     const int blk = tid >> 4, col = tid & 15;
     float x[16];
@@ -346,10 +346,10 @@ __device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid)
       sT[(16 * blk + r) * kLdT + 16 * blk + col] = x[r];
     }
   }
-  __syncthreads();
-  solve_level<1>(sA, sT, sM, tid);
-  solve_level<2>(sA, sT, sM, tid);
-  solve_level<3>(sA, sT, sM, tid);
+  named_bar_sync(bar_id, kPrepThreads);
+  solve_level<1>(sA, sT, sM, tid, bar_id);
+  solve_level<2>(sA, sT, sM, tid, bar_id);
+  solve_level<3>(sA, sT, sM, tid, bar_id);
 }
 
 // D (+)= A B^T with both operands as hi/lo pairs: A_hi B_hi + A_hi B_lo + A_lo B_hi
@@ -379,10 +379,25 @@ __device__ __forceinline__ void conv32_rows(const uint8_t* raw, int i, int off, 
 // One CTA per (chunk, key head).  Writes the chunk's K image for the key head
 // and, for each of its value heads, W^T, (gamma Q)^T, P, U0 and the gate vectors.
 // The operand images leave shared memory as bulk stores.
-__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) {
-  if (p.cu && *p.ws_flag) return;
-  extern __shared__ uint8_t prep_smem_raw[];
-  uint8_t* sm = align1024(prep_smem_raw);
+// Word of the gate area of (chunk gc, value head h) that the fused launch uses as the
+// ready flag of the chunk's operands (the gate vectors occupy words 0 .. 128).
+__device__ __forceinline__ int* ready_flag(const PrefillParams& p, long long gc, int h) {
+  return reinterpret_cast<int*>(p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate) +
+         kReadyFlagWord;
+}
+
+// Prep of one (chunk gc, key head kh) by 256 threads: the CTA's threads 256 half .. 256 half + 255,
+// shared memory at sm (1024-aligned), tensor-memory columns tbase .. tbase + 255 (allocated by
+// the caller), mbarriers bar[4].  Block-wide steps use named barrier 2 + half over the 256 threads.
+// `k` counts the items these threads ran before with the same mbarriers (initialised at k = 0;
+// every wait takes its phase parity from k).  When go_flag is given, it is set once the first
+// value head is done (or the item ends), which lets the other half of a CTA start out of phase.
+// Writes the chunk's K image for the key head and, for each of its value heads, W^T,
+// (gamma Q)^T, P, U0 and the gate vectors; the operand images leave shared memory as bulk
+// stores.  In a fused launch it then publishes the chunk through the value heads' ready flags.
+__device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, int kh, int half, uint8_t* sm,
+                                          uint32_t tbase, uint64_t* bar, int* abort_s, int k, int* go_flag) {
+  const int bar_id = 2 + half;
   uint8_t* sQK = sm + kPrepOffQK;
   uint8_t* sR = sm + kPrepOffR;
   float* sA = reinterpret_cast<float*>(sm + kPrepOffA);
@@ -392,13 +407,9 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
   float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
   uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2 + G) * 64] channel pairs: q | k | v heads
-  __shared__ uint64_t bar[4];  // [Q;K] K^T, W / U0 (per head), drain, q^T
-  __shared__ uint32_t tmem_base_s;
-  __shared__ int abort_s;
+  // bar: [Q;K] K^T, W / U0 (per head), drain, q^T
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long gc = blockIdx.x;
-  const int kh = blockIdx.y;
+  const int tid = threadIdx.x & (kPrepThreads - 1), warp = tid >> 5, lane = tid & 31;
   const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k;
   const long long C_conv = static_cast<long long>(2 * H_k + H_v) * kD;
 
@@ -419,14 +430,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - t0));
   const int nrows = L + kTaps - 1;  // raw rows of tokens t0 - 3 .. t0 + L - 1
 
-  Abort ab{p.err, &abort_s};
-  if (tid == 0) {
-    abort_s = 0;
+  Abort ab{p.err, abort_s};
+  const uint32_t ph = k & 1;  // phase parity of the once-per-item barriers
+  if (tid == 0 && k == 0) {
+    *abort_s = 0;
     for (int b = 0; b < 4; ++b) mbar_init(&bar[b], 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc<256>(&tmem_base_s);
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
 
   // ---- raw q | k rows into region R: 16-byte asynchronous copies by all threads (a warp
   // moves one 512-byte row per instruction); rows before the sequence start come from
@@ -480,16 +491,16 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       sB[j * 64 + i] = beta;
     }
   }
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
   for (int x = tid; x < G * 32; x += kPrepThreads) {
     const int j = x >> 5, i = 32 + (x & 31);
     sG[j * 64 + i] += sG[j * 64 + 31];
   }
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
   for (int x = tid; x < G * 64; x += kPrepThreads) sGam[x] = expf(sG[x]);
   // ---- front end of q and k from the staged rows: token i, channels 32*qq .. 32*qq+31
   cp_async_wait_all();
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
   {
     const int i = tid >> 2, qq = tid & 3;
     const bool valid = i < L;
@@ -521,9 +532,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   }
   fence_proxy_async_smem();
   tc_fence_before();
-  __syncthreads();
+  named_bar_sync(bar_id, kPrepThreads);
   tc_fence_after();
-  const uint32_t tbase = tmem_base_s;
 
   // ---- the K image to the workspace (the K rows of the four K-block halves), and
   // [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
@@ -558,7 +568,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       val = expf(Glast);
     }
     float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate);
-    gdst[k2] = val;
+    if (k2 != kReadyFlagWord) gdst[k2] = val;
   }
 
   // identity B image for the q^T transpose, in region R (the raw rows are dead)
@@ -580,21 +590,14 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   const int cbase = 32 * (warp >> 2);
   const bool isQ = row < 64;
   const int ri = row & 63;
-  float acc[32];
-  if (mbar_wait_warp(&bar[0], 0, ab)) {
-    tc_fence_after();
-    tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + cbase), acc);
-    tmem_wait_ld();
-  } else {
-#pragma unroll
-    for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
-  }
+  // (the [Q;K] K^T rows stay in tensor memory and are read again for each value head)
+  const bool qk_ok = mbar_wait_warp(&bar[0], ph, ab);
 
-  // ---- q^T (lane = d_k, column = token) into TMEM columns 0..63, which the [Q;K] K^T
-  // product no longer needs: Q_hi^T I + Q_lo^T I with an identity B, exact in fp32
+  // ---- q^T (lane = d_k, column = token) into TMEM columns 64..127: Q_hi^T I + Q_lo^T I
+  // with an identity B, exact in fp32
   fence_proxy_async_smem();
   tc_fence_before();
-  __syncthreads();  // the identity is complete; acc has been read
+  named_bar_sync(bar_id, kPrepThreads);  // the identity is complete
   tc_fence_after();
   if (tid == 0) {
     const uint32_t qk = smem_u32(sQK), id = smem_u32(sR);
@@ -602,20 +605,28 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
-      umma_bf16(tbase + kPrepColQK, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
-      umma_bf16(tbase + kPrepColQK, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
+      umma_bf16(tbase + kPrepColQT, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
+      umma_bf16(tbase + kPrepColQT, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
     }
     umma_commit(&bar[3]);
   }
   __syncwarp();
-  mbar_wait_warp(&bar[3], 0, ab);
+  mbar_wait_warp(&bar[3], ph, ab);
   tc_fence_after();
-  __syncthreads();  // Q and the identity are dead: the Q pieces and region R are scratch from here
+  named_bar_sync(bar_id, kPrepThreads);  // Q and the identity are dead: the Q pieces and region R are scratch from here
 
   for (int j = 0; j < G; ++j) {
     const int h = kh * G + j;
     uint8_t* hb = p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes);
     const float Gi = sG[j * 64 + ri];
+    float acc[32];
+    if (qk_ok) {
+      tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + cbase), acc);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) acc[e2] = 0.f;
+    }
     if (!isQ) {
       const float bi = sB[j * 64 + ri];
 #pragma unroll
@@ -642,15 +653,15 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       }
       fence_proxy_async_smem();
     }
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     if (tid == 0) {
       bulk_s2g(hb + kHeadOffP, sQK, kPImg);
       bulk_s2g(hb + kHeadOffP + kPImg, sQK + 32768, kPImg);
       bulk_commit();
     }
-    solve_unit_lower(sA, sT, sM, tid);
+    solve_unit_lower(sA, sT, sM, tid, bar_id);
     if (tid == 0) bulk_wait_read<0>();  // P has left the Q pieces
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     // B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
     for (int x = tid; x < 64 * 8; x += kPrepThreads) {
       const int r = x >> 3, cc = x & 7;
@@ -671,7 +682,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       *reinterpret_cast<uint4*>(sQK + kPrepOffBUhi + off) = hi;
       *reinterpret_cast<uint4*>(sQK + kPrepOffBUlo + off) = lo;
     }
-    __syncthreads();  // T is dead: region R takes the v_hat image
+    named_bar_sync(bar_id, kPrepThreads);  // T is dead: region R takes the v_hat image
     {
       // v_hat of value head h: token i, channels 32*qq .. 32*qq+31, as the MN-major image
       const int i = tid >> 2, qq = tid & 3;
@@ -694,7 +705,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
       // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
@@ -717,13 +728,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       umma_commit(&bar[1]);
     }
     __syncwarp();
-    if (mbar_wait_warp(&bar[1], j & 1, ab)) {
+    if (mbar_wait_warp(&bar[1], (k * G + j) & 1, ab)) {
       tc_fence_after();
       {
         // (gamma Q)^T row d_k = lane, tokens 32*(warp/4) .. +31: staged in region R, hi then lo
         const int kr = 32 * (warp & 3) + lane, half = warp >> 2;
         float qg[32];
-        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQK + 32 * half), qg);
+        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQT + 32 * half), qg);
         tmem_wait_ld();
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) {
@@ -766,7 +777,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
       uint8_t* wq = hb + kHeadOffWQ;  // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
@@ -778,20 +789,48 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
       bulk_commit();
       bulk_wait_read<0>();  // the staging areas are rewritten by the next value head
     }
-    __syncthreads();
+    named_bar_sync(bar_id, kPrepThreads);
+    if (go_flag && tid == 0) *reinterpret_cast<volatile int*>(go_flag) = 1;
   }
+  if (go_flag && tid == 0) *reinterpret_cast<volatile int*>(go_flag) = 1;
 
   // drain: every MMA this CTA issued and every bulk store has completed
   if (tid == 0) {
     umma_commit(&bar[2]);
     int drain_flag = 0;
     Abort drain{nullptr, &drain_flag};
-    mbar_wait(&bar[2], 0, drain);
+    mbar_wait(&bar[2], ph, drain);
     bulk_wait<0>();
   }
+  if (p.fused_scan_ctas > 0) {
+    // publish: every store of this chunk (bulk images drained above, U0 and gate vectors by
+    // all threads) is visible before the value heads' ready flags
+    __threadfence();
+    named_bar_sync(bar_id, kPrepThreads);
+    if (tid == 0) {
+      fence_proxy_async_global();
+      __threadfence();
+      for (int j = 0; j < G; ++j) st_release_gpu(ready_flag(p, gc, kh * G + j), 1);
+    }
+  }
+  tc_fence_before();
+  named_bar_sync(bar_id, kPrepThreads);
+}
+
+
+__global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) {
+  if (p.cu && *p.ws_flag) return;
+  extern __shared__ uint8_t prep_smem_raw[];
+  __shared__ uint64_t bar[4];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  if (threadIdx.x < 32) tmem_alloc<256>(&tmem_base_s);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc<256>(tbase);
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+  prep_body(p, blockIdx.x, blockIdx.y, 0, align1024(prep_smem_raw), tbase, bar, &abort_s, 0, nullptr);
+  if (threadIdx.x < 32) tmem_dealloc<256>(tbase);  // prep_body ends with a barrier after its last use
 }
 
 // ============================================================ scan kernel
@@ -813,6 +852,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // lane 0 issues the bulk copies (W, gamma Q, K, P single-buffered, gates and U0 double-buffered).
 
 constexpr int kScanThreads = 448;
+constexpr int kScanBar = 15;  // named barrier of the scan's CTA-wide steps
 constexpr int kWarpIssue = 12, kWarpProd = 13;
 // tensor memory columns (512 allocated)
 constexpr uint32_t kColS = 0;      // S fp32, 128 columns (d_k)
@@ -840,10 +880,10 @@ constexpr int kScOffO = kScOffU0 + 2 * kU0Bytes;       // o fp32 [64 tokens][128
 constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 
-__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) {
-  if (p.cu && *p.ws_flag) return;
-  extern __shared__ uint8_t scan_smem_raw[];
-  uint8_t* sm = align1024(scan_smem_raw);
+// The scan of one (sequence, value head) (`blk` = sequence rank * H_v + value head) by the
+// CTA's first 448 threads, with shared memory at sm (1024-aligned, kScSmem - 1024 bytes).
+// CTA-wide steps use named barrier kScanBar over those threads.
+__device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8_t* sm) {
   __shared__ uint64_t g_full[2], g_free[2];
   __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, u0_full[2], u0_free[2];
   __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
@@ -851,7 +891,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
   __shared__ int abort_s;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_rank = blockIdx.x / p.H_v, h = blockIdx.x % p.H_v;
+  const int n_rank = blk / p.H_v, h = blk % p.H_v;
   const int n = (p.seq_order && p.N <= kMaxOrdered) ? p.seq_order[n_rank] : n_rank;
   const int G = p.H_v / p.H_k, kh = h / G;
   const long long s = seq_start(p, n), e = seq_start(p, n + 1);
@@ -887,7 +927,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
   }
   if (warp == kWarpIssue) tmem_alloc<512>(&tmem_base_s);
   tc_fence_before();
-  __syncthreads();
+  named_bar_sync(kScanBar, kScanThreads);
   tc_fence_after();
   const uint32_t tbase = tmem_base_s;
 
@@ -1097,6 +1137,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
       auto load_gates_u0 = [&](int c) -> bool {  // chunk c into stage c & 1
         const int st = c & 1;
         const uint8_t* hb = head_blob(c);
+        // fused launch: chunk c's operands (read from here on) are published by its prep
+        if (p.fused_scan_ctas > 0 && !flag_wait(ready_flag(p, cb + c, h), ab, kBackoffNs)) return false;
         if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
         mbar_arrive_expect_tx(&g_full[st], kGateBytes);
         bulk_g2s(sm + kScOffG + st * kGateBytes, hb + kHeadOffGate, kGateBytes, &g_full[st]);
@@ -1251,8 +1293,109 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) 
   }
 
   tc_fence_before();
-  __syncthreads();
+  named_bar_sync(kScanBar, kScanThreads);
   if (warp == kWarpIssue) tmem_dealloc<512>(tbase);
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) {
+  if (p.cu && *p.ws_flag) return;
+  extern __shared__ uint8_t scan_smem_raw[];
+  scan_body(p, blockIdx.x, align1024(scan_smem_raw));
+}
+
+// ------------------------------------------------------------ fused launch
+//
+// When the scan has few (sequence, value head) CTAs (one long sequence: 48 at 16/48 heads),
+// its chain occupies a third of the SMs and the chunk-parallel prep would otherwise run
+// first, alone.  One launch then carries both: CTAs 0 .. fused_scan_ctas - 1 run the scan
+// (448 of their 512 threads), every later CTA runs two prep items, one per 256-thread half,
+// with its own 1024-aligned shared-memory half and 256 of the CTA's 512 tensor-memory
+// columns.  Prep items go chunk-major (item = chunk * H_k + key head), so chunks become
+// ready in order; the scan's producer waits (bounded) on a chunk's ready flag before its
+// first read of that chunk.  No prep CTA waits for anything, and the scan CTAs are at most
+// half of the SMs, so the prep always has SMs to run on, in any dispatch order.
+constexpr int kFusedThreads = 2 * kPrepThreads;
+constexpr int kMaxFusedScanFraction = 2;  // scan CTAs <= SMs / 2
+constexpr int kMinFusedItemsPerSm = 8;    // automatic plan: fuse only with >= 8 prep items per prep SM
+
+__host__ __device__ constexpr int prep_half_bytes(int G) { return (prep_smem_bytes(G) - 1024 + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr int fused_smem_bytes(int G) {
+  return 2 * prep_half_bytes(G) + 1024 > kScSmem ? 2 * prep_half_bytes(G) + 1024 : kScSmem;
+}
+
+__global__ void __launch_bounds__(kFusedThreads, 1) prefill_fused_kernel(PrefillParams p) {
+  if (p.cu && *p.ws_flag) return;
+  extern __shared__ uint8_t fused_smem_raw[];
+  uint8_t* sm = align1024(fused_smem_raw);
+  if (static_cast<int>(blockIdx.x) < p.fused_scan_ctas) {
+    if (threadIdx.x < kScanThreads) scan_body(p, blockIdx.x, sm);
+    return;
+  }
+  // prep CTAs: each half is a worker that takes the next item (chunk-major) from a counter in
+  // the workspace header until none is left
+  __shared__ uint64_t bar[2][4];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s[2];
+  __shared__ int go_s;
+  __shared__ long long item_s[2];
+  const int half = threadIdx.x / kPrepThreads, htid = threadIdx.x & (kPrepThreads - 1);
+  const long long n_items = p.n_chunks * p.H_k;
+  unsigned long long* counter = reinterpret_cast<unsigned long long*>(p.ws_flag) + 1;
+  if (threadIdx.x == 0) go_s = 0;
+  if (threadIdx.x < 32) tmem_alloc<512>(&tmem_base_s);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s + 256u * half;
+  uint8_t* smh = sm + half * prep_half_bytes(p.H_v / p.H_k);
+  if (half == 1 && htid == 0) {
+    // start once half 0 is through its first value head (or found nothing to do): the two
+    // halves then reach their latency-bound steps at different times
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile int*>(&go_s) == 0 && clock64() - t0 < kWaitLimitCycles) __nanosleep(256);
+  }
+  for (int k = 0;; ++k) {
+    if (htid == 0) item_s[half] = static_cast<long long>(atomicAdd(counter, 1ull));
+    named_bar_sync(2 + half, kPrepThreads);
+    const long long item = item_s[half];
+    if (item >= n_items) {
+      if (half == 0 && htid == 0) *reinterpret_cast<volatile int*>(&go_s) = 1;
+      break;
+    }
+    prep_body(p, item / p.H_k, static_cast<int>(item % p.H_k), half, smh, tbase, bar[half], &abort_s[half], k,
+              half == 0 && k == 0 ? &go_s : nullptr);
+    if (*reinterpret_cast<volatile int*>(&abort_s[half])) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) tmem_dealloc<512>(tmem_base_s);
+}
+
+// clears the ready flags of every (chunk, value head) before a fused launch
+// (and the prep work counter in the workspace header)
+__global__ void ready_flags_reset_kernel(PrefillParams p) {
+  const long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (x < p.n_chunks * p.H_v) *ready_flag(p, x / p.H_v, static_cast<int>(x % p.H_v)) = 0;
+  if (x == 0) reinterpret_cast<unsigned long long*>(p.ws_flag)[1] = 0ull;
+}
+
+// the number of scan CTAs of a fused launch, or 0 when the two phases go as two launches.
+// allow_fused: 0 = never, 1 = automatic (also needs enough prep items to keep the other SMs
+// busy for several rounds: with few, the prep's own latency dominates and two launches win),
+// 2 = whenever the scan fits in half the SMs.
+int fused_scan_ctas(const PrefillParams& p) {
+  if (!p.allow_fused || p.n_chunks <= 0) return 0;
+  const long long n_scan = static_cast<long long>(p.N) * p.H_v;
+  int dev = 0, n_sm = 0, smem_optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  if (n_scan * kMaxFusedScanFraction > n_sm) return 0;
+  if (p.allow_fused == 1 && p.n_chunks * p.H_k < static_cast<long long>(kMinFusedItemsPerSm) * (n_sm - n_scan)) return 0;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, prefill_fused_kernel) != cudaSuccess) return 0;
+  if (static_cast<long long>(attr.sharedSizeBytes) + fused_smem_bytes(p.H_v / p.H_k) > smem_optin) return 0;
+  return static_cast<int>(n_scan);
 }
 
 cudaError_t launch_scan(const PrefillParams& p, cudaStream_t stream) {
@@ -1264,8 +1407,10 @@ cudaError_t launch_scan(const PrefillParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* const* events) {
+cudaError_t launch_prefill(const PrefillParams& p_in, cudaStream_t stream, void* const* events) {
   cudaError_t err;
+  PrefillParams p = p_in;
+  p.fused_scan_ctas = fused_scan_ctas(p);
   if (p.cu) {
     setup_kernel<<<1, 1024, 0, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -1274,6 +1419,28 @@ cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* co
     const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
     conv_out_kernel<<<dim3(static_cast<unsigned>((C_conv + 255) / 256), p.N), 256, 0, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (p.fused_scan_ctas > 0) {
+    const long long n_flags = p.n_chunks * p.H_v;
+    ready_flags_reset_kernel<<<static_cast<unsigned>((n_flags + 255) / 256), 256, 0, stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int smem = fused_smem_bytes(p.H_v / p.H_k);
+    err = cudaFuncSetAttribute(prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    const long long n_items = p.n_chunks * p.H_k;
+    int dev = 0, n_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const long long n_prep = std::min<long long>(n_sm - p.fused_scan_ctas, n_items);
+    const unsigned grid = static_cast<unsigned>(p.fused_scan_ctas + n_prep);
+    if (events) {  // one launch: the prep / scan split is not observable; [1] sits next to [0]
+      cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
+      cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);
+    }
+    prefill_fused_kernel<<<grid, kFusedThreads, smem, stream>>>(p);
+    err = cudaGetLastError();
+    if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), stream);
+    return err;
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
   if (p.n_chunks > 0) {

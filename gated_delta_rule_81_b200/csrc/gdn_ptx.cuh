@@ -125,6 +125,38 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// orders this thread's generic-proxy and async-proxy (bulk copy) accesses of global memory
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until another CTA has published *flag != 0 with a release store; the
+// acquire plus the proxy fence order this thread's later bulk-copy reads after it.
+// False on timeout (error bit 1 raised) or abort.
+__device__ __forceinline__ bool flag_wait(const int* flag, const Abort& ab, unsigned sleep_ns) {
+  long long t0 = clock64();
+  while (ld_acquire_gpu(flag) == 0) {
+    if (ab.raised()) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      ab.raise(kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(sleep_ns);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }

@@ -38,7 +38,12 @@ class GdnInputs(ctypes.Structure):
         ("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
         ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("scale", ctypes.c_float),
         ("events", ctypes.c_void_p),
+        ("schedule", ctypes.c_int),
     ]
+
+SCHEDULE_AUTO = 0          # one overlapped launch when it pays (few scan units, many prep items)
+SCHEDULE_TWO_LAUNCHES = 1  # prep kernel, then scan kernel
+SCHEDULE_FUSED = 2         # one overlapped launch whenever the scan units fit in half the SMs
 
 
 _lib = None
@@ -89,7 +94,7 @@ def _tok_stride(t, T_tot):
     return t.stride(0)
 
 
-def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0) -> GdnInputs:
+def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0, schedule=SCHEDULE_AUTO) -> GdnInputs:
     T_tot = q.shape[0]
     H_k = q.shape[1] if q.dim() == 3 else q.shape[-1] // HEAD_DIM
     H_v = v.shape[1] if v.dim() == 3 else v.shape[-1] // HEAD_DIM
@@ -105,6 +110,7 @@ def make_inputs(q, k, v, a, b, z, conv_w, A_log, norm_w, scale=1.0) -> GdnInputs
     s.stride_z, s.stride_a, s.stride_b = (_tok_stride(t, T_tot) for t in (z, a, b))
     s.conv_w, s.A_log, s.norm_w = conv_w.data_ptr(), A_log.data_ptr(), norm_w.data_ptr()
     s.H_k, s.H_v, s.scale = int(H_k), int(H_v), float(scale)
+    s.schedule = int(schedule)
     return s
 
 

@@ -82,7 +82,16 @@ typedef struct {
   void* const* events;    /* optional timing hook: NULL, or caller-created cudaEvent_t handles that
                              the library records on `stream` around its kernels.  Prefill: 3 events,
                              [0] before the prep kernel, [1] between prep and scan, [2] after the
-                             scan.  Decode: 2 events, before and after the decode kernel. */
+                             scan; when both phases run as one fused launch (see `schedule`), [1] is
+                             recorded right after [0] and [2] after the launch.  Decode: 2 events,
+                             before and after the decode kernel. */
+  int schedule;           /* prefill launch plan.  1 = the chunk-parallel prep kernel, then the
+                             sequential scan kernel.  2 = one launch that overlaps them chunk by
+                             chunk (scan CTAs first, the prep on the other SMs publishing each
+                             chunk to the scan) whenever the scan's (sequence, value head) units
+                             fit in half the SMs, else as 1.  0 = automatic: as 2 when the prep
+                             also has at least 8 (chunk, key head) items per remaining SM, else
+                             as 1.  Results are bitwise identical under every plan. */
 } gdn_inputs;
 
 /*

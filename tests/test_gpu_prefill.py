@@ -28,8 +28,9 @@ def small_case(lengths, H_k=2, H_v=6, seed=11, a_mean=0.0, with_state=True, with
             "conv_in": gin.conv_state(N, H_k, H_v, seed + 2) if with_conv else None}
 
 
-def run_gpu(case, uniform=False, conv_in=None):
+def run_gpu(case, uniform=False, conv_in=None, schedule=gdn.SCHEDULE_AUTO):
     keep, s = device_inputs(case["inp"])
+    s.schedule = schedule
     st = case.get("state_in")
     st = st.cuda() if st is not None else None
     cv = conv_in if conv_in is not None else case.get("conv_in")
@@ -245,11 +246,13 @@ def test_other_head_groupings(H_k, H_v):
     check(case, out, S, C, run_oracle(case))
 
 
-def test_device_cu_seqlens_mismatch_is_reported_not_computed():
+@pytest.mark.parametrize("schedule", [gdn.SCHEDULE_TWO_LAUNCHES, gdn.SCHEDULE_FUSED])
+def test_device_cu_seqlens_mismatch_is_reported_not_computed(schedule):
     """The device copy of cu_seqlens disagrees with the host copy: the setup kernel
     detects it, sets error bit 4 and every other kernel skips its work."""
     case = small_case([64, 64])
     keep, s = device_inputs(case["inp"])
+    s.schedule = schedule
     cu_host = case["cu_seqlens"]
     cu_bad = torch.tensor([0, 64, 100], dtype=torch.int32, device="cuda")  # host says 128 tokens
     err = err_word()
@@ -258,3 +261,23 @@ def test_device_cu_seqlens_mismatch_is_reported_not_computed():
     torch.cuda.synchronize()
     assert int(err.item()) & 4
     assert torch.all(out == 7.0)  # nothing was written
+
+
+@pytest.mark.parametrize("kind", ["uniform-200-2x6", "varlen-2x6", "uniform-300-4x8", "layer-4096-16x48"])
+def test_fused_and_two_launch_schedules_bitwise_equal(kind):
+    """The fused schedule (prep and scan overlapped in one launch) and the plain
+    two-launch schedule run the same arithmetic."""
+    if kind == "uniform-200-2x6":
+        case, uniform = small_case([200], seed=41), True
+    elif kind == "varlen-2x6":
+        case, uniform = small_case([1, 64, 0, 65, 130, 3], seed=42, with_conv=True), False
+    elif kind == "uniform-300-4x8":
+        case, uniform = small_case([300], H_k=4, H_v=8, seed=43), True
+    else:
+        case, uniform = gin.prefill_case(1), True
+    a = run_gpu(case, uniform=uniform, schedule=gdn.SCHEDULE_FUSED)
+    b = run_gpu(case, uniform=uniform, schedule=gdn.SCHEDULE_TWO_LAUNCHES)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    if kind != "layer-4096-16x48":
+        check(case, *a, run_oracle(case))

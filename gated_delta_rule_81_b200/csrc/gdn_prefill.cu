@@ -466,7 +466,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     const long long ch0 = grp == 0 ? static_cast<long long>(kh) * kD
                         : grp == 1 ? static_cast<long long>(H_k + kh) * kD
                                    : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh * G + grp - 2) * kD;
-    sW[x] = __ldg(reinterpret_cast<const uint4*>(p.conv_w + (ch0 + 2 * pair) * kTaps));
+    cp_async16(&sW[x], p.conv_w + (ch0 + 2 * pair) * kTaps);  // waited for with the raw rows
   }
 
   // ---- gates of the key head's value heads
@@ -502,7 +502,9 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   cp_async_wait_all();
   named_bar_sync(bar_id, kPrepThreads);
   {
-    const int i = tid >> 2, qq = tid & 3;
+    // a quarter-warp takes 8 consecutive tokens of one 32-channel group: the raw rows are
+    // 528 bytes apart, so its 16-byte reads fall on 8 distinct bank groups
+    const int i = (tid & 7) | ((tid >> 5) << 3), qq = (tid >> 3) & 3;
     const bool valid = i < L;
     for (int which = 0; which < 2; ++which) {
       float y[32];
@@ -513,8 +515,8 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
         if (!valid) y[e2] = 0.f;
         ss = fmaf(y[e2], y[e2], ss);
       }
-      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
       const float inv = rsqrtf(ss + 1e-6f) * (which == 0 ? p.scale : 1.0f);
       const int row = which * 64 + i, kb = qq >> 1;
 #pragma unroll
@@ -685,7 +687,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     named_bar_sync(bar_id, kPrepThreads);  // T is dead: region R takes the v_hat image
     {
       // v_hat of value head h: token i, channels 32*qq .. 32*qq+31, as the MN-major image
-      const int i = tid >> 2, qq = tid & 3;
+      const int i = (tid & 7) | ((tid >> 5) << 3), qq = (tid >> 3) & 3;
       float y[32];
       if (i < L) {
         conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,

@@ -156,6 +156,23 @@ gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens
                         out, workspace, workspace_bytes, err, stream);
 }
 
+gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long ldb, void* C, long long ldc, int M,
+                         int N, int K, int* err, void* stream) {
+  if (M < 0 || N < 0 || K < 0) return GDN_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return GDN_OK;
+  if (!A || !B || !C || K == 0) return GDN_ERR_INVALID_ARG;
+  if (K % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  if (lda < K || ldb < K || ldc < N) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || ((lda | ldb | ldc) & 7)) return GDN_ERR_MISALIGNED;
+  const size_t a_bytes = (static_cast<size_t>(M - 1) * lda + K) * 2, b_bytes = (static_cast<size_t>(N - 1) * ldb + K) * 2;
+  const size_t c_bytes = (static_cast<size_t>(M - 1) * ldc + N) * 2;
+  if (overlap(C, c_bytes, A, a_bytes) || overlap(C, c_bytes, B, b_bytes)) return GDN_ERR_ALIAS;
+  const cudaError_t e = gdn::launch_gemm_bf16(static_cast<const bf16*>(A), lda, static_cast<const bf16*>(B), ldb,
+                                              static_cast<bf16*>(C), ldc, M, N, K, err,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,
                             const int* state_slot, int n_slots, void* out, int* err, void* stream) {
   if (N < 0 || T < 1 || T > gdn::kMaxDecodeTokens || n_slots < 0) return GDN_ERR_INVALID_ARG;

@@ -1,0 +1,247 @@
+// Dense bf16 projections around the mixer: C = A B^T with fp32 accumulation.
+//
+// Agnes-3.0-Flash model card, "Architecture" table: hidden size 5120, and the row
+// "Delta-rule layers" (16 key heads / 48 value heads, head dim 128).  The mixer's
+// inputs (q, k, v, the output gate z and the per-head gate logits a, b) come from
+// the hidden state through one input projection, and its 48 x 128 outputs go back
+// to the hidden size through one output projection.  Both are plain matrix products,
+// which this file computes on the tensor cores.
+//
+// One persistent CTA per SM walks 128 x 256 output tiles (M fastest, so the CTAs
+// running at the same time share B tiles through L2).  Per tile and 64-wide K step,
+// warp 0 lane 0 loads the A (128 x 64) and B (256 x 64) boxes with TMA (128-byte
+// swizzle, zero fill past the matrix edges) into a 4-stage ring; warp 1 lane 0
+// issues four tcgen05.mma (M 128, N 256, K 16) per step into one of two 256-column
+// fp32 accumulators in tensor memory; warps 2-5 read the other accumulator
+// (thread = row, lane quarter = warp % 4), round to bf16 and store, so each tile's
+// epilogue overlaps the next tile's products.  Every wait is bounded: a stuck
+// wait sets error bit 1 and the CTA unwinds (draining its copies and products).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "gdn_kernels.cuh"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
+constexpr int kGemmStages = 4;
+constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 16 KiB
+constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;  // 32 KiB
+constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
+constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024;
+constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kGemmEpiWarps = 4;
+
+struct GemmParams {
+  int M, N, K;
+  int tiles_m, tiles_n;
+  bf16* C;
+  long long ldc;
+  int* err;
+};
+
+__device__ __forceinline__ uint8_t* gemm_align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// 2-D tiled TMA load of the box at (x = column, y = row) into shared memory, completing on bar
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                     GemmParams g) {
+  extern __shared__ uint8_t gemm_smem_raw[];
+  uint8_t* sm = gemm_align1024(gemm_smem_raw);
+  __shared__ uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_empty[2], drain_b;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Abort ab{g.err, &abort_s};
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kGemmEpiWarps);
+    }
+    mbar_init(&drain_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc<512>(&tmem_base_s);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+  const int n_tiles = g.tiles_m * g.tiles_n;
+  const int k_steps = g.K / kGemmBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      long long it = 0;
+      for (int t = blockIdx.x; t < n_tiles && !ab.raised(); t += gridDim.x) {
+        const int m0 = (t % g.tiles_m) * kGemmBM, n0 = (t / g.tiles_m) * kGemmBN;
+        bool ok = true;
+        for (int kk = 0; kk < k_steps; ++kk, ++it) {
+          const int s = static_cast<int>(it % kGemmStages);
+          const long long use = it / kGemmStages;
+          if (use > 0 && !mbar_wait(&empty[s], static_cast<uint32_t>((use - 1) & 1), ab)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kGemmStageBytes);
+          uint8_t* st = sm + s * kGemmStageBytes;
+          tma_load_2d(st, &tma_a, kk * kGemmBK, m0, &full[s]);
+          tma_load_2d(st + kGemmABytes, &tma_b, kk * kGemmBK, n0, &full[s]);
+        }
+        if (!ok) break;
+      }
+      // loads still in flight (only after an abort) land before the CTA exits
+      int drain_flag = 0;
+      const Abort drain{nullptr, &drain_flag};
+      for (int s = 0; s < kGemmStages; ++s) {
+        const long long uses = it > s ? (it - 1 - s) / kGemmStages + 1 : 0;  // loads issued into stage s
+        if (uses > 0) mbar_wait(&full[s], static_cast<uint32_t>((uses - 1) & 1), drain);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, false, false);
+      long long it = 0;
+      int tile_i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tile_i) {
+        const int b = tile_i & 1, buse = tile_i >> 1;
+        if (buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t d = tbase + static_cast<uint32_t>(b * kGemmBN);
+        for (int kk = 0; kk < k_steps; ++kk, ++it) {
+          const int s = static_cast<int>(it % kGemmStages);
+          if (!mbar_wait(&full[s], static_cast<uint32_t>((it / kGemmStages) & 1), ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_s = smem_u32(sm + s * kGemmStageBytes), b_s = a_s + kGemmABytes;
+#pragma unroll
+          for (int ks = 0; ks < kGemmBK / 16; ++ks)
+            umma_bf16(d, smem_desc(a_s + ks * 32u, 16, 1024, Swz::k128), smem_desc(b_s + ks * 32u, 16, 1024, Swz::k128),
+                      idesc, kk > 0 || ks > 0);
+          umma_commit(&empty[s]);  // the stage is free once these products have read it
+        }
+        if (ok) umma_commit(&acc_full[b]);
+      }
+      // every product issued has completed before tensor memory is released
+      umma_commit(&drain_b);
+      int drain_flag = 0;
+      const Abort drain{nullptr, &drain_flag};
+      mbar_wait(&drain_b, 0, drain);
+    }
+  } else {
+    // ------------------------------------------------ epilogue: thread = output row
+    const int q = warp & 3;
+    int tile_i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tile_i) {
+      const int b = tile_i & 1;
+      if (!mbar_wait_warp(&acc_full[b], (tile_i >> 1) & 1, ab, false, 32)) break;
+      tc_fence_after();
+      const int m0 = (t % g.tiles_m) * kGemmBM, n0 = (t / g.tiles_m) * kGemmBN;
+      const int row = m0 + 32 * q + lane;
+      bf16* crow = g.C + static_cast<long long>(row) * g.ldc + n0;
+#pragma unroll 1
+      for (int c = 0; c < kGemmBN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_addr(tbase, 32 * q, static_cast<uint32_t>(b * kGemmBN + 32 * c)), v);
+        tmem_wait_ld();
+        const int col = n0 + 32 * c;
+        if (row < g.M && col < g.N) {
+          if (col + 32 <= g.N) {
+            uint4* dst = reinterpret_cast<uint4*>(crow + 32 * c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                  pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col + e < g.N) crow[32 * c + e] = __float2bfloat16(v[e]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc<512>(tbase);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// K-major bf16 matrix [rows][ld] (first `cols` columns used) as 64 x box_rows boxes, 128-byte swizzle
+bool encode_kmajor(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, long long rows,
+                   long long cols, long long ld, int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
+                             int M, int N, int K, int* err, cudaStream_t stream) {
+  static_assert(kGemmSmem <= 227 * 1024, "GEMM shared memory");
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap ta, tb;
+  if (!encode_kmajor(enc, &ta, A, M, K, lda, kGemmBM) || !encode_kmajor(enc, &tb, B, N, K, ldb, kGemmBN))
+    return cudaErrorInvalidValue;
+  GemmParams g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.tiles_m = (M + kGemmBM - 1) / kGemmBM;
+  g.tiles_n = (N + kGemmBN - 1) / kGemmBN;
+  g.C = C;
+  g.ldc = ldc;
+  g.err = err;
+  int dev = 0, n_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem)) !=
+      cudaSuccess)
+    return e;
+  const long long n_tiles = static_cast<long long>(g.tiles_m) * g.tiles_n;
+  const unsigned grid = static_cast<unsigned>(n_tiles < n_sm ? n_tiles : n_sm);
+  gemm_bf16_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

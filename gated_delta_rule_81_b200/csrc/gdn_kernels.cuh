@@ -87,5 +87,9 @@ struct PrefillParams {
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events);
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* const* events);
+// C[M][N] = A[M][K] B[N][K]^T in bf16 with fp32 accumulation (row-major, leading dimensions
+// in elements; K a multiple of 64; pointers and leading dimensions 16-byte aligned)
+cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
+                             int M, int N, int K, int* err, cudaStream_t stream);
 
 }  // namespace gdn

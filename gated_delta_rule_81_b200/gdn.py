@@ -50,7 +50,7 @@ _lib = None
 _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
-           "gdn_decode_multi", "gdn_status_string")
+           "gdn_decode_multi", "gdn_gemm_bf16", "gdn_status_string")
 MAX_DECODE_TOKENS = 8
 
 
@@ -74,6 +74,8 @@ def load(path: str | None = None):
     lib.gdn_decode_step.restype = _i
     lib.gdn_decode_multi.argtypes = [P, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]
     lib.gdn_decode_multi.restype = _i
+    lib.gdn_gemm_bf16.argtypes = [_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _vp, _vp]
+    lib.gdn_gemm_bf16.restype = _i
     lib.gdn_status_string.argtypes = [_i]
     lib.gdn_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -220,6 +222,24 @@ def decode_multi(inp: GdnInputs, N: int, T: int, state, conv_state, state_slot=N
     _check(lib.gdn_decode_multi(ctypes.byref(inp), N, T, _ptr(state), _ptr(conv_state), _ptr(state_slot), n_slots,
                                 _ptr(out), _ptr(err), _stream()),
            "gdn_decode_multi")
+    return out
+
+
+def gemm_bf16(a, b, out=None, err=None):
+    """gdn_gemm_bf16: out[M][N] = a[M][K] @ b[N][K]^T (bf16, fp32 accumulation).  a and b may be
+    row-strided views (last dimension contiguous)."""
+    lib = load()
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b disagree on K")
+    for name, t in (("a", a), ("b", b)):
+        if t.dtype != torch.bfloat16 or t.stride(1) != 1:
+            raise TypeError(f"{name} must be bf16 with a contiguous last dimension")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    _check(lib.gdn_gemm_bf16(_ptr(a), a.stride(0), _ptr(b), b.stride(0), _ptr(out), out.stride(0), M, N, K,
+                             _ptr(err), _stream()), "gdn_gemm_bf16")
     return out
 
 

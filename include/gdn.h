@@ -148,6 +148,21 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
                            int* err, void* stream);
 
 /*
+ * The dense projections on either side of the mixer (hidden size 5120 -> q|k|v|z|a|b,
+ * and 48*128 -> 5120): C = A B^T on the tensor cores, bf16 in and out, fp32
+ * accumulation, one rounding to bf16 per output element.
+ *   A  bf16 [M][lda], first K columns used        (activations, row-major)
+ *   B  bf16 [N][ldb], first K columns used        (weights, one output channel per row)
+ *   C  bf16 [M][ldc], first N columns written
+ * K must be a multiple of 64 (GDN_ERR_UNSUPPORTED otherwise); every pointer and
+ * leading dimension 16-byte aligned (GDN_ERR_MISALIGNED); C must not overlap A or
+ * B (GDN_ERR_ALIAS).  M or N = 0 is a no-op.  Error bit 1 of *err: a wait inside
+ * the kernel timed out.
+ */
+gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long ldb, void* C, long long ldc, int M,
+                         int N, int K, int* err, void* stream);
+
+/*
  * T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N sequences in one call
  * (decode with several tokens per step, e.g. verifying drafted tokens), with
  * the states held in slots of a state pool.  Token n * T + t of the inputs is

@@ -15,3 +15,4 @@ from .gdn_oracle import (  # noqa: F401
     recurrence,
 )
 from .chunked import chunked_recurrence  # noqa: F401
+from .projections import gemm, in_proj_layout, layer, round_bf16  # noqa: F401

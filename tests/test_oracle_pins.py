@@ -358,3 +358,53 @@ def test_mixer_identity_gate_through_full_path():
     for h in range(3):
         np.testing.assert_allclose(res["pre_norm"][:, h], qh @ st[0, h].double().numpy().T,
                                    rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ projections around the mixer
+
+
+def test_gemm_small_exact_and_orientation():
+    """C = A B^T: a hand-computed 2x2 product pins the orientation (B holds one output channel per row)."""
+    a = torch.tensor([[1.0, 2.0, 3.0], [4.0, 5.0, 6.0]], dtype=torch.bfloat16)
+    b = torch.tensor([[1.0, 0.0, 1.0], [0.0, 1.0, 0.0]], dtype=torch.bfloat16)
+    np.testing.assert_array_equal(oracle.gemm(a, b), np.array([[4.0, 2.0], [10.0, 5.0]]))
+
+
+def test_round_bf16_ties_and_library():
+    """Round to nearest bf16 with ties to even: values with a known answer, then agreement
+    with torch's own float32 -> bfloat16 conversion on random fp32 values."""
+    x = np.array([1 + 2.0**-8, 1 + 3 * 2.0**-9, 1 + 2.0**-7 + 2.0**-8, -2.5, 0.0, 3 * 2.0**-130])
+    want = np.array([1.0, 1 + 2.0**-7, 1 + 2.0**-6, -2.5, 0.0, 3 * 2.0**-130])
+    np.testing.assert_array_equal(oracle.round_bf16(x), want)
+    r = torch.randn(4096, generator=torch.Generator().manual_seed(3)) * 7.0
+    np.testing.assert_array_equal(oracle.round_bf16(r.double().numpy()), r.to(torch.bfloat16).double().numpy())
+
+
+def test_layer_routes_projection_columns():
+    """With permutation weights the layer is the mixer on permuted hidden channels: this pins
+    the q|k|v|z|a|b column order of the input projection and the output projection's
+    orientation, independently of the layer function's own bookkeeping."""
+    H_k, H_v, D, T = 1, 2, 128, 9
+    lay = oracle.in_proj_layout(H_k, H_v, D)
+    n_in = lay["total"][1]
+    hidden = n_in
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(T, hidden, generator=g).to(torch.bfloat16)
+    perm = torch.randperm(n_in, generator=g)
+    w_in = torch.zeros(n_in, hidden, dtype=torch.bfloat16)
+    w_in[torch.arange(n_in), perm] = 1.0  # proj[:, j] = x[:, perm[j]]
+    w_out = torch.zeros(hidden, H_v * D, dtype=torch.bfloat16)
+    rows = torch.arange(H_v * D)
+    w_out[rows, rows] = 1.0  # y[:, c] = out[:, c] for c < H_v*D, zero above
+    w = gin.weights(H_k, H_v, seed=5)
+    res = oracle.layer(x, w_in, w_out, w["conv_w"], w["A_log"], w["norm_w"], [0, T], H_k, H_v)
+    xp = x[:, perm]
+    inp = {n: xp[:, lay[n][0]:lay[n][1]].reshape(T, -1, D) for n in ("q", "k", "v", "z")}
+    inp.update({n: xp[:, lay[n][0]:lay[n][1]] for n in ("a", "b")})
+    inp.update(w)
+    inp["scale"] = 1.0
+    ref = oracle.mixer(inp, [0, T])
+    np.testing.assert_array_equal(res["out"], ref["out"])
+    o16 = torch.from_numpy(ref["out"]).to(torch.bfloat16).double().numpy().reshape(T, H_v * D)
+    np.testing.assert_array_equal(res["y"][:, :H_v * D], o16)
+    assert np.all(res["y"][:, H_v * D:] == 0)

@@ -18,6 +18,7 @@ host cores instead.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -351,6 +352,79 @@ def run_decode_ours(args, dev, steps_per_pass=64, T=1):
             "tokens_per_s": N * T / per_launch_s}
 
 
+def run_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120, H_k=16, H_v=48):
+    """One delta-rule layer, y = out_proj(mixer(in_proj(x))), B = 1, T = 4096, hidden 5120,
+    16/48 heads, random dense weights (std 1/sqrt(fan_in)); times the three parts with the
+    layer's event hook, and cuBLAS (torch.matmul) on the same two projection shapes beside."""
+    from gated_delta_rule_81_b200 import gdn
+
+    g = torch.Generator().manual_seed(100 + rank)
+    n_in = int(gdn.load().gdn_layer_n_in(H_k, H_v))
+    x = torch.randn(T, hidden, generator=g).to(torch.bfloat16).to(dev)
+    w_in = (torch.randn(n_in, hidden, generator=g) * hidden ** -0.5).to(torch.bfloat16).to(dev)
+    w_out = (torch.randn(hidden, H_v * 128, generator=g) * (H_v * 128) ** -0.5).to(torch.bfloat16).to(dev)
+    w = {k: v.to(dev) for k, v in gin.weights(H_k, H_v, seed=rank).items()}
+    st = gin.recurrent_state(1, H_v, seed=rank).to(dev)
+    L = gdn.make_layer(w_in, w_out, w["conv_w"], w["A_log"], w["norm_w"], H_k, H_v,
+                       schedule=SCHEDULES[args.schedule])
+    y = torch.empty(T, hidden, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(1, H_v, 128, 128, dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.layer_workspace_size(H_k, H_v, 1, T), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.layer_prefill(L, 1, T, x, st, None, y=y, state_out=S, want_conv=False, workspace=ws, err=err)
+
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for ev in evs:
+            flush_l2(flush)
+            arr = (ctypes.c_void_p * 4)(*[e.cuda_event or (e.record(stream) or e.cuda_event) for e in ev])
+            L.events = ctypes.cast(arr, ctypes.c_void_p)
+            step()
+        torch.cuda.synchronize()
+    L.events = None
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    parts = {"in_proj": [e[0].elapsed_time(e[1]) for e in evs], "mixer": [e[1].elapsed_time(e[2]) for e in evs],
+             "out_proj": [e[2].elapsed_time(e[3]) for e in evs]}
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    # cuBLAS on the same shapes, for comparison
+    proj = torch.empty(T, n_in, dtype=torch.bfloat16, device=dev)
+    mix = torch.randn(T, H_v * 128, device=dev).to(torch.bfloat16)
+
+    def cublas(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for _ in range(reps):
+            flush_l2(flush)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps
+
+    cub = {"in_proj": cublas(lambda: torch.matmul(x, w_in.t(), out=proj)),
+           "out_proj": cublas(lambda: torch.matmul(mix, w_out.t(), out=y))}
+    flops = {"in_proj": 2 * T * hidden * n_in, "out_proj": 2 * T * H_v * 128 * hidden,
+             "mixer": (scan_flop_per_token(H_v) + prep_flop_per_token(H_k, H_v)) * T}
+    return {"total_ms": total_ms, "T": T, "parts_ms": {k: statistics.mean(v) for k, v in parts.items()},
+            "cublas_ms": cub, "flops": flops, "clocks": clk.report(), "steps": args.steps}
+
+
 # ------------------------------------------------------------------ oracle (CPU) arm
 
 
@@ -413,7 +487,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode"], default="prefill4k",
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer"], default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
@@ -452,6 +526,33 @@ def main():
                                            "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"],
                                            "traffic": decode_traffic() if d["T"] == 1 else None},
                               "gpu_launches": d["launches"]}), flush=True)
+        return 0
+    if args.workload == "layer":
+        r = run_layer_ours(args, world, rank, dev, pk)
+        if rank == 0:
+            pm = r["parts_ms"]
+            dom = max(pm, key=pm.get)
+            achieved = r["flops"][dom] / (pm[dom] * 1e-3) / 1e12
+            gemm = {k: {"ms": round(pm[k], 5), "tflops": r["flops"][k] / (pm[k] * 1e-3) / 1e12,
+                        "frac_of_peak": r["flops"][k] / (pm[k] * 1e-3) / 1e12 / pk["bf16_tflops"],
+                        "cublas_ms": round(r["cublas_ms"][k], 5),
+                        "cublas_tflops": r["flops"][k] / (r["cublas_ms"][k] * 1e-3) / 1e12}
+                    for k in ("in_proj", "out_proj")}
+            ms_step = r["total_ms"] / r["steps"]
+            print(json.dumps({
+                "metric": "delta-layer prefill tokens/s (in_proj + mixer + out_proj)",
+                "value": world * r["T"] * r["steps"] / (r["total_ms"] / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": r["steps"], "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "delta-layer-prefill-T4096-hidden5120-16x48", "batch": 1, "seq_len": r["T"],
+                           "hidden": 5120, "H_k": 16, "H_v": 48, "weights": "random dense, std 1/sqrt(fan_in)",
+                           "l2": "flushed between timed steps"},
+                "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                             "peak_source": f"{pk['source']} (bf16 burst)",
+                             "parts_ms": {k: round(v, 5) for k, v in pm.items()}},
+                "gemm": gemm,
+                "gpu_launches": 4 * r["steps"], "clocks": r["clocks"]}), flush=True)
         return 0
     cfg_id = WORKLOADS[args.workload]
     res = run_prefill_ours(args, world, rank, dev, pk, cfg_id)

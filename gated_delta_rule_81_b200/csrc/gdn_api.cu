@@ -20,6 +20,11 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
+// leading dimension of the layer's projection buffer: n_in rounded up to 8 (16-byte rows)
+long long layer_ld_proj(int H_k, int H_v) {
+  return (2LL * H_k * GDN_HEAD_DIM + 2LL * H_v * GDN_HEAD_DIM + 2LL * H_v + 7) / 8 * 8;
+}
+
 // chunk_base[N+1] and seq_order[N] (ints) after the 1 KiB header
 size_t chunk_base_bytes(int N) { return round_up(sizeof(int) * (2 * static_cast<size_t>(N) + 1), 1024); }
 
@@ -46,12 +51,20 @@ gdn_status check_inputs(const gdn_inputs* in, long long T_tot) {
 }
 
 // `out` must not overlap any input read by the same call
+// bytes from the first element of a [T_tot] x stride input to the end of its last row's `width` channels
+size_t input_extent(long long T_tot, long long stride, long long width) {
+  return sizeof(bf16) * (static_cast<size_t>(T_tot - 1) * static_cast<size_t>(stride) + static_cast<size_t>(width));
+}
+
 gdn_status check_out_alias(const gdn_inputs* in, long long T_tot, const void* out) {
   const size_t ob = static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
-  const size_t tb = sizeof(bf16) * static_cast<size_t>(T_tot);
-  if (overlap(out, ob, in->q, tb * in->stride_q) || overlap(out, ob, in->k, tb * in->stride_k) ||
-      overlap(out, ob, in->v, tb * in->stride_v) || overlap(out, ob, in->z, tb * in->stride_z) ||
-      overlap(out, ob, in->a, tb * in->stride_a) || overlap(out, ob, in->b, tb * in->stride_b))
+  const long long qk = static_cast<long long>(in->H_k) * GDN_HEAD_DIM, vz = static_cast<long long>(in->H_v) * GDN_HEAD_DIM;
+  if (overlap(out, ob, in->q, input_extent(T_tot, in->stride_q, qk)) ||
+      overlap(out, ob, in->k, input_extent(T_tot, in->stride_k, qk)) ||
+      overlap(out, ob, in->v, input_extent(T_tot, in->stride_v, vz)) ||
+      overlap(out, ob, in->z, input_extent(T_tot, in->stride_z, vz)) ||
+      overlap(out, ob, in->a, input_extent(T_tot, in->stride_a, in->H_v)) ||
+      overlap(out, ob, in->b, input_extent(T_tot, in->stride_b, in->H_v)))
     return GDN_ERR_ALIAS;
   return GDN_OK;
 }
@@ -171,6 +184,76 @@ gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long 
                                               static_cast<bf16*>(C), ldc, M, N, K, err,
                                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+long long gdn_layer_n_in(int H_k, int H_v) {
+  if (H_k <= 0 || H_v <= 0) return 0;
+  return 2LL * H_k * GDN_HEAD_DIM + 2LL * H_v * GDN_HEAD_DIM + 2LL * H_v;
+}
+
+size_t gdn_layer_workspace_size(int H_k, int H_v, int B, int T) {
+  if (H_k <= 0 || H_v <= 0 || B < 0 || T < 0) return 0;
+  const long long T_tot = static_cast<long long>(B) * T;
+  const long long n_chunks = static_cast<long long>(B) * ((T + GDN_CHUNK - 1) / GDN_CHUNK);
+  const size_t proj = round_up(static_cast<size_t>(T_tot) * layer_ld_proj(H_k, H_v) * 2, 1024);
+  const size_t mix = round_up(static_cast<size_t>(T_tot) * H_v * GDN_HEAD_DIM * 2, 1024);
+  return proj + mix + gdn_prefill_workspace_size(H_k, H_v, B, n_chunks);
+}
+
+gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, long long ldx, const float* state_in,
+                             float* state_out, const void* conv_in, void* conv_out, void* y, long long ldy,
+                             void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  if (!L || B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+  if (L->H_k <= 0 || L->H_v <= 0 || L->hidden <= 0 || L->H_v % L->H_k != 0) return GDN_ERR_INVALID_ARG;
+  if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
+  if (T_tot == 0) return GDN_OK;
+  if (!x || !y || !L->w_in || !L->w_out) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_layer_workspace_size(L->H_k, L->H_v, B, T);
+  if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  const long long n_in = gdn_layer_n_in(L->H_k, L->H_v), ld_p = layer_ld_proj(L->H_k, L->H_v);
+  const long long d_v = static_cast<long long>(L->H_v) * GDN_HEAD_DIM;
+  if (ldy < L->hidden) return GDN_ERR_INVALID_ARG;
+  if (overlap(y, (static_cast<size_t>(T_tot - 1) * ldy + L->hidden) * 2, workspace, need)) return GDN_ERR_ALIAS;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  bf16* proj = reinterpret_cast<bf16*>(ws);
+  bf16* mix = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(T_tot) * ld_p * 2, 1024));
+  uint8_t* ws_mixer = reinterpret_cast<uint8_t*>(mix) + round_up(static_cast<size_t>(T_tot) * d_v * 2, 1024);
+  const size_t ws_mixer_bytes = workspace_bytes - static_cast<size_t>(ws_mixer - ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) {
+    if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
+  };
+  mark(0);
+  gdn_status s = gdn_gemm_bf16(x, ldx, L->w_in, L->ld_w_in, proj, ld_p, static_cast<int>(T_tot),
+                               static_cast<int>(n_in), L->hidden, err, stream);
+  if (s != GDN_OK) return s;
+  mark(1);
+  const long long HkD = static_cast<long long>(L->H_k) * GDN_HEAD_DIM;
+  gdn_inputs in = {};
+  in.q = proj;
+  in.k = proj + HkD;
+  in.v = proj + 2 * HkD;
+  in.z = proj + 2 * HkD + d_v;
+  in.a = proj + 2 * HkD + 2 * d_v;
+  in.b = proj + 2 * HkD + 2 * d_v + L->H_v;
+  in.stride_q = in.stride_k = in.stride_v = in.stride_z = in.stride_a = in.stride_b = ld_p;
+  in.conv_w = L->conv_w;
+  in.A_log = L->A_log;
+  in.norm_w = L->norm_w;
+  in.H_k = L->H_k;
+  in.H_v = L->H_v;
+  in.scale = L->scale;
+  in.schedule = L->schedule;
+  s = gdn_prefill(&in, B, T, state_in, state_out, conv_in, conv_out, mix, ws_mixer, ws_mixer_bytes, err, stream);
+  if (s != GDN_OK) return s;
+  mark(2);
+  s = gdn_gemm_bf16(mix, d_v, L->w_out, L->ld_w_out, y, ldy, static_cast<int>(T_tot), L->hidden,
+                    static_cast<int>(d_v), err, stream);
+  if (s != GDN_OK) return s;
+  mark(3);
+  return GDN_OK;
 }
 
 gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,

@@ -41,6 +41,18 @@ class GdnInputs(ctypes.Structure):
         ("schedule", ctypes.c_int),
     ]
 
+class GdnLayer(ctypes.Structure):
+    """gdn_layer: the weights of one delta-rule layer (device pointers)."""
+    _fields_ = [
+        ("w_in", ctypes.c_void_p), ("ld_w_in", ctypes.c_longlong),
+        ("w_out", ctypes.c_void_p), ("ld_w_out", ctypes.c_longlong),
+        ("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
+        ("H_k", ctypes.c_int), ("H_v", ctypes.c_int), ("hidden", ctypes.c_int),
+        ("scale", ctypes.c_float), ("schedule", ctypes.c_int),
+        ("events", ctypes.c_void_p),
+    ]
+
+
 SCHEDULE_AUTO = 0          # one overlapped launch when it pays (few scan units, many prep items)
 SCHEDULE_TWO_LAUNCHES = 1  # prep kernel, then scan kernel
 SCHEDULE_FUSED = 2         # one overlapped launch whenever the scan units fit in half the SMs
@@ -50,7 +62,8 @@ _lib = None
 _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
-           "gdn_decode_multi", "gdn_gemm_bf16", "gdn_status_string")
+           "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
+           "gdn_status_string")
 MAX_DECODE_TOKENS = 8
 
 
@@ -76,6 +89,13 @@ def load(path: str | None = None):
     lib.gdn_decode_multi.restype = _i
     lib.gdn_gemm_bf16.argtypes = [_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _vp, _vp]
     lib.gdn_gemm_bf16.restype = _i
+    lib.gdn_layer_n_in.argtypes = [_i, _i]
+    lib.gdn_layer_n_in.restype = _ll
+    lib.gdn_layer_workspace_size.argtypes = [_i, _i, _i, _i]
+    lib.gdn_layer_workspace_size.restype = _sz
+    lib.gdn_layer_prefill.argtypes = [ctypes.POINTER(GdnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _vp, _vp, _ll, _vp,
+                                      _sz, _vp, _vp]
+    lib.gdn_layer_prefill.restype = _i
     lib.gdn_status_string.argtypes = [_i]
     lib.gdn_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -241,6 +261,42 @@ def gemm_bf16(a, b, out=None, err=None):
     _check(lib.gdn_gemm_bf16(_ptr(a), a.stride(0), _ptr(b), b.stride(0), _ptr(out), out.stride(0), M, N, K,
                              _ptr(err), _stream()), "gdn_gemm_bf16")
     return out
+
+
+def make_layer(w_in, w_out, conv_w, A_log, norm_w, H_k, H_v, scale=1.0, schedule=SCHEDULE_AUTO) -> GdnLayer:
+    """gdn_layer from device tensors: w_in bf16 [n_in][hidden], w_out bf16 [hidden][H_v*128]."""
+    for name, t in (("w_in", w_in), ("w_out", w_out), ("conv_w", conv_w), ("norm_w", norm_w)):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise TypeError(f"{name} must be bf16 with a contiguous last dimension")
+    L = GdnLayer()
+    L.w_in, L.ld_w_in = w_in.data_ptr(), w_in.stride(0)
+    L.w_out, L.ld_w_out = w_out.data_ptr(), w_out.stride(0)
+    L.conv_w, L.A_log, L.norm_w = conv_w.data_ptr(), A_log.data_ptr(), norm_w.data_ptr()
+    L.H_k, L.H_v, L.hidden = int(H_k), int(H_v), int(w_in.shape[1])
+    L.scale, L.schedule = float(scale), int(schedule)
+    return L
+
+
+def layer_workspace_size(H_k, H_v, B, T) -> int:
+    return int(load().gdn_layer_workspace_size(H_k, H_v, B, T))
+
+
+def layer_prefill(L: GdnLayer, B: int, T: int, x, state_in=None, conv_in=None, *, want_state=True, want_conv=True,
+                  y=None, state_out=None, conv_out=None, workspace=None, err=None):
+    """gdn_layer_prefill: y = out_proj(mixer(in_proj(x))) for B sequences of T tokens.
+    Returns (y, state_out, conv_out)."""
+    lib = load()
+    dev = x.device
+    _, state_out, conv_out = _outputs(dev, 0, L.H_k, L.H_v, B, want_state, want_conv, torch.empty(0), state_out,
+                                      conv_out)
+    if y is None:
+        y = torch.empty(B * T, L.hidden, dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(layer_workspace_size(L.H_k, L.H_v, B, T), dtype=torch.uint8, device=dev)
+    _check(lib.gdn_layer_prefill(ctypes.byref(L), B, T, _ptr(x), x.stride(0), _ptr(state_in), _ptr(state_out),
+                                 _ptr(conv_in), _ptr(conv_out), _ptr(y), y.stride(0), _ptr(workspace),
+                                 workspace.numel(), _ptr(err), _stream()), "gdn_layer_prefill")
+    return y, state_out, conv_out
 
 
 def status_string(status: int) -> str:

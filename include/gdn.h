@@ -163,6 +163,48 @@ gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long 
                          int N, int K, int* err, void* stream);
 
 /*
+ * One delta-rule layer around the mixer: y = out_proj(mixer(in_proj(x))).
+ * The input projection's output channels are q (H_k*128) | k (H_k*128) | v (H_v*128) |
+ * z (H_v*128) | a (H_v) | b (H_v), n_in of them in all; no biases.
+ */
+typedef struct {
+  const void* w_in;       /* bf16 [n_in][ld_w_in], first `hidden` columns used */
+  long long ld_w_in;
+  const void* w_out;      /* bf16 [hidden][ld_w_out], first H_v*128 columns used */
+  long long ld_w_out;
+  const void* conv_w;     /* bf16 [C_conv][4] */
+  const float* A_log;     /* fp32 [H_v] */
+  const void* norm_w;     /* bf16 [128] */
+  int H_k, H_v;
+  int hidden;             /* model width; a multiple of 64 */
+  float scale;            /* as gdn_inputs.scale */
+  int schedule;           /* as gdn_inputs.schedule */
+  void* const* events;    /* optional timing hook: NULL, or 4 caller-created cudaEvent_t recorded on
+                             `stream` before the input projection, after it, after the mixer, and
+                             after the output projection */
+} gdn_layer;
+
+/* Channels of the input projection's output: 2 H_k 128 + 2 H_v 128 + 2 H_v. */
+long long gdn_layer_n_in(int H_k, int H_v);
+
+/* Bytes of workspace gdn_layer_prefill needs for B sequences of T tokens: the
+   projection output (bf16 [B T][n_in, padded to 8]), the mixer output (bf16 [B T][H_v 128])
+   and the mixer's own workspace.  0 on bad arguments. */
+size_t gdn_layer_workspace_size(int H_k, int H_v, int B, int T);
+
+/*
+ * Prefill of one delta-rule layer for B sequences of T tokens (packed [B*T]):
+ *   x  bf16 [B*T][ldx], first `hidden` columns used;  y  bf16 [B*T][ldy], first `hidden` written.
+ * state_in / state_out / conv_in / conv_out as in gdn_prefill.  Three launches
+ * groups on `stream`: gdn_gemm_bf16 (in_proj), gdn_prefill on the projection's
+ * columns (no copy: strided inputs), gdn_gemm_bf16 (out_proj).  Errors as those calls;
+ * y must not overlap x or the workspace.
+ */
+gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, long long ldx, const float* state_in,
+                             float* state_out, const void* conv_in, void* conv_out, void* y, long long ldy,
+                             void* workspace, size_t workspace_bytes, int* err, void* stream);
+
+/*
  * T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N sequences in one call
  * (decode with several tokens per step, e.g. verifying drafted tokens), with
  * the states held in slots of a state pool.  Token n * T + t of the inputs is

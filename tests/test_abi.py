@@ -20,7 +20,7 @@ def lib():
 
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "gdn.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:size_t|gdn_status|const char\*)\s+(gdn_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:size_t|gdn_status|const char\*|long long)\s+(gdn_\w+)\s*\(", text, re.M)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -128,3 +128,24 @@ def test_decode_multi_rejects_bad_arguments(lib):
     assert lib.gdn_decode_multi(ctypes.byref(s), 2, 2, st, cv, None, 2, st + 1024, None, None) == 4
     # N = 0 is a no-op
     assert lib.gdn_decode_multi(ctypes.byref(s), 0, 4, None, None, None, 0, None, None, None) == 0
+
+
+def test_layer_sizes_and_rejections(lib):
+    assert lib.gdn_layer_n_in(16, 48) == 2 * 16 * 128 + 2 * 48 * 128 + 2 * 48 == 16480
+    assert lib.gdn_layer_n_in(2, 6) == 2060 and lib.gdn_layer_n_in(0, 6) == 0
+    T = 4096
+    want = (-(-T * 16480 * 2 // 1024) * 1024) + (-(-T * 6144 * 2 // 1024) * 1024) + \
+        lib.gdn_prefill_workspace_size(16, 48, 1, T // 64)
+    assert lib.gdn_layer_workspace_size(16, 48, 1, T) == want
+    L = gdn.GdnLayer()
+    L.w_in, L.ld_w_in, L.w_out, L.ld_w_out = 0x100000, 5120, 0x200000, 6144
+    L.conv_w, L.A_log, L.norm_w = 0x300000, 0x310000, 0x320000
+    L.H_k, L.H_v, L.hidden, L.scale = 16, 48, 5120, 1.0
+    args = (1, 64, 0x400000, 5120, None, None, None, None, 0x900000, 5120, 0x2000000, 1 << 31, None, None)
+    L.hidden = 5000  # not a multiple of 64
+    assert lib.gdn_layer_prefill(ctypes.byref(L), *args) == 2
+    L.hidden = 5120
+    assert lib.gdn_layer_prefill(ctypes.byref(L), 1, 64, None, *args[3:]) == 1
+    small = args[:11] + (1024,) + args[12:]
+    assert lib.gdn_layer_prefill(ctypes.byref(L), *small) == 7
+    assert lib.gdn_layer_prefill(ctypes.byref(L), 0, 64, *args[2:]) == 0

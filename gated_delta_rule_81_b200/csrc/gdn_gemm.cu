@@ -7,15 +7,16 @@
 // to the hidden size through one output projection.  Both are plain matrix products,
 // which this file computes on the tensor cores.
 //
-// One persistent CTA per SM walks 128 x 256 output tiles (M fastest, so the CTAs
+// One persistent CTA per SM walks 128 x BN output tiles (M fastest, so the CTAs
 // running at the same time share B tiles through L2).  Per tile and 64-wide K step,
-// warp 0 lane 0 loads the A (128 x 64) and B (256 x 64) boxes with TMA (128-byte
-// swizzle, zero fill past the matrix edges) into a 4-stage ring; warp 1 lane 0
-// issues four tcgen05.mma (M 128, N 256, K 16) per step into one of two 256-column
-// fp32 accumulators in tensor memory; warps 2-5 read the other accumulator
+// warp 0 lane 0 loads the A (128 x 64) and B (BN x 64) boxes with TMA (128-byte
+// swizzle, zero fill past the matrix edges) into a ring of stages; warp 1 lane 0
+// issues four tcgen05.mma (M 128, N BN, K 16) per step into one of two fp32
+// accumulators in tensor memory (columns 0 and 256); warps 2-5 read the other accumulator
 // (thread = row, lane quarter = warp % 4), round to bf16 and store, so each tile's
-// epilogue overlaps the next tile's products.  Every wait is bounded: a stuck
-// wait sets error bit 1 and the CTA unwinds (draining its copies and products).
+// epilogue overlaps the next tile's products.  BN (256, 224, 192 or 160) is chosen
+// per shape (gemm_tile_width) so that the last round of tiles is not mostly idle.  Every wait is bounded: a
+// stuck wait sets error bit 1 and the CTA unwinds (draining its copies and products).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -25,14 +26,20 @@ namespace gdn {
 
 namespace {
 
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kGemmBM = 128, kGemmBK = 64;
 constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 16 KiB
-constexpr int kGemmBBytes = kGemmBN * kGemmBK * 2;  // 32 KiB
-constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
-constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 constexpr int kGemmEpiWarps = 4;
+constexpr int kGemmSmemBudget = 220 * 1024;
+
+template <int BN>
+struct GemmTile {
+  static constexpr int kBBytes = BN * kGemmBK * 2;
+  static constexpr int kStageBytes = kGemmABytes + kBBytes;
+  static constexpr int kStages = (kGemmSmemBudget - 1024) / kStageBytes > 6 ? 6 : (kGemmSmemBudget - 1024) / kStageBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 1024;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
+};
 
 struct GemmParams {
   int M, N, K;
@@ -55,9 +62,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                      GemmParams g) {
+  constexpr int kGemmBN = BN, kGemmStages = GemmTile<BN>::kStages, kGemmStageBytes = GemmTile<BN>::kStageBytes;
   extern __shared__ uint8_t gemm_smem_raw[];
   uint8_t* sm = gemm_align1024(gemm_smem_raw);
   __shared__ uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_empty[2], drain_b;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int b = tile_i & 1, buse = tile_i >> 1;
         if (buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1, ab)) break;
         tc_fence_after();
-        const uint32_t d = tbase + static_cast<uint32_t>(b * kGemmBN);
+        const uint32_t d = tbase + static_cast<uint32_t>(b * 256);
         for (int kk = 0; kk < k_steps; ++kk, ++it) {
           const int s = static_cast<int>(it % kGemmStages);
           if (!mbar_wait(&full[s], static_cast<uint32_t>((it / kGemmStages) & 1), ab)) {
@@ -163,7 +172,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kGemmBN / 32; ++c) {
         float v[32];
-        tmem_ld32(tmem_addr(tbase, 32 * q, static_cast<uint32_t>(b * kGemmBN + 32 * c)), v);
+        tmem_ld32(tmem_addr(tbase, 32 * q, static_cast<uint32_t>(b * 256 + 32 * c)), v);
         tmem_wait_ld();
         const int col = n0 + 32 * c;
         if (row < g.M && col < g.N) {
@@ -214,34 +223,70 @@ bool encode_kmajor(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, cons
 
 }  // namespace
 
-cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
-                             int M, int N, int K, int* err, cudaStream_t stream) {
-  static_assert(kGemmSmem <= 227 * 1024, "GEMM shared memory");
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
+namespace {
+
+template <int BN>
+cudaError_t launch_gemm_tile(PFN_cuTensorMapEncodeTiled_v12000 enc, const bf16* A, long long lda, const bf16* B,
+                             long long ldb, bf16* C, long long ldc, int M, int N, int K, int* err, int n_sm,
+                             cudaStream_t stream) {
   CUtensorMap ta, tb;
-  if (!encode_kmajor(enc, &ta, A, M, K, lda, kGemmBM) || !encode_kmajor(enc, &tb, B, N, K, ldb, kGemmBN))
+  if (!encode_kmajor(enc, &ta, A, M, K, lda, kGemmBM) || !encode_kmajor(enc, &tb, B, N, K, ldb, BN))
     return cudaErrorInvalidValue;
   GemmParams g;
   g.M = M;
   g.N = N;
   g.K = K;
   g.tiles_m = (M + kGemmBM - 1) / kGemmBM;
-  g.tiles_n = (N + kGemmBN - 1) / kGemmBN;
+  g.tiles_n = (N + BN - 1) / BN;
   g.C = C;
   g.ldc = ldc;
   g.err = err;
+  cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GemmTile<BN>::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long n_tiles = static_cast<long long>(g.tiles_m) * g.tiles_n;
+  const unsigned grid = static_cast<unsigned>(n_tiles < n_sm ? n_tiles : n_sm);
+  gemm_bf16_kernel<BN><<<grid, kGemmThreads, GemmTile<BN>::kSmem, stream>>>(ta, tb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// The tile width with the least time in its slowest CTA: rounds of tiles per SM times a
+// tile's time, which measures as growing with width + 512 (the A box and the per-step
+// hand-offs cost the same at every width); ties go to the wider tile.  At T = 4096 this
+// picks 256 for the input projection (N = 16480) and 224 for the output projection
+// (N = 5120: 5 rounds of 736 tiles instead of 5 of 640, the last one 32% full).
+int gemm_tile_width(int M, int N, int n_sm) {
+  static const int kWidths[] = {256, 224, 192, 160};
+  int best = 256;
+  long long best_cost = -1;
+  const long long tiles_m = (M + kGemmBM - 1) / kGemmBM;
+  for (int bn : kWidths) {
+    const long long tiles = tiles_m * ((N + bn - 1) / bn);
+    const long long cost = (tiles + n_sm - 1) / n_sm * (bn + 512);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
+                             int M, int N, int K, int* err, cudaStream_t stream) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
   int dev = 0, n_sm = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem)) !=
-      cudaSuccess)
-    return e;
-  const long long n_tiles = static_cast<long long>(g.tiles_m) * g.tiles_n;
-  const unsigned grid = static_cast<unsigned>(n_tiles < n_sm ? n_tiles : n_sm);
-  gemm_bf16_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ta, tb, g);
-  return cudaGetLastError();
+  switch (gemm_tile_width(M, N, n_sm)) {
+    case 224: return launch_gemm_tile<224>(enc, A, lda, B, ldb, C, ldc, M, N, K, err, n_sm, stream);
+    case 192: return launch_gemm_tile<192>(enc, A, lda, B, ldb, C, ldc, M, N, K, err, n_sm, stream);
+    case 160: return launch_gemm_tile<160>(enc, A, lda, B, ldb, C, ldc, M, N, K, err, n_sm, stream);
+    default: return launch_gemm_tile<256>(enc, A, lda, B, ldb, C, ldc, M, N, K, err, n_sm, stream);
+  }
 }
 
 }  // namespace gdn

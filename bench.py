@@ -56,8 +56,9 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {"scan": {"bytes": 442659072 + 44793088, "sha": "daba6480c7058e35"},   # ncu, T=4096 layer
-           "prep": {"bytes": 103497984 + 341519104, "sha": "daba6480c7058e35"}}
+TRAFFIC = {"scan": {"bytes": 442609664 + 44196608, "sha": "44d4966011593d14"},   # ncu, T=4096 layer
+           "prep": {"bytes": 101810688 + 334646272, "sha": "44d4966011593d14"},
+           "prefill_fused": {"bytes": 434084096 + 422704128, "sha": "44d4966011593d14"}}
 DECODE_TRAFFIC = {"bytes": 829675264 + 766249984, "sha": "852a2d42cccfe44d"}  # ncu, one step of 256 sequences
 
 

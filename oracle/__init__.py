@@ -16,3 +16,4 @@ from .gdn_oracle import (  # noqa: F401
 )
 from .chunked import chunked_recurrence  # noqa: F401
 from .projections import gemm, in_proj_layout, layer, round_bf16  # noqa: F401
+from . import attention as attn  # noqa: F401

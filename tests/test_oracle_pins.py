@@ -408,3 +408,106 @@ def test_layer_routes_projection_columns():
     o16 = torch.from_numpy(ref["out"]).to(torch.bfloat16).double().numpy().reshape(T, H_v * D)
     np.testing.assert_array_equal(res["y"][:, :H_v * D], o16)
     assert np.all(res["y"][:, H_v * D:] == 0)
+
+
+# ------------------------------------------------------------------ global-attention layer
+
+
+def test_rope_closed_forms():
+    """Position 0 is the identity; a basis vector e_i (i < 32) at position p turns into
+    cos(p theta_i) e_i + sin(p theta_i) e_{i+32} with theta_0 = 1; dims 64.. never move."""
+    A = oracle.attn
+    x = torch.randn(5, 2, 256, generator=torch.Generator().manual_seed(1), dtype=torch.float64)
+    np.testing.assert_allclose(A.rope(x, np.zeros(5)), x.numpy(), atol=0, rtol=0)
+    e = np.zeros((1, 1, 256))
+    e[0, 0, 0] = 1.0
+    for p in (1.0, 7.0, 1000.0):
+        r = A.rope(e, [p])
+        assert abs(r[0, 0, 0] - np.cos(p)) < 1e-12 and abs(r[0, 0, 32] - np.sin(p)) < 1e-12
+        assert np.count_nonzero(np.abs(r) > 1e-15) == 2
+    e2 = np.zeros((1, 1, 256))
+    e2[0, 0, 5] = 1.0
+    th = 1e7 ** (-5 / 32)
+    r = A.rope(e2, [3.0])
+    assert abs(r[0, 0, 5] - np.cos(3 * th)) < 1e-12 and abs(r[0, 0, 37] - np.sin(3 * th)) < 1e-12
+    r = A.rope(x, np.arange(5) * 11.0)
+    np.testing.assert_array_equal(r[..., 64:], x.numpy()[..., 64:])
+
+
+def test_rope_norm_and_relative_position():
+    """Rotations keep every pair's norm, and q_m . k_n depends on m - n only."""
+    A = oracle.attn
+    g = torch.Generator().manual_seed(2)
+    q = torch.randn(1, 1, 256, generator=g, dtype=torch.float64).numpy()
+    k = torch.randn(1, 1, 256, generator=g, dtype=torch.float64).numpy()
+    r = A.rope(q, [123.0])
+    np.testing.assert_allclose(r[..., :32] ** 2 + r[..., 32:64] ** 2, q[..., :32] ** 2 + q[..., 32:64] ** 2,
+                               rtol=1e-12)
+    d1 = (A.rope(q, [10.0]) * A.rope(k, [3.0])).sum()
+    d2 = (A.rope(q, [507.0]) * A.rope(k, [500.0])).sum()
+    assert abs(d1 - d2) < 1e-9 * abs(d1)
+
+
+def test_rms_norm_matches_library():
+    A = oracle.attn
+    x = torch.randn(7, 3, 256, generator=torch.Generator().manual_seed(3), dtype=torch.float64)
+    w = torch.rand(256, generator=torch.Generator().manual_seed(4), dtype=torch.float64) + 0.5
+    ref = F.rms_norm(x, (256,), w, eps=1e-6)
+    np.testing.assert_allclose(A.rms_norm(x, w), ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_matches_library_gqa_and_varlen():
+    """Causal GQA attention equals torch's scaled_dot_product_attention with the KV heads
+    repeated for their 6 query heads, per sequence; a packed call equals solo calls."""
+    A = oracle.attn
+    g = torch.Generator().manual_seed(5)
+    lens = [9, 1, 14]
+    T = sum(lens)
+    q = torch.randn(T, 24, 32, generator=g, dtype=torch.float64)
+    k = torch.randn(T, 4, 32, generator=g, dtype=torch.float64)
+    v = torch.randn(T, 4, 32, generator=g, dtype=torch.float64)
+    cu = [0, 9, 10, 24]
+    out = A.attention(q, k, v, cu)
+    for n in range(3):
+        s0, s1 = cu[n], cu[n + 1]
+        qq = q[s0:s1].transpose(0, 1)[None]
+        kk = k[s0:s1].repeat_interleave(6, dim=1).transpose(0, 1)[None]
+        vv = v[s0:s1].repeat_interleave(6, dim=1).transpose(0, 1)[None]
+        ref = F.scaled_dot_product_attention(qq, kk, vv, is_causal=True)[0].transpose(0, 1)
+        np.testing.assert_allclose(out[s0:s1], ref.numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(A.attention(q[s0:s1], k[s0:s1], v[s0:s1], [0, s1 - s0]), out[s0:s1],
+                                   rtol=0, atol=0)
+
+
+def test_attention_closed_forms():
+    """One token attends only to itself (output = v); with all keys equal the weights are
+    uniform, so each output is the mean of the values up to and including its position."""
+    A = oracle.attn
+    g = torch.Generator().manual_seed(6)
+    v = torch.randn(6, 4, 16, generator=g, dtype=torch.float64)
+    q = torch.randn(6, 24, 16, generator=g, dtype=torch.float64)
+    k1 = torch.randn(1, 4, 16, generator=g, dtype=torch.float64)
+    np.testing.assert_allclose(A.attention(q[:1], k1, v[:1], [0, 1])[0, 7], v[0, 1].numpy(), rtol=1e-14)
+    kc = k1.expand(6, 4, 16)
+    out = A.attention(q, kc, v, [0, 6])
+    prefix = np.cumsum(v.numpy(), axis=0) / np.arange(1, 7)[:, None, None]
+    for h in range(24):
+        np.testing.assert_allclose(out[:, h], prefix[:, h // 6], rtol=1e-12)
+
+
+def test_attn_mixer_gate_limits():
+    """A large positive gate passes the attention output, a zero gate halves it."""
+    A = oracle.attn
+    g = torch.Generator().manual_seed(7)
+    T = 5
+    q = torch.randn(T, 24, 256, generator=g).to(torch.bfloat16)
+    k = torch.randn(T, 4, 256, generator=g).to(torch.bfloat16)
+    v = torch.randn(T, 4, 256, generator=g).to(torch.bfloat16)
+    w = torch.ones(256, dtype=torch.bfloat16)
+    open_g = torch.full((T, 24, 256), 40.0).to(torch.bfloat16)
+    half_g = torch.zeros(T, 24, 256, dtype=torch.bfloat16)
+    a = A.attn_mixer(q, open_g, k, v, w, w, [0, T])
+    b = A.attn_mixer(q, half_g, k, v, w, w, [0, T])
+    o = A.attention(a["q_hat"], a["k_hat"], v, [0, T])
+    np.testing.assert_allclose(a["out"], o, rtol=1e-15)
+    np.testing.assert_allclose(b["out"], o / 2, rtol=1e-15)

@@ -256,6 +256,85 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
   return GDN_OK;
 }
 
+gdn_status gdn_attention_prefill(const void* q_hat, const void* k, const void* v, const void* g, long long ld_g,
+                                 int B, int T, void* out, int* err, void* stream) {
+  if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
+  if (T_tot == 0) return GDN_OK;
+  const long long hd = static_cast<long long>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
+  if (!q_hat || !k || !v || !g || !out || ld_g < hd) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q_hat) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out) || (ld_g & 7))
+    return GDN_ERR_MISALIGNED;
+  const size_t ob = static_cast<size_t>(T_tot) * hd * 2;
+  const size_t kvb = static_cast<size_t>(T_tot) * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM * 2;
+  if (overlap(out, ob, q_hat, ob) || overlap(out, ob, k, kvb) || overlap(out, ob, v, kvb) ||
+      overlap(out, ob, g, (static_cast<size_t>(T_tot - 1) * ld_g + hd) * 2))
+    return GDN_ERR_ALIAS;
+  return gdn::launch_flash_attn(static_cast<const bf16*>(q_hat), static_cast<const bf16*>(k),
+                                static_cast<const bf16*>(v), static_cast<const bf16*>(g), ld_g, B, T,
+                                static_cast<bf16*>(out), err, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? GDN_OK
+             : GDN_ERR_CUDA;
+}
+
+size_t gdn_attn_layer_workspace_size(int B, int T) {
+  if (B < 0 || T < 0) return 0;
+  const size_t T_tot = static_cast<size_t>(B) * T;
+  const size_t hd = static_cast<size_t>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
+  return round_up(T_tot * GDN_ATTN_N_IN * 2, 1024) + 2 * round_up(T_tot * hd * 2, 1024);
+}
+
+gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const void* x, long long ldx,
+                                  void* k_cache, void* v_cache, void* y, long long ldy, void* workspace,
+                                  size_t workspace_bytes, int* err, void* stream) {
+  if (!L || B < 0 || T < 0 || L->hidden <= 0) return GDN_ERR_INVALID_ARG;
+  if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
+  if (T_tot == 0) return GDN_OK;
+  if (!x || !y || !k_cache || !v_cache || !L->w_in || !L->w_out || !L->q_norm_w || !L->k_norm_w)
+    return GDN_ERR_INVALID_ARG;
+  if (ldy < L->hidden) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_attn_layer_workspace_size(B, T);
+  if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(L->q_norm_w) || !aligned16(L->k_norm_w) ||
+      !aligned16(workspace))
+    return GDN_ERR_MISALIGNED;
+  const size_t hd = static_cast<size_t>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
+  const size_t kv_bytes = static_cast<size_t>(T_tot) * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM * 2;
+  const size_t y_bytes = (static_cast<size_t>(T_tot - 1) * ldy + L->hidden) * 2;
+  if (overlap(y, y_bytes, workspace, need) || overlap(k_cache, kv_bytes, workspace, need) ||
+      overlap(v_cache, kv_bytes, workspace, need) || overlap(k_cache, kv_bytes, v_cache, kv_bytes) ||
+      overlap(y, y_bytes, k_cache, kv_bytes) || overlap(y, y_bytes, v_cache, kv_bytes))
+    return GDN_ERR_ALIAS;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  bf16* proj = reinterpret_cast<bf16*>(ws);
+  bf16* q_hat = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(T_tot) * GDN_ATTN_N_IN * 2, 1024));
+  bf16* att = reinterpret_cast<bf16*>(reinterpret_cast<uint8_t*>(q_hat) + round_up(static_cast<size_t>(T_tot) * hd * 2, 1024));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) {
+    if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
+  };
+  mark(0);
+  gdn_status s = gdn_gemm_bf16(x, ldx, L->w_in, L->ld_w_in, proj, GDN_ATTN_N_IN, static_cast<int>(T_tot),
+                               GDN_ATTN_N_IN, L->hidden, err, stream);
+  if (s != GDN_OK) return s;
+  mark(1);
+  if (gdn::launch_attn_qk(proj, GDN_ATTN_N_IN, static_cast<const bf16*>(L->q_norm_w),
+                          static_cast<const bf16*>(L->k_norm_w), B, T, q_hat, static_cast<bf16*>(k_cache),
+                          static_cast<bf16*>(v_cache), st) != cudaSuccess ||
+      gdn::launch_flash_attn(q_hat, static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache),
+                             proj + hd, GDN_ATTN_N_IN, B, T, att, err, st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  mark(2);
+  s = gdn_gemm_bf16(att, static_cast<long long>(hd), L->w_out, L->ld_w_out, y, ldy, static_cast<int>(T_tot),
+                    L->hidden, static_cast<int>(hd), err, stream);
+  if (s != GDN_OK) return s;
+  mark(3);
+  return GDN_OK;
+}
+
 gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,
                             const int* state_slot, int n_slots, void* out, int* err, void* stream) {
   if (N < 0 || T < 1 || T > gdn::kMaxDecodeTokens || n_slots < 0) return GDN_ERR_INVALID_ARG;

@@ -1,0 +1,441 @@
+// The global-attention layer of the hybrid decoder, between its two projections.
+//
+// Agnes-3.0-Flash model card, "Architecture" table: row "Global attention" (24 query
+// heads / 4 KV heads, 6 : 1 GQA, head dim 256, RMS-norm on q and k, sigmoid-gated
+// output) and row "Positions" (3-axis rotary, base 1e7, on the first 25 % of each head
+// dim = 64 dims); "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention Multimodal Model",
+// section "Attention Layer Details".  For text tokens the three rotary axes all carry
+// the token's position, so every one of the 32 frequencies turns by position * theta_i,
+// theta_i = 1e7^(-i/32), applied to the pairs (i, i + 32) of the first 64 dims.
+//
+// Two kernels:
+//   attn_qk_kernel     q_hat = rope(rms(q) w_q), k_hat = rope(rms(k) w_k) per head, both
+//                      stored bf16 (k_hat into the caller's K cache), v copied to the V cache;
+//   flash_attn_kernel  causal softmax attention, GQA, on the tensor cores, with the output
+//                      gate o * sigmoid(g) in its epilogue.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "gdn_kernels.cuh"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kAD = 256;          // head dim
+constexpr int kAHq = 24, kAHkv = 4, kAGrp = kAHq / kAHkv;
+constexpr int kARope = 64;        // rotary dims per head
+constexpr double kARopeBase = 1e7;
+
+// ------------------------------------------------------------ q / k norm and rotary
+//
+// One warp per (token, head): lane l holds dims 8l .. 8l+7 (16-byte loads); the rotary
+// pairs (i, i + 32) of dims 0 .. 63 sit in lanes l and l ^ 4 (l < 8).  The angles are
+// formed and reduced modulo 2 pi in fp64 (positions reach 262,144), then sincosf.
+constexpr int kQkThreads = 256;
+
+__device__ __forceinline__ void unpack8f(uint4 u, float* f) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8f(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+struct AttnQkParams {
+  const bf16* proj;  // [T_tot][ld_p]: q | g | k | v
+  long long ld_p;
+  const bf16* q_norm_w;  // [256]
+  const bf16* k_norm_w;
+  int T;                 // tokens per sequence (position = token index mod T)
+  long long T_tot;
+  bf16* q_hat;           // [T_tot][24][256]
+  bf16* k_cache;         // [T_tot][4][256]
+  bf16* v_cache;         // [T_tot][4][256]
+};
+
+__global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long item = static_cast<long long>(blockIdx.x) * (kQkThreads / 32) + warp;  // (token, head)
+  constexpr int kHeads = kAHq + kAHkv + kAHkv;  // q heads, k heads, v heads
+  if (item >= p.T_tot * kHeads) return;
+  const long long t = item / kHeads;
+  const int hh = static_cast<int>(item % kHeads);
+  const bf16* row = p.proj + t * p.ld_p;
+  if (hh >= kAHq + kAHkv) {  // v: a copy into the cache
+    const int h = hh - kAHq - kAHkv;
+    const uint4 u = reinterpret_cast<const uint4*>(row + 2 * kAHq * kAD + kAHkv * kAD + h * kAD)[lane];
+    reinterpret_cast<uint4*>(p.v_cache + (t * kAHkv + h) * kAD)[lane] = u;
+    return;
+  }
+  const bool is_q = hh < kAHq;
+  const int h = is_q ? hh : hh - kAHq;
+  const bf16* src = is_q ? row + h * kAD : row + 2 * kAHq * kAD + h * kAD;
+  float x[8], w[8];
+  unpack8f(reinterpret_cast<const uint4*>(src)[lane], x);
+  unpack8f(reinterpret_cast<const uint4*>(is_q ? p.q_norm_w : p.k_norm_w)[lane], w);
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss * (1.0f / kAD) + 1e-6f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = x[e] * inv * w[e];
+  // rotary on dims 0 .. 63 (lanes 0 .. 7): lane l < 4 holds x1 = dims 8l.., lane l + 4 holds x2
+  float partner[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, x[e], 4);
+  if (lane < 8) {
+    const double pos = static_cast<double>(t % p.T);
+    const int i0 = 8 * (lane & 3);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const double theta = exp(-static_cast<double>(i0 + e) / (kARope / 2) * log(kARopeBase));
+      const double ang = fmod(pos * theta, 6.283185307179586476925286766559);
+      float sn, cs;
+      sincosf(static_cast<float>(ang), &sn, &cs);
+      // x1' = x1 c - x2 s (lanes 0..3), x2' = x2 c + x1 s (lanes 4..7)
+      x[e] = lane < 4 ? fmaf(x[e], cs, -partner[e] * sn) : fmaf(x[e], cs, partner[e] * sn);
+    }
+  }
+  bf16* dst = is_q ? p.q_hat + (t * kAHq + h) * kAD : p.k_cache + (t * kAHkv + h) * kAD;
+  reinterpret_cast<uint4*>(dst)[lane] = pack8f(x);
+}
+
+// ------------------------------------------------------------ causal flash attention
+//
+// One CTA per (query tile of 128 tokens, query head); tiles of one sequence go longest
+// first.  Warps 0-3: softmax and epilogue (thread = query row, TMEM lane quarter = warp);
+// warp 4 lane 0: TMA (Q once, then K and V tiles of 64 keys into a 2-stage ring); warp 5
+// lane 0: tcgen05.mma.  Per key tile j:
+//   S_j  = Q K_j^T            M 128, N 64, K 256   (16 MMAs; A, B K-major from shared memory)
+//   P_j  = exp2(S_j log2(e)/16 - m)                (softmax warps; bf16 pairs into TMEM)
+//   O   += P_j V_j            M 128, N 256, K 64   (4 MMAs; A = P from TMEM, B = V MN-major)
+// S is double-buffered in TMEM, so S_{j+1} runs while the softmax works on S_j.  The
+// running max is lazy: O and l are rescaled only when a row's max grows by more than 8
+// (log2 units), after waiting for the products still writing O; the final 1/l makes the
+// result exact either way.  Masked scores (key past the query) are -inf.  Epilogue:
+// o / l * sigmoid(g) in bf16 into [T_tot][24 * 256].  Every wait is bounded.
+constexpr int kFaBM = 128, kFaBN = 64;
+constexpr int kFaThreads = 192;
+constexpr int kFaQBytes = kFaBM * kAD * 2;          // 64 KiB: 4 boxes of 128 rows x 64 dims
+constexpr int kFaKBytes = kFaBN * kAD * 2;          // 32 KiB: 4 boxes of 64 keys x 64 dims
+constexpr int kFaStageBytes = 2 * kFaKBytes;        // K | V
+constexpr int kFaSmem = kFaQBytes + 2 * kFaStageBytes + 1024;
+// tensor memory columns
+constexpr uint32_t kFaColO = 0;      // 256 fp32 columns
+constexpr uint32_t kFaColS = 256;    // 2 x 64
+constexpr uint32_t kFaColP = 384;    // 2 x 32 (bf16 pairs)
+constexpr float kFaRescale = 8.0f;   // lazy rescale threshold (log2 units)
+
+struct FaParams {
+  int T;              // tokens per sequence
+  int B;              // sequences
+  int tiles;          // query tiles per sequence
+  const bf16* g;      // gate: head h of token t at g + t * ld_g + h * 256
+  long long ld_g;
+  bf16* out;          // [T_tot][24*256]
+  int* err;
+  float scale_log2e;  // log2(e) / sqrt(256)
+};
+
+__device__ __forceinline__ uint8_t* fa_align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void fa_tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kFaThreads, 1)
+    flash_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, FaParams p) {
+  extern __shared__ uint8_t fa_smem_raw[];
+  uint8_t* sm = fa_align1024(fa_smem_raw);
+  uint8_t* sQ = sm;
+  uint8_t* sKV = sm + kFaQBytes;  // stage s: K at s * kFaStageBytes, V after it
+  __shared__ uint64_t q_full, kv_full[2], kv_free[2], s_full[2], p_full[2], pv_done[2], drain_b;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // work item: head h, sequence n, query tile mt (longest tiles first)
+  const int h = blockIdx.y;
+  const int n = blockIdx.x % p.B;
+  const int mt = p.tiles - 1 - static_cast<int>(blockIdx.x / p.B);
+  const int m0 = mt * kFaBM;                                  // first query position in the sequence
+  const int n_kv = min((m0 + kFaBM + kFaBN - 1) / kFaBN, (p.T + kFaBN - 1) / kFaBN);  // key tiles (causal)
+  const int kvh = h / kAGrp;
+  const int row0 = n * p.T;                                   // first token of the sequence
+
+  const Abort ab{p.err, &abort_s};
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(&q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&kv_full[b], 1);
+      mbar_init(&kv_free[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(&drain_b, 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) tmem_alloc<512>(&tmem_base_s);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      mbar_arrive_expect_tx(&q_full, kFaQBytes);
+      for (int kb = 0; kb < 4; ++kb)
+        fa_tma_load_2d(sQ + kb * (kFaBM * 128), &tm_q, h * kAD + kb * 64, row0 + m0, &q_full);
+      int issued[2] = {0, 0};
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&kv_free[s], ((j - 2) >> 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&kv_full[s], kFaStageBytes);
+        uint8_t* st = sKV + s * kFaStageBytes;
+        for (int kb = 0; kb < 4; ++kb) {
+          fa_tma_load_2d(st + kb * (kFaBN * 128), &tm_k, kvh * kAD + kb * 64, row0 + j * kFaBN, &kv_full[s]);
+          fa_tma_load_2d(st + kFaKBytes + kb * (kFaBN * 128), &tm_v, kvh * kAD + kb * 64, row0 + j * kFaBN,
+                         &kv_full[s]);
+        }
+        ++issued[s];
+      }
+      // copies still in flight (only after an abort) land before the CTA exits
+      int drain_flag = 0;
+      const Abort drain{nullptr, &drain_flag};
+      mbar_wait(&q_full, 0, drain);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s] > 0) mbar_wait(&kv_full[s], (issued[s] - 1) & 1, drain);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      const uint32_t idesc_s = idesc_bf16(kFaBM, kFaBN, false, false);  // Q K^T
+      const uint32_t idesc_o = idesc_bf16(kFaBM, kAD, false, true);     // P V, V MN-major (N = d)
+      const uint32_t q_s = smem_u32(sQ);
+      bool ok = mbar_wait(&q_full, 0, ab);
+      auto issue_pv = [&](int i) -> bool {  // O += P_i V_i
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t v_s = smem_u32(sKV + (i & 1) * kFaStageBytes + kFaKBytes);
+#pragma unroll
+        for (int ks = 0; ks < kFaBN / 16; ++ks)
+          umma_bf16_ts(tbase + kFaColO, tbase + kFaColP + 32u * (i & 1) + 8u * ks,
+                       smem_desc(v_s + ks * 2048u, kFaBN * 128, 1024, Swz::k128), idesc_o, i > 0 || ks > 0);
+        umma_commit(&pv_done[i & 1]);
+        umma_commit(&kv_free[i & 1]);
+        return true;
+      };
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, ab)) break;
+        // S buffer s was last read by the softmax of tile j - 2 (its p_full has arrived)
+        if (j >= 2 && !mbar_wait(&p_full[s], ((j - 2) >> 1) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t k_s = smem_u32(sKV + s * kFaStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < kAD / 16; ++ks) {
+          const uint32_t off_q = (ks >> 2) * (kFaBM * 128u) + (ks & 3) * 32u;
+          const uint32_t off_k = (ks >> 2) * (kFaBN * 128u) + (ks & 3) * 32u;
+          umma_bf16(tbase + kFaColS + 64u * s, smem_desc(q_s + off_q, 16, 1024, Swz::k128),
+                    smem_desc(k_s + off_k, 16, 1024, Swz::k128), idesc_s, ks > 0);
+        }
+        umma_commit(&s_full[s]);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && n_kv > 0) issue_pv(n_kv - 1);
+      umma_commit(&drain_b);
+      int drain_flag = 0;
+      const Abort drain{nullptr, &drain_flag};
+      mbar_wait(&drain_b, 0, drain);
+    }
+  } else {
+    // ------------------------------------------------ softmax + epilogue: thread = query row
+    const int r = 32 * warp + lane;  // warps 0-3: lane quarter = warp
+    const int qpos = m0 + r;
+    const uint32_t trow = tmem_addr(tbase, 32 * warp, 0);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait_warp(&s_full[s], (j >> 1) & 1, ab)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[kFaBN];
+      tmem_ld32(trow + kFaColS + 64u * s, sv);
+      tmem_ld32(trow + kFaColS + 64u * s + 32u, sv + 32);
+      tmem_wait_ld();
+      const int k0 = j * kFaBN;
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kFaBN; ++c) {
+        const float x = (k0 + c <= qpos) ? sv[c] * p.scale_log2e : -INFINITY;
+        sv[c] = x;
+        mloc = fmaxf(mloc, x);
+      }
+      // P buffer s was read by the products of tile j - 2
+      if (j >= 2 && !mbar_wait_warp(&pv_done[s], ((j - 2) >> 1) & 1, ab)) {
+        ok = false;
+        break;
+      }
+      // the rescale is decided per warp (its waits and tensor-memory accesses are warp-collective):
+      // lanes whose max grew by more than the threshold take the new max, the others keep theirs
+      const bool grow = mloc > m + kFaRescale;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_new = grow ? mloc : m;
+        if (j >= 1) {
+          // rescale the warp's rows of O once the products of tile j - 1 have written them
+          if (!mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = exp2f(m - m_new);  // 1 for lanes keeping their max
+#pragma unroll 1
+          for (int c = 0; c < kAD / 32; ++c) {
+            float o[32];
+            tmem_ld32(trow + kFaColO + 32u * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tmem_st32(trow + kFaColO + 32u * c, o);
+          }
+          l *= f;
+        }
+        m = m_new;
+      }
+      uint32_t pk[kFaBN / 2];
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kFaBN / 2; ++c) {
+        const float p0 = exp2f(sv[2 * c] - m), p1 = exp2f(sv[2 * c + 1] - m);
+        lsum += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l += lsum;
+      tmem_st16(trow + kFaColP + 32u * s, pk);
+      tmem_st16(trow + kFaColP + 32u * s + 16u, pk + 16);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
+    }
+    // epilogue: the last tile's products complete every write to O
+    if (ok && n_kv > 0 && mbar_wait_warp(&pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, ab)) {
+      tc_fence_after();
+      const bool valid = qpos < p.T;
+      const long long tok = static_cast<long long>(row0) + qpos;
+      const float inv_l = 1.0f / l;
+      const bf16* grow = p.g + tok * p.ld_g + h * kAD;
+      bf16* orow = p.out + tok * (kAHq * kAD) + h * kAD;
+#pragma unroll 1
+      for (int c = 0; c < kAD / 32; ++c) {
+        float o[32];
+        tmem_ld32(trow + kFaColO + 32u * c, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float gf[8], y[8];
+            unpack8f(reinterpret_cast<const uint4*>(grow + 32 * c)[u], gf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = o[8 * u + e] * inv_l / (1.0f + __expf(-gf[e]));
+            reinterpret_cast<uint4*>(orow + 32 * c)[u] = pack8f(y);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc<512>(tbase);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// bf16 [rows][ld] as 64-column x box_rows boxes, 128-byte swizzle, zero fill past the edges
+bool attn_encode(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, long long rows,
+                 long long cols, long long ld, int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_w, const bf16* k_norm_w, int B,
+                           int T, bf16* q_hat, bf16* k_cache, bf16* v_cache, cudaStream_t stream) {
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot == 0) return cudaSuccess;
+  AttnQkParams qp;
+  qp.proj = proj;
+  qp.ld_p = ld_p;
+  qp.q_norm_w = q_norm_w;
+  qp.k_norm_w = k_norm_w;
+  qp.T = T;
+  qp.T_tot = T_tot;
+  qp.q_hat = q_hat;
+  qp.k_cache = k_cache;
+  qp.v_cache = v_cache;
+  const long long items = T_tot * (kAHq + 2 * kAHkv);
+  attn_qk_kernel<<<static_cast<unsigned>((items + kQkThreads / 32 - 1) / (kQkThreads / 32)), kQkThreads, 0,
+                   stream>>>(qp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, const bf16* g, long long ld_g, int B,
+                              int T, bf16* out, int* err, cudaStream_t stream) {
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot == 0) return cudaSuccess;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = attn_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tq, tk, tv;
+  if (!attn_encode(enc, &tq, q_hat, T_tot, kAHq * kAD, kAHq * kAD, kFaBM) ||
+      !attn_encode(enc, &tk, k, T_tot, kAHkv * kAD, kAHkv * kAD, kFaBN) ||
+      !attn_encode(enc, &tv, v, T_tot, kAHkv * kAD, kAHkv * kAD, kFaBN))
+    return cudaErrorInvalidValue;
+  FaParams fp;
+  fp.T = T;
+  fp.B = B;
+  fp.tiles = (T + kFaBM - 1) / kFaBM;
+  fp.g = g;
+  fp.ld_g = ld_g;
+  fp.out = out;
+  fp.err = err;
+  fp.scale_log2e = 1.4426950408889634f / 16.0f;  // log2(e) / sqrt(256)
+  cudaError_t e = cudaFuncSetAttribute(flash_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmem);
+  if (e != cudaSuccess) return e;
+  flash_attn_kernel<<<dim3(static_cast<unsigned>(fp.tiles * B), kAHq), kFaThreads, kFaSmem, stream>>>(tq, tk, tv, fp);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

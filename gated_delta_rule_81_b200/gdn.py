@@ -53,6 +53,21 @@ class GdnLayer(ctypes.Structure):
     ]
 
 
+class GdnAttnLayer(ctypes.Structure):
+    """gdn_attn_layer: the weights of one global-attention layer (device pointers)."""
+    _fields_ = [
+        ("w_in", ctypes.c_void_p), ("ld_w_in", ctypes.c_longlong),
+        ("w_out", ctypes.c_void_p), ("ld_w_out", ctypes.c_longlong),
+        ("q_norm_w", ctypes.c_void_p), ("k_norm_w", ctypes.c_void_p),
+        ("hidden", ctypes.c_int),
+        ("events", ctypes.c_void_p),
+    ]
+
+
+ATTN_Q_HEADS, ATTN_KV_HEADS, ATTN_HEAD_DIM = 24, 4, 256
+ATTN_N_IN = 2 * 24 * 256 + 2 * 4 * 256
+
+
 SCHEDULE_AUTO = 0          # one overlapped launch when it pays (few scan units, many prep items)
 SCHEDULE_TWO_LAUNCHES = 1  # prep kernel, then scan kernel
 SCHEDULE_FUSED = 2         # one overlapped launch whenever the scan units fit in half the SMs
@@ -63,6 +78,7 @@ _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_lon
 
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
            "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
+           "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
            "gdn_status_string")
 MAX_DECODE_TOKENS = 8
 
@@ -96,6 +112,13 @@ def load(path: str | None = None):
     lib.gdn_layer_prefill.argtypes = [ctypes.POINTER(GdnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _vp, _vp, _ll, _vp,
                                       _sz, _vp, _vp]
     lib.gdn_layer_prefill.restype = _i
+    lib.gdn_attn_layer_workspace_size.argtypes = [_i, _i]
+    lib.gdn_attn_layer_workspace_size.restype = _sz
+    lib.gdn_attn_layer_prefill.argtypes = [ctypes.POINTER(GdnAttnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _ll, _vp,
+                                           _sz, _vp, _vp]
+    lib.gdn_attn_layer_prefill.restype = _i
+    lib.gdn_attention_prefill.argtypes = [_vp, _vp, _vp, _vp, _ll, _i, _i, _vp, _vp, _vp]
+    lib.gdn_attention_prefill.restype = _i
     lib.gdn_status_string.argtypes = [_i]
     lib.gdn_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -297,6 +320,49 @@ def layer_prefill(L: GdnLayer, B: int, T: int, x, state_in=None, conv_in=None, *
                                  _ptr(conv_in), _ptr(conv_out), _ptr(y), y.stride(0), _ptr(workspace),
                                  workspace.numel(), _ptr(err), _stream()), "gdn_layer_prefill")
     return y, state_out, conv_out
+
+
+def make_attn_layer(w_in, w_out, q_norm_w, k_norm_w) -> GdnAttnLayer:
+    """gdn_attn_layer from device tensors: w_in bf16 [ATTN_N_IN][hidden], w_out bf16 [hidden][24*256]."""
+    for name, t in (("w_in", w_in), ("w_out", w_out), ("q_norm_w", q_norm_w), ("k_norm_w", k_norm_w)):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise TypeError(f"{name} must be bf16 with a contiguous last dimension")
+    L = GdnAttnLayer()
+    L.w_in, L.ld_w_in = w_in.data_ptr(), w_in.stride(0)
+    L.w_out, L.ld_w_out = w_out.data_ptr(), w_out.stride(0)
+    L.q_norm_w, L.k_norm_w = q_norm_w.data_ptr(), k_norm_w.data_ptr()
+    L.hidden = int(w_in.shape[1])
+    return L
+
+
+def attn_layer_prefill(L: GdnAttnLayer, B: int, T: int, x, *, y=None, k_cache=None, v_cache=None, workspace=None,
+                       err=None):
+    """gdn_attn_layer_prefill.  Returns (y, k_cache, v_cache)."""
+    lib = load()
+    dev = x.device
+    if y is None:
+        y = torch.empty(B * T, L.hidden, dtype=torch.bfloat16, device=dev)
+    if k_cache is None:
+        k_cache = torch.empty(B * T, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    if v_cache is None:
+        v_cache = torch.empty(B * T, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(int(lib.gdn_attn_layer_workspace_size(B, T)), dtype=torch.uint8, device=dev)
+    _check(lib.gdn_attn_layer_prefill(ctypes.byref(L), B, T, _ptr(x), x.stride(0), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(y), y.stride(0), _ptr(workspace), workspace.numel(), _ptr(err),
+                                      _stream()), "gdn_attn_layer_prefill")
+    return y, k_cache, v_cache
+
+
+def attention_prefill(q_hat, k, v, g, B: int, T: int, out=None, err=None):
+    """gdn_attention_prefill on device tensors q_hat [B*T,24,256], k, v [B*T,4,256], g (rows of >= 24*256)."""
+    lib = load()
+    if out is None:
+        out = torch.empty(B * T, ATTN_Q_HEADS * ATTN_HEAD_DIM, dtype=torch.bfloat16, device=q_hat.device)
+    g2 = g.reshape(g.shape[0], -1) if g.dim() == 3 else g
+    _check(lib.gdn_attention_prefill(_ptr(q_hat), _ptr(k), _ptr(v), _ptr(g2), g2.stride(0), B, T, _ptr(out),
+                                     _ptr(err), _stream()), "gdn_attention_prefill")
+    return out
 
 
 def status_string(status: int) -> str:

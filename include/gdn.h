@@ -205,6 +205,59 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
                              void* workspace, size_t workspace_bytes, int* err, void* stream);
 
 /*
+ * The global-attention layer of the hybrid decoder (the fourth layer of every four):
+ * 24 query heads / 4 KV heads of dimension 256, RMS-norm on q and k, rotary position
+ * on the first 64 dims of each head (positions = token index within its sequence,
+ * base 1e7, pairs (i, i + 32)), causal softmax attention, output * sigmoid(gate).
+ * The input projection's output channels: q (24*256) | gate (24*256) | k (4*256) | v (4*256).
+ */
+#define GDN_ATTN_Q_HEADS 24
+#define GDN_ATTN_KV_HEADS 4
+#define GDN_ATTN_HEAD_DIM 256
+#define GDN_ATTN_N_IN (2 * GDN_ATTN_Q_HEADS * GDN_ATTN_HEAD_DIM + 2 * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM)
+typedef struct {
+  const void* w_in;       /* bf16 [GDN_ATTN_N_IN][ld_w_in], first `hidden` columns used */
+  long long ld_w_in;
+  const void* w_out;      /* bf16 [hidden][ld_w_out], first 24*256 columns used */
+  long long ld_w_out;
+  const void* q_norm_w;   /* bf16 [256] */
+  const void* k_norm_w;   /* bf16 [256] */
+  int hidden;             /* a multiple of 64 */
+  void* const* events;    /* optional timing hook: NULL or 4 cudaEvent_t, recorded before the input
+                             projection, after it, after the attention, after the output projection */
+} gdn_attn_layer;
+
+/*
+ * The attention itself, for B sequences of T tokens (packed [B*T]), on given operands:
+ *   q_hat  bf16 [B*T][24][256]  normalised, rotated queries
+ *   k, v   bf16 [B*T][4][256]   normalised, rotated keys and values (a KV cache)
+ *   g      bf16, gate of head h of token t at g + t*ld_g + h*256
+ *   out    bf16 [B*T][24*256] = softmax(q_hat k^T / 16, causal within each sequence) v * sigmoid(g),
+ *          query head h reading KV head h / 6.
+ * The probabilities enter the tensor cores as bf16 (relative error <= 2^-8 each).
+ */
+gdn_status gdn_attention_prefill(const void* q_hat, const void* k, const void* v, const void* g, long long ld_g,
+                                 int B, int T, void* out, int* err, void* stream);
+
+/* Workspace bytes of gdn_attn_layer_prefill for B sequences of T tokens. */
+size_t gdn_attn_layer_workspace_size(int B, int T);
+
+/*
+ * Prefill of the attention layer for B sequences of T tokens each (packed [B*T]):
+ *   x  bf16 [B*T][ldx] -> y bf16 [B*T][ldy] (first `hidden` columns);
+ *   k_cache, v_cache  bf16 [B*T][4][256], written: the normalised, rotated keys and the
+ *   values, i.e. the layer's KV cache after the prompt.
+ * Launches: gdn_gemm_bf16 (in_proj), the q/k norm + rotary kernel, the flash-attention
+ * kernel (tcgen05, gate in its epilogue), gdn_gemm_bf16 (out_proj).  Errors as the
+ * other entry points; y, the caches and the workspace must not overlap.  The workspace
+ * holds, each from a 1 KiB boundary: the projection [B*T][GDN_ATTN_N_IN], q_hat
+ * [B*T][24][256] and the attention output [B*T][24*256] (readable after the call).
+ */
+gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const void* x, long long ldx,
+                                  void* k_cache, void* v_cache, void* y, long long ldy, void* workspace,
+                                  size_t workspace_bytes, int* err, void* stream);
+
+/*
  * T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N sequences in one call
  * (decode with several tokens per step, e.g. verifying drafted tokens), with
  * the states held in slots of a state pool.  Token n * T + t of the inputs is

@@ -426,6 +426,80 @@ def run_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120, H_k=16, H_v=
             "cublas_ms": cub, "flops": flops, "clocks": clk.report(), "steps": args.steps}
 
 
+def run_attn_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120):
+    """One global-attention layer (24/4 GQA, head dim 256), B = 1, T = 4096, hidden 5120, random
+    dense weights (std 1/sqrt(fan_in)); times in_proj, attention (norm + rotary + flash) and
+    out_proj with the layer's event hook, and torch's scaled_dot_product_attention (GQA,
+    causal) on the same q, k, v shapes beside."""
+    from gated_delta_rule_81_b200 import gdn
+
+    g = torch.Generator().manual_seed(200 + rank)
+    x = torch.randn(T, hidden, generator=g).to(torch.bfloat16).to(dev)
+    w_in = (torch.randn(gdn.ATTN_N_IN, hidden, generator=g) * hidden ** -0.5).to(torch.bfloat16).to(dev)
+    w_out = (torch.randn(hidden, 24 * 256, generator=g) * (24 * 256) ** -0.5).to(torch.bfloat16).to(dev)
+    qn = (1.0 + 0.1 * torch.randn(256, generator=g)).to(torch.bfloat16).to(dev)
+    kn = (1.0 + 0.1 * torch.randn(256, generator=g)).to(torch.bfloat16).to(dev)
+    L = gdn.make_attn_layer(w_in, w_out, qn, kn)
+    y = torch.empty(T, hidden, dtype=torch.bfloat16, device=dev)
+    kc = torch.empty(T, 4, 256, dtype=torch.bfloat16, device=dev)
+    vc = torch.empty(T, 4, 256, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(int(gdn.load().gdn_attn_layer_workspace_size(1, T)), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.attn_layer_prefill(L, 1, T, x, y=y, k_cache=kc, v_cache=vc, workspace=ws, err=err)
+
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for ev in evs:
+            flush_l2(flush)
+            arr = (ctypes.c_void_p * 4)(*[e.cuda_event or (e.record(stream) or e.cuda_event) for e in ev])
+            L.events = ctypes.cast(arr, ctypes.c_void_p)
+            step()
+        torch.cuda.synchronize()
+    L.events = None
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    parts = {"in_proj": [e[0].elapsed_time(e[1]) for e in evs], "attention": [e[1].elapsed_time(e[2]) for e in evs],
+             "out_proj": [e[2].elapsed_time(e[3]) for e in evs]}
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    # torch SDPA on the same shapes (q [1, 24, T, 256], k / v [1, 4, T, 256], causal, GQA)
+    q_t = torch.randn(1, 24, T, 256, device=dev).to(torch.bfloat16)
+    k_t = torch.randn(1, 4, T, 256, device=dev).to(torch.bfloat16)
+    v_t = torch.randn(1, 4, T, 256, device=dev).to(torch.bfloat16)
+    sdpa_ms = None
+    try:
+        for _ in range(3):
+            torch.nn.functional.scaled_dot_product_attention(q_t, k_t, v_t, is_causal=True, enable_gqa=True)
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(10):
+            flush_l2(flush)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch.nn.functional.scaled_dot_product_attention(q_t, k_t, v_t, is_causal=True, enable_gqa=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        sdpa_ms = tot / 10
+    except RuntimeError as exc:  # no fused kernel for this shape on this build
+        print(f"note: torch SDPA unavailable for the comparison: {exc}", file=sys.stderr)
+    n_in = gdn.ATTN_N_IN
+    flops = {"in_proj": 2 * T * hidden * n_in, "out_proj": 2 * T * 24 * 256 * hidden,
+             "attention": 2 * 2 * 24 * 256 * T * (T + 1) // 2}  # causal QK^T and PV
+    return {"total_ms": total_ms, "T": T, "parts_ms": {k: statistics.mean(v) for k, v in parts.items()},
+            "sdpa_ms": sdpa_ms, "flops": flops, "clocks": clk.report(), "steps": args.steps}
+
+
 # ------------------------------------------------------------------ oracle (CPU) arm
 
 
@@ -488,7 +562,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer"], default="prefill4k",
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "attn_layer"], default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
@@ -527,6 +601,31 @@ def main():
                                            "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"],
                                            "traffic": decode_traffic() if d["T"] == 1 else None},
                               "gpu_launches": d["launches"]}), flush=True)
+        return 0
+    if args.workload == "attn_layer":
+        r = run_attn_layer_ours(args, world, rank, dev, pk)
+        if rank == 0:
+            pm = r["parts_ms"]
+            tf = {k: r["flops"][k] / (pm[k] * 1e-3) / 1e12 for k in pm}
+            ms_step = r["total_ms"] / r["steps"]
+            print(json.dumps({
+                "metric": "attention-layer prefill tokens/s (in_proj + norm/rotary + flash attention + out_proj)",
+                "value": world * r["T"] * r["steps"] / (r["total_ms"] / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": r["steps"], "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "attention-layer-prefill-T4096-hidden5120-24x4x256", "batch": 1,
+                           "seq_len": r["T"], "hidden": 5120, "q_heads": 24, "kv_heads": 4, "head_dim": 256,
+                           "weights": "random dense, std 1/sqrt(fan_in)", "l2": "flushed between timed steps"},
+                "roofline": {"kernel": "attention (norm/rotary + flash_attn_kernel)", "bound": "tensor",
+                             "achieved": tf["attention"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf["attention"] / pk["bf16_tflops"], "traffic": None,
+                             "peak_source": f"{pk['source']} (bf16 burst)",
+                             "algorithmic_flop_per_launch": r["flops"]["attention"],
+                             "parts_ms": {k: round(v, 5) for k, v in pm.items()},
+                             "parts_tflops": {k: round(v, 1) for k, v in tf.items()}},
+                "torch_sdpa": None if r["sdpa_ms"] is None else {
+                    "ms": round(r["sdpa_ms"], 5), "tflops": r["flops"]["attention"] / (r["sdpa_ms"] * 1e-3) / 1e12},
+                "gpu_launches": 4 * r["steps"], "clocks": r["clocks"]}), flush=True)
         return 0
     if args.workload == "layer":
         r = run_layer_ours(args, world, rank, dev, pk)

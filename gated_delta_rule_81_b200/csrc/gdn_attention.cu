@@ -109,26 +109,28 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
 //
 // One CTA per (query tile of 128 tokens, query head); tiles of one sequence go longest
 // first.  Warps 0-3: softmax and epilogue (thread = query row, TMEM lane quarter = warp);
-// warp 4 lane 0: TMA (Q once, then K and V tiles of 64 keys into a 2-stage ring); warp 5
+// warp 4 lanes 0 / 1: TMA (Q once and the K tiles / the V tiles of 128 keys, one buffer each); warp 5
 // lane 0: tcgen05.mma.  Per key tile j:
-//   S_j  = Q K_j^T            M 128, N 64, K 256   (16 MMAs; A, B K-major from shared memory)
-//   P_j  = exp2(S_j log2(e)/16 - m)                (softmax warps; bf16 pairs into TMEM)
-//   O   += P_j V_j            M 128, N 256, K 64   (4 MMAs; A = P from TMEM, B = V MN-major)
-// S is double-buffered in TMEM, so S_{j+1} runs while the softmax works on S_j.  The
+//   S_j  = Q K_j^T            M 128, N 128, K 256  (16 MMAs; A, B K-major from shared memory)
+//   P_j  = exp2(S_j log2(e)/16 - m)                (softmax warps; bf16 pairs written over the
+//                                                   first 64 columns of S_j's own TMEM buffer)
+//   O   += P_j V_j            M 128, N 256, K 128  (8 MMAs; A = P from TMEM, B = V MN-major)
+// TMEM: O in columns 0..255, S in two buffers of 128 columns, so S_{j+1} runs while the
+// softmax works on S_j; S_{j+2} reuses S_j's buffer once O += P_j V_j has read P_j.  The next
+// K tile loads as soon as S_j has read K_j, the next V tile once P_j V_j has read V_j.  The
 // running max is lazy: O and l are rescaled only when a row's max grows by more than 8
-// (log2 units), after waiting for the products still writing O; the final 1/l makes the
-// result exact either way.  Masked scores (key past the query) are -inf.  Epilogue:
-// o / l * sigmoid(g) in bf16 into [T_tot][24 * 256].  Every wait is bounded.
-constexpr int kFaBM = 128, kFaBN = 64;
+// (log2 units), decided per warp (the wait and the TMEM accesses are warp-collective), after
+// the products still writing O; the final 1/l makes the result exact either way.  Masked
+// scores (key past the query) are -inf.  Epilogue: o / l * sigmoid(g) in bf16 into
+// [T_tot][24 * 256].  Every wait is bounded.
+constexpr int kFaBM = 128, kFaBN = 128;
 constexpr int kFaThreads = 192;
 constexpr int kFaQBytes = kFaBM * kAD * 2;          // 64 KiB: 4 boxes of 128 rows x 64 dims
-constexpr int kFaKBytes = kFaBN * kAD * 2;          // 32 KiB: 4 boxes of 64 keys x 64 dims
-constexpr int kFaStageBytes = 2 * kFaKBytes;        // K | V
-constexpr int kFaSmem = kFaQBytes + 2 * kFaStageBytes + 1024;
+constexpr int kFaKBytes = kFaBN * kAD * 2;          // 64 KiB: 4 boxes of 128 keys x 64 dims
+constexpr int kFaSmem = kFaQBytes + 2 * kFaKBytes + 1024;  // Q | K | V
 // tensor memory columns
 constexpr uint32_t kFaColO = 0;      // 256 fp32 columns
-constexpr uint32_t kFaColS = 256;    // 2 x 64
-constexpr uint32_t kFaColP = 384;    // 2 x 32 (bf16 pairs)
+constexpr uint32_t kFaColS = 256;    // 2 x 128 (P of the tile in the first 64 of its buffer)
 constexpr float kFaRescale = 8.0f;   // lazy rescale threshold (log2 units)
 
 struct FaParams {
@@ -160,8 +162,9 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* sm = fa_align1024(fa_smem_raw);
   uint8_t* sQ = sm;
-  uint8_t* sKV = sm + kFaQBytes;  // stage s: K at s * kFaStageBytes, V after it
-  __shared__ uint64_t q_full, kv_full[2], kv_free[2], s_full[2], p_full[2], pv_done[2], drain_b;
+  uint8_t* sK = sm + kFaQBytes;
+  uint8_t* sV = sK + kFaKBytes;
+  __shared__ uint64_t q_full, k_full, k_free, v_full, v_free, s_full[2], p_full[2], pv_done[2], drain_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const int n = blockIdx.x % p.B;
   const int mt = p.tiles - 1 - static_cast<int>(blockIdx.x / p.B);
   const int m0 = mt * kFaBM;                                  // first query position in the sequence
-  const int n_kv = min((m0 + kFaBM + kFaBN - 1) / kFaBN, (p.T + kFaBN - 1) / kFaBN);  // key tiles (causal)
+  const int n_kv = (min(m0 + kFaBM, p.T) + kFaBN - 1) / kFaBN;  // key tiles (causal)
   const int kvh = h / kAGrp;
   const int row0 = n * p.T;                                   // first token of the sequence
 
@@ -179,9 +182,11 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   if (threadIdx.x == 0) {
     abort_s = 0;
     mbar_init(&q_full, 1);
+    mbar_init(&k_full, 1);
+    mbar_init(&k_free, 1);
+    mbar_init(&v_full, 1);
+    mbar_init(&v_free, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&kv_full[b], 1);
-      mbar_init(&kv_free[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 128);
       mbar_init(&pv_done[b], 1);
@@ -196,65 +201,70 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const uint32_t tbase = tmem_base_s;
 
   if (warp == 4) {
+    // ------------------------------------------------ TMA producers: lane 0 Q and the K tiles,
+    // lane 1 the V tiles, each waiting only for its own buffer
+    int drain_flag = 0;
+    const Abort drain{nullptr, &drain_flag};
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
       mbar_arrive_expect_tx(&q_full, kFaQBytes);
       for (int kb = 0; kb < 4; ++kb)
         fa_tma_load_2d(sQ + kb * (kFaBM * 128), &tm_q, h * kAD + kb * 64, row0 + m0, &q_full);
-      int issued[2] = {0, 0};
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_free[s], ((j - 2) >> 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&kv_full[s], kFaStageBytes);
-        uint8_t* st = sKV + s * kFaStageBytes;
-        for (int kb = 0; kb < 4; ++kb) {
-          fa_tma_load_2d(st + kb * (kFaBN * 128), &tm_k, kvh * kAD + kb * 64, row0 + j * kFaBN, &kv_full[s]);
-          fa_tma_load_2d(st + kFaKBytes + kb * (kFaBN * 128), &tm_v, kvh * kAD + kb * 64, row0 + j * kFaBN,
-                         &kv_full[s]);
-        }
-        ++issued[s];
+      int n_k = 0;
+      for (int j = 0; j < n_kv; ++j) {  // K_j once S_{j-1} has read K_{j-1}
+        if (j >= 1 && !mbar_wait(&k_free, (j - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&k_full, kFaKBytes);
+        for (int kb = 0; kb < 4; ++kb)
+          fa_tma_load_2d(sK + kb * (kFaBN * 128), &tm_k, kvh * kAD + kb * 64, row0 + j * kFaBN, &k_full);
+        ++n_k;
       }
       // copies still in flight (only after an abort) land before the CTA exits
-      int drain_flag = 0;
-      const Abort drain{nullptr, &drain_flag};
       mbar_wait(&q_full, 0, drain);
-      for (int s = 0; s < 2; ++s)
-        if (issued[s] > 0) mbar_wait(&kv_full[s], (issued[s] - 1) & 1, drain);
+      if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
+    } else if (lane == 1) {
+      int n_v = 0;
+      for (int j = 0; j < n_kv; ++j) {  // V_j once P_{j-1} V_{j-1} has read V_{j-1}
+        if (j >= 1 && !mbar_wait(&v_free, (j - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&v_full, kFaKBytes);
+        for (int kb = 0; kb < 4; ++kb)
+          fa_tma_load_2d(sV + kb * (kFaBN * 128), &tm_v, kvh * kAD + kb * 64, row0 + j * kFaBN, &v_full);
+        ++n_v;
+      }
+      if (n_v > 0) mbar_wait(&v_full, (n_v - 1) & 1, drain);
     }
   } else if (warp == 5) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
       const uint32_t idesc_s = idesc_bf16(kFaBM, kFaBN, false, false);  // Q K^T
       const uint32_t idesc_o = idesc_bf16(kFaBM, kAD, false, true);     // P V, V MN-major (N = d)
-      const uint32_t q_s = smem_u32(sQ);
+      const uint32_t q_s = smem_u32(sQ), k_s = smem_u32(sK), v_s = smem_u32(sV);
       bool ok = mbar_wait(&q_full, 0, ab);
       auto issue_pv = [&](int i) -> bool {  // O += P_i V_i
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, ab)) return false;
+        if (!mbar_wait(&v_full, i & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t v_s = smem_u32(sKV + (i & 1) * kFaStageBytes + kFaKBytes);
 #pragma unroll
         for (int ks = 0; ks < kFaBN / 16; ++ks)
-          umma_bf16_ts(tbase + kFaColO, tbase + kFaColP + 32u * (i & 1) + 8u * ks,
+          umma_bf16_ts(tbase + kFaColO, tbase + kFaColS + 128u * (i & 1) + 8u * ks,
                        smem_desc(v_s + ks * 2048u, kFaBN * 128, 1024, Swz::k128), idesc_o, i > 0 || ks > 0);
         umma_commit(&pv_done[i & 1]);
-        umma_commit(&kv_free[i & 1]);
+        umma_commit(&v_free);
         return true;
       };
       for (int j = 0; j < n_kv && ok; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, ab)) break;
-        // S buffer s was last read by the softmax of tile j - 2 (its p_full has arrived)
-        if (j >= 2 && !mbar_wait(&p_full[s], ((j - 2) >> 1) & 1, ab)) break;
+        if (!mbar_wait(&k_full, j & 1, ab)) break;
+        // S buffer s held P_{j-2}: its products must have read it
+        if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, ab)) break;
         tc_fence_after();
-        const uint32_t k_s = smem_u32(sKV + s * kFaStageBytes);
 #pragma unroll
         for (int ks = 0; ks < kAD / 16; ++ks) {
           const uint32_t off_q = (ks >> 2) * (kFaBM * 128u) + (ks & 3) * 32u;
           const uint32_t off_k = (ks >> 2) * (kFaBN * 128u) + (ks & 3) * 32u;
-          umma_bf16(tbase + kFaColS + 64u * s, smem_desc(q_s + off_q, 16, 1024, Swz::k128),
+          umma_bf16(tbase + kFaColS + 128u * s, smem_desc(q_s + off_q, 16, 1024, Swz::k128),
                     smem_desc(k_s + off_k, 16, 1024, Swz::k128), idesc_s, ks > 0);
         }
         umma_commit(&s_full[s]);
+        umma_commit(&k_free);
         if (j >= 1 && !issue_pv(j - 1)) {
           ok = false;
           break;
@@ -281,8 +291,8 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       }
       tc_fence_after();
       float sv[kFaBN];
-      tmem_ld32(trow + kFaColS + 64u * s, sv);
-      tmem_ld32(trow + kFaColS + 64u * s + 32u, sv + 32);
+#pragma unroll
+      for (int c4 = 0; c4 < kFaBN / 32; ++c4) tmem_ld32(trow + kFaColS + 128u * s + 32u * c4, sv + 32 * c4);
       tmem_wait_ld();
       const int k0 = j * kFaBN;
       float mloc = -INFINITY;
@@ -292,13 +302,8 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         sv[c] = x;
         mloc = fmaxf(mloc, x);
       }
-      // P buffer s was read by the products of tile j - 2
-      if (j >= 2 && !mbar_wait_warp(&pv_done[s], ((j - 2) >> 1) & 1, ab)) {
-        ok = false;
-        break;
-      }
-      // the rescale is decided per warp (its waits and tensor-memory accesses are warp-collective):
-      // lanes whose max grew by more than the threshold take the new max, the others keep theirs
+      // the rescale is decided per warp: lanes whose max grew by more than the threshold take
+      // the new max, the others keep theirs (factor 1)
       const bool grow = mloc > m + kFaRescale;
       if (__any_sync(0xffffffffu, grow)) {
         const float m_new = grow ? mloc : m;
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
             break;
           }
           tc_fence_after();
-          const float f = exp2f(m - m_new);  // 1 for lanes keeping their max
+          const float f = exp2f(m - m_new);
 #pragma unroll 1
           for (int c = 0; c < kAD / 32; ++c) {
             float o[32];
@@ -332,8 +337,8 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         pk[c] = pack_bf16x2(p0, p1);
       }
       l += lsum;
-      tmem_st16(trow + kFaColP + 32u * s, pk);
-      tmem_st16(trow + kFaColP + 32u * s + 16u, pk + 16);
+#pragma unroll
+      for (int c4 = 0; c4 < kFaBN / 32; ++c4) tmem_st16(trow + kFaColS + 128u * s + 16u * c4, pk + 16 * c4);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[s]);
@@ -344,7 +349,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       const bool valid = qpos < p.T;
       const long long tok = static_cast<long long>(row0) + qpos;
       const float inv_l = 1.0f / l;
-      const bf16* grow = p.g + tok * p.ld_g + h * kAD;
+      const bf16* grow_p = p.g + tok * p.ld_g + h * kAD;
       bf16* orow = p.out + tok * (kAHq * kAD) + h * kAD;
 #pragma unroll 1
       for (int c = 0; c < kAD / 32; ++c) {
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float gf[8], y[8];
-            unpack8f(reinterpret_cast<const uint4*>(grow + 32 * c)[u], gf);
+            unpack8f(reinterpret_cast<const uint4*>(grow_p + 32 * c)[u], gf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = o[8 * u + e] * inv_l / (1.0f + __expf(-gf[e]));
             reinterpret_cast<uint4*>(orow + 32 * c)[u] = pack8f(y);

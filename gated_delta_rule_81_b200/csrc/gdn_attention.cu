@@ -108,9 +108,11 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
 // ------------------------------------------------------------ causal flash attention
 //
 // One CTA per (query tile of 128 tokens, query head); tiles of one sequence go longest
-// first.  Warps 0-3: softmax and epilogue (thread = query row, TMEM lane quarter = warp);
-// warp 4 lanes 0 / 1: TMA (Q once and the K tiles / the V tiles of 128 keys, one buffer each); warp 5
-// lane 0: tcgen05.mma.  Per key tile j:
+// first.  Warps 0-7: softmax and epilogue (thread = query row, TMEM lane quarter = warp % 4;
+// warps w and w + 4 split the row's 128 score columns and O's 256 columns in halves and
+// trade their partial row maxima through shared memory); warp 8 lanes 0 / 1: TMA (Q once
+// and the K tiles / the V tiles of 128 keys, one buffer each); warp 9 lane 0: tcgen05.mma.
+// Per key tile j:
 //   S_j  = Q K_j^T            M 128, N 128, K 256  (16 MMAs; A, B K-major from shared memory)
 //   P_j  = exp2(S_j log2(e)/16 - m)                (softmax warps; bf16 pairs written over the
 //                                                   first 64 columns of S_j's own TMEM buffer)
@@ -124,7 +126,8 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
 // scores (key past the query) are -inf.  Epilogue: o / l * sigmoid(g) in bf16 into
 // [T_tot][24 * 256].  Every wait is bounded.
 constexpr int kFaBM = 128, kFaBN = 128;
-constexpr int kFaThreads = 192;
+constexpr int kFaThreads = 320;
+constexpr int kFaWarpTma = 8, kFaWarpMma = 9;
 constexpr int kFaQBytes = kFaBM * kAD * 2;          // 64 KiB: 4 boxes of 128 rows x 64 dims
 constexpr int kFaKBytes = kFaBN * kAD * 2;          // 64 KiB: 4 boxes of 128 keys x 64 dims
 constexpr int kFaSmem = kFaQBytes + 2 * kFaKBytes + 1024;  // Q | K | V
@@ -165,6 +168,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   uint8_t* sK = sm + kFaQBytes;
   uint8_t* sV = sK + kFaKBytes;
   __shared__ uint64_t q_full, k_full, k_free, v_full, v_free, s_full[2], p_full[2], pv_done[2], drain_b;
+  __shared__ float red_s[2][kFaBM];  // partial row maxima (and at the end partial sums), per column half
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,19 +192,19 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     mbar_init(&v_free, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], 256);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(&drain_b, 1);
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc<512>(&tmem_base_s);
+  if (warp == kFaWarpMma) tmem_alloc<512>(&tmem_base_s);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base_s;
 
-  if (warp == 4) {
+  if (warp == kFaWarpTma) {
     // ------------------------------------------------ TMA producers: lane 0 Q and the K tiles,
     // lane 1 the V tiles, each waiting only for its own buffer
     int drain_flag = 0;
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       }
       if (n_v > 0) mbar_wait(&v_full, (n_v - 1) & 1, drain);
     }
-  } else if (warp == 5) {
+  } else if (warp == kFaWarpMma) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
       const uint32_t idesc_s = idesc_bf16(kFaBM, kFaBN, false, false);  // Q K^T
@@ -277,84 +281,105 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       mbar_wait(&drain_b, 0, drain);
     }
   } else {
-    // ------------------------------------------------ softmax + epilogue: thread = query row
-    const int r = 32 * warp + lane;  // warps 0-3: lane quarter = warp
+    // ------------------------------------------------ softmax + epilogue: thread = query row,
+    // column half hc of the scores (keys 64 hc ..) and of O (d 128 hc ..)
+    const int q4 = warp & 3, hc = warp >> 2;
+    const int r = 32 * q4 + lane;
     const int qpos = m0 + r;
-    const uint32_t trow = tmem_addr(tbase, 32 * warp, 0);
-    float m = -INFINITY, l = 0.f;
+    const uint32_t trow = tmem_addr(tbase, 32 * q4, 0);
+    constexpr int kHalf = kFaBN / 2;  // 64 score columns per thread
+    float m = -INFINITY, l = 0.f;     // l: this half's partial sum
+    // no early exit: the two warps of a row pair meet at named barriers every tile, so after a
+    // failed wait a warp keeps its place in the loop and only skips its tensor-memory work
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int s = j & 1;
-      if (!mbar_wait_warp(&s_full[s], (j >> 1) & 1, ab)) {
-        ok = false;
-        break;
-      }
+      ok = ok && mbar_wait_warp(&s_full[s], (j >> 1) & 1, ab);
       tc_fence_after();
-      float sv[kFaBN];
+      float sv[kHalf];
+      if (ok) {
+        tmem_ld32(trow + kFaColS + 128u * s + kHalf * hc, sv);
+        tmem_ld32(trow + kFaColS + 128u * s + kHalf * hc + 32u, sv + 32);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int c4 = 0; c4 < kFaBN / 32; ++c4) tmem_ld32(trow + kFaColS + 128u * s + 32u * c4, sv + 32 * c4);
-      tmem_wait_ld();
-      const int k0 = j * kFaBN;
-      float mloc = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kFaBN; ++c) {
-        const float x = (k0 + c <= qpos) ? sv[c] * p.scale_log2e : -INFINITY;
-        sv[c] = x;
-        mloc = fmaxf(mloc, x);
+        for (int c = 0; c < kHalf; ++c) sv[c] = 0.f;
       }
-      // the rescale is decided per warp: lanes whose max grew by more than the threshold take
-      // the new max, the others keep theirs (factor 1)
+      const int k0 = j * kFaBN + kHalf * hc;
+      float mraw = -INFINITY;  // max of the raw scores (the scale is positive)
+      if (k0 + kHalf - 1 <= m0) {  // no key of this half lies past any query of the tile
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) mraw = fmaxf(mraw, sv[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) {
+          sv[c] = (k0 + c <= qpos) ? sv[c] : -INFINITY;
+          mraw = fmaxf(mraw, sv[c]);
+        }
+      }
+      // the row's max from both halves
+      red_s[hc][r] = mraw;
+      named_bar_sync(1 + q4, 64);
+      const float mloc = fmaxf(mraw, red_s[hc ^ 1][r]) * p.scale_log2e;
+      named_bar_sync(1 + q4, 64);  // both have read before the next tile's write
+      // the rescale is decided per warp (the wait and the TMEM accesses are warp-collective);
+      // both warps of a row pair see the same maxima, so they decide alike
       const bool grow = mloc > m + kFaRescale;
       if (__any_sync(0xffffffffu, grow)) {
         const float m_new = grow ? mloc : m;
         if (j >= 1) {
-          // rescale the warp's rows of O once the products of tile j - 1 have written them
-          if (!mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ab)) {
-            ok = false;
-            break;
-          }
+          // rescale the warp's half of its rows of O once the products of tile j - 1 have written them
+          ok = ok && mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ab);
+        }
+        if (j >= 1 && ok) {
           tc_fence_after();
-          const float f = exp2f(m - m_new);
+          const float f = exp2f(m - m_new);  // 1 for lanes keeping their max
 #pragma unroll 1
-          for (int c = 0; c < kAD / 32; ++c) {
+          for (int c = 0; c < kAD / 64; ++c) {
             float o[32];
-            tmem_ld32(trow + kFaColO + 32u * c, o);
+            tmem_ld32(trow + kFaColO + 128u * hc + 32u * c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(trow + kFaColO + 32u * c, o);
+            tmem_st32(trow + kFaColO + 128u * hc + 32u * c, o);
           }
           l *= f;
         }
         m = m_new;
       }
-      uint32_t pk[kFaBN / 2];
+      uint32_t pk[kHalf / 2];
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kFaBN / 2; ++c) {
-        const float p0 = exp2f(sv[2 * c] - m), p1 = exp2f(sv[2 * c + 1] - m);
+      for (int c = 0; c < kHalf / 2; ++c) {
+        const float p0 = exp2f(fmaf(sv[2 * c], p.scale_log2e, -m));
+        const float p1 = exp2f(fmaf(sv[2 * c + 1], p.scale_log2e, -m));
         lsum += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
       l += lsum;
-#pragma unroll
-      for (int c4 = 0; c4 < kFaBN / 32; ++c4) tmem_st16(trow + kFaColS + 128u * s + 16u * c4, pk + 16 * c4);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[s]);
+      if (ok) {
+        tmem_st16(trow + kFaColS + 128u * s + 32u * hc, pk);
+        tmem_st16(trow + kFaColS + 128u * s + 32u * hc + 16u, pk + 16);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[s]);
+      }
     }
-    // epilogue: the last tile's products complete every write to O
+    // epilogue: the last tile's products complete every write to O; l from both halves
+    red_s[hc][r] = l;
+    named_bar_sync(1 + q4, 64);
+    const float l_row = l + red_s[hc ^ 1][r];
     if (ok && n_kv > 0 && mbar_wait_warp(&pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, ab)) {
       tc_fence_after();
       const bool valid = qpos < p.T;
       const long long tok = static_cast<long long>(row0) + qpos;
-      const float inv_l = 1.0f / l;
-      const bf16* grow_p = p.g + tok * p.ld_g + h * kAD;
-      bf16* orow = p.out + tok * (kAHq * kAD) + h * kAD;
+      const float inv_l = 1.0f / l_row;
+      const bf16* grow_p = p.g + tok * p.ld_g + h * kAD + 128 * hc;
+      bf16* orow = p.out + tok * (kAHq * kAD) + h * kAD + 128 * hc;
 #pragma unroll 1
-      for (int c = 0; c < kAD / 32; ++c) {
+      for (int c = 0; c < kAD / 64; ++c) {
         float o[32];
-        tmem_ld32(trow + kFaColO + 32u * c, o);
+        tmem_ld32(trow + kFaColO + 128u * hc + 32u * c, o);
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -371,7 +396,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc<512>(tbase);
+  if (warp == kFaWarpMma) tmem_dealloc<512>(tbase);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {

@@ -272,7 +272,7 @@ gdn_status gdn_attention_prefill(const void* q_hat, const void* k, const void* v
       overlap(out, ob, g, (static_cast<size_t>(T_tot - 1) * ld_g + hd) * 2))
     return GDN_ERR_ALIAS;
   return gdn::launch_flash_attn(static_cast<const bf16*>(q_hat), static_cast<const bf16*>(k),
-                                static_cast<const bf16*>(v), static_cast<const bf16*>(g), ld_g, B, T,
+                                static_cast<const bf16*>(v), T, static_cast<const bf16*>(g), ld_g, B, T,
                                 static_cast<bf16*>(out), err, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? GDN_OK
              : GDN_ERR_CUDA;
@@ -286,9 +286,11 @@ size_t gdn_attn_layer_workspace_size(int B, int T) {
 }
 
 gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const void* x, long long ldx,
-                                  void* k_cache, void* v_cache, void* y, long long ldy, void* workspace,
-                                  size_t workspace_bytes, int* err, void* stream) {
-  if (!L || B < 0 || T < 0 || L->hidden <= 0) return GDN_ERR_INVALID_ARG;
+                                  void* k_cache, void* v_cache, int cache_cap, void* y, long long ldy,
+                                  void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  if (!L || B < 0 || T < 0 || L->hidden <= 0 || cache_cap < 0) return GDN_ERR_INVALID_ARG;
+  const int cap = cache_cap == 0 ? T : cache_cap;
+  if (cap < T) return GDN_ERR_INVALID_ARG;
   if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
@@ -302,7 +304,7 @@ gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const v
       !aligned16(workspace))
     return GDN_ERR_MISALIGNED;
   const size_t hd = static_cast<size_t>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
-  const size_t kv_bytes = static_cast<size_t>(T_tot) * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * cap * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM * 2;
   const size_t y_bytes = (static_cast<size_t>(T_tot - 1) * ldy + L->hidden) * 2;
   if (overlap(y, y_bytes, workspace, need) || overlap(k_cache, kv_bytes, workspace, need) ||
       overlap(v_cache, kv_bytes, workspace, need) || overlap(k_cache, kv_bytes, v_cache, kv_bytes) ||
@@ -322,14 +324,70 @@ gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const v
   if (s != GDN_OK) return s;
   mark(1);
   if (gdn::launch_attn_qk(proj, GDN_ATTN_N_IN, static_cast<const bf16*>(L->q_norm_w),
-                          static_cast<const bf16*>(L->k_norm_w), B, T, q_hat, static_cast<bf16*>(k_cache),
-                          static_cast<bf16*>(v_cache), st) != cudaSuccess ||
-      gdn::launch_flash_attn(q_hat, static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache),
+                          static_cast<const bf16*>(L->k_norm_w), B, T, nullptr, cap, q_hat,
+                          static_cast<bf16*>(k_cache), static_cast<bf16*>(v_cache), err, st) != cudaSuccess ||
+      gdn::launch_flash_attn(q_hat, static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache), cap,
                              proj + hd, GDN_ATTN_N_IN, B, T, att, err, st) != cudaSuccess)
     return GDN_ERR_CUDA;
   mark(2);
   s = gdn_gemm_bf16(att, static_cast<long long>(hd), L->w_out, L->ld_w_out, y, ldy, static_cast<int>(T_tot),
                     L->hidden, static_cast<int>(hd), err, stream);
+  if (s != GDN_OK) return s;
+  mark(3);
+  return GDN_OK;
+}
+
+size_t gdn_attn_decode_workspace_size(int N, int cache_cap) {
+  if (N < 0 || cache_cap < 0) return 0;
+  const size_t hd = static_cast<size_t>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
+  return round_up(static_cast<size_t>(N) * GDN_ATTN_N_IN * 2, 1024) + 2 * round_up(static_cast<size_t>(N) * hd * 2, 1024) +
+         round_up(gdn::attn_decode_part_bytes(N, cache_cap), 1024);
+}
+
+gdn_status gdn_attn_layer_decode_step(const gdn_attn_layer* L, int N, const void* x, long long ldx, void* k_cache,
+                                      void* v_cache, int cache_cap, int* cache_len, void* y, long long ldy,
+                                      void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  if (!L || N < 0 || cache_cap <= 0 || L->hidden <= 0) return GDN_ERR_INVALID_ARG;
+  if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!x || !y || !k_cache || !v_cache || !cache_len || !L->w_in || !L->w_out || !L->q_norm_w || !L->k_norm_w)
+    return GDN_ERR_INVALID_ARG;
+  if (ldy < L->hidden) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_attn_decode_workspace_size(N, cache_cap);
+  if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(L->q_norm_w) || !aligned16(L->k_norm_w) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(cache_len) & 3u))
+    return GDN_ERR_MISALIGNED;
+  const size_t hd = static_cast<size_t>(GDN_ATTN_Q_HEADS) * GDN_ATTN_HEAD_DIM;
+  const size_t kv_bytes = static_cast<size_t>(N) * cache_cap * GDN_ATTN_KV_HEADS * GDN_ATTN_HEAD_DIM * 2;
+  const size_t y_bytes = (static_cast<size_t>(N - 1) * ldy + L->hidden) * 2;
+  if (overlap(y, y_bytes, workspace, need) || overlap(k_cache, kv_bytes, workspace, need) ||
+      overlap(v_cache, kv_bytes, workspace, need) || overlap(k_cache, kv_bytes, v_cache, kv_bytes) ||
+      overlap(y, y_bytes, k_cache, kv_bytes) || overlap(y, y_bytes, v_cache, kv_bytes))
+    return GDN_ERR_ALIAS;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  bf16* proj = reinterpret_cast<bf16*>(ws);
+  bf16* q_hat = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(N) * GDN_ATTN_N_IN * 2, 1024));
+  bf16* att = reinterpret_cast<bf16*>(reinterpret_cast<uint8_t*>(q_hat) + round_up(static_cast<size_t>(N) * hd * 2, 1024));
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(att) + round_up(static_cast<size_t>(N) * hd * 2, 1024));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) {
+    if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
+  };
+  mark(0);
+  gdn_status s = gdn_gemm_bf16(x, ldx, L->w_in, L->ld_w_in, proj, GDN_ATTN_N_IN, N, GDN_ATTN_N_IN, L->hidden, err,
+                               stream);
+  if (s != GDN_OK) return s;
+  mark(1);
+  if (gdn::launch_attn_qk(proj, GDN_ATTN_N_IN, static_cast<const bf16*>(L->q_norm_w),
+                          static_cast<const bf16*>(L->k_norm_w), N, 1, cache_len, cache_cap, q_hat,
+                          static_cast<bf16*>(k_cache), static_cast<bf16*>(v_cache), err, st) != cudaSuccess ||
+      gdn::launch_attn_decode(q_hat, static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache),
+                              cache_cap, cache_len, proj + hd, GDN_ATTN_N_IN, N, part, att, st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  mark(2);
+  s = gdn_gemm_bf16(att, static_cast<long long>(hd), L->w_out, L->ld_w_out, y, ldy, N, L->hidden,
+                    static_cast<int>(hd), err, stream);
   if (s != GDN_OK) return s;
   mark(3);
   return GDN_OK;

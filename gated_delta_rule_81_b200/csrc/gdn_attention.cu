@@ -33,6 +33,7 @@ constexpr double kARopeBase = 1e7;
 // pairs (i, i + 32) of dims 0 .. 63 sit in lanes l and l ^ 4 (l < 8).  The angles are
 // formed and reduced modulo 2 pi in fp64 (positions reach 262,144), then sincosf.
 constexpr int kQkThreads = 256;
+constexpr int kDevErrCacheFull = 16;  // a sequence's KV cache has no row for its new token
 
 __device__ __forceinline__ void unpack8f(uint4 u, float* f) {
   f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
@@ -49,11 +50,14 @@ struct AttnQkParams {
   long long ld_p;
   const bf16* q_norm_w;  // [256]
   const bf16* k_norm_w;
-  int T;                 // tokens per sequence (position = token index mod T)
+  int T;                 // tokens per sequence in this call: token t is number t % T of sequence t / T
   long long T_tot;
+  const int* pos_base;   // null (positions 0 .. T-1) or [N]: position of each sequence's first token here
+  int cap;               // cache rows per sequence: token at position pos goes to row n * cap + pos
   bf16* q_hat;           // [T_tot][24][256]
-  bf16* k_cache;         // [T_tot][4][256]
-  bf16* v_cache;         // [T_tot][4][256]
+  bf16* k_cache;         // [N][cap][4][256]
+  bf16* v_cache;         // [N][cap][4][256]
+  int* err;
 };
 
 __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
@@ -63,11 +67,18 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
   if (item >= p.T_tot * kHeads) return;
   const long long t = item / kHeads;
   const int hh = static_cast<int>(item % kHeads);
+  const long long n = t / p.T;
+  const long long pos = (p.pos_base ? p.pos_base[n] : 0) + t % p.T;
+  if (pos >= p.cap) {  // no room in the cache: nothing is written for this sequence
+    if (lane == 0 && hh == 0 && p.err) atomicOr(p.err, kDevErrCacheFull);
+    return;
+  }
+  const long long crow = n * p.cap + pos;  // cache row of this token
   const bf16* row = p.proj + t * p.ld_p;
   if (hh >= kAHq + kAHkv) {  // v: a copy into the cache
     const int h = hh - kAHq - kAHkv;
     const uint4 u = reinterpret_cast<const uint4*>(row + 2 * kAHq * kAD + kAHkv * kAD + h * kAD)[lane];
-    reinterpret_cast<uint4*>(p.v_cache + (t * kAHkv + h) * kAD)[lane] = u;
+    reinterpret_cast<uint4*>(p.v_cache + (crow * kAHkv + h) * kAD)[lane] = u;
     return;
   }
   const bool is_q = hh < kAHq;
@@ -89,19 +100,19 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, x[e], 4);
   if (lane < 8) {
-    const double pos = static_cast<double>(t % p.T);
+    const double posd = static_cast<double>(pos);
     const int i0 = 8 * (lane & 3);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const double theta = exp(-static_cast<double>(i0 + e) / (kARope / 2) * log(kARopeBase));
-      const double ang = fmod(pos * theta, 6.283185307179586476925286766559);
+      const double ang = fmod(posd * theta, 6.283185307179586476925286766559);
       float sn, cs;
       sincosf(static_cast<float>(ang), &sn, &cs);
       // x1' = x1 c - x2 s (lanes 0..3), x2' = x2 c + x1 s (lanes 4..7)
       x[e] = lane < 4 ? fmaf(x[e], cs, -partner[e] * sn) : fmaf(x[e], cs, partner[e] * sn);
     }
   }
-  bf16* dst = is_q ? p.q_hat + (t * kAHq + h) * kAD : p.k_cache + (t * kAHkv + h) * kAD;
+  bf16* dst = is_q ? p.q_hat + (t * kAHq + h) * kAD : p.k_cache + (crow * kAHkv + h) * kAD;
   reinterpret_cast<uint4*>(dst)[lane] = pack8f(x);
 }
 
@@ -139,6 +150,8 @@ constexpr float kFaRescale = 8.0f;   // lazy rescale threshold (log2 units)
 struct FaParams {
   int T;              // tokens per sequence
   int B;              // sequences
+  // K, V: 3-D tensor maps (columns, T rows, B sequences at a stride of the cache capacity), so
+  // rows past a sequence's T tokens read as zeros, whatever the cache holds there
   int tiles;          // query tiles per sequence
   const bf16* g;      // gate: head h of token t at g + t * ld_g + h * 256
   long long ld_g;
@@ -156,6 +169,16 @@ __device__ __forceinline__ void fa_tma_load_2d(void* dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
       "[%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 3-D tiled TMA load of the box at (x = column, y = row, z = sequence)
+__device__ __forceinline__ void fa_tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                               uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -218,7 +241,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         if (j >= 1 && !mbar_wait(&k_free, (j - 1) & 1, ab)) break;
         mbar_arrive_expect_tx(&k_full, kFaKBytes);
         for (int kb = 0; kb < 4; ++kb)
-          fa_tma_load_2d(sK + kb * (kFaBN * 128), &tm_k, kvh * kAD + kb * 64, row0 + j * kFaBN, &k_full);
+          fa_tma_load_3d(sK + kb * (kFaBN * 128), &tm_k, kvh * kAD + kb * 64, j * kFaBN, n, &k_full);
         ++n_k;
       }
       // copies still in flight (only after an abort) land before the CTA exits
@@ -230,7 +253,7 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         if (j >= 1 && !mbar_wait(&v_free, (j - 1) & 1, ab)) break;
         mbar_arrive_expect_tx(&v_full, kFaKBytes);
         for (int kb = 0; kb < 4; ++kb)
-          fa_tma_load_2d(sV + kb * (kFaBN * 128), &tm_v, kvh * kAD + kb * 64, row0 + j * kFaBN, &v_full);
+          fa_tma_load_3d(sV + kb * (kFaBN * 128), &tm_v, kvh * kAD + kb * 64, j * kFaBN, n, &v_full);
         ++n_v;
       }
       if (n_v > 0) mbar_wait(&v_full, (n_v - 1) & 1, drain);
@@ -399,6 +422,159 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   if (warp == kFaWarpMma) tmem_dealloc<512>(tbase);
 }
 
+// ------------------------------------------------------------ decode over the KV cache
+//
+// One new token per sequence, already appended to the cache by attn_qk_kernel (at row
+// cache_len[n]); its 24 queries attend to rows 0 .. cache_len[n].  Split-K: CTA (split, KV
+// head, sequence) takes up to kDecSplit cache rows and the KV head's 6 query heads, in fp32:
+// pass 1 scores (warp = token, lane = 8 dims, a reduction over the lanes per head), per-head
+// max and exponentials, pass 2 the weighted V sum (lane = 8 dims of the 6 heads), partials
+// (o, m, l) to scratch.  attn_decode_combine_kernel merges the splits per (sequence, query
+// head), applies 1/l and sigmoid(g), writes bf16; a last small kernel advances cache_len.  The cache is read
+// once per KV head per step: HBM-bound by design.
+constexpr int kDecSplit = 256;
+constexpr int kDecThreads = 256;
+constexpr int kDecPart = kAD + 2;  // o[256], m, l
+
+struct AttnDecParams {
+  const bf16* q_hat;      // [N][24][256]
+  const bf16* k_cache;    // [N][cap][4][256]
+  const bf16* v_cache;
+  int cap;
+  const int* cache_len;   // [N] rows before this step; the new token sits at row cache_len[n]
+  int n_splits;
+  float* part;            // [N][4][n_splits][6][kDecPart]
+};
+
+__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecParams p) {
+  const int sp = blockIdx.x, kvh = blockIdx.y, n = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float qs[kAGrp][kAD];
+  __shared__ float sc[kAGrp][kDecSplit];
+  __shared__ float os[kAGrp][kAD];
+  __shared__ float mh[kAGrp], lh[kAGrp];
+  float* part = p.part + ((static_cast<long long>(n) * kAHkv + kvh) * p.n_splits + sp) * kAGrp * kDecPart;
+  const int len = p.cache_len[n] + 1;
+  const int t0 = sp * kDecSplit, t1 = min(t0 + kDecSplit, len);
+  if (len > p.cap || t0 >= t1) {  // nothing here (or no room in the cache): an empty partial
+    if (threadIdx.x < kAGrp) {
+      part[threadIdx.x * kDecPart + kAD] = -INFINITY;
+      part[threadIdx.x * kDecPart + kAD + 1] = 0.f;
+    }
+    return;
+  }
+  for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) {
+    const int j = x / kAD, d = x % kAD;
+    qs[j][d] = __bfloat162float(p.q_hat[(static_cast<long long>(n) * kAHq + kvh * kAGrp + j) * kAD + d]) * 0.0625f;
+  }
+  for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) os[x / kAD][x % kAD] = 0.f;
+  __syncthreads();
+  const bf16* kbase = p.k_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
+  const bf16* vbase = p.v_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
+  // pass 1: scores (already scaled by 1/sqrt(256) through q)
+  for (int t = t0 + warp; t < t1; t += kDecThreads / 32) {
+    float kf[8];
+    unpack8f(reinterpret_cast<const uint4*>(kbase + static_cast<long long>(t) * kAHkv * kAD)[lane], kf);
+    float dot[kAGrp];
+#pragma unroll
+    for (int j = 0; j < kAGrp; ++j) {
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a = fmaf(qs[j][8 * lane + e], kf[e], a);
+      dot[j] = a;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int j = 0; j < kAGrp; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], o);
+    if (lane < kAGrp) {
+      float v = dot[0];
+#pragma unroll
+      for (int j = 1; j < kAGrp; ++j)
+        if (lane == j) v = dot[j];
+      sc[lane][t - t0] = v;
+    }
+  }
+  __syncthreads();
+  // per-head max, exponentials and sum (warp j < 6 takes head j)
+  if (warp < kAGrp) {
+    float m = -INFINITY;
+    for (int i = lane; i < t1 - t0; i += 32) m = fmaxf(m, sc[warp][i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int i = lane; i < t1 - t0; i += 32) {
+      const float e = expf(sc[warp][i] - m);
+      sc[warp][i] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      mh[warp] = m;
+      lh[warp] = l;
+    }
+  }
+  __syncthreads();
+  // pass 2: o[j] = sum_t p[j][t] v[t]
+  float acc[kAGrp][8];
+#pragma unroll
+  for (int j = 0; j < kAGrp; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+  for (int t = t0 + warp; t < t1; t += kDecThreads / 32) {
+    float vf[8];
+    unpack8f(reinterpret_cast<const uint4*>(vbase + static_cast<long long>(t) * kAHkv * kAD)[lane], vf);
+#pragma unroll
+    for (int j = 0; j < kAGrp; ++j) {
+      const float pj = sc[j][t - t0];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(pj, vf[e], acc[j][e]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kAGrp; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicAdd(&os[j][8 * lane + e], acc[j][e]);
+  __syncthreads();
+  for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) part[(x / kAD) * kDecPart + x % kAD] = os[x / kAD][x % kAD];
+  if (threadIdx.x < kAGrp) {
+    part[threadIdx.x * kDecPart + kAD] = mh[threadIdx.x];
+    part[threadIdx.x * kDecPart + kAD + 1] = lh[threadIdx.x];
+  }
+}
+
+// merge the splits of (sequence n, query head h): o = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M}
+__global__ void __launch_bounds__(kAD) attn_decode_combine_kernel(AttnDecParams p, const bf16* g, long long ld_g,
+                                                                  bf16* out) {
+  const int n = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const int kvh = h / kAGrp, j = h % kAGrp;
+  const int len = p.cache_len[n] + 1;
+  if (len > p.cap) {  // reported by the cache write; nothing was attended: a zero output row
+    out[(static_cast<long long>(n) * kAHq + h) * kAD + d] = __float2bfloat16(0.f);
+    return;
+  }
+  const int used = (len + kDecSplit - 1) / kDecSplit;
+  const float* base = p.part + (static_cast<long long>(n) * kAHkv + kvh) * p.n_splits * kAGrp * kDecPart;
+  float M = -INFINITY;
+  for (int s2 = 0; s2 < used; ++s2) M = fmaxf(M, base[(s2 * kAGrp + j) * kDecPart + kAD]);
+  float L = 0.f, O = 0.f;
+  for (int s2 = 0; s2 < used; ++s2) {
+    const float* ps = base + (s2 * kAGrp + j) * kDecPart;
+    const float w = expf(ps[kAD] - M);
+    L = fmaf(ps[kAD + 1], w, L);
+    O = fmaf(ps[d], w, O);
+  }
+  const float gv = __bfloat162float(g[static_cast<long long>(n) * ld_g + h * kAD + d]);
+  out[(static_cast<long long>(n) * kAHq + h) * kAD + d] = __float2bfloat16(O / L / (1.0f + expf(-gv)));
+}
+
+// the step is complete: each sequence's cache holds one more row (unless it was full)
+__global__ void attn_cache_advance_kernel(int* cache_len, int N, int cap) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n < N && cache_len[n] < cap) cache_len[n] += 1;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -420,10 +596,23 @@ bool attn_encode(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 cache [B][cap][cols]: the first T rows of each sequence as 64-column x box_rows x 1 boxes
+bool attn_encode_cache(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base, int B, int T,
+                       int cap, long long cols, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cap) * cols * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_w, const bf16* k_norm_w, int B,
-                           int T, bf16* q_hat, bf16* k_cache, bf16* v_cache, cudaStream_t stream) {
+                           int T, const int* pos_base, int cap, bf16* q_hat, bf16* k_cache, bf16* v_cache, int* err,
+                           cudaStream_t stream) {
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot == 0) return cudaSuccess;
   AttnQkParams qp;
@@ -433,25 +622,28 @@ cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_
   qp.k_norm_w = k_norm_w;
   qp.T = T;
   qp.T_tot = T_tot;
+  qp.pos_base = pos_base;
+  qp.cap = cap;
   qp.q_hat = q_hat;
   qp.k_cache = k_cache;
   qp.v_cache = v_cache;
+  qp.err = err;
   const long long items = T_tot * (kAHq + 2 * kAHkv);
   attn_qk_kernel<<<static_cast<unsigned>((items + kQkThreads / 32 - 1) / (kQkThreads / 32)), kQkThreads, 0,
                    stream>>>(qp);
   return cudaGetLastError();
 }
 
-cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, const bf16* g, long long ld_g, int B,
-                              int T, bf16* out, int* err, cudaStream_t stream) {
+cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, int kv_cap, const bf16* g,
+                              long long ld_g, int B, int T, bf16* out, int* err, cudaStream_t stream) {
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot == 0) return cudaSuccess;
   PFN_cuTensorMapEncodeTiled_v12000 enc = attn_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tq, tk, tv;
   if (!attn_encode(enc, &tq, q_hat, T_tot, kAHq * kAD, kAHq * kAD, kFaBM) ||
-      !attn_encode(enc, &tk, k, T_tot, kAHkv * kAD, kAHkv * kAD, kFaBN) ||
-      !attn_encode(enc, &tv, v, T_tot, kAHkv * kAD, kAHkv * kAD, kFaBN))
+      !attn_encode_cache(enc, &tk, k, B, T, kv_cap, kAHkv * kAD, kFaBN) ||
+      !attn_encode_cache(enc, &tv, v, B, T, kv_cap, kAHkv * kAD, kFaBN))
     return cudaErrorInvalidValue;
   FaParams fp;
   fp.T = T;
@@ -465,6 +657,33 @@ cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, c
   cudaError_t e = cudaFuncSetAttribute(flash_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFaSmem);
   if (e != cudaSuccess) return e;
   flash_attn_kernel<<<dim3(static_cast<unsigned>(fp.tiles * B), kAHq), kFaThreads, kFaSmem, stream>>>(tq, tk, tv, fp);
+  return cudaGetLastError();
+}
+
+int attn_decode_splits(int cap) { return (cap + kDecSplit - 1) / kDecSplit; }
+
+size_t attn_decode_part_bytes(int N, int cap) {
+  return static_cast<size_t>(N) * kAHkv * attn_decode_splits(cap) * kAGrp * kDecPart * sizeof(float);
+}
+
+cudaError_t launch_attn_decode(const bf16* q_hat, const bf16* k_cache, const bf16* v_cache, int cap, int* cache_len,
+                               const bf16* g, long long ld_g, int N, float* part, bf16* out, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  AttnDecParams dp;
+  dp.q_hat = q_hat;
+  dp.k_cache = k_cache;
+  dp.v_cache = v_cache;
+  dp.cap = cap;
+  dp.cache_len = cache_len;
+  dp.n_splits = attn_decode_splits(cap);
+  dp.part = part;
+  attn_decode_kernel<<<dim3(static_cast<unsigned>(dp.n_splits), kAHkv, static_cast<unsigned>(N)), kDecThreads, 0,
+                       stream>>>(dp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_decode_combine_kernel<<<dim3(static_cast<unsigned>(N), kAHq), kAD, 0, stream>>>(dp, g, ld_g, out);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  attn_cache_advance_kernel<<<(N + 127) / 128, 128, 0, stream>>>(cache_len, N, cap);
   return cudaGetLastError();
 }
 

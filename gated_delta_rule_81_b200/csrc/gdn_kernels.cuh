@@ -91,14 +91,21 @@ cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* co
 // in elements; K a multiple of 64; pointers and leading dimensions 16-byte aligned)
 cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
                              int M, int N, int K, int* err, cudaStream_t stream);
-// The global-attention layer between its projections, B sequences of T tokens.
-// launch_attn_qk: proj [B T][ld_p] holds q (24 x 256) | g (24 x 256) | k (4 x 256) | v (4 x 256);
-// writes q_hat [B T][24][256] and the K and V caches [B T][4][256].
-cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_w, const bf16* k_norm_w, int B,
-                           int T, bf16* q_hat, bf16* k_cache, bf16* v_cache, cudaStream_t stream);
-// launch_flash_attn: out [B T][24 x 256] = causal softmax(q_hat k^T / 16) v * sigmoid(g), GQA 24 / 4;
-// g: head h of token t at g + t * ld_g + h * 256.
-cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, const bf16* g, long long ld_g, int B,
-                              int T, bf16* out, int* err, cudaStream_t stream);
+// The global-attention layer between its projections.
+// launch_attn_qk: proj [N T][ld_p] holds q (24 x 256) | g (24 x 256) | k (4 x 256) | v (4 x 256) of
+// T tokens for each of N sequences; writes q_hat [N T][24][256] and k_hat, v into the caches
+// [N][cap][4][256] at rows (pos_base ? pos_base[n] : 0) + t (error bit 16 past the capacity).
+cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_w, const bf16* k_norm_w, int N,
+                           int T, const int* pos_base, int cap, bf16* q_hat, bf16* k_cache, bf16* v_cache, int* err,
+                           cudaStream_t stream);
+// launch_flash_attn: out [B T][24 x 256] = causal softmax(q_hat k^T / 16) v * sigmoid(g), GQA 24 / 4, with
+// k, v the caches [B][kv_cap][4][256] (their first T rows); g: head h of token t at g + t * ld_g + h * 256.
+cudaError_t launch_flash_attn(const bf16* q_hat, const bf16* k, const bf16* v, int kv_cap, const bf16* g,
+                              long long ld_g, int B, int T, bf16* out, int* err, cudaStream_t stream);
+// Decode: one new token per sequence already in the caches at row cache_len[n]; out [N][24 x 256];
+// part: scratch of attn_decode_part_bytes(N, cap); cache_len advanced by one on the stream.
+size_t attn_decode_part_bytes(int N, int cap);
+cudaError_t launch_attn_decode(const bf16* q_hat, const bf16* k_cache, const bf16* v_cache, int cap, int* cache_len,
+                               const bf16* g, long long ld_g, int N, float* part, bf16* out, cudaStream_t stream);
 
 }  // namespace gdn

@@ -79,7 +79,7 @@ _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_lon
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
            "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
            "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
-           "gdn_status_string")
+           "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string")
 MAX_DECODE_TOKENS = 8
 
 
@@ -114,8 +114,13 @@ def load(path: str | None = None):
     lib.gdn_layer_prefill.restype = _i
     lib.gdn_attn_layer_workspace_size.argtypes = [_i, _i]
     lib.gdn_attn_layer_workspace_size.restype = _sz
-    lib.gdn_attn_layer_prefill.argtypes = [ctypes.POINTER(GdnAttnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _ll, _vp,
-                                           _sz, _vp, _vp]
+    lib.gdn_attn_layer_prefill.argtypes = [ctypes.POINTER(GdnAttnLayer), _i, _i, _vp, _ll, _vp, _vp, _i, _vp, _ll,
+                                           _vp, _sz, _vp, _vp]
+    lib.gdn_attn_decode_workspace_size.argtypes = [_i, _i]
+    lib.gdn_attn_decode_workspace_size.restype = _sz
+    lib.gdn_attn_layer_decode_step.argtypes = [ctypes.POINTER(GdnAttnLayer), _i, _vp, _ll, _vp, _vp, _i, _vp, _vp,
+                                               _ll, _vp, _sz, _vp, _vp]
+    lib.gdn_attn_layer_decode_step.restype = _i
     lib.gdn_attn_layer_prefill.restype = _i
     lib.gdn_attention_prefill.argtypes = [_vp, _vp, _vp, _vp, _ll, _i, _i, _vp, _vp, _vp]
     lib.gdn_attention_prefill.restype = _i
@@ -335,23 +340,39 @@ def make_attn_layer(w_in, w_out, q_norm_w, k_norm_w) -> GdnAttnLayer:
     return L
 
 
-def attn_layer_prefill(L: GdnAttnLayer, B: int, T: int, x, *, y=None, k_cache=None, v_cache=None, workspace=None,
-                       err=None):
-    """gdn_attn_layer_prefill.  Returns (y, k_cache, v_cache)."""
+def attn_layer_prefill(L: GdnAttnLayer, B: int, T: int, x, *, y=None, k_cache=None, v_cache=None, cache_cap=0,
+                       workspace=None, err=None):
+    """gdn_attn_layer_prefill.  Caches are [B][cache_cap or T][4][256].  Returns (y, k_cache, v_cache)."""
     lib = load()
     dev = x.device
+    cap = cache_cap or T
     if y is None:
         y = torch.empty(B * T, L.hidden, dtype=torch.bfloat16, device=dev)
     if k_cache is None:
-        k_cache = torch.empty(B * T, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        k_cache = torch.empty(B, cap, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
     if v_cache is None:
-        v_cache = torch.empty(B * T, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
+        v_cache = torch.empty(B, cap, ATTN_KV_HEADS, ATTN_HEAD_DIM, dtype=torch.bfloat16, device=dev)
     if workspace is None:
         workspace = torch.empty(int(lib.gdn_attn_layer_workspace_size(B, T)), dtype=torch.uint8, device=dev)
     _check(lib.gdn_attn_layer_prefill(ctypes.byref(L), B, T, _ptr(x), x.stride(0), _ptr(k_cache), _ptr(v_cache),
-                                      _ptr(y), y.stride(0), _ptr(workspace), workspace.numel(), _ptr(err),
-                                      _stream()), "gdn_attn_layer_prefill")
+                                      int(cache_cap), _ptr(y), y.stride(0), _ptr(workspace), workspace.numel(),
+                                      _ptr(err), _stream()), "gdn_attn_layer_prefill")
     return y, k_cache, v_cache
+
+
+def attn_layer_decode_step(L: GdnAttnLayer, x, k_cache, v_cache, cache_len, *, y=None, workspace=None, err=None):
+    """gdn_attn_layer_decode_step: one new token per sequence (x [N][hidden]); the caches
+    [N][cap][4][256] and cache_len (device int32 [N]) are updated in place.  Returns y."""
+    lib = load()
+    N, cap = x.shape[0], k_cache.shape[1]
+    if y is None:
+        y = torch.empty(N, L.hidden, dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib.gdn_attn_decode_workspace_size(N, cap)), dtype=torch.uint8, device=x.device)
+    _check(lib.gdn_attn_layer_decode_step(ctypes.byref(L), N, _ptr(x), x.stride(0), _ptr(k_cache), _ptr(v_cache),
+                                          cap, _ptr(cache_len), _ptr(y), y.stride(0), _ptr(workspace),
+                                          workspace.numel(), _ptr(err), _stream()), "gdn_attn_layer_decode_step")
+    return y
 
 
 def attention_prefill(q_hat, k, v, g, B: int, T: int, out=None, err=None):

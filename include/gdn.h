@@ -38,7 +38,7 @@
  *   - `err` (nullable) is a device int the kernels OR error bits into
  *     (1 = a bounded wait timed out, 2 = cluster exchange failed,
  *     4 = cu_seqlens on the device disagreed with cu_seqlens_host, 8 = a decode
- *     state_slot outside the pool).  It is
+ *     state_slot outside the pool, 16 = an attention KV cache with no row left).  It is
  *     never cleared by the library.  Read it after synchronising.
  */
 #ifndef GDN_H_
@@ -245,8 +245,9 @@ size_t gdn_attn_layer_workspace_size(int B, int T);
 /*
  * Prefill of the attention layer for B sequences of T tokens each (packed [B*T]):
  *   x  bf16 [B*T][ldx] -> y bf16 [B*T][ldy] (first `hidden` columns);
- *   k_cache, v_cache  bf16 [B*T][4][256], written: the normalised, rotated keys and the
- *   values, i.e. the layer's KV cache after the prompt.
+ *   k_cache, v_cache  bf16 [B][cache_cap][4][256] (cache_cap = 0: T), rows 0 .. T-1 of each
+ *   sequence written: the normalised, rotated keys and the values, i.e. the layer's KV
+ *   cache after the prompt (gdn_attn_layer_decode_step continues from it).
  * Launches: gdn_gemm_bf16 (in_proj), the q/k norm + rotary kernel, the flash-attention
  * kernel (tcgen05, gate in its epilogue), gdn_gemm_bf16 (out_proj).  Errors as the
  * other entry points; y, the caches and the workspace must not overlap.  The workspace
@@ -254,8 +255,25 @@ size_t gdn_attn_layer_workspace_size(int B, int T);
  * [B*T][24][256] and the attention output [B*T][24*256] (readable after the call).
  */
 gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const void* x, long long ldx,
-                                  void* k_cache, void* v_cache, void* y, long long ldy, void* workspace,
-                                  size_t workspace_bytes, int* err, void* stream);
+                                  void* k_cache, void* v_cache, int cache_cap, void* y, long long ldy,
+                                  void* workspace, size_t workspace_bytes, int* err, void* stream);
+
+/* Workspace bytes of gdn_attn_layer_decode_step for N sequences with caches of cache_cap rows. */
+size_t gdn_attn_decode_workspace_size(int N, int cache_cap);
+
+/*
+ * One decode step of the attention layer: one new token per sequence, x bf16 [N][ldx] -> y.
+ *   k_cache, v_cache  bf16 [N][cache_cap][4][256]; cache_len  device int32 [N], rows in use.
+ * The new token's normalised, rotated key and its value go to row cache_len[n] (its rotary
+ * position), its queries attend to rows 0 .. cache_len[n], and cache_len[n] grows by one,
+ * all on `stream`.  A full cache (cache_len[n] == cache_cap) gives that sequence a zero row of
+ * y, leaves its cache and cache_len as they were, and sets bit 16 of *err.  The attention runs in fp32 on the cache (split over
+ * blocks of 256 rows, merged exactly).  Workspace: the projection [N][GDN_ATTN_N_IN], q_hat,
+ * the attention output [N][24*256] (each from a 1 KiB boundary), then the split partials.
+ */
+gdn_status gdn_attn_layer_decode_step(const gdn_attn_layer* L, int N, const void* x, long long ldx, void* k_cache,
+                                      void* v_cache, int cache_cap, int* cache_len, void* y, long long ldy,
+                                      void* workspace, size_t workspace_bytes, int* err, void* stream);
 
 /*
  * T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N sequences in one call

@@ -28,10 +28,12 @@ from gpu_helpers import err_word, out_error
 pytestmark = pytest.mark.gpu
 
 
-def exact_attn_case(hidden, B, T, seed):
+def exact_attn_case(hidden, B, T, seed, extra=0):
+    """extra: further tokens per sequence (for decode), generated after the prompt's."""
     g = torch.Generator().manual_seed(seed)
     n_in = gdn.ATTN_N_IN
     x = (torch.randint(-16, 17, (B * T, hidden), generator=g).float() / 8).to(torch.bfloat16)
+    x_more = (torch.randint(-16, 17, (max(extra, 1), B, hidden), generator=g).float() / 8).to(torch.bfloat16)
     w_in = torch.zeros(n_in, hidden)
     cols = torch.stack([torch.randperm(hidden, generator=g)[:2] for _ in range(n_in)])
     vals = torch.tensor([1.0, -1.0, 0.5, -0.5, 0.25, -0.25])[torch.randint(0, 6, (n_in, 2), generator=g)]
@@ -40,7 +42,7 @@ def exact_attn_case(hidden, B, T, seed):
     w_out = (torch.randn(hidden, 24 * 256, generator=g) * (24 * 256) ** -0.5).to(torch.bfloat16)
     qn = (1.0 + 0.1 * torch.randn(256, generator=g)).to(torch.bfloat16)
     kn = (1.0 + 0.1 * torch.randn(256, generator=g)).to(torch.bfloat16)
-    return dict(x=x, w_in=w_in, w_out=w_out, qn=qn, kn=kn, B=B, T=T)
+    return dict(x=x, w_in=w_in, w_out=w_out, qn=qn, kn=kn, B=B, T=T, x_more=x_more[:extra])
 
 
 def run_attn(c):
@@ -50,6 +52,7 @@ def run_attn(c):
     B, T = c["B"], c["T"]
     ws = torch.empty(int(gdn.load().gdn_attn_layer_workspace_size(B, T)), dtype=torch.uint8, device="cuda")
     y, kc, vc = gdn.attn_layer_prefill(L, B, T, d["x"], err=err, workspace=ws)
+    kc, vc = kc.reshape(B * T, 4, 256), vc.reshape(B * T, 4, 256)
     torch.cuda.synchronize()
     assert int(err.item()) == 0, int(err.item())
     # the workspace holds [projection | q_hat | attention output], each 1 KiB aligned
@@ -117,3 +120,66 @@ def test_attn_layer_matches_oracle(hidden, B, T):
           f"(y_err rms form {e_y:.3e}); q_hat / K cache excess over 1 ulp {q_excess:.1e} / {k_excess:.1e}")
     assert q_excess <= 1e-6 and k_excess <= 1e-6
     assert r_att <= 1.0 and r_y <= 1.0
+
+
+def test_attn_decode_steps_continue_the_prefill():
+    """Prefill N prompts into caches with room for 3 more rows, then 3 decode steps: each
+    step's output and attention output match the oracle layer over the whole sequence at
+    its last position, the new cache rows match the oracle's, cache_len advances, and a 4th
+    step finds the caches full (error bit 16, zero rows of y, caches unchanged).  The decode attention runs in
+    fp32, so its bound keeps only a 2^-9 sum p|v| / l allowance for the rare one-ulp q_hat /
+    k_hat differences plus the output roundings."""
+    A = oracle.attn
+    N, T0, steps, hidden = 3, 150, 3, 256
+    c = exact_attn_case(hidden, N, T0, seed=77, extra=steps)
+    d = {k: c[k].cuda() for k in ("x", "w_in", "w_out", "qn", "kn")}
+    L = gdn.make_attn_layer(d["w_in"], d["w_out"], d["qn"], d["kn"])
+    err = err_word()
+    cap = T0 + steps
+    _, kc, vc = gdn.attn_layer_prefill(L, N, T0, d["x"], cache_cap=cap, err=err)
+    cache_len = torch.full((N,), T0, dtype=torch.int32, device="cuda")
+    ws = torch.empty(int(gdn.load().gdn_attn_decode_workspace_size(N, cap)), dtype=torch.uint8, device="cuda")
+    xs = [c["x"].reshape(N, T0, hidden)]
+    for st in range(steps):
+        xn = c["x_more"][st]
+        y = gdn.attn_layer_decode_step(L, xn.cuda(), kc, vc, cache_len, workspace=ws, err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert torch.equal(cache_len.cpu(), torch.full((N,), T0 + st + 1, dtype=torch.int32))
+        xs.append(xn[:, None])
+        T = T0 + st + 1
+        x_full = torch.cat(xs, dim=1).reshape(N * T, hidden)
+        cu = [i * T for i in range(N + 1)]
+        ref = A.attn_layer(x_full, c["w_in"], c["w_out"], c["qn"], c["kn"], cu)
+        last = [i * T + T - 1 for i in range(N)]
+        # attention output from the workspace: [projection | q_hat | attention], 1 KiB aligned
+        up = lambda n: -(-n // 1024) * 1024
+        off = up(N * gdn.ATTN_N_IN * 2) + up(N * 24 * 256 * 2)
+        att = ws[off:off + N * 24 * 256 * 2].view(torch.bfloat16).view(N, 24, 256).double().cpu().numpy()
+        lay = A.attn_in_proj_layout()
+        sig = 1.0 / (1.0 + np.exp(-ref["proj"][:, lay["g"][0]:lay["g"][1]].reshape(N * T, 24, 256)))
+        q_ref = oracle.round_bf16(A.rope(A.rms_norm(ref["proj"][:, :6144].reshape(N * T, 24, 256), c["qn"]),
+                                         A.positions(cu)))
+        o_abs = (A.attention(q_ref, ref["k_hat"], np.abs(ref["v"]), cu) * sig)[last]
+        att_ref = ref["out"][last]
+        bound_att = 2.0 ** -9 * o_abs + 2.0 ** -8 * np.abs(att_ref) + 1e-6
+        r_att = float(np.max(np.abs(att - att_ref) / bound_att))
+        bound_y = (bound_att + 2.0 ** -8 * np.abs(att_ref)).reshape(N, -1) @ np.abs(c["w_out"].double().numpy()).T \
+            + 2.0 ** -8 * np.abs(ref["y"][last]) + 1e-6
+        r_y = float(np.max(np.abs(y.double().cpu().numpy() - ref["y"][last]) / bound_y))
+        k_new = kc[:, T - 1].double().cpu().numpy()
+        k_ref = ref["k_hat"][last]
+        k_excess = float(np.max(np.abs(k_new - k_ref) - 2.0 ** -7 * np.abs(k_ref)))
+        np.testing.assert_array_equal(vc[:, T - 1].double().cpu().numpy(), ref["v"][last])
+        print(f"[parity] attention decode step {st + 1} (cache {T} rows): att/bound={r_att:.3f} y/bound={r_y:.3f} "
+              f"new K row excess over 1 ulp {k_excess:.1e}")
+        assert r_att <= 1.0 and r_y <= 1.0 and k_excess <= 1e-6
+    # the caches are full now
+    k_before = kc.clone()
+    y_full = torch.full((N, hidden), 5.0, dtype=torch.bfloat16, device="cuda")
+    gdn.attn_layer_decode_step(L, c["x_more"][0].cuda(), kc, vc, cache_len, y=y_full, workspace=ws, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 16
+    assert torch.equal(cache_len.cpu(), torch.full((N,), cap, dtype=torch.int32))
+    assert torch.all(y_full == 0)
+    assert torch.equal(kc, k_before)

@@ -500,6 +500,59 @@ def run_attn_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120):
             "sdpa_ms": sdpa_ms, "flops": flops, "clocks": clk.report(), "steps": args.steps}
 
 
+def run_attn_decode_ours(args, world, rank, dev, pk, N=64, ctx=4096, hidden=5120):
+    """One attention-layer decode step for N = 64 sequences whose KV caches hold 4095 rows
+    (the step appends row 4096 and attends to all 4096): in_proj GEMM, norm + rotary + cache
+    append, split-K attention over the cache, out_proj GEMM.  cache_len is reset before each
+    step, outside the timed events."""
+    from gated_delta_rule_81_b200 import gdn
+
+    g = torch.Generator().manual_seed(300 + rank)
+    x = torch.randn(N, hidden, generator=g).to(torch.bfloat16).to(dev)
+    w_in = (torch.randn(gdn.ATTN_N_IN, hidden, generator=g) * hidden ** -0.5).to(torch.bfloat16).to(dev)
+    w_out = (torch.randn(hidden, 24 * 256, generator=g) * (24 * 256) ** -0.5).to(torch.bfloat16).to(dev)
+    qn = torch.ones(256, dtype=torch.bfloat16, device=dev)
+    kc = torch.randn(N, ctx, 4, 256, device=dev).to(torch.bfloat16)
+    vc = torch.randn(N, ctx, 4, 256, device=dev).to(torch.bfloat16)
+    L = gdn.make_attn_layer(w_in, w_out, qn, qn)
+    y = torch.empty(N, hidden, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(int(gdn.load().gdn_attn_decode_workspace_size(N, ctx)), dtype=torch.uint8, device=dev)
+    start_len = torch.full((N,), ctx - 1, dtype=torch.int32, device=dev)
+    cache_len = start_len.clone()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gdn.attn_layer_decode_step(L, x, kc, vc, cache_len, y=y, workspace=ws, err=err)
+
+    for _ in range(args.warmup):
+        cache_len.copy_(start_len)
+        flush_l2(flush)
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for ev in evs:
+            cache_len.copy_(start_len)
+            flush_l2(flush)
+            arr = (ctypes.c_void_p * 4)(*[e.cuda_event or (e.record(stream) or e.cuda_event) for e in ev])
+            L.events = ctypes.cast(arr, ctypes.c_void_p)
+            step()
+        torch.cuda.synchronize()
+    L.events = None
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    parts = {"in_proj": [e[0].elapsed_time(e[1]) for e in evs], "attention": [e[1].elapsed_time(e[2]) for e in evs],
+             "out_proj": [e[2].elapsed_time(e[3]) for e in evs]}
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    kv_bytes = N * ctx * 4 * 256 * 2 * 2  # K and V rows read by the attention
+    return {"total_ms": max_over_ranks(sum(step_ms), world), "parts_ms": {k: statistics.mean(v) for k, v in parts.items()},
+            "kv_bytes": kv_bytes, "N": N, "ctx": ctx, "clocks": clk.report(), "steps": args.steps}
+
+
 # ------------------------------------------------------------------ oracle (CPU) arm
 
 
@@ -562,7 +615,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "attn_layer"], default="prefill4k",
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "attn_layer", "attn_decode"],
+                    default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
@@ -601,6 +655,26 @@ def main():
                                            "unit": "GB/s", "frac": d["gbs"] / pk["hbm_gbs"],
                                            "traffic": decode_traffic() if d["T"] == 1 else None},
                               "gpu_launches": d["launches"]}), flush=True)
+        return 0
+    if args.workload == "attn_decode":
+        r = run_attn_decode_ours(args, world, rank, dev, pk)
+        if rank == 0:
+            pm = r["parts_ms"]
+            gbs = r["kv_bytes"] / (pm["attention"] * 1e-3) / 1e9
+            ms_step = r["total_ms"] / r["steps"]
+            print(json.dumps({
+                "metric": "attention-layer decode: KV-cache GB/s of the attention segment",
+                "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": r["steps"], "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": {"workload": "attention-decode-64seq-ctx4096-hidden5120", "sequences": r["N"],
+                           "context": r["ctx"], "tokens_per_s": r["N"] / (ms_step * 1e-3),
+                           "l2": "flushed between timed steps"},
+                "roofline": {"kernel": "attention decode (norm/rotary + split-K attention + merge)", "bound": "hbm",
+                             "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                             "traffic": None, "algorithmic_bytes_per_launch": r["kv_bytes"],
+                             "parts_ms": {k: round(v, 5) for k, v in pm.items()}},
+                "gpu_launches": 7 * r["steps"], "clocks": r["clocks"]}), flush=True)
         return 0
     if args.workload == "attn_layer":
         r = run_attn_layer_ours(args, world, rank, dev, pk)

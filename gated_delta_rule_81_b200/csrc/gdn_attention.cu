@@ -446,7 +446,7 @@ struct AttnDecParams {
   float* part;            // [N][4][n_splits][6][kDecPart]
 };
 
-__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecParams p) {
+__global__ void __launch_bounds__(kDecThreads, 3) attn_decode_kernel(AttnDecParams p) {
   const int sp = blockIdx.x, kvh = blockIdx.y, n = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float qs[kAGrp][kAD];
@@ -471,28 +471,58 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecParams 
   __syncthreads();
   const bf16* kbase = p.k_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
   const bf16* vbase = p.v_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
-  // pass 1: scores (already scaled by 1/sqrt(256) through q)
-  for (int t = t0 + warp; t < t1; t += kDecThreads / 32) {
-    float kf[8];
-    unpack8f(reinterpret_cast<const uint4*>(kbase + static_cast<long long>(t) * kAHkv * kAD)[lane], kf);
-    float dot[kAGrp];
+  // pass 1: scores (already scaled by 1/sqrt(256) through q).  Lane = 8 dims; four tokens per
+  // step with their loads issued together; the 6 per-lane partial dot products (padded to 8)
+  // are summed over the 32 lanes by a transposed butterfly: at each of the first three steps a
+  // lane keeps half of its values and hands the other half to its partner, so lane l ends with
+  // the full sum of value (l >> 2) & 7 after 9 shuffles instead of 30.
+  float qr[kAGrp][8];
 #pragma unroll
-    for (int j = 0; j < kAGrp; ++j) {
-      float a = 0.f;
+  for (int j = 0; j < kAGrp; ++j)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaf(qs[j][8 * lane + e], kf[e], a);
-      dot[j] = a;
-    }
+    for (int e = 0; e < 8; ++e) qr[j][e] = qs[j][8 * lane + e];
+  const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+  for (int tb = t0 + 4 * warp; tb < t1; tb += 4 * (kDecThreads / 32)) {
+    uint4 kr[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
+    for (int u = 0; u < 4; ++u)
+      kr[u] = tb + u < t1 ? reinterpret_cast<const uint4*>(kbase + static_cast<long long>(tb + u) * kAHkv * kAD)[lane]
+                          : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int j = 0; j < kAGrp; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], o);
-    if (lane < kAGrp) {
-      float v = dot[0];
+    for (int u = 0; u < 4; ++u) {
+      float kf[8];
+      unpack8f(kr[u], kf);
+      float v8[8];
 #pragma unroll
-      for (int j = 1; j < kAGrp; ++j)
-        if (lane == j) v = dot[j];
-      sc[lane][t - t0] = v;
+      for (int j = 0; j < 8; ++j) {
+        float a = 0.f;
+        if (j < kAGrp) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a = fmaf(qr[j][e], kf[e], a);
+        }
+        v8[j] = a;
+      }
+      // step 1 (lanes l, l ^ 16): keep values 4 b4 .. 4 b4 + 3
+      float v4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float keep = b4 ? v8[i + 4] : v8[i], give = b4 ? v8[i] : v8[i + 4];
+        v4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
+      }
+      // step 2 (l ^ 8): keep 2 b3 .. 2 b3 + 1 of those
+      float v2[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float keep = b3 ? v4[i + 2] : v4[i], give = b3 ? v4[i] : v4[i + 2];
+        v2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+      }
+      // step 3 (l ^ 4): keep b2
+      const float keep = b2 ? v2[1] : v2[0], give = b2 ? v2[0] : v2[1];
+      float v1 = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+      const int head = 4 * b4 + 2 * b3 + b2;
+      if ((lane & 3) == 0 && head < kAGrp && tb + u < t1) sc[head][tb + u - t0] = v1;
     }
   }
   __syncthreads();
@@ -516,20 +546,29 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(AttnDecParams 
     }
   }
   __syncthreads();
-  // pass 2: o[j] = sum_t p[j][t] v[t]
+  // pass 2: o[j] = sum_t p[j][t] v[t], four tokens per step with their loads issued together
   float acc[kAGrp][8];
 #pragma unroll
   for (int j = 0; j < kAGrp; ++j)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
-  for (int t = t0 + warp; t < t1; t += kDecThreads / 32) {
-    float vf[8];
-    unpack8f(reinterpret_cast<const uint4*>(vbase + static_cast<long long>(t) * kAHkv * kAD)[lane], vf);
+  for (int tb = t0 + 4 * warp; tb < t1; tb += 4 * (kDecThreads / 32)) {
+    uint4 vr[4];
 #pragma unroll
-    for (int j = 0; j < kAGrp; ++j) {
-      const float pj = sc[j][t - t0];
+    for (int u = 0; u < 4; ++u)
+      vr[u] = tb + u < t1 ? reinterpret_cast<const uint4*>(vbase + static_cast<long long>(tb + u) * kAHkv * kAD)[lane]
+                          : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(pj, vf[e], acc[j][e]);
+    for (int u = 0; u < 4; ++u) {
+      if (tb + u >= t1) break;
+      float vf[8];
+      unpack8f(vr[u], vf);
+#pragma unroll
+      for (int j = 0; j < kAGrp; ++j) {
+        const float pj = sc[j][tb + u - t0];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(pj, vf[e], acc[j][e]);
+      }
     }
   }
 #pragma unroll

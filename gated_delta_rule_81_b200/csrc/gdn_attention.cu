@@ -426,13 +426,13 @@ __global__ void __launch_bounds__(kFaThreads, 1)
 //
 // One new token per sequence, already appended to the cache by attn_qk_kernel (at row
 // cache_len[n]); its 24 queries attend to rows 0 .. cache_len[n].  Split-K: CTA (split, KV
-// head, sequence) takes up to kDecSplit cache rows and the KV head's 6 query heads, in fp32:
-// pass 1 scores (warp = token, lane = 8 dims, a reduction over the lanes per head), per-head
-// max and exponentials, pass 2 the weighted V sum (lane = 8 dims of the 6 heads), partials
-// (o, m, l) to scratch.  attn_decode_combine_kernel merges the splits per (sequence, query
-// head), applies 1/l and sigmoid(g), writes bf16; a last small kernel advances cache_len.  The cache is read
-// once per KV head per step: HBM-bound by design.
-constexpr int kDecSplit = 256;
+// head, sequence) takes up to kDecSplit cache rows and the KV head's 6 query heads, in fp32
+// accumulation.  Both contractions run on the tensor cores as m16n8k16 bf16 MMAs (warp-level:
+// the 6 heads are far below the 64-row minimum of a tcgen05 tile), which leaves the CUDA cores
+// only the softmax; the kernel is HBM-bound by design (the cache is read once per KV head per
+// step).  attn_decode_combine_kernel merges the splits per (sequence, query head), applies 1/l
+// and sigmoid(g) and writes bf16; a last small kernel advances cache_len.
+constexpr int kDecSplit = 512;   // cache rows per CTA (a multiple of 128)
 constexpr int kDecThreads = 256;
 constexpr int kDecPart = kAD + 2;  // o[256], m, l
 
@@ -446,10 +446,21 @@ struct AttnDecParams {
   float* part;            // [N][4][n_splits][6][kDecPart]
 };
 
-__global__ void __launch_bounds__(kDecThreads, 3) attn_decode_kernel(AttnDecParams p) {
+// d (16 x 8 fp32) += A (16 x 16 bf16, row-major fragment a) B (16 x 8 bf16, column fragment b):
+// lane (g = lane / 4, c = lane % 4) holds A rows g, g + 8 at columns 2c, 2c + 1 (a0, a1) and
+// 2c + 8, 2c + 9 (a2, a3), B column g at rows 2c, 2c + 1 (b0) and 2c + 8, 2c + 9 (b1), and
+// D rows g (d0, d1), g + 8 (d2, d3) at columns 2c, 2c + 1.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(AttnDecParams p) {
   const int sp = blockIdx.x, kvh = blockIdx.y, n = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ float qs[kAGrp][kAD];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   __shared__ float sc[kAGrp][kDecSplit];
   __shared__ float os[kAGrp][kAD];
   __shared__ float mh[kAGrp], lh[kAGrp];
@@ -463,78 +474,89 @@ __global__ void __launch_bounds__(kDecThreads, 3) attn_decode_kernel(AttnDecPara
     }
     return;
   }
-  for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) {
-    const int j = x / kAD, d = x % kAD;
-    qs[j][d] = __bfloat162float(p.q_hat[(static_cast<long long>(n) * kAHq + kvh * kAGrp + j) * kAD + d]) * 0.0625f;
-  }
   for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) os[x / kAD][x % kAD] = 0.f;
-  __syncthreads();
+  const long long row_el = static_cast<long long>(kAHkv) * kAD;  // elements between cache rows
   const bf16* kbase = p.k_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
   const bf16* vbase = p.v_cache + (static_cast<long long>(n) * p.cap * kAHkv + kvh) * kAD;
-  // pass 1: scores (already scaled by 1/sqrt(256) through q).  Lane = 8 dims; four tokens per
-  // step with their loads issued together; the 6 per-lane partial dot products (padded to 8)
-  // are summed over the 32 lanes by a transposed butterfly: at each of the first three steps a
-  // lane keeps half of its values and hands the other half to its partner, so lane l ends with
-  // the full sum of value (l >> 2) & 7 after 9 shuffles instead of 30.
-  float qr[kAGrp][8];
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+
+  // pass 1: S[token][head] = K q^T, M = 16 tokens, N = 8 heads (6 used), K = 256 dims in 16
+  // MMAs.  The dot product does not depend on the order of the dims, so MMA 2m + h gives lane
+  // (g, c)'s four k slots {2c, 2c+1, 2c+8, 2c+9} the dims 8 (4m + c) + 4h + {0, 1, 2, 3}: each
+  // lane's operands are then whole 16-byte pieces of a K row (dims 8 (4m + c) .. + 7) and of its
+  // query head g, loaded straight into fragment order.  Warp w scores the 16-token blocks
+  // t0 + 16 (w + 8 blk); the two halves of the dims accumulate separately (shorter MMA chains).
+  {
+    uint4 qf[8];
+    const uint4* qrow = reinterpret_cast<const uint4*>(
+        p.q_hat + (static_cast<long long>(n) * kAHq + kvh * kAGrp + min(g, kAGrp - 1)) * kAD);
 #pragma unroll
-  for (int j = 0; j < kAGrp; ++j)
+    for (int m = 0; m < 8; ++m) qf[m] = g < kAGrp ? qrow[4 * m + c] : zero4;
+#pragma unroll 1
+    for (int blk = 0; blk < kDecSplit / 128; ++blk) {
+      const int tb = t0 + 16 * (warp + 8 * blk);
+      if (tb >= t1) break;  // warp-uniform
+      const int r0 = tb + g, r1 = tb + g + 8;
+      const uint4* k0 = reinterpret_cast<const uint4*>(kbase + r0 * row_el);
+      const uint4* k1 = reinterpret_cast<const uint4*>(kbase + r1 * row_el);
+      uint4 a0[8], a1[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qr[j][e] = qs[j][8 * lane + e];
-  const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
-  for (int tb = t0 + 4 * warp; tb < t1; tb += 4 * (kDecThreads / 32)) {
-    uint4 kr[4];
+      for (int m = 0; m < 8; ++m) {
+        a0[m] = r0 < t1 ? k0[4 * m + c] : zero4;
+        a1[m] = r1 < t1 ? k1[4 * m + c] : zero4;
+      }
+      float s4[4] = {0.f, 0.f, 0.f, 0.f}, t4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      kr[u] = tb + u < t1 ? reinterpret_cast<const uint4*>(kbase + static_cast<long long>(tb + u) * kAHkv * kAD)[lane]
-                          : make_uint4(0u, 0u, 0u, 0u);
+      for (int m = 0; m < 8; ++m) {
+        mma_16816(s4, a0[m].x, a1[m].x, a0[m].y, a1[m].y, qf[m].x, qf[m].y);
+        mma_16816(t4, a0[m].z, a1[m].z, a0[m].w, a1[m].w, qf[m].z, qf[m].w);
+      }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float kf[8];
-      unpack8f(kr[u], kf);
-      float v8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float a = 0.f;
-        if (j < kAGrp) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a = fmaf(qr[j][e], kf[e], a);
+      for (int e = 0; e < 4; ++e) s4[e] += t4[e];
+      if (c < kAGrp / 2) {  // heads 2c, 2c + 1; scores scaled by 1/sqrt(256)
+        if (r0 < t1) {
+          sc[2 * c][r0 - t0] = s4[0] * 0.0625f;
+          sc[2 * c + 1][r0 - t0] = s4[1] * 0.0625f;
         }
-        v8[j] = a;
+        if (r1 < t1) {
+          sc[2 * c][r1 - t0] = s4[2] * 0.0625f;
+          sc[2 * c + 1][r1 - t0] = s4[3] * 0.0625f;
+        }
       }
-      // step 1 (lanes l, l ^ 16): keep values 4 b4 .. 4 b4 + 3
-      float v4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float keep = b4 ? v8[i + 4] : v8[i], give = b4 ? v8[i] : v8[i + 4];
-        v4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
-      }
-      // step 2 (l ^ 8): keep 2 b3 .. 2 b3 + 1 of those
-      float v2[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float keep = b3 ? v4[i + 2] : v4[i], give = b3 ? v4[i] : v4[i + 2];
-        v2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
-      }
-      // step 3 (l ^ 4): keep b2
-      const float keep = b2 ? v2[1] : v2[0], give = b2 ? v2[0] : v2[1];
-      float v1 = keep + __shfl_xor_sync(0xffffffffu, give, 4);
-      v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-      v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-      const int head = 4 * b4 + 2 * b3 + b2;
-      if ((lane & 3) == 0 && head < kAGrp && tb + u < t1) sc[head][tb + u - t0] = v1;
     }
   }
+
+  // pass 2 operands.  O^T[dim][head] += V^T[dim][token] P^T[token][head]: M = 16 dims, N = 8
+  // heads, K = 16 tokens.  Warp pair wp = warp / 2 takes the 32-token groups t0 + 32 (wp + 4 it), warp
+  // parity dh the dims 128 dh .. + 127.  Lane (g, c) holds tokens 2c, 2c+1, 2c+8, 2c+9 of a 16-token
+  // block (slots u = 0..3) and, for each, the two 16-byte pieces at dims 128 dh + 8g and
+  // 128 dh + 64 + 8g; tile i (0..7) takes 32-bit word i of those 8: dims D_i, D_i + 1 as its
+  // rows g, g + 8, with the token pairs formed by byte permutes.  The pair's first 32-token group's loads
+  // are issued before the softmax.
+  const int dh = warp & 1, wp = warp >> 1;
+  const int tv0 = t0 + 32 * wp;
+  uint4 vr[2][4][2];
+#pragma unroll
+  for (int b = 0; b < 2; ++b)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t = tv0 + 16 * b + 2 * c + (u & 1) + 8 * (u >> 1);
+      const uint4* row = reinterpret_cast<const uint4*>(vbase + t * row_el + 128 * dh + 8 * g);
+      vr[b][u][0] = t < t1 ? row[0] : zero4;
+      vr[b][u][1] = t < t1 ? row[8] : zero4;
+    }
   __syncthreads();
-  // per-head max, exponentials and sum (warp j < 6 takes head j)
+  // per-head max, exponentials and sum (warp j < 6 takes head j); slots past the split's last
+  // token become 0 so that pass 2 reads no stale values
   if (warp < kAGrp) {
+    const int cnt = t1 - t0;
     float m = -INFINITY;
-    for (int i = lane; i < t1 - t0; i += 32) m = fmaxf(m, sc[warp][i]);
+    for (int i = lane; i < cnt; i += 32) m = fmaxf(m, sc[warp][i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float l = 0.f;
-    for (int i = lane; i < t1 - t0; i += 32) {
-      const float e = expf(sc[warp][i] - m);
+    for (int i = lane; i < kDecSplit; i += 32) {
+      const float e = i < cnt ? expf(sc[warp][i] - m) : 0.f;
       sc[warp][i] = e;
       l += e;
     }
@@ -546,35 +568,59 @@ __global__ void __launch_bounds__(kDecThreads, 3) attn_decode_kernel(AttnDecPara
     }
   }
   __syncthreads();
-  // pass 2: o[j] = sum_t p[j][t] v[t], four tokens per step with their loads issued together
-  float acc[kAGrp][8];
+  // pass 2: the weights p as a bf16 pair p_hi + p_lo (two MMAs), about 16 significant bits
+  float acc[8][4];
 #pragma unroll
-  for (int j = 0; j < kAGrp; ++j)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
-  for (int tb = t0 + 4 * warp; tb < t1; tb += 4 * (kDecThreads / 32)) {
-    uint4 vr[4];
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  const float* prow = &sc[min(g, kAGrp - 1)][0];
+#pragma unroll 1
+  for (int it = 0; it < kDecSplit / 128; ++it) {
+    const int tb = tv0 + 128 * it;
+    if (tb >= t1) break;  // warp-uniform
+    if (it > 0) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      vr[u] = tb + u < t1 ? reinterpret_cast<const uint4*>(vbase + static_cast<long long>(tb + u) * kAHkv * kAD)[lane]
-                          : make_uint4(0u, 0u, 0u, 0u);
+      for (int b = 0; b < 2; ++b)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (tb + u >= t1) break;
-      float vf[8];
-      unpack8f(vr[u], vf);
+        for (int u = 0; u < 4; ++u) {
+          const int t = tb + 16 * b + 2 * c + (u & 1) + 8 * (u >> 1);
+          const uint4* row = reinterpret_cast<const uint4*>(vbase + t * row_el + 128 * dh + 8 * g);
+          vr[b][u][0] = t < t1 ? row[0] : zero4;
+          vr[b][u][1] = t < t1 ? row[8] : zero4;
+        }
+    }
 #pragma unroll
-      for (int j = 0; j < kAGrp; ++j) {
-        const float pj = sc[j][tb + u - t0];
+    for (int b = 0; b < 2; ++b) {
+      const int tr = tb + 16 * b - t0 + 2 * c;  // this lane's first token, relative to t0
+      float2 p01 = *reinterpret_cast<const float2*>(prow + tr);
+      float2 p89 = *reinterpret_cast<const float2*>(prow + tr + 8);
+      if (g >= kAGrp) p01 = p89 = make_float2(0.f, 0.f);
+      const uint32_t b0h = pack_bf16x2(p01.x, p01.y), b1h = pack_bf16x2(p89.x, p89.y);
+      const uint32_t b0l = pack_bf16x2(p01.x - bf16_lo(b0h), p01.y - bf16_hi(b0h));
+      const uint32_t b1l = pack_bf16x2(p89.x - bf16_lo(b1h), p89.y - bf16_hi(b1h));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(pj, vf[e], acc[j][e]);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t w0 = (&vr[b][0][i >> 2].x)[i & 3], w1 = (&vr[b][1][i >> 2].x)[i & 3];
+        const uint32_t w8 = (&vr[b][2][i >> 2].x)[i & 3], w9 = (&vr[b][3][i >> 2].x)[i & 3];
+        const uint32_t x0 = __byte_perm(w0, w1, 0x5410), x1 = __byte_perm(w0, w1, 0x7632);
+        const uint32_t x2 = __byte_perm(w8, w9, 0x5410), x3 = __byte_perm(w8, w9, 0x7632);
+        mma_16816(acc[i], x0, x1, x2, x3, b0h, b1h);
+        mma_16816(acc[i], x0, x1, x2, x3, b0l, b1l);
       }
     }
   }
+  // the four warp pairs' partial sums of each (head, dim)
+  if (c < kAGrp / 2) {
 #pragma unroll
-  for (int j = 0; j < kAGrp; ++j)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) atomicAdd(&os[j][8 * lane + e], acc[j][e]);
+    for (int i = 0; i < 8; ++i) {
+      const int d = 128 * dh + 64 * (i >> 2) + 8 * g + 2 * (i & 3);
+      atomicAdd(&os[2 * c][d], acc[i][0]);
+      atomicAdd(&os[2 * c + 1][d], acc[i][1]);
+      atomicAdd(&os[2 * c][d + 1], acc[i][2]);
+      atomicAdd(&os[2 * c + 1][d + 1], acc[i][3]);
+    }
+  }
   __syncthreads();
   for (int x = threadIdx.x; x < kAGrp * kAD; x += kDecThreads) part[(x / kAD) * kDecPart + x % kAD] = os[x / kAD][x % kAD];
   if (threadIdx.x < kAGrp) {

@@ -183,3 +183,67 @@ def test_attn_decode_steps_continue_the_prefill():
     assert torch.equal(cache_len.cpu(), torch.full((N,), cap, dtype=torch.int32))
     assert torch.all(y_full == 0)
     assert torch.equal(kc, k_before)
+
+
+def test_attn_decode_long_ragged_caches():
+    """Decode over caches filled with seeded rows, cache_len = 0, 511, 1023 and 1300 (1, 512,
+    1024 and 1301 attended rows: one row, one full split, two full splits, three splits with a
+    ragged last one), so the split-K partials and their merge are all exercised.  q_hat and the
+    new K row must be within one bf16 ulp of the oracle's; the attention output is compared
+    with the oracle's causal attention over the whole sequence (last row) on the kernel's own
+    q_hat, where the fp32 scores and the p_hi + p_lo weights leave an error far below
+    2^-12 sum p|v| / l, plus the bf16 rounding of the stored output."""
+    A = oracle.attn
+    lens = [0, 511, 1023, 1300]
+    N, cap, hidden = len(lens), 1400, 256
+    c = exact_attn_case(hidden, N, 1, seed=91)
+    g = torch.Generator().manual_seed(92)
+    kc = torch.randn(N, cap, 4, 256, generator=g).to(torch.bfloat16)
+    vc = torch.randn(N, cap, 4, 256, generator=g).to(torch.bfloat16)
+    d = {k: c[k].cuda() for k in ("x", "w_in", "w_out", "qn", "kn")}
+    L = gdn.make_attn_layer(d["w_in"], d["w_out"], d["qn"], d["kn"])
+    err = err_word()
+    kcd, vcd = kc.cuda(), vc.cuda()
+    cache_len = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(int(gdn.load().gdn_attn_decode_workspace_size(N, cap)), dtype=torch.uint8, device="cuda")
+    gdn.attn_layer_decode_step(L, d["x"], kcd, vcd, cache_len, workspace=ws, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert cache_len.cpu().tolist() == [n + 1 for n in lens]
+    up = lambda n: -(-n // 1024) * 1024
+    off_q = up(N * gdn.ATTN_N_IN * 2)
+    off_att = off_q + up(N * 24 * 256 * 2)
+    q_gpu = ws[off_q:off_q + N * 24 * 256 * 2].view(torch.bfloat16).view(N, 24, 256).double().cpu().numpy()
+    att = ws[off_att:off_att + N * 24 * 256 * 2].view(torch.bfloat16).view(N, 24, 256).double().cpu().numpy()
+    proj = oracle.round_bf16(oracle.gemm(c["x"], c["w_in"]))
+    lay = A.attn_in_proj_layout()
+    part = lambda name: proj[:, lay[name][0]:lay[name][1]]
+    worst_att = worst_q = worst_k = 0.0
+    for n, ln in enumerate(lens):
+        pos = np.array([ln])
+        q_ref = oracle.round_bf16(A.rope(A.rms_norm(part("q")[n].reshape(1, 24, 256), c["qn"]), pos))[0]
+        k_ref = oracle.round_bf16(A.rope(A.rms_norm(part("k")[n].reshape(1, 4, 256), c["kn"]), pos))[0]
+        v_new = part("v")[n].reshape(4, 256)
+        worst_q = max(worst_q, float(np.max(np.abs(q_gpu[n] - q_ref) - 2.0 ** -7 * np.abs(q_ref))))
+        k_row = kcd[n, ln].double().cpu().numpy()
+        worst_k = max(worst_k, float(np.max(np.abs(k_row - k_ref) - 2.0 ** -7 * np.abs(k_ref))))
+        np.testing.assert_array_equal(vcd[n, ln].double().cpu().numpy(), v_new)
+        # the sequence as the oracle sees it: the cache rows, then the new token (the GPU's own
+        # new K row, checked above), whose query is the last row
+        T = ln + 1
+        keys = np.concatenate([kc[n, :ln].double().numpy(), k_row[None]], axis=0)
+        vals = np.concatenate([vc[n, :ln].double().numpy(), v_new[None]], axis=0)
+        qs = np.zeros((T, 24, 256))
+        qs[-1] = q_gpu[n]
+        sig = 1.0 / (1.0 + np.exp(-part("g")[n].reshape(24, 256)))
+        ref = A.attention(qs, keys, vals, [0, T])[-1] * sig
+        o_abs = A.attention(qs, keys, np.abs(vals), [0, T])[-1] * sig
+        bound = 2.0 ** -12 * o_abs + 2.0 ** -8 * np.abs(ref) + 1e-6
+        worst_att = max(worst_att, float(np.max(np.abs(att[n] - ref) / bound)))
+    print(f"[parity] attention decode over caches {lens}: att/bound={worst_att:.3f}; q_hat / new K row excess "
+          f"over 1 ulp {worst_q:.1e} / {worst_k:.1e}")
+    assert worst_q <= 1e-6 and worst_k <= 1e-6
+    assert worst_att <= 1.0
+    # rows other than the new ones are untouched
+    for n, ln in enumerate(lens):
+        assert torch.equal(kcd[n, :ln].cpu(), kc[n, :ln]) and torch.equal(kcd[n, ln + 1:].cpu(), kc[n, ln + 1:])

@@ -621,6 +621,8 @@ def main():
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
                          "overlapped in one launch whenever the scan units fit in half the SMs)")
+    ap.add_argument("--attn-seqs", type=int, default=64,
+                    help="attn_decode: sequences per step (each with a 4096-row KV cache)")
     ap.add_argument("--decode-tokens", type=int, default=1,
                     help="decode workload: new tokens per sequence per launch (1 .. 8)")
     args = ap.parse_args()
@@ -657,7 +659,7 @@ def main():
                               "gpu_launches": d["launches"]}), flush=True)
         return 0
     if args.workload == "attn_decode":
-        r = run_attn_decode_ours(args, world, rank, dev, pk)
+        r = run_attn_decode_ours(args, world, rank, dev, pk, N=args.attn_seqs)
         if rank == 0:
             pm = r["parts_ms"]
             gbs = r["kv_bytes"] / (pm["attention"] * 1e-3) / 1e9
@@ -667,7 +669,7 @@ def main():
                 "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": r["steps"], "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f32", "data": "synthetic",
-                "config": {"workload": "attention-decode-64seq-ctx4096-hidden5120", "sequences": r["N"],
+                "config": {"workload": f"attention-decode-{r['N']}seq-ctx4096-hidden5120", "sequences": r["N"],
                            "context": r["ctx"], "tokens_per_s": r["N"] / (ms_step * 1e-3),
                            "l2": "flushed between timed steps"},
                 "roofline": {"kernel": "attention decode (norm/rotary + split-K attention + merge)", "bound": "hbm",

@@ -8,11 +8,16 @@
 // the token's position, so every one of the 32 frequencies turns by position * theta_i,
 // theta_i = 1e7^(-i/32), applied to the pairs (i, i + 32) of the first 64 dims.
 //
-// Two kernels:
+// Kernels:
 //   attn_qk_kernel     q_hat = rope(rms(q) w_q), k_hat = rope(rms(k) w_k) per head, both
 //                      stored bf16 (k_hat into the caller's K cache), v copied to the V cache;
 //   flash_attn_kernel  causal softmax attention, GQA, on the tensor cores, with the output
-//                      gate o * sigmoid(g) in its epilogue.
+//                      gate o * sigmoid(g) in its epilogue (prefill);
+//   attn_decode_kernel, attn_decode_combine_kernel, attn_cache_advance_kernel
+//                      one new token per sequence against its KV cache: split-K partials,
+//                      their exact merge with the gate, and the cache length update.
+#include <cmath>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -30,8 +35,10 @@ constexpr double kARopeBase = 1e7;
 // ------------------------------------------------------------ q / k norm and rotary
 //
 // One warp per (token, head): lane l holds dims 8l .. 8l+7 (16-byte loads); the rotary
-// pairs (i, i + 32) of dims 0 .. 63 sit in lanes l and l ^ 4 (l < 8).  The angles are
-// formed and reduced modulo 2 pi in fp64 (positions reach 262,144), then sincosf.
+// pairs (i, i + 32) of dims 0 .. 63 sit in lanes l and l ^ 4 (l < 8).  The angles
+// pos * theta_i are formed in fp64 (positions reach 262,144) from frequencies the host
+// computes once per launch, reduced to [-pi, pi] by subtracting the nearest multiple of
+// 2 pi (one fp64 rounding and fma: error ~1e-10 rad at the largest positions), then sincosf.
 constexpr int kQkThreads = 256;
 constexpr int kDevErrCacheFull = 16;  // a sequence's KV cache has no row for its new token
 
@@ -58,6 +65,7 @@ struct AttnQkParams {
   bf16* k_cache;         // [N][cap][4][256]
   bf16* v_cache;         // [N][cap][4][256]
   int* err;
+  double theta[kARope / 2];  // rotary frequencies 1e7^(-i/32)
 };
 
 __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
@@ -102,12 +110,13 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
   if (lane < 8) {
     const double posd = static_cast<double>(pos);
     const int i0 = 8 * (lane & 3);
+    constexpr double kTwoPi = 6.283185307179586476925286766559, kInvTwoPi = 0.15915494309189533576888376337251;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const double theta = exp(-static_cast<double>(i0 + e) / (kARope / 2) * log(kARopeBase));
-      const double ang = fmod(posd * theta, 6.283185307179586476925286766559);
+      const double ang = posd * p.theta[i0 + e];
+      const double r = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
       float sn, cs;
-      sincosf(static_cast<float>(ang), &sn, &cs);
+      sincosf(static_cast<float>(r), &sn, &cs);
       // x1' = x1 c - x2 s (lanes 0..3), x2' = x2 c + x1 s (lanes 4..7)
       x[e] = lane < 4 ? fmaf(x[e], cs, -partner[e] * sn) : fmaf(x[e], cs, partner[e] * sn);
     }
@@ -713,6 +722,7 @@ cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_
   qp.k_cache = k_cache;
   qp.v_cache = v_cache;
   qp.err = err;
+  for (int i = 0; i < kARope / 2; ++i) qp.theta[i] = std::pow(kARopeBase, -static_cast<double>(i) / (kARope / 2));
   const long long items = T_tot * (kAHq + 2 * kAHkv);
   attn_qk_kernel<<<static_cast<unsigned>((items + kQkThreads / 32 - 1) / (kQkThreads / 32)), kQkThreads, 0,
                    stream>>>(qp);

@@ -34,12 +34,14 @@ constexpr double kARopeBase = 1e7;
 
 // ------------------------------------------------------------ q / k norm and rotary
 //
-// One warp per (token, head): lane l holds dims 8l .. 8l+7 (16-byte loads); the rotary
+// A warp per 4 (token, head) items of one token: lane l holds dims 8l .. 8l+7 (16-byte loads); the rotary
 // pairs (i, i + 32) of dims 0 .. 63 sit in lanes l and l ^ 4 (l < 8).  The angles
 // pos * theta_i are formed in fp64 (positions reach 262,144) from frequencies the host
 // computes once per launch, reduced to [-pi, pi] by subtracting the nearest multiple of
 // 2 pi (one fp64 rounding and fma: error ~1e-10 rad at the largest positions), then sincosf.
 constexpr int kQkThreads = 256;
+constexpr int kQkItems = 4;  // (token, head) items per warp, all of one token
+static_assert((kAHq + 2 * kAHkv) % kQkItems == 0, "a warp's items must belong to one token");
 constexpr int kDevErrCacheFull = 16;  // a sequence's KV cache has no row for its new token
 
 __device__ __forceinline__ void unpack8f(uint4 u, float* f) {
@@ -70,59 +72,85 @@ struct AttnQkParams {
 
 __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long item = static_cast<long long>(blockIdx.x) * (kQkThreads / 32) + warp;  // (token, head)
   constexpr int kHeads = kAHq + kAHkv + kAHkv;  // q heads, k heads, v heads
-  if (item >= p.T_tot * kHeads) return;
-  const long long t = item / kHeads;
-  const int hh = static_cast<int>(item % kHeads);
-  const long long n = t / p.T;
-  const long long pos = (p.pos_base ? p.pos_base[n] : 0) + t % p.T;
-  if (pos >= p.cap) {  // no room in the cache: nothing is written for this sequence
-    if (lane == 0 && hh == 0 && p.err) atomicOr(p.err, kDevErrCacheFull);
-    return;
-  }
-  const long long crow = n * p.cap + pos;  // cache row of this token
-  const bf16* row = p.proj + t * p.ld_p;
-  if (hh >= kAHq + kAHkv) {  // v: a copy into the cache
-    const int h = hh - kAHq - kAHkv;
-    const uint4 u = reinterpret_cast<const uint4*>(row + 2 * kAHq * kAD + kAHkv * kAD + h * kAD)[lane];
-    reinterpret_cast<uint4*>(p.v_cache + (crow * kAHkv + h) * kAD)[lane] = u;
-    return;
-  }
-  const bool is_q = hh < kAHq;
-  const int h = is_q ? hh : hh - kAHq;
-  const bf16* src = is_q ? row + h * kAD : row + 2 * kAHq * kAD + h * kAD;
-  float x[8], w[8];
-  unpack8f(reinterpret_cast<const uint4*>(src)[lane], x);
-  unpack8f(reinterpret_cast<const uint4*>(is_q ? p.q_norm_w : p.k_norm_w)[lane], w);
-  float ss = 0.f;
+  const long long n_items = p.T_tot * kHeads;
+  // a warp takes kQkItems consecutive (token, head) items of one token and issues their loads together
+  const long long item0 = (static_cast<long long>(blockIdx.x) * (kQkThreads / 32) + warp) * kQkItems;
+  if (item0 >= n_items) return;  // warp-uniform
+  uint4 raw[kQkItems];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float inv = rsqrtf(ss * (1.0f / kAD) + 1e-6f);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) x[e] = x[e] * inv * w[e];
-  // rotary on dims 0 .. 63 (lanes 0 .. 7): lane l < 4 holds x1 = dims 8l.., lane l + 4 holds x2
-  float partner[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, x[e], 4);
-  if (lane < 8) {
-    const double posd = static_cast<double>(pos);
-    const int i0 = 8 * (lane & 3);
-    constexpr double kTwoPi = 6.283185307179586476925286766559, kInvTwoPi = 0.15915494309189533576888376337251;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const double ang = posd * p.theta[i0 + e];
-      const double r = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
-      float sn, cs;
-      sincosf(static_cast<float>(r), &sn, &cs);
-      // x1' = x1 c - x2 s (lanes 0..3), x2' = x2 c + x1 s (lanes 4..7)
-      x[e] = lane < 4 ? fmaf(x[e], cs, -partner[e] * sn) : fmaf(x[e], cs, partner[e] * sn);
+  for (int u = 0; u < kQkItems; ++u) {
+    const long long item = item0 + u;
+    raw[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (item < n_items) {
+      const long long t = item / kHeads;
+      const int hh = static_cast<int>(item % kHeads);
+      const bf16* row = p.proj + t * p.ld_p;
+      const bf16* src = hh < kAHq ? row + hh * kAD : row + 2 * kAHq * kAD + (hh - kAHq) * kAD;  // k and v follow g
+      raw[u] = reinterpret_cast<const uint4*>(src)[lane];
     }
   }
-  bf16* dst = is_q ? p.q_hat + (t * kAHq + h) * kAD : p.k_cache + (crow * kAHkv + h) * kAD;
-  reinterpret_cast<uint4*>(dst)[lane] = pack8f(x);
+  float wq[8], wk[8];
+  unpack8f(reinterpret_cast<const uint4*>(p.q_norm_w)[lane], wq);
+  unpack8f(reinterpret_cast<const uint4*>(p.k_norm_w)[lane], wk);
+  // the rotation of this token, shared by its heads: lane i turns frequency i (its angle formed in
+  // fp64 and reduced to [-pi, pi]), then lanes 0..7 gather the 8 frequencies 8 (l % 4) + e they apply
+  const long long t_w = item0 / kHeads;
+  const long long pos_w = (p.pos_base ? p.pos_base[t_w / p.T] : 0) + t_w % p.T;
+  float cs8[8], sn8[8];
+  {
+    constexpr double kTwoPi = 6.283185307179586476925286766559, kInvTwoPi = 0.15915494309189533576888376337251;
+    const double ang = static_cast<double>(pos_w) * p.theta[lane];
+    const double r = fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
+    float sn, cs;
+    sincosf(static_cast<float>(r), &sn, &cs);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      cs8[e] = __shfl_sync(0xffffffffu, cs, 8 * (lane & 3) + e);
+      sn8[e] = __shfl_sync(0xffffffffu, sn, 8 * (lane & 3) + e);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kQkItems; ++u) {
+    const long long item = item0 + u;
+    if (item >= n_items) continue;  // warp-uniform
+    const long long t = item / kHeads;
+    const int hh = static_cast<int>(item % kHeads);
+    const long long n = t / p.T;
+    const long long pos = (p.pos_base ? p.pos_base[n] : 0) + t % p.T;
+    if (pos >= p.cap) {  // no room in the cache: nothing is written for this sequence
+      if (lane == 0 && hh == 0 && p.err) atomicOr(p.err, kDevErrCacheFull);
+      continue;
+    }
+    const long long crow = n * p.cap + pos;  // cache row of this token
+    if (hh >= kAHq + kAHkv) {  // v: a copy into the cache
+      reinterpret_cast<uint4*>(p.v_cache + (crow * kAHkv + (hh - kAHq - kAHkv)) * kAD)[lane] = raw[u];
+      continue;
+    }
+    const bool is_q = hh < kAHq;
+    const int h = is_q ? hh : hh - kAHq;
+    float x[8];
+    unpack8f(raw[u], x);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss * (1.0f / kAD) + 1e-6f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = x[e] * inv * (is_q ? wq[e] : wk[e]);
+    // rotary on dims 0 .. 63 (lanes 0 .. 7): lane l < 4 holds x1 = dims 8l.., lane l + 4 holds x2
+    float partner[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, x[e], 4);
+    if (lane < 8) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)  // x1' = x1 c - x2 s (lanes 0..3), x2' = x2 c + x1 s (lanes 4..7)
+        x[e] = lane < 4 ? fmaf(x[e], cs8[e], -partner[e] * sn8[e]) : fmaf(x[e], cs8[e], partner[e] * sn8[e]);
+    }
+    bf16* dst = is_q ? p.q_hat + (t * kAHq + h) * kAD : p.k_cache + (crow * kAHkv + h) * kAD;
+    reinterpret_cast<uint4*>(dst)[lane] = pack8f(x);
+  }
 }
 
 // ------------------------------------------------------------ causal flash attention
@@ -724,8 +752,8 @@ cudaError_t launch_attn_qk(const bf16* proj, long long ld_p, const bf16* q_norm_
   qp.err = err;
   for (int i = 0; i < kARope / 2; ++i) qp.theta[i] = std::pow(kARopeBase, -static_cast<double>(i) / (kARope / 2));
   const long long items = T_tot * (kAHq + 2 * kAHkv);
-  attn_qk_kernel<<<static_cast<unsigned>((items + kQkThreads / 32 - 1) / (kQkThreads / 32)), kQkThreads, 0,
-                   stream>>>(qp);
+  const long long per_cta = static_cast<long long>(kQkThreads / 32) * kQkItems;
+  attn_qk_kernel<<<static_cast<unsigned>((items + per_cta - 1) / per_cta), kQkThreads, 0, stream>>>(qp);
   return cudaGetLastError();
 }
 

@@ -206,6 +206,9 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
 
 /*
  * The global-attention layer of the hybrid decoder (the fourth layer of every four):
+ * model card "Agnes-3.0-Flash Preview", "Architecture" table, rows "Global attention"
+ * and "Positions"; "Agnes-3.0-Flash Deep Dive: A 33B Hybrid-Attention Multimodal Model",
+ * section "Attention Layer Details".
  * 24 query heads / 4 KV heads of dimension 256, RMS-norm on q and k, rotary position
  * on the first 64 dims of each head (positions = token index within its sequence,
  * base 1e7, pairs (i, i + 32)), causal softmax attention, output * sigmoid(gate).
@@ -267,9 +270,12 @@ size_t gdn_attn_decode_workspace_size(int N, int cache_cap);
  * The new token's normalised, rotated key and its value go to row cache_len[n] (its rotary
  * position), its queries attend to rows 0 .. cache_len[n], and cache_len[n] grows by one,
  * all on `stream`.  A full cache (cache_len[n] == cache_cap) gives that sequence a zero row of
- * y, leaves its cache and cache_len as they were, and sets bit 16 of *err.  The attention runs in fp32 on the cache (split over
- * blocks of 256 rows, merged exactly).  Workspace: the projection [N][GDN_ATTN_N_IN], q_hat,
- * the attention output [N][24*256] (each from a 1 KiB boundary), then the split partials.
+ * y, leaves its cache and cache_len as they were, and sets bit 16 of *err.  The attention
+ * is split over blocks of 512 cache rows and merged exactly; scores and weighted sums are
+ * bf16 tensor-core products with fp32 accumulation, the weights entering as a bf16 pair
+ * hi + lo (about 16 significant bits), the softmax in fp32.  Workspace: the projection
+ * [N][GDN_ATTN_N_IN], q_hat, the attention output [N][24*256] (each from a 1 KiB boundary),
+ * then the split partials.
  */
 gdn_status gdn_attn_layer_decode_step(const gdn_attn_layer* L, int N, const void* x, long long ldx, void* k_cache,
                                       void* v_cache, int cache_cap, int* cache_len, void* y, long long ldy,

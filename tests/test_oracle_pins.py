@@ -511,3 +511,38 @@ def test_attn_mixer_gate_limits():
     o = A.attention(a["q_hat"], a["k_hat"], v, [0, T])
     np.testing.assert_allclose(a["out"], o, rtol=1e-15)
     np.testing.assert_allclose(b["out"], o / 2, rtol=1e-15)
+
+
+def test_attn_layer_closed_form_routing():
+    """The attention layer end to end on a case with a closed-form answer.  Hidden states are
+    one-hot (x_t = e_t), so token t's projection is column t of W_in, chosen here: token 1's
+    query equals its own key r (a +-1 vector: both RMS-norms leave it as it is, and the two
+    rotations at the same position keep q.k = 256, a score of +16), token 0's key is -r (a score
+    near -16), so token 1 attends to itself alone up to e^-32; token 0 sees only itself.  The
+    values differ per KV head, so query head h must read KV head h // 6: out_t = v_t[h // 6] *
+    sigmoid(g_t[h]) and y_t = bf16(out_t) W_out^T (both products exact in fp64)."""
+    A = oracle.attn
+    Hq, Hkv, D, hidden = 24, 4, 256, 8
+    g = torch.Generator().manual_seed(11)
+    lay = A.attn_in_proj_layout()
+    r = (torch.randint(0, 2, (D,), generator=g) * 2 - 1).double()
+    cols = torch.zeros(lay["total"][1], hidden, dtype=torch.float64)
+    v = (torch.randn(2, Hkv, D, generator=g) * 0.5).to(torch.bfloat16).double()
+    gate = torch.randn(2, Hq, D, generator=g).to(torch.bfloat16).double()
+    for t in range(2):
+        col = cols[:, t]
+        col[lay["q"][0]:lay["q"][1]] = r.repeat(Hq)
+        col[lay["g"][0]:lay["g"][1]] = gate[t].reshape(-1)
+        col[lay["k"][0]:lay["k"][1]] = (r if t == 1 else -r).repeat(Hkv)
+        col[lay["v"][0]:lay["v"][1]] = v[t].reshape(-1)
+    w_in = cols.to(torch.bfloat16)  # every entry is exactly representable
+    assert torch.equal(w_in.double(), cols)
+    w_out = torch.randn(hidden, Hq * D, generator=g).to(torch.bfloat16)
+    x = torch.eye(2, hidden).to(torch.bfloat16)
+    ones = torch.ones(D, dtype=torch.bfloat16)
+    ref = A.attn_layer(x, w_in, w_out, ones, ones, [0, 2])
+    kv_of = torch.arange(Hq) // (Hq // Hkv)
+    out = np.stack([(v[t][kv_of] * torch.sigmoid(gate[t])).numpy() for t in range(2)])  # [2, 24, 256]
+    np.testing.assert_allclose(ref["out"].reshape(2, Hq, D), out, rtol=1e-12, atol=1e-13)
+    y = oracle.round_bf16(out).reshape(2, -1) @ w_out.double().numpy().T
+    np.testing.assert_allclose(ref["y"], y, rtol=1e-12, atol=1e-12)

@@ -666,11 +666,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(AttnDecPara
   }
 }
 
-// merge the splits of (sequence n, query head h): o = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M}
+// merge the splits of (sequence n, query head h): o = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M}.
+// The splits' weights e^{m_s - M} are formed once per CTA in shared memory (kDecMergeMax splits at
+// a time), then each thread (one output dim) sums its column with four loads in flight.
+constexpr int kDecMergeMax = 512;
 __global__ void __launch_bounds__(kAD) attn_decode_combine_kernel(AttnDecParams p, const bf16* g, long long ld_g,
                                                                   bf16* out) {
   const int n = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
   const int kvh = h / kAGrp, j = h % kAGrp;
+  __shared__ float w_s[kDecMergeMax];
+  __shared__ float red_s[kAD / 32];
   const int len = p.cache_len[n] + 1;
   if (len > p.cap) {  // reported by the cache write; nothing was attended: a zero output row
     out[(static_cast<long long>(n) * kAHq + h) * kAD + d] = __float2bfloat16(0.f);
@@ -678,14 +683,44 @@ __global__ void __launch_bounds__(kAD) attn_decode_combine_kernel(AttnDecParams 
   }
   const int used = (len + kDecSplit - 1) / kDecSplit;
   const float* base = p.part + (static_cast<long long>(n) * kAHkv + kvh) * p.n_splits * kAGrp * kDecPart;
+  // M = max over the splits of m_s
   float M = -INFINITY;
-  for (int s2 = 0; s2 < used; ++s2) M = fmaxf(M, base[(s2 * kAGrp + j) * kDecPart + kAD]);
-  float L = 0.f, O = 0.f;
-  for (int s2 = 0; s2 < used; ++s2) {
-    const float* ps = base + (s2 * kAGrp + j) * kDecPart;
-    const float w = expf(ps[kAD] - M);
-    L = fmaf(ps[kAD + 1], w, L);
-    O = fmaf(ps[d], w, O);
+  for (int s2 = d; s2 < used; s2 += kAD) M = fmaxf(M, base[(s2 * kAGrp + j) * kDecPart + kAD]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if ((d & 31) == 0) red_s[d >> 5] = M;
+  __syncthreads();
+  M = red_s[0];
+#pragma unroll
+  for (int w = 1; w < kAD / 32; ++w) M = fmaxf(M, red_s[w]);
+  float O = 0.f, L = 0.f;
+  for (int c0 = 0; c0 < used; c0 += kDecMergeMax) {
+    const int cn = min(kDecMergeMax, used - c0);
+    __syncthreads();  // red_s and w_s are free
+    float Lp = 0.f;
+    for (int s2 = d; s2 < cn; s2 += kAD) {
+      const float* ps = base + ((c0 + s2) * kAGrp + j) * kDecPart;
+      const float w = expf(ps[kAD] - M);
+      w_s[s2] = w;
+      Lp = fmaf(ps[kAD + 1], w, Lp);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+    if ((d & 31) == 0) red_s[d >> 5] = Lp;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kAD / 32; ++w) L += red_s[w];
+    const float* col = base + (static_cast<long long>(c0) * kAGrp + j) * kDecPart + d;
+    int s2 = 0;
+    for (; s2 + 4 <= cn; s2 += 4) {
+      const float o0 = col[(s2 + 0) * kAGrp * kDecPart], o1 = col[(s2 + 1) * kAGrp * kDecPart];
+      const float o2 = col[(s2 + 2) * kAGrp * kDecPart], o3 = col[(s2 + 3) * kAGrp * kDecPart];
+      O = fmaf(o0, w_s[s2], O);
+      O = fmaf(o1, w_s[s2 + 1], O);
+      O = fmaf(o2, w_s[s2 + 2], O);
+      O = fmaf(o3, w_s[s2 + 3], O);
+    }
+    for (; s2 < cn; ++s2) O = fmaf(col[s2 * kAGrp * kDecPart], w_s[s2], O);
   }
   const float gv = __bfloat162float(g[static_cast<long long>(n) * ld_g + h * kAD + d]);
   out[(static_cast<long long>(n) * kAHq + h) * kAD + d] = __float2bfloat16(O / L / (1.0f + expf(-gv)));

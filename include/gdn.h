@@ -36,7 +36,7 @@
  *   - Recurrent state: fp32 [N][H_v][128 (d_v)][128 (d_k)], row-major.
  *     Conv state: bf16 [N][3][C_conv], the 3 most recent raw tokens, oldest first.
  *   - `err` (nullable) is a device int the kernels OR error bits into
- *     (1 = a bounded wait timed out, 2 = cluster exchange failed,
+ *     (1 = a bounded wait timed out, 2 = reserved,
  *     4 = cu_seqlens on the device disagreed with cu_seqlens_host, 8 = a decode
  *     state_slot outside the pool, 16 = an attention KV cache with no row left).  It is
  *     never cleared by the library.  Read it after synchronising.

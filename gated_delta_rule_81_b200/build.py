@@ -23,7 +23,7 @@ NVCC_FLAGS = [
 
 TARGETS = {
     "libgdn.so": ["gdn_api.cu", "gdn_prefill.cu", "gdn_decode.cu", "gdn_noalloc.cu", "gdn_gemm.cu", "gdn_attention.cu"],
-    "libgdn_selftest.so": ["umma_selftest.cu"],
+    "libgdn_selftest.so": ["umma_selftest.cu", "wait_selftest.cu"],
 }
 
 

@@ -149,3 +149,52 @@ def test_layer_sizes_and_rejections(lib):
     small = args[:11] + (1024,) + args[12:]
     assert lib.gdn_layer_prefill(ctypes.byref(L), *small) == 7
     assert lib.gdn_layer_prefill(ctypes.byref(L), 0, 64, *args[2:]) == 0
+
+
+def _attn_layer(hidden=5120):
+    L = gdn.GdnAttnLayer()
+    L.w_in, L.ld_w_in, L.w_out, L.ld_w_out = 0x100000, hidden, 0x8000000, 24 * 256
+    L.q_norm_w, L.k_norm_w, L.hidden = 0x10000000, 0x10001000, hidden
+    return L
+
+
+def test_attention_sizes_and_rejections(lib):
+    up = lambda n: -(-n // 1024) * 1024
+    n_in, hd = 2 * 24 * 256 + 2 * 4 * 256, 24 * 256
+    assert lib.gdn_attn_layer_workspace_size(2, 100) == up(200 * n_in * 2) + 2 * up(200 * hd * 2)
+    assert lib.gdn_attn_layer_workspace_size(-1, 100) == 0
+    # decode: projection, q_hat, attention output, then fp32 partials (o[256], m, l) per
+    # (sequence, KV head, split of 512 cache rows, query head of the group)
+    for N, cap in ((64, 4096), (3, 153), (1, 513)):
+        parts = N * 4 * (-(-cap // 512)) * 6 * 258 * 4
+        assert lib.gdn_attn_decode_workspace_size(N, cap) == up(N * n_in * 2) + 2 * up(N * hd * 2) + up(parts)
+    assert lib.gdn_attn_decode_workspace_size(4, -1) == 0
+
+    L = _attn_layer()
+    B, T, cap = 1, 256, 512
+    ws_bytes = lib.gdn_attn_layer_workspace_size(B, T)
+    # x, k_cache, v_cache, cache_cap, y, ldy, workspace, bytes, err, stream
+    ok_args = [0x20000000, 5120, 0x30000000, 0x40000000, cap, 0x50000000, 5120, 0x60000000, ws_bytes, None, None]
+    bad = lambda **kw: [kw.get(str(i), a) for i, a in enumerate(ok_args)]
+    prefill = lambda L, B, T, args: lib.gdn_attn_layer_prefill(ctypes.byref(L), B, T, *args)
+    assert prefill(L, -1, T, ok_args) == 1                       # bad count
+    assert prefill(L, B, T, bad(**{"4": 100})) == 1              # cache smaller than the prompt
+    assert prefill(L, B, T, bad(**{"0": None})) == 1             # null input
+    assert prefill(L, B, T, bad(**{"8": ws_bytes - 1})) == 7     # workspace too small
+    assert prefill(L, B, T, bad(**{"2": 0x30000008})) == 3       # misaligned K cache
+    assert prefill(L, B, T, bad(**{"7": 0x50000000})) == 4       # workspace overlaps y
+    assert prefill(L, 0, T, ok_args) == 0                        # nothing to do, nothing launched
+    assert prefill(_attn_layer(5000), B, T, ok_args) == 2        # hidden not a multiple of 64
+
+    N = 4
+    dws = lib.gdn_attn_decode_workspace_size(N, cap)
+    # x, ldx, k_cache, v_cache, cache_cap, cache_len, y, ldy, workspace, bytes, err, stream
+    d_args = [0x20000000, 5120, 0x30000000, 0x40000000, cap, 0x70000000, 0x50000000, 5120, 0x60000000, dws, None,
+              None]
+    dbad = lambda **kw: [kw.get(str(i), a) for i, a in enumerate(d_args)]
+    step = lambda N, args: lib.gdn_attn_layer_decode_step(ctypes.byref(L), N, *args)
+    assert step(N, dbad(**{"4": 0})) == 1                        # no cache
+    assert step(N, dbad(**{"5": None})) == 1                     # no cache_len
+    assert step(N, dbad(**{"9": dws - 1})) == 7                  # workspace too small
+    assert step(N, dbad(**{"3": 0x40000004})) == 3               # misaligned V cache
+    assert step(0, d_args) == 0                                  # no sequences, nothing launched

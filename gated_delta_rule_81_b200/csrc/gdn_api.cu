@@ -169,6 +169,104 @@ gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens
                         out, workspace, workspace_bytes, err, stream);
 }
 
+// Device copies of gdn_prefill_host's host tensors, after the prefill workspace, each from a
+// 1 KiB boundary: q, k, v, z, a, b packed [T_tot][channels], then state, conv_in, conv_out, out.
+struct HostStage {
+  size_t q, k, v, z, a, b, state, conv_in, conv_out, out, end;
+};
+
+static HostStage host_stage_layout(int H_k, int H_v, int B, int T) {
+  const size_t T_tot = static_cast<size_t>(B) * T;
+  const size_t qk = T_tot * H_k * GDN_HEAD_DIM * 2, vz = T_tot * H_v * GDN_HEAD_DIM * 2, ab = T_tot * H_v * 2;
+  const size_t state = static_cast<size_t>(B) * H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * 4;
+  const size_t conv = static_cast<size_t>(B) * 3 * (2 * H_k + H_v) * GDN_HEAD_DIM * 2;
+  const long long n_chunks = static_cast<long long>(B) * ((T + GDN_CHUNK - 1) / GDN_CHUNK);
+  HostStage L;
+  size_t o = round_up(gdn_prefill_workspace_size(H_k, H_v, B, n_chunks), 1024);
+  L.q = o; o += round_up(qk, 1024);
+  L.k = o; o += round_up(qk, 1024);
+  L.v = o; o += round_up(vz, 1024);
+  L.z = o; o += round_up(vz, 1024);
+  L.a = o; o += round_up(ab, 1024);
+  L.b = o; o += round_up(ab, 1024);
+  L.state = o; o += round_up(state, 1024);
+  L.conv_in = o; o += round_up(conv, 1024);
+  L.conv_out = o; o += round_up(conv, 1024);
+  L.out = o; o += round_up(vz, 1024);
+  L.end = o;
+  return L;
+}
+
+size_t gdn_prefill_host_workspace_size(int H_k, int H_v, int B, int T) {
+  if (H_k <= 0 || H_v <= 0 || B < 0 || T < 0) return 0;
+  return host_stage_layout(H_k, H_v, B, T).end;
+}
+
+gdn_status gdn_prefill_host(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
+                            const void* conv_in, void* conv_out, void* out, void* workspace, size_t workspace_bytes,
+                            int* err, void* stream) {
+  if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+  const long long T_tot = static_cast<long long>(B) * T;
+  if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
+  gdn_status st = check_inputs(in, T_tot);
+  if (st != GDN_OK) return st;
+  if (B == 0) return GDN_OK;
+  if (T_tot > 0 && !out) return GDN_ERR_INVALID_ARG;
+  if (T_tot > 0 && (st = check_out_alias(in, T_tot, out)) != GDN_OK) return st;
+  const HostStage S = host_stage_layout(in->H_k, in->H_v, B, T);
+  if (!workspace || workspace_bytes < S.end) return GDN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  const size_t state_bytes = static_cast<size_t>(B) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(B) * 3 * (2 * in->H_k + in->H_v) * GDN_HEAD_DIM * sizeof(bf16);
+  const size_t out_bytes = static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
+  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
+  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
+    return GDN_ERR_ALIAS;
+  if (overlap(state_out, state_bytes, out, out_bytes) || overlap(conv_out, conv_bytes, out, out_bytes))
+    return GDN_ERR_ALIAS;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t qk_w = static_cast<size_t>(in->H_k) * GDN_HEAD_DIM, vz_w = static_cast<size_t>(in->H_v) * GDN_HEAD_DIM;
+  // inputs in: one (strided) copy per tensor into its packed device copy
+  struct Part { const void* src; long long stride; size_t width; size_t off; };
+  const Part parts[6] = {{in->q, in->stride_q, qk_w, S.q}, {in->k, in->stride_k, qk_w, S.k},
+                         {in->v, in->stride_v, vz_w, S.v}, {in->z, in->stride_z, vz_w, S.z},
+                         {in->a, in->stride_a, static_cast<size_t>(in->H_v), S.a},
+                         {in->b, in->stride_b, static_cast<size_t>(in->H_v), S.b}};
+  if (T_tot > 0) {
+    for (const Part& pt : parts) {
+      if (cudaMemcpy2DAsync(ws + pt.off, pt.width * 2, pt.src, static_cast<size_t>(pt.stride) * 2, pt.width * 2,
+                            static_cast<size_t>(T_tot), cudaMemcpyHostToDevice, cs) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    }
+  }
+  float* d_state = reinterpret_cast<float*>(ws + S.state);
+  if (state_in && cudaMemcpyAsync(d_state, state_in, state_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (conv_in && cudaMemcpyAsync(ws + S.conv_in, conv_in, conv_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  // the prefill on the device copies (state updated in place)
+  gdn_inputs d = *in;
+  d.q = ws + S.q; d.k = ws + S.k; d.v = ws + S.v; d.z = ws + S.z; d.a = ws + S.a; d.b = ws + S.b;
+  d.stride_q = d.stride_k = static_cast<long long>(qk_w);
+  d.stride_v = d.stride_z = static_cast<long long>(vz_w);
+  d.stride_a = d.stride_b = in->H_v;
+  const long long n_chunks = static_cast<long long>(B) * ((T + GDN_CHUNK - 1) / GDN_CHUNK);
+  st = prefill_common(&d, B, T_tot, n_chunks, nullptr, T, state_in ? d_state : nullptr,
+                      state_out ? d_state : nullptr, conv_in ? ws + S.conv_in : nullptr,
+                      conv_out ? ws + S.conv_out : nullptr, ws + S.out, workspace, workspace_bytes, err, stream);
+  if (st != GDN_OK) return st;
+  // outputs back
+  if (T_tot > 0 && cudaMemcpyAsync(out, ws + S.out, out_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (state_out && cudaMemcpyAsync(state_out, d_state, state_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (conv_out && cudaMemcpyAsync(conv_out, ws + S.conv_out, conv_bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return GDN_OK;
+}
+
 gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long ldb, void* C, long long ldc, int M,
                          int N, int K, int* err, void* stream) {
   if (M < 0 || N < 0 || K < 0) return GDN_ERR_INVALID_ARG;

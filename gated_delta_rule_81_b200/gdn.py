@@ -76,7 +76,8 @@ SCHEDULE_FUSED = 2         # one overlapped launch whenever the scan units fit i
 _lib = None
 _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_longlong
 
-EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_decode_step",
+EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_prefill_host_workspace_size",
+           "gdn_prefill_host", "gdn_decode_step",
            "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
            "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
            "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string")
@@ -97,6 +98,10 @@ def load(path: str | None = None):
     lib.gdn_prefill_workspace_size.restype = _sz
     lib.gdn_prefill.argtypes = [P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.gdn_prefill.restype = _i
+    lib.gdn_prefill_host_workspace_size.argtypes = [_i, _i, _i, _i]
+    lib.gdn_prefill_host_workspace_size.restype = _sz
+    lib.gdn_prefill_host.argtypes = [P, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+    lib.gdn_prefill_host.restype = _i
     lib.gdn_prefill_varlen.argtypes = [P, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
     lib.gdn_prefill_varlen.restype = _i
     lib.gdn_decode_step.argtypes = [P, _i, _vp, _vp, _vp, _vp, _vp]
@@ -222,6 +227,26 @@ def prefill(inp: GdnInputs, B: int, T: int, state_in=None, conv_in=None, *, want
                            _ptr(conv_out), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err), _stream()),
            "gdn_prefill")
     return out, state_out, conv_out
+
+
+def prefill_host_workspace_size(H_k: int, H_v: int, B: int, T: int) -> int:
+    return int(load().gdn_prefill_host_workspace_size(H_k, H_v, B, T))
+
+
+def prefill_host(inp: GdnInputs, B: int, T: int, out, state_in=None, state_out=None, conv_in=None, conv_out=None, *,
+                 workspace=None, err=None, stream=None):
+    """gdn_prefill_host: `inp` built from pinned host tensors (q, k, v, a, b, z) and device
+    weights; out, state_in / state_out, conv_in / conv_out are pinned host tensors (or None).
+    Asynchronous on `stream` (a torch.cuda.Stream, default the current one); returns out."""
+    lib = load()
+    if workspace is None:
+        workspace = torch.empty(prefill_host_workspace_size(inp.H_k, inp.H_v, B, T), dtype=torch.uint8,
+                                device=torch.device("cuda", torch.cuda.current_device()))
+    st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    _check(lib.gdn_prefill_host(ctypes.byref(inp), B, T, _ptr(state_in), _ptr(state_out), _ptr(conv_in),
+                                _ptr(conv_out), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(err), st),
+           "gdn_prefill_host")
+    return out
 
 
 def prefill_varlen(inp: GdnInputs, cu_seqlens, cu_seqlens_host, state_in=None, conv_in=None, *, want_state=True,

@@ -119,6 +119,25 @@ gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in
                        size_t workspace_bytes, int* err, void* stream);
 
 /*
+ * gdn_prefill for tensors that live in host memory.  The per-token inputs q, k, v, a, b, z
+ * of `in` (with its token strides), state_in, state_out, conv_in, conv_out and out are HOST
+ * pointers, page-locked for the copies to run asynchronously; conv_w, A_log and norm_w stay
+ * device pointers (the layer's weights live on the GPU).  On `stream`, in order: one copy
+ * per input tensor into packed device copies held in `workspace` (after the prefill's own
+ * scratch), gdn_prefill on them (the state updated in place on the device), one copy per
+ * output back to the host.  Semantics, nullable arguments and errors as gdn_prefill; the
+ * host buffers must stay valid and unmodified until the stream has passed the call.  Two
+ * calls on two streams with two workspaces overlap one call's input copies with the other's
+ * compute and output copies (the host link is full duplex).
+ *   workspace  device memory of gdn_prefill_host_workspace_size(H_k, H_v, B, T) bytes,
+ *              16-byte aligned, owned by the caller.
+ */
+size_t gdn_prefill_host_workspace_size(int H_k, int H_v, int B, int T);
+gdn_status gdn_prefill_host(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
+                            const void* conv_in, void* conv_out, void* out, void* workspace,
+                            size_t workspace_bytes, int* err, void* stream);
+
+/*
  * Prefill of N variable-length sequences packed back to back.
  *   cu_seqlens       device int32 [N+1], cu[0] = 0, non-decreasing; sequence n is
  *                    tokens cu[n] .. cu[n+1]-1

@@ -198,3 +198,29 @@ def test_attention_sizes_and_rejections(lib):
     assert step(N, dbad(**{"9": dws - 1})) == 7                  # workspace too small
     assert step(N, dbad(**{"3": 0x40000004})) == 3               # misaligned V cache
     assert step(0, d_args) == 0                                  # no sequences, nothing launched
+
+
+def test_prefill_host_sizes_and_rejections(lib):
+    up = lambda n: -(-n // 1024) * 1024
+    H_k, H_v, B, T = 16, 48, 2, 100
+    T_tot, C_conv = B * T, (2 * H_k + H_v) * 128
+    base = up(lib.gdn_prefill_workspace_size(H_k, H_v, B, B * 2))
+    staged = 2 * up(T_tot * H_k * 128 * 2) + 3 * up(T_tot * H_v * 128 * 2) + 2 * up(T_tot * H_v * 2) + \
+        up(B * H_v * 128 * 128 * 4) + 2 * up(B * 3 * C_conv * 2)
+    need = lib.gdn_prefill_host_workspace_size(H_k, H_v, B, T)
+    assert need == base + staged
+    assert lib.gdn_prefill_host_workspace_size(H_k, H_v, -1, T) == 0
+    s = gdn.GdnInputs()
+    s.q, s.k, s.v, s.a, s.b, s.z = 0x1000000, 0x2000000, 0x3000000, 0x4000000, 0x5000000, 0x6000000
+    s.stride_q, s.stride_k, s.stride_v, s.stride_z, s.stride_a, s.stride_b = 2048, 2048, 6144, 6144, 48, 48
+    s.conv_w, s.A_log, s.norm_w = 0x7000000, 0x7100000, 0x7200000
+    s.H_k, s.H_v, s.scale = H_k, H_v, 1.0
+    # state_in, state_out, conv_in, conv_out, out, workspace, bytes, err, stream
+    args = [None, None, None, None, 0x8000000, 0x10000000, need, None, None]
+    call = lambda B, a: lib.gdn_prefill_host(ctypes.byref(s), B, T, *a)
+    assert call(-1, args) == 1
+    assert call(B, args[:4] + [None] + args[5:]) == 1            # no output
+    assert call(B, args[:6] + [need - 1] + args[7:]) == 7        # workspace too small
+    assert call(B, args[:4] + [0x3000000] + args[5:]) == 4       # output over the v input
+    assert call(B, args[:5] + [0x10000008] + args[6:]) == 3      # misaligned workspace
+    assert call(0, args) == 0                                    # nothing to do

@@ -432,6 +432,84 @@ def run_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120, H_k=16, H_v=
             "cublas_ms": cub, "flops": flops, "clocks": clk.report(), "steps": args.steps}
 
 
+def run_layer_serve_ours(args, world, rank, dev, pk, N=1, T=4096, steps_dec=64, hidden=5120, H_k=16, H_v=48):
+    """Prefill -> decode handoff of one delta-rule layer: N prompts of T = 4096 tokens through
+    gdn_layer_prefill, then 64 single-token gdn_layer_decode steps that continue in place from
+    the prefill's final state and conv buffers (the handoff is the same buffers, no copy).
+    Random dense weights (std 1/sqrt(fan_in)); L2 flushed before every timed call."""
+    from gated_delta_rule_81_b200 import gdn
+
+    g = torch.Generator().manual_seed(500 + rank)
+    n_in = int(gdn.load().gdn_layer_n_in(H_k, H_v))
+    C_conv = (2 * H_k + H_v) * 128
+    x = torch.randn(N * T, hidden, generator=g).to(torch.bfloat16).to(dev)
+    xd = torch.randn(steps_dec, N, hidden, generator=g).to(torch.bfloat16).to(dev)
+    w_in = (torch.randn(n_in, hidden, generator=g) * hidden ** -0.5).to(torch.bfloat16).to(dev)
+    w_out = (torch.randn(hidden, H_v * 128, generator=g) * (H_v * 128) ** -0.5).to(torch.bfloat16).to(dev)
+    w = {k: v.to(dev) for k, v in gin.weights(H_k, H_v, seed=rank).items()}
+    L = gdn.make_layer(w_in, w_out, w["conv_w"], w["A_log"], w["norm_w"], H_k, H_v,
+                       schedule=SCHEDULES[args.schedule])
+    S = torch.empty(N, H_v, 128, 128, dtype=torch.float32, device=dev)
+    C = torch.empty(N, 3, C_conv, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(N * T, hidden, dtype=torch.bfloat16, device=dev)
+    yd = torch.empty(N, hidden, dtype=torch.bfloat16, device=dev)
+    ws_p = torch.empty(gdn.layer_workspace_size(H_k, H_v, N, T), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(int(gdn.load().gdn_layer_decode_workspace_size(H_k, H_v, N, 1)), dtype=torch.uint8,
+                       device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev).zero_()
+    stream = torch.cuda.current_stream()
+
+    def hook(ev):
+        if ev is None:
+            L.events = None
+            return None
+        arr = (ctypes.c_void_p * 4)(*[e.cuda_event or (e.record(stream) or e.cuda_event) for e in ev])
+        L.events = ctypes.cast(arr, ctypes.c_void_p)
+        return arr
+
+    def serve(evs_p=None, evs_d=None):
+        flush_l2(flush)
+        keep = hook(evs_p)
+        gdn.layer_prefill(L, N, T, x, None, None, y=y, state_out=S, conv_out=C, workspace=ws_p, err=err)
+        for i in range(steps_dec):
+            flush_l2(flush)
+            keep = hook(evs_d[i] if evs_d else None)
+            gdn.layer_decode(L, N, 1, xd[i], S, C, y=yd, workspace=ws_d, err=err)
+        hook(None)
+        return keep
+
+    for _ in range(max(args.warmup, 1)):
+        serve()
+    torch.cuda.synchronize()
+    barrier(world)
+    reps = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            evs_p = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            evs_d = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps_dec)]
+            serve(evs_p, evs_d)
+            reps.append((evs_p, evs_d))
+        torch.cuda.synchronize()
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    prefill_ms = [p[0].elapsed_time(p[3]) for p, _ in reps]
+    dec = {"in_proj": [], "mixer": [], "out_proj": [], "step": []}
+    for _, evs_d in reps:
+        for e in evs_d:
+            dec["in_proj"].append(e[0].elapsed_time(e[1]))
+            dec["mixer"].append(e[1].elapsed_time(e[2]))
+            dec["out_proj"].append(e[2].elapsed_time(e[3]))
+            dec["step"].append(e[0].elapsed_time(e[3]))
+    dec_total = max_over_ranks(sum(dec["step"]), world)
+    bytes_step = (n_in * hidden + hidden * H_v * 128) * 2 + N * (2 * H_v * 128 * 128 * 4 + 2 * 3 * C_conv * 2) + \
+        N * (hidden * 2 * 2 + n_in * 2 * 2 + H_v * 128 * 2 * 2)
+    return {"N": N, "T": T, "steps_dec": steps_dec, "prefill_ms": statistics.mean(prefill_ms),
+            "decode_ms": {k: statistics.mean(v) for k, v in dec.items()}, "decode_total_ms": dec_total,
+            "bytes_step": bytes_step, "clocks": clk.report(), "steps": args.steps}
+
+
 def run_attn_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120):
     """One global-attention layer (24/4 GQA, head dim 256), B = 1, T = 4096, hidden 5120, random
     dense weights (std 1/sqrt(fan_in)); times in_proj, attention (norm + rotary + flash) and
@@ -621,12 +699,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "attn_layer", "attn_decode"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "layer_serve", "attn_layer",
+                                                              "attn_decode"],
                     default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
                          "overlapped in one launch whenever the scan units fit in half the SMs)")
+    ap.add_argument("--serve-seqs", type=int, default=1,
+                    help="layer_serve: sequences prefilled and then decoded together")
     ap.add_argument("--attn-seqs", type=int, default=64,
                     help="attn_decode: sequences per step (each with a 4096-row KV cache)")
     ap.add_argument("--decode-tokens", type=int, default=1,
@@ -708,6 +789,29 @@ def main():
                 "torch_sdpa": None if r["sdpa_ms"] is None else {
                     "ms": round(r["sdpa_ms"], 5), "tflops": r["flops"]["attention"] / (r["sdpa_ms"] * 1e-3) / 1e12},
                 "gpu_launches": 4 * r["steps"], "clocks": r["clocks"]}), flush=True)
+        return 0
+    if args.workload == "layer_serve":
+        r = run_layer_serve_ours(args, world, rank, dev, pk, N=args.serve_seqs)
+        if rank == 0:
+            dm = r["decode_ms"]
+            tok_s = world * r["N"] * r["steps_dec"] * r["steps"] / (r["decode_total_ms"] / 1e3)
+            gbs = r["bytes_step"] / (dm["step"] * 1e-3) / 1e9
+            print(json.dumps({
+                "metric": "delta-layer decode tokens/s after a layer prefill (prefill -> decode handoff)",
+                "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": r["steps"], "warmup": args.warmup,
+                "ms_per_step": r["prefill_ms"] + dm["step"] * r["steps_dec"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"delta-layer-serve-{r['N']}seq-prompt{r['T']}-decode{r['steps_dec']}"
+                                       f"-hidden5120-16x48", "sequences": r["N"], "prompt": r["T"],
+                           "decode_steps": r["steps_dec"], "weights": "random dense, std 1/sqrt(fan_in)",
+                           "l2": "flushed before every timed call",
+                           "handoff": "decode continues in place on the prefill's state and conv buffers"},
+                "prefill_ms": round(r["prefill_ms"], 5),
+                "decode_step_ms": {k: round(v, 5) for k, v in dm.items()},
+                "roofline": {"kernel": "layer decode step (in_proj GEMM + decode + out_proj GEMM)", "bound": "hbm",
+                             "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                             "traffic": None, "algorithmic_bytes_per_step": r["bytes_step"]},
+                "gpu_launches": (5 + 3 * r["steps_dec"]) * r["steps"], "clocks": r["clocks"]}), flush=True)
         return 0
     if args.workload == "layer":
         r = run_layer_ours(args, world, rank, dev, pk)

@@ -354,6 +354,65 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
   return GDN_OK;
 }
 
+size_t gdn_layer_decode_workspace_size(int H_k, int H_v, int N, int T) {
+  if (H_k <= 0 || H_v <= 0 || N < 0 || T < 1 || T > gdn::kMaxDecodeTokens) return 0;
+  const size_t T_tot = static_cast<size_t>(N) * T;
+  return round_up(T_tot * layer_ld_proj(H_k, H_v) * 2, 1024) +
+         round_up(T_tot * static_cast<size_t>(H_v) * GDN_HEAD_DIM * 2, 1024);
+}
+
+gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, long long ldx, float* state,
+                            void* conv_state, const int* state_slot, int n_slots, void* y, long long ldy,
+                            void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  if (!L || N < 0 || T < 1 || T > gdn::kMaxDecodeTokens) return GDN_ERR_INVALID_ARG;
+  if (L->H_k <= 0 || L->H_v <= 0 || L->hidden <= 0 || L->H_v % L->H_k != 0) return GDN_ERR_INVALID_ARG;
+  if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
+  if (N == 0) return GDN_OK;
+  if (!x || !y || !L->w_in || !L->w_out) return GDN_ERR_INVALID_ARG;
+  const long long T_tot = static_cast<long long>(N) * T;
+  const size_t need = gdn_layer_decode_workspace_size(L->H_k, L->H_v, N, T);
+  if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  if (ldy < L->hidden) return GDN_ERR_INVALID_ARG;
+  if (overlap(y, (static_cast<size_t>(T_tot - 1) * ldy + L->hidden) * 2, workspace, need)) return GDN_ERR_ALIAS;
+  const long long n_in = gdn_layer_n_in(L->H_k, L->H_v), ld_p = layer_ld_proj(L->H_k, L->H_v);
+  const long long d_v = static_cast<long long>(L->H_v) * GDN_HEAD_DIM;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  bf16* proj = reinterpret_cast<bf16*>(ws);
+  bf16* mix = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(T_tot) * ld_p * 2, 1024));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) {
+    if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
+  };
+  mark(0);
+  gdn_status s = gdn_gemm_bf16(x, ldx, L->w_in, L->ld_w_in, proj, ld_p, static_cast<int>(T_tot),
+                               static_cast<int>(n_in), L->hidden, err, stream);
+  if (s != GDN_OK) return s;
+  mark(1);
+  const long long HkD = static_cast<long long>(L->H_k) * GDN_HEAD_DIM;
+  gdn_inputs in = {};
+  in.q = proj;
+  in.k = proj + HkD;
+  in.v = proj + 2 * HkD;
+  in.z = proj + 2 * HkD + d_v;
+  in.a = proj + 2 * HkD + 2 * d_v;
+  in.b = proj + 2 * HkD + 2 * d_v + L->H_v;
+  in.stride_q = in.stride_k = in.stride_v = in.stride_z = in.stride_a = in.stride_b = ld_p;
+  in.conv_w = L->conv_w;
+  in.A_log = L->A_log;
+  in.norm_w = L->norm_w;
+  in.H_k = L->H_k;
+  in.H_v = L->H_v;
+  in.scale = L->scale;
+  s = gdn_decode_multi(&in, N, T, state, conv_state, state_slot, state_slot ? n_slots : N, mix, err, stream);
+  if (s != GDN_OK) return s;
+  mark(2);
+  s = gdn_gemm_bf16(mix, d_v, L->w_out, L->ld_w_out, y, ldy, static_cast<int>(T_tot), L->hidden,
+                    static_cast<int>(d_v), err, stream);
+  if (s != GDN_OK) return s;
+  mark(3);
+  return GDN_OK;
+}
+
 gdn_status gdn_attention_prefill(const void* q_hat, const void* k, const void* v, const void* g, long long ld_g,
                                  int B, int T, void* out, int* err, void* stream) {
   if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;

@@ -79,6 +79,7 @@ _vp, _sz, _i, _ll = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_lon
 EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "gdn_prefill_host_workspace_size",
            "gdn_prefill_host", "gdn_decode_step",
            "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
+           "gdn_layer_decode_workspace_size", "gdn_layer_decode",
            "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
            "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string")
 MAX_DECODE_TOKENS = 8
@@ -117,6 +118,11 @@ def load(path: str | None = None):
     lib.gdn_layer_prefill.argtypes = [ctypes.POINTER(GdnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _vp, _vp, _ll, _vp,
                                       _sz, _vp, _vp]
     lib.gdn_layer_prefill.restype = _i
+    lib.gdn_layer_decode_workspace_size.argtypes = [_i, _i, _i, _i]
+    lib.gdn_layer_decode_workspace_size.restype = _sz
+    lib.gdn_layer_decode.argtypes = [ctypes.POINTER(GdnLayer), _i, _i, _vp, _ll, _vp, _vp, _vp, _i, _vp, _ll, _vp, _sz,
+                                     _vp, _vp]
+    lib.gdn_layer_decode.restype = _i
     lib.gdn_attn_layer_workspace_size.argtypes = [_i, _i]
     lib.gdn_attn_layer_workspace_size.restype = _sz
     lib.gdn_attn_layer_prefill.argtypes = [ctypes.POINTER(GdnAttnLayer), _i, _i, _vp, _ll, _vp, _vp, _i, _vp, _ll,
@@ -350,6 +356,24 @@ def layer_prefill(L: GdnLayer, B: int, T: int, x, state_in=None, conv_in=None, *
                                  _ptr(conv_in), _ptr(conv_out), _ptr(y), y.stride(0), _ptr(workspace),
                                  workspace.numel(), _ptr(err), _stream()), "gdn_layer_prefill")
     return y, state_out, conv_out
+
+
+def layer_decode(L: GdnLayer, N: int, T: int, x, state, conv_state, state_slot=None, n_slots=None, *, y=None,
+                 workspace=None, err=None):
+    """gdn_layer_decode: T new tokens for each of N sequences (x [N*T][hidden]); state and
+    conv_state (the pool, or one slot per sequence) are updated in place.  Returns y."""
+    lib = load()
+    if y is None:
+        y = torch.empty(N * T, L.hidden, dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(int(lib.gdn_layer_decode_workspace_size(L.H_k, L.H_v, N, T)), dtype=torch.uint8,
+                                device=x.device)
+    if n_slots is None:
+        n_slots = state.shape[0]
+    _check(lib.gdn_layer_decode(ctypes.byref(L), N, T, _ptr(x), x.stride(0), _ptr(state), _ptr(conv_state),
+                                _ptr(state_slot), int(n_slots), _ptr(y), y.stride(0), _ptr(workspace),
+                                workspace.numel(), _ptr(err), _stream()), "gdn_layer_decode")
+    return y
 
 
 def make_attn_layer(w_in, w_out, q_norm_w, k_norm_w) -> GdnAttnLayer:

@@ -223,6 +223,24 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
                              float* state_out, const void* conv_in, void* conv_out, void* y, long long ldy,
                              void* workspace, size_t workspace_bytes, int* err, void* stream);
 
+/* Workspace bytes of gdn_layer_decode for N sequences of T new tokens (0 on bad arguments). */
+size_t gdn_layer_decode_workspace_size(int H_k, int H_v, int N, int T);
+
+/*
+ * Decode of one delta-rule layer: T = 1 .. GDN_MAX_DECODE_TOKENS new tokens for each of N
+ * sequences (x bf16 [N*T][ldx], token n*T + t = new token t of sequence n) -> y bf16
+ * [N*T][ldy].  Three launch groups on `stream`: gdn_gemm_bf16 (in_proj), gdn_decode_multi on
+ * the projection's columns (strided, no copy) with the states in place, gdn_gemm_bf16
+ * (out_proj).  state, conv_state, state_slot and n_slots as in gdn_decode_multi (state_slot
+ * NULL: sequence n uses slot n and n_slots is ignored).  A state left by gdn_layer_prefill
+ * (state_out, conv_out) continues here unchanged: the handoff from prefill to decode is the
+ * same buffers.  L->events, when set, gets 4 records as in gdn_layer_prefill.  Errors as
+ * those calls; y must not overlap the workspace.
+ */
+gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, long long ldx, float* state,
+                            void* conv_state, const int* state_slot, int n_slots, void* y, long long ldy,
+                            void* workspace, size_t workspace_bytes, int* err, void* stream);
+
 /*
  * The global-attention layer of the hybrid decoder (the fourth layer of every four):
  * model card "Agnes-3.0-Flash Preview", "Architecture" table, rows "Global attention"

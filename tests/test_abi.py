@@ -224,3 +224,25 @@ def test_prefill_host_sizes_and_rejections(lib):
     assert call(B, args[:4] + [0x3000000] + args[5:]) == 4       # output over the v input
     assert call(B, args[:5] + [0x10000008] + args[6:]) == 3      # misaligned workspace
     assert call(0, args) == 0                                    # nothing to do
+
+
+def test_layer_decode_sizes_and_rejections(lib):
+    up = lambda n: -(-n // 1024) * 1024
+    assert lib.gdn_layer_decode_workspace_size(16, 48, 256, 1) == up(256 * 16480 * 2) + up(256 * 6144 * 2)
+    assert lib.gdn_layer_decode_workspace_size(16, 48, 4, 9) == 0 and lib.gdn_layer_decode_workspace_size(16, 48, 4, 0) == 0
+    L = gdn.GdnLayer()
+    L.w_in, L.ld_w_in, L.w_out, L.ld_w_out = 0x100000, 5120, 0x20000000, 6144
+    L.conv_w, L.A_log, L.norm_w = 0x300000, 0x310000, 0x320000
+    L.H_k, L.H_v, L.hidden, L.scale = 16, 48, 5120, 1.0
+    N, T = 4, 2
+    need = lib.gdn_layer_decode_workspace_size(16, 48, N, T)
+    # x, ldx, state, conv_state, state_slot, n_slots, y, ldy, workspace, bytes, err, stream
+    args = [0x400000, 5120, 0x40000000, 0x50000000, None, 0, 0x900000, 5120, 0x60000000, need, None, None]
+    call = lambda N, T, a: lib.gdn_layer_decode(ctypes.byref(L), N, T, *a)
+    assert call(N, 0, args) == 1 and call(N, 9, args) == 1      # tokens per call out of range
+    assert call(N, T, args[:9] + [need - 1] + args[10:]) == 7    # workspace too small
+    assert call(N, T, args[:6] + [0x60000000] + args[7:]) == 4   # y inside the workspace
+    assert call(N, T, [None] + args[1:]) == 1                    # no input
+    assert call(0, T, args) == 0                                 # no sequences, nothing launched
+    L.hidden = 5000
+    assert call(N, T, args) == 2

@@ -74,3 +74,35 @@ def test_layer_schedules_bitwise_equal():
     b = run_layer(c, gdn.SCHEDULE_TWO_LAUNCHES)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("T_dec", [1, 3])
+def test_layer_decode_continues_the_layer_prefill(T_dec):
+    """gdn_layer_prefill of a prompt, then two gdn_layer_decode calls of T_dec tokens each on
+    the prefill's own final state and conv buffers (the handoff is the same buffers): the
+    decoded tokens' outputs and the final states match the oracle layer run over the whole
+    sequences."""
+    H_k, H_v, hidden, B, T0, calls = 2, 6, 256, 2, 70, 2
+    T = T0 + calls * T_dec
+    c = exact_layer_case(H_k, H_v, hidden, B, T, seed=40 + T_dec)
+    d = {k: c[k].cuda() for k in ("x", "w_in", "w_out")}
+    w = {k: v.cuda() for k, v in c["w"].items()}
+    L = gdn.make_layer(d["w_in"], d["w_out"], w["conv_w"], w["A_log"], w["norm_w"], H_k, H_v)
+    err = err_word()
+    xs = d["x"].reshape(B, T, hidden)
+    _, S, C = gdn.layer_prefill(L, B, T0, xs[:, :T0].reshape(B * T0, hidden).contiguous(), c["state"].cuda(),
+                                c["conv"].cuda(), err=err)
+    ys = []
+    for i in range(calls):
+        xi = xs[:, T0 + i * T_dec:T0 + (i + 1) * T_dec].reshape(B * T_dec, hidden).contiguous()
+        ys.append(gdn.layer_decode(L, B, T_dec, xi, S, C, err=err).reshape(B, T_dec, hidden))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oracle_layer(c)
+    y_ref = ref["y"].reshape(B, T, hidden)[:, T0:]
+    y = torch.cat(ys, dim=1)
+    e_y, e_s = out_error(y.reshape(-1, hidden), y_ref.reshape(-1, hidden)), state_error(S, ref["state"])
+    print(f"[parity] layer decode after a {T0}-token layer prefill, {calls} x {T_dec} tokens: y_err={e_y:.3e} "
+          f"state_err={e_s:.3e}")
+    assert e_y <= OUT_TOL and e_s <= STATE_TOL
+    np.testing.assert_array_equal(C.float().cpu().numpy(), ref["conv"])

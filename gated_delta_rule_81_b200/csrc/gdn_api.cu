@@ -368,7 +368,8 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
   if (L->H_k <= 0 || L->H_v <= 0 || L->hidden <= 0 || L->H_v % L->H_k != 0) return GDN_ERR_INVALID_ARG;
   if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
-  if (!x || !y || !L->w_in || !L->w_out) return GDN_ERR_INVALID_ARG;
+  if (!x || !y || !L->w_in || !L->w_out || !state || !conv_state) return GDN_ERR_INVALID_ARG;
+  if (state_slot && n_slots < 1) return GDN_ERR_INVALID_ARG;
   const long long T_tot = static_cast<long long>(N) * T;
   const size_t need = gdn_layer_decode_workspace_size(L->H_k, L->H_v, N, T);
   if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;

@@ -243,6 +243,7 @@ def test_layer_decode_sizes_and_rejections(lib):
     assert call(N, T, args[:9] + [need - 1] + args[10:]) == 7    # workspace too small
     assert call(N, T, args[:6] + [0x60000000] + args[7:]) == 4   # y inside the workspace
     assert call(N, T, [None] + args[1:]) == 1                    # no input
+    assert call(N, T, args[:2] + [None] + args[3:]) == 1         # no state: rejected before any launch
     assert call(0, T, args) == 0                                 # no sequences, nothing launched
     L.hidden = 5000
     assert call(N, T, args) == 2

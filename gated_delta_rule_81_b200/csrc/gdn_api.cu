@@ -69,6 +69,22 @@ gdn_status check_out_alias(const gdn_inputs* in, long long T_tot, const void* ou
   return GDN_OK;
 }
 
+// The layer entry points check the states the mixer will take before their first launch, so
+// that a rejected call launches nothing: alignment, and the aliasing rules of the mixer calls.
+gdn_status check_layer_states(int H_k, int H_v, int n, const float* state_in, const float* state_out,
+                              const void* conv_in, const void* conv_out) {
+  if (!aligned16(state_in) || !aligned16(state_out) || !aligned16(conv_in) || !aligned16(conv_out))
+    return GDN_ERR_MISALIGNED;
+  const size_t state_bytes = static_cast<size_t>(n) * H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(n) * 3 * (2 * H_k + H_v) * GDN_HEAD_DIM * sizeof(bf16);
+  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
+    return GDN_ERR_ALIAS;
+  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
+  if (overlap(state_out ? state_out : state_in, state_bytes, conv_out ? conv_out : conv_in, conv_bytes))
+    return GDN_ERR_ALIAS;
+  return GDN_OK;
+}
+
 gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long long n_chunks, const int* cu,
                           int T_uniform, const float* state_in, float* state_out, const void* conv_in,
                           void* conv_out, void* out, void* workspace, size_t workspace_bytes, int* err,
@@ -308,6 +324,8 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
   if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
   if (T_tot == 0) return GDN_OK;
   if (!x || !y || !L->w_in || !L->w_out) return GDN_ERR_INVALID_ARG;
+  gdn_status cs = check_layer_states(L->H_k, L->H_v, B, state_in, state_out, conv_in, conv_out);
+  if (cs != GDN_OK) return cs;
   const size_t need = gdn_layer_workspace_size(L->H_k, L->H_v, B, T);
   if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
   const long long n_in = gdn_layer_n_in(L->H_k, L->H_v), ld_p = layer_ld_proj(L->H_k, L->H_v);
@@ -370,6 +388,8 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
   if (N == 0) return GDN_OK;
   if (!x || !y || !L->w_in || !L->w_out || !state || !conv_state) return GDN_ERR_INVALID_ARG;
   if (state_slot && n_slots < 1) return GDN_ERR_INVALID_ARG;
+  gdn_status cs = check_layer_states(L->H_k, L->H_v, state_slot ? n_slots : N, state, nullptr, conv_state, nullptr);
+  if (cs != GDN_OK) return cs;
   const long long T_tot = static_cast<long long>(N) * T;
   const size_t need = gdn_layer_decode_workspace_size(L->H_k, L->H_v, N, T);
   if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;

@@ -149,6 +149,17 @@ def test_layer_sizes_and_rejections(lib):
     small = args[:11] + (1024,) + args[12:]
     assert lib.gdn_layer_prefill(ctypes.byref(L), *small) == 7
     assert lib.gdn_layer_prefill(ctypes.byref(L), 0, 64, *args[2:]) == 0
+    # state and conv checks come before the input projection is launched
+    # (args: B, T, x, ldx, state_in, state_out, conv_in, conv_out, y, ldy, workspace, bytes, err, stream)
+    def with_(**kw):
+        a = list(args)
+        for k, val in kw.items():
+            a[int(k[1:])] = val
+        return lib.gdn_layer_prefill(ctypes.byref(L), *a)
+    assert with_(i4=0x40000000, i5=0x40000000 + 4096) == 4       # state_in, state_out overlapping, not equal
+    assert with_(i6=0x50000000, i7=0x50000000) == 4              # conv_out == conv_in
+    assert with_(i4=0x40000000, i6=0x40000000) == 4              # state and conv history in the same place
+    assert with_(i4=0x40000008) == 3                             # misaligned state_in
 
 
 def _attn_layer(hidden=5120):
@@ -244,6 +255,8 @@ def test_layer_decode_sizes_and_rejections(lib):
     assert call(N, T, args[:6] + [0x60000000] + args[7:]) == 4   # y inside the workspace
     assert call(N, T, [None] + args[1:]) == 1                    # no input
     assert call(N, T, args[:2] + [None] + args[3:]) == 1         # no state: rejected before any launch
+    assert call(N, T, args[:2] + [0x40000004] + args[3:]) == 3   # misaligned state
+    assert call(N, T, args[:3] + [0x40000000 + 1024] + args[4:]) == 4  # conv state inside the state pool
     assert call(0, T, args) == 0                                 # no sequences, nothing launched
     L.hidden = 5000
     assert call(N, T, args) == 2

@@ -168,8 +168,9 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
 
 /*
  * The dense projections on either side of the mixer (hidden size 5120 -> q|k|v|z|a|b,
- * and 48*128 -> 5120): C = A B^T on the tensor cores, bf16 in and out, fp32
- * accumulation, one rounding to bf16 per output element.
+ * and 48*128 -> 5120; model card "Agnes-3.0-Flash Preview", "Architecture" table, rows
+ * "Hidden size" and "Delta-rule layers"): C = A B^T on the tensor cores, bf16 in and out,
+ * fp32 accumulation, one rounding to bf16 per output element.
  *   A  bf16 [M][lda], first K columns used        (activations, row-major)
  *   B  bf16 [N][ldb], first K columns used        (weights, one output channel per row)
  *   C  bf16 [M][ldc], first N columns written
@@ -182,9 +183,11 @@ gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long 
                          int N, int K, int* err, void* stream);
 
 /*
- * One delta-rule layer around the mixer: y = out_proj(mixer(in_proj(x))).
- * The input projection's output channels are q (H_k*128) | k (H_k*128) | v (H_v*128) |
- * z (H_v*128) | a (H_v) | b (H_v), n_in of them in all; no biases.
+ * One delta-rule layer around the mixer: y = out_proj(mixer(in_proj(x))) (model card
+ * "Agnes-3.0-Flash Preview", "Architecture" table: hidden size 5120, delta-rule layers of
+ * 16 key / 48 value heads of 128).  The pages give no layout for the projections; this
+ * library's reading: the input projection's output channels are q (H_k*128) | k (H_k*128) |
+ * v (H_v*128) | z (H_v*128) | a (H_v) | b (H_v), n_in of them in all; no biases.
  */
 typedef struct {
   const void* w_in;       /* bf16 [n_in][ld_w_in], first `hidden` columns used */

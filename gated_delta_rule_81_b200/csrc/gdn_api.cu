@@ -69,6 +69,29 @@ gdn_status check_out_alias(const gdn_inputs* in, long long T_tot, const void* ou
   return GDN_OK;
 }
 
+// The mixer's inputs as columns of the layer's projection buffer [T_tot][ld_p]:
+// q | k | v | z | a | b, read through the row stride ld_p (no copy).
+gdn_inputs layer_mixer_inputs(const gdn_layer* L, const bf16* proj, long long ld_p) {
+  const long long HkD = static_cast<long long>(L->H_k) * GDN_HEAD_DIM;
+  const long long d_v = static_cast<long long>(L->H_v) * GDN_HEAD_DIM;
+  gdn_inputs in = {};
+  in.q = proj;
+  in.k = proj + HkD;
+  in.v = proj + 2 * HkD;
+  in.z = proj + 2 * HkD + d_v;
+  in.a = proj + 2 * HkD + 2 * d_v;
+  in.b = proj + 2 * HkD + 2 * d_v + L->H_v;
+  in.stride_q = in.stride_k = in.stride_v = in.stride_z = in.stride_a = in.stride_b = ld_p;
+  in.conv_w = L->conv_w;
+  in.A_log = L->A_log;
+  in.norm_w = L->norm_w;
+  in.H_k = L->H_k;
+  in.H_v = L->H_v;
+  in.scale = L->scale;
+  in.schedule = L->schedule;
+  return in;
+}
+
 // The layer entry points check the states the mixer will take before their first launch, so
 // that a rejected call launches nothing: alignment, and the aliasing rules of the mixer calls.
 gdn_status check_layer_states(int H_k, int H_v, int n, const float* state_in, const float* state_out,
@@ -346,22 +369,7 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
                                static_cast<int>(n_in), L->hidden, err, stream);
   if (s != GDN_OK) return s;
   mark(1);
-  const long long HkD = static_cast<long long>(L->H_k) * GDN_HEAD_DIM;
-  gdn_inputs in = {};
-  in.q = proj;
-  in.k = proj + HkD;
-  in.v = proj + 2 * HkD;
-  in.z = proj + 2 * HkD + d_v;
-  in.a = proj + 2 * HkD + 2 * d_v;
-  in.b = proj + 2 * HkD + 2 * d_v + L->H_v;
-  in.stride_q = in.stride_k = in.stride_v = in.stride_z = in.stride_a = in.stride_b = ld_p;
-  in.conv_w = L->conv_w;
-  in.A_log = L->A_log;
-  in.norm_w = L->norm_w;
-  in.H_k = L->H_k;
-  in.H_v = L->H_v;
-  in.scale = L->scale;
-  in.schedule = L->schedule;
+  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
   s = gdn_prefill(&in, B, T, state_in, state_out, conv_in, conv_out, mix, ws_mixer, ws_mixer_bytes, err, stream);
   if (s != GDN_OK) return s;
   mark(2);
@@ -409,21 +417,7 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
                                static_cast<int>(n_in), L->hidden, err, stream);
   if (s != GDN_OK) return s;
   mark(1);
-  const long long HkD = static_cast<long long>(L->H_k) * GDN_HEAD_DIM;
-  gdn_inputs in = {};
-  in.q = proj;
-  in.k = proj + HkD;
-  in.v = proj + 2 * HkD;
-  in.z = proj + 2 * HkD + d_v;
-  in.a = proj + 2 * HkD + 2 * d_v;
-  in.b = proj + 2 * HkD + 2 * d_v + L->H_v;
-  in.stride_q = in.stride_k = in.stride_v = in.stride_z = in.stride_a = in.stride_b = ld_p;
-  in.conv_w = L->conv_w;
-  in.A_log = L->A_log;
-  in.norm_w = L->norm_w;
-  in.H_k = L->H_k;
-  in.H_v = L->H_v;
-  in.scale = L->scale;
+  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
   s = gdn_decode_multi(&in, N, T, state, conv_state, state_slot, state_slot ? n_slots : N, mix, err, stream);
   if (s != GDN_OK) return s;
   mark(2);

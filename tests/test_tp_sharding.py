@@ -112,3 +112,15 @@ def test_two_gloo_ranks_sum_to_the_unsharded_layer():
         hr = tp.head_range(H_k, H_v, 2, rank)
         np.testing.assert_array_equal(S, full["state"][:, hr.v0:hr.v1])
         np.testing.assert_array_equal(C, full["conv"][:, :, tp.conv_channels(H_k, H_v, hr).numpy()])
+
+
+def test_layer_needs_a_group_or_explicit_rank():
+    """Without torch.distributed initialised, TPDeltaLayer must be told tp and rank; the shard
+    helpers pass absent states through."""
+    assert not dist.is_initialized()
+    w = torch.zeros(1)
+    with pytest.raises(RuntimeError):
+        tp.TPDeltaLayer(w, w, w, w, w, 16, 48)
+    assert tp.shard_state(None, 16, 48, 2, 0) is None and tp.shard_conv_state(None, 16, 48, 2, 1) is None
+    st = torch.arange(2 * 48 * 2 * 2, dtype=torch.float32).reshape(2, 48, 2, 2)
+    assert torch.equal(tp.shard_state(st, 16, 48, 2, 1), st[:, 24:])

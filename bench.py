@@ -5,9 +5,12 @@
 
 Default workload: one delta-layer prefill, B = 1, T = 4096 tokens, 16 key / 48
 value heads, head dim 128 (the headline configuration), metric tokens/s per
-layer.  One step = one gdn_prefill call (conv-state kernel, prep kernel, scan
-kernel) over the whole batch, inputs resident in HBM; the L2 is flushed
-(256 MiB write) between timed steps and the flush is outside the timed events.
+layer.  One step = one gdn_prefill call over the whole batch (the conv-state
+kernel, then the prefill proper: one overlapped launch of the chunk-parallel
+prep and the sequential scan, or the two as separate launches, as the
+library's automatic schedule decides), inputs resident in HBM; the L2 is
+flushed (256 MiB write) between timed steps and the flush is outside the
+timed events.
 A secondary line item measures batched decode (256 sequences x 64 steps),
 state GB/s.  Under torchrun (N > 1) every rank runs its own batch (weak
 scaling, no collective on the data path); the time is the max over ranks.
@@ -56,9 +59,9 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {"scan": {"bytes": 442609664 + 44196608, "sha": "44d4966011593d14"},   # ncu, T=4096 layer
-           "prep": {"bytes": 101810688 + 334646272, "sha": "44d4966011593d14"},
-           "prefill_fused": {"bytes": 434084096 + 422704128, "sha": "44d4966011593d14"}}
+TRAFFIC = {(1, "scan"): {"bytes": 442609664 + 44196608, "sha": "44d4966011593d14"},   # ncu, T=4096 layer
+           (1, "prep"): {"bytes": 101810688 + 334646272, "sha": "44d4966011593d14"},
+           (1, "prefill_fused"): {"bytes": 434084096 + 422704128, "sha": "44d4966011593d14"}}
 DECODE_TRAFFIC = {"bytes": 829675264 + 766249984, "sha": "852a2d42cccfe44d"}  # ncu, one step of 256 sequences
 
 
@@ -256,6 +259,55 @@ def run_prefill_ours(args, world, rank, dev, pk, cfg_id=1):
             "kernel_ms": {"prep": statistics.mean(prep_ms), "scan": statistics.mean(scan_ms),
                           "helpers+gaps": statistics.mean(step_ms) - statistics.mean(prep_ms)
                           - statistics.mean(scan_ms)}}
+
+
+def prefill_roofline(res, cfg_id, pk, ms_per_step):
+    """Roofline object of a prefill run: the dominant kernel's algorithmic TFLOP/s from its live
+    CUDA-event time (the library's event hook, on the launching stream), against the measured
+    bf16 peak; DRAM traffic from the ncu capture of that kernel and workload when the kernel
+    source is unchanged since."""
+    T = res["T"]
+    kt = res["kernel_ms"]
+    step_flops = (scan_flop_per_token(res["H_v"]) + prep_flop_per_token(res["H_k"], res["H_v"])) * T
+    if kt["prep"] < 0.02:  # one fused launch: the library records its prep/scan split event next to the start
+        dom, flops = "prefill_fused", step_flops
+        kt = {"prefill_fused": kt["scan"], "helpers+gaps": kt["helpers+gaps"]}
+    else:
+        dom = "scan" if kt["scan"] >= kt["prep"] else "prep"
+        flops = (scan_flop_per_token(res["H_v"]) if dom == "scan" else prep_flop_per_token(res["H_k"], res["H_v"])) * T
+    achieved = flops / (kt[dom] * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    tr = TRAFFIC.get((cfg_id, dom))
+    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") else None
+    return {"kernel": f"{dom}_kernel", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "traffic_note": tr.get("note") if tr and traffic is not None else None,
+            "peak_source": f"{pk['source']} (bf16 burst)",
+            "algorithmic_flop_per_launch": flops, "launch_ms": kt[dom],
+            "kernel_ms": {k: round(v, 5) for k, v in kt.items()},
+            "whole_step": {"achieved": step_flops / (ms_per_step * 1e-3) / 1e12,
+                           "frac": step_flops / (ms_per_step * 1e-3) / 1e12 / peak}}
+
+
+def prefill_secondaries(args, world, rank, dev, pk):
+    """The other prefill configurations, each a short run of its own (warm-up, then timed steps
+    with the L2 flushed between them), for the record beside the headline."""
+    out = []
+    for cfg_id, steps in ((0, 20), (2, 3), (3, 5)):
+        a = argparse.Namespace(**vars(args))
+        a.steps, a.warmup = steps, 3
+        res = run_prefill_ours(a, world, rank, dev, pk, cfg_id)
+        ms = res["total_ms"] / steps
+        c = gin.CONFIGS[cfg_id]
+        out.append({"workload": c["name"], "metric": "gated-delta prefill tokens/s per layer",
+                    "value": world * res["T"] / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+                    "warmup": 3, "sequences": res["N"], "tokens": res["T"],
+                    "l2": "flushed between timed steps" + (" (inputs L2-resident: 12 MB)" if cfg_id == 0 else ""),
+                    "roofline": prefill_roofline(res, cfg_id, pk, ms), "clocks": res["clocks"],
+                    "gpu_launches": res["launches_per_step"] * steps})
+        del res
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e_prefill(args, world, rank, dev, case):
@@ -658,30 +710,32 @@ def cpu_oracle_tokens_per_s(min_seconds=10.0, max_reps=8):
 
 
 def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores (all of them, OpenMP over value heads), one full step
+    per timed step: the whole T = 4096, 48-value-head layer, nothing extrapolated."""
     if rank != 0:
         return 0
     import oracle
 
     case = gin.prefill_case(1)
     cu = case["cu_seqlens"].tolist()
-    heads = list(range(8))  # bounded sample per step: 8 of 48 value heads, scaled to the layer
-    oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=[0], want_conv=False)
+    oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=[0], want_conv=False)  # build + warm
     for _ in range(args.warmup):
-        oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=heads, want_conv=False)
+        oracle.mixer(case["inp"], cu, state_in=case["state_in"], want_conv=False)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.mixer(case["inp"], cu, state_in=case["state_in"], heads=heads, want_conv=False)
+        oracle.mixer(case["inp"], cu, state_in=case["state_in"], want_conv=False)
     el = time.perf_counter() - t0
-    layer_s_per_step = el / args.steps * (48 / len(heads))
-    value = case["T_tot"] / layer_s_per_step
+    s_per_step = el / args.steps
+    value = case["T_tot"] / s_per_step
     cfg = {"workload": gin.CONFIGS[1]["name"], "batch": 1, "seq_len": case["T_tot"], "H_k": 16, "H_v": 48,
            "head_dim": 128}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s_per_step * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": cfg,
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"each step: value heads 0-7 of 48 over T=4096, time scaled x6"},
+                             "sample": f"each step: the whole layer, 48 value heads over T=4096, fp64 "
+                                       f"({args.steps} steps in {el:.1f} s)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -699,6 +753,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the configurations 0, 2 and 3 that the default line reports beside the headline")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["decode", "layer", "layer_serve", "attn_layer",
                                                               "attn_decode"],
                     default="prefill4k",
@@ -846,26 +902,7 @@ def main():
     total_ms = res["total_ms"]
     value = world * T * args.steps / (total_ms / 1e3)
     ms_per_step = total_ms / args.steps
-
-    # dominant kernel, timed live in the timed region with the library's event hook
-    kt = res["kernel_ms"]
-    step_flops = (scan_flop_per_token(res["H_v"]) + prep_flop_per_token(res["H_k"], res["H_v"])) * T
-    if kt["prep"] < 0.02:  # one fused launch: the library records its prep/scan split event next to the start
-        dom, flops = "prefill_fused", step_flops
-        kt = {"prefill_fused": kt["scan"], "helpers+gaps": kt["helpers+gaps"]}
-    else:
-        dom = "scan" if kt["scan"] >= kt["prep"] else "prep"
-        flops = (scan_flop_per_token(res["H_v"]) if dom == "scan" else prep_flop_per_token(res["H_k"], res["H_v"])) * T
-    achieved = flops / (kt[dom] * 1e-3) / 1e12
-    peak = pk["bf16_tflops"]
-    tr = TRAFFIC.get(dom)
-    traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") and cfg_id == 1 else None
-    roof = {"kernel": f"{dom}_kernel", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": traffic, "peak_source": f"{pk['source']} (bf16 burst)",
-            "algorithmic_flop_per_launch": flops, "launch_ms": kt[dom],
-            "kernel_ms": {k: round(v, 5) for k, v in kt.items()},
-            "whole_step": {"achieved": step_flops / (ms_per_step * 1e-3) / 1e12,
-                           "frac": step_flops / (ms_per_step * 1e-3) / 1e12 / peak}}
+    roof = prefill_roofline(res, cfg_id, pk, ms_per_step)
     if cfg_id != 1:
         if rank == 0:
             c = gin.CONFIGS[cfg_id]
@@ -890,6 +927,8 @@ def main():
                                "frac": d["gbs"] / pk["hbm_gbs"], "traffic": decode_traffic(),
                                "peak_source": pk["source"]}}
 
+    others = None if args.no_secondary else prefill_secondaries(args, world, rank, dev, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_tokens_per_s()
@@ -909,6 +948,7 @@ def main():
             "gpu_launches": res["launches_per_step"] * args.steps,
             "clocks": res["clocks"],
             "secondary": decode,
+            "secondary_prefill": others,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -92,20 +92,47 @@ gdn_inputs layer_mixer_inputs(const gdn_layer* L, const bf16* proj, long long ld
   return in;
 }
 
+// The aliasing rule of every prefill entry point, in one place: among the state and conv
+// buffers and the output (out_bytes of it; nullptr when the call has none), a buffer the call
+// writes (state_out, conv_out, out) overlaps no other one, except that state_out may be
+// exactly state_in (the state is updated in place, each row by the one CTA that reads it).
+gdn_status check_state_aliases(int H_k, int H_v, int n, const float* state_in, const float* state_out,
+                               const void* conv_in, const void* conv_out, const void* out, size_t out_bytes) {
+  const size_t state_bytes = static_cast<size_t>(n) * H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
+  const size_t conv_bytes = static_cast<size_t>(n) * 3 * (2 * H_k + H_v) * GDN_HEAD_DIM * sizeof(bf16);
+  struct Buf {
+    const void* p;
+    size_t bytes;
+    bool written;
+  };
+  const Buf b[5] = {{state_in, state_bytes, false}, {state_out, state_bytes, true}, {conv_in, conv_bytes, false},
+                    {conv_out, conv_bytes, true}, {out, out_bytes, true}};
+  for (int i = 0; i < 5; ++i)
+    for (int j = i + 1; j < 5; ++j) {
+      if (!b[i].written && !b[j].written) continue;
+      if (i == 0 && j == 1 && state_in == state_out) continue;
+      if (overlap(b[i].p, b[i].bytes, b[j].p, b[j].bytes)) return GDN_ERR_ALIAS;
+    }
+  return GDN_OK;
+}
+
 // The layer entry points check the states the mixer will take before their first launch, so
 // that a rejected call launches nothing: alignment, and the aliasing rules of the mixer calls.
 gdn_status check_layer_states(int H_k, int H_v, int n, const float* state_in, const float* state_out,
                               const void* conv_in, const void* conv_out) {
   if (!aligned16(state_in) || !aligned16(state_out) || !aligned16(conv_in) || !aligned16(conv_out))
     return GDN_ERR_MISALIGNED;
+  return check_state_aliases(H_k, H_v, n, state_in, state_out, conv_in, conv_out, nullptr, 0);
+}
+
+// None of the state and conv buffers of a layer call may lie in its workspace (the projection,
+// the mixer output and the mixer's scratch are written there).
+bool states_in_workspace(int H_k, int H_v, int n, const void* s0, const void* s1, const void* c0, const void* c1,
+                         const void* ws, size_t ws_bytes) {
   const size_t state_bytes = static_cast<size_t>(n) * H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
   const size_t conv_bytes = static_cast<size_t>(n) * 3 * (2 * H_k + H_v) * GDN_HEAD_DIM * sizeof(bf16);
-  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
-    return GDN_ERR_ALIAS;
-  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
-  if (overlap(state_out ? state_out : state_in, state_bytes, conv_out ? conv_out : conv_in, conv_bytes))
-    return GDN_ERR_ALIAS;
-  return GDN_OK;
+  return overlap(s0, state_bytes, ws, ws_bytes) || overlap(s1, state_bytes, ws, ws_bytes) ||
+         overlap(c0, conv_bytes, ws, ws_bytes) || overlap(c1, conv_bytes, ws, ws_bytes);
 }
 
 gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long long n_chunks, const int* cu,
@@ -117,19 +144,17 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   if (N == 0) return GDN_OK;
   if (T_tot > 0 && !out) return GDN_ERR_INVALID_ARG;
   if (T_tot > 0 && (st = check_out_alias(in, T_tot, out)) != GDN_OK) return st;
-  const long long C_conv = static_cast<long long>(2 * in->H_k + in->H_v) * GDN_HEAD_DIM;
-  const size_t state_bytes = static_cast<size_t>(N) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
-  const size_t conv_bytes = static_cast<size_t>(N) * 3 * C_conv * sizeof(bf16);
   if (!aligned16(out) || !aligned16(state_in) || !aligned16(state_out) || !aligned16(conv_in) ||
       !aligned16(conv_out) || !aligned16(workspace))
     return GDN_ERR_MISALIGNED;
-  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
-    return GDN_ERR_ALIAS;
-  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
-  if (state_out && overlap(state_out, state_bytes, out, static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * 2))
-    return GDN_ERR_ALIAS;
+  if ((st = check_state_aliases(in->H_k, in->H_v, N, state_in, state_out, conv_in, conv_out, out,
+                                static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16))) != GDN_OK)
+    return st;
   const size_t need = gdn_prefill_workspace_size(in->H_k, in->H_v, N, n_chunks);
   if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  if (states_in_workspace(in->H_k, in->H_v, N, state_in, state_out, conv_in, conv_out, workspace, need) ||
+      overlap(out, static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16), workspace, need))
+    return GDN_ERR_ALIAS;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   gdn::PrefillParams p = {};
@@ -258,11 +283,9 @@ gdn_status gdn_prefill_host(const gdn_inputs* in, int B, int T, const float* sta
   const size_t state_bytes = static_cast<size_t>(B) * in->H_v * GDN_HEAD_DIM * GDN_HEAD_DIM * sizeof(float);
   const size_t conv_bytes = static_cast<size_t>(B) * 3 * (2 * in->H_k + in->H_v) * GDN_HEAD_DIM * sizeof(bf16);
   const size_t out_bytes = static_cast<size_t>(T_tot) * in->H_v * GDN_HEAD_DIM * sizeof(bf16);
-  if (overlap(conv_out, conv_bytes, conv_in, conv_bytes)) return GDN_ERR_ALIAS;
-  if (state_out && state_in && state_out != state_in && overlap(state_out, state_bytes, state_in, state_bytes))
-    return GDN_ERR_ALIAS;
-  if (overlap(state_out, state_bytes, out, out_bytes) || overlap(conv_out, conv_bytes, out, out_bytes))
-    return GDN_ERR_ALIAS;
+  if ((st = check_state_aliases(in->H_k, in->H_v, B, state_in, state_out, conv_in, conv_out, out, out_bytes)) !=
+      GDN_OK)
+    return st;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -360,6 +383,12 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
   bf16* mix = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(T_tot) * ld_p * 2, 1024));
   uint8_t* ws_mixer = reinterpret_cast<uint8_t*>(mix) + round_up(static_cast<size_t>(T_tot) * d_v * 2, 1024);
   const size_t ws_mixer_bytes = workspace_bytes - static_cast<size_t>(ws_mixer - ws);
+  // everything the mixer call would reject is rejected here, before the first launch
+  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
+  if ((cs = check_inputs(&in, T_tot)) != GDN_OK) return cs;
+  if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  if (states_in_workspace(L->H_k, L->H_v, B, state_in, state_out, conv_in, conv_out, workspace, need))
+    return GDN_ERR_ALIAS;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) {
     if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
@@ -369,7 +398,6 @@ gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, lo
                                static_cast<int>(n_in), L->hidden, err, stream);
   if (s != GDN_OK) return s;
   mark(1);
-  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
   s = gdn_prefill(&in, B, T, state_in, state_out, conv_in, conv_out, mix, ws_mixer, ws_mixer_bytes, err, stream);
   if (s != GDN_OK) return s;
   mark(2);
@@ -396,7 +424,8 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
   if (N == 0) return GDN_OK;
   if (!x || !y || !L->w_in || !L->w_out || !state || !conv_state) return GDN_ERR_INVALID_ARG;
   if (state_slot && n_slots < 1) return GDN_ERR_INVALID_ARG;
-  gdn_status cs = check_layer_states(L->H_k, L->H_v, state_slot ? n_slots : N, state, nullptr, conv_state, nullptr);
+  // decode updates both in place: they are the written buffers of the rule
+  gdn_status cs = check_layer_states(L->H_k, L->H_v, state_slot ? n_slots : N, nullptr, state, nullptr, conv_state);
   if (cs != GDN_OK) return cs;
   const long long T_tot = static_cast<long long>(N) * T;
   const size_t need = gdn_layer_decode_workspace_size(L->H_k, L->H_v, N, T);
@@ -408,6 +437,13 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   bf16* proj = reinterpret_cast<bf16*>(ws);
   bf16* mix = reinterpret_cast<bf16*>(ws + round_up(static_cast<size_t>(T_tot) * ld_p * 2, 1024));
+  // everything the decode call would reject is rejected here, before the first launch
+  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
+  if ((cs = check_inputs(&in, T_tot)) != GDN_OK) return cs;
+  if (!aligned16(workspace) || (reinterpret_cast<uintptr_t>(state_slot) & 3u)) return GDN_ERR_MISALIGNED;
+  if (states_in_workspace(L->H_k, L->H_v, state_slot ? n_slots : N, state, nullptr, conv_state, nullptr, workspace,
+                          need))
+    return GDN_ERR_ALIAS;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) {
     if (L->events) cudaEventRecord(static_cast<cudaEvent_t>(L->events[i]), st);
@@ -417,7 +453,6 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
                                static_cast<int>(n_in), L->hidden, err, stream);
   if (s != GDN_OK) return s;
   mark(1);
-  const gdn_inputs in = layer_mixer_inputs(L, proj, ld_p);
   s = gdn_decode_multi(&in, N, T, state, conv_state, state_slot, state_slot ? n_slots : N, mix, err, stream);
   if (s != GDN_OK) return s;
   mark(2);
@@ -615,6 +650,12 @@ gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv
   return gdn_decode_multi(in, N, 1, state, conv_state, nullptr, N, out, err, stream);
 }
 
+gdn_status gdn_err_status(int err_word) {
+  if (err_word == 0) return GDN_OK;
+  if (err_word & gdn::kDevErrTimeout) return GDN_ERR_DEVICE_TIMEOUT;
+  return GDN_ERR_INVALID_ARG;
+}
+
 const char* gdn_status_string(gdn_status status) {
   switch (status) {
     case GDN_OK: return "GDN_OK";
@@ -623,7 +664,7 @@ const char* gdn_status_string(gdn_status status) {
     case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointer or stride not suitably aligned";
     case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: buffers that must be distinct overlap";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA launch failed";
-    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a device-side wait timed out";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a bounded device-side wait gave up (err bit 1)";
     case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing or too small";
   }
   return "unknown gdn_status";

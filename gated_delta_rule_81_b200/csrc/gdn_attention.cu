@@ -43,6 +43,7 @@ constexpr int kQkThreads = 256;
 constexpr int kQkItems = 4;  // (token, head) items per warp, all of one token
 static_assert((kAHq + 2 * kAHkv) % kQkItems == 0, "a warp's items must belong to one token");
 constexpr int kDevErrCacheFull = 16;  // a sequence's KV cache has no row for its new token
+constexpr int kDevErrCacheLen = 32;   // a decode cache_len outside [0, cap]: nothing written for that sequence
 
 __device__ __forceinline__ void unpack8f(uint4 u, float* f) {
   f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
@@ -118,8 +119,8 @@ __global__ void __launch_bounds__(kQkThreads) attn_qk_kernel(AttnQkParams p) {
     const int hh = static_cast<int>(item % kHeads);
     const long long n = t / p.T;
     const long long pos = (p.pos_base ? p.pos_base[n] : 0) + t % p.T;
-    if (pos >= p.cap) {  // no room in the cache: nothing is written for this sequence
-      if (lane == 0 && hh == 0 && p.err) atomicOr(p.err, kDevErrCacheFull);
+    if (pos < 0 || pos >= p.cap) {  // no room in the cache, or a bad length: nothing is written for it
+      if (lane == 0 && hh == 0 && p.err) atomicOr(p.err, pos == p.cap ? kDevErrCacheFull : kDevErrCacheLen);
       continue;
     }
     const long long crow = n * p.cap + pos;  // cache row of this token
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) attn_decode_kernel(AttnDecPara
   float* part = p.part + ((static_cast<long long>(n) * kAHkv + kvh) * p.n_splits + sp) * kAGrp * kDecPart;
   const int len = p.cache_len[n] + 1;
   const int t0 = sp * kDecSplit, t1 = min(t0 + kDecSplit, len);
-  if (len > p.cap || t0 >= t1) {  // nothing here (or no room in the cache): an empty partial
+  if (len <= 0 || len > p.cap || t0 >= t1) {  // nothing here (no room, or a bad length): an empty partial
     if (threadIdx.x < kAGrp) {
       part[threadIdx.x * kDecPart + kAD] = -INFINITY;
       part[threadIdx.x * kDecPart + kAD + 1] = 0.f;
@@ -677,7 +678,7 @@ __global__ void __launch_bounds__(kAD) attn_decode_combine_kernel(AttnDecParams 
   __shared__ float w_s[kDecMergeMax];
   __shared__ float red_s[kAD / 32];
   const int len = p.cache_len[n] + 1;
-  if (len > p.cap) {  // reported by the cache write; nothing was attended: a zero output row
+  if (len <= 0 || len > p.cap) {  // reported by the cache write; nothing was attended: a zero output row
     out[(static_cast<long long>(n) * kAHq + h) * kAD + d] = __float2bfloat16(0.f);
     return;
   }
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(kAD) attn_decode_combine_kernel(AttnDecParams 
 // the step is complete: each sequence's cache holds one more row (unless it was full)
 __global__ void attn_cache_advance_kernel(int* cache_len, int N, int cap) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n < N && cache_len[n] < cap) cache_len[n] += 1;
+  if (n < N && cache_len[n] >= 0 && cache_len[n] < cap) cache_len[n] += 1;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 attn_map_encoder() {

@@ -81,7 +81,8 @@ EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "g
            "gdn_decode_multi", "gdn_gemm_bf16", "gdn_layer_n_in", "gdn_layer_workspace_size", "gdn_layer_prefill",
            "gdn_layer_decode_workspace_size", "gdn_layer_decode",
            "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
-           "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string")
+           "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string",
+           "gdn_err_status")
 MAX_DECODE_TOKENS = 8
 
 
@@ -137,6 +138,8 @@ def load(path: str | None = None):
     lib.gdn_attention_prefill.restype = _i
     lib.gdn_status_string.argtypes = [_i]
     lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_err_status.argtypes = [_i]
+    lib.gdn_err_status.restype = _i
     _lib = lib
     return lib
 
@@ -437,3 +440,8 @@ def attention_prefill(q_hat, k, v, g, B: int, T: int, out=None, err=None):
 
 def status_string(status: int) -> str:
     return load().gdn_status_string(status).decode()
+
+
+def err_status(err_word: int) -> int:
+    """gdn_err_status: the gdn_status an error word read back from the device stands for."""
+    return load().gdn_err_status(int(err_word))

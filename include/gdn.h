@@ -38,8 +38,9 @@
  *   - `err` (nullable) is a device int the kernels OR error bits into
  *     (1 = a bounded wait timed out, 2 = reserved,
  *     4 = cu_seqlens on the device disagreed with cu_seqlens_host, 8 = a decode
- *     state_slot outside the pool, 16 = an attention KV cache with no row left).  It is
- *     never cleared by the library.  Read it after synchronising.
+ *     state_slot outside the pool, 16 = an attention KV cache with no row left, 32 = an
+ *     attention decode cache_len outside [0, cache_cap]).  It is never cleared by the
+ *     library.  Read it after synchronising; gdn_err_status maps it to a gdn_status.
  */
 #ifndef GDN_H_
 #define GDN_H_
@@ -61,7 +62,8 @@ typedef enum {
   GDN_ERR_MISALIGNED = 3,    /* a pointer or stride is not 16-byte aligned */
   GDN_ERR_ALIAS = 4,         /* buffers that must be distinct overlap */
   GDN_ERR_CUDA = 5,          /* a CUDA launch failed */
-  GDN_ERR_DEVICE_TIMEOUT = 6,/* reserved for callers mapping *err bit 1 */
+  GDN_ERR_DEVICE_TIMEOUT = 6,/* a bounded device-side wait gave up (bit 1 of *err): every call is
+                                asynchronous, so no call returns it; gdn_err_status maps the word */
   GDN_ERR_WORKSPACE = 7      /* workspace null or smaller than required */
 } gdn_status;
 
@@ -79,7 +81,10 @@ typedef struct {
   const void* norm_w;     /* bf16 [128] */
   int H_k, H_v;
   float scale;            /* multiplies the normalised q; 1.0 = o_t = S_t q_t as written above */
-  void* const* events;    /* optional timing hook: NULL, or caller-created cudaEvent_t handles that
+  void* const* events;    /* optional timing hook (benchmarking and profiling; NULL in normal use -- an
+                             addition to the plain tensor arguments of the mixer calls, kept in the
+                             struct so that timing a call does not need a second entry point):
+                             NULL, or caller-created cudaEvent_t handles that
                              the library records on `stream` around its kernels.  Prefill: 3 events,
                              [0] before the prep kernel, [1] between prep and scan, [2] after the
                              scan; when both phases run as one fused launch (see `schedule`), [1] is
@@ -105,6 +110,12 @@ size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks);
  * Prefill of B sequences of T tokens each, packed as [B*T] tokens (sequence n
  * holds tokens n*T .. n*T+T-1).  Computes out for every token, and optionally
  * the final recurrent state and conv state of each sequence.
+ * Departure from a launch that needs nothing but the tensors: the prefill takes a caller
+ * `workspace`.  Its chunk-parallel phase (front end, triangular solve and the state-independent
+ * products of every chunk, on all SMs at once) hands each chunk's operands to the sequential
+ * phase through that scratch, which the library does not allocate itself (see
+ * gdn_prefill_noalloc for callers that cannot provide one).  Both phases are described under
+ * gdn_inputs.schedule.
  *   state_in   fp32 [B][H_v][128][128] or NULL (zero initial state)
  *   state_out  fp32 [B][H_v][128][128] or NULL; may equal state_in (in place)
  *   conv_in    bf16 [B][3][C_conv] or NULL (zero history)
@@ -306,7 +317,9 @@ size_t gdn_attn_decode_workspace_size(int N, int cache_cap);
 
 /*
  * One decode step of the attention layer: one new token per sequence, x bf16 [N][ldx] -> y.
- *   k_cache, v_cache  bf16 [N][cache_cap][4][256]; cache_len  device int32 [N], rows in use.
+ *   k_cache, v_cache  bf16 [N][cache_cap][4][256]; cache_len  device int32 [N], rows in use,
+ *   0 <= cache_len[n] <= cache_cap (a value outside that range is treated like a full cache,
+ *   but sets bit 32 of *err instead of 16).
  * The new token's normalised, rotated key and its value go to row cache_len[n] (its rotary
  * position), its queries attend to rows 0 .. cache_len[n], and cache_len[n] grows by one,
  * all on `stream`.  A full cache (cache_len[n] == cache_cap) gives that sequence a zero row of
@@ -356,7 +369,9 @@ gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, vo
  *     GDN_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per device index for
+ *     the life of the process: do not use this call across a cudaDeviceReset
+ *     (the reset ends the context the address belongs to).
  *   - Every call on a device shares the one array and it keeps the previous
  *     call's contents (nothing in it needs to start at zero).  Calls whose work
  *     overlaps on the GPU -- on different streams, or from different host
@@ -370,6 +385,13 @@ gdn_status gdn_prefill_noalloc(const gdn_inputs* in, int B, int T, const float* 
 
 /* Static description of a status code. */
 const char* gdn_status_string(gdn_status status);
+
+/*
+ * The status that an `err` word (read back after synchronising the stream) stands for:
+ * GDN_OK for 0, GDN_ERR_DEVICE_TIMEOUT when bit 1 is set, GDN_ERR_INVALID_ARG for any
+ * other bit (device cu_seqlens, a state slot or a KV-cache length the call could not use).
+ */
+gdn_status gdn_err_status(int err_word);
 
 #ifdef __cplusplus
 }

@@ -90,11 +90,12 @@ def attention(q, k, v, cu_seqlens, scale=None) -> np.ndarray:
 
 def attn_mixer(q, g, k, v, q_norm_w, k_norm_w, cu_seqlens) -> dict:
     """The attention layer between its projections, on bf16 inputs q, g [T, 24, 256] and
-    k, v [T, 4, 256]: q_hat = rope(rms(q)), k_hat = rope(rms(k)) (both stored in bf16, the
-    format of the KV cache and of the attention operands), o = attention(q_hat, k_hat, v),
-    out = o * sigmoid(g).  Returns fp64 out and the bf16-rounded k_hat (cache) values."""
+    k, v [T, 4, 256]: q_hat = rope(rms(q)) in fp64, k_hat = rope(rms(k)) rounded to bf16
+    (the KV cache, a bf16 output of the layer that later steps read back),
+    o = attention(q_hat, k_hat, v), out = o * sigmoid(g).  Returns fp64 out, the fp64
+    q_hat and the bf16-rounded k_hat (cache) values."""
     pos = positions(cu_seqlens)
-    qh = round_bf16(rope(rms_norm(q, q_norm_w), pos))
+    qh = rope(rms_norm(q, q_norm_w), pos)
     kh = round_bf16(rope(rms_norm(k, k_norm_w), pos))
     o = attention(qh, kh, v, cu_seqlens)
     gate = 1.0 / (1.0 + np.exp(-_f64(g)))
@@ -120,4 +121,4 @@ def attn_layer(x, w_in, w_out, q_norm_w, k_norm_w, cu_seqlens, Hq: int = 24, Hkv
     m = attn_mixer(parts["q"], parts["g"], parts["k"], parts["v"], q_norm_w, k_norm_w, cu_seqlens)
     o = round_bf16(m["out"]).reshape(T, Hq * D)
     y = o @ _f64(w_out).T
-    return {"y": y, "proj": proj, "out": m["out"], "k_hat": m["k_hat"], "v": parts["v"]}
+    return {"y": y, "proj": proj, "out": m["out"], "q_hat": m["q_hat"], "k_hat": m["k_hat"], "v": parts["v"]}

@@ -90,8 +90,32 @@ def test_rejects_aliasing_and_small_workspace(lib):
     assert call_prefill(lib, s, conv_in=0x5000000, conv_out=0x5000000 + 16) == 4
     assert call_prefill(lib, s, out=0x10000) == 4  # out over the inputs
     assert call_prefill(lib, s, state_in=0x7000000, state_out=0x7000000 + 4096) == 4
+    assert call_prefill(lib, s, state_in=0x7000000, state_out=0x7000000) != 4  # in place is allowed
     assert call_prefill(lib, s, ws_bytes=1024) == 7
     assert call_prefill(lib, s, ws=None) == 7
+
+
+def test_prefill_rejects_every_written_buffer_overlap(lib):
+    """One rule for every prefill entry point: a buffer the call writes (state_out, conv_out,
+    out) overlaps no other state, conv or output buffer (state_out == state_in excepted), and
+    none of them lies in the workspace."""
+    s = fake_inputs()  # T = 64 tokens at 2 / 6 heads: out is 64 * 6 * 128 * 2 = 98,304 bytes
+    out = 0x900000
+    assert call_prefill(lib, s, conv_out=out + 1024) == 4                     # conv_out over out
+    assert call_prefill(lib, s, state_out=out + 4096) == 4                    # state_out over out
+    assert call_prefill(lib, s, conv_in=0x5000000, state_out=0x5000000) == 4  # state_out over conv_in
+    assert call_prefill(lib, s, conv_out=0x5000000, state_out=0x5000000) == 4  # state_out over conv_out
+    assert call_prefill(lib, s, state_in=0x5000000, conv_out=0x5000000) == 4  # conv_out over state_in
+    assert call_prefill(lib, s, state_in=0x2000000 + 4096) == 4               # state_in inside the workspace
+    assert call_prefill(lib, s, out=0x2000000 + 1024) == 4                    # out inside the workspace
+
+
+def test_err_status_maps_device_error_bits(lib):
+    assert gdn.err_status(0) == 0
+    assert gdn.err_status(1) == 6 and gdn.err_status(1 | 4) == 6   # a timed-out wait wins
+    for bit in (4, 8, 16, 32):
+        assert gdn.err_status(bit) == 1
+    assert gdn.status_string(6).startswith("GDN_ERR_DEVICE_TIMEOUT")
 
 
 def test_varlen_rejects_bad_cu_seqlens(lib):
@@ -160,6 +184,17 @@ def test_layer_sizes_and_rejections(lib):
     assert with_(i6=0x50000000, i7=0x50000000) == 4              # conv_out == conv_in
     assert with_(i4=0x40000000, i6=0x40000000) == 4              # state and conv history in the same place
     assert with_(i4=0x40000008) == 3                             # misaligned state_in
+    assert with_(i5=0x2000000 + 8192) == 4                       # state_out inside the workspace
+    # what the mixer call would reject is rejected before the input projection is launched
+    # (on this GPU-less host a launch would fail with GDN_ERR_CUDA = 5 instead)
+    L.H_k, L.H_v = 1, 16                                         # 16 value heads per key head
+    assert lib.gdn_layer_prefill(ctypes.byref(L), *args) == 2
+    L.H_k, L.H_v = 16, 48
+    L.conv_w = None
+    assert lib.gdn_layer_prefill(ctypes.byref(L), *args) == 1
+    L.conv_w = 0x300008                                          # misaligned conv weights
+    assert lib.gdn_layer_prefill(ctypes.byref(L), *args) == 3
+    L.conv_w = 0x300000
 
 
 def _attn_layer(hidden=5120):
@@ -258,5 +293,12 @@ def test_layer_decode_sizes_and_rejections(lib):
     assert call(N, T, args[:2] + [0x40000004] + args[3:]) == 3   # misaligned state
     assert call(N, T, args[:3] + [0x40000000 + 1024] + args[4:]) == 4  # conv state inside the state pool
     assert call(0, T, args) == 0                                 # no sequences, nothing launched
+    assert call(N, T, args[:2] + [0x60000000 + 2048] + args[3:]) == 4  # state inside the workspace
+    L.H_k, L.H_v = 1, 16                                         # decode-call rejections come first too
+    assert call(N, T, args) == 2
+    L.H_k, L.H_v = 16, 48
+    L.norm_w = None
+    assert call(N, T, args) == 1
+    L.norm_w = 0x320000
     L.hidden = 5000
     assert call(N, T, args) == 2

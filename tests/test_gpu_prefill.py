@@ -1,8 +1,11 @@
 """Parity of gdn_prefill / gdn_prefill_varlen (CUDA, through the C ABI) with the
 fp64 oracle, plus the bitwise properties of the varlen path.
 
-Tolerances (fixed for the mixer): max|y_gpu - y_ref| <= 1e-2 rms(y_ref) over
-the compared outputs, and ||S_gpu - S_ref||_F / ||S_ref||_F <= 5e-3 per sequence.
+Tolerances (gpu_helpers): element-wise |y_gpu - y_ref| <= 1e-2 rms(y_ref) + 2^-8 |y_ref|
+over the compared outputs -- the mixer's arithmetic bound plus the bf16 output's own
+rounding, which no bf16 result can avoid (outputs reach ~20 rms) -- with the plain
+max |y_gpu - y_ref| / rms(y_ref) printed beside it; and
+||S_gpu - S_ref||_F / ||S_ref||_F <= 5e-3 per sequence.
 """
 import numpy as np
 import pytest
@@ -104,6 +107,46 @@ def test_config2_full_context_sampled_heads():
     check(case, out, S, C, ref, heads)
     # every head: finite output, bounded by the gated norm (|y| <= sqrt(128) |w silu(z)|)
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.slow
+def test_full_context_slow_decay_stress():
+    """The long-horizon stress case at full length: T = 262,144 tokens, 16 / 48 heads, zero
+    initial state, a ~ N(-6, 1) so that alpha = e^g stays close to 1 (0.96 .. 0.998 per
+    token) and the state carries information over thousands of chunks; two sampled heads
+    against the oracle, the state at the 5e-3 bound."""
+    cfg = gin.CONFIGS[2]
+    T, H_k, H_v = cfg["T"], cfg["H_k"], cfg["H_v"]
+    inp = gin.token_inputs(T, H_k, H_v, seed=0, a_mean=-6.0)
+    inp.update(gin.weights(H_k, H_v, seed=0))
+    inp["scale"] = 1.0
+    case = {"inp": inp, "cu_seqlens": gin.cu_from_lengths([T]), "lengths": [T], "N": 1, "H_k": H_k, "H_v": H_v,
+            "state_in": None, "conv_in": None}
+    heads = [5, 40]
+    out, S, C = run_gpu(case, uniform=True)
+    ref = run_oracle(case, heads)
+    check(case, out, S, C, ref, heads)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(S).all()
+
+
+def test_config3_packed_equals_solo_bitwise():
+    """The packed 8-sequence workload at 16 / 48 heads: the shortest and the longest
+    sequence, run alone, give bitwise the same outputs, final states and conv states as
+    their slices of the packed call."""
+    case = gin.prefill_case(3)
+    out, S, C = run_gpu(case)
+    cu = case["cu_seqlens"].tolist()
+    lengths = case["lengths"]
+    for n in (min(range(len(lengths)), key=lambda i: lengths[i]), max(range(len(lengths)), key=lambda i: lengths[i])):
+        sub = {k: (v[cu[n]:cu[n + 1]] if k in ("q", "k", "v", "z", "a", "b") else v) for k, v in case["inp"].items()}
+        solo = {"inp": sub, "cu_seqlens": gin.cu_from_lengths([lengths[n]]), "lengths": [lengths[n]], "N": 1,
+                "H_k": case["H_k"], "H_v": case["H_v"], "state_in": None, "conv_in": None}
+        o1, S1, C1 = run_gpu(solo)
+        print(f"[parity] config 3 sequence {n} ({lengths[n]} tokens) alone vs packed: "
+              f"out equal {torch.equal(o1, out[cu[n]:cu[n + 1]])}, state equal {torch.equal(S1[0], S[n])}")
+        assert torch.equal(o1, out[cu[n]:cu[n + 1]])
+        assert torch.equal(S1[0], S[n])
+        assert torch.equal(C1[0], C[n])
 
 
 def test_long_decay_variant():

@@ -234,6 +234,26 @@ def test_gates_match_library_and_limits():
     assert be[0, 0] == 0.0 and be[0, 2] == 1.0
 
 
+def test_softplus_large_argument_branch():
+    """a > 30 takes softplus(a) = a + log1p(e^-a): compare with the library's log(1 + e^a)
+    (torch.logaddexp(0, a), exact for any a) at a in {31, 50, 100, 700}; g, alpha follow."""
+    A_log = np.log([1.0, 2.0, 16.0, 3.0])
+    a = np.array([[31.0, 50.0, 100.0, 700.0]])
+    b = np.zeros_like(a)
+    g, alpha, _ = oracle.gates(A_log, a, b)
+    sp = torch.logaddexp(torch.zeros(1, 4, dtype=torch.float64), torch.from_numpy(a)).numpy()
+    np.testing.assert_allclose(g, -np.exp(A_log)[None] * sp, rtol=1e-15)
+    # torch's softplus, told not to switch to the identity, computes log1p(e^a) directly
+    ref = F.softplus(torch.from_numpy(a[:, :3]), threshold=1e9).numpy()
+    np.testing.assert_allclose(-g[:, :3] / np.exp(A_log)[None, :3], ref, rtol=1e-15)
+    np.testing.assert_allclose(alpha, np.exp(-np.exp(A_log)[None] * sp), rtol=1e-13)
+    # the branch boundary: 30 and 30 + 1e-9 agree with the library on both sides
+    g2, _, _ = oracle.gates(np.zeros(2), np.array([[30.0, 30.0 + 1e-9]]), np.zeros((1, 2)))
+    sp2 = torch.logaddexp(torch.zeros(1, 2, dtype=torch.float64), torch.tensor([[30.0, 30.0 + 1e-9]],
+                                                                                 dtype=torch.float64)).numpy()
+    np.testing.assert_allclose(g2, -sp2, rtol=1e-15)
+
+
 # ---------------------------------------------------------------- whole mixer
 
 
@@ -298,6 +318,22 @@ def test_mixer_matches_library_composition():
     ref_out, ref_S = _torch_composition(case, st, cv)
     np.testing.assert_allclose(res["out"], ref_out, rtol=1e-10, atol=1e-11)
     np.testing.assert_allclose(res["state"], ref_S, rtol=1e-10, atol=1e-12)
+
+
+def test_mixer_scale_multiplies_the_query_only():
+    """scale multiplies the normalised query: o_t = S_t (s q_t) is linear in q_t and the state
+    S_t does not involve q at all, so the pre-norm output at scale s is s times the output at
+    scale 1 and the final state is the same.  (Applying s before the L2-norm would cancel it,
+    and applying it to k would change the state: both fail here.)"""
+    case = _small_case([70, 1, 130])
+    st = gin.recurrent_state(3, case["H_v"], seed=9)
+    inp1 = dict(case["inp"], scale=1.0)
+    ref = oracle.mixer(inp1, case["cu_seqlens"], state_in=st, want_pre_norm=True)
+    for s_ in (0.5, 128 ** -0.5, 3.0):
+        res = oracle.mixer(dict(case["inp"], scale=s_), case["cu_seqlens"], state_in=st, want_pre_norm=True)
+        np.testing.assert_allclose(res["pre_norm"], s_ * ref["pre_norm"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_array_equal(res["state"], ref["state"])
+        assert np.max(np.abs(res["pre_norm"] - ref["pre_norm"])) > 1e-3 * np.max(np.abs(ref["pre_norm"]))
 
 
 def test_mixer_conv_out_is_last_three_raw_tokens():

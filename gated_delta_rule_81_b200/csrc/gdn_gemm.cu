@@ -273,8 +273,98 @@ int gemm_tile_width(int M, int N, int n_sm) {
   return best;
 }
 
+// ============================================================ weight-streaming product (few rows)
+//
+// With a handful of rows of A (a decode step: one or a few tokens per sequence) the product is
+// bound by reading B, the weights, from HBM once; a 128-row tensor-core tile would be almost
+// empty and its few tiles would leave most SMs idle.  One warp takes kGemvCols rows of B (output
+// columns): A's rows sit in shared memory as fp32, each lane walks 16-byte pieces of its B rows
+// (several loads in flight per lane), multiplies them into fp32 sums per (row of A, column), and
+// the warp adds its lanes' sums with shuffles in a fixed order.  One bf16 rounding per output.
+constexpr int kGemvThreads = 256;
+constexpr int kGemvCols = 2;                                   // B rows (output columns) per warp
+constexpr int kGemvColsPerCta = kGemvCols * kGemvThreads / 32;
+
+template <int MR>
+__global__ void __launch_bounds__(kGemvThreads) gemv_bf16_kernel(const bf16* A, long long lda, const bf16* B,
+                                                                 long long ldb, bf16* C, long long ldc, int N, int K) {
+  extern __shared__ float4 gemv_x[];  // [MR][K / 4] fp32
+  const int kv = K / 8;               // 16-byte pieces per row (K is a multiple of 64)
+  for (int i = threadIdx.x; i < MR * kv; i += kGemvThreads) {
+    const int m = i / kv, c = i - m * kv;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(A + m * lda) + c);
+    gemv_x[m * 2 * kv + 2 * c] = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+    gemv_x[m * 2 * kv + 2 * c + 1] = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long n0 = static_cast<long long>(blockIdx.x) * kGemvColsPerCta + warp * kGemvCols;
+  if (n0 >= N) return;
+  const uint4* brow[kGemvCols];
+#pragma unroll
+  for (int r = 0; r < kGemvCols; ++r)
+    brow[r] = reinterpret_cast<const uint4*>(B + (n0 + r < N ? n0 + r : n0) * ldb);
+  float acc[kGemvCols][MR];
+#pragma unroll
+  for (int r = 0; r < kGemvCols; ++r)
+#pragma unroll
+    for (int m = 0; m < MR; ++m) acc[r][m] = 0.f;
+#pragma unroll 4
+  for (int c = lane; c < kv; c += 32) {
+    uint4 w[kGemvCols];
+#pragma unroll
+    for (int r = 0; r < kGemvCols; ++r) w[r] = __ldcs(brow[r] + c);  // read once: evict first
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+      const float4 x0 = gemv_x[m * 2 * kv + 2 * c], x1 = gemv_x[m * 2 * kv + 2 * c + 1];
+#pragma unroll
+      for (int r = 0; r < kGemvCols; ++r) {
+        float a = acc[r][m];
+        a = fmaf(bf16_lo(w[r].x), x0.x, a);
+        a = fmaf(bf16_hi(w[r].x), x0.y, a);
+        a = fmaf(bf16_lo(w[r].y), x0.z, a);
+        a = fmaf(bf16_hi(w[r].y), x0.w, a);
+        a = fmaf(bf16_lo(w[r].z), x1.x, a);
+        a = fmaf(bf16_hi(w[r].z), x1.y, a);
+        a = fmaf(bf16_lo(w[r].w), x1.z, a);
+        a = fmaf(bf16_hi(w[r].w), x1.w, a);
+        acc[r][m] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kGemvCols; ++r)
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+      float v = acc[r][m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == r * MR + m && n0 + r < N) C[m * ldc + n0 + r] = __float2bfloat16(v);
+    }
+}
+
+template <int MR>
+cudaError_t launch_gemv(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc, int N,
+                        int K, cudaStream_t stream) {
+  const int smem = MR * K * 4;
+  cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<MR>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((N + kGemvColsPerCta - 1) / kGemvColsPerCta);
+  gemv_bf16_kernel<MR><<<grid, kGemvThreads, smem, stream>>>(A, lda, B, ldb, C, ldc, N, K);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
                              int M, int N, int K, int* err, cudaStream_t stream) {
+  // a few rows: stream the weights once (A's rows in shared memory, MR * K * 4 bytes)
+  if (M <= kGemvMaxM && static_cast<long long>(M) * K * 4 <= 200 * 1024) {
+    switch (M) {
+      case 1: return launch_gemv<1>(A, lda, B, ldb, C, ldc, N, K, stream);
+      case 2: return launch_gemv<2>(A, lda, B, ldb, C, ldc, N, K, stream);
+      case 3: return launch_gemv<3>(A, lda, B, ldb, C, ldc, N, K, stream);
+      default: return launch_gemv<4>(A, lda, B, ldb, C, ldc, N, K, stream);
+    }
+  }
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   int dev = 0, n_sm = 0;

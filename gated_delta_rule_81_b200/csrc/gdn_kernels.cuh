@@ -82,13 +82,16 @@ struct PrefillParams {
   int allow_fused;        // 0 = two launches, 1 = automatic, 2 = one fused launch whenever possible
   int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, scan CTAs first, prep items
                           // published by ready flags; 0 = prep kernel, then scan kernel
+  int engine_prep;        // 1 = the persistent prep engine instead of the per-item prep kernel (two launches)
 };
 
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events);
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream, void* const* events);
 // C[M][N] = A[M][K] B[N][K]^T in bf16 with fp32 accumulation (row-major, leading dimensions
-// in elements; K a multiple of 64; pointers and leading dimensions 16-byte aligned)
+// in elements; K a multiple of 64; pointers and leading dimensions 16-byte aligned).  Up to
+// kGemvMaxM rows of A go through a weight-streaming kernel, more through tcgen05 tiles.
+constexpr int kGemvMaxM = 4;
 cudaError_t launch_gemm_bf16(const bf16* A, long long lda, const bf16* B, long long ldb, bf16* C, long long ldc,
                              int M, int N, int K, int* err, cudaStream_t stream);
 // The global-attention layer between its projections.

@@ -82,7 +82,7 @@ EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "g
            "gdn_layer_decode_workspace_size", "gdn_layer_decode",
            "gdn_attn_layer_workspace_size", "gdn_attn_layer_prefill", "gdn_attention_prefill",
            "gdn_attn_decode_workspace_size", "gdn_attn_layer_decode_step", "gdn_status_string",
-           "gdn_err_status")
+           "gdn_err_status", "gdn_prefill_fused_plan")
 MAX_DECODE_TOKENS = 8
 
 
@@ -140,6 +140,8 @@ def load(path: str | None = None):
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_err_status.argtypes = [_i]
     lib.gdn_err_status.restype = _i
+    lib.gdn_prefill_fused_plan.argtypes = [_i, _i, _i, _ll, _i, _i]
+    lib.gdn_prefill_fused_plan.restype = _i
     _lib = lib
     return lib
 

@@ -96,8 +96,23 @@ typedef struct {
                              chunk to the scan) whenever the scan's (sequence, value head) units
                              fit in half the SMs, else as 1.  0 = automatic: as 2 when the prep
                              also has at least 8 (chunk, key head) items per remaining SM, else
-                             as 1.  Results are bitwise identical under every plan. */
+                             as 1.  "The SMs" are those the calling context may use (see
+                             gdn_prefill_fused_plan).  Results are bitwise identical under every
+                             plan. */
 } gdn_inputs;
+
+/*
+ * The launch plan of a prefill: the number of scan CTAs of one overlapped launch, or 0 when
+ * the prep and the scan run as two launches, for N sequences of n_chunks chunks in all, under
+ * gdn_inputs.schedule `schedule`, on n_sm SMs.  The overlapped launch needs its scan CTAs
+ * (N * H_v) to fit in half the SMs, so that the prep, which the scan waits for, always has SMs
+ * of its own; the automatic plan (0) also wants at least 8 prep items (chunk, key head) per
+ * remaining SM.  The prefill calls take n_sm from the calling context: the SMs of its SM
+ * resource (a green context holds a partition of the device), scaled down by
+ * CUDA_MPS_ACTIVE_THREAD_PERCENTAGE when that is set, else the device's count.  Pure host
+ * function; 0 on bad arguments.
+ */
+int gdn_prefill_fused_plan(int H_k, int H_v, int N, long long n_chunks, int schedule, int n_sm);
 
 /*
  * Bytes of device workspace gdn_prefill / gdn_prefill_varlen need for a batch

@@ -20,7 +20,7 @@ def lib():
 
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "gdn.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:size_t|gdn_status|const char\*|long long)\s+(gdn_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:size_t|gdn_status|const char\*|long long|int)\s+(gdn_\w+)\s*\(", text, re.M)))
 
 
 def test_exports_every_declared_symbol(lib):
@@ -302,3 +302,22 @@ def test_layer_decode_sizes_and_rejections(lib):
     L.norm_w = 0x320000
     L.hidden = 5000
     assert call(N, T, args) == 2
+
+
+def test_fused_plan_follows_the_available_sms(lib):
+    """The overlapped prefill launch is chosen from the SMs the context may use: its scan CTAs
+    (N * H_v) must fit in half of them, and the automatic plan also wants >= 8 prep items per
+    remaining SM; a partition of the device (a green context, an MPS share) with fewer SMs
+    falls back to two launches instead of leaving the scan waiting for a prep with no SM."""
+    plan = lib.gdn_prefill_fused_plan
+    # one 4096-token prompt, 16 / 48 heads: 64 chunks x 16 key heads = 1024 prep items
+    assert plan(16, 48, 1, 64, 0, 148) == 48
+    assert plan(16, 48, 1, 64, 2, 148) == 48
+    assert plan(16, 48, 1, 64, 1, 148) == 0          # two launches asked for
+    assert plan(16, 48, 1, 64, 0, 95) == 0           # 48 scan CTAs need 96 SMs
+    assert plan(16, 48, 1, 64, 2, 96) == 48
+    assert plan(16, 48, 1, 8, 0, 148) == 0           # 128 items: too few for the other 100 SMs
+    assert plan(16, 48, 1, 8, 2, 148) == 48          # forced: fused all the same
+    assert plan(16, 48, 8, 1681, 0, 148) == 0        # 8 sequences: 384 scan units, two launches
+    assert plan(2, 6, 1, 8, 2, 148) == 6
+    assert plan(16, 48, 1, 64, 0, 0) == 0 and plan(0, 48, 1, 64, 0, 148) == 0

@@ -66,3 +66,25 @@ def test_gemm_projection_shapes_sampled_rows(N, K):
     e = gemm_error(c[rows], oracle.gemm(a[rows].cpu(), b.cpu()))
     print(f"[parity] gemm {M}x{N}x{K} (48 rows): excess over bound {e:.3e}")
     assert e <= 0
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K", [(16480, 5120), (5120, 6144), (1001, 640)])
+def test_few_rows_stream_the_weights(M, N, K):
+    """M <= 4 rows (a decode step) go through the weight-streaming kernel: the whole product
+    against fp64, with A a strided view (a row of the layer's input) and C's padding columns
+    untouched."""
+    a_full = rand_bf16(M, K + 64, seed=M * 31 + K)
+    a = a_full[:, 32:32 + K]
+    b = rand_bf16(N, K, seed=N + M, scale=K ** -0.5)
+    err = err_word()
+    ldc = (N + 7) // 8 * 8 + 8
+    c_full = torch.full((M, ldc), 3.0, dtype=torch.bfloat16, device="cuda")
+    c = c_full[:, :N]
+    gdn.gemm_bf16(a_full.cuda()[:, 32:32 + K], b.cuda(), out=c, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    e = gemm_error(c, oracle.gemm(a, b))
+    print(f"[parity] gemv {M}x{N}x{K}: excess over bound {e:.3e}")
+    assert e <= 0
+    assert torch.all(c_full[:, N:] == 3.0)

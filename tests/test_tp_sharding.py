@@ -124,3 +124,64 @@ def test_layer_needs_a_group_or_explicit_rank():
     assert tp.shard_state(None, 16, 48, 2, 0) is None and tp.shard_conv_state(None, 16, 48, 2, 1) is None
     st = torch.arange(2 * 48 * 2 * 2, dtype=torch.float32).reshape(2, 48, 2, 2)
     assert torch.equal(tp.shard_state(st, 16, 48, 2, 1), st[:, 24:])
+
+
+def _prefill_worker(rank, world, port, q, H_k, H_v, hidden, B, T):
+    """One rank of TPDeltaLayer.prefill with the library's layer call replaced by the fp64 oracle
+    on the rank's own shard (rounded to bf16, the layer's output format), so that the layer's own
+    plumbing runs on the CPU: the shard it keeps, the group it was given, and the in-place bf16
+    all-reduce of its partial output over that group."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        group = dist.new_group(list(range(world)))
+        c = _case(H_k, H_v, hidden, B, T, seed=9)
+        layer = tp.TPDeltaLayer(c["w_in"], c["w_out"], c["w"]["conv_w"], c["w"]["A_log"], c["w"]["norm_w"], H_k, H_v,
+                                group=group, device="cpu")
+        assert (layer.tp, layer.rank) == (world, rank)
+        partials = {}
+
+        def stand_in(L, B_, T_, x, state_in=None, conv_in=None, **kw):
+            assert L is layer.L
+            w = layer.w
+            res = oracle.layer(x, w["w_in"], w["w_out"], w["conv_w"], w["A_log"], layer.norm_w,
+                               [i * T_ for i in range(B_ + 1)], w["H_k"], w["H_v"], state_in=state_in, conv_in=conv_in)
+            y = torch.from_numpy(np.ascontiguousarray(res["y"])).to(torch.bfloat16)
+            partials["y"] = y.clone()
+            return y, torch.from_numpy(res["state"]), torch.from_numpy(res["conv"])
+
+        tp.gdn.layer_prefill = stand_in
+        y, S, C = layer.prefill(B, T, c["x"], layer.shard_state(c["state"]), layer.shard_conv_state(c["conv"]))
+        q.put((rank, partials["y"].float().numpy(), y.float().numpy(), S.numpy(), C.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tp_layer_prefill_all_reduces_its_partials_over_the_group():
+    H_k, H_v, hidden, B, T = 4, 12, 128, 1, 40
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_prefill_worker, args=(r, 2, port, q, H_k, H_v, hidden, B, T)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=300) for _ in procs), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (_, y0, out0, S0, C0), (_, y1, out1, S1, C1) = res
+    # both ranks hold the same sum, the bf16 rounding of the two bf16 partials' sum
+    np.testing.assert_array_equal(out0, out1)
+    want = torch.from_numpy(y0 + y1).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(out0, want)
+    # and it is the unsharded layer up to the bf16 roundings of the partials and of the sum
+    c = _case(H_k, H_v, hidden, B, T, seed=9)
+    full = _oracle_layer(c, c["w_in"], c["w_out"], c["w"]["conv_w"], c["w"]["A_log"], H_k, H_v, B, T, c["state"],
+                         c["conv"])
+    bound = 2.0 ** -8 * (np.abs(y0) + np.abs(y1)) + 2.0 ** -8 * np.abs(full["y"]) + 1e-6
+    assert np.all(np.abs(out0 - full["y"]) <= bound)
+    # the states stay sharded: each rank's are the unsharded layer's slices
+    for rank, S, C in ((0, S0, C0), (1, S1, C1)):
+        hr = tp.head_range(H_k, H_v, 2, rank)
+        np.testing.assert_array_equal(S, full["state"][:, hr.v0:hr.v1])
+        np.testing.assert_array_equal(C, full["conv"][:, :, tp.conv_channels(H_k, H_v, hr).numpy()])

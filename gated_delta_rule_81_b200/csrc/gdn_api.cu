@@ -189,7 +189,6 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.out = static_cast<bf16*>(out);
   p.err = err;
   p.allow_fused = in->schedule == 0 ? 1 : in->schedule == 2 ? 2 : 0;
-  p.engine_prep = in->schedule == 3;
   cudaError_t e = gdn::launch_prefill(p, static_cast<cudaStream_t>(stream), in->events);
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

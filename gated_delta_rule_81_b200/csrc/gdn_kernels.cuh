@@ -82,7 +82,6 @@ struct PrefillParams {
   int allow_fused;        // 0 = two launches, 1 = automatic, 2 = one fused launch whenever possible
   int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, scan CTAs first, prep items
                           // published by ready flags; 0 = prep kernel, then scan kernel
-  int engine_prep;        // 1 = the persistent prep engine instead of the per-item prep kernel (two launches)
 };
 
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)

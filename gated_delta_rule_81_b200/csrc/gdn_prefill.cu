@@ -242,7 +242,6 @@ __device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
 
 // The 4-tap conv + SiLU of 32 channels from their raw inputs (tap j = token t - 3 + j, 4 x 8 bf16
 // per tap): wsm holds the 32 channels' weights, 16 x uint4 (channels 2u, 2u+1; taps 0..3 each).
-template <bool kGlobalW = false>
 __device__ __forceinline__ void conv_taps(const uint4 (&xin)[kTaps][4], const uint4* wsm, float* y) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -251,7 +250,7 @@ __device__ __forceinline__ void conv_taps(const uint4 (&xin)[kTaps][4], const ui
     for (int j = 0; j < kTaps; ++j) unpack8(xin[j][g], x[j]);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {  // channel pair 8g + 2u, 8g + 2u + 1
-      const uint4 w = kGlobalW ? __ldg(wsm + 4 * g + u) : wsm[4 * g + u];
+      const uint4 w = wsm[4 * g + u];
       const int e0 = 2 * u, e1 = 2 * u + 1;
       float a0 = bf16_lo(w.x) * x[0][e0];
       a0 = fmaf(bf16_hi(w.x), x[1][e0], a0);
@@ -272,7 +271,6 @@ __device__ __forceinline__ void conv_taps(const uint4 (&xin)[kTaps][4], const ui
 //   sequence start come from conv_in (or are zero).  wsm: the 32 channels'
 //   weights in shared memory, 16 x uint4 (channels 2u, 2u+1; taps 0..3 each).
 //   All 16 input loads are issued before any arithmetic.
-template <bool kGlobalW = false>
 __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, long long src_stride,
                                        long long s, long long t, int n, long long conv_chan0, const uint4* wsm,
                                        float* y) {
@@ -289,18 +287,17 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
 #pragma unroll
     for (int g = 0; g < 4; ++g) xin[j][g] = row ? __ldg(row + g) : make_uint4(0u, 0u, 0u, 0u);
   }
-  conv_taps<kGlobalW>(xin, wsm, y);
+  conv_taps(xin, wsm, y);
 }
 
 // One block diagonal of the blocked inverse: for blocks (I, J = I - d),
 //   M = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II M
-// with 16x16 blocks; a work item is four adjacent columns of one row of one block, and the
-// kThreads threads of the named barrier bar_id walk the items.
-template <int d, int kThreads>
+// with 16x16 blocks; each thread computes four adjacent columns of one row.
+template <int d>
 __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* sM, int tid, int bar_id) {
   constexpr int nb = 4 - d;
-  for (int w = tid; w < nb * 64; w += kThreads) {
-    const int J = w >> 6, I = J + d, ii = (w >> 2) & 15, j4 = (w & 3) * 4;
+  if (tid < nb * 64) {
+    const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
     const float* arow = sA + (16 * I + ii) * kLdA + 16 * J;
     const float* tcol = sT + (16 * J) * kLdT + 16 * J + j4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -315,9 +312,9 @@ __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* s
     }
     *reinterpret_cast<float4*>(sM + (J << 8) + (ii << 4) + j4) = acc;
   }
-  named_bar_sync(bar_id, kThreads);
-  for (int w = tid; w < nb * 64; w += kThreads) {
-    const int J = w >> 6, I = J + d, ii = (w >> 2) & 15, j4 = (w & 3) * 4;
+  named_bar_sync(bar_id, kPrepThreads);
+  if (tid < nb * 64) {
+    const int J = tid >> 6, I = J + d, ii = (tid >> 2) & 15, j4 = (tid & 3) * 4;
     const float* trow = sT + (16 * I + ii) * kLdT + 16 * I;
     const float* mcol = sM + (J << 8) + j4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -332,13 +329,12 @@ __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* s
     }
     *reinterpret_cast<float4*>(sT + (16 * I + ii) * kLdT + 16 * J + j4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
   }
-  named_bar_sync(bar_id, kThreads);
+  named_bar_sync(bar_id, kPrepThreads);
 }
 
 // T = (I + A)^{-1} for a 64x64 strictly-lower A (fp32, shared memory), by 16x16
 // blocks: diagonal blocks by forward substitution, then the three block
-// diagonals below.  kThreads (>= 64) threads on named barrier bar_id.
-template <int kThreads>
+// diagonals below.  All 256 threads.
 __device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid, int bar_id) {
   if (tid < 64) {
     const int blk = tid >> 4, col = tid & 15;
@@ -357,10 +353,10 @@ __device__ void solve_unit_lower(const float* sA, float* sT, float* sM, int tid,
       sT[(16 * blk + r) * kLdT + 16 * blk + col] = x[r];
     }
   }
-  named_bar_sync(bar_id, kThreads);
-  solve_level<1, kThreads>(sA, sT, sM, tid, bar_id);
-  solve_level<2, kThreads>(sA, sT, sM, tid, bar_id);
-  solve_level<3, kThreads>(sA, sT, sM, tid, bar_id);
+  named_bar_sync(bar_id, kPrepThreads);
+  solve_level<1>(sA, sT, sM, tid, bar_id);
+  solve_level<2>(sA, sT, sM, tid, bar_id);
+  solve_level<3>(sA, sT, sM, tid, bar_id);
 }
 
 // D (+)= A B^T with both operands as hi/lo pairs: A_hi B_hi + A_hi B_lo + A_lo B_hi
@@ -672,7 +668,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
       bulk_s2g(hb + kHeadOffP + kPImg, sQK + 32768, kPImg);
       bulk_commit();
     }
-    solve_unit_lower<kPrepThreads>(sA, sT, sM, tid, bar_id);
+    solve_unit_lower(sA, sT, sM, tid, bar_id);
     if (tid == 0) bulk_wait_read<0>();  // P has left the Q pieces
     named_bar_sync(bar_id, kPrepThreads);
     // B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
@@ -846,644 +842,6 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
   if (threadIdx.x < 32) tmem_dealloc<256>(tbase);  // prep_body ends with a barrier after its last use
 }
 
-// ============================================================ prep engine
-//
-// The chunk-parallel phase as a persistent pipeline: one CTA per SM walks (chunk, key head)
-// items, and four roles, each on warps of its own, pass work to one another through
-// mbarriers so that the latency-bound steps of consecutive value heads and items overlap:
-//   F (warps 8-11): the item's gates and the q | k front end into the [Q;K] operand image,
-//     one item ahead of the others; then the item's K rows into the K buffer (once the
-//     previous item's last W^T product has read it) and from there to the workspace;
-//   S (warps 0-3): per value head, A and P from the [Q;K] K^T accumulator, the blocked solve
-//     T = (I + A)^{-1} and the B images B_W = T diag(beta gamma), B_U = T diag(beta);
-//     P goes straight to the workspace;
-//   V (warps 4-7): per value head, the v_hat operand image; then the epilogue of the
-//     previous value head: W^T, (gamma Q)^T and U0 from tensor memory to the workspace;
-//   M (warp 12, lane 0): the tcgen05 products ([Q;K] K^T and the q^T transpose per item;
-//     W^T = K^T B_W^T and U0^T = V^T B_U^T per value head) as soon as their operands are in.
-// The workspace receives exactly what the scan reads (layout in gdn_kernels.cuh).
-constexpr int kEngThreads = 416;
-constexpr int kEngWarpM = 12;
-constexpr int kEngBarS = 1, kEngBarV = 2, kEngBarF = 3, kEngBarAll = 4;  // named barriers
-constexpr int kEngMaxG = 8;
-// shared memory (offsets from a 1024-aligned base)
-constexpr int kEngOffQK = 0;                        // [Q;K] hi / lo (as the prep image above)
-constexpr int kEngOffKM = 65536;                    // K image: hi kb0 | hi kb1 | lo kb0 | lo kb1 (8 KiB each)
-constexpr int kEngOffAT = kEngOffKM + kKBytes;      // T, A, solve temp
-constexpr int kEngOffT = kEngOffAT;
-constexpr int kEngOffA = kEngOffT + 64 * kLdT * 4;
-constexpr int kEngOffM = kEngOffA + 64 * kLdA * 4;
-constexpr int kEngOffBI = kEngOffAT + 37888;        // B_W hi | B_U hi | B_W lo | B_U lo (8 KiB each)
-constexpr int kEngOffVI = kEngOffBI + 32768;        // v_hat hi | lo (MN-major, two 8 KiB channel blocks each)
-constexpr int kEngOffId = kEngOffVI + 2 * kImg64;   // identity B image of the q^T transpose (8 KiB)
-constexpr int kEngOffGate = kEngOffId + 8192;       // [2 item slots][G, beta, gamma][kEngMaxG][64] fp32
-constexpr int kEngGateSlot = 3 * kEngMaxG * 64 * 4;
-constexpr int kEngSmem = kEngOffGate + 2 * kEngGateSlot + 1024;
-static_assert(kEngOffM + 3 * 256 * 4 <= kEngOffBI, "T, A and the solve temp fit their region");
-static_assert(kEngOffBI % 1024 == 0 && kEngOffVI % 1024 == 0 && kEngOffId % 1024 == 0, "1024-aligned images");
-// tensor memory columns (512 allocated)
-constexpr uint32_t kEngColQK = 0;     // [Q;K] K^T of item slot s at 64 s
-constexpr uint32_t kEngColQT = 128;   // q^T of item slot s at 128 + 64 s
-constexpr uint32_t kEngColWU = 256;   // per value-head slot w at 256 + 128 w: W^T (64 columns), U0^T (64)
-
-struct EngBars {
-  uint64_t qk_full[2];   // F -> M, S, V: item in slot s staged ([Q;K] image, gates, item id)
-  uint64_t qkt_done[2];  // M -> S: [Q;K] K^T and q^T of slot s in tensor memory (or the end mark)
-  uint64_t tqk_free[2];  // S, V -> M, F: slot s (its accumulators and gates) read for the last time
-  uint64_t km_full;      // F -> M: the K buffer holds the current item's K
-  uint64_t km_free;      // M -> F: the products of the current item's last value head are done (K read)
-  uint64_t m_done[2];    // M -> S, V: value-head product k in slot k & 1 complete
-  uint64_t bi_full;      // S -> M: B images of value head k
-  uint64_t vi_full;      // V -> M: v_hat image of value head k
-  uint64_t wu_free[2];   // V -> M: W^T / U0^T slot read by the epilogue
-  uint64_t k_stored[2];  // F -> V: the K image of the item in slot s has reached global memory
-  uint64_t drain;
-};
-
-struct EngItem {  // where a (chunk, key head) item's tokens are
-  long long gc;   // global chunk index
-  int kh, n, L;   // key head, sequence, valid tokens (1..64)
-  long long s, t0;  // first token of the sequence, first token of the chunk
-};
-
-__device__ __forceinline__ EngItem eng_locate(const PrefillParams& p, long long item) {
-  EngItem it;
-  it.gc = item / p.H_k;
-  it.kh = static_cast<int>(item % p.H_k);
-  if (p.chunk_base) {
-    int lo = 0, hi = p.N - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.chunk_base[mid] <= it.gc) lo = mid; else hi = mid - 1;
-    }
-    it.n = lo;
-  } else {
-    it.n = static_cast<int>(it.gc / ((p.T_uniform + kChunk - 1) / kChunk));
-  }
-  it.s = seq_start(p, it.n);
-  const long long e = seq_start(p, it.n + 1);
-  it.t0 = it.s + (it.gc - chunk_base_of(p, it.n)) * kChunk;
-  it.L = static_cast<int>(min(static_cast<long long>(kChunk), e - it.t0));
-  return it;
-}
-
-__device__ __forceinline__ uint8_t* eng_head_blob(const PrefillParams& p, long long gc, int h) {
-  return p.ws_head + (gc * p.H_v + h) * static_cast<long long>(kHeadBytes);
-}
-
-// ---- F: gates and front end of one item into slot s
-__device__ __forceinline__ void eng_front(const PrefillParams& p, const EngItem& it, int G, uint8_t* sm, float* gate,
-                                          int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  float* sG = gate;
-  float* sB = gate + kEngMaxG * 64;
-  float* sGam = gate + 2 * kEngMaxG * 64;
-  // gates of the key head's value heads: g, beta, the cumulative sum of g within the chunk
-  for (int base = 0; base < G * 64; base += 128) {
-    const int x = base + tid;
-    if (x < G * 64) {  // warp-uniform: G * 64 is a multiple of 64
-      const int j = x >> 6, i = x & 63, h = it.kh * G + j;
-      float g = 0.f, beta = 0.f;
-      if (i < it.L) {
-        const long long t = it.t0 + i;
-        g = -expf(p.A_log[h]) * softplus_f(__bfloat162float(p.a[t * p.sa + h]));
-        beta = sigmoid_f(__bfloat162float(p.b[t * p.sb + h]));
-      }
-      float v = g;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-      }
-      sG[j * 64 + i] = v;
-      sB[j * 64 + i] = beta;
-    }
-  }
-  named_bar_sync(kEngBarF, 128);
-  for (int x = tid; x < G * 32; x += 128) {
-    const int j = x >> 5, i = 32 + (x & 31);
-    sG[j * 64 + i] += sG[j * 64 + 31];
-  }
-  named_bar_sync(kEngBarF, 128);
-  for (int x = tid; x < G * 64; x += 128) sGam[x] = expf(sG[x]);
-  named_bar_sync(kEngBarF, 128);
-  // gate vectors for the scan: gamma_i, decay-to-end_i (0 past the chunk's last token), gamma_C
-  for (int x = tid; x < G * 256; x += 128) {
-    const int j = x >> 8, k2 = x & 255, h = it.kh * G + j;
-    const float Glast = sG[j * 64 + (it.L - 1)];
-    float val = 0.f;
-    if (k2 < 64) val = sGam[j * 64 + k2];
-    else if (k2 < 128) val = (k2 - 64) < it.L ? expf(Glast - sG[j * 64 + (k2 - 64)]) : 0.f;
-    else if (k2 == 128) val = expf(Glast);
-    float* gdst = reinterpret_cast<float*>(eng_head_blob(p, it.gc, h) + kHeadOffGate);
-    if (k2 != kReadyFlagWord) gdst[k2] = val;
-  }
-  // q, k front end: token i, channels 32 qq .. 32 qq + 31 (a quarter-warp takes 8 consecutive
-  // tokens of one channel group); two token halves, q then k
-  const int qq = (tid >> 3) & 3;
-  for (int which = 0; which < 2; ++which) {
-    const bf16* src = (which ? p.k : p.q) + static_cast<long long>(it.kh) * kD + 32 * qq;
-    const long long sstr = which ? p.sk : p.sq;
-    const long long ch0 = static_cast<long long>(which * p.H_k + it.kh) * kD + 32 * qq;
-    const uint4* w = reinterpret_cast<const uint4*>(p.conv_w) + ch0 * kTaps / 8;
-    for (int tp = 0; tp < 2; ++tp) {
-      const int i = (tid & 7) | (warp << 3) | (tp << 5);
-      const bool valid = i < it.L;
-      float y[32];
-      if (valid) conv32<true>(p, src, sstr, it.s, it.t0 + i, it.n, ch0, w, y);
-      float ss = 0.f;
-#pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) {
-        if (!valid) y[e2] = 0.f;
-        ss = fmaf(y[e2], y[e2], ss);
-      }
-      ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-      const float inv = rsqrtf(ss + 1e-6f) * (which == 0 ? p.scale : 1.0f);
-      const int row = which * 64 + i, kb = qq >> 1;
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        float f[8];
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) f[e2] = y[8 * c2 + e2] * inv;
-        uint4 hi, lo;
-        split8(f, hi, lo);
-        const uint32_t soff = kb * 16384u + sw128_off(row, (qq & 1) * 4 + c2);
-        *reinterpret_cast<uint4*>(sm + kEngOffQK + soff) = hi;
-        *reinterpret_cast<uint4*>(sm + kEngOffQK + 32768 + soff) = lo;
-      }
-    }
-  }
-}
-
-// ---- S: A, P, the solve and the B images of value head j of an item
-__device__ __forceinline__ void eng_solve_head(const PrefillParams& p, const EngItem& it, int j, int G, uint8_t* sm,
-                                               const float* gate, uint32_t tbase, int slot, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  const float* sG = gate + j * 64;
-  const float* sB = gate + kEngMaxG * 64 + j * 64;
-  float* sA = reinterpret_cast<float*>(sm + kEngOffA);
-  float* sT = reinterpret_cast<float*>(sm + kEngOffT);
-  float* sM = reinterpret_cast<float*>(sm + kEngOffM);
-  const int h = it.kh * G + j;
-  uint8_t* hb = eng_head_blob(p, it.gc, h);
-  // row `row` of [Q;K] K^T: rows 0..63 give P, rows 64..127 give A
-  const int row = 32 * warp + lane;
-  const bool isQ = row < 64;
-  const int ri = row & 63;
-  const float Gi = sG[ri];
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    float acc[32];
-    tmem_ld32(tmem_addr(tbase, 32 * warp, kEngColQK + 64 * slot + 32 * half), acc);
-    tmem_wait_ld();
-    if (!isQ) {
-      const float bi = sB[ri];
-#pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) {
-        const int col = 32 * half + e2;
-        sA[ri * kLdA + col] = col < ri ? bi * __expf(Gi - sG[col]) * acc[e2] : 0.f;
-      }
-    } else {
-      // P_ij = e^{G_i - G_j} (q_i . k_j) for j <= i, K-major image (row i), straight to the workspace
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        float f[8];
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) {
-          const int col = 32 * half + 8 * c2 + e2;
-          f[e2] = col <= ri ? __expf(Gi - sG[col]) * acc[8 * c2 + e2] : 0.f;
-        }
-        uint4 hi, lo;
-        split8(f, hi, lo);
-        const uint32_t off = sw128_off(ri, 4 * half + c2);
-        *reinterpret_cast<uint4*>(hb + kHeadOffP + off) = hi;
-        *reinterpret_cast<uint4*>(hb + kHeadOffP + kPImg + off) = lo;
-      }
-    }
-  }
-  named_bar_sync(kEngBarS, 128);
-  solve_unit_lower<128>(sA, sT, sM, tid, kEngBarS);
-}
-
-// B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
-__device__ __forceinline__ void eng_b_images(uint8_t* sm, const float* gate, int j, int tid) {
-  const float* sB = gate + kEngMaxG * 64 + j * 64;
-  const float* sGam = gate + 2 * kEngMaxG * 64 + j * 64;
-  const float* sT = reinterpret_cast<const float*>(sm + kEngOffT);
-  uint8_t* bi = sm + kEngOffBI;
-  for (int x = tid; x < 64 * 8; x += 128) {
-    const int r = x >> 3, cc = x & 7;
-    float fu[8], fw[8];
-#pragma unroll
-    for (int e2 = 0; e2 < 8; ++e2) {
-      const int col = 8 * cc + e2;
-      const float tb = col <= r ? sT[r * kLdT + col] * sB[col] : 0.f;
-      fu[e2] = tb;
-      fw[e2] = tb * sGam[col];
-    }
-    uint4 hi, lo;
-    const uint32_t off = sw128_off(r, cc);
-    split8(fw, hi, lo);
-    *reinterpret_cast<uint4*>(bi + off) = hi;           // B_W hi
-    *reinterpret_cast<uint4*>(bi + 16384 + off) = lo;   // B_W lo
-    split8(fu, hi, lo);
-    *reinterpret_cast<uint4*>(bi + 8192 + off) = hi;    // B_U hi
-    *reinterpret_cast<uint4*>(bi + 24576 + off) = lo;   // B_U lo
-  }
-}
-
-// ---- V: the v_hat image of value head h (MN-major: rows = tokens, two 64-channel blocks, hi then lo)
-__device__ __forceinline__ void eng_vhat(const PrefillParams& p, const EngItem& it, int h, uint8_t* sm, int tid) {
-  const int warp = tid >> 5, qq = (tid >> 3) & 3;
-  const long long ch0 = 2LL * p.H_k * kD + static_cast<long long>(h) * kD + 32 * qq;
-  const uint4* w = reinterpret_cast<const uint4*>(p.conv_w) + ch0 * kTaps / 8;
-  for (int tp = 0; tp < 2; ++tp) {
-    const int i = (tid & 7) | (warp << 3) | (tp << 5);
-    float y[32];
-    if (i < it.L) {
-      conv32<true>(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, it.s, it.t0 + i, it.n, ch0, w, y);
-    } else {
-#pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
-    }
-#pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2) {
-      uint4 hi, lo;
-      split8(y + 8 * c2, hi, lo);
-      const uint32_t off = (qq >> 1) * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
-      *reinterpret_cast<uint4*>(sm + kEngOffVI + off) = hi;
-      *reinterpret_cast<uint4*>(sm + kEngOffVI + kImg64 + off) = lo;
-    }
-  }
-}
-
-// ---- V: the epilogue of value head j of an item: W^T, (gamma Q)^T, U0 to the workspace
-__device__ __forceinline__ void eng_epilogue(const PrefillParams& p, const EngItem& it, int j, int G,
-                                             const float* gate, uint32_t tbase, int slot, int wslot, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
-  const int q = warp & 3, kr = 32 * q + lane;  // TMEM lane = d_k row (W^T, q^T) or d_v row (U0^T)
-  const float* sGam = gate + 2 * kEngMaxG * 64 + j * 64;
-  uint8_t* hb = eng_head_blob(p, it.gc, it.kh * G + j);
-  const uint32_t wu = kEngColWU + 128u * wslot;
-  float o[32];
-  // W^T: lo image at 0, hi image at 16384 (rows = d_k, 64 tokens)
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    tmem_ld32(tmem_addr(tbase, 32 * q, wu + 32 * half), o);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2) {
-      uint4 hi, lo;
-      split8(o + 8 * c2, hi, lo);
-      const uint32_t off = sw128_off(kr, 4 * half + c2);
-      *reinterpret_cast<uint4*>(hb + kHeadOffWQ + off) = lo;
-      *reinterpret_cast<uint4*>(hb + kHeadOffWQ + kImg64 + off) = hi;
-    }
-  }
-  // (gamma Q)^T: hi image at 32768, lo at 49152
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    tmem_ld32(tmem_addr(tbase, 32 * q, kEngColQT + 64 * slot + 32 * half), o);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2) {
-      float f[8];
-#pragma unroll
-      for (int e2 = 0; e2 < 8; ++e2) f[e2] = o[8 * c2 + e2] * sGam[32 * half + 8 * c2 + e2];
-      uint4 hi, lo;
-      split8(f, hi, lo);
-      const uint32_t off = sw128_off(kr, 4 * half + c2);
-      *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 2 * kImg64 + off) = hi;
-      *reinterpret_cast<uint4*>(hb + kHeadOffWQ + 3 * kImg64 + off) = lo;
-    }
-  }
-  // U0 [token / 4][d_v][4] fp32: a warp writes 512 contiguous bytes per token quad
-  float4* u0 = reinterpret_cast<float4*>(hb + kHeadOffU0) + kr;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    tmem_ld32(tmem_addr(tbase, 32 * q, wu + 64 + 32 * half), o);
-    tmem_wait_ld();
-#pragma unroll
-    for (int q4 = 0; q4 < 8; ++q4)
-      u0[(8 * half + q4) * kD] = make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
-  }
-}
-
-// ---- M: the tensor-core products
-__device__ __forceinline__ void eng_mma_item(uint8_t* sm, uint32_t tbase, int slot) {
-  const uint32_t qh = smem_u32(sm + kEngOffQK), ql = qh + 32768;
-  const uint32_t idesc = idesc_bf16(128, 64, false, false);
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {  // [Q;K] K^T (rows 0..63: Q K^T, 64..127: K K^T)
-    const uint32_t ko = (ks >> 2) * 16384u + (ks & 3) * 32u;
-    umma_split(tbase + kEngColQK + 64 * slot, smem_desc(qh + ko, 16, 1024, Swz::k128),
-               smem_desc(ql + ko, 16, 1024, Swz::k128), smem_desc(qh + ko + 8192, 16, 1024, Swz::k128),
-               smem_desc(ql + ko + 8192, 16, 1024, Swz::k128), idesc, ks > 0);
-  }
-  // q^T (lane = d_k, column = token) = Q_hi^T I + Q_lo^T I, exact in fp32
-  const uint32_t id = smem_u32(sm + kEngOffId);
-  const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
-    umma_bf16(tbase + kEngColQT + 64 * slot, smem_desc(qh + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
-    umma_bf16(tbase + kEngColQT + 64 * slot, smem_desc(ql + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
-  }
-}
-
-__device__ __forceinline__ void eng_mma_head(uint8_t* sm, uint32_t tbase, int wslot) {
-  const uint32_t km = smem_u32(sm + kEngOffKM), bi = smem_u32(sm + kEngOffBI), vi = smem_u32(sm + kEngOffVI);
-  const uint32_t wu = tbase + kEngColWU + 128u * wslot;
-  const uint32_t idesc_w = idesc_bf16(128, 64, true, false);
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks)  // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
-    umma_split(wu, smem_desc(km + ks * 2048u, 8192, 1024, Swz::k128),
-               smem_desc(km + 16384u + ks * 2048u, 8192, 1024, Swz::k128),
-               smem_desc(bi + ks * 32u, 16, 1024, Swz::k128), smem_desc(bi + 16384u + ks * 32u, 16, 1024, Swz::k128),
-               idesc_w, ks > 0);
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks)  // U0^T = V^T B_U^T: A = v_hat (MN-major), B = B_U (K-major)
-    umma_split(wu + 64, smem_desc(vi + ks * 2048u, 8192, 1024, Swz::k128),
-               smem_desc(vi + kImg64 + ks * 2048u, 8192, 1024, Swz::k128),
-               smem_desc(bi + 8192u + ks * 32u, 16, 1024, Swz::k128),
-               smem_desc(bi + 24576u + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
-}
-
-// The engine of one CTA (threads 0 .. kEngThreads - 1, shared memory at sm, 1024-aligned).
-// Items: from the workspace counter when `dynamic` (the fused launch), else item0,
-// item0 + stride, ...  Every wait is bounded; a failed one raises the CTA's abort flag and
-// every role leaves its loop, drains what it issued and meets the others at the exit.
-__device__ void prep_engine(const PrefillParams& p, uint8_t* sm, bool dynamic, long long item0, long long stride) {
-  __shared__ EngBars B;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ int abort_s;
-  __shared__ long long item_s[2];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = p.H_v / p.H_k;
-  const long long n_items = p.n_chunks * p.H_k;
-  Abort ab{p.err, &abort_s};
-  if (tid == 0) {
-    abort_s = 0;
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&B.qk_full[b], 1);
-      mbar_init(&B.qkt_done[b], 1);
-      mbar_init(&B.tqk_free[b], 2);
-      mbar_init(&B.m_done[b], 1);
-      mbar_init(&B.wu_free[b], 1);
-      mbar_init(&B.k_stored[b], 1);
-    }
-    mbar_init(&B.km_full, 1);
-    mbar_init(&B.km_free, 1);
-    mbar_init(&B.bi_full, 1);
-    mbar_init(&B.vi_full, 1);
-    mbar_init(&B.drain, 1);
-    fence_mbar_init();
-  }
-  // identity B image for the q^T transpose
-  for (int x = tid; x < 64 * 8; x += kEngThreads) {
-    const int i = x >> 3, cc = x & 7;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (cc == (i >> 3)) {
-      const int e8 = i & 7;
-      w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
-    }
-    *reinterpret_cast<uint4*>(sm + kEngOffId + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  fence_proxy_async_smem();
-  if (warp == kEngWarpM) tmem_alloc<512>(&tmem_base_s);
-  tc_fence_before();
-  named_bar_sync(kEngBarAll, kEngThreads);
-  tc_fence_after();
-  const uint32_t tbase = tmem_base_s;
-  float* gates0 = reinterpret_cast<float*>(sm + kEngOffGate);
-
-  if (warp >= 8 && warp < 12) {
-    // ------------------------------------------------ F
-    const int ft = tid - 256;
-    unsigned long long* counter = reinterpret_cast<unsigned long long*>(p.ws_flag) + 1;
-    for (int n = 0;; ++n) {
-      const int s = n & 1;
-      bool ok = true;
-      if (n >= 2) ok = mbar_wait(&B.tqk_free[s], ((n - 2) >> 1) & 1, ab, false, kBackoffNs);
-      if (ok && n >= 1) ok = mbar_wait(&B.qkt_done[(n - 1) & 1], ((n - 1) >> 1) & 1, ab, false, kBackoffNs);
-      if (ft == 0) {
-        long long item = dynamic ? static_cast<long long>(atomicAdd(counter, 1ull)) : item0 + n * stride;
-        item_s[s] = ok && item < n_items ? item : -1;
-      }
-      if (bar_sync_or(kEngBarF, 128, !ok)) break;
-      const long long item = item_s[s];
-      if (item < 0) {
-        if (ft == 0) mbar_arrive(&B.qk_full[s]);
-        break;
-      }
-      const EngItem it = eng_locate(p, item);
-      if (!dynamic && item + stride < n_items) {
-        // the next item's raw rows into L2 while this one is processed: q | k of its key head
-        // (two 256-byte pieces per token) and v of its value heads (G * 256 bytes per token)
-        const EngItem nx = eng_locate(p, item + stride);
-        const int rows = nx.L + kTaps - 1;
-        for (int x = ft; x < rows * (4 + 2 * G); x += 128) {
-          const int r = x / (4 + 2 * G), piece = x % (4 + 2 * G);
-          const long long tau = nx.t0 - (kTaps - 1) + r;
-          if (tau < nx.s) continue;
-          const bf16* src = piece < 2 ? p.q + tau * p.sq + static_cast<long long>(nx.kh) * kD + piece * 64
-                          : piece < 4 ? p.k + tau * p.sk + static_cast<long long>(nx.kh) * kD + (piece - 2) * 64
-                                      : p.v + tau * p.sv + static_cast<long long>(nx.kh) * G * kD + (piece - 4) * 64;
-          prefetch_l2_line(src);
-        }
-      }
-      float* gate = gates0 + s * (kEngGateSlot / 4);
-      eng_front(p, it, G, sm, gate, ft);
-      fence_proxy_async_smem();
-      if (p.fused_scan_ctas > 0) __threadfence();  // the gate vectors reach global memory before the chunk is published
-      named_bar_sync(kEngBarF, 128);
-      if (ft == 0) mbar_arrive(&B.qk_full[s]);
-      // the item's K rows into the K buffer, once the previous item's last W^T product is done
-      // (one completion of km_free per item, waited for in order: a parity wait only tells
-      // the next phase from the one before it)
-      ok = n == 0 || mbar_wait(&B.km_free, (n - 1) & 1, ab, false, kBackoffNs);
-      if (ft == 0) bulk_wait_read<0>();  // the previous K image has left the buffer
-      if (bar_sync_or(kEngBarF, 128, !ok)) break;
-      for (int x = ft; x < kKBytes / 16; x += 128) {  // hi kb0 | hi kb1 | lo kb0 | lo kb1: the K rows (64..127)
-        const int piece = x >> 9, off = (x & 511) * 16;
-        const int src = (piece >> 1) * 32768 + (piece & 1) * 16384 + 8192 + off;
-        *reinterpret_cast<uint4*>(sm + kEngOffKM + piece * 8192 + off) =
-            *reinterpret_cast<const uint4*>(sm + kEngOffQK + src);
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(kEngBarF, 128);
-      if (ft == 0) {
-        mbar_arrive(&B.km_full);
-        bulk_s2g(p.ws_k + (it.gc * p.H_k + it.kh) * static_cast<long long>(kKBytes), sm + kEngOffKM, kKBytes);
-        bulk_commit();
-        if (p.fused_scan_ctas > 0) {
-          bulk_wait<0>();
-          fence_proxy_async_global();
-          mbar_arrive(&B.k_stored[s]);
-        }
-      }
-    }
-    if (ft == 0) bulk_wait<0>();
-  } else if (warp < 4) {
-    // ------------------------------------------------ S
-    for (int n = 0;; ++n) {
-      const int s = n & 1;
-      if (!mbar_wait_warp(&B.qkt_done[s], (n >> 1) & 1, ab)) break;
-      const long long item = item_s[s];
-      if (item < 0) break;
-      tc_fence_after();
-      const EngItem it = eng_locate(p, item);
-      const float* gate = gates0 + s * (kEngGateSlot / 4);
-      bool ok = true;
-      for (int j = 0; j < G && ok; ++j) {
-        const int k = n * G + j;
-        eng_solve_head(p, it, j, G, sm, gate, tbase, s, tid);
-        if (j == G - 1) {  // the slot's accumulator has been read for the last time (gates: below)
-          tc_fence_before();
-        }
-        ok = k == 0 || mbar_wait(&B.m_done[(k - 1) & 1], ((k - 1) >> 1) & 1, ab);  // B images free
-        if (bar_sync_or(kEngBarS, 128, !ok)) { ok = false; break; }
-        eng_b_images(sm, gate, j, tid);
-        fence_proxy_async_smem();
-        if (p.fused_scan_ctas > 0) __threadfence();  // P reaches global memory before the chunk is published
-        named_bar_sync(kEngBarS, 128);
-        if (tid == 0) {
-          mbar_arrive(&B.bi_full);
-          if (j == G - 1) mbar_arrive(&B.tqk_free[s]);
-        }
-      }
-      if (!ok) break;
-    }
-  } else if (warp < 8) {
-    // ------------------------------------------------ V
-    const int vt = tid - 128;
-    bool have_prev = false;
-    EngItem prev{};
-    int prev_j = 0, prev_s = 0, prev_k = 0;
-    bool ok = true;
-    auto epilogue_prev = [&]() {
-      // product prev_k is complete (waited by the caller)
-      tc_fence_after();
-      const float* gate = gates0 + prev_s * (kEngGateSlot / 4);
-      eng_epilogue(p, prev, prev_j, G, gate, tbase, prev_s, prev_k & 1, vt);
-      tc_fence_before();
-      if (p.fused_scan_ctas > 0) __threadfence();
-      named_bar_sync(kEngBarV, 128);
-      if (vt == 0) {
-        mbar_arrive(&B.wu_free[prev_k & 1]);
-        if (prev_j == G - 1) mbar_arrive(&B.tqk_free[prev_s]);
-        if (p.fused_scan_ctas > 0) {
-          // publish the chunk of this value head: K image stored (F), P (S), gates (F), and this
-          // epilogue's stores are all in global memory
-          const int pn = prev_k / G;
-          bool stored = mbar_wait(&B.k_stored[pn & 1], (pn >> 1) & 1, ab, false, kBackoffNs);
-          if (stored) {
-            fence_proxy_async_global();
-            __threadfence();
-            st_release_gpu(ready_flag(p, prev.gc, prev.kh * G + prev_j), 1);
-          }
-        }
-      }
-    };
-    for (int n = 0; ok; ++n) {
-      const int s = n & 1;
-      if (!mbar_wait(&B.qk_full[s], (n >> 1) & 1, ab, false, kBackoffNs)) { ok = false; break; }
-      const long long item = item_s[s];
-      if (item < 0) break;
-      const EngItem it = eng_locate(p, item);
-      for (int j = 0; j < G; ++j) {
-        const int k = n * G + j;
-        if (k > 0 && !mbar_wait(&B.m_done[(k - 1) & 1], ((k - 1) >> 1) & 1, ab, false, kBackoffNs)) {
-          ok = false;
-          break;
-        }
-        if (bar_sync_or(kEngBarV, 128, !ok)) { ok = false; break; }
-        eng_vhat(p, it, it.kh * G + j, sm, vt);
-        fence_proxy_async_smem();
-        named_bar_sync(kEngBarV, 128);
-        if (vt == 0) mbar_arrive(&B.vi_full);
-        if (have_prev) epilogue_prev();
-        have_prev = true;
-        prev = it;
-        prev_j = j;
-        prev_s = s;
-        prev_k = k;
-      }
-    }
-    // the last value head's epilogue
-    if (ok && have_prev) {
-      ok = mbar_wait(&B.m_done[prev_k & 1], (prev_k >> 1) & 1, ab, false, kBackoffNs);
-      if (!bar_sync_or(kEngBarV, 128, !ok)) epilogue_prev();
-    }
-  } else if (warp == kEngWarpM) {
-    // ------------------------------------------------ M
-    if (lane == 0) {
-      int n_qk = 0, k_m = 0, n_end = -1;
-      long long t_idle = clock64();
-      // polls with the non-blocking probe: a blocking try_wait on one barrier would hold up
-      // products whose operands are already in
-      while (true) {
-        bool progress = false;
-        if (k_m < n_qk * G) {  // the next value head's products (the critical path) first
-          const int nm = k_m / G;
-          if (mbar_test_wait(&B.km_full, nm & 1) && mbar_test_wait(&B.bi_full, k_m & 1) &&
-              mbar_test_wait(&B.vi_full, k_m & 1) &&
-              (k_m < 2 || mbar_test_wait(&B.wu_free[k_m & 1], ((k_m - 2) >> 1) & 1))) {
-            tc_fence_after();
-            eng_mma_head(sm, tbase, k_m & 1);
-            umma_commit(&B.m_done[k_m & 1]);
-            if (k_m % G == G - 1) umma_commit(&B.km_free);
-            ++k_m;
-            progress = true;
-          }
-        }
-        if (n_end < 0) {
-          const int s = n_qk & 1;
-          if (mbar_test_wait(&B.qk_full[s], (n_qk >> 1) & 1) &&
-              (n_qk < 2 || mbar_test_wait(&B.tqk_free[s], ((n_qk - 2) >> 1) & 1))) {
-            if (item_s[s] < 0) {
-              n_end = n_qk;
-              mbar_arrive(&B.qkt_done[s]);  // the end mark for S
-            } else {
-              tc_fence_after();
-              eng_mma_item(sm, tbase, s);
-              umma_commit(&B.qkt_done[s]);
-              ++n_qk;
-            }
-            progress = true;
-          }
-        }
-        if (n_end >= 0 && k_m == n_end * G) break;
-        if (progress) {
-          t_idle = clock64();
-        } else {
-          if (ab.raised()) break;
-          if (clock64() - t_idle > kWaitLimitCycles) {
-            ab.raise(kDevErrTimeout);
-            break;
-          }
-        }
-      }
-      // every product issued has completed before tensor memory is released
-      umma_commit(&B.drain);
-      int drain_flag = 0;
-      Abort drain{nullptr, &drain_flag};
-      mbar_wait(&B.drain, 0, drain);
-    }
-    __syncwarp();
-  }
-  tc_fence_before();
-  named_bar_sync(kEngBarAll, kEngThreads);
-  if (warp == kEngWarpM) tmem_dealloc<512>(tbase);
-}
-
-__global__ void __launch_bounds__(kEngThreads, 1) prep_engine_kernel(PrefillParams p) {
-  if (p.cu && *p.ws_flag) return;
-  extern __shared__ uint8_t eng_smem_raw[];
-  prep_engine(p, align1024(eng_smem_raw), false, blockIdx.x, gridDim.x);
-}
-
 // ============================================================ scan kernel
 //
 // One CTA per (sequence, value head); the whole 128 x 128 state lives in tensor
@@ -1498,13 +856,9 @@ __global__ void __launch_bounds__(kEngThreads, 1) prep_engine_kernel(PrefillPara
 // split its columns) convert S and U between fp32 accumulators and bf16 hi/lo
 // operands in tensor memory, each conversion publishing first the part the next
 // product waits for; warps 8-11 run the output stage; warp 12 lane 0 issues the
-// MMAs in the order S W^T, state update, S (gamma Q)^T, U^T P^T: the chain's two
-// products back to back, the output's behind them while the next S converts; warp 13
-// lane 0 issues the bulk copies: W, gamma Q, K and the gates in two stages, loaded
-// two chunks ahead (each stage refilled as soon as the product that reads it is done),
-// P in one.  The conversion warps read U0 straight from global memory, early in the
-// chunk.  The output stage stages o in the gamma Q half of the chunk's own stage (dead
-// once the chunk's products are done), and frees that half when it is through.
+// MMAs in the order S W^T, S (gamma Q)^T, state update, U^T P^T, so that the
+// output's products fill the tensor pipe while the chain converts; warp 13
+// lane 0 issues the bulk copies (W, gamma Q, K, P single-buffered, gates and U0 double-buffered).
 
 constexpr int kScanThreads = 448;
 constexpr int kScanBar = 15;  // named barrier of the scan's CTA-wide steps
@@ -1527,22 +881,21 @@ constexpr uint32_t kColUDH = 320;
 constexpr uint32_t kColUDL = 336;
 __host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base + 32u * (ks >> 1) + 8u * (ks & 1); }
 // shared memory (offsets from a 1024-aligned base)
-constexpr int kScOffWQ = 0;                            // 2 stages of W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
-constexpr int kScOffK = kScOffWQ + 2 * kWQBytes;       // 2 stages of K hi, lo
-constexpr int kScOffP = kScOffK + 2 * kKBytes;         // P hi, lo
-constexpr int kScOffG = kScOffP + 2 * kPImg;           // 2 stages of gates
+constexpr int kScOffWQ = 0;                            // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
+constexpr int kScOffK = kScOffWQ + kWQBytes;           // K hi, lo
+constexpr int kScOffP = kScOffK + kKBytes;             // P hi, lo
+constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // 2 stages of U0 fp32 [16 token quads][128][4]
+constexpr int kScOffO = kScOffU0 + 2 * kU0Bytes;       // o fp32 [64 tokens][128 d_v] for the token-major epilogue
+constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
-// o fp32 [64 tokens][128 d_v] for the token-major epilogue, in the (gamma Q)^T half of the chunk's stage
-constexpr int kScOffOInStage = 2 * kImg64;
-static_assert(64 * kD * 4 <= 2 * kImg64, "o fits the (gamma Q)^T half of a stage");
 
 // The scan of one (sequence, value head) (`blk` = sequence rank * H_v + value head) by the
 // CTA's first 448 threads, with shared memory at sm (1024-aligned, kScSmem - 1024 bytes).
 // CTA-wide steps use named barrier kScanBar over those threads.
 __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8_t* sm) {
   __shared__ uint64_t g_full[2], g_free[2];
-  __shared__ uint64_t w_full[2], w_free[2], q_full[2], q_free[2], k_full[2], k_free[2], p_full, p_free;
-  __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, o_done, y_done, o_free, drain_b;
+  __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, u0_full[2], u0_free[2];
+  __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -1560,13 +913,15 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     for (int b = 0; b < 2; ++b) {
       mbar_init(&g_full[b], 1);
       mbar_init(&g_free[b], 256);
-      mbar_init(&w_full[b], 1);
-      mbar_init(&w_free[b], 1);
-      mbar_init(&q_full[b], 1);
-      mbar_init(&q_free[b], 1);
-      mbar_init(&k_full[b], 1);
-      mbar_init(&k_free[b], 1);
+      mbar_init(&u0_full[b], 1);
+      mbar_init(&u0_free[b], 256);
     }
+    mbar_init(&w_full, 1);
+    mbar_init(&w_free, 1);
+    mbar_init(&q_full, 1);
+    mbar_init(&q_free, 1);
+    mbar_init(&k_full, 1);
+    mbar_init(&k_free, 1);
     mbar_init(&p_full, 1);
     mbar_init(&p_free, 1);
     mbar_init(&s_conv, 256);
@@ -1574,7 +929,6 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     mbar_init(&u_conv2, 256);
     mbar_init(&u_done, 1);
     mbar_init(&s_done, 1);
-    mbar_init(&o_done, 1);
     mbar_init(&y_done, 1);
     mbar_init(&o_free, 128);
     mbar_init(&drain_b, 1);
@@ -1596,67 +950,54 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     for (int c = 0; c < nc && ok; ++c) {
       const int gs = c & 1;
       const float* gates = reinterpret_cast<const float*>(sm + kScOffG + gs * kGateBytes);
-      // ---- S_c (columns 64 th .. +63) -> hi/lo operand, and S <- gamma_C S for the update.  The
-      // hi/lo copy of S_{c-1} may still be read by chunk c - 1's output product (issued after
-      // its state update), so the new copy is stored once that product is done (o_done).
+      // ---- S_c (columns 64 th .. +63) -> hi/lo operand; then S <- gamma_C S for the update
+      // (the previous chunk's products that read S hi/lo were issued before its state update)
       ok = c == 0 || mbar_wait_warp(&s_done, (c - 1) & 1, ab);
       if (ok) ok = mbar_wait_warp(&g_full[gs], (c >> 1) & 1, ab);
       if (!ok) break;
       tc_fence_after();
-      const float gC = gates[128];
-      uint32_t shi[32], slo[32];
+      float sv[64];
+      if (c == 0) {
+        if (p.state_in) {
+          const float4* src = reinterpret_cast<const float4*>(p.state_in + srow + 64 * th);
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {  // columns 64 th + 32 cc .. + 31
-        float sv[32];
-        if (c == 0) {
-          if (p.state_in) {
-            const float4* src = reinterpret_cast<const float4*>(p.state_in + srow + 64 * th + 32 * cc);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 f = __ldg(src + q4);
-              sv[4 * q4] = f.x; sv[4 * q4 + 1] = f.y; sv[4 * q4 + 2] = f.z; sv[4 * q4 + 3] = f.w;
-            }
-          } else {
-#pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) sv[e2] = 0.f;
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const float4 f = __ldg(src + q4);
+            sv[4 * q4] = f.x; sv[4 * q4 + 1] = f.y; sv[4 * q4 + 2] = f.z; sv[4 * q4 + 3] = f.w;
           }
         } else {
-          tmem_ld32(tl + kColS + 64 * th + 32 * cc, sv);
-          tmem_wait_ld();
-        }
-        split_pairs_x2<16>(sv, shi + 16 * cc, slo + 16 * cc);
 #pragma unroll
-        for (int e2 = 0; e2 < 32; e2 += 2) {
-          const float2 r = __fmul2_rn(make_float2(sv[e2], sv[e2 + 1]), make_float2(gC, gC));
-          sv[e2] = r.x;
-          sv[e2 + 1] = r.y;
+          for (int e2 = 0; e2 < 64; ++e2) sv[e2] = 0.f;
         }
-        tmem_st32(tl + kColS + 64 * th + 32 * cc, sv);
+      } else {
+        tmem_ld32(tl + kColS + 64 * th, sv);
+        tmem_ld32(tl + kColS + 64 * th + 32, sv + 32);
+        tmem_wait_ld();
       }
-      ok = c == 0 || mbar_wait_warp(&o_done, (c - 1) & 1, ab);
-      if (!ok) break;
-      tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        tmem_st16(tl + kColSH + 32 * th + 16 * cc, shi + 16 * cc);
-        tmem_st16(tl + kColSL + 32 * th + 16 * cc, slo + 16 * cc);
+        uint32_t hi[16], lo[16];
+        split_pairs_x2<16>(sv + 32 * cc, hi, lo);
+        tmem_st16(tl + kColSH + 32 * th + 16 * cc, hi);
+        tmem_st16(tl + kColSL + 32 * th + 16 * cc, lo);
       }
-      tmem_wait_st();  // the rescaled S too
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&s_conv);
-      // ---- U^T = U0^T - S W^T for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first
-      // (the state update waits for it), then U (the output product waits for it).  U0
-      // [token / 4][d_v][4] comes straight from global memory (published with the chunk's
-      // gates, which this warp has acquired), its loads issued before the wait.
-      float4 u0r[8];
-      {
-        const float4* U0g = reinterpret_cast<const float4*>(
-                                p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffU0) +
-                            (8 * th) * kD + v;
+      const float gC = gates[128];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) u0r[q4] = U0g[q4 * kD];
+      for (int e2 = 0; e2 < 64; e2 += 2) {
+        const float2 r = __fmul2_rn(make_float2(sv[e2], sv[e2 + 1]), make_float2(gC, gC));
+        sv[e2] = r.x;
+        sv[e2 + 1] = r.y;
       }
+      tmem_st32(tl + kColS + 64 * th, sv);
+      tmem_st32(tl + kColS + 64 * th + 32, sv + 32);
+      // ---- U^T = U0^T - S W^T for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first
+      // (the state update waits for it), then U (the output product waits for it)
       ok = mbar_wait_warp(&u_done, c & 1, ab);
+      if (ok) ok = mbar_wait_warp(&u0_full[gs], (c >> 1) & 1, ab);
+      const float* U0 = reinterpret_cast<const float*>(sm + kScOffU0 + gs * kU0Bytes);
       if (!ok) break;
       tc_fence_after();
       float u[32], ud[32];
@@ -1665,9 +1006,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tmem_ld32(tl + kColU2 + 32 * th, u);
         tmem_ld32(tl + kColU1 + 32 * th, u1);
         tmem_wait_ld();
+        const float4* U0q = reinterpret_cast<const float4*>(U0) + (8 * th) * kD + v;  // [token / 4][d_v][4]
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {  // u = U0 - (U1 + U2), packed in token pairs
-          const float4 u0 = u0r[q4];
+          const float4 u0 = U0q[q4 * kD];
           const int i = 4 * q4;
           const float2 a0 = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
           const float2 a1 = __fadd2_rn(make_float2(u1[i + 2], u1[i + 3]), make_float2(u[i + 2], u[i + 3]));
@@ -1676,6 +1018,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
           u[i] = r0.x; u[i + 1] = r0.y; u[i + 2] = r1.x; u[i + 3] = r1.y;
         }
       }
+      mbar_arrive(&u0_free[gs]);
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         const float2 d = *reinterpret_cast<const float2*>(gates + 64 + 32 * th + i);
@@ -1690,7 +1033,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tmem_st16(tl + kColUDH + 32 * th, hi);
         tmem_st16(tl + kColUDL + 32 * th, lo);
       }
-      tmem_wait_st();
+      tmem_wait_st();  // also covers the rescaled S
       tc_fence_before();
       mbar_arrive(&u_conv);
       {
@@ -1728,65 +1071,58 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
       const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
       const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
-      // Shared-memory descriptors of each stage's operands at K step 0, built once: a K step of an
-      // MN-major operand advances 2048 bytes (128 in the descriptor's 16-byte address field), of
-      // the K-major P 32 bytes (2), so issuing a product is one add and one instruction.
-      const uint32_t wq0 = smem_u32(sm + kScOffWQ), kb0 = smem_u32(sm + kScOffK);
-      const uint64_t d_w0 = smem_desc(wq0, kImg64, 1024, Swz::k128);               // [W_lo | W_hi], N = 128
-      const uint64_t d_wh0 = smem_desc(wq0 + kImg64, kImg64, 1024, Swz::k128);     // W_hi, N = 64
-      const uint64_t d_q0 = smem_desc(wq0 + 2 * kImg64, kImg64, 1024, Swz::k128);  // [gQ_hi | gQ_lo], N = 128
-      const uint64_t d_kh0 = smem_desc(kb0, 8192, 1024, Swz::k128);                // K hi (MN-major, N = d_k)
-      const uint64_t d_kl0 = smem_desc(kb0 + kImg64, 8192, 1024, Swz::k128);       // K lo
-      constexpr uint64_t kStageWQ = kWQBytes >> 4, kStageK = kKBytes >> 4;          // stage 1 = stage 0 + these
-      const uint64_t d_p = smem_desc(smem_u32(sm + kScOffP), 16, 1024, Swz::k128);  // 128 rows: P hi then P lo
-      constexpr uint64_t kStepMN = 2048 >> 4, kStepP = 32 >> 4;
+      const uint32_t wq = smem_u32(sm + kScOffWQ);
+      const uint32_t k_hi = smem_u32(sm + kScOffK), k_lo = k_hi + kImg64;
+      const uint32_t p_hi = smem_u32(sm + kScOffP);
       for (int c = 0; c < nc; ++c) {
-        const int st = c & 1;
-        const uint32_t sp = (c >> 1) & 1;  // phase parity of the chunk's stage barriers
-        const uint64_t d_w = d_w0 + st * kStageWQ, d_wh = d_wh0 + st * kStageWQ, d_q = d_q0 + st * kStageWQ;
-        const uint64_t d_kh = d_kh0 + st * kStageK, d_kl = d_kl0 + st * kStageK;
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
-        if (!mbar_wait(&w_full[st], sp, ab)) break;
+        if (!mbar_wait(&w_full, c & 1, ab)) break;
         if (c > 0 && !mbar_wait(&y_done, (c - 1) & 1, ab)) break;  // U^T P^T of the last chunk read the U columns
         tc_fence_after();
-        // the chain: [U2 | U1] = S_hi [W_lo | W_hi], U1 += S_lo W_hi
+        // the chain's product first: [U2 | U1] = S_hi [W_lo | W_hi], U1 += S_lo W_hi
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, d_w + ks * kStepMN, idesc_u, ks > 0);
-          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, d_wh + ks * kStepMN, idesc_u2, true);
+          const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
+          const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, ks > 0);
+          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
         }
         umma_commit(&u_done);
-        umma_commit(&w_free[st]);
-        // the chain: S += U_d^T K (onto gamma_C S)
-        if (!mbar_wait(&u_conv, c & 1, ab)) break;
-        if (!mbar_wait(&k_full[st], sp, ab)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), d_kh + ks * kStepMN, idesc_s, true);
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), d_kl + ks * kStepMN, idesc_s, true);
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), d_kh + ks * kStepMN, idesc_s, true);
-        }
-        umma_commit(&s_done);
-        umma_commit(&k_free[st]);
-        // the output, off the chain while the next chunk's S converts: [O1 | O2] = S_hi [gQ_hi | gQ_lo],
-        // O1 += S_lo gQ_hi once o(c-1) has been read, then [O1 | O2] += U_hi [P_hi | P_lo], O1 += U_lo P_hi
-        if (!mbar_wait(&q_full[st], sp, ab)) break;
+        umma_commit(&w_free);
+        // then the output's: [O1 | O2] = S_hi [gQ_hi | gQ_lo], O1 += S_lo gQ_hi, once o(c-1) has been read
+        if (!mbar_wait(&q_full, c & 1, ab)) break;
         if (c > 0 && !mbar_wait(&o_free, (c - 1) & 1, ab)) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, d_q + ks * kStepMN, idesc_u, ks > 0);
-          umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, d_q + ks * kStepMN, idesc_u2, true);
+          const uint64_t bq = smem_desc(wq + 2 * kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, ks > 0);
+          umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, bq, idesc_u2, true);
         }
-        umma_commit(&o_done);
+        umma_commit(&q_free);
+        if (!mbar_wait(&u_conv, c & 1, ab)) break;
+        if (!mbar_wait(&k_full, c & 1, ab)) break;
+        tc_fence_after();
+        // S += U_d^T K (onto gamma_C S)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
+          const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
+        }
+        umma_commit(&s_done);
+        umma_commit(&k_free);
         if (!mbar_wait(&u_conv2, c & 1, ab)) break;
         if (!mbar_wait(&p_full, c & 1, ab)) break;
         tc_fence_after();
+        // [O1 | O2] += U_hi [P_hi | P_lo], O1 += U_lo P_hi
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUH, ks), d_p + ks * kStepP, idesc_y, true);
-          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUL, ks), d_p + ks * kStepP, idesc_y2, true);
+          const uint64_t b2 = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);  // 128 rows: P hi then P lo
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUH, ks), b2, idesc_y, true);
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUL, ks), b2, idesc_y2, true);
         }
         umma_commit(&y_done);
         umma_commit(&p_free);
@@ -1801,79 +1137,51 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
   } else if (warp == kWarpProd) {
     // ------------------------------------------------ bulk-copy producer (lane 0)
     if (lane == 0) {
-      // Chunks 0 and 1 first; then at chunk c: P of chunk c + 1 (one stage) once chunk c's
-      // U^T P^T is done, and for chunk c + 2 into stage c & 1: W as soon as chunk c's S W^T is
-      // done, K after its state update, the gates once the conversion warps have read them,
-      // gamma Q once chunk c's output stage has released its half.
-      int n_g[2] = {0, 0}, n_w[2] = {0, 0}, n_q[2] = {0, 0}, n_k[2] = {0, 0}, n_p = 0;
+      // Order of need: W, gamma Q, K, P of chunk c (single stages, each refilled as soon as the
+      // product that reads it has completed), then the double-buffered gates and U0 of chunk c + 1.
+      int n_g[2] = {0, 0}, n_u0[2] = {0, 0}, n_w = 0, n_q = 0, n_k = 0, n_p = 0;
       auto head_blob = [&](int c) {
         return p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes);
       };
-      auto k_blob = [&](int c) { return p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes); };
-      // fused launch: chunk c's operands (read from here on) are published by its prep
-      auto ready = [&](int c) {
-        return p.fused_scan_ctas == 0 || flag_wait(ready_flag(p, cb + c, h), ab, kBackoffNs);
-      };
-      auto load_w = [&](int c) {
+      auto load_gates_u0 = [&](int c) -> bool {  // chunk c into stage c & 1
         const int st = c & 1;
-        mbar_arrive_expect_tx(&w_full[st], 2 * kImg64);
-        bulk_g2s(sm + kScOffWQ + st * kWQBytes, head_blob(c) + kHeadOffWQ, 2 * kImg64, &w_full[st]);
-        ++n_w[st];
-      };
-      auto load_q = [&](int c) {
-        const int st = c & 1;
-        mbar_arrive_expect_tx(&q_full[st], 2 * kImg64);
-        bulk_g2s(sm + kScOffWQ + st * kWQBytes + 2 * kImg64, head_blob(c) + kHeadOffWQ + 2 * kImg64, 2 * kImg64,
-                 &q_full[st]);
-        ++n_q[st];
-      };
-      auto load_k = [&](int c) {
-        const int st = c & 1;
-        mbar_arrive_expect_tx(&k_full[st], kKBytes);
-        bulk_g2s(sm + kScOffK + st * kKBytes, k_blob(c), kKBytes, &k_full[st]);
-        ++n_k[st];
-      };
-      auto load_g = [&](int c) {
-        const int st = c & 1;
+        const uint8_t* hb = head_blob(c);
+        // fused launch: chunk c's operands (read from here on) are published by its prep
+        if (p.fused_scan_ctas > 0 && !flag_wait(ready_flag(p, cb + c, h), ab, kBackoffNs)) return false;
+        if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
         mbar_arrive_expect_tx(&g_full[st], kGateBytes);
-        bulk_g2s(sm + kScOffG + st * kGateBytes, head_blob(c) + kHeadOffGate, kGateBytes, &g_full[st]);
+        bulk_g2s(sm + kScOffG + st * kGateBytes, hb + kHeadOffGate, kGateBytes, &g_full[st]);
         ++n_g[st];
+        if (c >= 2 && !mbar_wait(&u0_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
+        mbar_arrive_expect_tx(&u0_full[st], kU0Bytes);
+        bulk_g2s(sm + kScOffU0 + st * kU0Bytes, hb + kHeadOffU0, kU0Bytes, &u0_full[st]);
+        ++n_u0[st];
+        return true;
       };
-      auto load_p = [&](int c) {
-        mbar_arrive_expect_tx(&p_full, 2 * kPImg);
-        bulk_g2s(sm + kScOffP, head_blob(c) + kHeadOffP, 2 * kPImg, &p_full);
-        ++n_p;
-      };
-      bool ok = true;
-      for (int c = 0; c < 2 && c < nc && ok; ++c) {
-        if (!(ok = ready(c))) break;
-        load_g(c);
-        load_w(c);
-        load_k(c);
-        load_q(c);
-        if (c == 0) load_p(0);
-      }
+      bool ok = nc == 0 || load_gates_u0(0);
       for (int c = 0; c < nc && ok; ++c) {
-        const int st = c & 1;
-        const uint32_t sp = (c >> 1) & 1;
-        if (c + 1 < nc) {
-          if (!(ok = mbar_wait(&p_free, c & 1, ab, false, kBackoffNs))) break;
-          load_p(c + 1);
-        }
-        if (c + 2 < nc) {
-          if (!(ok = ready(c + 2))) break;
-          if (!(ok = mbar_wait(&w_free[st], sp, ab, false, kBackoffNs))) break;
-          load_w(c + 2);
-          if (!(ok = mbar_wait(&k_free[st], sp, ab, false, kBackoffNs))) break;
-          load_k(c + 2);
-          if (!(ok = mbar_wait(&g_free[st], sp, ab, false, kBackoffNs))) break;
-          load_g(c + 2);
-          if (!(ok = mbar_wait(&q_free[st], sp, ab, false, kBackoffNs))) break;
-          load_q(c + 2);
-        }
-        if (c + 3 < nc) {  // three chunks ahead into L2, behind this chunk's copies
-          prefetch_l2(head_blob(c + 3), kHeadBytes);
-          prefetch_l2(k_blob(c + 3), kKBytes);
+        const uint8_t* hb = head_blob(c);
+        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes);
+        if (c >= 1 && !mbar_wait(&w_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&w_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffWQ, hb + kHeadOffWQ, 2 * kImg64, &w_full);
+        ++n_w;
+        if (c >= 1 && !mbar_wait(&q_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&q_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffWQ + 2 * kImg64, hb + kHeadOffWQ + 2 * kImg64, 2 * kImg64, &q_full);
+        ++n_q;
+        if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&k_full, kKBytes);
+        bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
+        ++n_k;
+        if (c >= 1 && !mbar_wait(&p_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&p_full, 2 * kPImg);
+        bulk_g2s(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
+        ++n_p;
+        if (c + 1 < nc) ok = load_gates_u0(c + 1);
+        if (c + 2 < nc) {  // two chunks ahead into L2, behind this chunk's copies
+          prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
+          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
         }
       }
       // copies still in flight (only possible after an abort) land before the CTA exits
@@ -1881,10 +1189,11 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       Abort drain{nullptr, &drain_flag};
       for (int b = 0; b < 2; ++b) {
         if (n_g[b] > 0) mbar_wait(&g_full[b], (n_g[b] - 1) & 1, drain);
-        if (n_w[b] > 0) mbar_wait(&w_full[b], (n_w[b] - 1) & 1, drain);
-        if (n_q[b] > 0) mbar_wait(&q_full[b], (n_q[b] - 1) & 1, drain);
-        if (n_k[b] > 0) mbar_wait(&k_full[b], (n_k[b] - 1) & 1, drain);
+        if (n_u0[b] > 0) mbar_wait(&u0_full[b], (n_u0[b] - 1) & 1, drain);
       }
+      if (n_w > 0) mbar_wait(&w_full, (n_w - 1) & 1, drain);
+      if (n_q > 0) mbar_wait(&q_full, (n_q - 1) & 1, drain);
+      if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
       if (n_p > 0) mbar_wait(&p_full, (n_p - 1) & 1, drain);
     }
     __syncwarp();
@@ -1898,7 +1207,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     const int v = 32 * ow + lane;
     const int otid = tid - 256;           // 0..127 within the output group
     const uint32_t tl = tmem_addr(tbase, 32 * ow, 0);
-    // o of chunk c is staged in the (gamma Q)^T half of the chunk's stage
+    float* sO = reinterpret_cast<float*>(sm + kScOffO);
     const int v8 = (otid & 15) * 8;       // this thread's 8 channels; its tokens are otid / 16 + 8 m
     float w8[8];  // norm_w is only 2-byte aligned: element loads
 #pragma unroll
@@ -1921,7 +1230,6 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         zr[m] = r < L ? __ldg(reinterpret_cast<const uint4*>(p.z + (tok0 + r) * p.sz + static_cast<long long>(h) * kD + v8))
                       : make_uint4(0u, 0u, 0u, 0u);
       }
-      float* sO = reinterpret_cast<float*>(sm + kScOffWQ + (c & 1) * kWQBytes + kScOffOInStage);
       bool ok = mbar_wait_warp(&y_done, c & 1, ab, false, kBackoffNs);
       if (ok) {
         tc_fence_after();
@@ -1989,10 +1297,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
             *reinterpret_cast<uint4*>(p.out + ((tok0 + r) * p.H_v + h) * kD + v8) = pack8(y8[u]);
         }
       }
-      // the half goes back to the producer (which refills it by bulk copy for chunk c + 2)
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (otid == 0) mbar_arrive(&q_free[c & 1]);
+      named_bar_sync(1, 128);  // sO is rewritten by the next chunk
     }
   }
 
@@ -2181,20 +1486,11 @@ cudaError_t launch_prefill(const PrefillParams& p_in, cudaStream_t stream, void*
     return err;
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
-  if (p.n_chunks > 0 && !p.engine_prep) {
+  if (p.n_chunks > 0) {
     const int smem = prep_smem_bytes(p.H_v / p.H_k);
     err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, smem, stream>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  } else if (p.n_chunks > 0) {
-    err = cudaFuncSetAttribute(prep_engine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kEngSmem);
-    if (err != cudaSuccess) return err;
-    int dev = 0, n_sm = 0;
-    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-    if ((err = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-    const long long n_items = p.n_chunks * p.H_k;
-    prep_engine_kernel<<<static_cast<unsigned>(std::min<long long>(n_sm, n_items)), kEngThreads, kEngSmem, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);

@@ -16,15 +16,15 @@
 //
 // Two kernels (plus two small helpers):
 //   prep (one CTA per chunk x key head, all chunks in parallel): conv + SiLU +
-//     L2-norm front end, gates, [Q;K] K^T on tcgen05, the fp32 blocked
-//     triangular solve, and per value head W = T diag(b gamma) K and
-//     U0 = T diag(b) V on tcgen05 (so that U = U0 - W S^T).  It writes the
-//     chunk's operand images to the workspace.
+//     L2-norm front end of q and k, gates, [Q;K] K^T on tcgen05, the fp32 blocked
+//     triangular solve, and per value head B_U = T diag(b), P, W = T diag(b gamma) K on
+//     tcgen05 and v_hat = SiLU(conv(v)).  It writes the chunk's operand images to the
+//     workspace.
 //   scan (one CTA per sequence x value head): walks the chunks in order with
 //     the whole fp32 state in tensor memory (lane = value row), the state and
 //     U as bf16 hi/lo A operands read by tcgen05 straight from tensor memory.
-//     Per chunk four tcgen05 products (S W^T, S Q^T, U_d^T K, U^T P^T) and the
-//     gated RMS-norm epilogue.
+//     Per chunk five tcgen05 products (V^T B_U^T, S W^T, S Q^T, U_d^T K,
+//     U^T P^T) and the gated RMS-norm epilogue.
 #include <cuda.h>
 
 #include <algorithm>
@@ -176,16 +176,15 @@ constexpr int kLdT = 68;                               // fp32 row stride of T (
 // 64 kb .. 64 kb + 63) at kb * 16384, rows 0..63 = Q tokens, rows 64..127 = K tokens.
 // The K rows are the workspace's K image (four 8 KiB pieces, bulk-stored from here).
 constexpr int kPrepOffQK = 0;
-// Once the products that read Q have completed, the four 8 KiB Q pieces are scratch:
-// per value head they stage P (hi, lo), then hold the B images B_W = T diag(beta gamma)
-// and B_U = T diag(beta), then stage W^T (lo rows 0..63, 64..127, hi rows 0..63, 64..127).
-constexpr int kPrepOffBWhi = 0, kPrepOffBUhi = 16384, kPrepOffBWlo = 32768, kPrepOffBUlo = 49152;
+// The Q rows are the workspace's Q image too.  Once the product that reads Q has completed
+// and the Q image has left for the workspace, the four 8 KiB Q pieces are scratch: per
+// value head they stage P (hi, lo), then hold the B image B_W = T diag(beta gamma) (hi at 0,
+// lo at 32768), then stage -W^T (lo rows 0..63, 64..127, hi rows 0..63, 64..127).
+constexpr int kPrepOffBWhi = 0, kPrepOffBWlo = 32768;
 // Region R (37 KiB) changes role through the kernel:
 //   the raw q | k rows of the chunk (front-end input, rows of kRawStride bytes);
-//   the identity B image of the q^T transpose;
-//   per value head: T, A and the block-solve temp; then the v_hat image (A operand
-//   of U0^T, MN-major: rows = tokens, two 64-channel blocks, hi then lo); then the
-//   staged (gamma Q)^T images (hi, lo).
+//   per value head: T, A and the block-solve temp; then B_U = T diag(beta) (lo, hi) over
+//   the dead A, staged for the workspace.
 constexpr int kPrepOffR = 65536;
 constexpr int kRawStride = 2 * kD * 2 + 16;            // q row | k row, 16 B of padding against bank conflicts
 constexpr int kPrepOffT = kPrepOffR;                   // T fp32                64*68*4
@@ -195,15 +194,16 @@ constexpr int kPrepRBytes = 64 * kLdT * 4 + 64 * kLdA * 4 + 3 * 256 * 4;
 constexpr int kPrepOffG = kPrepOffR + kPrepRBytes;     // G cumsum   [8][64]
 constexpr int kPrepOffB = kPrepOffG + 8 * 64 * 4;      // beta       [8][64]
 constexpr int kPrepOffGam = kPrepOffB + 8 * 64 * 4;    // gamma = e^G [8][64]
-constexpr int kPrepOffW = kPrepOffGam + 8 * 64 * 4;    // conv weights of the q, k and v channels, (2+G)*128*8 B
-__host__ __device__ constexpr int prep_smem_bytes(int G) { return kPrepOffW + (2 + G) * 128 * 8 + 1024; }
-static_assert(2 * kImg64 <= kPrepRBytes, "the v_hat and (gamma Q)^T images must fit region R");
+constexpr int kPrepOffW = kPrepOffGam + 8 * 64 * 4;    // conv weights of the q and k channels, 2*128*8 B
+constexpr int kPrepOffBU = kPrepOffA;                  // B_U lo | hi, once A is dead
+constexpr int kVBatch = 3;                             // value heads whose raw v rows fit the [Q;K] region at once
+static_assert((kChunk + kTaps - 1) * (kVBatch * kD * 2 + 16) <= 65536, "the staged v rows must fit the [Q;K] region");
+constexpr int kPrepSmem = kPrepOffW + 2 * 128 * 8 + 1024;
 static_assert((kChunk + kTaps - 1) * kRawStride <= kPrepRBytes, "the raw q | k rows must fit region R");
+static_assert(kPrepOffBU % 1024 == 0 && 2 * kPImg <= 64 * kLdA * 4, "B_U must fit the A area");
 // tensor memory columns (256 per CTA, two CTAs per SM)
 constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns)
-constexpr uint32_t kPrepColQT = 64;   // q^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColW = 128;   // W^T (lane = d_k, column = token)
-constexpr uint32_t kPrepColU = 192;   // U0^T (lane = d_v, column = token)
 
 // W words of bf16 pairs from 2W fp32 values: hi[m] = (bf16(x[2m]), bf16(x[2m+1])) with
 // the even element in the low half, lo[m] the same for the residuals x - hi.  One paired
@@ -267,12 +267,12 @@ __device__ __forceinline__ void conv_taps(const uint4 (&xin)[kTaps][4], const ui
 }
 
 // Conv (4 taps) + SiLU of 32 consecutive channels of one token.
-//   src: the token-0 address of the group's first channel; rows before the
-//   sequence start come from conv_in (or are zero).  wsm: the 32 channels'
-//   weights in shared memory, 16 x uint4 (channels 2u, 2u+1; taps 0..3 each).
-//   All 16 input loads are issued before any arithmetic.
+//   src: the token-0 address of the group's first channel; rows before the sequence start
+//   come from conv_in (or are zero).  w: the 32 channels' weights, 16 x uint4 (channels 2u,
+//   2u+1; taps 0..3 each), in shared or global memory.  All 16 input loads are issued
+//   before any arithmetic.
 __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, long long src_stride,
-                                       long long s, long long t, int n, long long conv_chan0, const uint4* wsm,
+                                       long long s, long long t, int n, long long conv_chan0, const uint4* w,
                                        float* y) {
   const long long C_conv = static_cast<long long>(2 * p.H_k + p.H_v) * kD;
   uint4 xin[kTaps][4];
@@ -287,7 +287,7 @@ __device__ __forceinline__ void conv32(const PrefillParams& p, const bf16* src, 
 #pragma unroll
     for (int g = 0; g < 4; ++g) xin[j][g] = row ? __ldg(row + g) : make_uint4(0u, 0u, 0u, 0u);
   }
-  conv_taps(xin, wsm, y);
+  conv_taps(xin, w, y);
 }
 
 // One block diagonal of the blocked inverse: for blocks (I, J = I - d),
@@ -383,9 +383,6 @@ __device__ __forceinline__ void conv32_rows(const uint8_t* raw, int i, int off, 
   conv_taps(xin, wsm, y);
 }
 
-// One CTA per (chunk, key head).  Writes the chunk's K image for the key head
-// and, for each of its value heads, W^T, (gamma Q)^T, P, U0 and the gate vectors.
-// The operand images leave shared memory as bulk stores.
 // Word of the gate area of (chunk gc, value head h) that the fused launch uses as the
 // ready flag of the chunk's operands (the gate vectors occupy words 0 .. 128).
 __device__ __forceinline__ int* ready_flag(const PrefillParams& p, long long gc, int h) {
@@ -399,9 +396,9 @@ __device__ __forceinline__ int* ready_flag(const PrefillParams& p, long long gc,
 // `k` counts the items these threads ran before with the same mbarriers (initialised at k = 0;
 // every wait takes its phase parity from k).  When go_flag is given, it is set once the first
 // value head is done (or the item ends), which lets the other half of a CTA start out of phase.
-// Writes the chunk's K image for the key head and, for each of its value heads, W^T,
-// (gamma Q)^T, P, U0 and the gate vectors; the operand images leave shared memory as bulk
-// stores.  In a fused launch it then publishes the chunk through the value heads' ready flags.
+// Writes the chunk's K and Q images for the key head and, for each of its value heads,
+// -W^T, P, B_U, v_hat and the gate vectors; the operand images leave shared memory as bulk
+// stores (v_hat goes straight from registers).  In a fused launch it then publishes the chunk through the value heads' ready flags.
 __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, int kh, int half, uint8_t* sm,
                                           uint32_t tbase, uint64_t* bar, int* abort_s, int k, int* go_flag) {
   const int bar_id = 2 + half;
@@ -413,8 +410,8 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   float* sG = reinterpret_cast<float*>(sm + kPrepOffG);
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
   float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
-  uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [(2 + G) * 64] channel pairs: q | k | v heads
-  // bar: [Q;K] K^T, W / U0 (per head), drain, q^T
+  uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [2 * 64] channel pairs: q | k
+  // bar: [Q;K] K^T, W (per head), drain
 
   const int tid = threadIdx.x & (kPrepThreads - 1), warp = tid >> 5, lane = tid & 31;
   const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k;
@@ -446,33 +443,98 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   }
   named_bar_sync(bar_id, kPrepThreads);
 
-  // ---- raw q | k rows into region R: 16-byte asynchronous copies by all threads (a warp
-  // moves one 512-byte row per instruction); rows before the sequence start come from
-  // conv_in, or are zero.  The value heads' raw v rows are prefetched into L2 for later.
-  for (int x = tid; x < nrows * 32; x += kPrepThreads) {
-    const int r = x >> 5, piece = x & 31, which = piece >> 4;
-    const long long tau = t0 - (kTaps - 1) + r;
-    uint8_t* dst = sR + r * kRawStride + piece * 16;
-    const bf16* src = nullptr;
-    if (tau >= s) src = (which ? p.k + tau * p.sk : p.q + tau * p.sq) + static_cast<long long>(kh) * kD;
-    else if (p.conv_in)
-      src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + static_cast<long long>(which * H_k + kh) * kD;
-    if (src) cp_async16(dst, src + (piece & 15) * 8);
-    else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  cp_async_commit();
-  for (int x = tid; x < nrows * G * 2; x += kPrepThreads) {  // 128-byte lines of G*256-byte rows
-    const int r = x / (G * 2), line = x % (G * 2);
-    const long long tau = t0 - (kTaps - 1) + r;
-    if (tau >= s) prefetch_l2_line(p.v + tau * p.sv + static_cast<long long>(kh) * G * kD + line * 64);
+  // ---- v_hat = SiLU(conv(v)) of the value heads, kVBatch heads at a time: their raw rows
+  // (tokens t0 - 3 .. t0 + L - 1) are staged in the [Q;K] region with 16-byte asynchronous
+  // copies (rows before the sequence start from conv_in, or zero), then each thread takes
+  // 4 tokens x 8 channels of each head of the batch and stores the hi/lo pieces straight
+  // into the workspace's MN-major image (rows past the chunk's end zero).  The raw q | k rows
+  // of the front end are requested behind the first batch, so their latency overlaps it.
+  for (int jb = 0; jb < G; jb += kVBatch) {
+    const int nb = min(kVBatch, G - jb);
+    const int vstride = nb * kD * 2 + 16;  // one staged row: nb heads x 128 channels, 16 B of padding
+    for (int x = tid; x < nrows * nb * 16; x += kPrepThreads) {
+      const int r = x / (nb * 16), piece = x % (nb * 16);
+      const long long tau = t0 - (kTaps - 1) + r;
+      const long long ch = static_cast<long long>(kh * G + jb) * kD + piece * 8;  // v channel
+      uint8_t* dst = sQK + r * vstride + piece * 16;
+      const bf16* src = nullptr;
+      if (tau >= s) src = p.v + tau * p.sv + ch;
+      else if (p.conv_in) src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + 2LL * H_k * kD + ch;
+      if (src) cp_async16(dst, src);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+    if (jb == 0) {
+      // raw q | k rows into region R: 16-byte asynchronous copies by all threads (a warp moves
+      // one 512-byte row per instruction); rows before the sequence start come from conv_in,
+      // or are zero
+      for (int x = tid; x < nrows * 32; x += kPrepThreads) {
+        const int r = x >> 5, piece = x & 31, which = piece >> 4;
+        const long long tau = t0 - (kTaps - 1) + r;
+        uint8_t* dst = sR + r * kRawStride + piece * 16;
+        const bf16* src = nullptr;
+        if (tau >= s) src = (which ? p.k + tau * p.sk : p.q + tau * p.sq) + static_cast<long long>(kh) * kD;
+        else if (p.conv_in)
+          src = p.conv_in + (static_cast<long long>(n) * 3 + 3 + (tau - s)) * C_conv + static_cast<long long>(which * H_k + kh) * kD;
+        if (src) cp_async16(dst, src + (piece & 15) * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      cp_async_commit();
+      cp_async_wait_group<1>();  // the v rows (the q | k rows may still be in flight)
+    } else {
+      cp_async_wait_group<0>();
+    }
+    named_bar_sync(bar_id, kPrepThreads);
+    const int cg = tid & 15, tg = tid >> 4;  // 8 channels, 4 tokens
+    for (int jj = 0; jj < nb; ++jj) {
+      const int h = kh * G + jb + jj;
+      float2 wv[4][kTaps];
+      {
+        const uint4* wsrc = reinterpret_cast<const uint4*>(p.conv_w + (2LL * H_k * kD + static_cast<long long>(h) * kD + 8 * cg) * kTaps);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w = __ldg(wsrc + q);
+          wv[q][0] = make_float2(bf16_lo(w.x), bf16_lo(w.z));
+          wv[q][1] = make_float2(bf16_hi(w.x), bf16_hi(w.z));
+          wv[q][2] = make_float2(bf16_lo(w.y), bf16_lo(w.w));
+          wv[q][3] = make_float2(bf16_hi(w.y), bf16_hi(w.w));
+        }
+      }
+      const uint8_t* rsrc = sQK + jj * kD * 2 + cg * 16;
+      uint8_t* gv = p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffV + (cg >> 3) * 8192;
+      uint4 rw[4 + kTaps - 1];
+#pragma unroll
+      for (int r = 0; r < 4 + kTaps - 1; ++r) rw[r] = *reinterpret_cast<const uint4*>(rsrc + (4 * tg + r) * vstride);
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        const int i = 4 * tg + ii;
+        float y[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // channel pair q: taps on rows ii .. ii + 3
+          const uint32_t x0 = (&rw[ii].x)[q], x1 = (&rw[ii + 1].x)[q], x2 = (&rw[ii + 2].x)[q], x3 = (&rw[ii + 3].x)[q];
+          float2 a = __fmul2_rn(wv[q][0], make_float2(bf16_lo(x0), bf16_hi(x0)));
+          a = __ffma2_rn(wv[q][1], make_float2(bf16_lo(x1), bf16_hi(x1)), a);
+          a = __ffma2_rn(wv[q][2], make_float2(bf16_lo(x2), bf16_hi(x2)), a);
+          a = __ffma2_rn(wv[q][3], make_float2(bf16_lo(x3), bf16_hi(x3)), a);
+          y[2 * q] = i < L ? silu_fast(a.x) : 0.f;
+          y[2 * q + 1] = i < L ? silu_fast(a.y) : 0.f;
+        }
+        uint4 hi, lo;
+        split8(y, hi, lo);
+        const uint32_t off = sw128_off(i, cg & 7);
+        *reinterpret_cast<uint4*>(gv + off) = hi;
+        *reinterpret_cast<uint4*>(gv + kImg64 + off) = lo;
+      }
+    }
+    named_bar_sync(bar_id, kPrepThreads);  // the staged rows are read: the region is free
   }
 
-  // conv weights of this CTA's channels (q, k of key head kh; v of its G value heads)
-  for (int x = tid; x < (2 + G) * 64; x += kPrepThreads) {
-    const int pair = x % 64, grp = x / 64;  // grp 0 = q, 1 = k, 2.. = value head grp-2
-    const long long ch0 = grp == 0 ? static_cast<long long>(kh) * kD
-                        : grp == 1 ? static_cast<long long>(H_k + kh) * kD
-                                   : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh * G + grp - 2) * kD;
+  // (raw q | k rows: requested above, behind the first v batch)
+
+  // conv weights of this CTA's channels (q and k of key head kh)
+  for (int x = tid; x < 2 * 64; x += kPrepThreads) {
+    const int pair = x % 64, grp = x / 64;  // grp 0 = q, 1 = k
+    const long long ch0 = static_cast<long long>(grp * H_k + kh) * kD;
     cp_async16(&sW[x], p.conv_w + (ch0 + 2 * pair) * kTaps);  // waited for with the raw rows
   }
 
@@ -544,14 +606,15 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   named_bar_sync(bar_id, kPrepThreads);
   tc_fence_after();
 
-  // ---- the K image to the workspace (the K rows of the four K-block halves), and
-  // [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
+  // ---- the K and Q images to the workspace (the K rows, then the Q rows, of the four
+  // K-block halves), and [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
   if (tid == 0) {
-    uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
-    bulk_s2g(gK, sQK + 8192, 8192);
-    bulk_s2g(gK + 8192, sQK + 24576, 8192);
-    bulk_s2g(gK + 16384, sQK + 40960, 8192);
-    bulk_s2g(gK + 24576, sQK + 57344, 8192);
+    uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKQBytes);
+#pragma unroll
+    for (int piece = 0; piece < 4; ++piece) {  // hi block 0, hi block 1, lo block 0, lo block 1
+      bulk_s2g(gK + kKQOffK + piece * 8192, sQK + piece * 16384 + 8192, 8192);
+      bulk_s2g(gK + kKQOffQ + piece * 8192, sQK + piece * 16384, 8192);
+    }
     bulk_commit();
     const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
     const uint32_t idesc = idesc_bf16(128, 64, false, false);
@@ -580,20 +643,6 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     if (k2 != kReadyFlagWord) gdst[k2] = val;
   }
 
-  // identity B image for the q^T transpose, in region R (the raw rows are dead)
-  {
-    uint8_t* sId = sR;
-    for (int x = tid; x < 64 * 8; x += kPrepThreads) {
-      const int i = x >> 3, cc = x & 7;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (cc == (i >> 3)) {
-        const int e8 = i & 7;
-        w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;
-      }
-      *reinterpret_cast<uint4*>(sId + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
-
   // ---- K K^T and Q K^T rows into registers: thread row = 32*(warp%4)+lane, columns cbase..cbase+31
   const int row = 32 * (warp & 3) + lane;
   const int cbase = 32 * (warp >> 2);
@@ -601,28 +650,9 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   const int ri = row & 63;
   // (the [Q;K] K^T rows stay in tensor memory and are read again for each value head)
   const bool qk_ok = mbar_wait_warp(&bar[0], ph, ab);
-
-  // ---- q^T (lane = d_k, column = token) into TMEM columns 64..127: Q_hi^T I + Q_lo^T I
-  // with an identity B, exact in fp32
-  fence_proxy_async_smem();
-  tc_fence_before();
-  named_bar_sync(bar_id, kPrepThreads);  // the identity is complete
   tc_fence_after();
-  if (tid == 0) {
-    const uint32_t qk = smem_u32(sQK), id = smem_u32(sR);
-    const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
-      umma_bf16(tbase + kPrepColQT, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
-      umma_bf16(tbase + kPrepColQT, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
-    }
-    umma_commit(&bar[3]);
-  }
-  __syncwarp();
-  mbar_wait_warp(&bar[3], ph, ab);
-  tc_fence_after();
-  named_bar_sync(bar_id, kPrepThreads);  // Q and the identity are dead: the Q pieces and region R are scratch from here
+  if (tid == 0) bulk_wait_read<0>();  // the K and Q images have left shared memory
+  named_bar_sync(bar_id, kPrepThreads);  // Q is dead: the Q pieces and region R are scratch from here
 
   for (int j = 0; j < G; ++j) {
     const int h = kh * G + j;
@@ -671,7 +701,9 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     solve_unit_lower(sA, sT, sM, tid, bar_id);
     if (tid == 0) bulk_wait_read<0>();  // P has left the Q pieces
     named_bar_sync(bar_id, kPrepThreads);
-    // B_W = T diag(beta gamma), B_U = T diag(beta): K-major (row i, 64 j), lower triangle incl. diagonal
+    // B_W = T diag(beta gamma) into the Q pieces, B_U = T diag(beta) over the dead A: K-major
+    // (row i, 64 j), lower triangle incl. diagonal
+    uint8_t* sBU = sm + kPrepOffBU;  // lo | hi
     for (int x = tid; x < 64 * 8; x += kPrepThreads) {
       const int r = x >> 3, cc = x & 7;
       float fu[8], fw[8];
@@ -688,35 +720,16 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
       *reinterpret_cast<uint4*>(sQK + kPrepOffBWhi + off) = hi;
       *reinterpret_cast<uint4*>(sQK + kPrepOffBWlo + off) = lo;
       split8(fu, hi, lo);
-      *reinterpret_cast<uint4*>(sQK + kPrepOffBUhi + off) = hi;
-      *reinterpret_cast<uint4*>(sQK + kPrepOffBUlo + off) = lo;
-    }
-    named_bar_sync(bar_id, kPrepThreads);  // T is dead: region R takes the v_hat image
-    {
-      // v_hat of value head h: token i, channels 32*qq .. 32*qq+31, as the MN-major image
-      const int i = (tid & 7) | ((tid >> 5) << 3), qq = (tid >> 3) & 3;
-      float y[32];
-      if (i < L) {
-        conv32(p, p.v + static_cast<long long>(h) * kD + 32 * qq, p.sv, s, t0 + i, n,
-               2LL * H_k * kD + static_cast<long long>(h) * kD + 32 * qq, sW + (2 + j) * 64 + 16 * qq, y);
-      } else {
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) y[e2] = 0.f;
-      }
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-        uint4 hi, lo;
-        split8(y + 8 * c2, hi, lo);
-        const uint32_t off = (qq >> 1) * 8192u + sw128_off(i, (qq & 1) * 4 + c2);
-        *reinterpret_cast<uint4*>(sR + off) = hi;
-        *reinterpret_cast<uint4*>(sR + kImg64 + off) = lo;
-      }
+      *reinterpret_cast<uint4*>(sBU + off) = lo;
+      *reinterpret_cast<uint4*>(sBU + kPImg + off) = hi;
     }
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
+      bulk_s2g(hb + kHeadOffBU, sBU, 2 * kPImg);
+      bulk_commit();
       // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
       const uint32_t qk = smem_u32(sQK);
       const uint32_t idesc_w = idesc_bf16(128, 64, true, false);
@@ -726,62 +739,28 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
                    smem_desc(qk + 32768u + 8192u + ks * 2048u, 16384, 1024, Swz::k128),
                    smem_desc(qk + kPrepOffBWhi + ks * 32u, 16, 1024, Swz::k128),
                    smem_desc(qk + kPrepOffBWlo + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
-      // U0^T = V^T B_U^T: A = v_hat (MN-major, rows = tokens), B = B_U (K-major)
-      const uint32_t vv = smem_u32(sR);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        umma_split(tbase + kPrepColU, smem_desc(vv + ks * 2048u, 8192, 1024, Swz::k128),
-                   smem_desc(vv + kImg64 + ks * 2048u, 8192, 1024, Swz::k128),
-                   smem_desc(qk + kPrepOffBUhi + ks * 32u, 16, 1024, Swz::k128),
-                   smem_desc(qk + kPrepOffBUlo + ks * 32u, 16, 1024, Swz::k128), idesc_w, ks > 0);
       umma_commit(&bar[1]);
     }
     __syncwarp();
     if (mbar_wait_warp(&bar[1], (k * G + j) & 1, ab)) {
       tc_fence_after();
-      {
-        // (gamma Q)^T row d_k = lane, tokens 32*(warp/4) .. +31: staged in region R, hi then lo
-        const int kr = 32 * (warp & 3) + lane, half = warp >> 2;
-        float qg[32];
-        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQT + 32 * half), qg);
-        tmem_wait_ld();
+      // -W^T row d_k = 32 (warp % 4) + lane, tokens 32 (warp / 4) .. +31: staged lo rows
+      // 0..63 | 64..127 in the Q pieces at 0 | 16384, hi rows 0..63 | 64..127 at 32768 | 49152
+      const int kr = 32 * (warp & 3) + lane, half = warp >> 2;
+      float o[32];
+      tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColW + 32 * half), o);
+      tmem_wait_ld();
+      const uint32_t half_off = kr < 64 ? 0u : 16384u;
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          float f[8];
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float f[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) f[e2] = qg[8 * c2 + e2] * sGam[j * 64 + 32 * half + 8 * c2 + e2];
-          uint4 hi, lo;
-          split8(f, hi, lo);
-          const uint32_t off = sw128_off(kr, 4 * half + c2);
-          *reinterpret_cast<uint4*>(sR + off) = hi;
-          *reinterpret_cast<uint4*>(sR + kImg64 + off) = lo;
-        }
-      }
-      float o[64];
-      if (warp < 4) {
-        // W^T row d_k = lane (64 tokens): staged lo rows 0..63 | 64..127 in the Q pieces at 0 | 16384,
-        // hi rows 0..63 | 64..127 at 32768 | 49152
-        tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW), o);
-        tmem_ld32(tmem_addr(tbase, 32 * warp, kPrepColW + 32), o + 32);
-        tmem_wait_ld();
-        const int kr = 32 * warp + lane;
-        const uint32_t half_off = kr < 64 ? 0u : 16384u;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          uint4 hi, lo;
-          split8(o + 8 * cc, hi, lo);
-          const uint32_t off = sw128_off(kr & 63, cc);
-          *reinterpret_cast<uint4*>(sQK + half_off + off) = lo;
-          *reinterpret_cast<uint4*>(sQK + 32768 + half_off + off) = hi;
-        }
-      } else {
-        // U0 [token / 4][d_v][4] fp32: a warp writes 512 contiguous bytes per token quad
-        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU), o);
-        tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColU + 32), o + 32);
-        tmem_wait_ld();
-        float4* u0 = reinterpret_cast<float4*>(hb + kHeadOffU0) + 32 * (warp & 3) + lane;
-#pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) u0[q4 * kD] = make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
+        for (int e2 = 0; e2 < 8; ++e2) f[e2] = -o[8 * c2 + e2];
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t off = sw128_off(kr & 63, 4 * half + c2);
+        *reinterpret_cast<uint4*>(sQK + half_off + off) = lo;
+        *reinterpret_cast<uint4*>(sQK + 32768 + half_off + off) = hi;
       }
       fence_proxy_async_smem();
     }
@@ -789,14 +768,13 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
-      uint8_t* wq = hb + kHeadOffWQ;  // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
-      bulk_s2g(wq, sQK, 8192);
-      bulk_s2g(wq + 8192, sQK + 16384, 8192);
-      bulk_s2g(wq + 16384, sQK + 32768, 8192);
-      bulk_s2g(wq + 24576, sQK + 49152, 8192);
-      bulk_s2g(wq + 2 * kImg64, sR, 2 * kImg64);
+      uint8_t* wd = hb + kHeadOffW;  // -W^T lo | -W^T hi
+      bulk_s2g(wd, sQK, 8192);
+      bulk_s2g(wd + 8192, sQK + 16384, 8192);
+      bulk_s2g(wd + 16384, sQK + 32768, 8192);
+      bulk_s2g(wd + 24576, sQK + 49152, 8192);
       bulk_commit();
-      bulk_wait_read<0>();  // the staging areas are rewritten by the next value head
+      bulk_wait_read<0>();  // the staging areas (Q pieces, B_U) are rewritten by the next value head
     }
     named_bar_sync(bar_id, kPrepThreads);
     if (go_flag && tid == 0) *reinterpret_cast<volatile int*>(go_flag) = 1;
@@ -812,8 +790,8 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     bulk_wait<0>();
   }
   if (p.fused_scan_ctas > 0) {
-    // publish: every store of this chunk (bulk images drained above, U0 and gate vectors by
-    // all threads) is visible before the value heads' ready flags
+    // publish: every store of this chunk (bulk images drained above, v_hat and gate vectors
+    // by all threads) is visible before the value heads' ready flags
     __threadfence();
     named_bar_sync(bar_id, kPrepThreads);
     if (tid == 0) {
@@ -847,18 +825,19 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // One CTA per (sequence, value head); the whole 128 x 128 state lives in tensor
 // memory with lane = d_v row.  Per chunk, every product summed over the hi/lo
 // split terms (hi.hi + hi.lo + lo.hi):
-//   [U^T | O^T] = S [W^T | (gamma Q)^T]  (A = S hi/lo from TMEM; the U^T half first)
-//   U^T  = U0^T - (S W^T)
-//   S    = gamma_C S + (U^T diag(e^{G_C - G_j})) K   (A = U_d hi/lo from TMEM)
-//   O^T += U^T P^T                       (A = U hi/lo from TMEM)
-//   then the gated RMS-norm of o_i over d_v.
+//   U^T = V^T B_U^T + S (-W)^T          (A = v_hat from shared memory, then S hi/lo from TMEM)
+//   X   = S Q^T                         (the state's part of o, before the decay gamma_i)
+//   S   = gamma_C S + (U^T diag(e^{G_C - G_j})) K   (A = U_d hi/lo from TMEM)
+//   Y   = U^T P^T                       (A = U hi/lo from TMEM)
+//   o_i = gamma_i X_i + Y_i, then the gated RMS-norm of o_i over d_v.
+// V^T B_U^T (the state-independent part of U, U0) is accumulated first, off the chain:
+// once the previous chunk's products have read the U columns and before S is converted.
 // Warps 0-7 (thread = d_v row; warps w and w + 4 share a TMEM lane quarter and
 // split its columns) convert S and U between fp32 accumulators and bf16 hi/lo
 // operands in tensor memory, each conversion publishing first the part the next
 // product waits for; warps 8-11 run the output stage; warp 12 lane 0 issues the
-// MMAs in the order S W^T, S (gamma Q)^T, state update, U^T P^T, so that the
-// output's products fill the tensor pipe while the chain converts; warp 13
-// lane 0 issues the bulk copies (W, gamma Q, K, P single-buffered, gates and U0 double-buffered).
+// MMAs; warp 13 lane 0 issues the bulk copies (v_hat, B_U, W, Q, K, P single-buffered,
+// gates double-buffered).
 
 constexpr int kScanThreads = 448;
 constexpr int kScanBar = 15;  // named barrier of the scan's CTA-wide steps
@@ -867,10 +846,11 @@ constexpr int kWarpIssue = 12, kWarpProd = 13;
 constexpr uint32_t kColS = 0;      // S fp32, 128 columns (d_k)
 constexpr uint32_t kColSH = 128;   // S hi, bf16 pairs along d_k (64 columns)
 constexpr uint32_t kColSL = 192;   // S lo
-// [S_hi W_lo^T | (S_hi + S_lo) W_hi^T | O part 1 | O part 2], 4 x 64 columns
-constexpr uint32_t kColU2 = 256;   //   U^T = U0^T - (U2 + U1)
+// [V_hi B_U_lo - S_hi W_lo | V_hi B_U_hi + V_lo B_U_hi - S_hi W_hi - S_lo W_hi], 2 x 64 columns
+constexpr uint32_t kColU2 = 256;   //   U^T = U2 + U1
 constexpr uint32_t kColU1 = 320;
-constexpr uint32_t kColO = 384;    //   o = O1 + O2 (gamma Q S^T, then + P U accumulated by the last product)
+constexpr uint32_t kColX = 384;    // X = S Q^T (64 columns)
+constexpr uint32_t kColY = 448;    // Y = U^T P^T (64 columns)
 // After the U conversion, in place: the chain warp of token half th (tokens 32 th .. +31)
 // read U2 / U1 columns 256 + 32 th / 320 + 32 th and writes there, 16 columns each,
 //   U hi at 256 + 32 th, U lo at 272 + 32 th, U_d hi at 320 + 32 th, U_d lo at 336 + 32 th,
@@ -881,20 +861,23 @@ constexpr uint32_t kColUDH = 320;
 constexpr uint32_t kColUDL = 336;
 __host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base + 32u * (ks >> 1) + 8u * (ks & 1); }
 // shared memory (offsets from a 1024-aligned base)
-constexpr int kScOffWQ = 0;                            // W^T lo | W^T hi | (gQ)^T hi | (gQ)^T lo
-constexpr int kScOffK = kScOffWQ + kWQBytes;           // K hi, lo
-constexpr int kScOffP = kScOffK + kKBytes;             // P hi, lo
-constexpr int kScOffU0 = kScOffP + 2 * kPImg;          // 2 stages of U0 fp32 [16 token quads][128][4]
-constexpr int kScOffO = kScOffU0 + 2 * kU0Bytes;       // o fp32 [64 tokens][128 d_v] for the token-major epilogue
+constexpr int kScOffW = 0;                             // -W^T lo | -W^T hi
+constexpr int kScOffQ = kScOffW + kWBytes;             // Q hi | Q lo
+constexpr int kScOffK = kScOffQ + 2 * kImg64;          // K hi | K lo
+constexpr int kScOffP = kScOffK + 2 * kImg64;          // P hi | P lo
+constexpr int kScOffBU = kScOffP + 2 * kPImg;          // B_U lo | B_U hi
+constexpr int kScOffV = kScOffBU + 2 * kPImg;          // v_hat hi | lo (MN-major: row = token, two 64-channel blocks)
+constexpr int kScOffO = kScOffV + 2 * kImg64;          // o fp32 [64 tokens][128 d_v] for the token-major epilogue
 constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 
 // The scan of one (sequence, value head) (`blk` = sequence rank * H_v + value head) by the
 // CTA's first 448 threads, with shared memory at sm (1024-aligned, kScSmem - 1024 bytes).
-// CTA-wide steps use named barrier kScanBar over those threads.
+// CTA-wide steps use named barrier kScanBar.
 __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8_t* sm) {
   __shared__ uint64_t g_full[2], g_free[2];
-  __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, u0_full[2], u0_free[2];
+  __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, bu_full, bu_free;
+  __shared__ uint64_t v_full, v_free;
   __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
@@ -912,9 +895,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     abort_s = 0;
     for (int b = 0; b < 2; ++b) {
       mbar_init(&g_full[b], 1);
-      mbar_init(&g_free[b], 256);
-      mbar_init(&u0_full[b], 1);
-      mbar_init(&u0_free[b], 256);
+      mbar_init(&g_free[b], 256 + 128);  // the conversion and output warps
     }
     mbar_init(&w_full, 1);
     mbar_init(&w_free, 1);
@@ -924,6 +905,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     mbar_init(&k_free, 1);
     mbar_init(&p_full, 1);
     mbar_init(&p_free, 1);
+    mbar_init(&bu_full, 1);
+    mbar_init(&bu_free, 1);
+    mbar_init(&v_full, 1);
+    mbar_init(&v_free, 1);
     mbar_init(&s_conv, 256);
     mbar_init(&u_conv, 256);
     mbar_init(&u_conv2, 256);
@@ -951,7 +936,6 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       const int gs = c & 1;
       const float* gates = reinterpret_cast<const float*>(sm + kScOffG + gs * kGateBytes);
       // ---- S_c (columns 64 th .. +63) -> hi/lo operand; then S <- gamma_C S for the update
-      // (the previous chunk's products that read S hi/lo were issued before its state update)
       ok = c == 0 || mbar_wait_warp(&s_done, (c - 1) & 1, ab);
       if (ok) ok = mbar_wait_warp(&g_full[gs], (c >> 1) & 1, ab);
       if (!ok) break;
@@ -974,6 +958,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tmem_ld32(tl + kColS + 64 * th + 32, sv + 32);
         tmem_wait_ld();
       }
+      // the previous chunk's X = S Q^T (issued around the state update) still reads S hi/lo
+      if (c > 0) ok = mbar_wait_warp(&q_free, (c - 1) & 1, ab);
+      if (!ok) break;
+      tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t hi[16], lo[16];
@@ -993,11 +981,9 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       }
       tmem_st32(tl + kColS + 64 * th, sv);
       tmem_st32(tl + kColS + 64 * th + 32, sv + 32);
-      // ---- U^T = U0^T - S W^T for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first
-      // (the state update waits for it), then U (the output product waits for it)
+      // ---- U^T = U2 + U1 for tokens 32 th .. +31: U_d = U^T diag(decay-to-end) first (the
+      // state update waits for it), then U (the output product waits for it)
       ok = mbar_wait_warp(&u_done, c & 1, ab);
-      if (ok) ok = mbar_wait_warp(&u0_full[gs], (c >> 1) & 1, ab);
-      const float* U0 = reinterpret_cast<const float*>(sm + kScOffU0 + gs * kU0Bytes);
       if (!ok) break;
       tc_fence_after();
       float u[32], ud[32];
@@ -1006,19 +992,13 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tmem_ld32(tl + kColU2 + 32 * th, u);
         tmem_ld32(tl + kColU1 + 32 * th, u1);
         tmem_wait_ld();
-        const float4* U0q = reinterpret_cast<const float4*>(U0) + (8 * th) * kD + v;  // [token / 4][d_v][4]
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {  // u = U0 - (U1 + U2), packed in token pairs
-          const float4 u0 = U0q[q4 * kD];
-          const int i = 4 * q4;
-          const float2 a0 = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
-          const float2 a1 = __fadd2_rn(make_float2(u1[i + 2], u1[i + 3]), make_float2(u[i + 2], u[i + 3]));
-          const float2 r0 = __ffma2_rn(a0, make_float2(-1.f, -1.f), make_float2(u0.x, u0.y));
-          const float2 r1 = __ffma2_rn(a1, make_float2(-1.f, -1.f), make_float2(u0.z, u0.w));
-          u[i] = r0.x; u[i + 1] = r0.y; u[i + 2] = r1.x; u[i + 3] = r1.y;
+        for (int i = 0; i < 32; i += 2) {
+          const float2 r = __fadd2_rn(make_float2(u1[i], u1[i + 1]), make_float2(u[i], u[i + 1]));
+          u[i] = r.x;
+          u[i + 1] = r.y;
         }
       }
-      mbar_arrive(&u0_free[gs]);
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         const float2 d = *reinterpret_cast<const float2*>(gates + 64 + 32 * th + i);
@@ -1026,7 +1006,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         ud[i] = r.x;
         ud[i + 1] = r.y;
       }
-      mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time
+      mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time by this warp
       {
         uint32_t hi[16], lo[16];
         split_pairs_x2<16>(ud, hi, lo);
@@ -1066,63 +1046,104 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
   } else if (warp == kWarpIssue) {
     // ------------------------------------------------ tensor-core issue (one thread)
     if (lane == 0) {
-      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [W_lo | W_hi], S_hi [gQ_hi | gQ_lo]
-      const uint32_t idesc_u2 = idesc_bf16(128, 64, false, true);   // S_lo W_hi, S_lo gQ_hi
+      const uint32_t idesc_v = idesc_bf16(128, 128, true, false);   // v_hi^T [B_U lo | B_U hi] (A MN-major)
+      const uint32_t idesc_v2 = idesc_bf16(128, 64, true, false);   // v_lo^T B_U hi
+      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [-W_lo | -W_hi] (B MN-major)
+      const uint32_t idesc_u2 = idesc_bf16(128, 64, false, true);   // S_lo (-W_hi)
+      const uint32_t idesc_x = idesc_bf16(128, 64, false, false);   // S Q^T (Q K-major: N = tokens)
       const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
-      const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
-      const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
-      const uint32_t wq = smem_u32(sm + kScOffWQ);
+      const uint32_t idesc_y = idesc_bf16(128, 64, false, false);   // U P^T (K-major)
+      const uint32_t w_lo = smem_u32(sm + kScOffW), w_hi = w_lo + kImg64;
+      const uint32_t q_hi = smem_u32(sm + kScOffQ), q_lo = q_hi + kImg64;
       const uint32_t k_hi = smem_u32(sm + kScOffK), k_lo = k_hi + kImg64;
-      const uint32_t p_hi = smem_u32(sm + kScOffP);
+      const uint32_t p_hi = smem_u32(sm + kScOffP), p_lo = p_hi + kPImg;
+      const uint32_t bu_lo = smem_u32(sm + kScOffBU), bu_hi = bu_lo + kPImg;
+      const uint32_t v_hi = smem_u32(sm + kScOffV), v_lo = v_hi + kImg64;
       for (int c = 0; c < nc; ++c) {
+        // U0 = v_hat^T B_U^T into [U2 | U1], once the previous chunk's update and output
+        // products (their commit covers every earlier MMA) have read the U columns
+        if (c > 0 && !mbar_wait(&y_done, (c - 1) & 1, ab)) break;
+        if (!mbar_wait(&v_full, c & 1, ab)) break;
+        if (!mbar_wait(&bu_full, c & 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ah = smem_desc(v_hi + ks * 2048u, 8192, 1024, Swz::k128);
+          const uint64_t al = smem_desc(v_lo + ks * 2048u, 8192, 1024, Swz::k128);
+          const uint64_t b2 = smem_desc(bu_lo + ks * 32u, 16, 1024, Swz::k128);  // 128 rows: B_U lo then hi
+          const uint64_t bh = smem_desc(bu_hi + ks * 32u, 16, 1024, Swz::k128);
+          umma_bf16(tbase + kColU2, ah, b2, idesc_v, ks > 0);
+          umma_bf16(tbase + kColU1, al, bh, idesc_v2, true);
+        }
+        umma_commit(&v_free);
+        umma_commit(&bu_free);
+        // the chain's product: [U2 | U1] += S_hi [-W_lo | -W_hi], U1 += S_lo (-W_hi)
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
         if (!mbar_wait(&w_full, c & 1, ab)) break;
-        if (c > 0 && !mbar_wait(&y_done, (c - 1) & 1, ab)) break;  // U^T P^T of the last chunk read the U columns
         tc_fence_after();
-        // the chain's product first: [U2 | U1] = S_hi [W_lo | W_hi], U1 += S_lo W_hi
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
-          const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
-          umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, ks > 0);
+          const uint64_t bw = smem_desc(w_lo + ks * 2048u, kImg64, 1024, Swz::k128);
+          const uint64_t bw2 = smem_desc(w_hi + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, true);
           umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
         }
         umma_commit(&u_done);
         umma_commit(&w_free);
-        // then the output's: [O1 | O2] = S_hi [gQ_hi | gQ_lo], O1 += S_lo gQ_hi, once o(c-1) has been read
+        // X = S Q^T, once x(c-1) and y(c-1) have been read, in groups of two K steps; the state
+        // update (the chain's next product) goes out between two groups as soon as U_d and K
+        // are in place
         if (!mbar_wait(&q_full, c & 1, ab)) break;
         if (c > 0 && !mbar_wait(&o_free, (c - 1) & 1, ab)) break;
         tc_fence_after();
+        bool s_issued = false;
+        auto issue_update = [&]() {  // S += U_d^T K (onto gamma_C S)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bq = smem_desc(wq + 2 * kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
-          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, ks > 0);
-          umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, bq, idesc_u2, true);
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
+            const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
+            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
+            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
+            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
+          }
+          umma_commit(&s_done);
+          umma_commit(&k_free);
+          s_issued = true;
+        };
+#pragma unroll
+        for (int kg = 0; kg < 4; ++kg) {
+          if (!s_issued && mbar_test_wait(&u_conv, c & 1) && mbar_test_wait(&k_full, c & 1)) {
+            tc_fence_after();
+            issue_update();
+          }
+#pragma unroll
+          for (int ks = 2 * kg; ks < 2 * kg + 2; ++ks) {
+            const uint32_t ko = (ks >> 2) * 8192u + (ks & 3) * 32u;
+            const uint64_t bh = smem_desc(q_hi + ko, 16, 1024, Swz::k128);
+            const uint64_t bl = smem_desc(q_lo + ko, 16, 1024, Swz::k128);
+            umma_bf16_ts(tbase + kColX, tbase + kColSH + 8 * ks, bh, idesc_x, ks > 0);
+            umma_bf16_ts(tbase + kColX, tbase + kColSH + 8 * ks, bl, idesc_x, true);
+            umma_bf16_ts(tbase + kColX, tbase + kColSL + 8 * ks, bh, idesc_x, true);
+          }
         }
         umma_commit(&q_free);
-        if (!mbar_wait(&u_conv, c & 1, ab)) break;
-        if (!mbar_wait(&k_full, c & 1, ab)) break;
-        tc_fence_after();
-        // S += U_d^T K (onto gamma_C S)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
-          const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
-          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
+        if (!s_issued) {
+          if (!mbar_wait(&u_conv, c & 1, ab)) break;
+          if (!mbar_wait(&k_full, c & 1, ab)) break;
+          tc_fence_after();
+          issue_update();
         }
-        umma_commit(&s_done);
-        umma_commit(&k_free);
         if (!mbar_wait(&u_conv2, c & 1, ab)) break;
         if (!mbar_wait(&p_full, c & 1, ab)) break;
         tc_fence_after();
-        // [O1 | O2] += U_hi [P_hi | P_lo], O1 += U_lo P_hi
+        // Y = U_hi P_hi + U_hi P_lo + U_lo P_hi
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t b2 = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);  // 128 rows: P hi then P lo
-          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUH, ks), b2, idesc_y, true);
-          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUL, ks), b2, idesc_y2, true);
+          const uint64_t bh = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);
+          const uint64_t bl = smem_desc(p_lo + ks * 32u, 16, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUH, ks), bh, idesc_y, ks > 0);
+          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUH, ks), bl, idesc_y, true);
+          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUL, ks), bh, idesc_y, true);
         }
         umma_commit(&y_done);
         umma_commit(&p_free);
@@ -1137,60 +1158,63 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
   } else if (warp == kWarpProd) {
     // ------------------------------------------------ bulk-copy producer (lane 0)
     if (lane == 0) {
-      // Order of need: W, gamma Q, K, P of chunk c (single stages, each refilled as soon as the
-      // product that reads it has completed), then the double-buffered gates and U0 of chunk c + 1.
-      int n_g[2] = {0, 0}, n_u0[2] = {0, 0}, n_w = 0, n_q = 0, n_k = 0, n_p = 0;
+      // Order of need: v_hat, B_U, W, Q, K, P of chunk c (single stages, each refilled as soon
+      // as the product that reads it has completed), then the double-buffered gates of chunk c + 1.
+      int n_g[2] = {0, 0}, n_v = 0, n_bu = 0, n_w = 0, n_q = 0, n_k = 0, n_p = 0;
       auto head_blob = [&](int c) {
         return p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes);
       };
-      auto load_gates_u0 = [&](int c) -> bool {  // chunk c into stage c & 1
+      auto load_gates = [&](int c) -> bool {  // chunk c into stage c & 1
         const int st = c & 1;
-        const uint8_t* hb = head_blob(c);
         // fused launch: chunk c's operands (read from here on) are published by its prep
         if (p.fused_scan_ctas > 0 && !flag_wait(ready_flag(p, cb + c, h), ab, kBackoffNs)) return false;
         if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
         mbar_arrive_expect_tx(&g_full[st], kGateBytes);
-        bulk_g2s(sm + kScOffG + st * kGateBytes, hb + kHeadOffGate, kGateBytes, &g_full[st]);
+        bulk_g2s(sm + kScOffG + st * kGateBytes, head_blob(c) + kHeadOffGate, kGateBytes, &g_full[st]);
         ++n_g[st];
-        if (c >= 2 && !mbar_wait(&u0_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
-        mbar_arrive_expect_tx(&u0_full[st], kU0Bytes);
-        bulk_g2s(sm + kScOffU0 + st * kU0Bytes, hb + kHeadOffU0, kU0Bytes, &u0_full[st]);
-        ++n_u0[st];
         return true;
       };
-      bool ok = nc == 0 || load_gates_u0(0);
+      bool ok = nc == 0 || load_gates(0);
       for (int c = 0; c < nc && ok; ++c) {
         const uint8_t* hb = head_blob(c);
-        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes);
+        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKQBytes);
+        if (c >= 1 && !mbar_wait(&v_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&v_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffV, hb + kHeadOffV, 2 * kImg64, &v_full);
+        ++n_v;
+        if (c >= 1 && !mbar_wait(&bu_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
+        mbar_arrive_expect_tx(&bu_full, 2 * kPImg);
+        bulk_g2s(sm + kScOffBU, hb + kHeadOffBU, 2 * kPImg, &bu_full);
+        ++n_bu;
         if (c >= 1 && !mbar_wait(&w_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&w_full, 2 * kImg64);
-        bulk_g2s(sm + kScOffWQ, hb + kHeadOffWQ, 2 * kImg64, &w_full);
+        mbar_arrive_expect_tx(&w_full, kWBytes);
+        bulk_g2s(sm + kScOffW, hb + kHeadOffW, kWBytes, &w_full);
         ++n_w;
         if (c >= 1 && !mbar_wait(&q_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&q_full, 2 * kImg64);
-        bulk_g2s(sm + kScOffWQ + 2 * kImg64, hb + kHeadOffWQ + 2 * kImg64, 2 * kImg64, &q_full);
+        bulk_g2s(sm + kScOffQ, kb + kKQOffQ, 2 * kImg64, &q_full);
         ++n_q;
         if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&k_full, kKBytes);
-        bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
+        mbar_arrive_expect_tx(&k_full, 2 * kImg64);
+        bulk_g2s(sm + kScOffK, kb + kKQOffK, 2 * kImg64, &k_full);
         ++n_k;
         if (c >= 1 && !mbar_wait(&p_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&p_full, 2 * kPImg);
         bulk_g2s(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
         ++n_p;
-        if (c + 1 < nc) ok = load_gates_u0(c + 1);
+        if (c + 1 < nc) ok = load_gates(c + 1);
         if (c + 2 < nc) {  // two chunks ahead into L2, behind this chunk's copies
           prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
-          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
+          prefetch_l2(kb + 2LL * p.H_k * kKQBytes, kKQBytes);
         }
       }
       // copies still in flight (only possible after an abort) land before the CTA exits
       int drain_flag = 0;
       Abort drain{nullptr, &drain_flag};
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < 2; ++b)
         if (n_g[b] > 0) mbar_wait(&g_full[b], (n_g[b] - 1) & 1, drain);
-        if (n_u0[b] > 0) mbar_wait(&u0_full[b], (n_u0[b] - 1) & 1, drain);
-      }
+      if (n_v > 0) mbar_wait(&v_full, (n_v - 1) & 1, drain);
+      if (n_bu > 0) mbar_wait(&bu_full, (n_bu - 1) & 1, drain);
       if (n_w > 0) mbar_wait(&w_full, (n_w - 1) & 1, drain);
       if (n_q > 0) mbar_wait(&q_full, (n_q - 1) & 1, drain);
       if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
@@ -1199,8 +1223,8 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     __syncwarp();
   } else {
     // ------------------------------------------------ output stage (warps 8-11)
-    // o leaves tensor memory row-wise (thread = d_v row) into shared memory as fp32
-    // [token][d_v]; then each thread owns 8 consecutive d_v of a token, 16 threads per
+    // o = gamma X + Y leaves tensor memory row-wise (thread = d_v row) into shared memory as
+    // fp32 [token][d_v]; then each thread owns 8 consecutive d_v of a token, 16 threads per
     // token: the sum of o^2 over d_v is a 4-step shuffle inside that group (a fixed
     // order), z is read and out written with 16-byte accesses.
     const int ow = warp & 3;              // TMEM lane quarter
@@ -1215,6 +1239,8 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     // Every output warp reaches every named barrier; a failed wait is OR-ed into the
     // first barrier so that the four warps leave the loop together.
     for (int c = 0; c < nc; ++c) {
+      const int gs = c & 1;
+      const float* gam = reinterpret_cast<const float*>(sm + kScOffG + gs * kGateBytes);
       const long long tok0 = s + static_cast<long long>(c) * kChunk;
       const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - tok0));
       // z of the next chunk into L2 (one 128-byte line per thread), z of this chunk into
@@ -1231,23 +1257,26 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
                       : make_uint4(0u, 0u, 0u, 0u);
       }
       bool ok = mbar_wait_warp(&y_done, c & 1, ab, false, kBackoffNs);
+      if (ok) ok = mbar_wait_warp(&g_full[gs], (c >> 1) & 1, ab);  // (complete: the chain read these gates)
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          float o1[32], o2[32];
-          tmem_ld32(tl + kColO + 32 * cc, o1);
-          tmem_ld32(tl + kColO + 64 + 32 * cc, o2);
+          float xv[32], yv[32];
+          tmem_ld32(tl + kColX + 32 * cc, xv);
+          tmem_ld32(tl + kColY + 32 * cc, yv);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float2 r = __fadd2_rn(make_float2(o1[i], o1[i + 1]), make_float2(o2[i], o2[i + 1]));
+            const float2 g2 = *reinterpret_cast<const float2*>(gam + 32 * cc + i);
+            const float2 r = __ffma2_rn(make_float2(xv[i], xv[i + 1]), g2, make_float2(yv[i], yv[i + 1]));
             sO[(32 * cc + i) * kD + v] = r.x;
             sO[(32 * cc + i + 1) * kD + v] = r.y;
           }
         }
         tc_fence_before();
         mbar_arrive(&o_free);
+        mbar_arrive(&g_free[gs]);
       }
       if (bar_sync_or(1, 128, !ok)) break;
       // the eight tokens' sums of squares side by side (independent shuffles), then the outputs
@@ -1327,10 +1356,9 @@ constexpr int kFusedThreads = 2 * kPrepThreads;
 constexpr int kMaxFusedScanFraction = 2;  // scan CTAs <= SMs / 2
 constexpr int kMinFusedItemsPerSm = 8;    // automatic plan: fuse only with >= 8 prep items per prep SM
 
-__host__ __device__ constexpr int prep_half_bytes(int G) { return (prep_smem_bytes(G) - 1024 + 1023) / 1024 * 1024; }
-__host__ __device__ constexpr int fused_smem_bytes(int G) {
-  return 2 * prep_half_bytes(G) + 1024 > kScSmem ? 2 * prep_half_bytes(G) + 1024 : kScSmem;
-}
+constexpr int kPrepHalfBytes = (kPrepSmem - 1024 + 1023) / 1024 * 1024;
+constexpr int kFusedSmem = 2 * kPrepHalfBytes + 1024 > kScSmem ? 2 * kPrepHalfBytes + 1024 : kScSmem;
+static_assert(kFusedThreads >= kScanThreads, "a fused launch's scan CTAs run the scan on their first threads");
 
 __global__ void __launch_bounds__(kFusedThreads, 1) prefill_fused_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;
@@ -1356,7 +1384,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_fused_kernel(Prefill
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base_s + 256u * half;
-  uint8_t* smh = sm + half * prep_half_bytes(p.H_v / p.H_k);
+  uint8_t* smh = sm + half * kPrepHalfBytes;
   if (half == 1 && htid == 0) {
     // start once half 0 is through its first value head (or found nothing to do): the two
     // halves then reach their latency-bound steps at different times
@@ -1439,7 +1467,7 @@ int fused_scan_ctas(const PrefillParams& p) {
   if (cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
   cudaFuncAttributes attr;
   if (cudaFuncGetAttributes(&attr, prefill_fused_kernel) != cudaSuccess) return 0;
-  if (static_cast<long long>(attr.sharedSizeBytes) + fused_smem_bytes(p.H_v / p.H_k) > smem_optin) return 0;
+  if (static_cast<long long>(attr.sharedSizeBytes) + kFusedSmem > smem_optin) return 0;
   return n_scan;
 }
 
@@ -1469,7 +1497,7 @@ cudaError_t launch_prefill(const PrefillParams& p_in, cudaStream_t stream, void*
     const long long n_flags = p.n_chunks * p.H_v;
     ready_flags_reset_kernel<<<static_cast<unsigned>((n_flags + 255) / 256), 256, 0, stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    const int smem = fused_smem_bytes(p.H_v / p.H_k);
+    const int smem = kFusedSmem;
     err = cudaFuncSetAttribute(prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     const long long n_items = p.n_chunks * p.H_k;
@@ -1487,7 +1515,7 @@ cudaError_t launch_prefill(const PrefillParams& p_in, cudaStream_t stream, void*
   }
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
   if (p.n_chunks > 0) {
-    const int smem = prep_smem_bytes(p.H_v / p.H_k);
+    const int smem = kPrepSmem;
     err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     prep_kernel<<<dim3(static_cast<unsigned>(p.n_chunks), p.H_k), kPrepThreads, smem, stream>>>(p);

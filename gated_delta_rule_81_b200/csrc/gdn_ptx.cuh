@@ -72,6 +72,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of phase `parity` (try_wait may suspend the thread for a while when the
+// phase is not complete).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -204,6 +218,12 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// wait until at most N of this thread's committed cp.async groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // hint: bring the 128-byte line holding `src` into L2
 __device__ __forceinline__ void prefetch_l2_line(const void* src) {
@@ -371,8 +391,14 @@ __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u 
 
 __device__ __forceinline__ float silu_f(float y) { return y / (1.0f + __expf(-y)); }
 
-// SiLU with the fast approximate division (about 2 ulp; y -> -inf gives -0)
-__device__ __forceinline__ float silu_fast(float y) { return __fdividef(y, 1.0f + __expf(-y)); }
+// SiLU y / (1 + 2^(-y log2 e)) on the approximate base-2 exponential and reciprocal (a few ulp;
+// denormal inputs and results flushed to zero; y -> -inf gives -0, y -> +inf gives +inf)
+__device__ __forceinline__ float silu_fast(float y) {
+  float t, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(y * -1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + t));
+  return y * r;
+}
 
 // softplus(a) = log(1 + e^a), computed as max(a, 0) + log1p(e^{-|a|})
 __device__ __forceinline__ float softplus_f(float a) { return fmaxf(a, 0.0f) + log1pf(expf(-fabsf(a))); }

@@ -25,6 +25,7 @@
 //     U as bf16 hi/lo A operands read by tcgen05 straight from tensor memory.
 //     Per chunk five tcgen05 products (V^T B_U^T, S W^T, S Q^T, U_d^T K,
 //     U^T P^T) and the gated RMS-norm epilogue.
+#define GDN_WAIT_OUT_OF_LINE  // the prefill kernels' waits share one polling loop (gdn_ptx.cuh)
 #include <cuda.h>
 
 #include <algorithm>
@@ -301,7 +302,7 @@ __device__ __forceinline__ void solve_level(const float* sA, float* sT, float* s
     const float* arow = sA + (16 * I + ii) * kLdA + 16 * J;
     const float* tcol = sT + (16 * J) * kLdT + 16 * J + j4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+#pragma unroll 8
     for (int kk = 0; kk < 16 * d; ++kk) {
       const float a = arow[kk];
       const float4 t = *reinterpret_cast<const float4*>(tcol + kk * kLdT);
@@ -872,8 +873,9 @@ constexpr int kScOffG = kScOffO + 64 * kD * 4;         // 2 stages of gates
 constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 
 // The scan of one (sequence, value head) (`blk` = sequence rank * H_v + value head) by the
-// CTA's first 448 threads, with shared memory at sm (1024-aligned, kScSmem - 1024 bytes).
+// CTA's first 448 threads (kIssueUnroll: unrolling of the MMA issue loops), with shared memory at sm (1024-aligned, kScSmem - 1024 bytes).
 // CTA-wide steps use named barrier kScanBar.
+template <int kIssueUnroll>
 __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8_t* sm) {
   __shared__ uint64_t g_full[2], g_free[2];
   __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, bu_full, bu_free;
@@ -1066,7 +1068,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         if (!mbar_wait(&v_full, c & 1, ab)) break;
         if (!mbar_wait(&bu_full, c & 1, ab)) break;
         tc_fence_after();
-#pragma unroll
+#pragma unroll kIssueUnroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ah = smem_desc(v_hi + ks * 2048u, 8192, 1024, Swz::k128);
           const uint64_t al = smem_desc(v_lo + ks * 2048u, 8192, 1024, Swz::k128);
@@ -1081,7 +1083,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
         if (!mbar_wait(&w_full, c & 1, ab)) break;
         tc_fence_after();
-#pragma unroll
+#pragma unroll kIssueUnroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bw = smem_desc(w_lo + ks * 2048u, kImg64, 1024, Swz::k128);
           const uint64_t bw2 = smem_desc(w_hi + ks * 2048u, kImg64, 1024, Swz::k128);
@@ -1098,7 +1100,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tc_fence_after();
         bool s_issued = false;
         auto issue_update = [&]() {  // S += U_d^T K (onto gamma_C S)
-#pragma unroll
+#pragma unroll kIssueUnroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
             const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
@@ -1110,13 +1112,13 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
           umma_commit(&k_free);
           s_issued = true;
         };
-#pragma unroll
+#pragma unroll kIssueUnroll
         for (int kg = 0; kg < 4; ++kg) {
           if (!s_issued && mbar_test_wait(&u_conv, c & 1) && mbar_test_wait(&k_full, c & 1)) {
             tc_fence_after();
             issue_update();
           }
-#pragma unroll
+#pragma unroll kIssueUnroll
           for (int ks = 2 * kg; ks < 2 * kg + 2; ++ks) {
             const uint32_t ko = (ks >> 2) * 8192u + (ks & 3) * 32u;
             const uint64_t bh = smem_desc(q_hi + ko, 16, 1024, Swz::k128);
@@ -1137,7 +1139,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         if (!mbar_wait(&p_full, c & 1, ab)) break;
         tc_fence_after();
         // Y = U_hi P_hi + U_hi P_lo + U_lo P_hi
-#pragma unroll
+#pragma unroll kIssueUnroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t bh = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);
           const uint64_t bl = smem_desc(p_lo + ks * 32u, 16, 1024, Swz::k128);
@@ -1338,7 +1340,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(PrefillParams p) {
   if (p.cu && *p.ws_flag) return;
   extern __shared__ uint8_t scan_smem_raw[];
-  scan_body(p, blockIdx.x, align1024(scan_smem_raw));
+  scan_body<8>(p, blockIdx.x, align1024(scan_smem_raw));
 }
 
 // ------------------------------------------------------------ fused launch
@@ -1365,7 +1367,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) prefill_fused_kernel(Prefill
   extern __shared__ uint8_t fused_smem_raw[];
   uint8_t* sm = align1024(fused_smem_raw);
   if (static_cast<int>(blockIdx.x) < p.fused_scan_ctas) {
-    if (threadIdx.x < kScanThreads) scan_body(p, blockIdx.x, sm);
+    // the MMA issue loops unrolled by two only: this launch runs the prep's code on the other
+    // SMs, and the smaller scan code keeps the two from evicting each other's instructions
+    if (threadIdx.x < kScanThreads) scan_body<2>(p, blockIdx.x, sm);
     return;
   }
   // prep CTAs: each half is a worker that takes the next item (chunk-major) from a counter in

@@ -101,6 +101,29 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 // Bounded wait for phase `parity` of `bar`.  False on timeout or abort.
 // sleep_ns > 0 backs off between polls: for waits off the critical path, so that
 // the polling warp leaves issue slots to the warps it shares a sub-partition with.
+#ifdef GDN_WAIT_OUT_OF_LINE
+// (this translation unit: the first probe inline, the polling loop one out-of-line function
+// shared by every call site, which keeps large kernels' code small)
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const Abort& ab, bool cluster_scope,
+                                                   unsigned sleep_ns) {
+  long long t0 = clock64();
+  while (true) {
+    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (ab.raised()) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      ab.raise(kDevErrTimeout);
+      return false;
+    }
+    if (sleep_ns) __nanosleep(sleep_ns);
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
+                                          bool cluster_scope = false, unsigned sleep_ns = 0) {
+  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ab, cluster_scope, sleep_ns);
+}
+#else
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
                                           bool cluster_scope = false, unsigned sleep_ns = 0) {
   if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
@@ -115,6 +138,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (sleep_ns) __nanosleep(sleep_ns);
   }
 }
+#endif
 
 // Warp-collective bounded wait: every lane of the warp calls it and all get the
 // same answer, so a following warp-aligned instruction (tcgen05.ld/st) is

@@ -41,14 +41,14 @@ from gated_delta_rule_81_b200 import inputs as gin  # noqa: E402
 METRIC = "gated-delta prefill tokens/s per layer; decode state GB/s vs B200 HBM peak"
 
 # Algorithmic work per token of a chunk-64 prefill with d = 128 (16 key / 48 value heads):
-#   prep kernel: [Q;K]K^T per key head (4 C d) and the two T-products per value head (4 C d)
-#   scan kernel: W S^T, Q S^T, U^T K per value head (6 d^2) and P U (2 C d)
+#   prep kernel: [Q;K]K^T per key head (4 C d) and W = B_W K per value head (2 C d)
+#   scan kernel: W S^T, Q S^T, U^T K per value head (6 d^2), U0 = B_U V and P U (4 C d)
 def prep_flop_per_token(H_k=16, H_v=48, C=64, d=128):
-    return H_k * 4 * C * d + H_v * 4 * C * d          # 2,097,152 at 16/48 heads
+    return H_k * 4 * C * d + H_v * 2 * C * d          # 1,310,720 at 16/48 heads
 
 
 def scan_flop_per_token(H_v=48, C=64, d=128):
-    return H_v * (6 * d * d + 2 * C * d)              # 5,505,024 at 48 value heads
+    return H_v * (6 * d * d + 4 * C * d)              # 6,291,456 at 48 value heads
 
 
 PREP_FLOP_PER_TOKEN = prep_flop_per_token()

@@ -181,7 +181,7 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.chunk_base = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) : nullptr;
   p.seq_order = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) + (N + 1) : nullptr;
   p.ws_k = ws + gdn::kWsHeader + chunk_base_bytes(N);
-  p.ws_head = p.ws_k + static_cast<size_t>(n_chunks) * in->H_k * gdn::kKQBytes;
+  p.ws_head = p.ws_k + static_cast<size_t>(n_chunks) * in->H_k * gdn::kKBytes;
   p.state_in = state_in;
   p.state_out = state_out;
   p.conv_in = static_cast<const bf16*>(conv_in);
@@ -200,7 +200,7 @@ extern "C" {
 size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks) {
   if (H_k <= 0 || H_v <= 0 || N < 0 || n_chunks < 0) return 0;
   return gdn::kWsHeader + chunk_base_bytes(N) +
-         static_cast<size_t>(n_chunks) * (static_cast<size_t>(H_k) * gdn::kKQBytes +
+         static_cast<size_t>(n_chunks) * (static_cast<size_t>(H_k) * gdn::kKBytes +
                                           static_cast<size_t>(H_v) * gdn::kHeadBytes);
 }
 

@@ -11,13 +11,13 @@ using bf16 = __nv_bfloat16;
 // Every tensor-core operand is stored as a bf16 pair (hi = bf16(x), lo =
 // bf16(x - hi)) so that products keep ~16 significant bits.  Operand images use
 // the 128-byte swizzled layout (rows of 64 bf16 = 128 B, 8-row groups of 1 KiB).
-//   per (chunk, key head), kKQBytes:
-//     K hi | K lo | Q hi | Q lo: 64 tokens x 128 channels each, as two 8 KiB blocks of
-//     64 channels (row = token).  The scan reads K as an MN-major operand (N = channels)
-//     and Q as a K-major one (N = tokens, K = channels).
+//   per (chunk, key head), kKBytes:
+//     K hi | K lo: 64 tokens x 128 channels each, as two 8 KiB blocks of 64 channels
+//     (row = token), read by the scan as an MN-major operand (N = channels).
 //   per (chunk, value head), kHeadBytes:
-//     -W^T lo | -W^T hi: two 16 KiB images of 128 rows (d_k) x 64 tokens,
-//       W = T diag(beta gamma) K, negated; side by side one MN-major operand of N = 128
+//     -W^T lo | -W^T hi | (gamma Q)^T hi | (gamma Q)^T lo: four 16 KiB images of 128 rows
+//       (d_k) x 64 tokens, W = T diag(beta gamma) K (negated) and gamma Q = diag(gamma) Q;
+//       side by side one MN-major operand of N = 256 (or, from the second, N = 128)
 //     P hi | P lo: P_ij = e^{G_i - G_j} q_i.k_j for j <= i, row = i, 64 j per row
 //     B_U lo | B_U hi: B_U = T diag(beta), row = i, 64 j per row (K-major); side by side
 //       one operand of N = 128
@@ -25,19 +25,18 @@ using bf16 = __nv_bfloat16;
 //       two 8 KiB blocks of 64 channels each (read by the scan as an MN-major operand, M = d_v)
 //     gates fp32: gamma_i [64], e^{G_C - G_i} [64], gamma_C
 constexpr int kImg64 = 16384;                                // 64 rows x 128 channels (or 128 x 64), bf16
-constexpr int kKQOffK = 0;                                   // K hi, K lo
-constexpr int kKQOffQ = 2 * kImg64;                          // Q hi, Q lo
-constexpr int kKQBytes = 4 * kImg64;
+constexpr int kKBytes = 2 * kImg64;                          // K hi, K lo
 constexpr int kHeadOffW = 0;                                 // -W^T lo, -W^T hi
 constexpr int kWBytes = 2 * kImg64;
+constexpr int kHeadOffGQ = kHeadOffW + kWBytes;              // (gamma Q)^T hi, lo
 constexpr int kPImg = 8192;                                  // one 64 x 64 bf16 image
-constexpr int kHeadOffP = kHeadOffW + kWBytes;               // P hi, lo
+constexpr int kHeadOffP = kHeadOffGQ + 2 * kImg64;           // P hi, lo
 constexpr int kHeadOffBU = kHeadOffP + 2 * kPImg;            // B_U lo, hi
 constexpr int kHeadOffV = kHeadOffBU + 2 * kPImg;            // v_hat hi, lo
 constexpr int kHeadOffGate = kHeadOffV + 2 * kImg64;
 constexpr int kGateBytes = 1024;
 constexpr int kReadyFlagWord = 255;  // word of the gate area a fused prefill launch uses as a ready flag
-constexpr int kHeadBytes = kHeadOffGate + kGateBytes;        // 99328
+constexpr int kHeadBytes = kHeadOffGate + kGateBytes;        // 132096
 constexpr int kWsHeader = 1024;                              // error/consistency word
 
 constexpr int kMaxDecodeTokens = 8;   // new tokens per sequence in one decode call
@@ -76,7 +75,7 @@ struct PrefillParams {
   int* chunk_base;        // [N+1] in the workspace (varlen), or null (uniform)
   int* seq_order;         // [N] scan order, longest first (varlen), or null
   int* ws_flag;           // workspace header word: nonzero = inconsistent cu_seqlens
-  uint8_t* ws_k;          // [n_chunks][H_k][kKQBytes]
+  uint8_t* ws_k;          // [n_chunks][H_k][kKBytes]
   uint8_t* ws_head;       // [n_chunks][H_v][kHeadBytes]
   const float* state_in;  // [N][H_v][128][128] or null (zeros)
   float* state_out;       // [N][H_v][128][128] or null

@@ -177,15 +177,15 @@ constexpr int kLdT = 68;                               // fp32 row stride of T (
 // 64 kb .. 64 kb + 63) at kb * 16384, rows 0..63 = Q tokens, rows 64..127 = K tokens.
 // The K rows are the workspace's K image (four 8 KiB pieces, bulk-stored from here).
 constexpr int kPrepOffQK = 0;
-// The Q rows are the workspace's Q image too.  Once the product that reads Q has completed
-// and the Q image has left for the workspace, the four 8 KiB Q pieces are scratch: per
+// Once the products that read Q have completed, the four 8 KiB Q pieces are scratch: per
 // value head they stage P (hi, lo), then hold the B image B_W = T diag(beta gamma) (hi at 0,
 // lo at 32768), then stage -W^T (lo rows 0..63, 64..127, hi rows 0..63, 64..127).
 constexpr int kPrepOffBWhi = 0, kPrepOffBWlo = 32768;
 // Region R (37 KiB) changes role through the kernel:
 //   the raw q | k rows of the chunk (front-end input, rows of kRawStride bytes);
+//   the identity B image of the q^T transpose;
 //   per value head: T, A and the block-solve temp; then B_U = T diag(beta) (lo, hi) over
-//   the dead A, staged for the workspace.
+//   the dead A, staged for the workspace; then the staged (gamma Q)^T images (hi, lo).
 constexpr int kPrepOffR = 65536;
 constexpr int kRawStride = 2 * kD * 2 + 16;            // q row | k row, 16 B of padding against bank conflicts
 constexpr int kPrepOffT = kPrepOffR;                   // T fp32                64*68*4
@@ -202,8 +202,10 @@ static_assert((kChunk + kTaps - 1) * (kVBatch * kD * 2 + 16) <= 65536, "the stag
 constexpr int kPrepSmem = kPrepOffW + 2 * 128 * 8 + 1024;
 static_assert((kChunk + kTaps - 1) * kRawStride <= kPrepRBytes, "the raw q | k rows must fit region R");
 static_assert(kPrepOffBU % 1024 == 0 && 2 * kPImg <= 64 * kLdA * 4, "B_U must fit the A area");
+static_assert(2 * kImg64 <= kPrepRBytes, "the (gamma Q)^T images must fit region R");
 // tensor memory columns (256 per CTA, two CTAs per SM)
 constexpr uint32_t kPrepColQK = 0;    // [Q;K] K^T: rows 0..63 Q K^T, rows 64..127 K K^T (64 columns)
+constexpr uint32_t kPrepColQT = 64;   // q^T (lane = d_k, column = token)
 constexpr uint32_t kPrepColW = 128;   // W^T (lane = d_k, column = token)
 
 // W words of bf16 pairs from 2W fp32 values: hi[m] = (bf16(x[2m]), bf16(x[2m+1])) with
@@ -397,9 +399,9 @@ __device__ __forceinline__ int* ready_flag(const PrefillParams& p, long long gc,
 // `k` counts the items these threads ran before with the same mbarriers (initialised at k = 0;
 // every wait takes its phase parity from k).  When go_flag is given, it is set once the first
 // value head is done (or the item ends), which lets the other half of a CTA start out of phase.
-// Writes the chunk's K and Q images for the key head and, for each of its value heads,
-// -W^T, P, B_U, v_hat and the gate vectors; the operand images leave shared memory as bulk
-// stores (v_hat goes straight from registers).  In a fused launch it then publishes the chunk through the value heads' ready flags.
+// Writes the chunk's K image for the key head and, for each of its value heads, -W^T,
+// (gamma Q)^T, P, B_U, v_hat and the gate vectors; the operand images leave shared memory as
+// bulk stores (v_hat goes straight from registers).  In a fused launch it then publishes the chunk through the value heads' ready flags.
 __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, int kh, int half, uint8_t* sm,
                                           uint32_t tbase, uint64_t* bar, int* abort_s, int k, int* go_flag) {
   const int bar_id = 2 + half;
@@ -412,7 +414,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   float* sB = reinterpret_cast<float*>(sm + kPrepOffB);
   float* sGam = reinterpret_cast<float*>(sm + kPrepOffGam);
   uint4* sW = reinterpret_cast<uint4*>(sm + kPrepOffW);  // [2 * 64] channel pairs: q | k
-  // bar: [Q;K] K^T, W (per head), drain
+  // bar: [Q;K] K^T, W (per head), drain, q^T
 
   const int tid = threadIdx.x & (kPrepThreads - 1), warp = tid >> 5, lane = tid & 31;
   const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k;
@@ -607,15 +609,13 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   named_bar_sync(bar_id, kPrepThreads);
   tc_fence_after();
 
-  // ---- the K and Q images to the workspace (the K rows, then the Q rows, of the four
-  // K-block halves), and [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
+  // ---- the K image to the workspace (the K rows of the four K-block halves), and
+  // [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
   if (tid == 0) {
-    uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKQBytes);
+    uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
 #pragma unroll
-    for (int piece = 0; piece < 4; ++piece) {  // hi block 0, hi block 1, lo block 0, lo block 1
-      bulk_s2g(gK + kKQOffK + piece * 8192, sQK + piece * 16384 + 8192, 8192);
-      bulk_s2g(gK + kKQOffQ + piece * 8192, sQK + piece * 16384, 8192);
-    }
+    for (int piece = 0; piece < 4; ++piece)  // hi block 0, hi block 1, lo block 0, lo block 1
+      bulk_s2g(gK + piece * 8192, sQK + piece * 16384 + 8192, 8192);
     bulk_commit();
     const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
     const uint32_t idesc = idesc_bf16(128, 64, false, false);
@@ -644,6 +644,17 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     if (k2 != kReadyFlagWord) gdst[k2] = val;
   }
 
+  // identity B image for the q^T transpose, in region R (the raw rows are dead)
+  for (int x = tid; x < 64 * 8; x += kPrepThreads) {
+    const int i = x >> 3, cc = x & 7;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (cc == (i >> 3)) {
+      const int e8 = i & 7;
+      w[e8 >> 1] = (e8 & 1) ? 0x3F800000u : 0x00003F80u;  // bf16 1.0 in the element's half
+    }
+    *reinterpret_cast<uint4*>(sR + sw128_off(i, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+
   // ---- K K^T and Q K^T rows into registers: thread row = 32*(warp%4)+lane, columns cbase..cbase+31
   const int row = 32 * (warp & 3) + lane;
   const int cbase = 32 * (warp >> 2);
@@ -651,9 +662,29 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   const int ri = row & 63;
   // (the [Q;K] K^T rows stay in tensor memory and are read again for each value head)
   const bool qk_ok = mbar_wait_warp(&bar[0], ph, ab);
+
+  // ---- q^T (lane = d_k, column = token) into TMEM columns 64..127: Q_hi^T I + Q_lo^T I
+  // with an identity B, exact in fp32
+  fence_proxy_async_smem();
+  tc_fence_before();
+  named_bar_sync(bar_id, kPrepThreads);  // the identity is complete
   tc_fence_after();
-  if (tid == 0) bulk_wait_read<0>();  // the K and Q images have left shared memory
-  named_bar_sync(bar_id, kPrepThreads);  // Q is dead: the Q pieces and region R are scratch from here
+  if (tid == 0) {
+    const uint32_t qk = smem_u32(sQK), id = smem_u32(sR);
+    const uint32_t idesc_t = idesc_bf16(128, 64, true, false);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint64_t b = smem_desc(id + ks * 32u, 16, 1024, Swz::k128);
+      umma_bf16(tbase + kPrepColQT, smem_desc(qk + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, ks > 0);
+      umma_bf16(tbase + kPrepColQT, smem_desc(qk + 32768u + ks * 2048u, 16384, 1024, Swz::k128), b, idesc_t, true);
+    }
+    umma_commit(&bar[3]);
+  }
+  __syncwarp();
+  mbar_wait_warp(&bar[3], ph, ab);
+  tc_fence_after();
+  if (tid == 0) bulk_wait_read<0>();  // the K image has left shared memory
+  named_bar_sync(bar_id, kPrepThreads);  // Q and the identity are dead: the Q pieces and region R are scratch
 
   for (int j = 0; j < G; ++j) {
     const int h = kh * G + j;
@@ -731,6 +762,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     if (tid == 0) {
       bulk_s2g(hb + kHeadOffBU, sBU, 2 * kPImg);
       bulk_commit();
+      bulk_wait_read<0>();  // B_U has left region R before the product's completion frees it
       // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
       const uint32_t qk = smem_u32(sQK);
       const uint32_t idesc_w = idesc_bf16(128, 64, true, false);
@@ -763,19 +795,36 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
         *reinterpret_cast<uint4*>(sQK + half_off + off) = lo;
         *reinterpret_cast<uint4*>(sQK + 32768 + half_off + off) = hi;
       }
+      // (gamma Q)^T row d_k = kr, the same 32 tokens: staged in region R, hi rows 0..63 | 64..127
+      // then lo rows 0..63 | 64..127
+      tmem_ld32(tmem_addr(tbase, 32 * (warp & 3), kPrepColQT + 32 * half), o);
+      tmem_wait_ld();
+      const uint32_t rhalf = kr < 64 ? 0u : 8192u;
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float f[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) f[e2] = o[8 * c2 + e2] * sGam[j * 64 + 32 * half + 8 * c2 + e2];
+        uint4 hi, lo;
+        split8(f, hi, lo);
+        const uint32_t off = rhalf + sw128_off(kr & 63, 4 * half + c2);
+        *reinterpret_cast<uint4*>(sR + off) = hi;
+        *reinterpret_cast<uint4*>(sR + kImg64 + off) = lo;
+      }
       fence_proxy_async_smem();
     }
     tc_fence_before();
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
-      uint8_t* wd = hb + kHeadOffW;  // -W^T lo | -W^T hi
+      uint8_t* wd = hb + kHeadOffW;  // -W^T lo | -W^T hi | (gamma Q)^T hi | (gamma Q)^T lo
       bulk_s2g(wd, sQK, 8192);
       bulk_s2g(wd + 8192, sQK + 16384, 8192);
       bulk_s2g(wd + 16384, sQK + 32768, 8192);
       bulk_s2g(wd + 24576, sQK + 49152, 8192);
+      bulk_s2g(hb + kHeadOffGQ, sR, 2 * kImg64);
       bulk_commit();
-      bulk_wait_read<0>();  // the staging areas (Q pieces, B_U) are rewritten by the next value head
+      bulk_wait_read<0>();  // the staging areas (Q pieces, region R) are rewritten by the next value head
     }
     named_bar_sync(bar_id, kPrepThreads);
     if (go_flag && tid == 0) *reinterpret_cast<volatile int*>(go_flag) = 1;
@@ -826,19 +875,17 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // One CTA per (sequence, value head); the whole 128 x 128 state lives in tensor
 // memory with lane = d_v row.  Per chunk, every product summed over the hi/lo
 // split terms (hi.hi + hi.lo + lo.hi):
-//   U^T = V^T B_U^T + S (-W)^T          (A = v_hat from shared memory, then S hi/lo from TMEM)
-//   X   = S Q^T                         (the state's part of o, before the decay gamma_i)
+//   [U^T | O^T]  = V^T [B_U^T | 0] + S [-W^T | (gamma Q)^T]   (U0 from shared-memory operands
+//                  first, off the chain; then one product of N = 256 for both halves)
 //   S   = gamma_C S + (U^T diag(e^{G_C - G_j})) K   (A = U_d hi/lo from TMEM)
-//   Y   = U^T P^T                       (A = U hi/lo from TMEM)
-//   o_i = gamma_i X_i + Y_i, then the gated RMS-norm of o_i over d_v.
-// V^T B_U^T (the state-independent part of U, U0) is accumulated first, off the chain:
-// once the previous chunk's products have read the U columns and before S is converted.
+//   O^T += U^T P^T                      (A = U hi/lo from TMEM)
+//   then the gated RMS-norm of o_i over d_v.
 // Warps 0-7 (thread = d_v row; warps w and w + 4 share a TMEM lane quarter and
 // split its columns) convert S and U between fp32 accumulators and bf16 hi/lo
 // operands in tensor memory, each conversion publishing first the part the next
-// product waits for; warps 8-11 run the output stage; warp 12 lane 0 issues the
-// MMAs; warp 13 lane 0 issues the bulk copies (v_hat, B_U, W, Q, K, P single-buffered,
-// gates double-buffered).
+// product waits for; warps 8-11 run the output stage (and clear O for the next chunk's
+// accumulation); warp 12 lane 0 issues the MMAs; warp 13 lane 0 issues the bulk copies
+// (v_hat, B_U, W | gamma Q, K, P single-buffered, gates double-buffered).
 
 constexpr int kScanThreads = 448;
 constexpr int kScanBar = 15;  // named barrier of the scan's CTA-wide steps
@@ -847,11 +894,12 @@ constexpr int kWarpIssue = 12, kWarpProd = 13;
 constexpr uint32_t kColS = 0;      // S fp32, 128 columns (d_k)
 constexpr uint32_t kColSH = 128;   // S hi, bf16 pairs along d_k (64 columns)
 constexpr uint32_t kColSL = 192;   // S lo
-// [V_hi B_U_lo - S_hi W_lo | V_hi B_U_hi + V_lo B_U_hi - S_hi W_hi - S_lo W_hi], 2 x 64 columns
+// [U2 | U1 | O1 | O2], 4 x 64 columns:
+//   U2 = V_hi B_U_lo - S_hi W_lo,  U1 = V_hi B_U_hi + V_lo B_U_hi - S_hi W_hi - S_lo W_hi,
+//   O1 = S_hi gQ_hi + S_lo gQ_hi + U_hi P_hi + U_lo P_hi,  O2 = S_hi gQ_lo + U_hi P_lo
 constexpr uint32_t kColU2 = 256;   //   U^T = U2 + U1
 constexpr uint32_t kColU1 = 320;
-constexpr uint32_t kColX = 384;    // X = S Q^T (64 columns)
-constexpr uint32_t kColY = 448;    // Y = U^T P^T (64 columns)
+constexpr uint32_t kColO = 384;    //   o = O1 + O2
 // After the U conversion, in place: the chain warp of token half th (tokens 32 th .. +31)
 // read U2 / U1 columns 256 + 32 th / 320 + 32 th and writes there, 16 columns each,
 //   U hi at 256 + 32 th, U lo at 272 + 32 th, U_d hi at 320 + 32 th, U_d lo at 336 + 32 th,
@@ -862,9 +910,8 @@ constexpr uint32_t kColUDH = 320;
 constexpr uint32_t kColUDL = 336;
 __host__ __device__ constexpr uint32_t ucol(uint32_t base, int ks) { return base + 32u * (ks >> 1) + 8u * (ks & 1); }
 // shared memory (offsets from a 1024-aligned base)
-constexpr int kScOffW = 0;                             // -W^T lo | -W^T hi
-constexpr int kScOffQ = kScOffW + kWBytes;             // Q hi | Q lo
-constexpr int kScOffK = kScOffQ + 2 * kImg64;          // K hi | K lo
+constexpr int kScOffW = 0;                             // -W^T lo | -W^T hi | (gQ)^T hi | (gQ)^T lo
+constexpr int kScOffK = kScOffW + 2 * kWBytes;         // K hi | K lo
 constexpr int kScOffP = kScOffK + 2 * kImg64;          // P hi | P lo
 constexpr int kScOffBU = kScOffP + 2 * kPImg;          // B_U lo | B_U hi
 constexpr int kScOffV = kScOffBU + 2 * kPImg;          // v_hat hi | lo (MN-major: row = token, two 64-channel blocks)
@@ -878,7 +925,7 @@ constexpr int kScSmem = kScOffG + 2 * kGateBytes + 1024;
 template <int kIssueUnroll>
 __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8_t* sm) {
   __shared__ uint64_t g_full[2], g_free[2];
-  __shared__ uint64_t w_full, w_free, q_full, q_free, k_full, k_free, p_full, p_free, bu_full, bu_free;
+  __shared__ uint64_t w_full, w_free, k_full, k_free, p_full, p_free, bu_full, bu_free;
   __shared__ uint64_t v_full, v_free;
   __shared__ uint64_t s_conv, u_conv, u_conv2, u_done, s_done, y_done, o_free, drain_b;
   __shared__ uint32_t tmem_base_s;
@@ -897,12 +944,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     abort_s = 0;
     for (int b = 0; b < 2; ++b) {
       mbar_init(&g_full[b], 1);
-      mbar_init(&g_free[b], 256 + 128);  // the conversion and output warps
+      mbar_init(&g_free[b], 256);
     }
     mbar_init(&w_full, 1);
     mbar_init(&w_free, 1);
-    mbar_init(&q_full, 1);
-    mbar_init(&q_free, 1);
     mbar_init(&k_full, 1);
     mbar_init(&k_free, 1);
     mbar_init(&p_full, 1);
@@ -960,10 +1005,6 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         tmem_ld32(tl + kColS + 64 * th + 32, sv + 32);
         tmem_wait_ld();
       }
-      // the previous chunk's X = S Q^T (issued around the state update) still reads S hi/lo
-      if (c > 0) ok = mbar_wait_warp(&q_free, (c - 1) & 1, ab);
-      if (!ok) break;
-      tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t hi[16], lo[16];
@@ -1008,7 +1049,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         ud[i] = r.x;
         ud[i + 1] = r.y;
       }
-      mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time by this warp
+      mbar_arrive(&g_free[gs]);  // the chunk's gates have been read for the last time
       {
         uint32_t hi[16], lo[16];
         split_pairs_x2<16>(ud, hi, lo);
@@ -1050,15 +1091,14 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     if (lane == 0) {
       const uint32_t idesc_v = idesc_bf16(128, 128, true, false);   // v_hi^T [B_U lo | B_U hi] (A MN-major)
       const uint32_t idesc_v2 = idesc_bf16(128, 64, true, false);   // v_lo^T B_U hi
-      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [-W_lo | -W_hi] (B MN-major)
-      const uint32_t idesc_u2 = idesc_bf16(128, 64, false, true);   // S_lo (-W_hi)
-      const uint32_t idesc_x = idesc_bf16(128, 64, false, false);   // S Q^T (Q K-major: N = tokens)
+      const uint32_t idesc_u = idesc_bf16(128, 256, false, true);   // S_hi [-W_lo | -W_hi | gQ_hi | gQ_lo] (B MN-major)
+      const uint32_t idesc_u2 = idesc_bf16(128, 128, false, true);  // S_lo [-W_hi | gQ_hi]
       const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
-      const uint32_t idesc_y = idesc_bf16(128, 64, false, false);   // U P^T (K-major)
-      const uint32_t w_lo = smem_u32(sm + kScOffW), w_hi = w_lo + kImg64;
-      const uint32_t q_hi = smem_u32(sm + kScOffQ), q_lo = q_hi + kImg64;
+      const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
+      const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
+      const uint32_t wq = smem_u32(sm + kScOffW);
       const uint32_t k_hi = smem_u32(sm + kScOffK), k_lo = k_hi + kImg64;
-      const uint32_t p_hi = smem_u32(sm + kScOffP), p_lo = p_hi + kPImg;
+      const uint32_t p_hi = smem_u32(sm + kScOffP);
       const uint32_t bu_lo = smem_u32(sm + kScOffBU), bu_hi = bu_lo + kPImg;
       const uint32_t v_hi = smem_u32(sm + kScOffV), v_lo = v_hi + kImg64;
       for (int c = 0; c < nc; ++c) {
@@ -1079,73 +1119,45 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         }
         umma_commit(&v_free);
         umma_commit(&bu_free);
-        // the chain's product: [U2 | U1] += S_hi [-W_lo | -W_hi], U1 += S_lo (-W_hi)
+        // the chain's product and the state's part of o together, onto U0 and onto the O that
+        // the output warps cleared: [U2 | U1 | O1 | O2] += S_hi [-W_lo | -W_hi | gQ_hi | gQ_lo],
+        // [U1 | O1] += S_lo [-W_hi | gQ_hi]
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
         if (!mbar_wait(&w_full, c & 1, ab)) break;
+        if (!mbar_wait(&o_free, c & 1, ab)) break;
         tc_fence_after();
 #pragma unroll kIssueUnroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bw = smem_desc(w_lo + ks * 2048u, kImg64, 1024, Swz::k128);
-          const uint64_t bw2 = smem_desc(w_hi + ks * 2048u, kImg64, 1024, Swz::k128);
+          const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
+          const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
           umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, true);
           umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
         }
         umma_commit(&u_done);
         umma_commit(&w_free);
-        // X = S Q^T, once x(c-1) and y(c-1) have been read, in groups of two K steps; the state
-        // update (the chain's next product) goes out between two groups as soon as U_d and K
-        // are in place
-        if (!mbar_wait(&q_full, c & 1, ab)) break;
-        if (c > 0 && !mbar_wait(&o_free, (c - 1) & 1, ab)) break;
+        if (!mbar_wait(&u_conv, c & 1, ab)) break;
+        if (!mbar_wait(&k_full, c & 1, ab)) break;
         tc_fence_after();
-        bool s_issued = false;
-        auto issue_update = [&]() {  // S += U_d^T K (onto gamma_C S)
+        // S += U_d^T K (onto gamma_C S)
 #pragma unroll kIssueUnroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
-            const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
-            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
-            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
-            umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
-          }
-          umma_commit(&s_done);
-          umma_commit(&k_free);
-          s_issued = true;
-        };
-#pragma unroll kIssueUnroll
-        for (int kg = 0; kg < 4; ++kg) {
-          if (!s_issued && mbar_test_wait(&u_conv, c & 1) && mbar_test_wait(&k_full, c & 1)) {
-            tc_fence_after();
-            issue_update();
-          }
-#pragma unroll kIssueUnroll
-          for (int ks = 2 * kg; ks < 2 * kg + 2; ++ks) {
-            const uint32_t ko = (ks >> 2) * 8192u + (ks & 3) * 32u;
-            const uint64_t bh = smem_desc(q_hi + ko, 16, 1024, Swz::k128);
-            const uint64_t bl = smem_desc(q_lo + ko, 16, 1024, Swz::k128);
-            umma_bf16_ts(tbase + kColX, tbase + kColSH + 8 * ks, bh, idesc_x, ks > 0);
-            umma_bf16_ts(tbase + kColX, tbase + kColSH + 8 * ks, bl, idesc_x, true);
-            umma_bf16_ts(tbase + kColX, tbase + kColSL + 8 * ks, bh, idesc_x, true);
-          }
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bh = smem_desc(k_hi + ks * 2048u, 8192, 1024, Swz::k128);
+          const uint64_t bl = smem_desc(k_lo + ks * 2048u, 8192, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bh, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDH, ks), bl, idesc_s, true);
+          umma_bf16_ts(tbase + kColS, tbase + ucol(kColUDL, ks), bh, idesc_s, true);
         }
-        umma_commit(&q_free);
-        if (!s_issued) {
-          if (!mbar_wait(&u_conv, c & 1, ab)) break;
-          if (!mbar_wait(&k_full, c & 1, ab)) break;
-          tc_fence_after();
-          issue_update();
-        }
+        umma_commit(&s_done);
+        umma_commit(&k_free);
         if (!mbar_wait(&u_conv2, c & 1, ab)) break;
         if (!mbar_wait(&p_full, c & 1, ab)) break;
         tc_fence_after();
-        // Y = U_hi P_hi + U_hi P_lo + U_lo P_hi
+        // [O1 | O2] += U_hi [P_hi | P_lo], O1 += U_lo P_hi
 #pragma unroll kIssueUnroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bh = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);
-          const uint64_t bl = smem_desc(p_lo + ks * 32u, 16, 1024, Swz::k128);
-          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUH, ks), bh, idesc_y, ks > 0);
-          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUH, ks), bl, idesc_y, true);
-          umma_bf16_ts(tbase + kColY, tbase + ucol(kColUL, ks), bh, idesc_y, true);
+          const uint64_t b2 = smem_desc(p_hi + ks * 32u, 16, 1024, Swz::k128);  // 128 rows: P hi then P lo
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUH, ks), b2, idesc_y, true);
+          umma_bf16_ts(tbase + kColO, tbase + ucol(kColUL, ks), b2, idesc_y2, true);
         }
         umma_commit(&y_done);
         umma_commit(&p_free);
@@ -1160,9 +1172,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
   } else if (warp == kWarpProd) {
     // ------------------------------------------------ bulk-copy producer (lane 0)
     if (lane == 0) {
-      // Order of need: v_hat, B_U, W, Q, K, P of chunk c (single stages, each refilled as soon
-      // as the product that reads it has completed), then the double-buffered gates of chunk c + 1.
-      int n_g[2] = {0, 0}, n_v = 0, n_bu = 0, n_w = 0, n_q = 0, n_k = 0, n_p = 0;
+      // Order of need: v_hat, B_U, W | gamma Q, K, P of chunk c (single stages, each refilled as
+      // soon as the product that reads it has completed), then the double-buffered gates of
+      // chunk c + 1.
+      int n_g[2] = {0, 0}, n_v = 0, n_bu = 0, n_w = 0, n_k = 0, n_p = 0;
       auto head_blob = [&](int c) {
         return p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes);
       };
@@ -1179,7 +1192,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       bool ok = nc == 0 || load_gates(0);
       for (int c = 0; c < nc && ok; ++c) {
         const uint8_t* hb = head_blob(c);
-        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKQBytes);
+        const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes);
         if (c >= 1 && !mbar_wait(&v_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&v_full, 2 * kImg64);
         bulk_g2s(sm + kScOffV, hb + kHeadOffV, 2 * kImg64, &v_full);
@@ -1189,16 +1202,12 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         bulk_g2s(sm + kScOffBU, hb + kHeadOffBU, 2 * kPImg, &bu_full);
         ++n_bu;
         if (c >= 1 && !mbar_wait(&w_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&w_full, kWBytes);
-        bulk_g2s(sm + kScOffW, hb + kHeadOffW, kWBytes, &w_full);
+        mbar_arrive_expect_tx(&w_full, 2 * kWBytes);
+        bulk_g2s(sm + kScOffW, hb + kHeadOffW, 2 * kWBytes, &w_full);  // W and gamma Q side by side
         ++n_w;
-        if (c >= 1 && !mbar_wait(&q_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&q_full, 2 * kImg64);
-        bulk_g2s(sm + kScOffQ, kb + kKQOffQ, 2 * kImg64, &q_full);
-        ++n_q;
         if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&k_full, 2 * kImg64);
-        bulk_g2s(sm + kScOffK, kb + kKQOffK, 2 * kImg64, &k_full);
+        mbar_arrive_expect_tx(&k_full, kKBytes);
+        bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
         ++n_k;
         if (c >= 1 && !mbar_wait(&p_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
         mbar_arrive_expect_tx(&p_full, 2 * kPImg);
@@ -1207,7 +1216,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         if (c + 1 < nc) ok = load_gates(c + 1);
         if (c + 2 < nc) {  // two chunks ahead into L2, behind this chunk's copies
           prefetch_l2(hb + 2LL * p.H_v * kHeadBytes, kHeadBytes);
-          prefetch_l2(kb + 2LL * p.H_k * kKQBytes, kKQBytes);
+          prefetch_l2(kb + 2LL * p.H_k * kKBytes, kKBytes);
         }
       }
       // copies still in flight (only possible after an abort) land before the CTA exits
@@ -1218,17 +1227,17 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       if (n_v > 0) mbar_wait(&v_full, (n_v - 1) & 1, drain);
       if (n_bu > 0) mbar_wait(&bu_full, (n_bu - 1) & 1, drain);
       if (n_w > 0) mbar_wait(&w_full, (n_w - 1) & 1, drain);
-      if (n_q > 0) mbar_wait(&q_full, (n_q - 1) & 1, drain);
       if (n_k > 0) mbar_wait(&k_full, (n_k - 1) & 1, drain);
       if (n_p > 0) mbar_wait(&p_full, (n_p - 1) & 1, drain);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------ output stage (warps 8-11)
-    // o = gamma X + Y leaves tensor memory row-wise (thread = d_v row) into shared memory as
-    // fp32 [token][d_v]; then each thread owns 8 consecutive d_v of a token, 16 threads per
-    // token: the sum of o^2 over d_v is a 4-step shuffle inside that group (a fixed
-    // order), z is read and out written with 16-byte accesses.
+    // o = O1 + O2 leaves tensor memory row-wise (thread = d_v row) into shared memory as
+    // fp32 [token][d_v], and O is cleared for the next chunk's accumulation; then each thread
+    // owns 8 consecutive d_v of a token, 16 threads per token: the sum of o^2 over d_v is a
+    // 4-step shuffle inside that group (a fixed order), z is read and out written with
+    // 16-byte accesses.
     const int ow = warp & 3;              // TMEM lane quarter
     const int v = 32 * ow + lane;
     const int otid = tid - 256;           // 0..127 within the output group
@@ -1238,11 +1247,19 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     float w8[8];  // norm_w is only 2-byte aligned: element loads
 #pragma unroll
     for (int e2 = 0; e2 < 8; ++e2) w8[e2] = __bfloat162float(p.norm_w[v8 + e2]);
+    {  // O starts cleared: the first chunk's product accumulates onto it
+      float zero[32];
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) zero[e2] = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_st32(tl + kColO + 32 * cc, zero);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&o_free);
+    }
     // Every output warp reaches every named barrier; a failed wait is OR-ed into the
     // first barrier so that the four warps leave the loop together.
     for (int c = 0; c < nc; ++c) {
-      const int gs = c & 1;
-      const float* gam = reinterpret_cast<const float*>(sm + kScOffG + gs * kGateBytes);
       const long long tok0 = s + static_cast<long long>(c) * kChunk;
       const int L = static_cast<int>(min(static_cast<long long>(kChunk), e - tok0));
       // z of the next chunk into L2 (one 128-byte line per thread), z of this chunk into
@@ -1259,26 +1276,29 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
                       : make_uint4(0u, 0u, 0u, 0u);
       }
       bool ok = mbar_wait_warp(&y_done, c & 1, ab, false, kBackoffNs);
-      if (ok) ok = mbar_wait_warp(&g_full[gs], (c >> 1) & 1, ab);  // (complete: the chain read these gates)
       if (ok) {
         tc_fence_after();
+        float zero[32];
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) zero[e2] = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          float xv[32], yv[32];
-          tmem_ld32(tl + kColX + 32 * cc, xv);
-          tmem_ld32(tl + kColY + 32 * cc, yv);
+          float o1[32], o2[32];
+          tmem_ld32(tl + kColO + 32 * cc, o1);
+          tmem_ld32(tl + kColO + 64 + 32 * cc, o2);
           tmem_wait_ld();
+          tmem_st32(tl + kColO + 32 * cc, zero);
+          tmem_st32(tl + kColO + 64 + 32 * cc, zero);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float2 g2 = *reinterpret_cast<const float2*>(gam + 32 * cc + i);
-            const float2 r = __ffma2_rn(make_float2(xv[i], xv[i + 1]), g2, make_float2(yv[i], yv[i + 1]));
+            const float2 r = __fadd2_rn(make_float2(o1[i], o1[i + 1]), make_float2(o2[i], o2[i + 1]));
             sO[(32 * cc + i) * kD + v] = r.x;
             sO[(32 * cc + i + 1) * kD + v] = r.y;
           }
         }
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&o_free);
-        mbar_arrive(&g_free[gs]);
       }
       if (bar_sync_or(1, 128, !ok)) break;
       // the eight tokens' sums of squares side by side (independent shuffles), then the outputs

@@ -379,7 +379,7 @@ gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, vo
  * GDN_NOALLOC_SCRATCH_BYTES inside libgdn.so, which every GPU that loads the
  * library holds until the process exits.
  *   - Limit: gdn_prefill_workspace_size(H_k, H_v, B, B*ceil(T/64)) must not
- *     exceed GDN_NOALLOC_SCRATCH_BYTES (64 MiB: e.g. up to 11 chunks of 64
+ *     exceed GDN_NOALLOC_SCRATCH_BYTES (64 MiB: e.g. up to 9 chunks of 64
  *     tokens in total at 16/48 heads, 88 at 2/6 heads); larger requests return
  *     GDN_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the array's device address

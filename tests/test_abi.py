@@ -39,7 +39,7 @@ def test_workspace_size(lib):
     base = gdn.workspace_size(16, 48, 1, 0)
     assert base > 0
     per_chunk = gdn.workspace_size(16, 48, 1, 1) - base
-    assert per_chunk == 16 * 65536 + 48 * 99328  # K, Q images per key head; W, P, B_U, v_hat, gates per value head
+    assert per_chunk == 16 * 32768 + 48 * 132096  # K image per key head; W, gamma Q, P, B_U, v_hat, gates per value head
     assert gdn.workspace_size(0, 48, 1, 1) == 0
     assert gdn.workspace_size(16, 48, -1, 1) == 0
 

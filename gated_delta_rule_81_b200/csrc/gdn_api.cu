@@ -2,6 +2,9 @@
 // and kernel launches.  Declared in include/gdn.h.
 #include <limits.h>
 #include <stdint.h>
+#include <stdlib.h>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/gdn.h"
 #include "gdn_kernels.cuh"
@@ -9,6 +12,26 @@
 using gdn::bf16;
 
 namespace {
+
+// NVTX ranges named after the entry points, when GDN_NVTX is set (to anything but 0) in the
+// environment; read once.  NVTX3 is header-only and loads nothing unless a profiler injects it.
+bool nvtx_on() {
+  static const bool on = [] {
+    const char* e = getenv("GDN_NVTX");
+    return e && *e && !(e[0] == '0' && e[1] == 0);
+  }();
+  return on;
+}
+
+struct NvtxRange {
+  bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_on()) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -207,6 +230,7 @@ size_t gdn_prefill_workspace_size(int H_k, int H_v, int N, long long n_chunks) {
 gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
                        const void* conv_in, void* conv_out, void* out, void* workspace, size_t workspace_bytes,
                        int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_prefill");
   if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
@@ -218,6 +242,7 @@ gdn_status gdn_prefill(const gdn_inputs* in, int B, int T, const float* state_in
 gdn_status gdn_prefill_varlen(const gdn_inputs* in, int N, const int* cu_seqlens, const int* cu_seqlens_host,
                               const float* state_in, float* state_out, const void* conv_in, void* conv_out,
                               void* out, void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_prefill_varlen");
   if (N < 0) return GDN_ERR_INVALID_ARG;
   if (N == 0) return check_inputs(in, 0);
   if (!cu_seqlens || !cu_seqlens_host) return GDN_ERR_INVALID_ARG;
@@ -269,6 +294,7 @@ size_t gdn_prefill_host_workspace_size(int H_k, int H_v, int B, int T) {
 gdn_status gdn_prefill_host(const gdn_inputs* in, int B, int T, const float* state_in, float* state_out,
                             const void* conv_in, void* conv_out, void* out, void* workspace, size_t workspace_bytes,
                             int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_prefill_host");
   if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
@@ -331,6 +357,7 @@ gdn_status gdn_prefill_host(const gdn_inputs* in, int B, int T, const float* sta
 
 gdn_status gdn_gemm_bf16(const void* A, long long lda, const void* B, long long ldb, void* C, long long ldc, int M,
                          int N, int K, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_gemm_bf16");
   if (M < 0 || N < 0 || K < 0) return GDN_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return GDN_OK;
   if (!A || !B || !C || K == 0) return GDN_ERR_INVALID_ARG;
@@ -363,6 +390,7 @@ size_t gdn_layer_workspace_size(int H_k, int H_v, int B, int T) {
 gdn_status gdn_layer_prefill(const gdn_layer* L, int B, int T, const void* x, long long ldx, const float* state_in,
                              float* state_out, const void* conv_in, void* conv_out, void* y, long long ldy,
                              void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_layer_prefill");
   if (!L || B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
   if (L->H_k <= 0 || L->H_v <= 0 || L->hidden <= 0 || L->H_v % L->H_k != 0) return GDN_ERR_INVALID_ARG;
   if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
@@ -418,6 +446,7 @@ size_t gdn_layer_decode_workspace_size(int H_k, int H_v, int N, int T) {
 gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, long long ldx, float* state,
                             void* conv_state, const int* state_slot, int n_slots, void* y, long long ldy,
                             void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_layer_decode");
   if (!L || N < 0 || T < 1 || T > gdn::kMaxDecodeTokens) return GDN_ERR_INVALID_ARG;
   if (L->H_k <= 0 || L->H_v <= 0 || L->hidden <= 0 || L->H_v % L->H_k != 0) return GDN_ERR_INVALID_ARG;
   if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
@@ -465,6 +494,7 @@ gdn_status gdn_layer_decode(const gdn_layer* L, int N, int T, const void* x, lon
 
 gdn_status gdn_attention_prefill(const void* q_hat, const void* k, const void* v, const void* g, long long ld_g,
                                  int B, int T, void* out, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_attention_prefill");
   if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
   const long long T_tot = static_cast<long long>(B) * T;
   if (T_tot > INT_MAX) return GDN_ERR_UNSUPPORTED;
@@ -495,6 +525,7 @@ size_t gdn_attn_layer_workspace_size(int B, int T) {
 gdn_status gdn_attn_layer_prefill(const gdn_attn_layer* L, int B, int T, const void* x, long long ldx,
                                   void* k_cache, void* v_cache, int cache_cap, void* y, long long ldy,
                                   void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_attn_layer_prefill");
   if (!L || B < 0 || T < 0 || L->hidden <= 0 || cache_cap < 0) return GDN_ERR_INVALID_ARG;
   const int cap = cache_cap == 0 ? T : cache_cap;
   if (cap < T) return GDN_ERR_INVALID_ARG;
@@ -554,6 +585,7 @@ size_t gdn_attn_decode_workspace_size(int N, int cache_cap) {
 gdn_status gdn_attn_layer_decode_step(const gdn_attn_layer* L, int N, const void* x, long long ldx, void* k_cache,
                                       void* v_cache, int cache_cap, int* cache_len, void* y, long long ldy,
                                       void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_attn_layer_decode_step");
   if (!L || N < 0 || cache_cap <= 0 || L->hidden <= 0) return GDN_ERR_INVALID_ARG;
   if (L->hidden % 64 != 0) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
@@ -602,6 +634,7 @@ gdn_status gdn_attn_layer_decode_step(const gdn_attn_layer* L, int N, const void
 
 gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, void* conv_state,
                             const int* state_slot, int n_slots, void* out, int* err, void* stream) {
+  const NvtxRange nvtx_range("gdn_decode_multi");
   if (N < 0 || T < 1 || T > gdn::kMaxDecodeTokens || n_slots < 0) return GDN_ERR_INVALID_ARG;
   const long long T_tot = static_cast<long long>(N) * T;
   gdn_status st = check_inputs(in, T_tot);
@@ -647,6 +680,7 @@ gdn_status gdn_decode_multi(const gdn_inputs* in, int N, int T, float* state, vo
 
 gdn_status gdn_decode_step(const gdn_inputs* in, int N, float* state, void* conv_state, void* out, int* err,
                            void* stream) {
+  const NvtxRange nvtx_range("gdn_decode_step");
   return gdn_decode_multi(in, N, 1, state, conv_state, nullptr, N, out, err, stream);
 }
 

@@ -41,6 +41,10 @@
  *     state_slot outside the pool, 16 = an attention KV cache with no row left, 32 = an
  *     attention decode cache_len outside [0, cache_cap]).  It is never cleared by the
  *     library.  Read it after synchronising; gdn_err_status maps it to a gdn_status.
+ *   - With GDN_NVTX set in the environment (to anything but "0", read on the first
+ *     call), every launching entry point pushes an NVTX range named after itself for
+ *     its duration on the host (NVTX3, header-only: nothing is loaded unless a
+ *     profiler injects its library).
  */
 #ifndef GDN_H_
 #define GDN_H_

@@ -321,3 +321,22 @@ def test_fused_plan_follows_the_available_sms(lib):
     assert plan(16, 48, 8, 1681, 0, 148) == 0        # 8 sequences: 384 scan units, two launches
     assert plan(2, 6, 1, 8, 2, 148) == 6
     assert plan(16, 48, 1, 64, 0, 0) == 0 and plan(0, 48, 1, 64, 0, 148) == 0
+
+
+def test_nvtx_ranges_switch_on_from_the_environment():
+    """GDN_NVTX=1: the entry points push NVTX ranges (no profiler attached, so no-ops); a call
+    that fails validation still returns its status and pops its range."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, sys; sys.path.insert(0, %r)\n"
+        "from gated_delta_rule_81_b200 import gdn\n"
+        "lib = gdn.load()\n"
+        "s = gdn.GdnInputs()\n"
+        "rc = lib.gdn_prefill(ctypes.byref(s), -1, 4, None, None, None, None, None, None, 0, None, None)\n"
+        "rc2 = lib.gdn_decode_step(ctypes.byref(s), -1, None, None, None, None, None)\n"
+        "print(rc, rc2)\n" % ROOT)
+    env = dict(os.environ, GDN_NVTX="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == ["1", "1"]  # GDN_ERR_INVALID_ARG, from both

@@ -59,9 +59,19 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
-TRAFFIC = {(1, "scan"): {"bytes": 442609664 + 44196608, "sha": "44d4966011593d14"},   # ncu, T=4096 layer
-           (1, "prep"): {"bytes": 101810688 + 334646272, "sha": "44d4966011593d14"},
-           (1, "prefill_fused"): {"bytes": 434084096 + 422704128, "sha": "44d4966011593d14"}}
+TRAFFIC = {
+    (1, "prefill_fused"): {"bytes": 443626496 + 462670848, "sha": "71336e0501319143"},  # ncu, T=4096 16/48, one launch
+    (1, "prep"): {"bytes": 87340032 + 383146240, "sha": "71336e0501319143"},
+    (1, "scan"): {"bytes": 493061888 + 41922048, "sha": "71336e0501319143"},
+    (0, "prep"): {"bytes": 1435648 + 0, "sha": "71336e0501319143"},                  # ncu, T=512 2/6
+    (0, "scan"): {"bytes": 7726848 + 0, "sha": "71336e0501319143"},
+    (2, "prefill_fused"): {"bytes": 16 * (1945085184 + 1959130112), "sha": "71336e0501319143",
+                           "note": "ncu capture of the first 16,384 tokens (fused launch), x16 by tokens"},
+    (3, "prep"): {"bytes": round(8.004909618388753 * (305648896 + 1423295488)), "sha": "71336e0501319143",
+                 "note": "ncu capture with every packed length scaled to 13,443 tokens in all, x107610/13443"},
+    (3, "scan"): {"bytes": round(8.004909618388753 * (1669312768 + 174477824)), "sha": "71336e0501319143",
+                 "note": "ncu capture with every packed length scaled to 13,443 tokens in all, x107610/13443"},
+}
 DECODE_TRAFFIC = {"bytes": 829675264 + 766249984, "sha": "852a2d42cccfe44d"}  # ncu, one step of 256 sequences
 
 
@@ -200,10 +210,23 @@ WORKLOADS = {"prefill4k": 1, "tiny": 0, "fullctx": 2, "varlen": 3}
 SCHEDULES = {"auto": 0, "two-launches": 1, "fused": 2}
 
 
+def case_overrides(args, cfg_id, seed):
+    """--tokens: a configuration on a prefix of its tokens (uniform cases) or with every packed
+    length scaled to about that total (varlen), the same distributions otherwise."""
+    if not getattr(args, "tokens", None):
+        return {}
+    c = gin.CONFIGS[cfg_id]
+    if c["kind"] == "varlen":
+        full = gin.varlen_lengths(c["N"], c["len_lo"], c["len_hi"], seed)
+        f = args.tokens / sum(full)
+        return {"lengths": [max(64, int(n * f)) for n in full]}
+    return {"T": args.tokens}
+
+
 def run_prefill_ours(args, world, rank, dev, pk, cfg_id=1):
     from gated_delta_rule_81_b200 import gdn
 
-    case = gin.prefill_case(cfg_id, seed=rank)
+    case = gin.prefill_case(cfg_id, seed=rank, **case_overrides(args, cfg_id, rank))
     inp = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in case["inp"].items()}
     st = case["state_in"].to(dev) if case["state_in"] is not None else None
     varlen = gin.CONFIGS[cfg_id]["kind"] == "varlen"
@@ -255,6 +278,7 @@ def run_prefill_ours(args, world, rank, dev, pk, cfg_id=1):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item())}")
     return {"total_ms": total_ms, "step_ms": step_ms, "T": T_tot, "clocks": clk.report(),
+            "prefix": bool(getattr(args, "tokens", None)),
             "launches_per_step": 4 if varlen else 3, "case": case, "H_k": H_k, "H_v": H_v, "N": N,
             "kernel_ms": {"prep": statistics.mean(prep_ms), "scan": statistics.mean(scan_ms),
                           "helpers+gaps": statistics.mean(step_ms) - statistics.mean(prep_ms)
@@ -277,7 +301,7 @@ def prefill_roofline(res, cfg_id, pk, ms_per_step):
         flops = (scan_flop_per_token(res["H_v"]) if dom == "scan" else prep_flop_per_token(res["H_k"], res["H_v"])) * T
     achieved = flops / (kt[dom] * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
-    tr = TRAFFIC.get((cfg_id, dom))
+    tr = None if res.get("prefix") else TRAFFIC.get((cfg_id, dom))  # (the ncu figures are for the full case)
     traffic = tr["bytes"] if tr and tr.get("sha") == src_sha("gdn_prefill.cu") else None
     return {"kernel": f"{dom}_kernel", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic,
@@ -295,7 +319,7 @@ def prefill_secondaries(args, world, rank, dev, pk):
     out = []
     for cfg_id, steps in ((0, 20), (2, 3), (3, 5)):
         a = argparse.Namespace(**vars(args))
-        a.steps, a.warmup = steps, 3
+        a.steps, a.warmup, a.tokens = steps, 3, None
         res = run_prefill_ours(a, world, rank, dev, pk, cfg_id)
         ms = res["total_ms"] / steps
         c = gin.CONFIGS[cfg_id]
@@ -759,6 +783,9 @@ def main():
                                                               "attn_decode"],
                     default="prefill4k",
                     help="prefill4k (default, the headline line) or another configuration for the record")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="prefill workloads: run on a prefix of this many tokens (packed sequences: every "
+                         "length scaled to about this total), e.g. for a profiler capture of a smaller case")
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto",
                     help="prefill launch plan (gdn_inputs.schedule): auto, two-launches, or fused (prep and scan "
                          "overlapped in one launch whenever the scan units fit in half the SMs)")

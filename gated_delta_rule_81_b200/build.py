@@ -1,6 +1,8 @@
 """Compile the sm_100a libraries in-tree with nvcc.
 
   libgdn.so          the mixer (C ABI declared in include/gdn.h)
+  libgdn_debug.so    the same with GDN_DEBUG: every workspace access of the prefill kernels is
+                     bounds-checked (an access outside is skipped and reported, error bit 64)
   libgdn_selftest.so tcgen05/UMMA layout self-test kernel used by the GPU tests
 """
 from __future__ import annotations
@@ -21,10 +23,13 @@ NVCC_FLAGS = [
     "-diag-suppress", "177",
 ]
 
+_GDN_SOURCES = ["gdn_api.cu", "gdn_prefill.cu", "gdn_decode.cu", "gdn_noalloc.cu", "gdn_gemm.cu", "gdn_attention.cu"]
 TARGETS = {
-    "libgdn.so": ["gdn_api.cu", "gdn_prefill.cu", "gdn_decode.cu", "gdn_noalloc.cu", "gdn_gemm.cu", "gdn_attention.cu"],
+    "libgdn.so": _GDN_SOURCES,
+    "libgdn_debug.so": _GDN_SOURCES,
     "libgdn_selftest.so": ["umma_selftest.cu", "wait_selftest.cu"],
 }
+EXTRA_FLAGS = {"libgdn_debug.so": ["-DGDN_DEBUG"]}
 
 
 def _nvcc() -> str:
@@ -53,7 +58,8 @@ def build(force: bool = False, verbose: bool = False) -> list[str]:
             os.path.getmtime(f) > os.path.getmtime(out) for f in _deps(srcs))
         if stale:
             tmp = out + f".tmp{os.getpid()}"
-            cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *[os.path.join(CSRC, s) for s in srcs]]
+            cmd = [_nvcc(), *NVCC_FLAGS, *EXTRA_FLAGS.get(name, []), "-I", INCLUDE, "-o", tmp,
+                   *[os.path.join(CSRC, s) for s in srcs]]
             if verbose:
                 print(" ".join(cmd))
             subprocess.run(cmd, check=True)

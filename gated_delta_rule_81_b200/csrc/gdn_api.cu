@@ -205,6 +205,7 @@ gdn_status prefill_common(const gdn_inputs* in, int N, long long T_tot, long lon
   p.seq_order = cu ? reinterpret_cast<int*>(ws + gdn::kWsHeader) + (N + 1) : nullptr;
   p.ws_k = ws + gdn::kWsHeader + chunk_base_bytes(N);
   p.ws_head = p.ws_k + static_cast<size_t>(n_chunks) * in->H_k * gdn::kKBytes;
+  p.ws_end = ws + need;  // the layout's own end (a caller may pass more)
   p.state_in = state_in;
   p.state_out = state_out;
   p.conv_in = static_cast<const bf16*>(conv_in);

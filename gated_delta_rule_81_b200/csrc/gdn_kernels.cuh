@@ -77,6 +77,7 @@ struct PrefillParams {
   int* ws_flag;           // workspace header word: nonzero = inconsistent cu_seqlens
   uint8_t* ws_k;          // [n_chunks][H_k][kKBytes]
   uint8_t* ws_head;       // [n_chunks][H_v][kHeadBytes]
+  const uint8_t* ws_end;  // one past the caller's workspace (checked by the debug build)
   const float* state_in;  // [N][H_v][128][128] or null (zeros)
   float* state_out;       // [N][H_v][128][128] or null
   const bf16* conv_in;    // [N][3][C_conv] or null (zeros)
@@ -87,6 +88,22 @@ struct PrefillParams {
   int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, scan CTAs first, prep items
                           // published by ready flags; 0 = prep kernel, then scan kernel
 };
+
+constexpr int kDevErrBounds = 64;  // (debug build) an access outside the workspace was skipped
+
+// Debug build (GDN_DEBUG, libgdn_debug.so): every workspace access of the prefill kernels is
+// checked against [ws_k, ws_end); one outside sets kDevErrBounds and is skipped (never a trap).
+// In the product build the check is the constant true and compiles away.
+#ifdef GDN_DEBUG
+__device__ __forceinline__ bool ws_ok(const PrefillParams& p, const void* ptr, long long bytes) {
+  const uint8_t* a = static_cast<const uint8_t*>(ptr);
+  const bool ok = a >= p.ws_k && bytes >= 0 && a + bytes <= p.ws_end;
+  if (!ok && p.err) atomicOr(p.err, kDevErrBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool ws_ok(const PrefillParams&, const void*, long long) { return true; }
+#endif
 
 // events: null, or cudaEvent_t handles recorded around the kernels (see gdn_inputs.events)
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events);

@@ -525,8 +525,10 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
         uint4 hi, lo;
         split8(y, hi, lo);
         const uint32_t off = sw128_off(i, cg & 7);
-        *reinterpret_cast<uint4*>(gv + off) = hi;
-        *reinterpret_cast<uint4*>(gv + kImg64 + off) = lo;
+        if (ws_ok(p, gv + off, 16) && ws_ok(p, gv + kImg64 + off, 16)) {
+          *reinterpret_cast<uint4*>(gv + off) = hi;
+          *reinterpret_cast<uint4*>(gv + kImg64 + off) = lo;
+        }
       }
     }
     named_bar_sync(bar_id, kPrepThreads);  // the staged rows are read: the region is free
@@ -613,9 +615,11 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
   // [Q;K] K^T -> TMEM columns 0..63 (rows 0..63: Q K^T, rows 64..127: K K^T)
   if (tid == 0) {
     uint8_t* gK = p.ws_k + (gc * H_k + kh) * static_cast<long long>(kKBytes);
+    if (ws_ok(p, gK, kKBytes)) {
 #pragma unroll
-    for (int piece = 0; piece < 4; ++piece)  // hi block 0, hi block 1, lo block 0, lo block 1
-      bulk_s2g(gK + piece * 8192, sQK + piece * 16384 + 8192, 8192);
+      for (int piece = 0; piece < 4; ++piece)  // hi block 0, hi block 1, lo block 0, lo block 1
+        bulk_s2g(gK + piece * 8192, sQK + piece * 16384 + 8192, 8192);
+    }
     bulk_commit();
     const uint32_t qh = smem_u32(sQK), ql = qh + 32768;
     const uint32_t idesc = idesc_bf16(128, 64, false, false);
@@ -641,7 +645,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
       val = expf(Glast);
     }
     float* gdst = reinterpret_cast<float*>(p.ws_head + (gc * H_v + h) * static_cast<long long>(kHeadBytes) + kHeadOffGate);
-    if (k2 != kReadyFlagWord) gdst[k2] = val;
+    if (k2 != kReadyFlagWord && ws_ok(p, gdst + k2, 4)) gdst[k2] = val;
   }
 
   // identity B image for the q^T transpose, in region R (the raw rows are dead)
@@ -726,8 +730,10 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     }
     named_bar_sync(bar_id, kPrepThreads);
     if (tid == 0) {
-      bulk_s2g(hb + kHeadOffP, sQK, kPImg);
-      bulk_s2g(hb + kHeadOffP + kPImg, sQK + 32768, kPImg);
+      if (ws_ok(p, hb + kHeadOffP, 2 * kPImg)) {
+        bulk_s2g(hb + kHeadOffP, sQK, kPImg);
+        bulk_s2g(hb + kHeadOffP + kPImg, sQK + 32768, kPImg);
+      }
       bulk_commit();
     }
     solve_unit_lower(sA, sT, sM, tid, bar_id);
@@ -760,7 +766,7 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     named_bar_sync(bar_id, kPrepThreads);
     tc_fence_after();
     if (tid == 0) {
-      bulk_s2g(hb + kHeadOffBU, sBU, 2 * kPImg);
+      if (ws_ok(p, hb + kHeadOffBU, 2 * kPImg)) bulk_s2g(hb + kHeadOffBU, sBU, 2 * kPImg);
       bulk_commit();
       bulk_wait_read<0>();  // B_U has left region R before the product's completion frees it
       // W^T = K^T B_W^T: A = K (MN-major, rows = tokens), B = B_W (K-major)
@@ -818,11 +824,13 @@ __device__ __forceinline__ void prep_body(const PrefillParams& p, long long gc, 
     tc_fence_after();
     if (tid == 0) {
       uint8_t* wd = hb + kHeadOffW;  // -W^T lo | -W^T hi | (gamma Q)^T hi | (gamma Q)^T lo
-      bulk_s2g(wd, sQK, 8192);
-      bulk_s2g(wd + 8192, sQK + 16384, 8192);
-      bulk_s2g(wd + 16384, sQK + 32768, 8192);
-      bulk_s2g(wd + 24576, sQK + 49152, 8192);
-      bulk_s2g(hb + kHeadOffGQ, sR, 2 * kImg64);
+      if (ws_ok(p, wd, 2 * kWBytes)) {
+        bulk_s2g(wd, sQK, 8192);
+        bulk_s2g(wd + 8192, sQK + 16384, 8192);
+        bulk_s2g(wd + 16384, sQK + 32768, 8192);
+        bulk_s2g(wd + 24576, sQK + 49152, 8192);
+        bulk_s2g(hb + kHeadOffGQ, sR, 2 * kImg64);
+      }
       bulk_commit();
       bulk_wait_read<0>();  // the staging areas (Q pieces, region R) are rewritten by the next value head
     }
@@ -1176,6 +1184,16 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       // soon as the product that reads it has completed), then the double-buffered gates of
       // chunk c + 1.
       int n_g[2] = {0, 0}, n_v = 0, n_bu = 0, n_w = 0, n_k = 0, n_p = 0;
+      // a bulk load into shared memory with its byte count on `bar`; one outside the workspace
+      // (debug build) is skipped and the barrier completes without data
+      auto load = [&](void* dst, const uint8_t* src, uint32_t bytes, uint64_t* bar) {
+        if (ws_ok(p, src, bytes)) {
+          mbar_arrive_expect_tx(bar, bytes);
+          bulk_g2s(dst, src, bytes, bar);
+        } else {
+          mbar_arrive(bar);
+        }
+      };
       auto head_blob = [&](int c) {
         return p.ws_head + ((cb + c) * p.H_v + h) * static_cast<long long>(kHeadBytes);
       };
@@ -1184,8 +1202,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         // fused launch: chunk c's operands (read from here on) are published by its prep
         if (p.fused_scan_ctas > 0 && !flag_wait(ready_flag(p, cb + c, h), ab, kBackoffNs)) return false;
         if (c >= 2 && !mbar_wait(&g_free[st], ((c >> 1) - 1) & 1, ab, false, kBackoffNs)) return false;
-        mbar_arrive_expect_tx(&g_full[st], kGateBytes);
-        bulk_g2s(sm + kScOffG + st * kGateBytes, head_blob(c) + kHeadOffGate, kGateBytes, &g_full[st]);
+        load(sm + kScOffG + st * kGateBytes, head_blob(c) + kHeadOffGate, kGateBytes, &g_full[st]);
         ++n_g[st];
         return true;
       };
@@ -1194,24 +1211,19 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         const uint8_t* hb = head_blob(c);
         const uint8_t* kb = p.ws_k + ((cb + c) * p.H_k + kh) * static_cast<long long>(kKBytes);
         if (c >= 1 && !mbar_wait(&v_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&v_full, 2 * kImg64);
-        bulk_g2s(sm + kScOffV, hb + kHeadOffV, 2 * kImg64, &v_full);
+        load(sm + kScOffV, hb + kHeadOffV, 2 * kImg64, &v_full);
         ++n_v;
         if (c >= 1 && !mbar_wait(&bu_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&bu_full, 2 * kPImg);
-        bulk_g2s(sm + kScOffBU, hb + kHeadOffBU, 2 * kPImg, &bu_full);
+        load(sm + kScOffBU, hb + kHeadOffBU, 2 * kPImg, &bu_full);
         ++n_bu;
         if (c >= 1 && !mbar_wait(&w_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&w_full, 2 * kWBytes);
-        bulk_g2s(sm + kScOffW, hb + kHeadOffW, 2 * kWBytes, &w_full);  // W and gamma Q side by side
+        load(sm + kScOffW, hb + kHeadOffW, 2 * kWBytes, &w_full);  // W and gamma Q side by side
         ++n_w;
         if (c >= 1 && !mbar_wait(&k_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&k_full, kKBytes);
-        bulk_g2s(sm + kScOffK, kb, kKBytes, &k_full);
+        load(sm + kScOffK, kb, kKBytes, &k_full);
         ++n_k;
         if (c >= 1 && !mbar_wait(&p_free, (c - 1) & 1, ab, false, kBackoffNs)) break;
-        mbar_arrive_expect_tx(&p_full, 2 * kPImg);
-        bulk_g2s(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
+        load(sm + kScOffP, hb + kHeadOffP, 2 * kPImg, &p_full);
         ++n_p;
         if (c + 1 < nc) ok = load_gates(c + 1);
         if (c + 2 < nc) {  // two chunks ahead into L2, behind this chunk's copies

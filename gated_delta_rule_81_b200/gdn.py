@@ -86,10 +86,12 @@ EXPORTS = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_prefill_varlen", "g
 MAX_DECODE_TOKENS = 8
 
 
-def load(path: str | None = None):
-    """Load libgdn.so from the package directory (it must have been built)."""
+def load(path: str | None = None, fresh: bool = False):
+    """Load libgdn.so from the package directory (it must have been built).  The first library
+    loaded is kept for every later call; `fresh` loads `path` (e.g. libgdn_debug.so) and
+    returns it without making it that library."""
     global _lib
-    if _lib is not None:
+    if _lib is not None and not fresh:
         return _lib
     path = path or _build.lib_path("libgdn.so")
     if not os.path.exists(path):
@@ -142,7 +144,8 @@ def load(path: str | None = None):
     lib.gdn_err_status.restype = _i
     lib.gdn_prefill_fused_plan.argtypes = [_i, _i, _i, _ll, _i, _i]
     lib.gdn_prefill_fused_plan.restype = _i
-    _lib = lib
+    if not fresh:
+        _lib = lib
     return lib
 
 

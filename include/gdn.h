@@ -39,8 +39,13 @@
  *     (1 = a bounded wait timed out, 2 = reserved,
  *     4 = cu_seqlens on the device disagreed with cu_seqlens_host, 8 = a decode
  *     state_slot outside the pool, 16 = an attention KV cache with no row left, 32 = an
- *     attention decode cache_len outside [0, cache_cap]).  It is never cleared by the
- *     library.  Read it after synchronising; gdn_err_status maps it to a gdn_status.
+ *     attention decode cache_len outside [0, cache_cap], 64 = (libgdn_debug.so only) a
+ *     prefill kernel found a workspace access outside the workspace and skipped it).
+ *     It is never cleared by the library.  Read it after synchronising; gdn_err_status
+ *     maps it to a gdn_status.
+ *   - libgdn_debug.so exports the same calls, built with every workspace access of the
+ *     prefill kernels checked against the workspace's bounds (a failed check sets bit 64
+ *     and skips the access; nothing traps).  Same results as libgdn.so on valid calls.
  *   - With GDN_NVTX set in the environment (to anything but "0", read on the first
  *     call), every launching entry point pushes an NVTX range named after itself for
  *     its duration on the host (NVTX3, header-only: nothing is loaded unless a

@@ -30,6 +30,14 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_debug_library_exports_the_same_symbols(lib):
+    """libgdn_debug.so (bounds-checked workspace accesses) is a drop-in for libgdn.so."""
+    dbg = gdn.load(build.lib_path("libgdn_debug.so"), fresh=True)
+    assert dbg is not lib
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert gdn.status_string(code).startswith("GDN_")

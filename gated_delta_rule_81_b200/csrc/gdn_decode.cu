@@ -13,9 +13,14 @@
 // T updates run on the row in registers, so the call's HBM traffic is one state
 // round trip for T tokens.
 //
-// One CTA per (sequence, key head): it owns the key head's q/k conv channels
-// and the value channels and state rows of the key head's value heads, so the
-// conv state and the recurrent state are updated in place without races.
+// One CTA per (sequence, key head), or, when that grid would leave SMs idle (few
+// sequences), one CTA per (sequence, value head) with the G CTAs of a key head in one
+// thread-block cluster.  A CTA owns the state rows and value channels of its value heads,
+// so the recurrent state and the v part of the conv state are updated in place without
+// races; the q/k conv channels of a key head are read by every CTA of its cluster and
+// written by the cluster's first CTA after a cluster barrier, i.e. after all of them
+// have read the history.  Each CTA of a cluster normalises q and k itself (the same code
+// on the same data), so both grids give bitwise equal results.
 // Every token goes through the same code whatever T is, so T calls with one token
 // and one call with T tokens give bitwise equal results.
 //
@@ -73,17 +78,24 @@ __host__ __device__ inline DecodeSmem decode_smem(int T, int G) {
   return L;
 }
 
-// global channel of CTA channel j: q head kh, k head kh, v heads kh G .. kh G + G - 1
-__device__ __forceinline__ long long conv_channel(int j, int kh, int H_k, int G) {
+// global channel of CTA channel j: q head kh, k head kh, then the CTA's value heads from hv0 on
+__device__ __forceinline__ long long conv_channel(int j, int kh, int H_k, int hv0) {
   return j < kD       ? static_cast<long long>(kh) * kD + j
          : j < 2 * kD ? static_cast<long long>(H_k + kh) * kD + (j - kD)
-                      : static_cast<long long>(2 * H_k) * kD + static_cast<long long>(kh) * G * kD + (j - 2 * kD);
+                      : static_cast<long long>(2 * H_k + hv0) * kD + (j - 2 * kD);
+}
+
+// every thread of the cluster arrives, then waits for all the others (release / acquire)
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams p) {
-  const int kh = blockIdx.x, n = blockIdx.y;
+  // grid (parts, H_k, N): a part takes G / parts consecutive value heads of key head kh
+  const int part = blockIdx.x, parts = gridDim.x, kh = blockIdx.y, n = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k, T = p.T;
+  const int H_k = p.H_k, H_v = p.H_v, G = H_v / H_k / parts, T = p.T;
+  const int hv0 = (kh * parts + part) * G;  // the CTA's first value head; G = its value heads
   const long long C_conv = static_cast<long long>(2 * H_k + H_v) * kD;
   const int slot = p.state_slot ? p.state_slot[n] : n;
   if (slot < 0 || slot >= p.n_slots) {  // the same value in every thread: the CTA leaves together
@@ -91,7 +103,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
     return;
   }
   const int n_ch = (2 + G) * kD, n_rows = G * kD;
-  float* S = p.state + (static_cast<long long>(slot) * H_v + static_cast<long long>(kh) * G) * kD * kD;
+  float* S = p.state + (static_cast<long long>(slot) * H_v + hv0) * kD * kD;
   // the first block of state rows of each warp starts on its way to L2 now
   if (lane == 0) prefetch_l2(S + static_cast<long long>(warp) * kRowsPerIter * kD, kRowBlockBytes);
 
@@ -116,26 +128,26 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
     const long long tok = static_cast<long long>(n) * T + t;
     const bf16* src = e < kD       ? p.q + tok * p.sq + static_cast<long long>(kh) * kD + e
                       : e < 2 * kD ? p.k + tok * p.sk + static_cast<long long>(kh) * kD + (e - kD)
-                                   : p.v + tok * p.sv + static_cast<long long>(kh) * G * kD + (e - 2 * kD);
+                                   : p.v + tok * p.sv + static_cast<long long>(hv0) * kD + (e - 2 * kD);
     cp_async16(xraw + t * n_ch + e, src);
   }
   const bf16* cs_in = p.conv_state + static_cast<long long>(slot) * 3 * C_conv;
   for (int i = tid; i < 3 * n_p16; i += kDecThreads) {  // conv history rows
     const int row = i / n_p16, e = (i % n_p16) * 8;
-    cp_async16(hist + row * n_ch + e, cs_in + row * C_conv + conv_channel(e, kh, H_k, G));
+    cp_async16(hist + row * n_ch + e, cs_in + row * C_conv + conv_channel(e, kh, H_k, hv0));
   }
   for (int i = tid; i < n_ch / 2; i += kDecThreads) {  // conv taps: one piece = 2 channels x 4 taps
     const int e = 2 * i;
-    cp_async16(taps + e * kTaps, p.conv_w + conv_channel(e, kh, H_k, G) * kTaps);
+    cp_async16(taps + e * kTaps, p.conv_w + conv_channel(e, kh, H_k, hv0) * kTaps);
   }
   for (int i = tid; i < T * G * (kD / 8); i += kDecThreads) {  // z of the T tokens and G heads
     const int t = i / (G * (kD / 8)), rem = i % (G * (kD / 8)), jh = rem / (kD / 8), e = (rem % (kD / 8)) * 8;
     const long long tok = static_cast<long long>(n) * T + t;
-    cp_async16(z_s + (t * G + jh) * kD + e, p.z + tok * p.sz + static_cast<long long>(kh * G + jh) * kD + e);
+    cp_async16(z_s + (t * G + jh) * kD + e, p.z + tok * p.sz + static_cast<long long>(hv0 + jh) * kD + e);
   }
   cp_async_commit();
   for (int x = tid; x < T * G; x += kDecThreads) {  // gates (a and b are only 2-byte aligned)
-    const int t = x / G, jh = x % G, h = kh * G + jh;
+    const int t = x / G, jh = x % G, h = hv0 + jh;
     const long long tok = static_cast<long long>(n) * T + t;
     const float a = __bfloat162float(p.a[tok * p.sa + h]);
     const float b = __bfloat162float(p.b[tok * p.sb + h]);
@@ -145,6 +157,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
   if (tid < kD) normw_s[tid] = __bfloat162float(p.norm_w[tid]);
   cp_async_wait_all();
   __syncthreads();
+  if (parts > 1) cluster_barrier();  // every CTA of the key head holds the old q/k history now
 
   // ---- causal conv over the T new tokens (a sliding window over the 3 history rows);
   // the conv state takes the last three raw tokens
@@ -167,10 +180,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
       h1 = h2;
       h2 = x;
     }
-    const long long c = conv_channel(j, kh, H_k, G);
-    cs_out[c] = __float2bfloat16(h0);
-    cs_out[C_conv + c] = __float2bfloat16(h1);
-    cs_out[2 * C_conv + c] = __float2bfloat16(h2);
+    if (part == 0 || j >= 2 * kD) {  // q/k channels: the cluster's first CTA alone
+      const long long c = conv_channel(j, kh, H_k, hv0);
+      cs_out[c] = __float2bfloat16(h0);
+      cs_out[C_conv + c] = __float2bfloat16(h1);
+      cs_out[2 * C_conv + c] = __float2bfloat16(h2);
+    }
   }
   __syncthreads();
   // L2 norms of q and k of every token (item = 2 t + which)
@@ -297,7 +312,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
 
   // ---- gated RMS-norm per (token, value head): one warp per pair
   for (int pr = warp; pr < T * G; pr += kDecThreads / 32) {
-    const int t = pr / G, jh = pr % G, h = kh * G + jh;
+    const int t = pr / G, jh = pr % G, h = hv0 + jh;
     const long long tok = static_cast<long long>(n) * T + t;
     const float* ot = o_s + t * n_rows + jh * kD;
     const bf16* zt = z_s + (t * G + jh) * kD;
@@ -314,17 +329,39 @@ __global__ void __launch_bounds__(kDecThreads, 2) gdn_decode_kernel(DecodeParams
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events) {
+// CTAs per key head: G (one per value head, a cluster of G <= 8) while one CTA per
+// (sequence, key head) would leave SMs idle, else 1.
+int decode_parts(const DecodeParams& p) {
   const int G = p.H_v / p.H_k;
-  const int smem = decode_smem(p.T, G).total;
+  if (G == 1) return 1;
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 1;
+  return static_cast<long long>(p.N) * p.H_k < n_sm ? G : 1;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream, void* const* events) {
+  const int parts = decode_parts(p);
+  const int smem = decode_smem(p.T, p.H_v / p.H_k / parts).total;
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(gdn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(p.H_k, p.N);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(parts, p.H_k, p.N);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = parts;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = parts > 1 ? 1 : 0;
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream);
-  gdn_decode_kernel<<<grid, kDecThreads, smem, stream>>>(p);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = cudaLaunchKernelEx(&cfg, gdn_decode_kernel, p);
+  if (err == cudaSuccess) err = cudaGetLastError();
   if (events) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream);
   return err;
 }

@@ -1,7 +1,8 @@
 """gdn_decode_multi (CUDA, through the C ABI): T new tokens per sequence in one call,
 with the states in slots of a pool.  Checked against the fp64 oracle run over the
-same tokens, against T single-token decode steps (bitwise), and for the slot
-indirection (permuted slots, untouched slots, a slot outside the pool)."""
+same tokens, against T single-token decode steps (bitwise), across the two launch
+grids (bitwise), and for the slot indirection (permuted slots, untouched slots, a
+slot outside the pool)."""
 import numpy as np
 import pytest
 import torch
@@ -86,6 +87,37 @@ def test_decode_multi_bitwise_equals_single_steps(T):
     assert torch.equal(y_multi, y_one)
     assert torch.equal(S_multi, S_one)
     assert torch.equal(C_multi, C_one)
+
+
+@pytest.mark.parametrize("T,heads", [(1, (2, 6)), (3, (1, 8))])
+def test_decode_multi_value_head_grid_bitwise_equals_key_head_grid(T, heads):
+    """Few sequences run one CTA per value head (the G CTAs of a key head in a cluster),
+    a batch that fills the SMs one CTA per key head: the same sequences give bitwise
+    equal outputs, states and conv states either way."""
+    H_k, H_v = heads
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    N_big, N_small = -(-n_sm // H_k) + 1, 3
+    assert N_big * H_k >= n_sm and N_small * H_k < n_sm  # the two calls take different grids
+    case = gin.decode_case(N=N_big, steps=T, H_k=H_k, H_v=H_v, seed=90 + T)
+    tok = seq_major(case, T)
+    keep, inp = make_dev_inputs(tok, case["w"], case["scale"])
+    S_big = case["state"].cuda().clone()
+    C_big = case["conv_state"].cuda().clone()
+    y_big = gdn.decode_multi(inp, N_big, T, S_big, C_big)
+    dev_w = keep[1]
+    for n0 in range(0, N_big, N_small):
+        seqs = list(range(n0, min(n0 + N_small, N_big)))
+        rows = [n * T + t for n in seqs for t in range(T)]
+        part = {k: tok[k][rows].cuda() for k in TOKEN_KEYS}
+        pin = gdn.make_inputs(*(part[k] for k in ("q", "k", "v", "a", "b", "z")), dev_w["conv_w"], dev_w["A_log"],
+                              dev_w["norm_w"], scale=case["scale"])
+        S = case["state"][seqs].cuda()
+        C = case["conv_state"][seqs].cuda()
+        y = gdn.decode_multi(pin, len(seqs), T, S, C)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_big[rows[0]:rows[-1] + 1])
+        assert torch.equal(S, S_big[seqs])
+        assert torch.equal(C, C_big[seqs])
 
 
 def test_decode_multi_state_slots():

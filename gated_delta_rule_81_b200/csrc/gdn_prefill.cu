@@ -884,7 +884,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // memory with lane = d_v row.  Per chunk, every product summed over the hi/lo
 // split terms (hi.hi + hi.lo + lo.hi):
 //   [U^T | O^T]  = V^T [B_U^T | 0] + S [-W^T | (gamma Q)^T]   (U0 from shared-memory operands
-//                  first, off the chain; then one product of N = 256 for both halves)
+//                  first, off the chain; then the U half, committed on its own so that the U
+//                  conversion starts early, then the O half behind it)
 //   S   = gamma_C S + (U^T diag(e^{G_C - G_j})) K   (A = U_d hi/lo from TMEM)
 //   O^T += U^T P^T                      (A = U hi/lo from TMEM)
 //   then the gated RMS-norm of o_i over d_v.
@@ -1099,8 +1100,8 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     if (lane == 0) {
       const uint32_t idesc_v = idesc_bf16(128, 128, true, false);   // v_hi^T [B_U lo | B_U hi] (A MN-major)
       const uint32_t idesc_v2 = idesc_bf16(128, 64, true, false);   // v_lo^T B_U hi
-      const uint32_t idesc_u = idesc_bf16(128, 256, false, true);   // S_hi [-W_lo | -W_hi | gQ_hi | gQ_lo] (B MN-major)
-      const uint32_t idesc_u2 = idesc_bf16(128, 128, false, true);  // S_lo [-W_hi | gQ_hi]
+      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [-W_lo | -W_hi], S_lo [-W_hi | gQ_hi],
+                                                                    // S_hi [gQ_hi | gQ_lo] (B MN-major)
       const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
       const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
       const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
@@ -1127,9 +1128,10 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         }
         umma_commit(&v_free);
         umma_commit(&bu_free);
-        // the chain's product and the state's part of o together, onto U0 and onto the O that
-        // the output warps cleared: [U2 | U1 | O1 | O2] += S_hi [-W_lo | -W_hi | gQ_hi | gQ_lo],
-        // [U1 | O1] += S_lo [-W_hi | gQ_hi]
+        // the chain's product onto U0 (and onto the O that the output warps cleared):
+        // [U2 | U1] += S_hi [-W_lo | -W_hi], [U1 | O1] += S_lo [-W_hi | gQ_hi]; its commit lets
+        // the U conversion start while the state's part of o, [O1 | O2] += S_hi [gQ_hi | gQ_lo],
+        // is issued and runs behind it
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
         if (!mbar_wait(&w_full, c & 1, ab)) break;
         if (!mbar_wait(&o_free, c & 1, ab)) break;
@@ -1139,9 +1141,14 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
           const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
           const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
           umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, true);
-          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
+          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u, true);
         }
         umma_commit(&u_done);
+#pragma unroll kIssueUnroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bq = smem_desc(wq + 2 * kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
+          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, true);
+        }
         umma_commit(&w_free);
         if (!mbar_wait(&u_conv, c & 1, ab)) break;
         if (!mbar_wait(&k_full, c & 1, ab)) break;

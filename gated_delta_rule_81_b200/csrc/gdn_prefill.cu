@@ -892,8 +892,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prep_kernel(PrefillParams p) 
 // Warps 0-7 (thread = d_v row; warps w and w + 4 share a TMEM lane quarter and
 // split its columns) convert S and U between fp32 accumulators and bf16 hi/lo
 // operands in tensor memory, each conversion publishing first the part the next
-// product waits for; warps 8-11 run the output stage (and clear O for the next chunk's
-// accumulation); warp 12 lane 0 issues the MMAs; warp 13 lane 0 issues the bulk copies
+// product waits for; warps 8-11 run the output stage (the first product of o overwrites
+// O once they have read it); warp 12 lane 0 issues the MMAs; warp 13 lane 0 issues the bulk copies
 // (v_hat, B_U, W | gamma Q, K, P single-buffered, gates double-buffered).
 
 constexpr int kScanThreads = 448;
@@ -906,6 +906,7 @@ constexpr uint32_t kColSL = 192;   // S lo
 // [U2 | U1 | O1 | O2], 4 x 64 columns:
 //   U2 = V_hi B_U_lo - S_hi W_lo,  U1 = V_hi B_U_hi + V_lo B_U_hi - S_hi W_hi - S_lo W_hi,
 //   O1 = S_hi gQ_hi + S_lo gQ_hi + U_hi P_hi + U_lo P_hi,  O2 = S_hi gQ_lo + U_hi P_lo
+//   (O1 | O2 start from the first K step of S_hi gQ, without accumulation)
 constexpr uint32_t kColU2 = 256;   //   U^T = U2 + U1
 constexpr uint32_t kColU1 = 320;
 constexpr uint32_t kColO = 384;    //   o = O1 + O2
@@ -1100,8 +1101,8 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     if (lane == 0) {
       const uint32_t idesc_v = idesc_bf16(128, 128, true, false);   // v_hi^T [B_U lo | B_U hi] (A MN-major)
       const uint32_t idesc_v2 = idesc_bf16(128, 64, true, false);   // v_lo^T B_U hi
-      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [-W_lo | -W_hi], S_lo [-W_hi | gQ_hi],
-                                                                    // S_hi [gQ_hi | gQ_lo] (B MN-major)
+      const uint32_t idesc_u = idesc_bf16(128, 128, false, true);   // S_hi [-W_lo | -W_hi], S_hi [gQ_hi | gQ_lo] (B MN-major)
+      const uint32_t idesc_u2 = idesc_bf16(128, 64, false, true);   // S_lo (-W_hi), S_lo gQ_hi
       const uint32_t idesc_s = idesc_bf16(128, 128, false, true);   // U_d K (K MN-major, N = d_k)
       const uint32_t idesc_y = idesc_bf16(128, 128, false, false);  // U_hi [P_hi | P_lo] (K-major)
       const uint32_t idesc_y2 = idesc_bf16(128, 64, false, false);  // U_lo P_hi
@@ -1128,26 +1129,28 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
         }
         umma_commit(&v_free);
         umma_commit(&bu_free);
-        // the chain's product onto U0 (and onto the O that the output warps cleared):
-        // [U2 | U1] += S_hi [-W_lo | -W_hi], [U1 | O1] += S_lo [-W_hi | gQ_hi]; its commit lets
-        // the U conversion start while the state's part of o, [O1 | O2] += S_hi [gQ_hi | gQ_lo],
-        // is issued and runs behind it
+        // the chain's product onto U0: [U2 | U1] += S_hi [-W_lo | -W_hi], U1 += S_lo (-W_hi); its
+        // commit lets the U conversion start while the state's part of o is issued and runs
+        // behind it, [O1 | O2] = S_hi [gQ_hi | gQ_lo], O1 += S_lo gQ_hi, once the output warps
+        // have read the previous chunk's O (the first product overwrites it)
         if (!mbar_wait(&s_conv, c & 1, ab)) break;
         if (!mbar_wait(&w_full, c & 1, ab)) break;
-        if (!mbar_wait(&o_free, c & 1, ab)) break;
         tc_fence_after();
 #pragma unroll kIssueUnroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bw = smem_desc(wq + ks * 2048u, kImg64, 1024, Swz::k128);
           const uint64_t bw2 = smem_desc(wq + kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
           umma_bf16_ts(tbase + kColU2, tbase + kColSH + 8 * ks, bw, idesc_u, true);
-          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u, true);
+          umma_bf16_ts(tbase + kColU1, tbase + kColSL + 8 * ks, bw2, idesc_u2, true);
         }
         umma_commit(&u_done);
+        if (!mbar_wait(&o_free, c & 1, ab)) break;
+        tc_fence_after();
 #pragma unroll kIssueUnroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t bq = smem_desc(wq + 2 * kImg64 + ks * 2048u, kImg64, 1024, Swz::k128);
-          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, true);
+          umma_bf16_ts(tbase + kColO, tbase + kColSH + 8 * ks, bq, idesc_u, ks > 0);
+          umma_bf16_ts(tbase + kColO, tbase + kColSL + 8 * ks, bq, idesc_u2, true);
         }
         umma_commit(&w_free);
         if (!mbar_wait(&u_conv, c & 1, ab)) break;
@@ -1266,16 +1269,7 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
     float w8[8];  // norm_w is only 2-byte aligned: element loads
 #pragma unroll
     for (int e2 = 0; e2 < 8; ++e2) w8[e2] = __bfloat162float(p.norm_w[v8 + e2]);
-    {  // O starts cleared: the first chunk's product accumulates onto it
-      float zero[32];
-#pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) zero[e2] = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_st32(tl + kColO + 32 * cc, zero);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&o_free);
-    }
+    mbar_arrive(&o_free);  // the first chunk's state product writes O afresh
     // Every output warp reaches every named barrier; a failed wait is OR-ed into the
     // first barrier so that the four warps leave the loop together.
     for (int c = 0; c < nc; ++c) {
@@ -1297,17 +1291,16 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
       bool ok = mbar_wait_warp(&y_done, c & 1, ab, false, kBackoffNs);
       if (ok) {
         tc_fence_after();
-        float zero[32];
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) zero[e2] = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           float o1[32], o2[32];
           tmem_ld32(tl + kColO + 32 * cc, o1);
           tmem_ld32(tl + kColO + 64 + 32 * cc, o2);
           tmem_wait_ld();
-          tmem_st32(tl + kColO + 32 * cc, zero);
-          tmem_st32(tl + kColO + 64 + 32 * cc, zero);
+          if (cc == 1) {  // O is read: the next chunk's product may overwrite it
+            tc_fence_before();
+            mbar_arrive(&o_free);
+          }
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float2 r = __fadd2_rn(make_float2(o1[i], o1[i + 1]), make_float2(o2[i], o2[i + 1]));
@@ -1315,9 +1308,6 @@ __device__ __forceinline__ void scan_body(const PrefillParams& p, int blk, uint8
             sO[(32 * cc + i + 1) * kD + v] = r.y;
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&o_free);
       }
       if (bar_sync_or(1, 128, !ok)) break;
       // the eight tokens' sums of squares side by side (independent shuffles), then the outputs

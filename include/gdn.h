@@ -101,9 +101,9 @@ typedef struct {
                              before and after the decode kernel. */
   int schedule;           /* prefill launch plan.  1 = the chunk-parallel prep kernel, then the
                              sequential scan kernel.  2 = one launch that overlaps them chunk by
-                             chunk (scan CTAs first, the prep on the other SMs publishing each
-                             chunk to the scan) whenever the scan's (sequence, value head) units
-                             fit in half the SMs, else as 1.  0 = automatic: as 2 when the prep
+                             chunk (the scan on the launch's last CTAs, the prep on the others
+                             publishing each chunk to the scan) whenever the scan's (sequence,
+                             value head) units fit in half the SMs, else as 1.  0 = automatic: as 2 when the prep
                              also has at least 8 (chunk, key head) items per remaining SM, else
                              as 1.  "The SMs" are those the calling context may use (see
                              gdn_prefill_fused_plan).  Results are bitwise identical under every

@@ -60,19 +60,19 @@ DECODE_BYTES_PER_SEQ = 2 * 48 * 128 * 128 * 4                          # fp32 st
 # DRAM traffic of one launch from an ncu capture, valid only for the kernel source
 # it was taken on (sha256 of the .cu file, first 16 hex digits).
 TRAFFIC = {
-    (1, "prefill_fused"): {"bytes": 443626496 + 462670848, "sha": "71336e0501319143"},  # ncu, T=4096 16/48, one launch
-    (1, "prep"): {"bytes": 87340032 + 383146240, "sha": "71336e0501319143"},
-    (1, "scan"): {"bytes": 493061888 + 41922048, "sha": "71336e0501319143"},
-    (0, "prep"): {"bytes": 1435648 + 0, "sha": "71336e0501319143"},                  # ncu, T=512 2/6
-    (0, "scan"): {"bytes": 7726848 + 0, "sha": "71336e0501319143"},
-    (2, "prefill_fused"): {"bytes": 16 * (1945085184 + 1959130112), "sha": "71336e0501319143",
+    (1, "prefill_fused"): {"bytes": 502739968 + 470943744, "sha": "f1c941c89f236f35"},  # ncu, T=4096 16/48, one launch
+    (1, "prep"): {"bytes": 87277824 + 383108608, "sha": "f1c941c89f236f35"},
+    (1, "scan"): {"bytes": 493164800 + 41825536, "sha": "f1c941c89f236f35"},
+    (0, "prep"): {"bytes": 1435904 + 0, "sha": "f1c941c89f236f35"},                  # ncu, T=512 2/6
+    (0, "scan"): {"bytes": 7730176 + 0, "sha": "f1c941c89f236f35"},
+    (2, "prefill_fused"): {"bytes": 16 * (2214828800 + 1960944128), "sha": "f1c941c89f236f35",
                            "note": "ncu capture of the first 16,384 tokens (fused launch), x16 by tokens"},
-    (3, "prep"): {"bytes": round(8.004909618388753 * (305648896 + 1423295488)), "sha": "71336e0501319143",
+    (3, "prep"): {"bytes": round(8.004909618388753 * (306098432 + 1422825216)), "sha": "f1c941c89f236f35",
                  "note": "ncu capture with every packed length scaled to 13,443 tokens in all, x107610/13443"},
-    (3, "scan"): {"bytes": round(8.004909618388753 * (1669312768 + 174477824)), "sha": "71336e0501319143",
+    (3, "scan"): {"bytes": round(8.004909618388753 * (1687225856 + 172754176)), "sha": "f1c941c89f236f35",
                  "note": "ncu capture with every packed length scaled to 13,443 tokens in all, x107610/13443"},
 }
-DECODE_TRAFFIC = {"bytes": 829675264 + 766249984, "sha": "852a2d42cccfe44d"}  # ncu, one step of 256 sequences
+DECODE_TRAFFIC = {"bytes": 829711104 + 765053696, "sha": "d1cb6c7e2cc2e513"}  # ncu, one step of 256 sequences
 
 
 def src_sha(name):

@@ -17,7 +17,8 @@ using bf16 = __nv_bfloat16;
 //   per (chunk, value head), kHeadBytes:
 //     -W^T lo | -W^T hi | (gamma Q)^T hi | (gamma Q)^T lo: four 16 KiB images of 128 rows
 //       (d_k) x 64 tokens, W = T diag(beta gamma) K (negated) and gamma Q = diag(gamma) Q;
-//       side by side one MN-major operand of N = 256 (or, from the second, N = 128)
+//       read by the scan as MN-major operands of N = 128 (-W^T lo | hi, -W^T hi | (gamma Q)^T hi,
+//       (gamma Q)^T hi | lo)
 //     P hi | P lo: P_ij = e^{G_i - G_j} q_i.k_j for j <= i, row = i, 64 j per row
 //     B_U lo | B_U hi: B_U = T diag(beta), row = i, 64 j per row (K-major); side by side
 //       one operand of N = 128
@@ -85,8 +86,8 @@ struct PrefillParams {
   bf16* out;              // [T_tot][H_v][128]
   int* err;
   int allow_fused;        // 0 = two launches, 1 = automatic, 2 = one fused launch whenever possible
-  int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, scan CTAs first, prep items
-                          // published by ready flags; 0 = prep kernel, then scan kernel
+  int fused_scan_ctas;    // set by launch_prefill: > 0 = one fused launch, the scan on its last CTAs,
+                          // prep items published by ready flags; 0 = prep kernel, then scan kernel
 };
 
 constexpr int kDevErrBounds = 64;  // (debug build) an access outside the workspace was skipped

@@ -14,6 +14,6 @@ from .gdn_oracle import (  # noqa: F401
     num_threads,
     recurrence,
 )
-from .chunked import chunked_recurrence  # noqa: F401
+from .chunked import chunked_recurrence, chunked_transfer_recurrence  # noqa: F401
 from .projections import gemm, in_proj_layout, layer, round_bf16  # noqa: F401
 from . import attention as attn  # noqa: F401

@@ -21,6 +21,17 @@ Unrolling inside one chunk that starts from S_0, with gamma_i = prod_{j<=i} alph
 This is the chunkwise (UT-transform) form of the published Gated Delta Networks
 and DeltaNet-parallelisation papers, re-derived here.  A library triangular
 solve and matmuls are its only primitives.
+
+chunked_transfer_recurrence writes the same chunk step with the state dependence
+gathered into one product per chunk.  With T = (I + A)^{-1}, W = T diag(beta gamma) K,
+U0 = T diag(beta) V, P = M * Q K^T and D = diag(exp(G_C - G_j)), the solve above is
+U = U0 - W S_0^T, so
+
+  O   = (diag(gamma) Q - P W) S_0^T + P U0
+  S_C = S_0 (gamma_C I - W^T D K) + U0^T D K
+
+i.e. S_C = S_0 M + N with M and N independent of the state (a transfer matrix and a
+drive per chunk).
 """
 from __future__ import annotations
 
@@ -51,4 +62,33 @@ def chunked_recurrence(q, k, v, g, beta, S0=None, chunk=64):
         o[sl] = gam[:, None] * (Q @ S.T) + (M * (Q @ K.T)) @ U
         dec = np.exp(G[-1] - G)
         S = gam[-1] * S + U.T @ (dec[:, None] * K)
+    return o, S
+
+
+def chunked_transfer_recurrence(q, k, v, g, beta, S0=None, chunk=64):
+    """The same chunk step as chunked_recurrence, written as O = Q' S_0^T + P U0 and
+    S_C = S_0 M + N (module docstring).  Arguments and results as chunked_recurrence."""
+    q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
+    T, dk = k.shape
+    dv = v.shape[1]
+    S = np.zeros((dv, dk)) if S0 is None else np.array(S0, dtype=np.float64)
+    o = np.zeros((T, dv))
+    for c0 in range(0, T, chunk):
+        sl = slice(c0, min(c0 + chunk, T))
+        Q, K, V, b = q[sl], k[sl], v[sl], beta[sl]
+        L = K.shape[0]
+        G = np.cumsum(g[sl])
+        gam = np.exp(G)
+        ii, jj = np.meshgrid(np.arange(L), np.arange(L), indexing="ij")
+        M_ij = np.exp(np.where(jj <= ii, G[:, None] - G[None, :], -np.inf))
+        A = b[:, None] * np.where(jj < ii, M_ij, 0.0) * (K @ K.T)
+        Tinv = np.linalg.inv(np.eye(L) + A)
+        W = Tinv @ ((b * gam)[:, None] * K)
+        U0 = Tinv @ (b[:, None] * V)
+        P = M_ij * (Q @ K.T)
+        DK = np.exp(G[-1] - G)[:, None] * K
+        transfer = gam[-1] * np.eye(dk) - W.T @ DK
+        drive = U0.T @ DK
+        o[sl] = (gam[:, None] * Q - P @ W) @ S.T + P @ U0
+        S = S @ transfer + drive
     return o, S

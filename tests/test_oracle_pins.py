@@ -149,6 +149,28 @@ def test_chunked_form_agrees(chunk, T):
     assert np.max(np.abs(S_ch - S_seq[0, 0])) <= 1e-12 * scale_s
 
 
+@pytest.mark.parametrize("chunk", [1, 16, 64])
+@pytest.mark.parametrize("T", [1, 63, 65, 200])
+def test_chunked_transfer_form_agrees(chunk, T):
+    """The chunk step with the state dependence gathered into S_0 M + N (transfer matrix
+    and drive per chunk) equals the sequential recurrence to 1e-12, slow and fast decay."""
+    D = 128
+    for g_hi in (0.05, 1.5):
+        q = RNG.standard_normal((T, 1, D))
+        k = unit_rows(np.abs(RNG.standard_normal((T, 1, D))) + 0.3)
+        v = RNG.standard_normal((T, 1, D))
+        g = -RNG.uniform(0.0, g_hi, (T, 1))
+        beta = RNG.uniform(0, 1, (T, 1))
+        S0 = 0.1 * RNG.standard_normal((1, 1, D, D))
+        o_seq, S_seq = oracle.recurrence(q, k, v, np.exp(g), beta, [0, T], S0)
+        o_tr, S_tr = oracle.chunked_transfer_recurrence(q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0], S0[0, 0],
+                                                        chunk)
+        scale_o = max(1.0, np.sqrt(np.mean(o_seq**2)))
+        scale_s = max(1.0, np.sqrt(np.mean(S_seq**2)))
+        assert np.max(np.abs(o_tr - o_seq[:, 0])) <= 1e-12 * scale_o
+        assert np.max(np.abs(S_tr - S_seq[0, 0])) <= 1e-12 * scale_s
+
+
 def test_value_rows_are_independent():
     """Changing value channel r of head h changes only output channel r of head h
     and state row r (the state is d_v x d_k and o = S q)."""

@@ -107,7 +107,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.002):
         self.samples, self.reasons, self.period = [], 0, period
         self._stop = threading.Event()
         self.ok = False

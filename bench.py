@@ -651,7 +651,7 @@ def run_attn_layer_ours(args, world, rank, dev, pk, T=4096, hidden=5120):
             torch.cuda.synchronize()
             tot += e0.elapsed_time(e1)
         sdpa_ms = tot / 10
-    except RuntimeError as exc:  # no fused kernel for this shape on this build
+    except RuntimeError as exc:  # no fused kernel for this shape in the library
         print(f"note: torch SDPA unavailable for the comparison: {exc}", file=sys.stderr)
     n_in = gdn.ATTN_N_IN
     flops = {"in_proj": 2 * T * hidden * n_in, "out_proj": 2 * T * 24 * 256 * hidden,

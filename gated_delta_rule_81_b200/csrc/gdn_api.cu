@@ -695,7 +695,7 @@ const char* gdn_status_string(gdn_status status) {
   switch (status) {
     case GDN_OK: return "GDN_OK";
     case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: null pointer, bad count or bad shape";
-    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: request outside what this build implements";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: request outside what this library implements";
     case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointer or stride not suitably aligned";
     case GDN_ERR_ALIAS: return "GDN_ERR_ALIAS: buffers that must be distinct overlap";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA launch failed";

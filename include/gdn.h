@@ -67,7 +67,7 @@ extern "C" {
 typedef enum {
   GDN_OK = 0,
   GDN_ERR_INVALID_ARG = 1,   /* null required pointer, bad count, bad shape */
-  GDN_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  GDN_ERR_UNSUPPORTED = 2,   /* valid request this library does not implement */
   GDN_ERR_MISALIGNED = 3,    /* a pointer or stride is not 16-byte aligned */
   GDN_ERR_ALIAS = 4,         /* buffers that must be distinct overlap */
   GDN_ERR_CUDA = 5,          /* a CUDA launch failed */
